@@ -1,0 +1,216 @@
+"""Thin ctypes binding of libcf.so (include/cf.h), same names as the C ABI.
+
+Argument marshalling only: tensors become raw device pointers, the stream
+defaults to torch's current stream, and a non-zero cf_status raises
+CFError.  Every step of the compression runs in the library's CUDA kernels;
+there is no Python or CPU fallback.  If libcf.so is missing, the first call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcf.so")
+
+CF_OK = 0
+STATUS_NAMES = {0: "CF_OK", 1: "CF_ERR_INVALID_ARG", 2: "CF_ERR_ALIGNMENT",
+                3: "CF_ERR_UNSUPPORTED", 4: "CF_ERR_WORKSPACE", 5: "CF_ERR_CUDA",
+                6: "CF_ERR_NUMERIC", 7: "CF_ERR_TIMEOUT"}
+
+# Every symbol include/cf.h declares (checked by the ABI test).
+EXPORTS = ("cf_status_string", "cf_abi_version", "cf_codes_words_per_row",
+           "cf_payload_bytes", "cf_state_init", "cf_encode", "cf_decode",
+           "cf_encode_batched", "cf_decode_batched", "cf_lowrank_workspace_bytes",
+           "cf_lowrank_factor_bytes", "cf_lowrank_encode", "cf_lowrank_decode",
+           "cf_lowrank_status", "cf_set_launch_override")
+
+
+class CFError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib().cf_status_string(status).decode() if _lib is not None else str(status)
+        super().__init__(f"{where}: {msg}")
+
+
+class cf_desc(ctypes.Structure):
+    _fields_ = [("tokens", ctypes.c_int64), ("channels", ctypes.c_int64),
+                ("bits", ctypes.c_int32), ("rank", ctypes.c_int32),
+                ("iters", ctypes.c_int32), ("scale_kind", ctypes.c_int32)]
+
+
+class cf_enc_buffer(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("recon_s", ctypes.c_void_p),
+                ("err", ctypes.c_void_p), ("codes", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p)]
+
+
+class cf_dec_buffer(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("recon_r", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libcf.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libcf.so not built ({LIB_PATH}); run "
+                               "`python -m activation_residual_compression_cf_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        D = ctypes.POINTER(cf_desc)
+        sig = {
+            "cf_status_string": ([ctypes.c_int], ctypes.c_char_p),
+            "cf_abi_version": ([], i32),
+            "cf_codes_words_per_row": ([D], i64),
+            "cf_payload_bytes": ([D], i64),
+            "cf_state_init": ([D, vp, vp, vp, vp], ctypes.c_int),
+            "cf_encode": ([D, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+            "cf_decode": ([D, vp, vp, vp, vp], ctypes.c_int),
+            "cf_encode_batched": ([D, i32, vp, vp, vp], ctypes.c_int),
+            "cf_decode_batched": ([D, i32, vp, vp, vp], ctypes.c_int),
+            "cf_lowrank_workspace_bytes": ([D], i64),
+            "cf_lowrank_factor_bytes": ([i64, i32], i64),
+            "cf_lowrank_encode": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+            "cf_lowrank_decode": ([D, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+            "cf_lowrank_status": ([vp, vp], ctypes.c_int),
+            "cf_set_launch_override": ([i32, i32, i32, i32], ctypes.c_int),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes, f.restype = args, res
+        _lib = L
+    return _lib
+
+
+def desc(tokens: int, channels: int, bits: int = 0, rank: int = 0, iters: int = 0,
+         scale_kind: int = 0) -> cf_desc:
+    return cf_desc(tokens, channels, bits, rank, iters, scale_kind)
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _s(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _chk(st: int, where: str):
+    if st != CF_OK:
+        raise CFError(st, where)
+
+
+def cf_status_string(status: int) -> str:
+    return lib().cf_status_string(status).decode()
+
+
+def cf_abi_version() -> int:
+    return lib().cf_abi_version()
+
+
+def cf_codes_words_per_row(d: cf_desc) -> int:
+    return lib().cf_codes_words_per_row(ctypes.byref(d))
+
+
+def cf_payload_bytes(d: cf_desc) -> int:
+    return lib().cf_payload_bytes(ctypes.byref(d))
+
+
+def cf_state_init(d, x0, recon, err=None, stream=None):
+    _chk(lib().cf_state_init(ctypes.byref(d), _p(x0), _p(recon), _p(err), _s(stream)),
+         "cf_state_init")
+
+
+def cf_encode(d, x, recon_s, err, codes, scales, stream=None):
+    _chk(lib().cf_encode(ctypes.byref(d), _p(x), _p(recon_s), _p(err), _p(codes),
+                         _p(scales), _s(stream)), "cf_encode")
+
+
+def cf_decode(d, codes, scales, recon_r, stream=None):
+    _chk(lib().cf_decode(ctypes.byref(d), _p(codes), _p(scales), _p(recon_r), _s(stream)),
+         "cf_decode")
+
+
+def cf_encode_batched(d, n, bufs_dev, status_dev=None, stream=None):
+    _chk(lib().cf_encode_batched(ctypes.byref(d), n, _p(bufs_dev), _p(status_dev), _s(stream)),
+         "cf_encode_batched")
+
+
+def cf_decode_batched(d, n, bufs_dev, status_dev=None, stream=None):
+    _chk(lib().cf_decode_batched(ctypes.byref(d), n, _p(bufs_dev), _p(status_dev), _s(stream)),
+         "cf_decode_batched")
+
+
+def cf_lowrank_workspace_bytes(d) -> int:
+    return lib().cf_lowrank_workspace_bytes(ctypes.byref(d))
+
+
+def cf_lowrank_factor_bytes(rows: int, rank: int) -> int:
+    return lib().cf_lowrank_factor_bytes(rows, rank)
+
+
+def cf_lowrank_encode(d, x, recon_s, err, omega, p_codes, p_scales, q_codes, q_scales,
+                      workspace, workspace_bytes=None, stream=None):
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _chk(lib().cf_lowrank_encode(ctypes.byref(d), _p(x), _p(recon_s), _p(err), _p(omega),
+                                 _p(p_codes), _p(p_scales), _p(q_codes), _p(q_scales),
+                                 _p(workspace), nbytes, _s(stream)), "cf_lowrank_encode")
+
+
+def cf_lowrank_decode(d, p_codes, p_scales, q_codes, q_scales, recon_r, stream=None):
+    _chk(lib().cf_lowrank_decode(ctypes.byref(d), _p(p_codes), _p(p_scales), _p(q_codes),
+                                 _p(q_scales), _p(recon_r), _s(stream)), "cf_lowrank_decode")
+
+
+def cf_lowrank_status(workspace, stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the workspace status."""
+    return lib().cf_lowrank_status(_p(workspace), _s(stream))
+
+
+def cf_set_launch_override(kernel: int, groups_per_thread: int = 0, threads: int = 0,
+                           blocks_per_sm: int = 0):
+    _chk(lib().cf_set_launch_override(kernel, groups_per_thread, threads, blocks_per_sm),
+         "cf_set_launch_override")
+
+
+# ----------------------------------------------------------- small helpers
+# Allocation helpers for callers that hold their buffers in torch tensors.
+# They only size and place memory; the library itself never allocates.
+
+def enc_buffer_array(sets, device) -> torch.Tensor:
+    """Device array of cf_enc_buffer from [(x, recon_s, err, codes, scales), ...]."""
+    arr = (cf_enc_buffer * len(sets))()
+    for i, (x, r, e, c, s) in enumerate(sets):
+        arr[i] = cf_enc_buffer(_p(x), _p(r), _p(e), _p(c), _p(s))
+    host = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8)
+    return host.to(device)
+
+
+def dec_buffer_array(sets, device) -> torch.Tensor:
+    """Device array of cf_dec_buffer from [(codes, scales, recon_r), ...]."""
+    arr = (cf_dec_buffer * len(sets))()
+    for i, (c, s, r) in enumerate(sets):
+        arr[i] = cf_dec_buffer(_p(c), _p(s), _p(r))
+    host = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8)
+    return host.to(device)
+
+
+def bf16_as_u16(x: torch.Tensor) -> torch.Tensor:
+    """View a bf16 tensor as its 16-bit patterns (no copy)."""
+    return x.view(torch.int16)

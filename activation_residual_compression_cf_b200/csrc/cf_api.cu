@@ -1,0 +1,288 @@
+// cf_api.cu -- host side of libcf.so: argument validation, launch-shape
+// choice and kernel launches behind the C ABI declared in cf.h.
+//
+// Nothing here allocates device memory or synchronises a stream (except
+// cf_lowrank_status, documented as synchronising).
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "cf.h"
+#include "lowrank_api.cuh"
+#include "quant_kernels.cuh"
+
+namespace {
+
+// ---------------------------------------------------------------- helpers
+
+constexpr int kMaxGroupsPerThread = 4;
+constexpr int kMaxThreads = 512;
+constexpr int64_t kMaxChannels = 8LL * kMaxGroupsPerThread * kMaxThreads;  // 16384
+
+struct Override {
+    int gpt = 0, threads = 0, blocks_per_sm = 0;
+};
+Override g_override[2];
+std::mutex g_mu;
+
+int device_sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    static int cache[64] = {0};
+    if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < 64) cache[dev] = n;
+    return n;
+}
+
+bool is_aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cf_status check_dev_ptr(const void *p) {
+    if (!p) return CF_ERR_INVALID_ARG;
+    if (!is_aligned16(p)) return CF_ERR_ALIGNMENT;
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return CF_ERR_INVALID_ARG;
+    }
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return CF_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return CF_ERR_CUDA;
+    if (a.type == cudaMemoryTypeDevice && a.device != dev) return CF_ERR_INVALID_ARG;
+    return CF_OK;
+}
+
+#define CF_TRY(expr)                         \
+    do {                                     \
+        cf_status _s = (expr);               \
+        if (_s != CF_OK) return _s;          \
+    } while (0)
+
+cf_status check_quant_desc(const cf_desc *d) {
+    if (!d) return CF_ERR_INVALID_ARG;
+    if (d->tokens < 0 || d->channels < 1) return CF_ERR_INVALID_ARG;
+    if (d->scale_kind != 0) return CF_ERR_UNSUPPORTED;
+    if (d->bits != 1 && d->bits != 2) return CF_ERR_UNSUPPORTED;
+    if (d->rank != 0 || d->iters != 0) return CF_ERR_INVALID_ARG;
+    if (d->channels > kMaxChannels) return CF_ERR_UNSUPPORTED;
+    if (d->tokens > (int64_t(1) << 40) / d->channels) return CF_ERR_INVALID_ARG;
+    return CF_OK;
+}
+
+struct Shape {
+    int gpt;
+    int threads;
+    int blocks_per_sm;
+};
+
+// Smallest thread count (multiple of 32) with at most 4 groups of 8
+// channels per thread, aiming at ~128 threads per row.
+Shape choose_shape(int kernel, int64_t C) {
+    const int64_t G = (C + 7) / 8;
+    Shape s;
+    int gpt = (int)((G + 127) / 128);
+    if (gpt < 1) gpt = 1;
+    if (gpt > kMaxGroupsPerThread) gpt = kMaxGroupsPerThread;
+    int64_t thr = (G + gpt - 1) / gpt;
+    thr = (thr + 31) / 32 * 32;
+    s.gpt = gpt;
+    s.threads = (int)thr;
+    s.blocks_per_sm = 0;
+    std::lock_guard<std::mutex> lk(g_mu);
+    const Override &o = g_override[kernel];
+    if (o.gpt > 0 && o.threads > 0 && (int64_t)o.gpt * o.threads >= G) {
+        s.gpt = o.gpt;
+        s.threads = o.threads;
+    }
+    if (o.blocks_per_sm > 0) s.blocks_per_sm = o.blocks_per_sm;
+    return s;
+}
+
+template <class K>
+int grid_for(K kernel, int threads, int blocks_per_sm_cap, int64_t rows) {
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, 0) != cudaSuccess ||
+        occ < 1) {
+        (void)cudaGetLastError();
+        occ = 1;
+    }
+    if (blocks_per_sm_cap > 0 && blocks_per_sm_cap < occ) occ = blocks_per_sm_cap;
+    int64_t g = (int64_t)device_sm_count() * occ;
+    if (g < 1) g = 1;
+    if (rows < g) g = rows;
+    return (int)g;
+}
+
+cf_status launch_result() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? CF_OK : CF_ERR_CUDA;
+}
+
+template <int BITS, int GPT, bool VEC, class Src>
+cf_status launch_encode_t(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t *status,
+                          const Shape &s, cudaStream_t st) {
+    auto k = cf::encode_rows_kernel<BITS, GPT, VEC, Src>;
+    const int grid = grid_for(k, s.threads, s.blocks_per_sm, rows);
+    k<<<grid, s.threads, 0, st>>>(src, T, C, rows, status);
+    return launch_result();
+}
+
+template <int BITS, int GPT, bool VEC, class Src>
+cf_status launch_decode_t(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t *status,
+                          const Shape &s, cudaStream_t st) {
+    auto k = cf::decode_rows_kernel<BITS, GPT, VEC, Src>;
+    const int grid = grid_for(k, s.threads, s.blocks_per_sm, rows);
+    k<<<grid, s.threads, 0, st>>>(src, T, C, rows, status);
+    return launch_result();
+}
+
+template <bool ENC, int BITS, int GPT, bool VEC, class Src>
+cf_status launch_one(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t *status,
+                     const Shape &s, cudaStream_t st) {
+    if constexpr (ENC)
+        return launch_encode_t<BITS, GPT, VEC>(src, T, C, rows, status, s, st);
+    else
+        return launch_decode_t<BITS, GPT, VEC>(src, T, C, rows, status, s, st);
+}
+
+// Runtime (bits, gpt, vec) -> template instance.
+template <bool ENC, class Src>
+cf_status dispatch(const Src &src, int bits, int64_t T, int64_t C, int64_t rows,
+                   int32_t *status, cudaStream_t st) {
+    const Shape s = choose_shape(ENC ? 0 : 1, C);
+    const bool vec = (C % 8) == 0;
+#define CF_CASE(B, G, V)                                     \
+    if (bits == B && s.gpt == G && vec == V)                 \
+        return launch_one<ENC, B, G, V>(src, T, C, rows, status, s, st);
+#define CF_CASES_G(B, V) CF_CASE(B, 1, V) CF_CASE(B, 2, V) CF_CASE(B, 3, V) CF_CASE(B, 4, V)
+    CF_CASES_G(1, true)
+    CF_CASES_G(1, false)
+    CF_CASES_G(2, true)
+    CF_CASES_G(2, false)
+#undef CF_CASES_G
+#undef CF_CASE
+    return CF_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ C ABI
+
+extern "C" {
+
+const char *cf_status_string(cf_status s) {
+    switch (s) {
+        case CF_OK: return "CF_OK";
+        case CF_ERR_INVALID_ARG: return "CF_ERR_INVALID_ARG: null, host or out-of-range argument";
+        case CF_ERR_ALIGNMENT: return "CF_ERR_ALIGNMENT: device pointer not 16-byte aligned";
+        case CF_ERR_UNSUPPORTED: return "CF_ERR_UNSUPPORTED: bits/rank/scale_kind/shape not supported";
+        case CF_ERR_WORKSPACE: return "CF_ERR_WORKSPACE: low-rank workspace too small";
+        case CF_ERR_CUDA: return "CF_ERR_CUDA: CUDA runtime call or kernel launch failed";
+        case CF_ERR_NUMERIC: return "CF_ERR_NUMERIC: Gram matrix not positive definite";
+        case CF_ERR_TIMEOUT: return "CF_ERR_TIMEOUT: bounded device wait gave up";
+    }
+    return "unknown cf_status";
+}
+
+int32_t cf_abi_version(void) { return CF_ABI_VERSION; }
+
+int64_t cf_codes_words_per_row(const cf_desc *d) {
+    if (check_quant_desc(d) != CF_OK) return 0;
+    return (d->channels * d->bits + 31) / 32;
+}
+
+int64_t cf_payload_bytes(const cf_desc *d) {
+    if (!d) return 0;
+    if (d->bits == 0 && d->rank > 0) {
+        if (cf_lowrank::check_desc(d) != CF_OK) return 0;
+        const int64_t nb = (d->rank + 1) / 2;
+        return d->tokens * nb + d->channels * nb + 8LL * d->rank;
+    }
+    if (check_quant_desc(d) != CF_OK) return 0;
+    return d->tokens * cf_codes_words_per_row(d) * 4 + d->tokens * 4;
+}
+
+cf_status cf_state_init(const cf_desc *d, const uint16_t *x0, float *recon, float *err,
+                        void *stream) {
+    if (!d || d->tokens < 0 || d->channels < 1) return CF_ERR_INVALID_ARG;
+    if (d->tokens > (int64_t(1) << 40) / d->channels) return CF_ERR_INVALID_ARG;
+    const int64_t n = d->tokens * d->channels;
+    if (n == 0) return CF_OK;
+    CF_TRY(check_dev_ptr(x0));
+    CF_TRY(check_dev_ptr(recon));
+    if (err) CF_TRY(check_dev_ptr(err));
+    const int threads = 256;
+    int64_t blocks = (n / 8 + threads - 1) / threads;
+    const int64_t cap = (int64_t)device_sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    cf::state_init_kernel<<<(int)blocks, threads, 0, (cudaStream_t)stream>>>(x0, recon, err, n);
+    return launch_result();
+}
+
+cf_status cf_encode(const cf_desc *d, const uint16_t *x, float *recon_s, float *err,
+                    uint32_t *codes, float *scales, void *stream) {
+    CF_TRY(check_quant_desc(d));
+    if (d->tokens == 0) return CF_OK;
+    CF_TRY(check_dev_ptr(x));
+    CF_TRY(check_dev_ptr(recon_s));
+    CF_TRY(check_dev_ptr(err));
+    CF_TRY(check_dev_ptr(codes));
+    CF_TRY(check_dev_ptr(scales));
+    cf::EncSingle src{{x, recon_s, err, codes, scales}};
+    return dispatch<true>(src, d->bits, d->tokens, d->channels, d->tokens, nullptr,
+                          (cudaStream_t)stream);
+}
+
+cf_status cf_decode(const cf_desc *d, const uint32_t *codes, const float *scales, float *recon_r,
+                    void *stream) {
+    CF_TRY(check_quant_desc(d));
+    if (d->tokens == 0) return CF_OK;
+    CF_TRY(check_dev_ptr(codes));
+    CF_TRY(check_dev_ptr(scales));
+    CF_TRY(check_dev_ptr(recon_r));
+    cf::DecSingle src{{codes, scales, recon_r}};
+    return dispatch<false>(src, d->bits, d->tokens, d->channels, d->tokens, nullptr,
+                           (cudaStream_t)stream);
+}
+
+cf_status cf_encode_batched(const cf_desc *d, int32_t n, const cf_enc_buffer *bufs_dev,
+                            int32_t *status_dev, void *stream) {
+    CF_TRY(check_quant_desc(d));
+    if (n < 0) return CF_ERR_INVALID_ARG;
+    if (n == 0 || d->tokens == 0) return CF_OK;
+    CF_TRY(check_dev_ptr(bufs_dev));
+    if (status_dev) CF_TRY(check_dev_ptr(status_dev));
+    cf::EncArray src{bufs_dev};
+    return dispatch<true>(src, d->bits, d->tokens, d->channels, d->tokens * (int64_t)n,
+                          status_dev, (cudaStream_t)stream);
+}
+
+cf_status cf_decode_batched(const cf_desc *d, int32_t n, const cf_dec_buffer *bufs_dev,
+                            int32_t *status_dev, void *stream) {
+    CF_TRY(check_quant_desc(d));
+    if (n < 0) return CF_ERR_INVALID_ARG;
+    if (n == 0 || d->tokens == 0) return CF_OK;
+    CF_TRY(check_dev_ptr(bufs_dev));
+    if (status_dev) CF_TRY(check_dev_ptr(status_dev));
+    cf::DecArray src{bufs_dev};
+    return dispatch<false>(src, d->bits, d->tokens, d->channels, d->tokens * (int64_t)n,
+                           status_dev, (cudaStream_t)stream);
+}
+
+cf_status cf_set_launch_override(int32_t kernel, int32_t groups_per_thread, int32_t threads,
+                                 int32_t blocks_per_sm) {
+    if (kernel < 0 || kernel > 1) return CF_ERR_INVALID_ARG;
+    if (groups_per_thread < 0 || groups_per_thread > kMaxGroupsPerThread) return CF_ERR_INVALID_ARG;
+    if (threads < 0 || threads > kMaxThreads || threads % 32 != 0) return CF_ERR_INVALID_ARG;
+    if (blocks_per_sm < 0 || blocks_per_sm > 64) return CF_ERR_INVALID_ARG;
+    if ((groups_per_thread == 0) != (threads == 0)) return CF_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_override[kernel].gpt = groups_per_thread;
+    g_override[kernel].threads = threads;
+    g_override[kernel].blocks_per_sm = blocks_per_sm;
+    return CF_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,382 @@
+// quant_kernels.cuh -- fused quantize-mode encode and decode kernels.
+//
+// Method: "Accelerating Parallel Diffusion Model Serving with Residual
+// Compression" (CompactFusion summary), "Approach": the sender compresses
+// the residual against the previous reconstruction and keeps an error
+// feedback buffer; the "Measured effects" table names the 1-bit and 2-bit
+// quantisers.  The per-row arithmetic is the one documented in cf.h.
+//
+// Design (B200, HBM bound: 14.1-14.3 B/element encode, 8.1-8.3 decode):
+//  * One CTA owns one token row at a time and walks rows in a grid-stride
+//    loop over ALL buffers of a batched call (row = buffer * T + token), so a
+//    step of 114 buffers is one launch with no tail per buffer.
+//  * A thread owns GPT groups of 8 consecutive channels; group g of the row
+//    goes to thread g % blockDim, so each warp-wide access is contiguous.
+//    x is read with one 16-byte load per group, recon with two, and the
+//    whole row stays in registers between the scale reduction and the
+//    quantise/update phase: every state byte crosses HBM once.
+//  * Scale reduction: warp shuffles, then one shared-memory slot per warp
+//    (double-buffered by row parity so one __syncthreads per row suffices),
+//    combined by every thread in the same fixed order.  The 1-bit mean-abs
+//    sum is accumulated in fp64 like the definition, so the fp32 scale
+//    agrees with a sequential fp64 sum except in the rare case where the
+//    two fp64 sums straddle an fp32 rounding boundary.
+//  * Packing: a group yields 8*BITS code bits; the 4/BITS lanes that share a
+//    32-bit word OR their fields together with xor-shuffles and the first of
+//    them stores the word.
+//  * All state arithmetic uses __fadd_rn/__fsub_rn/__fmul_rn so nothing is
+//    contracted into an FMA: sender mirror and receiver update compute the
+//    identical rounded value.
+#pragma once
+
+#include "cf.h"
+#include "cf_common.cuh"
+
+namespace cf {
+
+struct EncPtrs {
+    const uint16_t *x;
+    float *recon;
+    float *err;
+    uint32_t *codes;
+    float *scales;
+};
+
+struct DecPtrs {
+    const uint32_t *codes;
+    const float *scales;
+    float *recon;
+};
+
+template <class P>
+__device__ __forceinline__ P ldg_ptr(P const *field) {
+    return reinterpret_cast<P>(
+        __ldg(reinterpret_cast<const unsigned long long *>(field)));
+}
+
+// Pointer sources: a single buffer passed by value (validated on the host)
+// or a device array of buffers (validated per buffer on the device).
+struct EncSingle {
+    EncPtrs p;
+    static constexpr bool kChecked = false;
+    __device__ __forceinline__ EncPtrs get(int64_t) const { return p; }
+};
+struct EncArray {
+    const cf_enc_buffer *a;
+    static constexpr bool kChecked = true;
+    __device__ __forceinline__ EncPtrs get(int64_t i) const {
+        const cf_enc_buffer *e = a + i;
+        EncPtrs p;
+        p.x = ldg_ptr(&e->x);
+        p.recon = ldg_ptr(&e->recon_s);
+        p.err = ldg_ptr(&e->err);
+        p.codes = ldg_ptr(&e->codes);
+        p.scales = ldg_ptr(&e->scales);
+        return p;
+    }
+};
+struct DecSingle {
+    DecPtrs p;
+    static constexpr bool kChecked = false;
+    __device__ __forceinline__ DecPtrs get(int64_t) const { return p; }
+};
+struct DecArray {
+    const cf_dec_buffer *a;
+    static constexpr bool kChecked = true;
+    __device__ __forceinline__ DecPtrs get(int64_t i) const {
+        const cf_dec_buffer *e = a + i;
+        DecPtrs p;
+        p.codes = ldg_ptr(&e->codes);
+        p.scales = ldg_ptr(&e->scales);
+        p.recon = ldg_ptr(&e->recon_r);
+        return p;
+    }
+};
+
+__device__ __forceinline__ int enc_ptr_status(const EncPtrs &p) {
+    if (!p.x || !p.recon || !p.err || !p.codes || !p.scales) return CF_ERR_INVALID_ARG;
+    if (misaligned16(p.x) || misaligned16(p.recon) || misaligned16(p.err) ||
+        misaligned16(p.codes) || misaligned16(p.scales))
+        return CF_ERR_ALIGNMENT;
+    return CF_OK;
+}
+__device__ __forceinline__ int dec_ptr_status(const DecPtrs &p) {
+    if (!p.codes || !p.scales || !p.recon) return CF_ERR_INVALID_ARG;
+    if (misaligned16(p.codes) || misaligned16(p.scales) || misaligned16(p.recon))
+        return CF_ERR_ALIGNMENT;
+    return CF_OK;
+}
+
+__device__ __forceinline__ void report(int32_t *status, int code) {
+    if (status) atomicCAS(status, (int32_t)CF_OK, (int32_t)code);
+}
+
+// Code of one residual value.  1 bit: [v >= 0].  2 bits: number of the
+// thresholds -A/2, 0, A/2 that v reaches (ties go to the upper bin).
+template <int BITS>
+__device__ __forceinline__ uint32_t quantize(float v, float half) {
+    if (BITS == 1) return v >= 0.0f ? 1u : 0u;
+    return (uint32_t)(v >= -half) + (uint32_t)(v >= 0.0f) + (uint32_t)(v >= half);
+}
+
+// Reconstruction level: 1 bit +-s; 2 bits (2k-3)/4 * A, i.e. the centres of
+// the four equal bins of [-A, A].  (2k-3)/4 is exact; one rounded product.
+template <int BITS>
+__device__ __forceinline__ float dequantize(uint32_t code, float scale) {
+    if (BITS == 1) return code ? scale : -scale;
+    const float lvl = (float)((int)(2u * code) - 3) * 0.25f;
+    return __fmul_rn(lvl, scale);
+}
+
+template <int BITS, int GPT, bool VEC, class Src>
+__global__ void __launch_bounds__(512)
+encode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status) {
+    constexpr int GPW = 4 / BITS;  // 8-channel groups per 32-bit code word
+    const int tid = threadIdx.x;
+    const int nt = blockDim.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int nw = nt >> 5;
+    const int64_t G = (C + 7) >> 3;
+    const int64_t W = (C * BITS + 31) >> 5;
+
+    __shared__ double sh_sum[2][32];
+    __shared__ float sh_max[2][32];
+
+    int par = 0;
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x, par ^= 1) {
+        const int64_t b = row / T;
+        const int64_t t = row - b * T;
+        const EncPtrs p = src.get(b);
+        if (Src::kChecked) {
+            const int st = enc_ptr_status(p);
+            if (st != CF_OK) {
+                if (tid == 0) report(status, st);
+                continue;  // uniform across the CTA
+            }
+        }
+        const uint16_t *xr = p.x + t * C;
+        float *rr = p.recon + t * C;
+        float *er = p.err + t * C;
+        uint32_t *cw = p.codes + t * W;
+
+        // Phase 1: issue every load of this thread's groups.
+        uint4 xraw[GPT];
+        float r[GPT][8];
+#pragma unroll
+        for (int j = 0; j < GPT; ++j) {
+            const int64_t g = (int64_t)j * nt + tid;
+            if (VEC) {
+                if (g < G) {
+                    xraw[j] = ld_ro_v4(xr + 8 * g);
+                    const float4 a = ld_state_v4(rr + 8 * g);
+                    const float4 c = ld_state_v4(rr + 8 * g + 4);
+                    r[j][0] = a.x; r[j][1] = a.y; r[j][2] = a.z; r[j][3] = a.w;
+                    r[j][4] = c.x; r[j][5] = c.y; r[j][6] = c.z; r[j][7] = c.w;
+                } else {
+                    xraw[j] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) r[j][e] = 0.0f;
+                }
+            } else {
+                uint32_t h[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int64_t c = 8 * g + e;
+                    const bool ok = (g < G) && (c < C);
+                    h[e] = ok ? (uint32_t)xr[c] : 0u;
+                    r[j][e] = ok ? rr[c] : 0.0f;
+                }
+                xraw[j] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16),
+                                     h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+            }
+        }
+
+        // Phase 2: residual (padding lanes hold x = recon = 0, so v = 0).
+        float v[GPT][8];
+#pragma unroll
+        for (int j = 0; j < GPT; ++j) {
+            const uint32_t w4[4] = {xraw[j].x, xraw[j].y, xraw[j].z, xraw[j].w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t h = (w4[e >> 1] >> ((e & 1) * 16)) & 0xffffu;
+                v[j][e] = __fsub_rn(bf16_bits_to_f32(h), r[j][e]);
+            }
+        }
+
+        // Phase 3: per-token scale.
+        float scale;
+        if (BITS == 1) {
+            double acc = 0.0;
+#pragma unroll
+            for (int j = 0; j < GPT; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc += (double)fabsf(v[j][e]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFullMask, acc, o);
+            if (lane == 0) sh_sum[par][warp] = acc;
+            __syncthreads();
+            double tot = 0.0;
+            for (int w = 0; w < nw; ++w) tot += sh_sum[par][w];
+            scale = __fdiv_rn(__double2float_rn(tot), (float)C);
+        } else {
+            float m = 0.0f;
+#pragma unroll
+            for (int j = 0; j < GPT; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[j][e]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+            if (lane == 0) sh_max[par][warp] = m;
+            __syncthreads();
+            float tot = 0.0f;
+            for (int w = 0; w < nw; ++w) tot = fmaxf(tot, sh_max[par][w]);
+            scale = tot;
+        }
+        const float half = __fmul_rn(0.5f, scale);
+
+        // Phase 4: quantise, error feedback, mirror update, pack, store.
+#pragma unroll
+        for (int j = 0; j < GPT; ++j) {
+            const int64_t g = (int64_t)j * nt + tid;
+            uint32_t field = 0;
+            float eo[8], ro[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const bool ok = VEC ? (g < G) : ((g < G) && (8 * g + e < C));
+                uint32_t code = quantize<BITS>(v[j][e], half);
+                code = ok ? code : 0u;
+                field |= code << (e * BITS);
+                const float d = dequantize<BITS>(code, scale);
+                eo[e] = __fsub_rn(v[j][e], d);
+                ro[e] = __fadd_rn(r[j][e], d);
+            }
+            uint32_t word = field << ((lane % GPW) * 8 * BITS);
+#pragma unroll
+            for (int o = 1; o < GPW; o <<= 1) word |= __shfl_xor_sync(kFullMask, word, o);
+            if (g < G) {
+                if (VEC) {
+                    st_stream_v4(er + 8 * g, make_float4(eo[0], eo[1], eo[2], eo[3]));
+                    st_stream_v4(er + 8 * g + 4, make_float4(eo[4], eo[5], eo[6], eo[7]));
+                    st_state_v4(rr + 8 * g, make_float4(ro[0], ro[1], ro[2], ro[3]));
+                    st_state_v4(rr + 8 * g + 4, make_float4(ro[4], ro[5], ro[6], ro[7]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int64_t c = 8 * g + e;
+                        if (c < C) {
+                            er[c] = eo[e];
+                            rr[c] = ro[e];
+                        }
+                    }
+                }
+                if ((lane % GPW) == 0) cw[g / GPW] = word;
+            }
+        }
+        if (tid == 0) p.scales[t] = scale;
+    }
+}
+
+template <int BITS, int GPT, bool VEC, class Src>
+__global__ void __launch_bounds__(512)
+decode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status) {
+    constexpr uint32_t MASK = (1u << BITS) - 1u;
+    const int tid = threadIdx.x;
+    const int nt = blockDim.x;
+    const int64_t G = (C + 7) >> 3;
+    const int64_t W = (C * BITS + 31) >> 5;
+
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+        const int64_t b = row / T;
+        const int64_t t = row - b * T;
+        const DecPtrs p = src.get(b);
+        if (Src::kChecked) {
+            const int st = dec_ptr_status(p);
+            if (st != CF_OK) {
+                if (tid == 0) report(status, st);
+                continue;
+            }
+        }
+        const float scale = __ldg(p.scales + t);
+        const uint32_t *cw = p.codes + t * W;
+        float *rr = p.recon + t * C;
+
+        uint32_t field[GPT];
+        float r[GPT][8];
+#pragma unroll
+        for (int j = 0; j < GPT; ++j) {
+            const int64_t g = (int64_t)j * nt + tid;
+            if (g < G) {
+                // group g's 8*BITS bits: byte g (1 bit) or half-word g (2 bits)
+                if (BITS == 1)
+                    field[j] = __ldg(reinterpret_cast<const uint8_t *>(cw) + g);
+                else
+                    field[j] = __ldg(reinterpret_cast<const uint16_t *>(cw) + g);
+            } else {
+                field[j] = 0u;
+            }
+            if (VEC) {
+                if (g < G) {
+                    const float4 a = ld_state_v4(rr + 8 * g);
+                    const float4 c = ld_state_v4(rr + 8 * g + 4);
+                    r[j][0] = a.x; r[j][1] = a.y; r[j][2] = a.z; r[j][3] = a.w;
+                    r[j][4] = c.x; r[j][5] = c.y; r[j][6] = c.z; r[j][7] = c.w;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int64_t c = 8 * g + e;
+                    r[j][e] = ((g < G) && (c < C)) ? rr[c] : 0.0f;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < GPT; ++j) {
+            const int64_t g = (int64_t)j * nt + tid;
+            if (g >= G) continue;
+            float ro[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t code = (field[j] >> (e * BITS)) & MASK;
+                ro[e] = __fadd_rn(r[j][e], dequantize<BITS>(code, scale));
+            }
+            if (VEC) {
+                st_state_v4(rr + 8 * g, make_float4(ro[0], ro[1], ro[2], ro[3]));
+                st_state_v4(rr + 8 * g + 4, make_float4(ro[4], ro[5], ro[6], ro[7]));
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int64_t c = 8 * g + e;
+                    if (c < C) rr[c] = ro[e];
+                }
+            }
+        }
+    }
+}
+
+// Warmup: recon = (float)x0, err = 0 (err may be null).  Flat over n
+// elements; 8-element vector body, scalar tail.
+__global__ void state_init_kernel(const uint16_t *x0, float *recon, float *err, int64_t n) {
+    const int64_t groups = n >> 3;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += stride) {
+        const uint4 xv = ld_ro_v4(x0 + 8 * g);
+        const uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = bf16_bits_to_f32((w4[e >> 1] >> ((e & 1) * 16)) & 0xffffu);
+        st_state_v4(recon + 8 * g, make_float4(f[0], f[1], f[2], f[3]));
+        st_state_v4(recon + 8 * g + 4, make_float4(f[4], f[5], f[6], f[7]));
+        if (err) {
+            st_stream_v4(err + 8 * g, make_float4(0.f, 0.f, 0.f, 0.f));
+            st_stream_v4(err + 8 * g + 4, make_float4(0.f, 0.f, 0.f, 0.f));
+        }
+    }
+    if (blockIdx.x == 0 && (int64_t)threadIdx.x < n - 8 * groups) {
+        const int64_t i = 8 * groups + threadIdx.x;
+        recon[i] = bf16_bits_to_f32(x0[i]);
+        if (err) err[i] = 0.0f;
+    }
+}
+
+}  // namespace cf

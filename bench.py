@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Throughput of the residual-compression hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload flux_sp]
+                    [--impl ours|reference] [--no-cpu-baseline] [--no-e2e]
+
+A "step" is one denoising step of the workload: every exchanged buffer is
+encoded by the sender (residual + error feedback + per-token scale +
+quantise + pack + error/mirror update) and decoded by the receiver (unpack
++ dequantise + accumulate), each as ONE batched launch over all buffers.
+
+Metric: GB/s of bf16 activation processed = 2 bytes * T * C * buffers *
+steps / (encode + decode time), whole job (all ranks).  Inputs are the
+seeded synthetic drift trajectories, pre-generated in HBM before timing; one
+step touches ~5 GB (FLUX-like shard), far more than the 126 MB L2, so no L2
+flush is needed between steps.
+
+Multi-GPU: the path has no exchange between GPUs in this build (sender and
+receiver share a device), so N ranks run N independent replicas of the
+workload ("weak" scaling); the timed region is bracketed by barriers and the
+max over ranks is reported.
+
+--impl reference times the CPU oracle (plain C, one core) on a bounded
+sample of the same workload, with the same metric and unit.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from activation_residual_compression_cf_b200 import workloads as W  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "encode+decode GB/s of bf16 activation processed; % of B200 HBM roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="flux_sp", choices=[k for k, v in W.WORKLOADS.items()
+                                                               if v.mode == "quant"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="budget of the oracle timing sample")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------ environment
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(
+            "nccl" if torch.cuda.is_available() else "gloo",
+            timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the GPU is under load."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev):
+        try:
+            self.index = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+        except Exception:
+            self.index = str(dev.index or 0)
+        self.rows, self.proc = [], None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [c.strip() for c in line.split(",")]))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [r for ts, r in self.rows if t0 - 0.1 <= ts <= t1 + 0.1] or [r for _, r in self.rows]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "activation_residual_compression_cf_b200", "csrc")
+    for fn in ("quant_kernels.cuh", "cf_common.cuh"):
+        h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(f"{kernel}:{workload}")
+    if not d or d.get("source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ CPU oracle leg
+
+def oracle_sample(wl, seconds, max_buffer_steps=10**9):
+    """Times the oracle's encode+decode on host copies of buffer 0's
+    trajectory (cycled) until `seconds` of work; returns (GB/s, detail)."""
+    import oracle
+    xs = W.trajectory(wl, 0, steps=min(wl.steps, 4), device="cpu")
+    xb = [W.bf16_bits(x) for x in xs]
+    recon_s, _ = oracle.state_init(xb[0])
+    recon_r = recon_s.copy()
+    done, t_work, i = 0, 0.0, 0
+    while t_work < seconds and done < max_buffer_steps:
+        x = xb[1 + i % (len(xb) - 1)]
+        t0 = time.perf_counter()
+        codes, scales, _ = oracle.encode(x, recon_s, wl.bits)
+        oracle.decode(codes, scales, recon_r, wl.bits)
+        t_work += time.perf_counter() - t0
+        done += 1
+        i += 1
+    gbs = 2 * wl.elems * done / t_work / 1e9
+    return gbs, done, t_work
+
+
+# ------------------------------------------------------------ GPU leg
+
+def run_ours(args, world, rank, local):
+    from activation_residual_compression_cf_b200 import build, cf
+    build.build()
+    cf.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = W.WORKLOADS[args.workload]
+    n, T, C, bits = wl.buffers, wl.tokens, wl.channels, wl.bits
+    d = cf.desc(T, C, bits)
+    Wd = cf.cf_codes_words_per_row(d)
+
+    # Pre-generate the trajectory (as many steps as fit a 40 GB budget).
+    step_bytes = n * T * C * 2
+    S = max(2, min(wl.steps, int(40e9 // step_bytes)))
+    X = torch.empty((S, n, T, C), dtype=torch.bfloat16, device=dev)
+    for b in range(n):
+        tr = W.Trajectory(wl, b, device=dev, seed=rank)
+        for s in range(S):
+            X[s, b] = tr.next()
+    del tr
+    f32 = dict(dtype=torch.float32, device=dev)
+    recon_s = torch.empty((n, T, C), **f32)
+    recon_r = torch.empty((n, T, C), **f32)
+    err = torch.empty((n, T, C), **f32)
+    codes = torch.empty((n, T, Wd), dtype=torch.int32, device=dev)
+    scales = torch.empty((n, T), **f32)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    X16 = X.view(torch.int16)
+    for b in range(n):
+        cf.cf_state_init(d, X16[0, b], recon_s[b], err[b])
+        cf.cf_state_init(d, X16[0, b], recon_r[b], None)
+    enc = [cf.enc_buffer_array([(X16[s, b], recon_s[b], err[b], codes[b], scales[b])
+                                for b in range(n)], dev) for s in range(S)]
+    dec = cf.dec_buffer_array([(codes[b], scales[b], recon_r[b]) for b in range(n)], dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        cf.cf_encode_batched(d, n, enc[1 + i % (S - 1)], status, stream)
+        cf.cf_decode_batched(d, n, dec, status, stream)
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t_start.record(stream)
+    for i in range(args.steps):
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        cf.cf_encode_batched(d, n, enc[1 + (args.warmup + i) % (S - 1)], status, stream)
+        e1.record(stream)
+        cf.cf_decode_batched(d, n, dec, status, stream)
+        e2.record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    wall1 = time.time()
+    clocks = sampler.stop(wall0, wall1)
+    assert int(status.item()) == 0, cf.cf_status_string(int(status.item()))
+    ms = t_start.elapsed_time(t_end)
+    enc_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1, _ in ev)
+    dec_ms = statistics.mean(e1.elapsed_time(e2) for _, e1, e2 in ev)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    bytes_processed = 2 * T * C * n * args.steps * world
+    value = bytes_processed / (ms / 1e3) / 1e9
+    enc_bytes = n * T * (C * 2 + C * 4 * 3 + Wd * 4 + 4)     # x, recon r/w, err w, codes, scale
+    dec_bytes = n * T * (Wd * 4 + 4 + C * 4 * 2)             # codes, scale, recon r/w
+    peak, peak_kind = peaks()
+    enc_gbs = enc_bytes / (enc_ms / 1e3) / 1e9
+    dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9
+
+    # End to end through the public API: pinned host x in, payload out.
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, status)
+        if world > 1:
+            t = torch.tensor([e2e["ms"]], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e["ms"] = float(t.item())
+        e2e = {"value": round(bytes_processed / (e2e["ms"] / 1e3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+               "ms_per_step": round(e2e["ms"] / args.steps, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, done, tw = oracle_sample(wl, args.cpu_seconds)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{done} buffer-steps of {args.workload} buffer 0 ({T}x{C}, "
+                         f"{bits}-bit encode+decode), {tw:.1f} s single-threaded C"}
+
+    traffic = recorded_traffic("encode", args.workload)
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 in, fp32 state", "data": "synthetic",
+        "config": {"workload": args.workload, "tokens": T, "channels": C, "buffers": n,
+                   "bits": bits, "mode": f"{bits}-bit {'mean-abs' if bits == 1 else 'absmax'} + EF",
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2 ({n * T * C * 14 / 1e9:.1f} GB touched per step)",
+                   "launches_per_step": 2},
+        "roofline": {"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(enc_gbs / peak, 4), "traffic": traffic,
+                     "kernel": "encode_rows_kernel (batched)", "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": enc_bytes, "avg_launch_ms": round(enc_ms, 4)},
+        "decode": {"achieved": round(dec_gbs, 1), "frac": round(dec_gbs / peak, 4),
+                   "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_ms": round(dec_ms, 4)},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    return out
+
+
+def run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, status):
+    n, T, C = wl.buffers, wl.tokens, wl.channels
+    # Two host steps of pinned input (buffer 0's trajectory replicated over
+    # the buffers), alternated so consecutive steps see a real residual.
+    tr = W.Trajectory(wl, 0, device=dev)
+    tr.next()
+    x_host = []
+    for _ in range(2):
+        xk = tr.next().unsqueeze(0).expand(n, T, C).contiguous().cpu()
+        x_host.append(xk.pin_memory())
+        del xk
+    x_dev = torch.empty((n, T, C), dtype=torch.bfloat16, device=dev)
+    x16 = x_dev.view(torch.int16)
+    enc = cf.enc_buffer_array([(x16[b], recon_s[b], err[b], codes[b], scales[b])
+                               for b in range(n)], dev)
+    dec = cf.dec_buffer_array([(codes[b], scales[b], recon_r[b]) for b in range(n)], dev)
+    codes_h = torch.empty(codes.shape, dtype=codes.dtype).pin_memory()
+    scales_h = torch.empty(scales.shape, dtype=scales.dtype).pin_memory()
+
+    def step(i):
+        x_dev.copy_(x_host[i % 2], non_blocking=True)
+        cf.cf_encode_batched(d, n, enc, status, stream)
+        cf.cf_decode_batched(d, n, dec, status, stream)
+        codes_h.copy_(codes, non_blocking=True)
+        scales_h.copy_(scales, non_blocking=True)
+
+    for i in range(max(3, args.warmup // 4)):
+        step(i)
+    torch.cuda.synchronize()
+    steps = args.steps
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return {"ms": a.elapsed_time(b), "h2d": n * T * C * 2,
+            "d2h": codes.numel() * 4 + scales.numel() * 4}
+
+
+def run_reference(args, world, rank):
+    """CPU oracle on the host cores, same metric/unit/config; rank 0 only."""
+    if rank != 0:
+        return None
+    wl = W.WORKLOADS[args.workload]
+    per_step = 1
+    import oracle
+    xs = W.trajectory(wl, 0, steps=min(wl.steps, 4), device="cpu")
+    xb = [W.bf16_bits(x) for x in xs]
+    recon_s, _ = oracle.state_init(xb[0])
+    recon_r = recon_s.copy()
+
+    def one(i):
+        for _ in range(per_step):
+            x = xb[1 + i % (len(xb) - 1)]
+            c, s, _ = oracle.encode(x, recon_s, wl.bits)
+            oracle.decode(c, s, recon_r, wl.bits)
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(i)
+    sec = time.perf_counter() - t0
+    value = 2 * wl.elems * per_step * args.steps / sec / 1e9
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sec * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 state",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "tokens": wl.tokens, "channels": wl.channels,
+                   "buffers": wl.buffers, "bits": wl.bits,
+                   "sample": f"each step = {per_step} of the {wl.buffers} buffers"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{per_step} buffer(s) per step, {args.steps} steps, "
+                                   "single-threaded C oracle"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        world, rank = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        out = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

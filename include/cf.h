@@ -1,0 +1,209 @@
+/*
+ * cf.h -- C ABI of libcf.so: B200 (sm_100a) CompactFusion-style residual
+ * compression of exchanged activations.
+ *
+ * Method: "Accelerating Parallel Diffusion Model Serving with Residual
+ * Compression" (atlas.scime.ai summary of the CompactFusion paper).  Per
+ * the page's "Approach": the sender transmits the step-wise residual against
+ * the previously reconstructed activation instead of the activation, keeps
+ * a sender-side error-feedback buffer so compression error does not build
+ * up, and compresses either to 1/2-bit codes or to low-rank factors
+ * quantised to INT4.  The receiver decodes and accumulates into its own
+ * reconstruction.  The "Measured effects" table names the 1-bit and 2-bit
+ * variants, the 1-step warmup and subspace iteration; "Key results" gives
+ * about 100x compression at rank 32 with INT4 factors.
+ *
+ * Conventions for every entry point
+ *  - Ownership: the caller allocates and owns every buffer.  The library
+ *    allocates nothing, frees nothing and never synchronises the stream
+ *    (except cf_lowrank_status, which says so).
+ *  - All device work is enqueued asynchronously on `stream`, a
+ *    cudaStream_t passed as void* (NULL = the legacy default stream).
+ *  - Pointers named *_dev or documented as device pointers must be device
+ *    (or managed) memory of the current device.  Single-buffer calls check
+ *    this with cudaPointerGetAttributes and return CF_ERR_INVALID_ARG for
+ *    host memory instead of launching.
+ *  - Every device pointer must be 16-byte aligned (CF_ERR_ALIGNMENT).
+ *  - Argument errors are reported synchronously and launch nothing.  A
+ *    failed launch returns CF_ERR_CUDA.  Numeric trouble found on the
+ *    device (low-rank mode) is written to a status word in the workspace.
+ *  - Layouts are row-major and dense: an activation is [tokens][channels].
+ *  - bf16 values are passed as their 16-bit patterns (the upper half of an
+ *    IEEE binary32).
+ *  - Inputs must be finite; NaN/Inf give unspecified codes.
+ *
+ * Quantize-mode arithmetic (fp32 IEEE round-to-nearest-even, no fused
+ * multiply-add anywhere on the state path), per token row:
+ *   v      = (float)x - recon_s
+ *   1 bit: s = (float)(sum |v| accumulated in fp64) / C ;  code = [v >= 0] ;
+ *          deq = code ? s : -s
+ *   2 bit: A = max |v| ; code = [v >= -A/2] + [v >= 0] + [v >= A/2] ;
+ *          deq = lvl[code] * A with lvl = {-3/4, -1/4, 1/4, 3/4}
+ *   err    = v - deq ;  recon_s = recon_s + deq
+ *   decode: recon_r = recon_r + deq (same expression, so recon_r == recon_s
+ *           bit for bit when both started from the same cf_state_init)
+ * Code layout: row t of the codes is ceil(C*bits/32) uint32 words; element
+ * c sits in word (c*bits)/32 at bit (c*bits)%32, least significant first;
+ * unused tail bits are zero.  One fp32 scale per token (s or A).
+ */
+#ifndef CF_H
+#define CF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CF_ABI_VERSION 1
+
+typedef enum cf_status {
+    CF_OK = 0,
+    CF_ERR_INVALID_ARG = 1,  /* null/host pointer, negative size, bad field */
+    CF_ERR_ALIGNMENT = 2,    /* a device pointer is not 16-byte aligned     */
+    CF_ERR_UNSUPPORTED = 3,  /* bits/rank/scale_kind outside what is built  */
+    CF_ERR_WORKSPACE = 4,    /* low-rank workspace too small                 */
+    CF_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed         */
+    CF_ERR_NUMERIC = 6,      /* low-rank: Gram matrix not positive definite */
+    CF_ERR_TIMEOUT = 7       /* reserved: a bounded device wait gave up      */
+} cf_status;
+
+/* Problem description, as the pages state the problem: one exchanged
+ * activation buffer of `tokens` x `channels`, compressed at `bits` (quantize
+ * mode) or at `rank` with `iters` subspace iterations (low-rank mode). */
+typedef struct cf_desc {
+    int64_t tokens;      /* T >= 0 (T == 0 is a no-op)                     */
+    int64_t channels;    /* C >= 1; quantize mode C <= 16384                */
+    int32_t bits;        /* quantize mode: 1 or 2; low-rank mode: 0         */
+    int32_t rank;        /* low-rank mode: 1..64, <= min(T, C); else 0      */
+    int32_t iters;       /* low-rank mode: 1..16; else 0                    */
+    int32_t scale_kind;  /* 0 = 1-bit mean-abs / 2-bit absmax (only value)  */
+} cf_desc;
+
+/* One sender buffer set for the batched encode (all device pointers). */
+typedef struct cf_enc_buffer {
+    const uint16_t *x;   /* bf16 [T][C], this step's activation             */
+    float *recon_s;      /* fp32 [T][C], sender copy of the reconstruction  */
+    float *err;          /* fp32 [T][C], error-feedback buffer (written)    */
+    uint32_t *codes;     /* uint32 [T][ceil(C*bits/32)] (written)           */
+    float *scales;       /* fp32 [T] (written)                              */
+} cf_enc_buffer;
+
+/* One receiver buffer set for the batched decode (all device pointers). */
+typedef struct cf_dec_buffer {
+    const uint32_t *codes;
+    const float *scales;
+    float *recon_r;      /* fp32 [T][C], receiver reconstruction (updated)  */
+} cf_dec_buffer;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *cf_status_string(cf_status s);
+
+/* CF_ABI_VERSION of the loaded library. */
+int32_t cf_abi_version(void);
+
+/* uint32 code words per token row: ceil(channels * bits / 32); 0 for an
+ * invalid descriptor. */
+int64_t cf_codes_words_per_row(const cf_desc *d);
+
+/* Bytes on the wire for one buffer: codes + scales (quantize mode) or INT4
+ * factors + scales (low-rank mode); 0 for an invalid descriptor. */
+int64_t cf_payload_bytes(const cf_desc *d);
+
+/* Warmup step ("Measured effects": the first step is sent uncompressed).
+ * recon[i] = (float)x0[i]; err[i] = 0 when err != NULL.  Call it for the
+ * sender (with err) and for the receiver (err = NULL) on the same x0.
+ * x0: bf16 [T][C] device; recon, err: fp32 [T][C] device. */
+cf_status cf_state_init(const cf_desc *d, const uint16_t *x0, float *recon,
+                        float *err, void *stream);
+
+/* Sender, quantize mode, one buffer: residual with error feedback, per-token
+ * scale, quantise, pack, error update and mirror update in one pass.
+ * x: bf16 [T][C]; recon_s: fp32 [T][C] read and updated in place;
+ * err: fp32 [T][C] written; codes: uint32 [T][words_per_row] written;
+ * scales: fp32 [T] written.  All device pointers, non-overlapping. */
+cf_status cf_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
+                    float *err, uint32_t *codes, float *scales, void *stream);
+
+/* Receiver, quantize mode, one buffer: unpack, dequantise, accumulate.
+ * codes, scales as written by cf_encode; recon_r: fp32 [T][C] updated. */
+cf_status cf_decode(const cf_desc *d, const uint32_t *codes,
+                    const float *scales, float *recon_r, void *stream);
+
+/* Batched forms: `n` buffers of the same shape in ONE launch, with the same
+ * per-buffer semantics as cf_encode / cf_decode.  `bufs_dev` is a DEVICE
+ * array of n descriptors (it must stay valid until the work completes).
+ * Pointers inside it are checked on the device: a buffer with a null or
+ * misaligned pointer is skipped and, when `status_dev` (device int32) is
+ * not NULL, the first such error code is stored there with atomicCAS over
+ * an initial CF_OK (the caller zeroes it).  Pointers inside must be device
+ * memory: the host cannot check them. */
+cf_status cf_encode_batched(const cf_desc *d, int32_t n,
+                            const cf_enc_buffer *bufs_dev, int32_t *status_dev,
+                            void *stream);
+cf_status cf_decode_batched(const cf_desc *d, int32_t n,
+                            const cf_dec_buffer *bufs_dev, int32_t *status_dev,
+                            void *stream);
+
+/* ------------------------------------------------------------------------
+ * Low-rank mode ("Approach", "Key results", "Builds on": PowerSGD-style
+ * subspace iteration, INT4 factors).  With V = (float)x - recon_s:
+ *   Q = omega ; repeat iters: Y = V Q ; P = orth(Y) ; Q = V^T P
+ *   INT4 per column of P [T][r] and Q [C][r]: s_j = max|col_j| / 7,
+ *   q = clamp(rint(col / s_j), -7, 7)
+ *   D = (q_P s_P)(q_Q s_Q)^T ; err = V - D ; recon_s = recon_s + D
+ * orth() is CholeskyQR with an fp64 Gram matrix: P = Y R^-1 with R the
+ * Cholesky factor of Y^T Y, i.e. the unique thin QR with diag(R) > 0.
+ * Factor layout: row-major [rows][ceil(r/2)] bytes, two's-complement
+ * nibbles, even column in the low nibble.  Scales: fp32 [r] per factor.
+ * ---------------------------------------------------------------------- */
+
+/* Device workspace bytes cf_lowrank_encode needs for this descriptor. */
+int64_t cf_lowrank_workspace_bytes(const cf_desc *d);
+
+/* Bytes of one packed INT4 factor with `rows` rows at rank `rank`. */
+int64_t cf_lowrank_factor_bytes(int64_t rows, int32_t rank);
+
+/* Sender, low-rank mode.  x: bf16 [T][C]; recon_s: fp32 [T][C] updated;
+ * err: fp32 [T][C] written; omega: fp32 [C][r] Gaussian start block chosen
+ * by the caller; p_codes: [T][ceil(r/2)] bytes, p_scales: fp32 [r];
+ * q_codes: [C][ceil(r/2)] bytes, q_scales: fp32 [r] (all written);
+ * workspace: device, >= cf_lowrank_workspace_bytes(d) bytes, 256-byte
+ * aligned, contents need not be initialised.  If the fp64 Gram matrix of an
+ * iteration is not positive definite (Y rank deficient, e.g. a zero
+ * residual) the affected columns of P are set to zero, which still yields a
+ * valid (lower-rank) D, and CF_ERR_NUMERIC is recorded in the workspace
+ * status word (see cf_lowrank_status). */
+cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
+                            float *err, const float *omega, uint8_t *p_codes,
+                            float *p_scales, uint8_t *q_codes, float *q_scales,
+                            void *workspace, size_t workspace_bytes,
+                            void *stream);
+
+/* Receiver, low-rank mode: recon_r += D, with D formed from the payload by
+ * the same device routine the sender uses (so recon_r == recon_s bit for
+ * bit).  recon_r: fp32 [T][C] device, updated. */
+cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes,
+                            const float *p_scales, const uint8_t *q_codes,
+                            const float *q_scales, float *recon_r,
+                            void *stream);
+
+/* Synchronises `stream`, then returns the status word the last
+ * cf_lowrank_encode on `workspace` recorded (CF_OK or CF_ERR_NUMERIC) and
+ * clears it.  Returns CF_ERR_CUDA if the copy or the sync fails. */
+cf_status cf_lowrank_status(void *workspace, void *stream);
+
+/* Launch-shape override for tuning sweeps: kernel 0 = encode, 1 = decode;
+ * groups_per_thread in 1..4 (8 channels per group), threads a multiple of
+ * 32 in 32..512, or 0 to restore the built-in choice; blocks_per_sm caps
+ * the persistent grid (0 = occupancy limit).  Affects later launches in
+ * this process only.  Returns CF_ERR_INVALID_ARG for out-of-range values. */
+cf_status cf_set_launch_override(int32_t kernel, int32_t groups_per_thread,
+                                 int32_t threads, int32_t blocks_per_sm);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CF_H */

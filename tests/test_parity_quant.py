@@ -1,0 +1,196 @@
+"""GPU parity of the quantize-mode kernels (cf_encode / cf_decode and the
+batched forms) against the CPU oracle, through the C ABI.
+
+Sizes: every workload shape, small enough for the oracle to finish in
+seconds yet spanning many rows and a ragged tail of channel groups; the
+scalar path (channels not a multiple of 8); the largest supported row; an
+empty problem; and the full FLUX-like step (114 buffers in one batched
+launch, as bench.py times it) checked on sampled buffers against the oracle
+and on all buffers through properties that hold at any size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from activation_residual_compression_cf_b200 import cf
+from activation_residual_compression_cf_b200 import workloads as W
+
+from _parity import GpuBuffer, compare_step, f32_of, oracle_step
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_trajectory(wl, buffer, steps, stats=None):
+    xs = W.trajectory(wl, buffer, steps=steps, device="cuda")
+    xb = [W.bf16_bits(x) for x in xs]
+    g = GpuBuffer(wl.tokens, wl.channels, wl.bits)
+    g.init(xs[0])
+    recon_o, _ = oracle.state_init(xb[0])
+    h = g.host()
+    assert np.array_equal(h["recon_s"], recon_o) and not np.any(h["err"])
+    for s in range(1, steps):
+        g.step(xs[s])
+        v, ora = oracle_step(xb[s], recon_o, wl.bits)
+        gh = g.host()
+        compare_step(wl.bits, v, ora, gh, stats)
+        # receiver tracks sender bit for bit on the GPU
+        assert np.array_equal(gh["recon_r"].view(np.uint32), gh["recon_s"].view(np.uint32))
+        # free-running: the oracle continues from its own state
+    return stats
+
+
+def test_tiny_full_trajectory():
+    stats = _run_trajectory(W.WORKLOADS["tiny"], 0, 8, {})
+    assert stats["code_diffs"] == 0
+
+
+@pytest.mark.parametrize("name,tokens", [("flux_sp", 96), ("flux_full", 80), ("cogvideox", 70)])
+def test_workload_shapes_trajectory(name, tokens):
+    wl = W.replace(W.WORKLOADS[name], tokens=tokens)
+    _run_trajectory(wl, 1, 5, {})
+
+
+@pytest.mark.parametrize("T,C,bits", [
+    (37, 3072, 1), (37, 3072, 2), (50, 1920, 1), (19, 200, 2), (64, 64, 2),
+    (13, 33, 2), (9, 33, 1), (5, 1, 1), (6, 7, 2), (11, 1000, 1),   # scalar path: C % 8 != 0
+    (3, 16384, 1), (3, 16384, 2),                                   # largest supported row
+])
+def test_shapes_and_ragged_tails(T, C, bits):
+    wl = W.replace(W.WORKLOADS["flux_sp"], tokens=T, channels=C, bits=bits)
+    _run_trajectory(wl, 0, 3, {})
+
+
+def test_empty_tokens_is_noop():
+    g = GpuBuffer(0, 64, 1)
+    g.step(torch.empty(0, 64, dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+
+
+def test_zero_residual_on_gpu():
+    wl = W.replace(W.WORKLOADS["flux_sp"], tokens=16)
+    x = W.trajectory(wl, 0, steps=1, device="cuda")[0]
+    for bits in (1, 2):
+        g = GpuBuffer(16, 3072, bits)
+        g.init(x)
+        before = g.host()["recon_s"].copy()
+        g.step(x)
+        h = g.host()
+        assert np.array_equal(h["recon_s"], before) and np.array_equal(h["recon_r"], before)
+        assert not np.any(h["scales"]) and not np.any(h["err"])
+
+
+@pytest.mark.parametrize("bits", [1, 2])
+def test_launch_shapes_agree_bitwise(bits):
+    """Every launch shape the override allows gives the same bits."""
+    wl = W.replace(W.WORKLOADS["flux_sp"], tokens=64, bits=bits)
+    xs = W.trajectory(wl, 2, steps=2, device="cuda")
+    ref = None
+    try:
+        for gpt, thr, bps in [(0, 0, 0), (3, 128, 0), (4, 96, 0), (2, 192, 2), (1, 384, 1), (4, 128, 0)]:
+            cf.cf_set_launch_override(0, gpt, thr, bps)
+            cf.cf_set_launch_override(1, gpt, thr, bps)
+            g = GpuBuffer(64, 3072, bits)
+            g.init(xs[0])
+            g.step(xs[1])
+            h = g.host()
+            if ref is None:
+                ref = h
+            for k in ("codes", "scales", "err", "recon_s", "recon_r"):
+                assert np.array_equal(h[k].view(np.uint8), ref[k].view(np.uint8)), (gpt, thr, k)
+    finally:
+        cf.cf_set_launch_override(0, 0, 0, 0)
+        cf.cf_set_launch_override(1, 0, 0, 0)
+
+
+def test_host_pointer_is_rejected():
+    d = cf.desc(4, 64, 1)
+    host = torch.zeros(4, 64)
+    dev = torch.zeros(4, 64, device="cuda")
+    with pytest.raises(cf.CFError) as ei:
+        cf.cf_encode(d, host.view(torch.int16), dev, dev, dev, dev)
+    assert ei.value.status == 1
+
+
+def _batched_state(wl, n, dev="cuda"):
+    T, C = wl.tokens, wl.channels
+    Wd = (C * wl.bits + 31) // 32
+    f32 = dict(dtype=torch.float32, device=dev)
+    st = dict(recon_s=torch.empty(n, T, C, **f32), recon_r=torch.empty(n, T, C, **f32),
+              err=torch.empty(n, T, C, **f32),
+              codes=torch.empty(n, T, Wd, dtype=torch.int32, device=dev),
+              scales=torch.empty(n, T, **f32))
+    return st
+
+
+def test_batched_bad_buffer_is_skipped_and_reported():
+    wl = W.replace(W.WORKLOADS["flux_sp"], tokens=32, buffers=3)
+    xs = torch.stack([W.trajectory(wl, b, steps=2, device="cuda") for b in range(3)], 1)  # [S,n,T,C]
+    st = _batched_state(wl, 3)
+    d = cf.desc(32, 3072, 2)
+    for b in range(3):
+        cf.cf_state_init(d, xs[0, b].view(torch.int16), st["recon_s"][b], st["err"][b])
+    before = st["recon_s"].clone()
+    x16 = xs[1].view(torch.int16)
+    sets = [(x16[b], st["recon_s"][b], st["err"][b], st["codes"][b], st["scales"][b]) for b in range(3)]
+    bad = list(sets[1])
+    bad[1] = st["recon_s"][1].data_ptr() + 4           # misaligned recon
+    bufs = cf.enc_buffer_array([sets[0], tuple(bad), sets[2]], "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cf.cf_encode_batched(d, 3, bufs, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 2
+    assert torch.equal(st["recon_s"][1], before[1])     # skipped buffer untouched
+    assert not torch.equal(st["recon_s"][0], before[0])
+    bad[1] = 0                                           # null pointer
+    bufs = cf.enc_buffer_array([tuple(bad)], "cuda")
+    status.zero_()
+    cf.cf_encode_batched(d, 1, bufs, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1
+
+
+@pytest.mark.parametrize("name,steps,sample", [("flux_sp", 3, (0, 57, 113))])
+def test_full_size_batched_step(name, steps, sample):
+    """The bench's launch: all buffers of a step in one batched encode and one
+    batched decode.  Sampled buffers are checked against the oracle over all
+    steps; every buffer is checked for the EF identity and for
+    receiver == sender."""
+    wl = W.WORKLOADS[name]
+    n, T, C = wl.buffers, wl.tokens, wl.channels
+    trs = [W.Trajectory(wl, b, device="cuda") for b in range(n)]
+    st = _batched_state(wl, n)
+    d = cf.desc(T, C, wl.bits)
+    x = torch.stack([t.next() for t in trs])
+    for b in range(n):
+        cf.cf_state_init(d, x[b].view(torch.int16), st["recon_s"][b], st["err"][b])
+        cf.cf_state_init(d, x[b].view(torch.int16), st["recon_r"][b], None)
+    recon_o = {b: oracle.state_init(W.bf16_bits(x[b]))[0] for b in sample}
+    x_buf = torch.empty_like(x)
+    x16 = x_buf.view(torch.int16)
+    enc = cf.enc_buffer_array([(x16[b], st["recon_s"][b], st["err"][b], st["codes"][b],
+                                st["scales"][b]) for b in range(n)], "cuda")
+    dec = cf.dec_buffer_array([(st["codes"][b], st["scales"][b], st["recon_r"][b])
+                               for b in range(n)], "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for s in range(1, steps):
+        x_buf.copy_(torch.stack([t.next() for t in trs]))
+        v = x_buf.float() - st["recon_s"]                  # one fp32 rounding, as the kernel
+        cf.cf_encode_batched(d, n, enc, status)
+        cf.cf_decode_batched(d, n, dec, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.equal(st["recon_r"].view(torch.int32), st["recon_s"].view(torch.int32))
+        # EF identity: recon_s + err == x within the three fp32 roundings
+        gap = (st["recon_s"].double() + st["err"].double() - x_buf.double()).abs()
+        bound = (v.abs().double() + st["err"].abs().double() + st["recon_s"].abs().double()) \
+            * 2.0**-24 * (1 + 1e-9) + 3 * 2.0**-149
+        assert bool((gap <= bound).all())
+        del v, gap, bound
+        for b in sample:
+            xb = W.bf16_bits(x_buf[b])
+            v, ora = oracle_step(xb, recon_o[b], wl.bits)
+            gh = dict(codes=st["codes"][b].cpu().numpy().view(np.uint32),
+                      scales=st["scales"][b].cpu().numpy(), err=st["err"][b].cpu().numpy(),
+                      recon_s=st["recon_s"][b].cpu().numpy())
+            compare_step(wl.bits, v, ora, gh)
