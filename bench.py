@@ -58,6 +58,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="budget of the oracle timing sample")
+    ap.add_argument("--buffers", type=int, default=0,
+                    help="override the buffer count (smaller cases for profiling)")
+    ap.add_argument("--gen-steps", type=int, default=0,
+                    help="distinct pre-generated steps to cycle through (0 = all that fit)")
     return ap.parse_args()
 
 
@@ -84,52 +88,75 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples while the GPU is under load."""
+    """nvidia-smi clock/throttle samples while the GPU is under load.
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Queries every GPU and keeps the rows of the one torch is using (matched
+    by UUID, else by the CUDA_VISIBLE_DEVICES ordinal, else index 0)."""
+
+    FIELDS = ("uuid,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, dev):
+        self.uuid = None
         try:
-            self.index = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+            self.uuid = str(torch.cuda.get_device_properties(dev).uuid).lower()
         except Exception:
-            self.index = str(dev.index or 0)
-        self.rows, self.proc = [], None
+            pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        k = dev.index or 0
+        self.fallback_index = ids[k] if k < len(ids) and ids[k].isdigit() else str(k)
+        self.rows, self.proc, self.note = [], None, None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        except (OSError, FileNotFoundError) as e:
+            self.proc, self.note = None, f"nvidia-smi unavailable: {e}"
 
     def _read(self):
         for line in self.proc.stdout:
             self.rows.append((time.time(), [c.strip() for c in line.split(",")]))
 
+    def _mine(self, r):
+        if self.uuid and self.uuid in r[0].lower():
+            return True
+        return False
+
     def stop(self, t0, t1):
         if self.proc is None:
-            return None
-        time.sleep(0.15)
+            return {"note": self.note}
+        time.sleep(0.25)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        rows = [r for ts, r in self.rows if t0 - 0.1 <= ts <= t1 + 0.1] or [r for _, r in self.rows]
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        allrows = [(ts, r) for ts, r in self.rows if len(r) >= 10]
+        mine = [(ts, r) for ts, r in allrows if self._mine(r)]
+        if not mine:
+            mine = [(ts, r) for ts, r in allrows if r[1] == self.fallback_index]
+        if not mine:
+            return {"note": "no nvidia-smi samples", "raw_rows": len(self.rows)}
+        win = [r for ts, r in mine if t0 - 0.15 <= ts <= t1 + 0.15]
+        rows = win or [r for _, r in mine]
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [x for x in (num(r[2]) for r in rows) if x is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({n for r in rows for n, v in zip(names, r[6:10]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][3]),
+                "reasons": reasons, "samples": len(rows),
+                "window": "timed region" if win else "whole run (timed region shorter than one sample)"}
 
 
 def kernel_source_hash():
@@ -184,6 +211,8 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     wl = W.WORKLOADS[args.workload]
+    if args.buffers:
+        wl = W.replace(wl, buffers=args.buffers)
     n, T, C, bits = wl.buffers, wl.tokens, wl.channels, wl.bits
     d = cf.desc(T, C, bits)
     Wd = cf.cf_codes_words_per_row(d)
@@ -191,6 +220,8 @@ def run_ours(args, world, rank, local):
     # Pre-generate the trajectory (as many steps as fit a 40 GB budget).
     step_bytes = n * T * C * 2
     S = max(2, min(wl.steps, int(40e9 // step_bytes)))
+    if args.gen_steps:
+        S = max(2, min(S, args.gen_steps))
     X = torch.empty((S, n, T, C), dtype=torch.bfloat16, device=dev)
     for b in range(n):
         tr = W.Trajectory(wl, b, device=dev, seed=rank)

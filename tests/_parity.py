@@ -60,8 +60,8 @@ def compare_step(bits, v_oracle, ora, gpu, stats=None):
     for key in ("recon_s", "err", "recon_r"):
         if key not in gpu:
             continue
-        o, g = ora[key].astype(np.float64), gpu[key].astype(np.float64)
         ref = ora["recon_s"] if key == "recon_r" else ora[key]
+        o, g = ref.astype(np.float64), gpu[key].astype(np.float64)
         rowmax = np.max(np.abs(ref.astype(np.float64)), axis=1, keepdims=True) if C else 0
         assert np.all(np.abs(g - o) <= STATE_RTOL * rowmax + 1e-37), \
             f"{key} mismatch: max abs diff {np.max(np.abs(g - o))}"

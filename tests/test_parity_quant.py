@@ -25,12 +25,12 @@ def _run_trajectory(wl, buffer, steps, stats=None):
     xs = W.trajectory(wl, buffer, steps=steps, device="cuda")
     xb = [W.bf16_bits(x) for x in xs]
     g = GpuBuffer(wl.tokens, wl.channels, wl.bits)
-    g.init(xs[0])
+    g.init(xs[0].clone())
     recon_o, _ = oracle.state_init(xb[0])
     h = g.host()
     assert np.array_equal(h["recon_s"], recon_o) and not np.any(h["err"])
     for s in range(1, steps):
-        g.step(xs[s])
+        g.step(xs[s].clone())          # a fresh allocation is 16-byte aligned
         v, ora = oracle_step(xb[s], recon_o, wl.bits)
         gh = g.host()
         compare_step(wl.bits, v, ora, gh, stats)
