@@ -1,6 +1,9 @@
-// lowrank_api.cuh -- internal interface between the C-ABI translation unit
-// and the low-rank implementation (lowrank.cu).
+// lowrank_api.cuh -- internal interface of the low-rank implementation:
+// limits, tile constants and the workspace layout.
 #pragma once
+
+#include <stddef.h>
+#include <stdint.h>
 
 #include "cf.h"
 
@@ -9,7 +12,27 @@ namespace cf_lowrank {
 constexpr int kMaxRank = 64;
 constexpr int kMaxIters = 16;
 
+constexpr int64_t kChunkA = 512;   // channels per split of the Y = V Q pass
+constexpr int64_t kChunkB = 256;   // tokens per split of the Q = V^T P pass
+constexpr int kGramTok = 64;       // tokens per partial Gram block
+constexpr int kApplyTok = 32;      // D tile: tokens
+constexpr int kApplyCh = 256;      // D tile: channels
+constexpr int kApplyThreads = 256;
+
+// Workspace layout (byte offsets, each region 256-byte aligned).  rp is
+// the rank padded to a multiple of 16 (MMA N granularity); Tp the token
+// count padded to a multiple of 8 (16-byte rows of the bf16 P^T copy).
+struct Layout {
+    int64_t T, C;
+    int r, rp;
+    int64_t Tp;
+    int splitsA, splitsB, nGram;
+    size_t off_status, off_gp, off_rinv, off_amax, off_vb, off_qt, off_yp, off_y, off_p, off_pt,
+        off_zp, off_q, total;
+};
+
 // Descriptor checks shared by cf_payload_bytes and the low-rank entry points.
 cf_status check_desc(const cf_desc *d);
+Layout make_layout(int64_t T, int64_t C, int r);
 
 }  // namespace cf_lowrank

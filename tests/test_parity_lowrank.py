@@ -1,0 +1,173 @@
+"""GPU parity of the low-rank mode (cf_lowrank_encode / cf_lowrank_decode)
+against the fp64 CPU oracle, through the C ABI.
+
+Bar: the relative Frobenius error ||V - D||_F / ||V||_F of the GPU payload is
+within 1% of the oracle's on the same input (teacher-forced: both sides start
+each step from the GPU's pre-step state).  Also checked at every step: the
+error-feedback identity recon_s + err == x, receiver == sender bit for bit,
+INT4 codes in [-7, 7] with the column maximum at +-7, and the payload ratio.
+"""
+import numpy as np
+import pytest
+import torch
+
+from activation_residual_compression_cf_b200 import cf
+from activation_residual_compression_cf_b200 import workloads as W
+from oracle import lowrank as L
+
+pytestmark = pytest.mark.gpu
+
+REL_FROB_TOL = 0.01
+
+
+class GpuLowrank:
+    def __init__(self, T, C, r, iters, dev="cuda"):
+        self.d = cf.desc(T, C, 0, r, iters)
+        self.T, self.C, self.r = T, C, r
+        nb = (r + 1) // 2
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.recon_s = torch.empty(T, C, **f32)
+        self.recon_r = torch.empty(T, C, **f32)
+        self.err = torch.empty(T, C, **f32)
+        self.pc = torch.empty(T * nb + 16, dtype=torch.uint8, device=dev)
+        self.qc = torch.empty(C * nb + 16, dtype=torch.uint8, device=dev)
+        self.ps = torch.empty(r, **f32)
+        self.qs = torch.empty(r, **f32)
+        self.ws = torch.empty(cf.cf_lowrank_workspace_bytes(self.d), dtype=torch.uint8, device=dev)
+
+    def init(self, x0):
+        cf.cf_state_init(self.d, x0.view(torch.int16), self.recon_s, self.err)
+        cf.cf_state_init(self.d, x0.view(torch.int16), self.recon_r, None)
+
+    def step(self, x, omega):
+        cf.cf_lowrank_encode(self.d, x.view(torch.int16), self.recon_s, self.err, omega,
+                             self.pc, self.ps, self.qc, self.qs, self.ws)
+        cf.cf_lowrank_decode(self.d, self.pc, self.ps, self.qc, self.qs, self.recon_r)
+
+    def payload(self):
+        nb = (self.r + 1) // 2
+        return (self.pc[: self.T * nb].cpu().numpy().reshape(self.T, nb), self.ps.cpu().numpy(),
+                self.qc[: self.C * nb].cpu().numpy().reshape(self.C, nb), self.qs.cpu().numpy())
+
+
+def _rel_err(v, d):
+    v64 = v.astype(np.float64)
+    return np.linalg.norm(v64 - d.astype(np.float64)) / np.linalg.norm(v64)
+
+
+def _check_codes(packed, scales, r):
+    q = L.int4_unpack(packed, r)
+    assert q.min() >= -7 and q.max() <= 7
+    live = scales > 0
+    assert np.all(np.abs(q[:, live]).max(axis=0) == 7)
+    assert not np.any(q[:, ~live])
+
+
+def _run(wl, steps, buffer=0, check_frob=True):
+    T, C, r, it = wl.tokens, wl.channels, wl.rank, wl.iters
+    xs = W.trajectory(wl, buffer, steps=steps, device="cuda")
+    g = GpuLowrank(T, C, r, it)
+    g.init(xs[0].clone())
+    errs = []
+    for s in range(1, steps):
+        x = xs[s].clone()
+        om = W.omega(wl, buffer, s, device="cuda")
+        recon_before = g.recon_s.cpu().numpy()
+        g.step(x, om)
+        torch.cuda.synchronize()
+        assert cf.cf_lowrank_status(g.ws) in (0,)
+        xb = W.bf16_bits(x)
+        xf = L.bf16_bits_to_f32(xb)
+        v = (xf - recon_before).astype(np.float32)
+        rs, er, rr = g.recon_s.cpu().numpy(), g.err.cpu().numpy(), g.recon_r.cpu().numpy()
+        # D as the GPU applied it, and the EF identity
+        d_gpu = (rs.astype(np.float64) - recon_before)
+        gap = np.abs(rs.astype(np.float64) + er - xf)
+        assert gap.max() <= 4 * np.spacing(np.float32(np.abs(xf).max() + np.abs(v).max()))
+        assert np.array_equal(rr.view(np.uint32), rs.view(np.uint32))
+        pc, ps, qc, qs = g.payload()
+        _check_codes(pc, ps, r)
+        _check_codes(qc, qs, r)
+        # the D the payload encodes (oracle reconstruction of the GPU payload)
+        d_pay = L.reconstruct(pc, ps, qc, qs, r)
+        tol = 4 * np.spacing(np.float32(np.abs(rs).max())) + 1e-5 * np.abs(d_pay).max()
+        assert np.max(np.abs(d_pay - d_gpu)) <= tol
+        # oracle on the same input
+        ro = recon_before.copy()
+        out = L.lowrank_encode(xb, ro, om.cpu().numpy(), it)
+        e_gpu, e_ora = _rel_err(v, d_pay), _rel_err(out["V"], out["D"])
+        errs.append((e_gpu, e_ora))
+        if check_frob:
+            assert abs(e_gpu - e_ora) <= REL_FROB_TOL * e_ora, (s, e_gpu, e_ora)
+    return errs
+
+
+def test_small_lowrank_trajectory():
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=256, channels=192, rank=8)
+    _run(wl, 4)
+
+
+@pytest.mark.parametrize("T,C,r,iters", [(100, 200, 5, 1), (300, 136, 16, 3), (77, 64, 33, 2),
+                                         (640, 512, 64, 2), (1000, 1000, 32, 2)])
+def test_lowrank_ragged_shapes(T, C, r, iters):
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r, iters=iters)
+    _run(wl, 3)
+
+
+def test_lowrank_full_size_sampled():
+    """The low-rank workload at full size (4096 x 3072, rank 32, 2
+    iterations), one buffer, three compressed steps."""
+    errs = _run(W.WORKLOADS["lowrank"], 4, buffer=7)
+    assert all(e < 0.5 for e, _ in errs)
+
+
+def test_lowrank_zero_residual_and_status():
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=128, channels=64, rank=4)
+    x = W.trajectory(wl, 0, steps=1, device="cuda")[0].clone()
+    g = GpuLowrank(128, 64, 4, 2)
+    g.init(x)
+    before = g.recon_s.clone()
+    g.step(x, W.omega(wl, 0, 1, device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(g.recon_s, before) and torch.equal(g.recon_r, before)
+    assert not bool(g.err.any())
+    assert cf.cf_lowrank_status(g.ws) == 6          # CF_ERR_NUMERIC: Y has no rank
+    assert cf.cf_lowrank_status(g.ws) == 0          # cleared by the read
+
+
+def test_lowrank_exact_rank_input():
+    """A residual of rank 3 < r: Y has only 3 independent columns, the other
+    Cholesky pivots are dead (status CF_ERR_NUMERIC, zero P columns), and the
+    remaining error is the INT4 factor error, within 1% of the oracle's."""
+    T, C, r = 256, 128, 8
+    g = GpuLowrank(T, C, r, 2)
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    x0 = torch.zeros(T, C, dtype=torch.bfloat16, device="cuda")
+    g.init(x0)
+    u = torch.randn(T, 3, generator=gen, device="cuda")
+    w = torch.randn(C, 3, generator=gen, device="cuda")
+    x = (u @ w.T).to(torch.bfloat16)
+    om = torch.randn(C, r, generator=gen, device="cuda")
+    g.step(x, om)
+    torch.cuda.synchronize()
+    assert cf.cf_lowrank_status(g.ws) == 6
+    xb = W.bf16_bits(x)
+    v = L.bf16_bits_to_f32(xb)
+    d = g.recon_s.cpu().numpy()
+    ro = np.zeros((T, C), np.float32)
+    out = L.lowrank_encode(xb, ro, om.cpu().numpy(), 2)
+    e_gpu, e_ora = _rel_err(v, d), _rel_err(out["V"], out["D"])
+    assert abs(e_gpu - e_ora) <= REL_FROB_TOL * e_ora, (e_gpu, e_ora)
+    pc, ps, qc, qs = g.payload()
+    assert int((ps > 0).sum()) == 3 and int((qs > 0).sum()) == 3
+
+
+def test_workspace_too_small_is_rejected():
+    g = GpuLowrank(64, 64, 4, 1)
+    small = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    x = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
+    om = torch.zeros(64, 4, device="cuda")
+    with pytest.raises(cf.CFError) as ei:
+        cf.cf_lowrank_encode(g.d, x.view(torch.int16), g.recon_s, g.err, om, g.pc, g.ps, g.qc,
+                             g.qs, small)
+    assert ei.value.status == 4
