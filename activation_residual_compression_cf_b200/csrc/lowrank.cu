@@ -18,13 +18,17 @@
 //
 // The workspace is caller-allocated (cf_lowrank_workspace_bytes); its
 // layout is computed here from (T, C, r).
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <atomic>
 
 #include "cf.h"
 #include "cf_common.cuh"
 #include "lowrank_api.cuh"
 #include "lowrank_kernels.cuh"
+#include "lowrank_umma.cuh"
 
 namespace cf_lowrank {
 
@@ -109,6 +113,107 @@ int sm_count() {
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     return n;
+}
+
+std::atomic<int> g_engine{0};  // 0 = tensor cores (tcgen05), 1 = CUDA cores
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::atomic<bool> tried{false};
+    if (!fn && !tried.exchange(true)) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            (void)cudaGetLastError();
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows][cols] array (row pitch `pitch`
+// elements), box {64 columns, box_rows rows}, 128-byte swizzle, zero fill
+// outside the array.
+bool make_map(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, int64_t pitch,
+              uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)pitch * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN>
+cf_status launch_project(const Layout &L, const __nv_bfloat16 *vb, const __nv_bfloat16 *qt,
+                         float *yp, int32_t *status, cudaStream_t st) {
+    CUtensorMap mv, mq;
+    if (!make_map(&mv, vb, L.C, L.T, L.C, 128) || !make_map(&mq, qt, L.C, L.rp, L.C, BN))
+        return CF_ERR_CUDA;
+    auto k = cf::umma::project_kernel<BN>;
+    const int smem = cf::umma::StageGeom<BN>::kSmem;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return CF_ERR_CUDA;
+    dim3 grid((unsigned)((L.T + 127) / 128), (unsigned)L.splitsA);
+    k<<<grid, 128, smem, st>>>(mv, mq, yp, L.T, L.C, kChunkA, status);
+    return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
+}
+
+template <int BN>
+cf_status launch_backproject(const Layout &L, const __nv_bfloat16 *vb, const __nv_bfloat16 *pt,
+                             float *zp, int32_t *status, cudaStream_t st) {
+    CUtensorMap mv, mp;
+    if (!make_map(&mv, vb, L.C, L.T, L.C, 64) || !make_map(&mp, pt, L.Tp, L.rp, L.Tp, BN))
+        return CF_ERR_CUDA;
+    auto k = cf::umma::backproject_kernel<BN>;
+    const int smem = cf::umma::StageGeom<BN>::kSmem;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return CF_ERR_CUDA;
+    dim3 grid((unsigned)((L.C + 127) / 128), (unsigned)L.splitsB);
+    k<<<grid, 128, smem, st>>>(mv, mp, zp, L.T, L.C, kChunkB, status);
+    return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
+}
+
+cf_status project(const Layout &L, const __nv_bfloat16 *vb, const __nv_bfloat16 *qt, float *yp,
+                  int32_t *status, cudaStream_t st) {
+    if (g_engine.load() == 0) {
+        switch (L.rp) {
+            case 16: return launch_project<16>(L, vb, qt, yp, status, st);
+            case 32: return launch_project<32>(L, vb, qt, yp, status, st);
+            case 48: return launch_project<48>(L, vb, qt, yp, status, st);
+            case 64: return launch_project<64>(L, vb, qt, yp, status, st);
+        }
+    }
+    cf::lr_project_simt<<<dim3((unsigned)((L.T + 63) / 64), (unsigned)L.splitsA), 256, 0, st>>>(
+        vb, qt, yp, L.T, L.C, L.rp);
+    return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
+}
+
+cf_status backproject(const Layout &L, const __nv_bfloat16 *vb, const __nv_bfloat16 *pt, float *zp,
+                      int32_t *status, cudaStream_t st) {
+    if (g_engine.load() == 0) {
+        switch (L.rp) {
+            case 16: return launch_backproject<16>(L, vb, pt, zp, status, st);
+            case 32: return launch_backproject<32>(L, vb, pt, zp, status, st);
+            case 48: return launch_backproject<48>(L, vb, pt, zp, status, st);
+            case 64: return launch_backproject<64>(L, vb, pt, zp, status, st);
+        }
+    }
+    cf::lr_backproject_simt<<<dim3((unsigned)((L.C + 63) / 64), (unsigned)L.splitsB), 256, 0, st>>>(
+        vb, pt, zp, L.T, L.Tp, L.C, L.rp);
+    return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 
 template <class T>
@@ -200,9 +305,7 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
         LR_LAUNCHED();
     }
     for (int it = 0; it < d->iters; ++it) {
-        cf::lr_project_simt<<<dim3((unsigned)((T + 63) / 64), (unsigned)L.splitsA), 256, 0, st>>>(
-            vb, qt, yp, T, C, rp);
-        LR_LAUNCHED();
+        LR_TRY(project(L, vb, qt, yp, status, st));
         cf::lr_reduce_gram_kernel<<<(unsigned)L.nGram, 256, 0, st>>>(yp, y, gp, T, rp, L.splitsA);
         LR_LAUNCHED();
         {
@@ -216,9 +319,7 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
         const int64_t np = (int64_t)L.Tp * rp;
         cf::lr_orth_kernel<<<(unsigned)((np + 255) / 256), 256, 0, st>>>(y, rinv, p, pt, T, L.Tp, r, rp);
         LR_LAUNCHED();
-        cf::lr_backproject_simt<<<dim3((unsigned)((C + 63) / 64), (unsigned)L.splitsB), 256, 0, st>>>(
-            vb, pt, zp, T, L.Tp, C, rp);
-        LR_LAUNCHED();
+        LR_TRY(backproject(L, vb, pt, zp, status, st));
         const int64_t nz = C * rp;
         cf::lr_reduce_q_kernel<<<(unsigned)((nz + 255) / 256), 256, 0, st>>>(zp, q, qt, C, rp, L.splitsB);
         LR_LAUNCHED();
@@ -249,6 +350,12 @@ cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes, const floa
     const Layout L = make_layout(d->tokens, d->channels, d->rank);
     return apply(false, L, nullptr, recon_r, nullptr, p_codes, p_scales, q_codes, q_scales,
                  (cudaStream_t)stream);
+}
+
+cf_status cf_set_lowrank_engine(int32_t engine) {
+    if (engine < 0 || engine > 1) return CF_ERR_INVALID_ARG;
+    g_engine.store(engine);
+    return CF_OK;
 }
 
 cf_status cf_lowrank_status(void *workspace, void *stream) {

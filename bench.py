@@ -51,8 +51,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="flux_sp", choices=[k for k, v in W.WORKLOADS.items()
-                                                               if v.mode == "quant"])
+    ap.add_argument("--workload", default="flux_sp", choices=list(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -335,6 +334,115 @@ def run_ours(args, world, rank, local):
     return out
 
 
+def run_lowrank(args, world, rank, local):
+    """Low-rank mode: per step, cf_lowrank_encode then cf_lowrank_decode for
+    every buffer (one workspace, reused in stream order)."""
+    from activation_residual_compression_cf_b200 import build, cf
+    build.build()
+    cf.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = W.WORKLOADS[args.workload]
+    if args.buffers:
+        wl = W.replace(wl, buffers=args.buffers)
+    n, T, C, r, it = wl.buffers, wl.tokens, wl.channels, wl.rank, wl.iters
+    d = cf.desc(T, C, 0, r, it)
+    step_bytes = n * T * C * 2
+    S = max(2, min(wl.steps, int(30e9 // step_bytes)))
+    if args.gen_steps:
+        S = max(2, min(S, args.gen_steps))
+    X = torch.empty((S, n, T, C), dtype=torch.bfloat16, device=dev)
+    OM = torch.empty((S, n, C, r), dtype=torch.float32, device=dev)
+    for b in range(n):
+        tr = W.Trajectory(wl, b, device=dev, seed=rank)
+        for s in range(S):
+            X[s, b] = tr.next()
+            OM[s, b] = W.omega(wl, b, s, device=dev, seed=rank)
+    f32 = dict(dtype=torch.float32, device=dev)
+    recon_s = torch.empty((n, T, C), **f32)
+    recon_r = torch.empty((n, T, C), **f32)
+    err = torch.empty((n, T, C), **f32)
+    nb = (r + 1) // 2
+    pc = torch.empty((n, T * nb + 16), dtype=torch.uint8, device=dev)
+    qc = torch.empty((n, C * nb + 16), dtype=torch.uint8, device=dev)
+    ps = torch.empty((n, max(r, 4)), **f32)
+    qs = torch.empty((n, max(r, 4)), **f32)
+    ws = torch.empty(cf.cf_lowrank_workspace_bytes(d), dtype=torch.uint8, device=dev)
+    X16 = X.view(torch.int16)
+    for b in range(n):
+        cf.cf_state_init(d, X16[0, b], recon_s[b], err[b])
+        cf.cf_state_init(d, X16[0, b], recon_r[b], None)
+    stream = torch.cuda.current_stream(dev)
+
+    def enc(i):
+        s = 1 + i % (S - 1)
+        for b in range(n):
+            cf.cf_lowrank_encode(d, X16[s, b], recon_s[b], err[b], OM[s, b], pc[b], ps[b],
+                                 qc[b], qs[b], ws, stream=stream)
+
+    def dec():
+        for b in range(n):
+            cf.cf_lowrank_decode(d, pc[b], ps[b], qc[b], qs[b], recon_r[b], stream=stream)
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for i in range(args.warmup):
+        enc(i)
+        dec()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    for i in range(args.steps):
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        enc(args.warmup + i)
+        e1.record(stream)
+        dec()
+        e2.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop(wall0, time.time())
+    ms = ev[0][0].elapsed_time(ev[-1][2])
+    enc_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    dec_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    peak, peak_kind = peaks()
+    value = 2 * T * C * n * args.steps * world / (ms / 1e3) / 1e9
+    enc_bytes = n * T * C * 14
+    dec_bytes = n * T * C * 8
+    status = cf.cf_lowrank_status(ws)
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 in, fp32 state, bf16 tensor products", "data": "synthetic",
+        "config": {"workload": args.workload, "tokens": T, "channels": C, "buffers": n,
+                   "rank": r, "iters": it, "mode": "low-rank INT4 + EF",
+                   "parallelism": f"replicas x{world}", "l2": "inputs larger than L2",
+                   "launches_per_step": None},
+        "roofline": {"bound": "hbm", "achieved": round(enc_bytes / (enc_ms / 1e3) / 1e9, 1),
+                     "peak": peak, "unit": "GB/s",
+                     "frac": round(enc_bytes / (enc_ms / 1e3) / 1e9 / peak, 4), "traffic": None,
+                     "kernel": "cf_lowrank_encode (whole call, 14 B/elem unavoidable I/O)",
+                     "peak_kind": peak_kind},
+        "decode": {"achieved": round(dec_bytes / (dec_ms / 1e3) / 1e9, 1),
+                   "frac": round(dec_bytes / (dec_ms / 1e3) / 1e9 / peak, 4),
+                   "avg_ms_per_step": round(dec_ms, 4)},
+        "encode_ms_per_step": round(enc_ms, 4), "lowrank_status": status,
+        "payload_ratio": round(2 * T * C / cf.cf_payload_bytes(d), 2),
+        "cpu_baseline": None, "e2e": None, "gpu_launches": None, "clocks": clocks,
+    }
+    return out
+
+
 def run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, status):
     n, T, C = wl.buffers, wl.tokens, wl.channels
     # Two host steps of pinned input (buffer 0's trajectory replicated over
@@ -427,7 +535,10 @@ def main():
         return
     world, rank, local = dist_setup(args)
     try:
-        out = run_ours(args, world, rank, local)
+        if W.WORKLOADS[args.workload].mode == "lowrank":
+            out = run_lowrank(args, world, rank, local)
+        else:
+            out = run_ours(args, world, rank, local)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

@@ -66,7 +66,8 @@ typedef enum cf_status {
     CF_ERR_WORKSPACE = 4,    /* low-rank workspace too small                 */
     CF_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed         */
     CF_ERR_NUMERIC = 6,      /* low-rank: Gram matrix not positive definite */
-    CF_ERR_TIMEOUT = 7       /* reserved: a bounded device wait gave up      */
+    CF_ERR_TIMEOUT = 7       /* a bounded device wait gave up (tensor-core
+                                products); recorded in the workspace status */
 } cf_status;
 
 /* Problem description, as the pages state the problem: one exchanged
@@ -193,6 +194,13 @@ cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes,
  * cf_lowrank_encode on `workspace` recorded (CF_OK or CF_ERR_NUMERIC) and
  * clears it.  Returns CF_ERR_CUDA if the copy or the sync fails. */
 cf_status cf_lowrank_status(void *workspace, void *stream);
+
+/* Engine of the two subspace-iteration products in this process: 0 (the
+ * default) = tcgen05 tensor cores (bf16 operands, fp32 accumulation in
+ * TMEM), 1 = CUDA cores (same bf16 operands, fp32 FMA).  For cross-checks
+ * and diagnosis; both satisfy the same parity bar.  Returns
+ * CF_ERR_INVALID_ARG for any other value. */
+cf_status cf_set_lowrank_engine(int32_t engine);
 
 /* Launch-shape override for tuning sweeps: kernel 0 = encode, 1 = decode;
  * groups_per_thread in 1..4 (8 channels per group), threads a multiple of

@@ -144,9 +144,11 @@ def test_lowrank_exact_rank_input():
     gen = torch.Generator(device="cuda").manual_seed(5)
     x0 = torch.zeros(T, C, dtype=torch.bfloat16, device="cuda")
     g.init(x0)
-    u = torch.randn(T, 3, generator=gen, device="cuda")
-    w = torch.randn(C, 3, generator=gen, device="cuda")
+    # small integers: u w^T is exact in bf16, so the input has rank exactly 3
+    u = torch.randint(-3, 4, (T, 3), generator=gen, device="cuda").float()
+    w = torch.randint(-3, 4, (C, 3), generator=gen, device="cuda").float()
     x = (u @ w.T).to(torch.bfloat16)
+    assert torch.equal(x.float(), u @ w.T)
     om = torch.randn(C, r, generator=gen, device="cuda")
     g.step(x, om)
     torch.cuda.synchronize()
@@ -160,6 +162,38 @@ def test_lowrank_exact_rank_input():
     assert abs(e_gpu - e_ora) <= REL_FROB_TOL * e_ora, (e_gpu, e_ora)
     pc, ps, qc, qs = g.payload()
     assert int((ps > 0).sum()) == 3 and int((qs > 0).sum()) == 3
+
+
+@pytest.mark.parametrize("T,C,r", [(4096, 3072, 32), (300, 136, 16), (640, 512, 64), (77, 64, 33)])
+def test_tensor_core_and_cuda_core_products_agree(T, C, r):
+    """The tcgen05 products and the CUDA-core products read the same bf16
+    operands and accumulate in fp32; the payloads they produce agree up to
+    summation order, and both meet the oracle bar."""
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r)
+    xs = W.trajectory(wl, 3, steps=2, device="cuda")
+    om = W.omega(wl, 3, 1, device="cuda")
+    outs = []
+    try:
+        for engine in (1, 0):
+            cf.cf_set_lowrank_engine(engine)
+            g = GpuLowrank(T, C, r, 2)
+            g.init(xs[0].clone())
+            g.step(xs[1].clone(), om)
+            torch.cuda.synchronize()
+            assert cf.cf_lowrank_status(g.ws) == 0
+            outs.append((g.payload(), g.recon_s.cpu().numpy()))
+    finally:
+        cf.cf_set_lowrank_engine(0)
+    (p1, r1), (p0, r0) = outs
+    # per-column scales of the weak (noise) directions may rotate with the
+    # summation order; the leading columns and the product must agree
+    assert np.allclose(p0[1][:8], p1[1][:8], rtol=1e-3)
+    d0 = L.reconstruct(p0[0], p0[1], p0[2], p0[3], r)
+    d1 = L.reconstruct(p1[0], p1[1], p1[2], p1[3], r)
+    v = L.bf16_bits_to_f32(W.bf16_bits(xs[1])) - L.bf16_bits_to_f32(W.bf16_bits(xs[0]))
+    e0, e1 = _rel_err(v, d0), _rel_err(v, d1)
+    assert abs(e0 - e1) <= REL_FROB_TOL * e1, (e0, e1)
+    assert np.linalg.norm(d0 - d1) <= 5e-2 * np.linalg.norm(d1)
 
 
 def test_workspace_too_small_is_rejected():
