@@ -26,7 +26,8 @@ EXPORTS = ("cf_status_string", "cf_abi_version", "cf_codes_words_per_row",
            "cf_payload_bytes", "cf_state_init", "cf_encode", "cf_decode",
            "cf_encode_batched", "cf_decode_batched", "cf_lowrank_workspace_bytes",
            "cf_lowrank_factor_bytes", "cf_lowrank_encode", "cf_lowrank_decode",
-           "cf_lowrank_status", "cf_set_lowrank_engine", "cf_set_launch_override")
+           "cf_lowrank_status", "cf_set_lowrank_engine", "cf_set_quant_pipeline",
+           "cf_set_launch_override")
 
 
 class CFError(RuntimeError):
@@ -83,6 +84,7 @@ def lib():
             "cf_lowrank_status": ([vp, vp], ctypes.c_int),
             "cf_set_launch_override": ([i32, i32, i32, i32], ctypes.c_int),
             "cf_set_lowrank_engine": ([i32], ctypes.c_int),
+            "cf_set_quant_pipeline": ([i32, i32, i32], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -186,6 +188,10 @@ def cf_lowrank_status(workspace, stream=None) -> int:
 
 def cf_set_lowrank_engine(engine: int):
     _chk(lib().cf_set_lowrank_engine(engine), "cf_set_lowrank_engine")
+
+
+def cf_set_quant_pipeline(kernel: int, pipeline: int, stages: int = 0):
+    _chk(lib().cf_set_quant_pipeline(kernel, pipeline, stages), "cf_set_quant_pipeline")
 
 
 def cf_set_launch_override(kernel: int, groups_per_thread: int = 0, threads: int = 0,

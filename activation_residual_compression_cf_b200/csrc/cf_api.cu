@@ -10,6 +10,7 @@
 #include "cf.h"
 #include "lowrank_api.cuh"
 #include "quant_kernels.cuh"
+#include "quant_tma.cuh"
 
 namespace {
 
@@ -23,6 +24,8 @@ struct Override {
     int gpt = 0, threads = 0, blocks_per_sm = 0;
 };
 Override g_override[2];
+int g_pipeline[2] = {1, 1};  // 0 = register-resident rows, 1 = TMA row staging (default)
+int g_stages[2] = {0, 0};    // TMA ring depth (0 = built-in choice)
 std::mutex g_mu;
 
 int device_sm_count() {
@@ -137,9 +140,52 @@ cf_status launch_decode_t(const Src &src, int64_t T, int64_t C, int64_t rows, in
     return launch_result();
 }
 
+// TMA-staged variants: C % 8 == 0 (16-byte rows) and, for decode, 16-byte
+// code rows (W % 4 == 0); at most 480 consumer threads.
+template <bool ENC, int BITS, int GPT, class Src>
+cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t *status,
+                     const Shape &s, int stages_req, cudaStream_t st) {
+    const int64_t W = (C * BITS + 31) / 32;
+    const int64_t slot = ENC ? 6 * C : 4 * W + 4 * C;
+    int stages = stages_req > 0 ? stages_req : (int)(100000 / slot);
+    if (stages > 8) stages = 8;
+    if (stages < 2) stages = 2;
+    const size_t smem = (size_t)stages * slot + 16 * (size_t)stages;
+    const int threads = 32 + s.threads;
+    void (*k)(Src, int64_t, int64_t, int64_t, int32_t *, int);
+    if constexpr (ENC)
+        k = cf::tma::encode_tma_kernel<BITS, GPT, Src>;
+    else
+        k = cf::tma::decode_tma_kernel<BITS, GPT, Src>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return CF_ERR_CUDA;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, threads, smem) != cudaSuccess || occ < 1) {
+        (void)cudaGetLastError();
+        occ = 1;
+    }
+    if (s.blocks_per_sm > 0 && s.blocks_per_sm < occ) occ = s.blocks_per_sm;
+    int64_t grid = (int64_t)device_sm_count() * occ;
+    if (grid > rows) grid = rows;
+    if (grid < 1) grid = 1;
+    k<<<(unsigned)grid, threads, smem, st>>>(src, T, C, rows, status, stages);
+    return launch_result();
+}
+
 template <bool ENC, int BITS, int GPT, bool VEC, class Src>
 cf_status launch_one(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t *status,
                      const Shape &s, cudaStream_t st) {
+    if constexpr (VEC) {
+        int pipe, stages;
+        {
+            std::lock_guard<std::mutex> lk(g_mu);
+            pipe = g_pipeline[ENC ? 0 : 1];
+            stages = g_stages[ENC ? 0 : 1];
+        }
+        const bool codes_ok = ENC || ((C * BITS + 31) / 32) % 4 == 0;
+        if (pipe == 1 && codes_ok && s.threads <= 480 && 2 * (ENC ? 6 * C : 4 * C + C * BITS / 8) <= 200000)
+            return launch_tma<ENC, BITS, GPT>(src, T, C, rows, status, s, stages, st);
+    }
     if constexpr (ENC)
         return launch_encode_t<BITS, GPT, VEC>(src, T, C, rows, status, s, st);
     else
@@ -269,6 +315,16 @@ cf_status cf_decode_batched(const cf_desc *d, int32_t n, const cf_dec_buffer *bu
     cf::DecArray src{bufs_dev};
     return dispatch<false>(src, d->bits, d->tokens, d->channels, d->tokens * (int64_t)n,
                            status_dev, (cudaStream_t)stream);
+}
+
+cf_status cf_set_quant_pipeline(int32_t kernel, int32_t pipeline, int32_t stages) {
+    if (kernel < 0 || kernel > 1) return CF_ERR_INVALID_ARG;
+    if (pipeline < 0 || pipeline > 1) return CF_ERR_INVALID_ARG;
+    if (stages < 0 || stages == 1 || stages > 8) return CF_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_pipeline[kernel] = pipeline;
+    g_stages[kernel] = stages;
+    return CF_OK;
 }
 
 cf_status cf_set_launch_override(int32_t kernel, int32_t groups_per_thread, int32_t threads,

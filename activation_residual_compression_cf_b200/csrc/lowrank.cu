@@ -62,7 +62,7 @@ Layout make_layout(int64_t T, int64_t C, int r) {
     };
     L.off_status = take(16);
     L.off_gp = take((size_t)L.nGram * L.rp * L.rp * 8);
-    L.off_rinv = take((size_t)L.rp * L.rp * 4);
+    L.off_rmat = take((size_t)L.rp * L.rp * 4 + (size_t)L.rp * 4);
     L.off_amax = take((size_t)2 * L.rp * 4);
     L.off_vb = take((size_t)T * C * 2);
     L.off_qt = take((size_t)L.rp * C * 2);
@@ -216,6 +216,36 @@ cf_status backproject(const Layout &L, const __nv_bfloat16 *vb, const __nv_bfloa
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 
+cf_status orth(const Layout &L, const float *y, const float *rmat, const float *rinvd, float *p,
+               __nv_bfloat16 *pt, uint32_t *amax, cudaStream_t st) {
+    const unsigned grid = (unsigned)((L.Tp + 63) / 64);
+#define CF_ORTH(RP) cf::lr_orth_kernel<RP><<<grid, 64, 0, st>>>(y, rmat, rinvd, p, pt, L.T, L.Tp, amax)
+    switch (L.rp) {
+        case 16: CF_ORTH(16); break;
+        case 32: CF_ORTH(32); break;
+        case 48: CF_ORTH(48); break;
+        case 64: CF_ORTH(64); break;
+        default: return CF_ERR_UNSUPPORTED;
+    }
+#undef CF_ORTH
+    return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
+}
+
+cf_status reduce_q(const Layout &L, const float *zp, float *q, __nv_bfloat16 *qt, uint32_t *amax,
+                   cudaStream_t st) {
+    const unsigned grid = (unsigned)((L.C + 31) / 32);
+#define CF_RQ(RP) cf::lr_reduce_q_kernel<RP><<<grid, 32, 0, st>>>(zp, q, qt, L.C, L.splitsB, amax)
+    switch (L.rp) {
+        case 16: CF_RQ(16); break;
+        case 32: CF_RQ(32); break;
+        case 48: CF_RQ(48); break;
+        case 64: CF_RQ(64); break;
+        default: return CF_ERR_UNSUPPORTED;
+    }
+#undef CF_RQ
+    return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
+}
+
 template <class T>
 T *at(void *ws, size_t off) {
     return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
@@ -224,7 +254,12 @@ T *at(void *ws, size_t off) {
 cf_status apply(bool sender, const Layout &L, const uint16_t *x, float *recon, float *err,
                 const uint8_t *pc, const float *ps, const uint8_t *qc, const float *qs,
                 cudaStream_t st) {
-    dim3 grid((unsigned)((L.C + kApplyCh - 1) / kApplyCh), (unsigned)((L.T + kApplyTok - 1) / kApplyTok));
+    const int64_t gx = (L.C + kApplyCh - 1) / kApplyCh;
+    const int64_t ntiles = (L.T + kApplyTok - 1) / kApplyTok;
+    int64_t gy = (2 * (int64_t)sm_count() + gx - 1) / gx;
+    if (gy > ntiles) gy = ntiles;
+    if (gy < 1) gy = 1;
+    dim3 grid((unsigned)gx, (unsigned)gy);
     const size_t smem = (size_t)L.r * (kApplyTok + kApplyCh) * sizeof(float);
     if (sender) {
         auto k = cf::lr_apply_kernel<true>;
@@ -280,7 +315,9 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
 
     int32_t *status = at<int32_t>(ws, L.off_status);
     double *gp = at<double>(ws, L.off_gp);
-    float *rinv = at<float>(ws, L.off_rinv);
+    float *rmat = at<float>(ws, L.off_rmat);
+    float *rinvd = rmat + rp * rp;
+    uint32_t *ticket = reinterpret_cast<uint32_t *>(status + 1);
     uint32_t *amax = at<uint32_t>(ws, L.off_amax);
     __nv_bfloat16 *vb = at<__nv_bfloat16>(ws, L.off_vb);
     __nv_bfloat16 *qt = at<__nv_bfloat16>(ws, L.off_qt);
@@ -306,29 +343,15 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
     }
     for (int it = 0; it < d->iters; ++it) {
         LR_TRY(project(L, vb, qt, yp, status, st));
-        cf::lr_reduce_gram_kernel<<<(unsigned)L.nGram, 256, 0, st>>>(yp, y, gp, T, rp, L.splitsA);
+        cf::lr_gram_chol_kernel<<<(unsigned)L.nGram, 256, 0, st>>>(
+            yp, y, gp, T, r, rp, L.splitsA, L.nGram, rmat, rinvd, ticket, status);
         LR_LAUNCHED();
-        {
-            const size_t cs = cf::lr_chol_smem_bytes(rp);
-            if (cudaFuncSetAttribute(cf::lr_chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)cs) != cudaSuccess)
-                return CF_ERR_CUDA;
-            cf::lr_chol_kernel<<<1, 256, cs, st>>>(gp, L.nGram, rinv, r, rp, status);
-        }
-        LR_LAUNCHED();
-        const int64_t np = (int64_t)L.Tp * rp;
-        cf::lr_orth_kernel<<<(unsigned)((np + 255) / 256), 256, 0, st>>>(y, rinv, p, pt, T, L.Tp, r, rp);
-        LR_LAUNCHED();
+        const bool last = (it == d->iters - 1);
+        LR_TRY(orth(L, y, rmat, rinvd, p, pt, last ? amax : nullptr, st));
         LR_TRY(backproject(L, vb, pt, zp, status, st));
-        const int64_t nz = C * rp;
-        cf::lr_reduce_q_kernel<<<(unsigned)((nz + 255) / 256), 256, 0, st>>>(zp, q, qt, C, rp, L.splitsB);
-        LR_LAUNCHED();
+        LR_TRY(reduce_q(L, zp, q, qt, last ? amax + rp : nullptr, st));
     }
-    // INT4 factors: column absmax, then quantise and pack.
-    cf::lr_absmax_kernel<<<(unsigned)((T + 255) / 256), 256, 0, st>>>(p, T, r, rp, amax);
-    LR_LAUNCHED();
-    cf::lr_absmax_kernel<<<(unsigned)((C + 255) / 256), 256, 0, st>>>(q, C, r, rp, amax + rp);
-    LR_LAUNCHED();
+    // INT4 factors: quantise and pack against the column maxima.
     const int nb = (r + 1) / 2;
     cf::lr_int4_pack_kernel<<<(unsigned)((T * nb + 255) / 256), 256, 0, st>>>(p, T, r, rp, amax, p_codes, p_scales);
     LR_LAUNCHED();

@@ -13,7 +13,7 @@ constexpr int kMaxRank = 64;
 constexpr int kMaxIters = 16;
 
 constexpr int64_t kChunkA = 512;   // channels per split of the Y = V Q pass
-constexpr int64_t kChunkB = 256;   // tokens per split of the Q = V^T P pass
+constexpr int64_t kChunkB = 512;   // tokens per split of the Q = V^T P pass
 constexpr int kGramTok = 64;       // tokens per partial Gram block
 constexpr int kApplyTok = 32;      // D tile: tokens
 constexpr int kApplyCh = 256;      // D tile: channels
@@ -27,7 +27,7 @@ struct Layout {
     int r, rp;
     int64_t Tp;
     int splitsA, splitsB, nGram;
-    size_t off_status, off_gp, off_rinv, off_amax, off_vb, off_qt, off_yp, off_y, off_p, off_pt,
+    size_t off_status, off_gp, off_rmat, off_amax, off_vb, off_qt, off_yp, off_y, off_p, off_pt,
         off_zp, off_q, total;
 };
 

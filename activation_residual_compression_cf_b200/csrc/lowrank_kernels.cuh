@@ -91,14 +91,88 @@ lr_project_simt(const bf16 *vb, const bf16 *qt, float *yp, int64_t T, int64_t C,
     }
 }
 
-// Y = sum of the split partials (fixed order), and this block's partial Gram
-// matrix Gp[blk] = Y_blk^T Y_blk in fp64 over its 64 tokens.
+// Cholesky of the rp x rp matrix in shared memory A (leading dimension ld,
+// upper triangle valid), in one warp with every column in registers:
+// lane c owns column c (r <= 32).  Step j broadcasts row j of R by
+// shuffles; no shared-memory round trips inside the factorisation.
+// On return A's upper triangle holds R and dead[j] flags dead pivots.
+template <int RPW>
+__device__ __forceinline__ void warp_cholesky_regs(double *A, int ld, int r, const double *gdiag,
+                                                   int *dead) {
+    const int lane = threadIdx.x & 31;
+    double col[RPW];
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) col[i] = (lane < r && i <= lane) ? A[i * ld + lane] : 0.0;
+#pragma unroll
+    for (int j = 0; j < RPW; ++j) {
+        if (j >= r) break;
+        const double ajj = __shfl_sync(kFullMask, col[j], j);
+        const bool bad = !(ajj > 1e-10 * gdiag[j]);
+        const double rjj = bad ? 0.0 : sqrt(ajj);
+        const double inv = bad ? 0.0 : 1.0 / rjj;
+        // row j of R: lane c > j scales its entry; lane j holds the diagonal
+        if (lane > j) col[j] *= inv;
+        if (lane == j) col[j] = rjj;
+        const double rjc = col[j];
+#pragma unroll
+        for (int i = j + 1; i < RPW; ++i) {
+            const double rji = __shfl_sync(kFullMask, rjc, i);  // R[j][i] from lane i
+            if (lane >= i) col[i] = fma(-rji, rjc, col[i]);
+        }
+        if (lane == 0) dead[j] = bad ? 1 : 0;
+    }
+#pragma unroll
+    for (int i = 0; i < RPW; ++i)
+        if (lane < r && i <= lane) A[i * ld + lane] = col[i];
+}
+
+// Same factorisation for r up to 64 with the matrix in shared memory (lane
+// l owns columns l and l + 32).
+__device__ __forceinline__ void warp_cholesky_smem(double *A, int ld, int r, const double *gdiag,
+                                                   int *dead) {
+    const int lane = threadIdx.x & 31;
+    for (int j = 0; j < r; ++j) {
+        const double ajj = A[j * ld + j];
+        const bool bad = !(ajj > 1e-10 * gdiag[j]);
+        const double rjj = bad ? 0.0 : sqrt(ajj);
+        const double inv = bad ? 0.0 : 1.0 / rjj;
+        for (int c = lane; c < r; c += 32)
+            if (c > j) A[j * ld + c] *= inv;
+        __syncwarp();
+        if (lane == 0) {
+            A[j * ld + j] = rjj;
+            dead[j] = bad ? 1 : 0;
+        }
+        for (int c = lane; c < r; c += 32) {
+            if (c <= j) continue;
+            const double rjc = A[j * ld + c];
+            for (int i = j + 1; i <= c; ++i) A[i * ld + c] = fma(-A[j * ld + i], rjc, A[i * ld + c]);
+        }
+        __syncwarp();
+    }
+}
+
+// Fused Gram + Cholesky.  Every CTA: Y = sum of the split partials (fixed
+// order) for its 64 tokens, and its partial Gram block Gp[blk] = Y^T Y
+// (upper triangle, fp64).  The last CTA to finish (atomic ticket after a
+// fence) sums the partials in block order -- deterministic -- and factors
+// G = R^T R in one warp (right-looking, lane l owns columns l and l + 32).
+// A pivot that is not above 1e-10 of its original diagonal entry marks the
+// column dead: its row of R and its inverse diagonal are zero, so P gets a
+// zero column, and CF_ERR_NUMERIC is recorded.  Output: R (fp32 [rp][rp],
+// upper) and 1/diag(R) (fp32 [rp], 0 where dead).  The ticket is reset for
+// the next iteration.
 __global__ void __launch_bounds__(256)
-lr_reduce_gram_kernel(const float *yp, float *y, double *gp, int64_t T, int rp, int splits) {
-    __shared__ float Ys[64][65];
+lr_gram_chol_kernel(const float *yp, float *y, double *gp, int64_t T, int r, int rp, int splits,
+                    int nblk, float *rmat, float *rinvd, uint32_t *ticket, int32_t *status) {
+    __shared__ double S[64 * 65];  // Y block (fp64), later the matrix being factored
+    __shared__ double gdiag[64];
+    __shared__ int dead[64];
+    __shared__ int is_last;
     const int tid = threadIdx.x;
     const int64_t t0 = (int64_t)blockIdx.x * cf_lowrank::kGramTok;
-    for (int i = tid; i < 64 * rp; i += 256) {
+    const int ldy = rp + 1;
+    for (int i = tid; i < 64 * rp; i += blockDim.x) {
         const int tt = i / rp, k = i - (i / rp) * rp;
         const int64_t t = t0 + tt;
         float v = 0.0f;
@@ -106,102 +180,141 @@ lr_reduce_gram_kernel(const float *yp, float *y, double *gp, int64_t T, int rp, 
             for (int s = 0; s < splits; ++s) v += yp[((int64_t)s * T + t) * rp + k];
             y[t * rp + k] = v;
         }
-        Ys[tt][k] = v;
+        S[tt * ldy + k] = (double)v;
     }
     __syncthreads();
     double *g = gp + (int64_t)blockIdx.x * rp * rp;
-    for (int e = tid; e < rp * rp; e += 256) {
+    for (int e = tid; e < rp * rp; e += blockDim.x) {
         const int i = e / rp, j = e - (e / rp) * rp;
+        if (i > j) continue;
         double acc = 0.0;
-        for (int tt = 0; tt < 64; ++tt) acc += (double)Ys[tt][i] * (double)Ys[tt][j];
+        for (int tt = 0; tt < 64; ++tt) acc = fma(S[tt * ldy + i], S[tt * ldy + j], acc);
         g[e] = acc;
     }
-}
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = (atomicAdd(ticket, 1u) == (uint32_t)(nblk - 1)) ? 1 : 0;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
 
-// One CTA: G = sum of the partial Grams; upper Cholesky G = R^T R in fp64;
-// Rinv = R^-1 (fp32, zero padded to rp x rp).  A pivot that is not positive,
-// or below 1e-10 of its diagonal entry (the column is numerically in the
-// span of the earlier ones), marks the column dead: its row of R and its
-// column of Rinv are zero, so P gets a zero column, and CF_ERR_NUMERIC is
-// recorded in the status word.
-__global__ void __launch_bounds__(256)
-lr_chol_kernel(const double *gp, int nblk, float *rinv, int r, int rp, int32_t *status) {
-    // dynamic shared memory: G, R, X as [rp][rp+1] fp64, then dead flags
-    extern __shared__ double dsm[];
     const int ld = rp + 1;
-    double *G = dsm;
-    double *R = G + rp * ld;
-    double *X = R + rp * ld;
-    int *dead = reinterpret_cast<int *>(X + rp * ld);
-    __shared__ int any_dead;
-    const int tid = threadIdx.x;
-    for (int e = tid; e < rp * rp; e += blockDim.x) {
-        double acc = 0.0;
-        for (int b = 0; b < nblk; ++b) acc += gp[(int64_t)b * rp * rp + e];
-        G[(e / rp) * ld + e % rp] = acc;
-    }
-    for (int e = tid; e < rp * ld; e += blockDim.x) {
-        R[e] = 0.0;
-        X[e] = 0.0;
-    }
-    if (tid == 0) any_dead = 0;
-    __syncthreads();
-    for (int j = 0; j < r; ++j) {
-        if (tid == 0) {
-            double d = G[j * ld + j];
-            for (int k = 0; k < j; ++k) d -= R[k * ld + j] * R[k * ld + j];
-            const bool bad = !(d > 0.0) || !(d > 1e-10 * G[j * ld + j]);
-            dead[j] = bad ? 1 : 0;
-            R[j * ld + j] = bad ? 0.0 : sqrt(d);
-            if (bad) any_dead = 1;
-        }
-        __syncthreads();
-        for (int i = j + 1 + tid; i < r; i += blockDim.x) {
-            double s = G[j * ld + i];
-            for (int k = 0; k < j; ++k) s -= R[k * ld + j] * R[k * ld + i];
-            R[j * ld + i] = dead[j] ? 0.0 : s / R[j * ld + j];
-        }
-        __syncthreads();
-    }
-    // X = R^-1 by back substitution, one column per thread.
-    if (tid < r) {
-        const int c = tid;
-        if (!dead[c]) {
-            X[c * ld + c] = 1.0 / R[c * ld + c];
-            for (int i = c - 1; i >= 0; --i) {
-                if (dead[i]) continue;
-                double s = 0.0;
-                for (int k = i + 1; k <= c; ++k) s += R[i * ld + k] * X[k * ld + c];
-                X[i * ld + c] = -s / R[i * ld + i];
+    double *A = S;
+    // final reduction of the partial Grams: the sum for entry e is split
+    // over 4 adjacent lanes (blocks q, q+4, ...) and combined by xor
+    // shuffles as (p0 + p1) + (p2 + p3), the same order on every run.
+    // 4 * rp * rp is a multiple of the block size, so every thread runs the
+    // same number of iterations and all lanes reach the shuffles.
+    const int ne = rp * rp;
+    for (int idx = tid; idx < 4 * ne; idx += blockDim.x) {
+        const int e = idx >> 2, q = idx & 3;
+        const int i = e / rp, j = e - (e / rp) * rp;
+        double a[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+        if (i <= j) {
+            // 8 independent accumulators keep 8 L2 loads in flight; the
+            // association order depends only on nblk, so it is reproducible
+            int b = q;
+            for (; b + 28 < nblk; b += 32) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) a[u] += __ldcg(gp + (int64_t)(b + 4 * u) * ne + e);
             }
+            for (int u = 0; b < nblk; b += 4, ++u) a[u & 7] += __ldcg(gp + (int64_t)b * ne + e);
+        }
+        double acc = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+        acc += __shfl_xor_sync(kFullMask, acc, 1);
+        acc += __shfl_xor_sync(kFullMask, acc, 2);
+        if (q == 0 && i <= j) {
+            A[i * ld + j] = acc;
+            if (i == j) gdiag[i] = acc;
         }
     }
     __syncthreads();
+    if (tid < 32) {
+        if (r <= 16)
+            warp_cholesky_regs<16>(A, ld, r, gdiag, dead);
+        else if (r <= 32)
+            warp_cholesky_regs<32>(A, ld, r, gdiag, dead);
+        else
+            warp_cholesky_smem(A, ld, r, gdiag, dead);
+    }
+    __syncthreads();
+    int nd = 0;
     for (int e = tid; e < rp * rp; e += blockDim.x) {
-        const int i = e / rp, c = e % rp;
-        rinv[e] = (i < r && c < r) ? (float)X[i * ld + c] : 0.0f;
+        const int i = e / rp, c = e - (e / rp) * rp;
+        rmat[e] = (i <= c && c < r) ? (float)A[i * ld + c] : 0.0f;
     }
-    if (tid == 0 && any_dead) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_NUMERIC);
+    for (int j = tid; j < rp; j += blockDim.x) {
+        const bool live = j < r && !dead[j];
+        rinvd[j] = live ? (float)(1.0 / A[j * ld + j]) : 0.0f;
+        nd += (j < r && dead[j]) ? 1 : 0;
+    }
+    if (nd) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_NUMERIC);
+    if (tid == 0) *ticket = 0u;
 }
 
-inline size_t lr_chol_smem_bytes(int rp) {
-    return (size_t)3 * rp * (rp + 1) * sizeof(double) + (size_t)rp * sizeof(int);
-}
-
-// P = Y Rinv (fp32 [T][rp]) and its bf16 transpose Pt [rp][Tp] (zero past T).
-__global__ void lr_orth_kernel(const float *y, const float *rinv, float *p, bf16 *pt, int64_t T,
-                               int64_t Tp, int r, int rp) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= Tp * rp) return;
-    const int64_t t = i / rp;
-    const int k = (int)(i - t * rp);
-    float v = 0.0f;
-    if (t < T && k < r) {
-        const float *yr = y + t * rp;
-        for (int j = 0; j <= k; ++j) v = fmaf(yr[j], rinv[j * rp + k], v);
+// P = Y R^-1 by forward substitution, one token row per thread:
+//   P[t][k] = (Y[t][k] - sum_{j<k} P[t][j] R[j][k]) / R[k][k]
+// written as fp32 P [T][rp] and as the bf16 transpose Pt [rp][Tp] (zero
+// past T) that the back-projection reads.  On the last iteration (amax !=
+// null) it also folds max |P[:, k]| into amax[k] (float bits, atomicMax once
+// per CTA and column).
+template <int RP>
+__global__ void __launch_bounds__(128)
+lr_orth_kernel(const float *y, const float *rmat, const float *rinvd, float *p, bf16 *pt,
+               int64_t T, int64_t Tp, uint32_t *amax) {
+    __shared__ float Rs[RP * RP];
+    __shared__ float Id[RP];
+    __shared__ float Wm[4][RP];
+    for (int i = threadIdx.x; i < RP * RP; i += blockDim.x) Rs[i] = rmat[i];
+    for (int i = threadIdx.x; i < RP; i += blockDim.x) Id[i] = rinvd[i];
+    __syncthreads();
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    float pv[RP];
+    if (t < T) {
+        const float4 *yr = reinterpret_cast<const float4 *>(y + t * RP);
+#pragma unroll
+        for (int q = 0; q < RP / 4; ++q) {
+            const float4 v = yr[q];
+            pv[4 * q] = v.x;
+            pv[4 * q + 1] = v.y;
+            pv[4 * q + 2] = v.z;
+            pv[4 * q + 3] = v.w;
+        }
+#pragma unroll
+        for (int k = 0; k < RP; ++k) {
+            float acc = pv[k];
+#pragma unroll
+            for (int j = 0; j < k; ++j) acc = fmaf(-pv[j], Rs[j * RP + k], acc);
+            pv[k] = acc * Id[k];
+        }
+        float4 *pr = reinterpret_cast<float4 *>(p + t * RP);
+#pragma unroll
+        for (int q = 0; q < RP / 4; ++q)
+            pr[q] = make_float4(pv[4 * q], pv[4 * q + 1], pv[4 * q + 2], pv[4 * q + 3]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < RP; ++k) pv[k] = 0.0f;
     }
-    if (t < T) p[t * rp + k] = v;
-    pt[(int64_t)k * Tp + t] = __float2bfloat16_rn(v);
+    if (t < Tp) {
+#pragma unroll
+        for (int k = 0; k < RP; ++k) pt[(int64_t)k * Tp + t] = __float2bfloat16_rn(pv[k]);
+    }
+    if (amax) {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+        for (int k = 0; k < RP; ++k) {
+            float m = fabsf(pv[k]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+            if (lane == 0) Wm[warp][k] = m;
+        }
+        __syncthreads();
+        for (int k = threadIdx.x; k < RP; k += blockDim.x) {
+            float m = 0.0f;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, Wm[w][k]);
+            atomicMax(amax + k, __float_as_uint(m));
+        }
+    }
 }
 
 // Zp[s][c][k] = sum over the tokens of split s of Vb[t][c] * Pt[k][t].
@@ -247,28 +360,65 @@ lr_backproject_simt(const bf16 *vb, const bf16 *pt, float *zp, int64_t T, int64_
     }
 }
 
-// Q = sum of the split partials (fixed order): fp32 [C][rp] and bf16 Qt.
-__global__ void lr_reduce_q_kernel(const float *zp, float *q, bf16 *qt, int64_t C, int rp,
-                                   int splits) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= C * rp) return;
-    const int64_t c = i / rp;
-    const int k = (int)(i - c * rp);
-    float v = 0.0f;
-    for (int s = 0; s < splits; ++s) v += zp[(int64_t)s * C * rp + i];
-    q[i] = v;
-    qt[(int64_t)k * C + c] = __float2bfloat16_rn(v);
-}
-
-// amax[k] = max over rows of |f[row][k]| as float bits (non-negative floats
-// order like their bit patterns).
-__global__ void lr_absmax_kernel(const float *f, int64_t rows, int r, int rp, uint32_t *amax) {
-    const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (int k = 0; k < r; ++k) {
-        float m = (row < rows) ? fabsf(f[row * rp + k]) : 0.0f;
+// Q = sum of the split partials (fixed order), one channel per thread:
+// fp32 Q [C][rp] and the bf16 transpose Qt [rp][C] for the next projection.
+// On the last iteration (amax != null) it folds max |Q[:, k]| into amax[k].
+template <int RP>
+__global__ void __launch_bounds__(128)
+lr_reduce_q_kernel(const float *zp, float *q, bf16 *qt, int64_t C, int splits, uint32_t *amax) {
+    __shared__ float Wm[4][RP];
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    float v[RP];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
-        if ((threadIdx.x & 31) == 0) atomicMax(amax + k, __float_as_uint(m));
+    for (int k = 0; k < RP; ++k) v[k] = 0.0f;
+    if (c < C) {
+        // splits in pairs: two rows of loads in flight per step, fixed order
+        int s = 0;
+        for (; s + 1 < splits; s += 2) {
+            const float4 *z0 = reinterpret_cast<const float4 *>(zp + ((int64_t)s * C + c) * RP);
+            const float4 *z1 = reinterpret_cast<const float4 *>(zp + ((int64_t)(s + 1) * C + c) * RP);
+#pragma unroll
+            for (int qd = 0; qd < RP / 4; ++qd) {
+                const float4 a = __ldcg(z0 + qd), b = __ldcg(z1 + qd);
+                v[4 * qd] += a.x + b.x;
+                v[4 * qd + 1] += a.y + b.y;
+                v[4 * qd + 2] += a.z + b.z;
+                v[4 * qd + 3] += a.w + b.w;
+            }
+        }
+        for (; s < splits; ++s) {
+            const float4 *zr = reinterpret_cast<const float4 *>(zp + ((int64_t)s * C + c) * RP);
+#pragma unroll
+            for (int qd = 0; qd < RP / 4; ++qd) {
+                const float4 z = __ldcg(zr + qd);
+                v[4 * qd] += z.x;
+                v[4 * qd + 1] += z.y;
+                v[4 * qd + 2] += z.z;
+                v[4 * qd + 3] += z.w;
+            }
+        }
+        float4 *qr = reinterpret_cast<float4 *>(q + c * RP);
+#pragma unroll
+        for (int qd = 0; qd < RP / 4; ++qd)
+            qr[qd] = make_float4(v[4 * qd], v[4 * qd + 1], v[4 * qd + 2], v[4 * qd + 3]);
+#pragma unroll
+        for (int k = 0; k < RP; ++k) qt[(int64_t)k * C + c] = __float2bfloat16_rn(v[k]);
+    }
+    if (amax) {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+        for (int k = 0; k < RP; ++k) {
+            float m = fabsf(v[k]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+            if (lane == 0) Wm[warp][k] = m;
+        }
+        __syncthreads();
+        for (int k = threadIdx.x; k < RP; k += blockDim.x) {
+            float m = 0.0f;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, Wm[w][k]);
+            atomicMax(amax + k, __float_as_uint(m));
+        }
     }
 }
 
@@ -302,76 +452,100 @@ __device__ __forceinline__ float int4_dequant(const uint8_t *row_codes, int k, c
     return __fmul_rn((float)q, __ldg(scales + k));
 }
 
-// D = (qP sP)(qQ sQ)^T on a 32-token x 256-channel tile, then
+// D = (qP sP)(qQ sQ)^T, then
 //   sender:   v = x - recon ; err = v - D ; recon = recon + D
 //   receiver: recon = recon + D
-// D is a fixed chain of fused multiply-adds in k order, so sender and
-// receiver form bit-identical values from the same payload.
+// A CTA owns one 256-channel slice (blockIdx.x): it dequantises that slice
+// of Q once into shared memory, then walks 32-token tiles (blockIdx.y,
+// stride gridDim.y).  Thread (w, l) owns tokens 4w..4w+3 x channels
+// 8l..8l+7 of a tile; its x/recon loads are issued before the rank-r FMA
+// loop so the HBM traffic overlaps the arithmetic.  D is a fixed chain of
+// fused multiply-adds in k order, so sender and receiver form bit-identical
+// values from the same payload.
 template <bool SENDER>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 lr_apply_kernel(const uint16_t *x, float *recon, float *err, const uint8_t *pc, const float *ps,
                 const uint8_t *qc, const float *qs, int64_t T, int64_t C, int r) {
+    constexpr int TM = cf_lowrank::kApplyTok, TN = cf_lowrank::kApplyCh;
     extern __shared__ float sm[];
-    float *As = sm;                                // [r][32]
-    float *Bs = sm + (size_t)r * cf_lowrank::kApplyTok;  // [r][256]
+    float *Bs = sm;                   // [r][TN]
+    float *As = sm + (size_t)r * TN;  // [r][TM]
     const int tid = threadIdx.x;
-    const int64_t t0 = (int64_t)blockIdx.y * cf_lowrank::kApplyTok;
-    const int64_t c0 = (int64_t)blockIdx.x * cf_lowrank::kApplyCh;
+    const int64_t c0 = (int64_t)blockIdx.x * TN;
     const int nb = (r + 1) / 2;
-    for (int i = tid; i < cf_lowrank::kApplyTok * r; i += blockDim.x) {
-        const int tt = i / r, k = i - (i / r) * r;
-        const int64_t t = t0 + tt;
-        As[k * cf_lowrank::kApplyTok + tt] = (t < T) ? int4_dequant(pc + t * nb, k, ps) : 0.0f;
-    }
-    for (int i = tid; i < cf_lowrank::kApplyCh * r; i += blockDim.x) {
+    for (int i = tid; i < TN * r; i += blockDim.x) {
         const int cc = i / r, k = i - (i / r) * r;
         const int64_t c = c0 + cc;
-        Bs[k * cf_lowrank::kApplyCh + cc] = (c < C) ? int4_dequant(qc + c * nb, k, qs) : 0.0f;
+        Bs[k * TN + cc] = (c < C) ? int4_dequant(qc + c * nb, k, qs) : 0.0f;
     }
-    __syncthreads();
     const int w = tid >> 5, l = tid & 31;
-    float acc[4][8];
+    const int64_t c = c0 + 8 * l;
+    const bool col_ok = c < C;  // C % 8 == 0: 8 channels are all in or all out
+    const int64_t ntiles = (T + TM - 1) / TM;
+    for (int64_t tile = blockIdx.y; tile < ntiles; tile += gridDim.y) {
+        const int64_t t0 = tile * TM;
+        float ro[4][8];
+        uint4 xv[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 4; ++i) {
+            const int64_t t = t0 + 4 * w + i;
+            if (col_ok && t < T) {
+                const float4 a = ld_state_v4(recon + t * C + c);
+                const float4 b = ld_state_v4(recon + t * C + c + 4);
+                ro[i][0] = a.x; ro[i][1] = a.y; ro[i][2] = a.z; ro[i][3] = a.w;
+                ro[i][4] = b.x; ro[i][5] = b.y; ro[i][6] = b.z; ro[i][7] = b.w;
+                xv[i] = SENDER ? ld_ro_v4(x + t * C + c) : make_uint4(0, 0, 0, 0);
+            } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-    for (int k = 0; k < r; ++k) {
-        const float4 a = *reinterpret_cast<const float4 *>(As + k * cf_lowrank::kApplyTok + 4 * w);
-        const float4 b0 = *reinterpret_cast<const float4 *>(Bs + k * cf_lowrank::kApplyCh + 8 * l);
-        const float4 b1 = *reinterpret_cast<const float4 *>(Bs + k * cf_lowrank::kApplyCh + 8 * l + 4);
-        const float av[4] = {a.x, a.y, a.z, a.w};
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                for (int j = 0; j < 8; ++j) ro[i][j] = 0.0f;
+                xv[i] = make_uint4(0, 0, 0, 0);
+            }
+        }
+        __syncthreads();  // the previous tile's reads of As are done
+        for (int i = tid; i < TM * r; i += blockDim.x) {
+            const int tt = i / r, k = i - (i / r) * r;
+            const int64_t t = t0 + tt;
+            As[k * TM + tt] = (t < T) ? int4_dequant(pc + t * nb, k, ps) : 0.0f;
+        }
+        __syncthreads();
+        float acc[4][8];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] = __fmaf_rn(av[i], bv[j], acc[i][j]);
-    }
-    const int64_t c = c0 + 8 * l;
-    if (c >= C) return;  // C % 8 == 0: a group of 8 channels is all in or all out
+            for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+        for (int k = 0; k < r; ++k) {
+            const float4 a = *reinterpret_cast<const float4 *>(As + k * TM + 4 * w);
+            const float4 b0 = *reinterpret_cast<const float4 *>(Bs + k * TN + 8 * l);
+            const float4 b1 = *reinterpret_cast<const float4 *>(Bs + k * TN + 8 * l + 4);
+            const float av[4] = {a.x, a.y, a.z, a.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t t = t0 + 4 * w + i;
-        if (t >= T) break;
-        float *rr = recon + t * C + c;
-        const float4 ra = ld_state_v4(rr), rb = ld_state_v4(rr + 4);
-        const float ro[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-        float rn[8];
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) rn[j] = __fadd_rn(ro[j], acc[i][j]);
-        if (SENDER) {
-            const uint4 xv = ld_ro_v4(x + t * C + c);
-            const uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
-            float eo[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float v = __fsub_rn(bf16_bits_to_f32((w4[j >> 1] >> ((j & 1) * 16)) & 0xffffu), ro[j]);
-                eo[j] = __fsub_rn(v, acc[i][j]);
-            }
-            st_stream_v4(err + t * C + c, make_float4(eo[0], eo[1], eo[2], eo[3]));
-            st_stream_v4(err + t * C + c + 4, make_float4(eo[4], eo[5], eo[6], eo[7]));
+                for (int j = 0; j < 8; ++j) acc[i][j] = __fmaf_rn(av[i], bv[j], acc[i][j]);
         }
-        st_state_v4(rr, make_float4(rn[0], rn[1], rn[2], rn[3]));
-        st_state_v4(rr + 4, make_float4(rn[4], rn[5], rn[6], rn[7]));
+        if (!col_ok) continue;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t t = t0 + 4 * w + i;
+            if (t >= T) break;
+            float rn[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) rn[j] = __fadd_rn(ro[i][j], acc[i][j]);
+            if (SENDER) {
+                const uint32_t w4[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+                float eo[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float xf = bf16_bits_to_f32((w4[j >> 1] >> ((j & 1) * 16)) & 0xffffu);
+                    eo[j] = __fsub_rn(__fsub_rn(xf, ro[i][j]), acc[i][j]);
+                }
+                st_stream_v4(err + t * C + c, make_float4(eo[0], eo[1], eo[2], eo[3]));
+                st_stream_v4(err + t * C + c + 4, make_float4(eo[4], eo[5], eo[6], eo[7]));
+            }
+            st_state_v4(recon + t * C + c, make_float4(rn[0], rn[1], rn[2], rn[3]));
+            st_state_v4(recon + t * C + c + 4, make_float4(rn[4], rn[5], rn[6], rn[7]));
+        }
     }
 }
 

@@ -59,6 +59,9 @@ def parse():
                     help="budget of the oracle timing sample")
     ap.add_argument("--buffers", type=int, default=0,
                     help="override the buffer count (smaller cases for profiling)")
+    ap.add_argument("--pipeline", type=int, default=-1,
+                    help="quantize kernels: 0 register-resident rows, 1 TMA row staging, "
+                         "-1 the library default")
     ap.add_argument("--gen-steps", type=int, default=0,
                     help="distinct pre-generated steps to cycle through (0 = all that fit)")
     return ap.parse_args()
@@ -212,6 +215,9 @@ def run_ours(args, world, rank, local):
     wl = W.WORKLOADS[args.workload]
     if args.buffers:
         wl = W.replace(wl, buffers=args.buffers)
+    if args.pipeline >= 0:
+        cf.cf_set_quant_pipeline(0, args.pipeline, 0)
+        cf.cf_set_quant_pipeline(1, args.pipeline, 0)
     n, T, C, bits = wl.buffers, wl.tokens, wl.channels, wl.bits
     d = cf.desc(T, C, bits)
     Wd = cf.cf_codes_words_per_row(d)

@@ -202,6 +202,17 @@ cf_status cf_lowrank_status(void *workspace, void *stream);
  * CF_ERR_INVALID_ARG for any other value. */
 cf_status cf_set_lowrank_engine(int32_t engine);
 
+/* Memory pipeline of the quantize-mode kernels in this process: kernel 0 =
+ * encode, 1 = decode; pipeline 0 = register-resident rows (each thread
+ * loads its channel groups straight into registers), 1 = TMA row staging
+ * (a producer warp streams whole rows into a ring of `stages` shared-memory
+ * slots with 1-D bulk copies; consumer warps compute from shared memory;
+ * the default).  stages 0 = built-in choice, else 2..8.  Both give bit-identical results;
+ * the TMA pipeline applies when C % 8 == 0 (decode also needs
+ * ceil(C*bits/32) % 4 == 0) and otherwise the call uses pipeline 0.
+ * Returns CF_ERR_INVALID_ARG for out-of-range values. */
+cf_status cf_set_quant_pipeline(int32_t kernel, int32_t pipeline, int32_t stages);
+
 /* Launch-shape override for tuning sweeps: kernel 0 = encode, 1 = decode;
  * groups_per_thread in 1..4 (8 channels per group), threads a multiple of
  * 32 in 32..512, or 0 to restore the built-in choice; blocks_per_sm caps

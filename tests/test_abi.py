@@ -97,6 +97,18 @@ def test_launch_override_validation(L):
     assert L.cf_set_launch_override(0, 0, 0, 0) == 0
 
 
+def test_pipeline_and_engine_knobs_validate(L):
+    assert L.cf_set_quant_pipeline(2, 0, 0) == 1
+    assert L.cf_set_quant_pipeline(0, 2, 0) == 1
+    assert L.cf_set_quant_pipeline(0, 1, 1) == 1
+    assert L.cf_set_quant_pipeline(0, 1, 9) == 1
+    assert L.cf_set_quant_pipeline(0, 1, 4) == 0
+    assert L.cf_set_quant_pipeline(0, 0, 0) == 0
+    assert L.cf_set_quant_pipeline(0, 1, 0) == 0   # restore the default
+    assert L.cf_set_lowrank_engine(2) == 1
+    assert L.cf_set_lowrank_engine(0) == 0
+
+
 def test_binding_raises_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(cf, "_lib", None)
     monkeypatch.setattr(cf, "LIB_PATH", str(tmp_path / "nope.so"))

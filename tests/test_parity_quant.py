@@ -103,6 +103,32 @@ def test_launch_shapes_agree_bitwise(bits):
         cf.cf_set_launch_override(1, 0, 0, 0)
 
 
+@pytest.mark.parametrize("T,C,bits", [(64, 3072, 2), (64, 3072, 1), (33, 1920, 2), (17, 256, 1),
+                                      (9, 64, 2), (5, 16384, 2), (40, 200, 2)])
+@pytest.mark.parametrize("stages", [0, 2, 5])
+def test_tma_pipeline_bit_identical(T, C, bits, stages):
+    """The TMA row-staging pipeline computes the same bits as the
+    register-resident one (and falls back to it where its alignment
+    conditions fail, e.g. C = 200 at 2 bits for decode)."""
+    wl = W.replace(W.WORKLOADS["flux_sp"], tokens=T, channels=C, bits=bits)
+    xs = W.trajectory(wl, 4, steps=3, device="cuda")
+    res = []
+    try:
+        for pipe in (0, 1):
+            cf.cf_set_quant_pipeline(0, pipe, stages if pipe else 0)
+            cf.cf_set_quant_pipeline(1, pipe, stages if pipe else 0)
+            g = GpuBuffer(T, C, bits)
+            g.init(xs[0].clone())
+            g.step(xs[1].clone())
+            g.step(xs[2].clone())
+            res.append(g.host())
+    finally:
+        cf.cf_set_quant_pipeline(0, 1, 0)   # the library default
+        cf.cf_set_quant_pipeline(1, 1, 0)
+    for k in ("codes", "scales", "err", "recon_s", "recon_r"):
+        assert np.array_equal(res[0][k].view(np.uint8), res[1][k].view(np.uint8)), k
+
+
 def test_host_pointer_is_rejected():
     d = cf.desc(4, 64, 1)
     host = torch.zeros(4, 64)
@@ -150,8 +176,9 @@ def test_batched_bad_buffer_is_skipped_and_reported():
     assert int(status.item()) == 1
 
 
+@pytest.mark.parametrize("pipe", [0, 1])
 @pytest.mark.parametrize("name,steps,sample", [("flux_sp", 3, (0, 57, 113))])
-def test_full_size_batched_step(name, steps, sample):
+def test_full_size_batched_step(name, steps, sample, pipe):
     """The bench's launch: all buffers of a step in one batched encode and one
     batched decode.  Sampled buffers are checked against the oracle over all
     steps; every buffer is checked for the EF identity and for
@@ -173,6 +200,16 @@ def test_full_size_batched_step(name, steps, sample):
     dec = cf.dec_buffer_array([(st["codes"][b], st["scales"][b], st["recon_r"][b])
                                for b in range(n)], "cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cf.cf_set_quant_pipeline(0, pipe, 0)
+    cf.cf_set_quant_pipeline(1, pipe, 0)
+    try:
+        _full_size_steps(wl, d, n, steps, sample, trs, st, x_buf, enc, dec, status, recon_o)
+    finally:
+        cf.cf_set_quant_pipeline(0, 1, 0)   # the library default
+        cf.cf_set_quant_pipeline(1, 1, 0)
+
+
+def _full_size_steps(wl, d, n, steps, sample, trs, st, x_buf, enc, dec, status, recon_o):
     for s in range(1, steps):
         x_buf.copy_(torch.stack([t.next() for t in trs]))
         v = x_buf.float() - st["recon_s"]                  # one fp32 rounding, as the kernel
