@@ -29,6 +29,7 @@
 #include "lowrank_api.cuh"
 #include "lowrank_kernels.cuh"
 #include "lowrank_umma.cuh"
+#include "lowrank_apply_tc.cuh"
 
 namespace cf_lowrank {
 
@@ -251,9 +252,32 @@ T *at(void *ws, size_t off) {
     return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
 }
 
+template <bool SENDER, int KP>
+cf_status launch_apply_tc(const Layout &L, const uint16_t *x, float *recon, float *err,
+                          const uint8_t *pc, const float *ps, const uint8_t *qc, const float *qs,
+                          int32_t *status, cudaStream_t st) {
+    auto k = cf::umma::lr_apply_tc_kernel<SENDER, KP>;
+    constexpr int smem = cf::umma::apply_tc_smem<KP>();
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return CF_ERR_CUDA;
+    dim3 grid((unsigned)((L.C + 127) / 128), (unsigned)((L.T + 127) / 128));
+    k<<<grid, 256, smem, st>>>(x, recon, err, pc, ps, qc, qs, L.T, L.C, L.r, status);
+    return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
+}
+
+// D = P^ Q^T applied to the state.  Engine 0: tensor cores (tcgen05 tf32,
+// hi/lo split); engine 1: CUDA-core FMA chain.  A buffer's sender and
+// receiver must use the same engine to stay bit-identical.
 cf_status apply(bool sender, const Layout &L, const uint16_t *x, float *recon, float *err,
                 const uint8_t *pc, const float *ps, const uint8_t *qc, const float *qs,
-                cudaStream_t st) {
+                int32_t *status, cudaStream_t st) {
+    if (g_engine.load() == 0) {
+        if (L.rp <= 32)
+            return sender ? launch_apply_tc<true, 32>(L, x, recon, err, pc, ps, qc, qs, status, st)
+                          : launch_apply_tc<false, 32>(L, x, recon, err, pc, ps, qc, qs, status, st);
+        return sender ? launch_apply_tc<true, 64>(L, x, recon, err, pc, ps, qc, qs, status, st)
+                      : launch_apply_tc<false, 64>(L, x, recon, err, pc, ps, qc, qs, status, st);
+    }
     const int64_t gx = (L.C + kApplyCh - 1) / kApplyCh;
     const int64_t ntiles = (L.T + kApplyTok - 1) / kApplyTok;
     int64_t gy = (2 * (int64_t)sm_count() + gx - 1) / gx;
@@ -343,9 +367,15 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
     }
     for (int it = 0; it < d->iters; ++it) {
         LR_TRY(project(L, vb, qt, yp, status, st));
-        cf::lr_gram_chol_kernel<<<(unsigned)L.nGram, 256, 0, st>>>(
-            yp, y, gp, T, r, rp, L.splitsA, L.nGram, rmat, rinvd, ticket, status);
-        LR_LAUNCHED();
+        {
+            const size_t gs = cf::lr_gram_smem_bytes(rp);
+            if (cudaFuncSetAttribute(cf::lr_gram_chol_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gs) != cudaSuccess)
+                return CF_ERR_CUDA;
+            cf::lr_gram_chol_kernel<<<(unsigned)L.nGram, 256, gs, st>>>(
+                yp, y, gp, T, r, rp, L.splitsA, L.nGram, rmat, rinvd, ticket, status);
+            LR_LAUNCHED();
+        }
         const bool last = (it == d->iters - 1);
         LR_TRY(orth(L, y, rmat, rinvd, p, pt, last ? amax : nullptr, st));
         LR_TRY(backproject(L, vb, pt, zp, status, st));
@@ -357,7 +387,7 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
     LR_LAUNCHED();
     cf::lr_int4_pack_kernel<<<(unsigned)((C * nb + 255) / 256), 256, 0, st>>>(q, C, r, rp, amax + rp, q_codes, q_scales);
     LR_LAUNCHED();
-    return apply(true, L, x, recon_s, err, p_codes, p_scales, q_codes, q_scales, st);
+    return apply(true, L, x, recon_s, err, p_codes, p_scales, q_codes, q_scales, status, st);
 }
 
 cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes, const float *p_scales,
@@ -372,7 +402,7 @@ cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes, const floa
     LR_TRY(check_ptr(recon_r));
     const Layout L = make_layout(d->tokens, d->channels, d->rank);
     return apply(false, L, nullptr, recon_r, nullptr, p_codes, p_scales, q_codes, q_scales,
-                 (cudaStream_t)stream);
+                 nullptr, (cudaStream_t)stream);
 }
 
 cf_status cf_set_lowrank_engine(int32_t engine) {

@@ -14,7 +14,7 @@ constexpr int kMaxIters = 16;
 
 constexpr int64_t kChunkA = 512;   // channels per split of the Y = V Q pass
 constexpr int64_t kChunkB = 512;   // tokens per split of the Q = V^T P pass
-constexpr int kGramTok = 64;       // tokens per partial Gram block
+constexpr int kGramTok = 256;      // tokens per partial Gram block
 constexpr int kApplyTok = 32;      // D tile: tokens
 constexpr int kApplyCh = 256;      // D tile: channels
 constexpr int kApplyThreads = 256;

@@ -152,44 +152,71 @@ __device__ __forceinline__ void warp_cholesky_smem(double *A, int ld, int r, con
     }
 }
 
-// Fused Gram + Cholesky.  Every CTA: Y = sum of the split partials (fixed
-// order) for its 64 tokens, and its partial Gram block Gp[blk] = Y^T Y
-// (upper triangle, fp64).  The last CTA to finish (atomic ticket after a
-// fence) sums the partials in block order -- deterministic -- and factors
-// G = R^T R in one warp (right-looking, lane l owns columns l and l + 32).
-// A pivot that is not above 1e-10 of its original diagonal entry marks the
-// column dead: its row of R and its inverse diagonal are zero, so P gets a
-// zero column, and CF_ERR_NUMERIC is recorded.  Output: R (fp32 [rp][rp],
+// Fused Gram + Cholesky.  CTA b owns tokens [256 b, 256 b + 256):
+//  1. Y = sum of the split partials (float4 rows, every split's load in
+//     flight at once, summed in split order), written to y and to shared
+//     memory;
+//  2. its partial Gram block Gp[b] = Y_b^T Y_b (upper triangle, fp64, four
+//     interleaved accumulators per entry combined in a fixed order).
+// The last CTA to finish (atomic ticket after a fence) sums the partial
+// blocks in block order -- deterministic -- and factors G = R^T R in one
+// warp.  A pivot not above 1e-10 of its original diagonal entry marks the
+// column dead: its row of R and its inverse diagonal are zero (P gets a
+// zero column) and CF_ERR_NUMERIC is recorded.  Output: R (fp32 [rp][rp],
 // upper) and 1/diag(R) (fp32 [rp], 0 where dead).  The ticket is reset for
 // the next iteration.
 __global__ void __launch_bounds__(256)
 lr_gram_chol_kernel(const float *yp, float *y, double *gp, int64_t T, int r, int rp, int splits,
                     int nblk, float *rmat, float *rinvd, uint32_t *ticket, int32_t *status) {
-    __shared__ double S[64 * 65];  // Y block (fp64), later the matrix being factored
+    extern __shared__ float ys[];  // [kGramTok][rp + 1]
+    __shared__ double A[64 * 65];
     __shared__ double gdiag[64];
     __shared__ int dead[64];
     __shared__ int is_last;
     const int tid = threadIdx.x;
-    const int64_t t0 = (int64_t)blockIdx.x * cf_lowrank::kGramTok;
     const int ldy = rp + 1;
-    for (int i = tid; i < 64 * rp; i += blockDim.x) {
-        const int tt = i / rp, k = i - (i / rp) * rp;
+    const int64_t t0 = (int64_t)blockIdx.x * cf_lowrank::kGramTok;
+    const int q4 = rp / 4;
+    for (int idx = tid; idx < cf_lowrank::kGramTok * q4; idx += blockDim.x) {
+        const int tt = idx / q4, k = (idx - tt * q4) * 4;
         const int64_t t = t0 + tt;
-        float v = 0.0f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (t < T) {
-            for (int s = 0; s < splits; ++s) v += yp[((int64_t)s * T + t) * rp + k];
-            y[t * rp + k] = v;
+            const float4 *src = reinterpret_cast<const float4 *>(yp + t * rp + k);
+            const int64_t sstride = T * rp / 4;
+            int s = 0;
+            for (; s + 8 <= splits; s += 8) {
+                float4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (s + u) * sstride);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
+                }
+            }
+            for (; s < splits; ++s) {
+                const float4 v = __ldcg(src + s * sstride);
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            }
+            *reinterpret_cast<float4 *>(y + t * rp + k) = acc;
         }
-        S[tt * ldy + k] = (double)v;
+        float *row = ys + tt * ldy + k;
+        row[0] = acc.x; row[1] = acc.y; row[2] = acc.z; row[3] = acc.w;
     }
     __syncthreads();
-    double *g = gp + (int64_t)blockIdx.x * rp * rp;
-    for (int e = tid; e < rp * rp; e += blockDim.x) {
+    const int ne = rp * rp;
+    double *g = gp + (int64_t)blockIdx.x * ne;
+    for (int e = tid; e < ne; e += blockDim.x) {
         const int i = e / rp, j = e - (e / rp) * rp;
         if (i > j) continue;
-        double acc = 0.0;
-        for (int tt = 0; tt < 64; ++tt) acc = fma(S[tt * ldy + i], S[tt * ldy + j], acc);
-        g[e] = acc;
+        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+        for (int tt = 0; tt < cf_lowrank::kGramTok; tt += 4) {
+            a0 = fma((double)ys[tt * ldy + i], (double)ys[tt * ldy + j], a0);
+            a1 = fma((double)ys[(tt + 1) * ldy + i], (double)ys[(tt + 1) * ldy + j], a1);
+            a2 = fma((double)ys[(tt + 2) * ldy + i], (double)ys[(tt + 2) * ldy + j], a2);
+            a3 = fma((double)ys[(tt + 3) * ldy + i], (double)ys[(tt + 3) * ldy + j], a3);
+        }
+        g[e] = (a0 + a1) + (a2 + a3);
     }
     __threadfence();
     __syncthreads();
@@ -199,34 +226,21 @@ lr_gram_chol_kernel(const float *yp, float *y, double *gp, int64_t T, int r, int
     __threadfence();
 
     const int ld = rp + 1;
-    double *A = S;
-    // final reduction of the partial Grams: the sum for entry e is split
-    // over 4 adjacent lanes (blocks q, q+4, ...) and combined by xor
-    // shuffles as (p0 + p1) + (p2 + p3), the same order on every run.
-    // 4 * rp * rp is a multiple of the block size, so every thread runs the
-    // same number of iterations and all lanes reach the shuffles.
-    const int ne = rp * rp;
-    for (int idx = tid; idx < 4 * ne; idx += blockDim.x) {
-        const int e = idx >> 2, q = idx & 3;
+    for (int e = tid; e < ne; e += blockDim.x) {
         const int i = e / rp, j = e - (e / rp) * rp;
+        if (i > j) continue;
+        // 8 independent accumulators keep 8 L2 loads in flight; the
+        // association order depends only on nblk, so it is reproducible
         double a[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-        if (i <= j) {
-            // 8 independent accumulators keep 8 L2 loads in flight; the
-            // association order depends only on nblk, so it is reproducible
-            int b = q;
-            for (; b + 28 < nblk; b += 32) {
+        int b = 0;
+        for (; b + 8 <= nblk; b += 8) {
 #pragma unroll
-                for (int u = 0; u < 8; ++u) a[u] += __ldcg(gp + (int64_t)(b + 4 * u) * ne + e);
-            }
-            for (int u = 0; b < nblk; b += 4, ++u) a[u & 7] += __ldcg(gp + (int64_t)b * ne + e);
+            for (int u = 0; u < 8; ++u) a[u] += __ldcg(gp + (int64_t)(b + u) * ne + e);
         }
-        double acc = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
-        acc += __shfl_xor_sync(kFullMask, acc, 1);
-        acc += __shfl_xor_sync(kFullMask, acc, 2);
-        if (q == 0 && i <= j) {
-            A[i * ld + j] = acc;
-            if (i == j) gdiag[i] = acc;
-        }
+        for (; b < nblk; ++b) a[0] += __ldcg(gp + (int64_t)b * ne + e);
+        const double v = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+        A[i * ld + j] = v;
+        if (i == j) gdiag[i] = v;
     }
     __syncthreads();
     if (tid < 32) {
@@ -239,7 +253,7 @@ lr_gram_chol_kernel(const float *yp, float *y, double *gp, int64_t T, int r, int
     }
     __syncthreads();
     int nd = 0;
-    for (int e = tid; e < rp * rp; e += blockDim.x) {
+    for (int e = tid; e < ne; e += blockDim.x) {
         const int i = e / rp, c = e - (e / rp) * rp;
         rmat[e] = (i <= c && c < r) ? (float)A[i * ld + c] : 0.0f;
     }
@@ -250,6 +264,10 @@ lr_gram_chol_kernel(const float *yp, float *y, double *gp, int64_t T, int r, int
     }
     if (nd) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_NUMERIC);
     if (tid == 0) *ticket = 0u;
+}
+
+inline size_t lr_gram_smem_bytes(int rp) {
+    return (size_t)cf_lowrank::kGramTok * (rp + 1) * sizeof(float);
 }
 
 // P = Y R^-1 by forward substitution, one token row per thread:

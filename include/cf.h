@@ -195,11 +195,14 @@ cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes,
  * clears it.  Returns CF_ERR_CUDA if the copy or the sync fails. */
 cf_status cf_lowrank_status(void *workspace, void *stream);
 
-/* Engine of the two subspace-iteration products in this process: 0 (the
- * default) = tcgen05 tensor cores (bf16 operands, fp32 accumulation in
- * TMEM), 1 = CUDA cores (same bf16 operands, fp32 FMA).  For cross-checks
- * and diagnosis; both satisfy the same parity bar.  Returns
- * CF_ERR_INVALID_ARG for any other value. */
+/* Engine of the low-rank dense products in this process: 0 (the default) =
+ * tcgen05 tensor cores (the two subspace-iteration products with bf16
+ * operands, and D = P^ Q^T in tf32 with a hi/lo split of the scaled P
+ * factor, fp32 accumulation in TMEM), 1 = CUDA cores (same operands, fp32
+ * FMA).  For cross-checks and diagnosis; both satisfy the same parity bar.
+ * The sender and the receiver of a buffer must use the same engine: D is
+ * bit-identical only within one engine.  Returns CF_ERR_INVALID_ARG for any
+ * other value. */
 cf_status cf_set_lowrank_engine(int32_t engine);
 
 /* Memory pipeline of the quantize-mode kernels in this process: kernel 0 =
