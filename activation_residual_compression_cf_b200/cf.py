@@ -27,7 +27,7 @@ EXPORTS = ("cf_status_string", "cf_abi_version", "cf_codes_words_per_row",
            "cf_encode_batched", "cf_decode_batched", "cf_lowrank_workspace_bytes",
            "cf_lowrank_factor_bytes", "cf_lowrank_encode", "cf_lowrank_decode",
            "cf_lowrank_status", "cf_set_lowrank_engine", "cf_set_quant_pipeline",
-           "cf_set_launch_override")
+           "cf_set_launch_override", "cf_lowrank_encode_noalloc")
 
 
 class CFError(RuntimeError):
@@ -85,6 +85,7 @@ def lib():
             "cf_set_launch_override": ([i32, i32, i32, i32], ctypes.c_int),
             "cf_set_lowrank_engine": ([i32], ctypes.c_int),
             "cf_set_quant_pipeline": ([i32, i32, i32], ctypes.c_int),
+            "cf_lowrank_encode_noalloc": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -174,6 +175,16 @@ def cf_lowrank_encode(d, x, recon_s, err, omega, p_codes, p_scales, q_codes, q_s
     _chk(lib().cf_lowrank_encode(ctypes.byref(d), _p(x), _p(recon_s), _p(err), _p(omega),
                                  _p(p_codes), _p(p_scales), _p(q_codes), _p(q_scales),
                                  _p(workspace), nbytes, _s(stream)), "cf_lowrank_encode")
+
+
+def cf_lowrank_encode_noalloc(d, x, recon_s, err, omega, p_codes, p_scales, q_codes, q_scales,
+                              stream=None):
+    """cf_lowrank_encode without a workspace, for callers that cannot allocate
+    device memory: the library's fixed device scratch array is used instead
+    (see include/cf.h for its size and sharing rules)."""
+    _chk(lib().cf_lowrank_encode_noalloc(ctypes.byref(d), _p(x), _p(recon_s), _p(err),
+                                         _p(omega), _p(p_codes), _p(p_scales), _p(q_codes),
+                                         _p(q_scales), _s(stream)), "cf_lowrank_encode_noalloc")
 
 
 def cf_lowrank_decode(d, p_codes, p_scales, q_codes, q_scales, recon_r, stream=None):

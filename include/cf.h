@@ -190,6 +190,36 @@ cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes,
                             const float *q_scales, float *recon_r,
                             void *stream);
 
+/* Size of the device scratch array behind cf_lowrank_encode_noalloc: 40 MiB,
+ * enough for 4096 tokens x 3072 channels at rank 32 (about 33.5 MB). */
+#define CF_LOWRANK_NOALLOC_SCRATCH_BYTES (40ull << 20)
+
+/* Low-rank sender for callers that cannot allocate device memory.  The
+ * paper has no counterpart to this call; it exists for callers such as a
+ * plug-in running inside a framework that owns all device memory and gives
+ * it no allocator, or a serving loop that must not call cudaMalloc mid-step
+ * (the call can synchronise the device).  Same arguments and results as
+ * cf_lowrank_encode without the workspace pair: the scratch lives in one
+ * file-scope device array of CF_LOWRANK_NOALLOC_SCRATCH_BYTES bytes that
+ * every GPU using the library holds until the process exits.  The call
+ * allocates nothing and calls no allocating routine; inputs and outputs are
+ * still the caller's.
+ *  - Problems whose cf_lowrank_workspace_bytes exceeds the array return
+ *    CF_ERR_WORKSPACE without launching anything.
+ *  - The first call on a device looks up the array's device address on the
+ *    current device (cudaGetSymbolAddress) and caches it; make that first
+ *    call before any stream capture on that device.
+ *  - Every call on a device shares the one array, which keeps the previous
+ *    call's contents (the implementation clears what must start at zero).
+ *    Calls whose work overlaps on the GPU -- different streams without
+ *    ordering between them -- race on the array and corrupt each other.
+ *  - The status word is in the array as well: cf_lowrank_status cannot
+ *    reach it; CF_ERR_NUMERIC cases still yield a valid, lower-rank D. */
+cf_status cf_lowrank_encode_noalloc(const cf_desc *d, const uint16_t *x, float *recon_s,
+                                    float *err, const float *omega, uint8_t *p_codes,
+                                    float *p_scales, uint8_t *q_codes, float *q_scales,
+                                    void *stream);
+
 /* Synchronises `stream`, then returns the status word the last
  * cf_lowrank_encode on `workspace` recorded (CF_OK or CF_ERR_NUMERIC) and
  * clears it.  Returns CF_ERR_CUDA if the copy or the sync fails. */
