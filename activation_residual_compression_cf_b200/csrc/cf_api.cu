@@ -39,11 +39,9 @@ int device_sm_count() {
     return n;
 }
 
-bool is_aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-cf_status check_dev_ptr(const void *p) {
+cf_status check_dev_ptr(const void *p, uintptr_t align = 16) {
     if (!p) return CF_ERR_INVALID_ARG;
-    if (!is_aligned16(p)) return CF_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(p) & (align - 1)) != 0) return CF_ERR_ALIGNMENT;
     cudaPointerAttributes a;
     if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
         (void)cudaGetLastError();
@@ -77,18 +75,31 @@ struct Shape {
     int gpt;
     int threads;
     int blocks_per_sm;
+    int pipeline = 0;
 };
 
-// Smallest thread count (multiple of 32) with at most 4 groups of 8
-// channels per thread, aiming at ~128 threads per row.
-Shape choose_shape(int kernel, int64_t C) {
+// Launch shape per row: threads (a multiple of 32) x groups of 8 channels
+// per thread.  Measured on B200 at C = 3072 (114 x 1024 rows): the TMA
+// pipeline is fastest with 4 groups per thread (fewer, busier consumer
+// warps), the register pipeline with 2 groups per thread.
+Shape choose_shape(int kernel, int64_t C, int pipeline) {
     const int64_t G = (C + 7) / 8;
     Shape s;
-    int gpt = (int)((G + 127) / 128);
-    if (gpt < 1) gpt = 1;
+    int gpt;
+    if (pipeline == 1) {
+        gpt = kMaxGroupsPerThread;
+    } else {
+        gpt = (int)((G + 191) / 192);
+        if (gpt < 2) gpt = 2;
+    }
     if (gpt > kMaxGroupsPerThread) gpt = kMaxGroupsPerThread;
+    while (gpt > 1 && (G + gpt - 1) / gpt < 32 && (G + gpt - 2) / (gpt - 1) <= 32) --gpt;
     int64_t thr = (G + gpt - 1) / gpt;
     thr = (thr + 31) / 32 * 32;
+    while (thr > kMaxThreads && gpt < kMaxGroupsPerThread) {
+        ++gpt;
+        thr = ((G + gpt - 1) / gpt + 31) / 32 * 32;
+    }
     s.gpt = gpt;
     s.threads = (int)thr;
     s.blocks_per_sm = 0;
@@ -147,7 +158,14 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
                      const Shape &s, int stages_req, cudaStream_t st) {
     const int64_t W = (C * BITS + 31) / 32;
     const int64_t slot = ENC ? 6 * C : 4 * W + 4 * C;
-    int stages = stages_req > 0 ? stages_req : (int)(100000 / slot);
+    // Ring depth: measured on B200 (C = 1920 and 3072), 5 slots for encode
+    // and 6 for decode are at or near the best; deeper rings cost CTAs per SM.
+    int stages = stages_req;
+    if (stages <= 0) {
+        stages = (int)(120000 / slot);
+        const int cap = ENC ? 5 : 6;
+        if (stages > cap) stages = cap;
+    }
     if (stages > 8) stages = 8;
     if (stages < 2) stages = 2;
     const size_t smem = (size_t)stages * slot + 16 * (size_t)stages;
@@ -176,15 +194,14 @@ template <bool ENC, int BITS, int GPT, bool VEC, class Src>
 cf_status launch_one(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t *status,
                      const Shape &s, cudaStream_t st) {
     if constexpr (VEC) {
-        int pipe, stages;
-        {
-            std::lock_guard<std::mutex> lk(g_mu);
-            pipe = g_pipeline[ENC ? 0 : 1];
-            stages = g_stages[ENC ? 0 : 1];
-        }
-        const bool codes_ok = ENC || ((C * BITS + 31) / 32) % 4 == 0;
-        if (pipe == 1 && codes_ok && s.threads <= 480 && 2 * (ENC ? 6 * C : 4 * C + C * BITS / 8) <= 200000)
+        if (s.pipeline == 1) {
+            int stages;
+            {
+                std::lock_guard<std::mutex> lk(g_mu);
+                stages = g_stages[ENC ? 0 : 1];
+            }
             return launch_tma<ENC, BITS, GPT>(src, T, C, rows, status, s, stages, st);
+        }
     }
     if constexpr (ENC)
         return launch_encode_t<BITS, GPT, VEC>(src, T, C, rows, status, s, st);
@@ -193,10 +210,26 @@ cf_status launch_one(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
 }
 
 // Runtime (bits, gpt, vec) -> template instance.
+// The TMA pipeline applies when rows are 16-byte multiples (C % 8 == 0),
+// decode code rows too (ceil(C*bits/32) % 4 == 0), and a 2-slot ring fits.
+bool tma_applies(bool enc, int bits, int64_t C) {
+    if (C % 8 != 0) return false;
+    if (!enc && ((C * bits + 31) / 32) % 4 != 0) return false;
+    return 2 * (enc ? 6 * C : 4 * C + C * bits / 8) <= 200000;
+}
+
 template <bool ENC, class Src>
 cf_status dispatch(const Src &src, int bits, int64_t T, int64_t C, int64_t rows,
                    int32_t *status, cudaStream_t st) {
-    const Shape s = choose_shape(ENC ? 0 : 1, C);
+    int pipe;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        pipe = g_pipeline[ENC ? 0 : 1];
+    }
+    if (pipe == 1 && !tma_applies(ENC, bits, C)) pipe = 0;
+    Shape s = choose_shape(ENC ? 0 : 1, C, pipe);
+    if (pipe == 1 && s.threads > 480) s = choose_shape(ENC ? 0 : 1, C, pipe = 0);
+    s.pipeline = pipe;
     const bool vec = (C % 8) == 0;
 #define CF_CASE(B, G, V)                                     \
     if (bits == B && s.gpt == G && vec == V)                 \
@@ -275,7 +308,7 @@ cf_status cf_encode(const cf_desc *d, const uint16_t *x, float *recon_s, float *
     CF_TRY(check_dev_ptr(recon_s));
     CF_TRY(check_dev_ptr(err));
     CF_TRY(check_dev_ptr(codes));
-    CF_TRY(check_dev_ptr(scales));
+    CF_TRY(check_dev_ptr(scales, 4));
     cf::EncSingle src{{x, recon_s, err, codes, scales}};
     return dispatch<true>(src, d->bits, d->tokens, d->channels, d->tokens, nullptr,
                           (cudaStream_t)stream);
@@ -286,7 +319,7 @@ cf_status cf_decode(const cf_desc *d, const uint32_t *codes, const float *scales
     CF_TRY(check_quant_desc(d));
     if (d->tokens == 0) return CF_OK;
     CF_TRY(check_dev_ptr(codes));
-    CF_TRY(check_dev_ptr(scales));
+    CF_TRY(check_dev_ptr(scales, 4));
     CF_TRY(check_dev_ptr(recon_r));
     cf::DecSingle src{{codes, scales, recon_r}};
     return dispatch<false>(src, d->bits, d->tokens, d->channels, d->tokens, nullptr,

@@ -55,14 +55,17 @@ Layout make_layout(int64_t T, int64_t C, int r) {
     L.splitsA = (int)((C + kChunkA - 1) / kChunkA);
     L.splitsB = (int)((T + kChunkB - 1) / kChunkB);
     L.nGram = (int)((T + kGramTok - 1) / kGramTok);
+    L.nGroups = (L.nGram + kGramGroup - 1) / kGramGroup;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         size_t o = off;
         off += (bytes + 255) / 256 * 256;
         return o;
     };
-    L.off_status = take(16);
+    L.off_status = take(16);                          // status word, final ticket
+    L.off_gt = take((size_t)L.nGroups * 4);           // group tickets
     L.off_gp = take((size_t)L.nGram * L.rp * L.rp * 8);
+    L.off_gg = take((size_t)L.nGroups * L.rp * L.rp * 8);
     L.off_rmat = take((size_t)L.rp * L.rp * 4 + (size_t)L.rp * 4);
     L.off_amax = take((size_t)2 * L.rp * 4);
     L.off_vb = take((size_t)T * C * 2);
@@ -339,6 +342,8 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
 
     int32_t *status = at<int32_t>(ws, L.off_status);
     double *gp = at<double>(ws, L.off_gp);
+    double *gg = at<double>(ws, L.off_gg);
+    uint32_t *gticket = at<uint32_t>(ws, L.off_gt);
     float *rmat = at<float>(ws, L.off_rmat);
     float *rinvd = rmat + rp * rp;
     uint32_t *ticket = reinterpret_cast<uint32_t *>(status + 1);
@@ -352,7 +357,8 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
     float *zp = at<float>(ws, L.off_zp);
     float *q = at<float>(ws, L.off_q);
 
-    if (cudaMemsetAsync(status, 0, 16, st) != cudaSuccess) return CF_ERR_CUDA;
+    // status word and tickets start at zero
+    if (cudaMemsetAsync(status, 0, L.off_gp, st) != cudaSuccess) return CF_ERR_CUDA;
     if (cudaMemsetAsync(amax, 0, (size_t)2 * rp * 4, st) != cudaSuccess) return CF_ERR_CUDA;
     const int sms = sm_count();
     {
@@ -368,12 +374,8 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
     for (int it = 0; it < d->iters; ++it) {
         LR_TRY(project(L, vb, qt, yp, status, st));
         {
-            const size_t gs = cf::lr_gram_smem_bytes(rp);
-            if (cudaFuncSetAttribute(cf::lr_gram_chol_kernel,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gs) != cudaSuccess)
-                return CF_ERR_CUDA;
-            cf::lr_gram_chol_kernel<<<(unsigned)L.nGram, 256, gs, st>>>(
-                yp, y, gp, T, r, rp, L.splitsA, L.nGram, rmat, rinvd, ticket, status);
+            cf::lr_gram_chol_kernel<<<(unsigned)L.nGram, 256, 0, st>>>(
+                yp, y, gp, gg, T, r, rp, L.splitsA, rmat, rinvd, gticket, ticket, status);
             LR_LAUNCHED();
         }
         const bool last = (it == d->iters - 1);

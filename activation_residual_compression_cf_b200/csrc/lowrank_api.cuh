@@ -14,7 +14,8 @@ constexpr int kMaxIters = 16;
 
 constexpr int64_t kChunkA = 512;   // channels per split of the Y = V Q pass
 constexpr int64_t kChunkB = 512;   // tokens per split of the Q = V^T P pass
-constexpr int kGramTok = 256;      // tokens per partial Gram block
+constexpr int kGramTok = 32;       // tokens per Gram CTA
+constexpr int kGramGroup = 16;     // Gram partial blocks summed per first-level group
 constexpr int kApplyTok = 32;      // D tile: tokens
 constexpr int kApplyCh = 256;      // D tile: channels
 constexpr int kApplyThreads = 256;
@@ -26,8 +27,8 @@ struct Layout {
     int64_t T, C;
     int r, rp;
     int64_t Tp;
-    int splitsA, splitsB, nGram;
-    size_t off_status, off_gp, off_rmat, off_amax, off_vb, off_qt, off_yp, off_y, off_p, off_pt,
+    int splitsA, splitsB, nGram, nGroups;
+    size_t off_status, off_gt, off_gp, off_gg, off_rmat, off_amax, off_vb, off_qt, off_yp, off_y, off_p, off_pt,
         off_zp, off_q, total;
 };
 

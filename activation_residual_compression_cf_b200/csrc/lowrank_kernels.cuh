@@ -98,7 +98,7 @@ lr_project_simt(const bf16 *vb, const bf16 *qt, float *yp, int64_t T, int64_t C,
 // On return A's upper triangle holds R and dead[j] flags dead pivots.
 template <int RPW>
 __device__ __forceinline__ void warp_cholesky_regs(double *A, int ld, int r, const double *gdiag,
-                                                   int *dead) {
+                                                   int *dead, double *invd) {
     const int lane = threadIdx.x & 31;
     double col[RPW];
 #pragma unroll
@@ -108,9 +108,9 @@ __device__ __forceinline__ void warp_cholesky_regs(double *A, int ld, int r, con
         if (j >= r) break;
         const double ajj = __shfl_sync(kFullMask, col[j], j);
         const bool bad = !(ajj > 1e-10 * gdiag[j]);
-        const double rjj = bad ? 0.0 : sqrt(ajj);
-        const double inv = bad ? 0.0 : 1.0 / rjj;
-        // row j of R: lane c > j scales its entry; lane j holds the diagonal
+        // one reciprocal square root gives both R[j][j] = ajj * inv and 1/R[j][j]
+        const double inv = bad ? 0.0 : rsqrt(ajj);
+        const double rjj = ajj * inv;
         if (lane > j) col[j] *= inv;
         if (lane == j) col[j] = rjj;
         const double rjc = col[j];
@@ -119,7 +119,10 @@ __device__ __forceinline__ void warp_cholesky_regs(double *A, int ld, int r, con
             const double rji = __shfl_sync(kFullMask, rjc, i);  // R[j][i] from lane i
             if (lane >= i) col[i] = fma(-rji, rjc, col[i]);
         }
-        if (lane == 0) dead[j] = bad ? 1 : 0;
+        if (lane == 0) {
+            dead[j] = bad ? 1 : 0;
+            invd[j] = inv;
+        }
     }
 #pragma unroll
     for (int i = 0; i < RPW; ++i)
@@ -129,19 +132,20 @@ __device__ __forceinline__ void warp_cholesky_regs(double *A, int ld, int r, con
 // Same factorisation for r up to 64 with the matrix in shared memory (lane
 // l owns columns l and l + 32).
 __device__ __forceinline__ void warp_cholesky_smem(double *A, int ld, int r, const double *gdiag,
-                                                   int *dead) {
+                                                   int *dead, double *invd) {
     const int lane = threadIdx.x & 31;
     for (int j = 0; j < r; ++j) {
         const double ajj = A[j * ld + j];
         const bool bad = !(ajj > 1e-10 * gdiag[j]);
-        const double rjj = bad ? 0.0 : sqrt(ajj);
-        const double inv = bad ? 0.0 : 1.0 / rjj;
+        const double inv = bad ? 0.0 : rsqrt(ajj);
+        const double rjj = ajj * inv;
         for (int c = lane; c < r; c += 32)
             if (c > j) A[j * ld + c] *= inv;
         __syncwarp();
         if (lane == 0) {
             A[j * ld + j] = rjj;
             dead[j] = bad ? 1 : 0;
+            invd[j] = inv;
         }
         for (int c = lane; c < r; c += 32) {
             if (c <= j) continue;
@@ -152,51 +156,116 @@ __device__ __forceinline__ void warp_cholesky_smem(double *A, int ld, int r, con
     }
 }
 
-// Fused Gram + Cholesky.  CTA b owns tokens [256 b, 256 b + 256):
-//  1. Y = sum of the split partials (float4 rows, every split's load in
-//     flight at once, summed in split order), written to y and to shared
-//     memory;
-//  2. its partial Gram block Gp[b] = Y_b^T Y_b (upper triangle, fp64, four
-//     interleaved accumulators per entry combined in a fixed order).
-// The last CTA to finish (atomic ticket after a fence) sums the partial
-// blocks in block order -- deterministic -- and factors G = R^T R in one
-// warp.  A pivot not above 1e-10 of its original diagonal entry marks the
-// column dead: its row of R and its inverse diagonal are zero (P gets a
-// zero column) and CF_ERR_NUMERIC is recorded.  Output: R (fp32 [rp][rp],
-// upper) and 1/diag(R) (fp32 [rp], 0 where dead).  The ticket is reset for
-// the next iteration.
+// Cholesky of the upper triangle of A (leading dimension ld, r <= 32) by
+// the first 128 threads of the block: thread (w, c) = (tid / 32, tid % 32)
+// owns column c and the rows i = w, w + 4, ... of it in registers, so every
+// warp (one per SM sub-partition) shares the fp64 update work of a step.
+// Row j of R is broadcast through shared memory (double-buffered, one
+// barrier per step among the 128 threads).  Results as warp_cholesky_regs.
+__device__ __forceinline__ void quad_cholesky(double *A, int ld, int r, const double *gdiag,
+                                              int *dead, double *invd, double (*rowbuf)[33]) {
+    const int tid = threadIdx.x;
+    const int w = tid >> 5, c = tid & 31;
+    double a[8];  // A[w + 4m][c]
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const int i = w + 4 * m;
+        a[m] = (c < r && i <= c) ? A[i * ld + c] : 0.0;
+    }
+    for (int j = 0; j < r; ++j) {
+        const int wj = j & 3, mj = j >> 2;
+        double *row = rowbuf[j & 1];
+        if (w == wj) {
+            // this warp holds row j: finish it and publish it
+            double ajj = 0.0;
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+                if (m == mj) ajj = a[m];
+            ajj = __shfl_sync(kFullMask, ajj, j);
+            const bool bad = !(ajj > 1e-10 * gdiag[j]);
+            const double inv = bad ? 0.0 : rsqrt(ajj);
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+                if (m == mj) {
+                    if (c > j) a[m] *= inv;
+                    if (c == j) a[m] = ajj * inv;
+                    row[c] = (c >= j && c < r) ? a[m] : 0.0;
+                }
+            if (c == 0) {
+                dead[j] = bad ? 1 : 0;
+                invd[j] = inv;
+            }
+        }
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+        // trailing update of this thread's rows i > j: A[i][c] -= R[j][i] R[j][c]
+        if (c > j) {
+            const double rjc = row[c];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int i = w + 4 * m;
+                if (i > j && i <= c) a[m] = fma(-row[i], rjc, a[m]);
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const int i = w + 4 * m;
+        if (c < r && i <= c) A[i * ld + c] = a[m];
+    }
+}
+
+// Fused Gram + Cholesky, deterministic.  CTA b owns 32 tokens:
+//  1. Y = sum of the split partials for its tokens (float4 rows; the loads
+//     of up to 8 splits are issued before any is summed; summed in split
+//     order), written to y and to shared memory;
+//  2. its fp64 partial Gram Gp[b] = Y_b^T Y_b (upper triangle).
+// Reduction in two ticketed levels, each summing in a fixed order: the last
+// CTA to finish in each group of 16 blocks sums the group's partials into
+// Gg[group]; the last group to finish sums the groups in order into G and
+// factors G = R^T R in one warp.  (A reduction whose order varied from run
+// to run would be amplified by the bf16 operand roundings of later
+// iterations into visible differences.)  A pivot not above 1e-10 of its
+// original diagonal entry marks the column dead: its row of R and its
+// inverse diagonal are zero (P gets a zero column) and CF_ERR_NUMERIC is
+// recorded.  Output: R (fp32 [rp][rp], upper) and 1/diag(R) (fp32 [rp], 0
+// where dead).  All tickets are reset by their last user.
 __global__ void __launch_bounds__(256)
-lr_gram_chol_kernel(const float *yp, float *y, double *gp, int64_t T, int r, int rp, int splits,
-                    int nblk, float *rmat, float *rinvd, uint32_t *ticket, int32_t *status) {
-    extern __shared__ float ys[];  // [kGramTok][rp + 1]
-    __shared__ double A[64 * 65];
+lr_gram_chol_kernel(const float *yp, float *y, double *gp, double *gg, int64_t T, int r, int rp,
+                    int splits, float *rmat, float *rinvd, uint32_t *gticket, uint32_t *ticket,
+                    int32_t *status) {
+    constexpr int TOK = cf_lowrank::kGramTok;
+    // one buffer: the fp32 Y block in phases 1-2, the fp64 matrix afterwards
+    __shared__ double buf[64 * 65];
+    static_assert(TOK * 65 * sizeof(float) <= sizeof(buf), "Y block does not fit");
+    float *ys = reinterpret_cast<float *>(buf);
+    double *A = buf;
     __shared__ double gdiag[64];
+    __shared__ double invd[64];
+    __shared__ double rowbuf[2][33];
     __shared__ int dead[64];
     __shared__ int is_last;
     const int tid = threadIdx.x;
     const int ldy = rp + 1;
-    const int64_t t0 = (int64_t)blockIdx.x * cf_lowrank::kGramTok;
+    const int64_t t0 = (int64_t)blockIdx.x * TOK;
     const int q4 = rp / 4;
-    for (int idx = tid; idx < cf_lowrank::kGramTok * q4; idx += blockDim.x) {
+    for (int idx = tid; idx < TOK * q4; idx += blockDim.x) {
         const int tt = idx / q4, k = (idx - tt * q4) * 4;
         const int64_t t = t0 + tt;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (t < T) {
             const float4 *src = reinterpret_cast<const float4 *>(yp + t * rp + k);
             const int64_t sstride = T * rp / 4;
-            int s = 0;
-            for (; s + 8 <= splits; s += 8) {
+            // batches of 8 splits: all 8 loads issued before any is summed
+            for (int s0 = 0; s0 < splits; s0 += 8) {
                 float4 v[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (s + u) * sstride);
+                for (int u = 0; u < 8; ++u)
+                    if (s0 + u < splits) v[u] = __ldcg(src + (s0 + u) * sstride);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
-                }
-            }
-            for (; s < splits; ++s) {
-                const float4 v = __ldcg(src + s * sstride);
-                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+                for (int u = 0; u < 8; ++u)
+                    if (s0 + u < splits) {
+                        acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
+                    }
             }
             *reinterpret_cast<float4 *>(y + t * rp + k) = acc;
         }
@@ -205,22 +274,49 @@ lr_gram_chol_kernel(const float *yp, float *y, double *gp, int64_t T, int r, int
     }
     __syncthreads();
     const int ne = rp * rp;
-    double *g = gp + (int64_t)blockIdx.x * ne;
     for (int e = tid; e < ne; e += blockDim.x) {
         const int i = e / rp, j = e - (e / rp) * rp;
         if (i > j) continue;
-        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-        for (int tt = 0; tt < cf_lowrank::kGramTok; tt += 4) {
+        double a0 = 0.0, a1 = 0.0;
+#pragma unroll 4
+        for (int tt = 0; tt < TOK; tt += 2) {
             a0 = fma((double)ys[tt * ldy + i], (double)ys[tt * ldy + j], a0);
             a1 = fma((double)ys[(tt + 1) * ldy + i], (double)ys[(tt + 1) * ldy + j], a1);
-            a2 = fma((double)ys[(tt + 2) * ldy + i], (double)ys[(tt + 2) * ldy + j], a2);
-            a3 = fma((double)ys[(tt + 3) * ldy + i], (double)ys[(tt + 3) * ldy + j], a3);
         }
-        g[e] = (a0 + a1) + (a2 + a3);
+        gp[(int64_t)blockIdx.x * ne + e] = a0 + a1;
     }
+    // level 1: the last CTA of each group of kGramGroup blocks sums them
+    const int nblk = gridDim.x;
+    const int grp = blockIdx.x / cf_lowrank::kGramGroup;
+    const int gb0 = grp * cf_lowrank::kGramGroup;
+    const int gn = min(cf_lowrank::kGramGroup, nblk - gb0);
+    const int ngrp = (nblk + cf_lowrank::kGramGroup - 1) / cf_lowrank::kGramGroup;
     __threadfence();
     __syncthreads();
-    if (tid == 0) is_last = (atomicAdd(ticket, 1u) == (uint32_t)(nblk - 1)) ? 1 : 0;
+    if (tid == 0) is_last = (atomicAdd(gticket + grp, 1u) == (uint32_t)(gn - 1)) ? 1 : 0;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    for (int e = tid; e < ne; e += blockDim.x) {
+        const int i = e / rp, j = e - (e / rp) * rp;
+        if (i > j) continue;
+        // batches of 16 loads in flight, summed in block order
+        double acc = 0.0;
+        for (int u0 = 0; u0 < gn; u0 += 16) {
+            double v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                v[u] = (u0 + u < gn) ? __ldcg(gp + (int64_t)(gb0 + u0 + u) * ne + e) : 0.0;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) acc += v[u];
+        }
+        gg[(int64_t)grp * ne + e] = acc;
+    }
+    if (tid == 0) gticket[grp] = 0u;
+    // level 2: the last group sums the groups in order
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = (atomicAdd(ticket, 1u) == (uint32_t)(ngrp - 1)) ? 1 : 0;
     __syncthreads();
     if (!is_last) return;
     __threadfence();
@@ -229,27 +325,22 @@ lr_gram_chol_kernel(const float *yp, float *y, double *gp, int64_t T, int r, int
     for (int e = tid; e < ne; e += blockDim.x) {
         const int i = e / rp, j = e - (e / rp) * rp;
         if (i > j) continue;
-        // 8 independent accumulators keep 8 L2 loads in flight; the
-        // association order depends only on nblk, so it is reproducible
         double a[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-        int b = 0;
-        for (; b + 8 <= nblk; b += 8) {
+        int g = 0;
+        for (; g + 8 <= ngrp; g += 8) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) a[u] += __ldcg(gp + (int64_t)(b + u) * ne + e);
+            for (int u = 0; u < 8; ++u) a[u] += __ldcg(gg + (int64_t)(g + u) * ne + e);
         }
-        for (; b < nblk; ++b) a[0] += __ldcg(gp + (int64_t)b * ne + e);
+        for (; g < ngrp; ++g) a[0] += __ldcg(gg + (int64_t)g * ne + e);
         const double v = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
         A[i * ld + j] = v;
         if (i == j) gdiag[i] = v;
     }
     __syncthreads();
-    if (tid < 32) {
-        if (r <= 16)
-            warp_cholesky_regs<16>(A, ld, r, gdiag, dead);
-        else if (r <= 32)
-            warp_cholesky_regs<32>(A, ld, r, gdiag, dead);
-        else
-            warp_cholesky_smem(A, ld, r, gdiag, dead);
+    if (r <= 32) {
+        if (tid < 128) quad_cholesky(A, ld, r, gdiag, dead, invd, rowbuf);
+    } else if (tid < 32) {
+        warp_cholesky_smem(A, ld, r, gdiag, dead, invd);
     }
     __syncthreads();
     int nd = 0;
@@ -259,15 +350,11 @@ lr_gram_chol_kernel(const float *yp, float *y, double *gp, int64_t T, int r, int
     }
     for (int j = tid; j < rp; j += blockDim.x) {
         const bool live = j < r && !dead[j];
-        rinvd[j] = live ? (float)(1.0 / A[j * ld + j]) : 0.0f;
+        rinvd[j] = live ? (float)invd[j] : 0.0f;
         nd += (j < r && dead[j]) ? 1 : 0;
     }
     if (nd) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_NUMERIC);
     if (tid == 0) *ticket = 0u;
-}
-
-inline size_t lr_gram_smem_bytes(int rp) {
-    return (size_t)cf_lowrank::kGramTok * (rp + 1) * sizeof(float);
 }
 
 // P = Y R^-1 by forward substitution, one token row per thread:

@@ -93,16 +93,20 @@ struct DecArray {
     }
 };
 
+// Scales are per-token fp32 scalars: 4-byte alignment suffices for them.
+__device__ __forceinline__ bool misaligned4(const void *p) {
+    return (reinterpret_cast<uintptr_t>(p) & 3u) != 0;
+}
 __device__ __forceinline__ int enc_ptr_status(const EncPtrs &p) {
     if (!p.x || !p.recon || !p.err || !p.codes || !p.scales) return CF_ERR_INVALID_ARG;
     if (misaligned16(p.x) || misaligned16(p.recon) || misaligned16(p.err) ||
-        misaligned16(p.codes) || misaligned16(p.scales))
+        misaligned16(p.codes) || misaligned4(p.scales))
         return CF_ERR_ALIGNMENT;
     return CF_OK;
 }
 __device__ __forceinline__ int dec_ptr_status(const DecPtrs &p) {
     if (!p.codes || !p.scales || !p.recon) return CF_ERR_INVALID_ARG;
-    if (misaligned16(p.codes) || misaligned16(p.scales) || misaligned16(p.recon))
+    if (misaligned16(p.codes) || misaligned4(p.scales) || misaligned16(p.recon))
         return CF_ERR_ALIGNMENT;
     return CF_OK;
 }

@@ -40,6 +40,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
+from activation_residual_compression_cf_b200 import replicas as R  # noqa: E402
 from activation_residual_compression_cf_b200 import workloads as W  # noqa: E402
 
 FALLBACK_HBM_GBS = 6650.0
@@ -70,15 +71,11 @@ def parse():
 # ------------------------------------------------------------ environment
 
 def dist_setup(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group(
-            "nccl" if torch.cuda.is_available() else "gloo",
-            timeout=datetime.timedelta(seconds=120))
-    return world, rank, local
+    info = R.rank_info_from_env()
+    if info.distributed:
+        torch.cuda.set_device(info.local)
+        R.init(info, timeout_s=120.0)
+    return info.world, info.rank, info.local
 
 
 def peaks():
@@ -261,32 +258,24 @@ def run_ours(args, world, rank, local):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    wall0 = time.time()
-    t_start.record(stream)
-    for i in range(args.steps):
-        e0, e1, e2 = ev[i]
-        e0.record(stream)
-        cf.cf_encode_batched(d, n, enc[1 + (args.warmup + i) % (S - 1)], status, stream)
-        e1.record(stream)
-        cf.cf_decode_batched(d, n, dec, status, stream)
-        e2.record(stream)
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    with R.bracket():
+        wall0 = time.time()
+        t_start.record(stream)
+        for i in range(args.steps):
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            cf.cf_encode_batched(d, n, enc[1 + (args.warmup + i) % (S - 1)], status, stream)
+            e1.record(stream)
+            cf.cf_decode_batched(d, n, dec, status, stream)
+            e2.record(stream)
+        t_end.record(stream)
     wall1 = time.time()
     clocks = sampler.stop(wall0, wall1)
     assert int(status.item()) == 0, cf.cf_status_string(int(status.item()))
     ms = t_start.elapsed_time(t_end)
     enc_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1, _ in ev)
     dec_ms = statistics.mean(e1.elapsed_time(e2) for _, e1, e2 in ev)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = R.reduce_scalar(ms, "max")
 
     bytes_processed = 2 * T * C * n * args.steps * world
     value = bytes_processed / (ms / 1e3) / 1e9
@@ -300,10 +289,7 @@ def run_ours(args, world, rank, local):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, status)
-        if world > 1:
-            t = torch.tensor([e2e["ms"]], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e["ms"] = float(t.item())
+        e2e["ms"] = R.reduce_scalar(e2e["ms"], "max")
         e2e = {"value": round(bytes_processed / (e2e["ms"] / 1e3) / 1e9, 3), "unit": "GB/s",
                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                "ms_per_step": round(e2e["ms"] / args.steps, 4)}
@@ -398,28 +384,20 @@ def run_lowrank(args, world, rank, local):
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    wall0 = time.time()
-    for i in range(args.steps):
-        e0, e1, e2 = ev[i]
-        e0.record(stream)
-        enc(args.warmup + i)
-        e1.record(stream)
-        dec()
-        e2.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    with R.bracket():
+        wall0 = time.time()
+        for i in range(args.steps):
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            enc(args.warmup + i)
+            e1.record(stream)
+            dec()
+            e2.record(stream)
     clocks = sampler.stop(wall0, time.time())
     ms = ev[0][0].elapsed_time(ev[-1][2])
     enc_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
     dec_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = R.reduce_scalar(ms, "max")
     peak, peak_kind = peaks()
     value = 2 * T * C * n * args.steps * world / (ms / 1e3) / 1e9
     enc_bytes = n * T * C * 14
@@ -548,8 +526,7 @@ def main():
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:
-        if world > 1:
-            torch.distributed.destroy_process_group()
+        R.finish()
 
 
 if __name__ == "__main__":

@@ -23,7 +23,9 @@
  *    (or managed) memory of the current device.  Single-buffer calls check
  *    this with cudaPointerGetAttributes and return CF_ERR_INVALID_ARG for
  *    host memory instead of launching.
- *  - Every device pointer must be 16-byte aligned (CF_ERR_ALIGNMENT).
+ *  - Every device pointer must be 16-byte aligned (CF_ERR_ALIGNMENT), except
+ *    the per-token scale arrays of the quantize mode, which need 4 bytes
+ *    (so [n][T] packed scales of any T are valid).
  *  - Argument errors are reported synchronously and launch nothing.  A
  *    failed launch returns CF_ERR_CUDA.  Numeric trouble found on the
  *    device (low-rank mode) is written to a status word in the workspace.

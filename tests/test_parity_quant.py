@@ -177,7 +177,9 @@ def test_batched_bad_buffer_is_skipped_and_reported():
 
 
 @pytest.mark.parametrize("pipe", [0, 1])
-@pytest.mark.parametrize("name,steps,sample", [("flux_sp", 3, (0, 57, 113))])
+@pytest.mark.parametrize("name,steps,sample", [("flux_sp", 3, (0, 57, 113)),
+                                               ("flux_full", 2, (0, 113)),
+                                               ("cogvideox", 2, (0, 59))])
 def test_full_size_batched_step(name, steps, sample, pipe):
     """The bench's launch: all buffers of a step in one batched encode and one
     batched decode.  Sampled buffers are checked against the oracle over all
@@ -211,19 +213,24 @@ def test_full_size_batched_step(name, steps, sample, pipe):
 
 def _full_size_steps(wl, d, n, steps, sample, trs, st, x_buf, enc, dec, status, recon_o):
     for s in range(1, steps):
-        x_buf.copy_(torch.stack([t.next() for t in trs]))
-        v = x_buf.float() - st["recon_s"]                  # one fp32 rounding, as the kernel
+        for b in range(n):
+            x_buf[b].copy_(trs[b].next())
+        v = [x_buf[b].float() - st["recon_s"][b] for b in range(n)]   # one fp32 rounding
         cf.cf_encode_batched(d, n, enc, status)
         cf.cf_decode_batched(d, n, dec, status)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
         assert torch.equal(st["recon_r"].view(torch.int32), st["recon_s"].view(torch.int32))
-        # EF identity: recon_s + err == x within the three fp32 roundings
-        gap = (st["recon_s"].double() + st["err"].double() - x_buf.double()).abs()
-        bound = (v.abs().double() + st["err"].abs().double() + st["recon_s"].abs().double()) \
-            * 2.0**-24 * (1 + 1e-9) + 3 * 2.0**-149
-        assert bool((gap <= bound).all())
-        del v, gap, bound
+        # EF identity per buffer: recon_s + err == x within the three fp32
+        # roundings (residual, error, mirror update)
+        for b in range(n):
+            rs, er, xb = st["recon_s"][b].double(), st["err"][b].double(), x_buf[b].double()
+            vb = v[b].double().abs()
+            gap = (rs + er - xb).abs()
+            bound = (vb + er.abs() + rs.abs()) * 2.0**-24 * (1 + 1e-9) + 3 * 2.0**-149
+            assert bool((gap <= bound).all()), b
+            del rs, er, xb, vb, gap, bound
+        del v
         for b in sample:
             xb = W.bf16_bits(x_buf[b])
             v, ora = oracle_step(xb, recon_o[b], wl.bits)
