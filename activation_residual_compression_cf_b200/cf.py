@@ -27,7 +27,8 @@ EXPORTS = ("cf_status_string", "cf_abi_version", "cf_codes_words_per_row",
            "cf_encode_batched", "cf_decode_batched", "cf_lowrank_workspace_bytes",
            "cf_lowrank_factor_bytes", "cf_lowrank_encode", "cf_lowrank_decode",
            "cf_lowrank_status", "cf_set_lowrank_engine", "cf_set_quant_pipeline",
-           "cf_set_launch_override", "cf_lowrank_encode_noalloc")
+           "cf_set_launch_override", "cf_lowrank_encode_noalloc", "cf_decode_emit",
+           "cf_decode_emit_batched")
 
 
 class CFError(RuntimeError):
@@ -54,6 +55,11 @@ class cf_dec_buffer(ctypes.Structure):
                 ("recon_r", ctypes.c_void_p)]
 
 
+class cf_dec_emit_buffer(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("recon_r", ctypes.c_void_p), ("out", ctypes.c_void_p)]
+
+
 _lib = None
 
 
@@ -77,6 +83,8 @@ def lib():
             "cf_decode": ([D, vp, vp, vp, vp], ctypes.c_int),
             "cf_encode_batched": ([D, i32, vp, vp, vp], ctypes.c_int),
             "cf_decode_batched": ([D, i32, vp, vp, vp], ctypes.c_int),
+            "cf_decode_emit": ([D, vp, vp, vp, vp, vp], ctypes.c_int),
+            "cf_decode_emit_batched": ([D, i32, vp, vp, vp], ctypes.c_int),
             "cf_lowrank_workspace_bytes": ([D], i64),
             "cf_lowrank_factor_bytes": ([i64, i32], i64),
             "cf_lowrank_encode": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
@@ -149,6 +157,16 @@ def cf_encode(d, x, recon_s, err, codes, scales, stream=None):
 def cf_decode(d, codes, scales, recon_r, stream=None):
     _chk(lib().cf_decode(ctypes.byref(d), _p(codes), _p(scales), _p(recon_r), _s(stream)),
          "cf_decode")
+
+
+def cf_decode_emit(d, codes, scales, recon_r, out, stream=None):
+    _chk(lib().cf_decode_emit(ctypes.byref(d), _p(codes), _p(scales), _p(recon_r), _p(out),
+                              _s(stream)), "cf_decode_emit")
+
+
+def cf_decode_emit_batched(d, n, bufs_dev, status_dev=None, stream=None):
+    _chk(lib().cf_decode_emit_batched(ctypes.byref(d), n, _p(bufs_dev), _p(status_dev),
+                                      _s(stream)), "cf_decode_emit_batched")
 
 
 def cf_encode_batched(d, n, bufs_dev, status_dev=None, stream=None):
@@ -229,6 +247,15 @@ def dec_buffer_array(sets, device) -> torch.Tensor:
     arr = (cf_dec_buffer * len(sets))()
     for i, (c, s, r) in enumerate(sets):
         arr[i] = cf_dec_buffer(_p(c), _p(s), _p(r))
+    host = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8)
+    return host.to(device)
+
+
+def dec_emit_buffer_array(sets, device) -> torch.Tensor:
+    """Device array of cf_dec_emit_buffer from [(codes, scales, recon_r, out), ...]."""
+    arr = (cf_dec_emit_buffer * len(sets))()
+    for i, (c, s, r, o) in enumerate(sets):
+        arr[i] = cf_dec_emit_buffer(_p(c), _p(s), _p(r), _p(o))
     host = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8)
     return host.to(device)
 

@@ -326,6 +326,31 @@ cf_status cf_decode(const cf_desc *d, const uint32_t *codes, const float *scales
                            (cudaStream_t)stream);
 }
 
+cf_status cf_decode_emit(const cf_desc *d, const uint32_t *codes, const float *scales,
+                         float *recon_r, uint16_t *out, void *stream) {
+    CF_TRY(check_quant_desc(d));
+    if (d->tokens == 0) return CF_OK;
+    CF_TRY(check_dev_ptr(codes));
+    CF_TRY(check_dev_ptr(scales, 4));
+    CF_TRY(check_dev_ptr(recon_r));
+    CF_TRY(check_dev_ptr(out));
+    cf::DecEmitSingle src{{codes, scales, recon_r, out}};
+    return dispatch<false>(src, d->bits, d->tokens, d->channels, d->tokens, nullptr,
+                           (cudaStream_t)stream);
+}
+
+cf_status cf_decode_emit_batched(const cf_desc *d, int32_t n, const cf_dec_emit_buffer *bufs_dev,
+                                 int32_t *status_dev, void *stream) {
+    CF_TRY(check_quant_desc(d));
+    if (n < 0) return CF_ERR_INVALID_ARG;
+    if (n == 0 || d->tokens == 0) return CF_OK;
+    CF_TRY(check_dev_ptr(bufs_dev));
+    if (status_dev) CF_TRY(check_dev_ptr(status_dev));
+    cf::DecEmitArray src{bufs_dev};
+    return dispatch<false>(src, d->bits, d->tokens, d->channels, d->tokens * (int64_t)n,
+                           status_dev, (cudaStream_t)stream);
+}
+
 cf_status cf_encode_batched(const cf_desc *d, int32_t n, const cf_enc_buffer *bufs_dev,
                             int32_t *status_dev, void *stream) {
     CF_TRY(check_quant_desc(d));

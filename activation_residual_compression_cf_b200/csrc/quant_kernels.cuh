@@ -29,6 +29,8 @@
 //    identical rounded value.
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include "cf.h"
 #include "cf_common.cuh"
 
@@ -46,6 +48,7 @@ struct DecPtrs {
     const uint32_t *codes;
     const float *scales;
     float *recon;
+    uint16_t *out;  // bf16 copy of the new reconstruction (emitting decode only)
 };
 
 template <class P>
@@ -75,23 +78,54 @@ struct EncArray {
         return p;
     }
 };
-struct DecSingle {
+template <bool EMIT>
+struct DecSingleT {
     DecPtrs p;
     static constexpr bool kChecked = false;
+    static constexpr bool kEmit = EMIT;
     __device__ __forceinline__ DecPtrs get(int64_t) const { return p; }
 };
+using DecSingle = DecSingleT<false>;
+using DecEmitSingle = DecSingleT<true>;
 struct DecArray {
     const cf_dec_buffer *a;
     static constexpr bool kChecked = true;
+    static constexpr bool kEmit = false;
     __device__ __forceinline__ DecPtrs get(int64_t i) const {
         const cf_dec_buffer *e = a + i;
         DecPtrs p;
         p.codes = ldg_ptr(&e->codes);
         p.scales = ldg_ptr(&e->scales);
         p.recon = ldg_ptr(&e->recon_r);
+        p.out = nullptr;
         return p;
     }
 };
+struct DecEmitArray {
+    const cf_dec_emit_buffer *a;
+    static constexpr bool kChecked = true;
+    static constexpr bool kEmit = true;
+    __device__ __forceinline__ DecPtrs get(int64_t i) const {
+        const cf_dec_emit_buffer *e = a + i;
+        DecPtrs p;
+        p.codes = ldg_ptr(&e->codes);
+        p.scales = ldg_ptr(&e->scales);
+        p.recon = ldg_ptr(&e->recon_r);
+        p.out = ldg_ptr(&e->out);
+        return p;
+    }
+};
+
+// 8 fp32 values -> 8 bf16 (round to nearest even) packed in 16 bytes.
+__device__ __forceinline__ uint4 pack_bf16x8(const float *v) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+        w[k] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
 
 // Scales are per-token fp32 scalars: 4-byte alignment suffices for them.
 __device__ __forceinline__ bool misaligned4(const void *p) {
@@ -104,9 +138,11 @@ __device__ __forceinline__ int enc_ptr_status(const EncPtrs &p) {
         return CF_ERR_ALIGNMENT;
     return CF_OK;
 }
+template <bool EMIT>
 __device__ __forceinline__ int dec_ptr_status(const DecPtrs &p) {
-    if (!p.codes || !p.scales || !p.recon) return CF_ERR_INVALID_ARG;
-    if (misaligned16(p.codes) || misaligned4(p.scales) || misaligned16(p.recon))
+    if (!p.codes || !p.scales || !p.recon || (EMIT && !p.out)) return CF_ERR_INVALID_ARG;
+    if (misaligned16(p.codes) || misaligned4(p.scales) || misaligned16(p.recon) ||
+        (EMIT && misaligned16(p.out)))
         return CF_ERR_ALIGNMENT;
     return CF_OK;
 }
@@ -295,7 +331,7 @@ decode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
         const int64_t t = row - b * T;
         const DecPtrs p = src.get(b);
         if (Src::kChecked) {
-            const int st = dec_ptr_status(p);
+            const int st = dec_ptr_status<Src::kEmit>(p);
             if (st != CF_OK) {
                 if (tid == 0) report(status, st);
                 continue;
@@ -347,11 +383,19 @@ decode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
             if (VEC) {
                 st_state_v4(rr + 8 * g, make_float4(ro[0], ro[1], ro[2], ro[3]));
                 st_state_v4(rr + 8 * g + 4, make_float4(ro[4], ro[5], ro[6], ro[7]));
+                if (Src::kEmit)
+                    *reinterpret_cast<uint4 *>(p.out + t * C + 8 * g) = pack_bf16x8(ro);
             } else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int64_t c = 8 * g + e;
-                    if (c < C) rr[c] = ro[e];
+                    if (c < C) {
+                        rr[c] = ro[e];
+                        if (Src::kEmit) {
+                            const __nv_bfloat16 h = __float2bfloat16_rn(ro[e]);
+                            p.out[t * C + c] = *reinterpret_cast<const uint16_t *>(&h);
+                        }
+                    }
                 }
             }
         }

@@ -160,7 +160,11 @@ encode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
                 for (int e = 0; e < 8; ++e) r[j][e] = v[j][e] = 0.0f;
             }
         }
-        // the slot is no longer read: release it to the producer
+        // the slot is no longer read: release it to the producer.  The reads
+        // above are generic-proxy accesses and the producer's next bulk copy
+        // into this slot is an async-proxy write: the proxy fence orders them
+        // (without it a late read can see the next row's bytes).
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0) bar_arrive(bars + 8u * (stages + s));
         ++i;
@@ -260,7 +264,7 @@ decode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
         for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
             const int64_t b = row / T, t = row - b * T;
             const DecPtrs p = src.get(b);
-            if (Src::kChecked && dec_ptr_status(p) != CF_OK) continue;
+            if (Src::kChecked && dec_ptr_status<Src::kEmit>(p) != CF_OK) continue;
             const int s = i % stages;
             const uint32_t ph = (uint32_t)(i / stages) & 1u;
             if (!bar_wait(bars + 8u * (stages + s), ph ^ 1u)) {
@@ -285,7 +289,7 @@ decode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
         const int64_t b = row / T, t = row - b * T;
         const DecPtrs p = src.get(b);
         if (Src::kChecked) {
-            const int st = dec_ptr_status(p);
+            const int st = dec_ptr_status<Src::kEmit>(p);
             if (st != CF_OK) {
                 if (ct == 0) report(status, st);
                 continue;
@@ -323,6 +327,8 @@ decode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
                 for (int e = 0; e < 8; ++e) r[j][e] = 0.0f;
             }
         }
+        // release the slot; proxy fence as in the encode kernel
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0) bar_arrive(bars + 8u * (stages + s));
         ++i;
@@ -338,6 +344,7 @@ decode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
             }
             st_state_v4(rr + 8 * g, make_float4(ro[0], ro[1], ro[2], ro[3]));
             st_state_v4(rr + 8 * g + 4, make_float4(ro[4], ro[5], ro[6], ro[7]));
+            if (Src::kEmit) *reinterpret_cast<uint4 *>(p.out + t * C + 8 * g) = pack_bf16x8(ro);
         }
     }
 }

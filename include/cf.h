@@ -100,6 +100,14 @@ typedef struct cf_dec_buffer {
     float *recon_r;      /* fp32 [T][C], receiver reconstruction (updated)  */
 } cf_dec_buffer;
 
+/* One receiver buffer set for the batched emitting decode. */
+typedef struct cf_dec_emit_buffer {
+    const uint32_t *codes;
+    const float *scales;
+    float *recon_r;      /* fp32 [T][C], receiver reconstruction (updated)  */
+    uint16_t *out;       /* bf16 [T][C], written: bf16_rne(new recon_r)     */
+} cf_dec_emit_buffer;
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *cf_status_string(cf_status s);
 
@@ -134,6 +142,14 @@ cf_status cf_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
 cf_status cf_decode(const cf_desc *d, const uint32_t *codes,
                     const float *scales, float *recon_r, void *stream);
 
+/* Receiver that also emits the reconstruction in bf16, the dtype the
+ * attention layer consumes (the decoded K/V go straight to attention), in
+ * the same pass: recon_r is updated exactly as by cf_decode and
+ * out[t][c] = bf16 round-to-nearest-even of the new recon_r[t][c].
+ * out: bf16 [T][C] device, written. */
+cf_status cf_decode_emit(const cf_desc *d, const uint32_t *codes, const float *scales,
+                         float *recon_r, uint16_t *out, void *stream);
+
 /* Batched forms: `n` buffers of the same shape in ONE launch, with the same
  * per-buffer semantics as cf_encode / cf_decode.  `bufs_dev` is a DEVICE
  * array of n descriptors (it must stay valid until the work completes).
@@ -148,6 +164,9 @@ cf_status cf_encode_batched(const cf_desc *d, int32_t n,
 cf_status cf_decode_batched(const cf_desc *d, int32_t n,
                             const cf_dec_buffer *bufs_dev, int32_t *status_dev,
                             void *stream);
+cf_status cf_decode_emit_batched(const cf_desc *d, int32_t n,
+                                 const cf_dec_emit_buffer *bufs_dev,
+                                 int32_t *status_dev, void *stream);
 
 /* ------------------------------------------------------------------------
  * Low-rank mode ("Approach", "Key results", "Builds on": PowerSGD-style

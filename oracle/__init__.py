@@ -38,6 +38,10 @@ def _load():
         lib.orc_encode.restype = ctypes.c_int
         lib.orc_decode.argtypes = [i64, i64, i32, vp, vp, vp]
         lib.orc_decode.restype = ctypes.c_int
+        lib.orc_decode_emit.argtypes = [i64, i64, i32, vp, vp, vp, vp]
+        lib.orc_decode_emit.restype = ctypes.c_int
+        lib.orc_f32_to_bf16.argtypes = [ctypes.c_float]
+        lib.orc_f32_to_bf16.restype = ctypes.c_uint16
         _lib = lib
     return _lib
 
@@ -95,6 +99,28 @@ def decode(codes: np.ndarray, scales: np.ndarray, recon_r: np.ndarray, bits: int
     rc = _load().orc_decode(T, C, bits, _ptr(codes), _ptr(scales), _ptr(recon_r))
     if rc != 0:
         raise ValueError(f"oracle decode: unsupported bits={bits}")
+
+
+def decode_emit(codes: np.ndarray, scales: np.ndarray, recon_r: np.ndarray, bits: int):
+    """Receiver step that also returns the bf16 reconstruction (uint16 bit
+    patterns, round to nearest even); ``recon_r`` is updated in place."""
+    T, C = recon_r.shape
+    W = words_per_row(C, bits)
+    _check(codes, np.uint32, (T, W), "codes")
+    _check(scales, np.float32, (T,), "scales")
+    _check(recon_r, np.float32, (T, C), "recon_r")
+    out = np.empty((T, C), np.uint16)
+    rc = _load().orc_decode_emit(T, C, bits, _ptr(codes), _ptr(scales), _ptr(recon_r), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle decode: unsupported bits={bits}")
+    return out
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Element-wise fp32 -> bf16 (round to nearest even) through the C oracle."""
+    f = _load().orc_f32_to_bf16
+    flat = np.ascontiguousarray(a, np.float32).ravel()
+    return np.array([f(float(v)) for v in flat], np.uint16).reshape(np.shape(a))
 
 
 def quant_payload_bytes(tokens: int, channels: int, bits: int) -> int:

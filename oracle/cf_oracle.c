@@ -133,6 +133,22 @@ int orc_encode(int64_t T, int64_t C, int32_t bits, const uint16_t *x,
     return 0;
 }
 
+/* fp32 -> bf16 bit pattern, round to nearest, ties to even; NaN stays a
+ * (quiet) NaN.  The attention layer that consumes the reconstruction reads
+ * bf16, so a receiver that also emits bf16 writes this rounding of recon_r. */
+uint16_t orc_f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu)) return (uint16_t)((u >> 16) | 0x0040u);
+    const uint32_t lsb = (u >> 16) & 1u;
+    return (uint16_t)((u + 0x7fffu + lsb) >> 16);
+}
+
+/* Receiver that also emits the bf16 reconstruction: recon_r as orc_decode,
+ * then out[i] = bf16_rne(recon_r[i]). */
+int orc_decode_emit(int64_t T, int64_t C, int32_t bits, const uint32_t *codes,
+                    const float *scales, float *recon_r, uint16_t *out);
+
 /* Receiver: unpack, dequantise and accumulate into recon_r. */
 int orc_decode(int64_t T, int64_t C, int32_t bits, const uint32_t *codes,
                const float *scales, float *recon_r) {
@@ -148,5 +164,13 @@ int orc_decode(int64_t T, int64_t C, int32_t bits, const uint32_t *codes,
             rr[c] = rr[c] + dequant(bits, code, scales[t]);
         }
     }
+    return 0;
+}
+
+int orc_decode_emit(int64_t T, int64_t C, int32_t bits, const uint32_t *codes,
+                    const float *scales, float *recon_r, uint16_t *out) {
+    int rc = orc_decode(T, C, bits, codes, scales, recon_r);
+    if (rc != 0) return rc;
+    for (int64_t i = 0; i < T * C; ++i) out[i] = orc_f32_to_bf16(recon_r[i]);
     return 0;
 }

@@ -202,3 +202,33 @@ def test_payload_ratio_closed_form():
     assert oracle.quant_payload_bytes(1024, 3072, 1) == 1024 * (3072 // 8 + 4)
     r1 = 2 * 1024 * 3072 / oracle.quant_payload_bytes(1024, 3072, 1)
     assert abs(r1 - 16 / (1 + 32 / 3072)) < 1e-9
+
+
+def test_bf16_rounding_matches_torch_and_ties_to_even():
+    """The emitted bf16 reconstruction is round-to-nearest-even: checked
+    against torch's CPU conversion (a library routine) on random values and on
+    hand-picked ties."""
+    rng = np.random.default_rng(11)
+    vals = np.concatenate([
+        rng.standard_normal(2000).astype(np.float32) * 10 ** rng.uniform(-30, 30, 2000).astype(np.float32),
+        np.array([0.0, -0.0, 1.0, -1.0, 3.0e38, -3.0e38, 1e-40, np.inf, -np.inf], np.float32)])
+    ties = np.array([0x3f808000, 0x3f818000, 0xbf808000, 0x3f80c000], np.uint32).view(np.float32)
+    vals = np.concatenate([vals, ties])
+    ours = oracle.f32_to_bf16_bits(vals)
+    ref = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+    # 1.00390625 = 0x3F808000 is a tie between 0x3F80 and 0x3F81: even -> 0x3F80
+    assert ours[-4] == 0x3F80 and ours[-3] == 0x3F82 and ours[-2] == 0xBF80 and ours[-1] == 0x3F81
+    nan = oracle.f32_to_bf16_bits(np.array([np.nan], np.float32))[0]
+    assert (nan & 0x7F80) == 0x7F80 and (nan & 0x7F)
+
+
+def test_decode_emit_is_decode_then_bf16():
+    wl, xs = _traj("tiny", steps=2)
+    recon_s, _ = oracle.state_init(xs[0])
+    recon_r = recon_s.copy()
+    codes, scales, _ = oracle.encode(xs[1], recon_s, 1)
+    out = oracle.decode_emit(codes, scales, recon_r, 1)
+    assert np.array_equal(recon_r, recon_s)
+    ref = torch.from_numpy(recon_r).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(out, ref)
