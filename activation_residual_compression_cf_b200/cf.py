@@ -28,7 +28,7 @@ EXPORTS = ("cf_status_string", "cf_abi_version", "cf_codes_words_per_row",
            "cf_lowrank_factor_bytes", "cf_lowrank_encode", "cf_lowrank_decode",
            "cf_lowrank_status", "cf_set_lowrank_engine", "cf_set_quant_pipeline",
            "cf_set_launch_override", "cf_lowrank_encode_noalloc", "cf_decode_emit",
-           "cf_decode_emit_batched")
+           "cf_decode_emit_batched", "cf_lowrank_encode_batched", "cf_lowrank_decode_batched")
 
 
 class CFError(RuntimeError):
@@ -52,6 +52,19 @@ class cf_enc_buffer(ctypes.Structure):
 
 class cf_dec_buffer(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("recon_r", ctypes.c_void_p)]
+
+
+class cf_lowrank_buffer(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("recon_s", ctypes.c_void_p), ("err", ctypes.c_void_p),
+                ("omega", ctypes.c_void_p), ("p_codes", ctypes.c_void_p),
+                ("p_scales", ctypes.c_void_p), ("q_codes", ctypes.c_void_p),
+                ("q_scales", ctypes.c_void_p)]
+
+
+class cf_lowrank_dec_buffer(ctypes.Structure):
+    _fields_ = [("p_codes", ctypes.c_void_p), ("p_scales", ctypes.c_void_p),
+                ("q_codes", ctypes.c_void_p), ("q_scales", ctypes.c_void_p),
                 ("recon_r", ctypes.c_void_p)]
 
 
@@ -90,6 +103,8 @@ def lib():
             "cf_lowrank_encode": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
             "cf_lowrank_decode": ([D, vp, vp, vp, vp, vp, vp], ctypes.c_int),
             "cf_lowrank_status": ([vp, vp], ctypes.c_int),
+            "cf_lowrank_encode_batched": ([D, i32, vp, vp, sz, vp], ctypes.c_int),
+            "cf_lowrank_decode_batched": ([D, i32, vp, vp, vp], ctypes.c_int),
             "cf_set_launch_override": ([i32, i32, i32, i32], ctypes.c_int),
             "cf_set_lowrank_engine": ([i32], ctypes.c_int),
             "cf_set_quant_pipeline": ([i32, i32, i32], ctypes.c_int),
@@ -210,6 +225,17 @@ def cf_lowrank_decode(d, p_codes, p_scales, q_codes, q_scales, recon_r, stream=N
                                  _p(q_scales), _p(recon_r), _s(stream)), "cf_lowrank_decode")
 
 
+def cf_lowrank_encode_batched(d, n, bufs_dev, workspace, workspace_bytes=None, stream=None):
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _chk(lib().cf_lowrank_encode_batched(ctypes.byref(d), n, _p(bufs_dev), _p(workspace), nbytes,
+                                         _s(stream)), "cf_lowrank_encode_batched")
+
+
+def cf_lowrank_decode_batched(d, n, bufs_dev, status_dev=None, stream=None):
+    _chk(lib().cf_lowrank_decode_batched(ctypes.byref(d), n, _p(bufs_dev), _p(status_dev),
+                                         _s(stream)), "cf_lowrank_decode_batched")
+
+
 def cf_lowrank_status(workspace, stream=None) -> int:
     """Synchronises the stream; returns (and clears) the workspace status."""
     return lib().cf_lowrank_status(_p(workspace), _s(stream))
@@ -249,6 +275,24 @@ def dec_buffer_array(sets, device) -> torch.Tensor:
         arr[i] = cf_dec_buffer(_p(c), _p(s), _p(r))
     host = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8)
     return host.to(device)
+
+
+def lowrank_buffer_array(sets, device) -> torch.Tensor:
+    """Device array of cf_lowrank_buffer from
+    [(x, recon_s, err, omega, p_codes, p_scales, q_codes, q_scales), ...]."""
+    arr = (cf_lowrank_buffer * len(sets))()
+    for i, t in enumerate(sets):
+        arr[i] = cf_lowrank_buffer(*[_p(v) for v in t])
+    return torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
+
+
+def lowrank_dec_buffer_array(sets, device) -> torch.Tensor:
+    """Device array of cf_lowrank_dec_buffer from
+    [(p_codes, p_scales, q_codes, q_scales, recon_r), ...]."""
+    arr = (cf_lowrank_dec_buffer * len(sets))()
+    for i, t in enumerate(sets):
+        arr[i] = cf_lowrank_dec_buffer(*[_p(v) for v in t])
+    return torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
 
 
 def dec_emit_buffer_array(sets, device) -> torch.Tensor:

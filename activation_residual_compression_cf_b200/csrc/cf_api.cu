@@ -79,15 +79,16 @@ struct Shape {
 };
 
 // Launch shape per row: threads (a multiple of 32) x groups of 8 channels
-// per thread.  Measured on B200 at C = 3072 (114 x 1024 rows): the TMA
-// pipeline is fastest with 4 groups per thread (fewer, busier consumer
-// warps), the register pipeline with 2 groups per thread.
-Shape choose_shape(int kernel, int64_t C, int pipeline) {
+// per thread.  Chosen from sweeps on B200 timed in the encode -> decode
+// sequence (C = 3072, 114 x 1024 and 114 x 4096 rows): TMA encode is fastest
+// with 4 groups per thread at 2 bits and 3 at 1 bit, TMA decode with 3; the
+// register pipeline with 2.
+Shape choose_shape(int kernel, int64_t C, int pipeline, int bits) {
     const int64_t G = (C + 7) / 8;
     Shape s;
     int gpt;
     if (pipeline == 1) {
-        gpt = kMaxGroupsPerThread;
+        gpt = kernel == 0 ? (bits == 1 ? 3 : 4) : 3;
     } else {
         gpt = (int)((G + 191) / 192);
         if (gpt < 2) gpt = 2;
@@ -158,13 +159,12 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
                      const Shape &s, int stages_req, cudaStream_t st) {
     const int64_t W = (C * BITS + 31) / 32;
     const int64_t slot = ENC ? 6 * C : 4 * W + 4 * C;
-    // Ring depth: measured on B200 (C = 1920 and 3072), 5 slots for encode
-    // and 6 for decode are at or near the best; deeper rings cost CTAs per SM.
+    // Ring depth: measured on B200 (C = 1920 and 3072), 5 slots for both
+    // kernels are at or near the best; deeper rings cost CTAs per SM.
     int stages = stages_req;
     if (stages <= 0) {
         stages = (int)(120000 / slot);
-        const int cap = ENC ? 5 : 6;
-        if (stages > cap) stages = cap;
+        if (stages > 5) stages = 5;
     }
     if (stages > 8) stages = 8;
     if (stages < 2) stages = 2;
@@ -227,8 +227,8 @@ cf_status dispatch(const Src &src, int bits, int64_t T, int64_t C, int64_t rows,
         pipe = g_pipeline[ENC ? 0 : 1];
     }
     if (pipe == 1 && !tma_applies(ENC, bits, C)) pipe = 0;
-    Shape s = choose_shape(ENC ? 0 : 1, C, pipe);
-    if (pipe == 1 && s.threads > 480) s = choose_shape(ENC ? 0 : 1, C, pipe = 0);
+    Shape s = choose_shape(ENC ? 0 : 1, C, pipe, bits);
+    if (pipe == 1 && s.threads > 480) s = choose_shape(ENC ? 0 : 1, C, pipe = 0, bits);
     s.pipeline = pipe;
     const bool vec = (C % 8) == 0;
 #define CF_CASE(B, G, V)                                     \

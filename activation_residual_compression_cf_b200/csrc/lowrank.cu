@@ -86,9 +86,9 @@ namespace {
 
 using namespace cf_lowrank;
 
-cf_status check_ptr(const void *p) {
+cf_status check_ptr(const void *p, uintptr_t align = 16) {
     if (!p) return CF_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0) return CF_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(p) & (align - 1)) != 0) return CF_ERR_ALIGNMENT;
     cudaPointerAttributes a;
     if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
         (void)cudaGetLastError();
@@ -107,15 +107,14 @@ cf_status check_ptr(const void *p) {
         if (_s != CF_OK) return _s; \
     } while (0)
 
-#define LR_LAUNCHED()                                                  \
-    do {                                                               \
-        if (cudaGetLastError() != cudaSuccess) return CF_ERR_CUDA;     \
+#define LR_LAUNCHED()                                              \
+    do {                                                           \
+        if (cudaGetLastError() != cudaSuccess) return CF_ERR_CUDA; \
     } while (0)
 
 int sm_count() {
     int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     return n;
 }
 
@@ -144,86 +143,83 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor map over a row-major [rows][cols] array (row pitch `pitch`
-// elements), box {64 columns, box_rows rows}, 128-byte swizzle, zero fill
-// outside the array.
+// 3-D bf16 tensor map over n buffers of a row-major [rows][cols] array each
+// (row pitch `pitch` elements, buffer stride `bstride` bytes), box {64
+// columns, box_rows rows, 1 buffer}, 128-byte swizzle, zero fill outside.
 bool make_map(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, int64_t pitch,
-              uint32_t box_rows) {
+              int64_t n, int64_t bstride, uint32_t box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)pitch * 2};
-    const cuuint32_t box[2] = {64, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+    const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)n};
+    const cuuint64_t strides[2] = {(cuuint64_t)pitch * 2, (cuuint64_t)bstride};
+    const cuuint32_t box[3] = {64, box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int BN>
-cf_status launch_project(const Layout &L, const __nv_bfloat16 *vb, const __nv_bfloat16 *qt,
-                         float *yp, int32_t *status, cudaStream_t st) {
+cf_status launch_project(const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
     CUtensorMap mv, mq;
-    if (!make_map(&mv, vb, L.C, L.T, L.C, 128) || !make_map(&mq, qt, L.C, L.rp, L.C, BN))
+    if (!make_map(&mv, B.ws + L.off_vb, L.C, L.T, L.C, n, B.ws_stride, 128) ||
+        !make_map(&mq, B.ws + L.off_qt, L.C, L.rp, L.C, n, B.ws_stride, BN))
         return CF_ERR_CUDA;
     auto k = cf::umma::project_kernel<BN>;
     const int smem = cf::umma::StageGeom<BN>::kSmem;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return CF_ERR_CUDA;
-    dim3 grid((unsigned)((L.T + 127) / 128), (unsigned)L.splitsA);
-    k<<<grid, 128, smem, st>>>(mv, mq, yp, L.T, L.C, kChunkA, status);
+    dim3 grid((unsigned)((L.T + 127) / 128), (unsigned)L.splitsA, (unsigned)n);
+    k<<<grid, 128, smem, st>>>(mv, mq, B, L);
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 
 template <int BN>
-cf_status launch_backproject(const Layout &L, const __nv_bfloat16 *vb, const __nv_bfloat16 *pt,
-                             float *zp, int32_t *status, cudaStream_t st) {
+cf_status launch_backproject(const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
     CUtensorMap mv, mp;
-    if (!make_map(&mv, vb, L.C, L.T, L.C, 64) || !make_map(&mp, pt, L.Tp, L.rp, L.Tp, BN))
+    if (!make_map(&mv, B.ws + L.off_vb, L.C, L.T, L.C, n, B.ws_stride, 64) ||
+        !make_map(&mp, B.ws + L.off_pt, L.Tp, L.rp, L.Tp, n, B.ws_stride, BN))
         return CF_ERR_CUDA;
     auto k = cf::umma::backproject_kernel<BN>;
     const int smem = cf::umma::StageGeom<BN>::kSmem;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return CF_ERR_CUDA;
-    dim3 grid((unsigned)((L.C + 127) / 128), (unsigned)L.splitsB);
-    k<<<grid, 128, smem, st>>>(mv, mp, zp, L.T, L.C, kChunkB, status);
+    dim3 grid((unsigned)((L.C + 127) / 128), (unsigned)L.splitsB, (unsigned)n);
+    k<<<grid, 128, smem, st>>>(mv, mp, B, L);
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 
-cf_status project(const Layout &L, const __nv_bfloat16 *vb, const __nv_bfloat16 *qt, float *yp,
-                  int32_t *status, cudaStream_t st) {
+cf_status project(const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
     if (g_engine.load() == 0) {
         switch (L.rp) {
-            case 16: return launch_project<16>(L, vb, qt, yp, status, st);
-            case 32: return launch_project<32>(L, vb, qt, yp, status, st);
-            case 48: return launch_project<48>(L, vb, qt, yp, status, st);
-            case 64: return launch_project<64>(L, vb, qt, yp, status, st);
+            case 16: return launch_project<16>(B, L, n, st);
+            case 32: return launch_project<32>(B, L, n, st);
+            case 48: return launch_project<48>(B, L, n, st);
+            case 64: return launch_project<64>(B, L, n, st);
         }
     }
-    cf::lr_project_simt<<<dim3((unsigned)((L.T + 63) / 64), (unsigned)L.splitsA), 256, 0, st>>>(
-        vb, qt, yp, L.T, L.C, L.rp);
+    cf::lr_project_simt<<<dim3((unsigned)((L.T + 63) / 64), (unsigned)L.splitsA, (unsigned)n), 256, 0,
+                          st>>>(B, L);
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 
-cf_status backproject(const Layout &L, const __nv_bfloat16 *vb, const __nv_bfloat16 *pt, float *zp,
-                      int32_t *status, cudaStream_t st) {
+cf_status backproject(const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
     if (g_engine.load() == 0) {
         switch (L.rp) {
-            case 16: return launch_backproject<16>(L, vb, pt, zp, status, st);
-            case 32: return launch_backproject<32>(L, vb, pt, zp, status, st);
-            case 48: return launch_backproject<48>(L, vb, pt, zp, status, st);
-            case 64: return launch_backproject<64>(L, vb, pt, zp, status, st);
+            case 16: return launch_backproject<16>(B, L, n, st);
+            case 32: return launch_backproject<32>(B, L, n, st);
+            case 48: return launch_backproject<48>(B, L, n, st);
+            case 64: return launch_backproject<64>(B, L, n, st);
         }
     }
-    cf::lr_backproject_simt<<<dim3((unsigned)((L.C + 63) / 64), (unsigned)L.splitsB), 256, 0, st>>>(
-        vb, pt, zp, L.T, L.Tp, L.C, L.rp);
+    cf::lr_backproject_simt<<<dim3((unsigned)((L.C + 63) / 64), (unsigned)L.splitsB, (unsigned)n), 256,
+                              0, st>>>(B, L);
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 
-cf_status orth(const Layout &L, const float *y, const float *rmat, const float *rinvd, float *p,
-               __nv_bfloat16 *pt, uint32_t *amax, cudaStream_t st) {
-    const unsigned grid = (unsigned)((L.Tp + 63) / 64);
-#define CF_ORTH(RP) cf::lr_orth_kernel<RP><<<grid, 64, 0, st>>>(y, rmat, rinvd, p, pt, L.T, L.Tp, amax)
+cf_status orth(const LrBatch &B, const Layout &L, int n, bool last, cudaStream_t st) {
+    const dim3 grid((unsigned)((L.Tp + 63) / 64), 1, (unsigned)n);
+#define CF_ORTH(RP) cf::lr_orth_kernel<RP><<<grid, 64, 0, st>>>(B, L, last ? 1 : 0)
     switch (L.rp) {
         case 16: CF_ORTH(16); break;
         case 32: CF_ORTH(32); break;
@@ -235,10 +231,9 @@ cf_status orth(const Layout &L, const float *y, const float *rmat, const float *
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 
-cf_status reduce_q(const Layout &L, const float *zp, float *q, __nv_bfloat16 *qt, uint32_t *amax,
-                   cudaStream_t st) {
-    const unsigned grid = (unsigned)((L.C + 31) / 32);
-#define CF_RQ(RP) cf::lr_reduce_q_kernel<RP><<<grid, 32, 0, st>>>(zp, q, qt, L.C, L.splitsB, amax)
+cf_status reduce_q(const LrBatch &B, const Layout &L, int n, bool last, cudaStream_t st) {
+    const dim3 grid((unsigned)((L.C + 31) / 32), 1, (unsigned)n);
+#define CF_RQ(RP) cf::lr_reduce_q_kernel<RP><<<grid, 32, 0, st>>>(B, L, last ? 1 : 0)
     switch (L.rp) {
         case 16: CF_RQ(16); break;
         case 32: CF_RQ(32); break;
@@ -250,57 +245,79 @@ cf_status reduce_q(const Layout &L, const float *zp, float *q, __nv_bfloat16 *qt
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 
-template <class T>
-T *at(void *ws, size_t off) {
-    return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
-}
-
 template <bool SENDER, int KP>
-cf_status launch_apply_tc(const Layout &L, const uint16_t *x, float *recon, float *err,
-                          const uint8_t *pc, const float *ps, const uint8_t *qc, const float *qs,
-                          int32_t *status, cudaStream_t st) {
+cf_status launch_apply_tc(const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
     auto k = cf::umma::lr_apply_tc_kernel<SENDER, KP>;
-    constexpr int smem = cf::umma::apply_tc_smem<KP>();
+    constexpr int smem = cf::umma::apply_tc_smem<SENDER, KP>();
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return CF_ERR_CUDA;
-    dim3 grid((unsigned)((L.C + 127) / 128), (unsigned)((L.T + 127) / 128));
-    k<<<grid, 256, smem, st>>>(x, recon, err, pc, ps, qc, qs, L.T, L.C, L.r, status);
+    dim3 grid((unsigned)((L.C + 127) / 128), (unsigned)((L.T + 127) / 128), (unsigned)n);
+    k<<<grid, cf::umma::kApplyThreads, smem, st>>>(B, L);
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 
 // D = P^ Q^T applied to the state.  Engine 0: tensor cores (tcgen05 tf32,
 // hi/lo split); engine 1: CUDA-core FMA chain.  A buffer's sender and
 // receiver must use the same engine to stay bit-identical.
-cf_status apply(bool sender, const Layout &L, const uint16_t *x, float *recon, float *err,
-                const uint8_t *pc, const float *ps, const uint8_t *qc, const float *qs,
-                int32_t *status, cudaStream_t st) {
+cf_status apply(bool sender, const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
     if (g_engine.load() == 0) {
         if (L.rp <= 32)
-            return sender ? launch_apply_tc<true, 32>(L, x, recon, err, pc, ps, qc, qs, status, st)
-                          : launch_apply_tc<false, 32>(L, x, recon, err, pc, ps, qc, qs, status, st);
-        return sender ? launch_apply_tc<true, 64>(L, x, recon, err, pc, ps, qc, qs, status, st)
-                      : launch_apply_tc<false, 64>(L, x, recon, err, pc, ps, qc, qs, status, st);
+            return sender ? launch_apply_tc<true, 32>(B, L, n, st) : launch_apply_tc<false, 32>(B, L, n, st);
+        return sender ? launch_apply_tc<true, 64>(B, L, n, st) : launch_apply_tc<false, 64>(B, L, n, st);
     }
     const int64_t gx = (L.C + kApplyCh - 1) / kApplyCh;
     const int64_t ntiles = (L.T + kApplyTok - 1) / kApplyTok;
     int64_t gy = (2 * (int64_t)sm_count() + gx - 1) / gx;
     if (gy > ntiles) gy = ntiles;
     if (gy < 1) gy = 1;
-    dim3 grid((unsigned)gx, (unsigned)gy);
+    dim3 grid((unsigned)gx, (unsigned)gy, (unsigned)n);
     const size_t smem = (size_t)L.r * (kApplyTok + kApplyCh) * sizeof(float);
     if (sender) {
         auto k = cf::lr_apply_kernel<true>;
         if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return CF_ERR_CUDA;
-        k<<<grid, kApplyThreads, smem, st>>>(x, recon, err, pc, ps, qc, qs, L.T, L.C, L.r);
+        k<<<grid, kApplyThreads, smem, st>>>(B, L);
     } else {
         auto k = cf::lr_apply_kernel<false>;
         if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return CF_ERR_CUDA;
-        k<<<grid, kApplyThreads, smem, st>>>(nullptr, recon, nullptr, pc, ps, qc, qs, L.T, L.C, L.r);
+        k<<<grid, kApplyThreads, smem, st>>>(B, L);
     }
     LR_LAUNCHED();
     return CF_OK;
+}
+
+// The whole sender for n buffers (n = 1 for the single-buffer call).
+cf_status encode_impl(const cf_desc *d, const Layout &L, int n, const LrBatch &B, cudaStream_t st) {
+    const int nb = (L.r + 1) / 2;
+    cf::lr_prep_kernel<<<(unsigned)n, 128, 0, st>>>(B, L);
+    LR_LAUNCHED();
+    {
+        const int64_t groups = L.T * L.C / 8;
+        int64_t blocks = (groups + 255) / 256;
+        const int64_t cap = (int64_t)sm_count() * 8 / n + 1;
+        if (blocks > cap) blocks = cap;
+        cf::lr_residual_kernel<<<dim3((unsigned)blocks, 1, (unsigned)n), 256, 0, st>>>(B, L);
+        LR_LAUNCHED();
+        const int64_t nq = (int64_t)L.rp * L.C;
+        cf::lr_omega_kernel<<<dim3((unsigned)((nq + 255) / 256), 1, (unsigned)n), 256, 0, st>>>(B, L);
+        LR_LAUNCHED();
+    }
+    for (int it = 0; it < d->iters; ++it) {
+        const bool last = (it == d->iters - 1);
+        LR_TRY(project(B, L, n, st));
+        cf::lr_gram_chol_kernel<<<dim3((unsigned)L.nGram, 1, (unsigned)n), 256, 0, st>>>(B, L);
+        LR_LAUNCHED();
+        LR_TRY(orth(B, L, n, last, st));
+        LR_TRY(backproject(B, L, n, st));
+        LR_TRY(reduce_q(B, L, n, last, st));
+    }
+    // INT4 factors: quantise and pack against the column maxima.
+    cf::lr_int4_pack_kernel<<<dim3((unsigned)((L.T * nb + 255) / 256), 1, (unsigned)n), 256, 0, st>>>(B, L, 0);
+    LR_LAUNCHED();
+    cf::lr_int4_pack_kernel<<<dim3((unsigned)((L.C * nb + 255) / 256), 1, (unsigned)n), 256, 0, st>>>(B, L, 1);
+    LR_LAUNCHED();
+    return apply(true, B, L, n, st);
 }
 
 }  // namespace
@@ -328,68 +345,43 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
     LR_TRY(check_ptr(x));
     LR_TRY(check_ptr(recon_s));
     LR_TRY(check_ptr(err));
-    LR_TRY(check_ptr(omega));
-    LR_TRY(check_ptr(p_codes));
-    LR_TRY(check_ptr(p_scales));
-    LR_TRY(check_ptr(q_codes));
-    LR_TRY(check_ptr(q_scales));
+    LR_TRY(check_ptr(omega, 4));
+    LR_TRY(check_ptr(p_codes, 1));
+    LR_TRY(check_ptr(p_scales, 4));
+    LR_TRY(check_ptr(q_codes, 1));
+    LR_TRY(check_ptr(q_scales, 4));
     LR_TRY(check_ptr(workspace));
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return CF_ERR_ALIGNMENT;
-    cudaStream_t st = (cudaStream_t)stream;
-    void *ws = workspace;
-    const int64_t T = L.T, C = L.C;
-    const int r = L.r, rp = L.rp;
+    LrBatch B = {};
+    B.one.x = x;
+    B.one.recon = recon_s;
+    B.one.err = err;
+    B.one.omega = omega;
+    B.one.pc = B.one.pc_out = p_codes;
+    B.one.ps = B.one.ps_out = p_scales;
+    B.one.qc = B.one.qc_out = q_codes;
+    B.one.qs = B.one.qs_out = q_scales;
+    B.ws = static_cast<uint8_t *>(workspace);
+    B.ws_stride = (int64_t)L.total;
+    return encode_impl(d, L, 1, B, (cudaStream_t)stream);
+}
 
-    int32_t *status = at<int32_t>(ws, L.off_status);
-    double *gp = at<double>(ws, L.off_gp);
-    double *gg = at<double>(ws, L.off_gg);
-    uint32_t *gticket = at<uint32_t>(ws, L.off_gt);
-    float *rmat = at<float>(ws, L.off_rmat);
-    float *rinvd = rmat + rp * rp;
-    uint32_t *ticket = reinterpret_cast<uint32_t *>(status + 1);
-    uint32_t *amax = at<uint32_t>(ws, L.off_amax);
-    __nv_bfloat16 *vb = at<__nv_bfloat16>(ws, L.off_vb);
-    __nv_bfloat16 *qt = at<__nv_bfloat16>(ws, L.off_qt);
-    float *yp = at<float>(ws, L.off_yp);
-    float *y = at<float>(ws, L.off_y);
-    float *p = at<float>(ws, L.off_p);
-    __nv_bfloat16 *pt = at<__nv_bfloat16>(ws, L.off_pt);
-    float *zp = at<float>(ws, L.off_zp);
-    float *q = at<float>(ws, L.off_q);
-
-    // status word and tickets start at zero
-    if (cudaMemsetAsync(status, 0, L.off_gp, st) != cudaSuccess) return CF_ERR_CUDA;
-    if (cudaMemsetAsync(amax, 0, (size_t)2 * rp * 4, st) != cudaSuccess) return CF_ERR_CUDA;
-    const int sms = sm_count();
-    {
-        const int64_t groups = T * C / 8;
-        int64_t blocks = (groups + 255) / 256;
-        if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-        cf::lr_residual_kernel<<<(unsigned)blocks, 256, 0, st>>>(x, recon_s, vb, T * C);
-        LR_LAUNCHED();
-        const int64_t nq = (int64_t)rp * C;
-        cf::lr_omega_kernel<<<(unsigned)((nq + 255) / 256), 256, 0, st>>>(omega, qt, C, r, rp);
-        LR_LAUNCHED();
-    }
-    for (int it = 0; it < d->iters; ++it) {
-        LR_TRY(project(L, vb, qt, yp, status, st));
-        {
-            cf::lr_gram_chol_kernel<<<(unsigned)L.nGram, 256, 0, st>>>(
-                yp, y, gp, gg, T, r, rp, L.splitsA, rmat, rinvd, gticket, ticket, status);
-            LR_LAUNCHED();
-        }
-        const bool last = (it == d->iters - 1);
-        LR_TRY(orth(L, y, rmat, rinvd, p, pt, last ? amax : nullptr, st));
-        LR_TRY(backproject(L, vb, pt, zp, status, st));
-        LR_TRY(reduce_q(L, zp, q, qt, last ? amax + rp : nullptr, st));
-    }
-    // INT4 factors: quantise and pack against the column maxima.
-    const int nb = (r + 1) / 2;
-    cf::lr_int4_pack_kernel<<<(unsigned)((T * nb + 255) / 256), 256, 0, st>>>(p, T, r, rp, amax, p_codes, p_scales);
-    LR_LAUNCHED();
-    cf::lr_int4_pack_kernel<<<(unsigned)((C * nb + 255) / 256), 256, 0, st>>>(q, C, r, rp, amax + rp, q_codes, q_scales);
-    LR_LAUNCHED();
-    return apply(true, L, x, recon_s, err, p_codes, p_scales, q_codes, q_scales, status, st);
+cf_status cf_lowrank_encode_batched(const cf_desc *d, int32_t n, const cf_lowrank_buffer *bufs_dev,
+                                    void *workspace, size_t workspace_bytes, void *stream) {
+    LR_TRY(check_desc(d));
+    if (n < 0) return CF_ERR_INVALID_ARG;
+    if (n == 0 || d->tokens == 0) return CF_OK;
+    if (n > 65535) return CF_ERR_UNSUPPORTED;
+    const Layout L = make_layout(d->tokens, d->channels, d->rank);
+    if (workspace_bytes / (size_t)n < L.total) return CF_ERR_WORKSPACE;
+    LR_TRY(check_ptr(bufs_dev));
+    LR_TRY(check_ptr(workspace));
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return CF_ERR_ALIGNMENT;
+    LrBatch B = {};
+    B.enc = bufs_dev;
+    B.ws = static_cast<uint8_t *>(workspace);
+    B.ws_stride = (int64_t)L.total;
+    return encode_impl(d, L, n, B, (cudaStream_t)stream);
 }
 
 cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes, const float *p_scales,
@@ -397,14 +389,34 @@ cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes, const floa
                             void *stream) {
     LR_TRY(check_desc(d));
     if (d->tokens == 0) return CF_OK;
-    LR_TRY(check_ptr(p_codes));
-    LR_TRY(check_ptr(p_scales));
-    LR_TRY(check_ptr(q_codes));
-    LR_TRY(check_ptr(q_scales));
+    LR_TRY(check_ptr(p_codes, 1));
+    LR_TRY(check_ptr(p_scales, 4));
+    LR_TRY(check_ptr(q_codes, 1));
+    LR_TRY(check_ptr(q_scales, 4));
     LR_TRY(check_ptr(recon_r));
     const Layout L = make_layout(d->tokens, d->channels, d->rank);
-    return apply(false, L, nullptr, recon_r, nullptr, p_codes, p_scales, q_codes, q_scales,
-                 nullptr, (cudaStream_t)stream);
+    LrBatch B = {};
+    B.one.pc = p_codes;
+    B.one.ps = p_scales;
+    B.one.qc = q_codes;
+    B.one.qs = q_scales;
+    B.one.recon = recon_r;
+    return apply(false, B, L, 1, (cudaStream_t)stream);
+}
+
+cf_status cf_lowrank_decode_batched(const cf_desc *d, int32_t n, const cf_lowrank_dec_buffer *bufs_dev,
+                                    int32_t *status_dev, void *stream) {
+    LR_TRY(check_desc(d));
+    if (n < 0) return CF_ERR_INVALID_ARG;
+    if (n == 0 || d->tokens == 0) return CF_OK;
+    if (n > 65535) return CF_ERR_UNSUPPORTED;
+    LR_TRY(check_ptr(bufs_dev));
+    if (status_dev) LR_TRY(check_ptr(status_dev, 4));
+    const Layout L = make_layout(d->tokens, d->channels, d->rank);
+    LrBatch B = {};
+    B.dec = bufs_dev;
+    B.dec_status = status_dev;
+    return apply(false, B, L, n, (cudaStream_t)stream);
 }
 
 cf_status cf_set_lowrank_engine(int32_t engine) {

@@ -11,15 +11,18 @@
 // The split keeps ~21 significant bits of every product, so D matches the
 // exact product of the payload to ~1e-6 relative.  Sender and receiver run
 // this same kernel on the same payload, so their D is bit-identical.
-// Epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (channels), token
-// columns 64 (w / 4) .. +63, 16 at a time; for each token its 32 lanes touch
-// 32 consecutive channels, i.e. one 128-byte transaction per warp per array.
+// Epilogue: x and recon arrive in shared memory through bulk copies issued
+// by a producer warp (below); warp w reads TMEM lanes 32 (w % 4) .. +31
+// (channels) and, of every 16-token stage, the token columns of half w / 4;
+// for each token its 32 lanes write 32 consecutive channels, one 128-byte
+// transaction per warp per array.
 #pragma once
 
 #include <cuda_bf16.h>
 
 #include "cf.h"
 #include "cf_common.cuh"
+#include "lowrank_kernels.cuh"
 #include "lowrank_umma.cuh"
 
 namespace cf {
@@ -59,26 +62,100 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v) {
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Staging of x and recon: the tile's 128 tokens are 8 stages of 16 token
+// rows; a stage holds the rows' recon (16 x 128 fp32) and, for the sender,
+// x (16 x 128 bf16).  Ring depth per kernel, sized so that the sender with
+// rank <= 32 keeps two CTAs per SM.
+constexpr int kApplyStageTok = 16;
+constexpr int kApplyStagesPerTile = kApplyTile / kApplyStageTok;
+constexpr int kApplyConsumers = 256;            // 8 warps: 4 channel quarters x 2 token halves
+constexpr int kApplyThreads = kApplyConsumers + 32;  // + one producer warp
+
+template <bool SENDER>
+__host__ __device__ constexpr int apply_stage_bytes() {
+    return kApplyStageTok * kApplyTile * (SENDER ? 6 : 4);
+}
 template <bool SENDER, int KP>
-__global__ void __launch_bounds__(256, 2)
-lr_apply_tc_kernel(const uint16_t *x, float *recon, float *err, const uint8_t *pc, const float *ps,
-                   const uint8_t *qc, const float *qs, int64_t T, int64_t C, int r, int32_t *status) {
+__host__ __device__ constexpr int apply_ring() {
+    return KP <= 32 ? (SENDER ? 4 : 6) : 8;
+}
+template <bool SENDER, int KP>
+__host__ __device__ constexpr int apply_tc_smem() {
+    return 1024 + 3 * (KP / 32) * 16384 + apply_ring<SENDER, KP>() * apply_stage_bytes<SENDER>() + 256;
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void consumers_sync() {
+    asm volatile("bar.sync 1, %0;" ::"r"(kApplyConsumers) : "memory");
+}
+
+// Warp roles (288 threads):
+//   warps 0-7 : build the MMA operands, thread 0 issues the MMAs; then each
+//               warp combines one channel quarter (w % 4, its TMEM lanes) x
+//               one half (w / 4) of every 16-token stage, reading x and recon
+//               from shared memory and D from TMEM, and writes err and recon
+//               to global memory;
+//   warp 8    : one lane issues 1-D bulk copies (cp.async.bulk, no multicast)
+//               of every token row's 128-channel segment of recon (and x)
+//               into the ring, from the kernel's first instructions on, so the
+//               HBM reads overlap the operand build and the MMA.
+// Every wait is bounded; on expiry CF_ERR_TIMEOUT goes to the buffer's status
+// word, the warps stop, the producer waits (bounded) for its copies still in
+// flight, and TMEM is freed.
+template <bool SENDER, int KP>
+__global__ void __launch_bounds__(kApplyThreads, (KP <= 32 ? 2 : 1))
+lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L) {
+    const int bz = blockIdx.z;
+    if (lr_skipped(B, L, bz)) return;
+    const cf_lowrank::LrPtrs pp = B.get(bz);
+    if (!SENDER && B.dec && !lr_dec_ptrs_ok(B, pp)) return;
+    const uint16_t *x = pp.x;
+    float *recon = pp.recon, *err = pp.err;
+    const uint8_t *pc = pp.pc, *qc = pp.qc;
+    const float *ps = pp.ps, *qs = pp.qs;
+    const int64_t T = L.T, C = L.C;
+    const int r = L.r;
+    int32_t *status = B.ws ? B.at<int32_t>(bz, L.off_status) + cf_lowrank::kStatusWord
+                           : (SENDER ? nullptr : B.dec_status);
     constexpr int NA = KP / 32;       // 128-byte K atoms per operand
     constexpr int OPB = NA * 16384;   // bytes per operand tile
+    constexpr int S = apply_ring<SENDER, KP>();
+    constexpr int SB = apply_stage_bytes<SENDER>();
+    constexpr int RB = kApplyStageTok * kApplyTile * 4;  // recon part of a stage
     extern __shared__ uint8_t dsm[];
     const uint32_t base = (smem_u32(dsm) + 1023u) & ~1023u;
     uint8_t *gb = dsm + (base - smem_u32(dsm));
     const uint32_t sA = base, sBh = base + OPB, sBl = base + 2 * OPB;
-    const uint32_t bar = base + 3 * OPB;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(gb + 3 * OPB + 8);
+    const uint32_t ring = base + 3 * OPB;
+    uint8_t *gring = gb + 3 * OPB;
+    const uint32_t bars = ring + S * SB;       // mma, full[S], empty[S]
+    const uint32_t mma_bar = bars;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(gring + S * SB + 8 * (1 + 2 * S));
+    int *abort_flag = reinterpret_cast<int *>(tslot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t c0 = (int64_t)blockIdx.x * kApplyTile;
     const int64_t t0 = (int64_t)blockIdx.y * kApplyTile;
     const int nb = (r + 1) / 2;
+    const int64_t cw = (C - c0 < kApplyTile) ? C - c0 : kApplyTile;   // channels in this tile
+    const int64_t tw = (T - t0 < kApplyTile) ? T - t0 : kApplyTile;   // tokens in this tile
+    const int ns = (int)((tw + kApplyStageTok - 1) / kApplyStageTok);  // stages in this tile
 
     if (tid == 0) {
-        mbar_init(bar, 1);
+        mbar_init(mma_bar, 1);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(bars + 8u * (1 + s), 1);                  // full: producer + tx bytes
+            mbar_init(bars + 8u * (1 + S + s), kApplyConsumers / 32);  // empty: one per warp
+        }
+        *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -88,82 +165,125 @@ lr_apply_tc_kernel(const uint16_t *x, float *recon, float *err, const uint8_t *p
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // operands: 16-byte chunks of 4 consecutive k per store
-    for (int idx = tid; idx < kApplyTile * (KP / 4); idx += blockDim.x) {
-        const int row = idx / (KP / 4), k0 = (idx - row * (KP / 4)) * 4;
-        const int64_t c = c0 + row, t = t0 + row;
-        float a[4], h[4], l[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int k = k0 + u;
-            a[u] = (c < C && k < r) ? (float)int4_code_at(qc + c * nb, k) : 0.0f;
-            float b = 0.0f;
-            if (t < T && k < r)
-                b = __fmul_rn((float)int4_code_at(pc + t * nb, k), __fmul_rn(__ldg(ps + k), __ldg(qs + k)));
-            h[u] = __uint_as_float(__float_as_uint(b) & 0xFFFFE000u);
-            l[u] = __fsub_rn(b, h[u]);
-        }
-        const uint32_t off = sw128_f32_offset(row, k0);
-        *reinterpret_cast<float4 *>(gb + off) = make_float4(a[0], a[1], a[2], a[3]);
-        *reinterpret_cast<float4 *>(gb + OPB + off) = make_float4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<float4 *>(gb + 2 * OPB + off) = make_float4(l[0], l[1], l[2], l[3]);
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tslot;
-    if (tid == 0) {
-        constexpr uint32_t idesc = idesc_tf32(kApplyTile);
-        const int ksteps = (r + 7) / 8;
-        for (int kk = 0; kk < ksteps; ++kk) {
-            const uint32_t off = (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32);
-            const uint64_t da = sw128_desc(sA + off, 16, 1024);
-            mma_tf32(tmem, da, sw128_desc(sBh + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
-            mma_tf32(tmem, da, sw128_desc(sBl + off, 16, 1024), idesc, 1u);
+
+    if (warp == kApplyConsumers / 32) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            const uint32_t rbytes = (uint32_t)cw * 4u, xbytes = (uint32_t)cw * 2u;
+            int issued = 0;
+            bool ok = true;
+            for (int st = 0; st < ns; ++st) {
+                const int slot = st % S;
+                if (st >= S && !mbar_wait(bars + 8u * (1 + S + slot), (uint32_t)((st / S - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                const int64_t tb = t0 + (int64_t)st * kApplyStageTok;
+                const int rows = (int)((T - tb < kApplyStageTok) ? T - tb : kApplyStageTok);
+                const uint32_t full = bars + 8u * (1 + slot);
+                const uint32_t dst = ring + (uint32_t)(slot * SB);
+                mbar_expect_tx(full, (uint32_t)rows * (rbytes + (SENDER ? xbytes : 0u)));
+                for (int j = 0; j < rows; ++j) {
+                    const int64_t o = (tb + j) * C + c0;
+                    bulk_g2s(dst + (uint32_t)(j * kApplyTile * 4), recon + o, rbytes, full);
+                    if (SENDER)
+                        bulk_g2s(dst + (uint32_t)(RB + j * kApplyTile * 2), x + o, xbytes, full);
+                }
+                ++issued;
+            }
+            if (!ok && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+            // Copies of the last stages issued may still be landing if a
+            // consumer gave up: wait for them (bounded) before this CTA's
+            // shared memory is released.  In a normal run these phases have
+            // completed already and each wait returns at once.
+            for (int st = (issued > S ? issued - S : 0); st < issued; ++st)
+                (void)mbar_wait(bars + 8u * (1 + st % S), (uint32_t)((st / S) & 1));
         }
-        mma_commit(bar);
-    }
-    bool ok = true;
-    if (lane == 0) ok = mbar_wait(bar, 0);
-    ok = __shfl_sync(kFullMask, ok ? 1 : 0, 0) != 0;
-    const bool failed = __syncthreads_or(ok ? 0 : 1) != 0;
-    if (!failed) {
+    } else {
+        // ---------------- operands + MMA ----------------
+        // 16-byte chunks of 4 consecutive k per store
+        for (int idx = tid; idx < kApplyTile * (KP / 4); idx += kApplyConsumers) {
+            const int row = idx / (KP / 4), k0 = (idx - row * (KP / 4)) * 4;
+            const int64_t c = c0 + row, t = t0 + row;
+            float a[4], h[4], l[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int k = k0 + u;
+                a[u] = (c < C && k < r) ? (float)int4_code_at(qc + c * nb, k) : 0.0f;
+                float b = 0.0f;
+                if (t < T && k < r)
+                    b = __fmul_rn((float)int4_code_at(pc + t * nb, k), __fmul_rn(__ldg(ps + k), __ldg(qs + k)));
+                h[u] = __uint_as_float(__float_as_uint(b) & 0xFFFFE000u);
+                l[u] = __fsub_rn(b, h[u]);
+            }
+            const uint32_t off = sw128_f32_offset(row, k0);
+            *reinterpret_cast<float4 *>(gb + off) = make_float4(a[0], a[1], a[2], a[3]);
+            *reinterpret_cast<float4 *>(gb + OPB + off) = make_float4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<float4 *>(gb + 2 * OPB + off) = make_float4(l[0], l[1], l[2], l[3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        fence_before_sync();
+        consumers_sync();
         fence_after_sync();
-        const int q = warp & 3, half = warp >> 2;
-        const int64_t c = c0 + 32 * q + lane;
-        const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
-#pragma unroll 1
-        for (int ch = 0; ch < 8; ++ch) {
-            const int col = 64 * half + 8 * ch;
-            float dv[8];
-            tmem_ld8(trow + col, dv);
-            if (c < C) {
-                const int64_t tb = t0 + col;
-                float *rb = recon + tb * C + c;
-                float rv[8];
-                uint32_t xv[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const bool in = tb + j < T;
-                    const size_t o = (size_t)j * (size_t)C;
-                    rv[j] = in ? __ldcs(rb + o) : 0.0f;
-                    if (SENDER) xv[j] = in ? (uint32_t)__ldcs(x + tb * C + c + o) : 0u;
+        if (tid == 0) {
+            constexpr uint32_t idesc = idesc_tf32(kApplyTile);
+            const int ksteps = (r + 7) / 8;
+            for (int kk = 0; kk < ksteps; ++kk) {
+                const uint32_t off = (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32);
+                const uint64_t da = sw128_desc(sA + off, 16, 1024);
+                mma_tf32(tmem, da, sw128_desc(sBh + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                mma_tf32(tmem, da, sw128_desc(sBl + off, 16, 1024), idesc, 1u);
+            }
+            mma_commit(mma_bar);
+        }
+        const bool ok = __all_sync(kFullMask, mbar_wait(mma_bar, 0));
+        if (!ok && lane == 0) *(volatile int *)abort_flag = 1;
+        consumers_sync();
+        if (*(volatile int *)abort_flag) {
+            if (tid == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+        } else {
+            fence_after_sync();
+            // ---------------- combine ----------------
+            const int q = warp & 3, half = warp >> 2;
+            const int cl = 32 * q + lane;              // channel within the tile
+            const int64_t c = c0 + cl;
+            const bool col_ok = cl < cw;
+            const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
+            for (int st = 0; st < ns; ++st) {
+                const int slot = st % S;
+                const bool got = __all_sync(kFullMask, mbar_wait(bars + 8u * (1 + slot), (uint32_t)((st / S) & 1)));
+                if (!got) {
+                    if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+                    break;
                 }
+                const int tl = st * kApplyStageTok + 8 * half;   // first token column of this warp
+                float dv[8];
+                tmem_ld8(trow + (uint32_t)tl, dv);
+                const float *sr = reinterpret_cast<const float *>(gring + slot * SB) + 8 * half * kApplyTile;
+                const uint16_t *sx = reinterpret_cast<const uint16_t *>(gring + slot * SB + RB) + 8 * half * kApplyTile;
+                if (col_ok) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (tb + j >= T) break;
-                    const size_t o = (size_t)j * (size_t)C;
-                    if (SENDER) {
-                        const float v = __fsub_rn(bf16_bits_to_f32(xv[j]), rv[j]);
-                        __stcs(err + tb * C + c + o, __fsub_rn(v, dv[j]));
+                    for (int j = 0; j < 8; ++j) {
+                        if (tl + j >= tw) break;
+                        const float rv = sr[j * kApplyTile + cl];
+                        const int64_t o = (t0 + tl + j) * C + c;
+                        if (SENDER) {
+                            const float v = __fsub_rn(bf16_bits_to_f32(sx[j * kApplyTile + cl]), rv);
+                            __stcs(err + o, __fsub_rn(v, dv[j]));
+                        }
+                        __stcs(recon + o, __fadd_rn(rv, dv[j]));
                     }
-                    rb[o] = __fadd_rn(rv[j], dv[j]);
                 }
+                // generic reads of the slot before the next async copy into it
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + 8u * (1 + S + slot));
             }
         }
-    } else if (tid == 0 && status) {
-        atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
     }
     fence_before_sync();
     __syncthreads();
@@ -172,11 +292,6 @@ lr_apply_tc_kernel(const uint16_t *x, float *recon, float *err, const uint8_t *p
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128u)
                      : "memory");
     }
-}
-
-template <int KP>
-constexpr int apply_tc_smem() {
-    return 3 * (KP / 32) * 16384 + 1024 + 64;
 }
 
 }  // namespace umma

@@ -16,9 +16,52 @@
 namespace cf {
 
 using bf16 = __nv_bfloat16;
+using cf_lowrank::Layout;
+using cf_lowrank::LrBatch;
+using cf_lowrank::LrPtrs;
+
+// Every kernel of a (batched) low-rank call handles buffer blockIdx.z.  A
+// buffer whose pointers failed validation in lr_prep_kernel is skipped by all.
+__device__ __forceinline__ bool lr_skipped(const LrBatch &B, const Layout &L, int b) {
+    return B.ws != nullptr && B.at<int32_t>(b, L.off_status)[cf_lowrank::kSkipWord] != 0;
+}
+
+// Per-buffer set-up of a low-rank encode: zero the status word, the Gram
+// tickets and the column maxima of this buffer's workspace slice, then check
+// its pointers (x, recon, err: 16-byte aligned; omega, scales: 4-byte; all
+// non-null) and mark the buffer skipped with the error in its status word.
+__global__ void lr_prep_kernel(const LrBatch B, const Layout L) {
+    const int b = blockIdx.x;
+    int32_t *st = B.at<int32_t>(b, L.off_status);
+    uint32_t *gt = B.at<uint32_t>(b, L.off_gt);
+    uint32_t *amax = B.at<uint32_t>(b, L.off_amax);
+    for (int i = threadIdx.x; i < 4; i += blockDim.x) st[i] = 0;
+    for (int i = threadIdx.x; i < L.nGroups; i += blockDim.x) gt[i] = 0u;
+    for (int i = threadIdx.x; i < 2 * L.rp; i += blockDim.x) amax[i] = 0u;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const LrPtrs p = B.get(b);
+        int code = CF_OK;
+        if (!p.x || !p.recon || !p.err || !p.omega || !p.pc_out || !p.ps_out || !p.qc_out || !p.qs_out)
+            code = CF_ERR_INVALID_ARG;
+        else if (misaligned16(p.x) || misaligned16(p.recon) || misaligned16(p.err) ||
+                 (reinterpret_cast<uintptr_t>(p.omega) & 3u) || (reinterpret_cast<uintptr_t>(p.ps_out) & 3u) ||
+                 (reinterpret_cast<uintptr_t>(p.qs_out) & 3u))
+            code = CF_ERR_ALIGNMENT;
+        st[cf_lowrank::kStatusWord] = code;
+        st[cf_lowrank::kSkipWord] = code != CF_OK ? 1 : 0;
+    }
+}
 
 // Vb = bf16_rn((float)x - recon): the residual the projections read.
-__global__ void lr_residual_kernel(const uint16_t *x, const float *recon, bf16 *vb, int64_t n) {
+__global__ void lr_residual_kernel(const LrBatch B, const Layout L) {
+    const int bz = blockIdx.z;
+    if (lr_skipped(B, L, bz)) return;
+    const LrPtrs pp = B.get(bz);
+    const uint16_t *x = pp.x;
+    const float *recon = pp.recon;
+    bf16 *vb = B.at<bf16>(bz, L.off_vb);
+    const int64_t n = L.T * L.C;
     const int64_t groups = n >> 3;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += stride) {
@@ -40,7 +83,13 @@ __global__ void lr_residual_kernel(const uint16_t *x, const float *recon, bf16 *
 }
 
 // Qt[k][c] = bf16(omega[c][k]) for k < r, 0 for the padding rows.
-__global__ void lr_omega_kernel(const float *omega, bf16 *qt, int64_t C, int r, int rp) {
+__global__ void lr_omega_kernel(const LrBatch B, const Layout L) {
+    const int bz = blockIdx.z;
+    if (lr_skipped(B, L, bz)) return;
+    const float *omega = B.get(bz).omega;
+    bf16 *qt = B.at<bf16>(bz, L.off_qt);
+    const int64_t C = L.C;
+    const int r = L.r, rp = L.rp;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (int64_t)rp * C) return;
     const int k = (int)(i / C);
@@ -51,7 +100,14 @@ __global__ void lr_omega_kernel(const float *omega, bf16 *qt, int64_t C, int r, 
 // Yp[s][t][k] = sum over the channels of split s of Vb[t][c] * Qt[k][c].
 // Block: 64 tokens; thread (tok = tid/4, kg = tid%4) owns k = kg + 4j.
 __global__ void __launch_bounds__(256)
-lr_project_simt(const bf16 *vb, const bf16 *qt, float *yp, int64_t T, int64_t C, int rp) {
+lr_project_simt(const LrBatch B, const Layout L) {
+    const int bz = blockIdx.z;
+    if (lr_skipped(B, L, bz)) return;
+    const bf16 *vb = B.at<bf16>(bz, L.off_vb);
+    const bf16 *qt = B.at<bf16>(bz, L.off_qt);
+    float *yp = B.at<float>(bz, L.off_yp);
+    const int64_t T = L.T, C = L.C;
+    const int rp = L.rp;
     __shared__ float Vs[64][65];
     __shared__ float Qs[64][65];
     const int tid = threadIdx.x;
@@ -230,9 +286,20 @@ __device__ __forceinline__ void quad_cholesky(double *A, int ld, int r, const do
 // recorded.  Output: R (fp32 [rp][rp], upper) and 1/diag(R) (fp32 [rp], 0
 // where dead).  All tickets are reset by their last user.
 __global__ void __launch_bounds__(256)
-lr_gram_chol_kernel(const float *yp, float *y, double *gp, double *gg, int64_t T, int r, int rp,
-                    int splits, float *rmat, float *rinvd, uint32_t *gticket, uint32_t *ticket,
-                    int32_t *status) {
+lr_gram_chol_kernel(const LrBatch B, const Layout L) {
+    const int bz = blockIdx.z;
+    if (lr_skipped(B, L, bz)) return;
+    const float *yp = B.at<float>(bz, L.off_yp);
+    float *y = B.at<float>(bz, L.off_y);
+    double *gp = B.at<double>(bz, L.off_gp);
+    double *gg = B.at<double>(bz, L.off_gg);
+    const int64_t T = L.T;
+    const int r = L.r, rp = L.rp, splits = L.splitsA;
+    float *rmat = B.at<float>(bz, L.off_rmat);
+    float *rinvd = rmat + rp * rp;
+    uint32_t *gticket = B.at<uint32_t>(bz, L.off_gt);
+    int32_t *status = B.at<int32_t>(bz, L.off_status) + cf_lowrank::kStatusWord;
+    uint32_t *ticket = B.at<uint32_t>(bz, L.off_status) + cf_lowrank::kTicketWord;
     constexpr int TOK = cf_lowrank::kGramTok;
     // one buffer: the fp32 Y block in phases 1-2, the fp64 matrix afterwards
     __shared__ double buf[64 * 65];
@@ -365,8 +432,16 @@ lr_gram_chol_kernel(const float *yp, float *y, double *gp, double *gg, int64_t T
 // per CTA and column).
 template <int RP>
 __global__ void __launch_bounds__(128)
-lr_orth_kernel(const float *y, const float *rmat, const float *rinvd, float *p, bf16 *pt,
-               int64_t T, int64_t Tp, uint32_t *amax) {
+lr_orth_kernel(const LrBatch B, const Layout L, int want_amax) {
+    const int bz = blockIdx.z;
+    if (lr_skipped(B, L, bz)) return;
+    const float *y = B.at<float>(bz, L.off_y);
+    const float *rmat = B.at<float>(bz, L.off_rmat);
+    const float *rinvd = rmat + RP * RP;
+    float *p = B.at<float>(bz, L.off_p);
+    bf16 *pt = B.at<bf16>(bz, L.off_pt);
+    const int64_t T = L.T, Tp = L.Tp;
+    uint32_t *amax = want_amax ? B.at<uint32_t>(bz, L.off_amax) : nullptr;
     __shared__ float Rs[RP * RP];
     __shared__ float Id[RP];
     __shared__ float Wm[4][RP];
@@ -424,8 +499,14 @@ lr_orth_kernel(const float *y, const float *rmat, const float *rinvd, float *p, 
 
 // Zp[s][c][k] = sum over the tokens of split s of Vb[t][c] * Pt[k][t].
 __global__ void __launch_bounds__(256)
-lr_backproject_simt(const bf16 *vb, const bf16 *pt, float *zp, int64_t T, int64_t Tp, int64_t C,
-                    int rp) {
+lr_backproject_simt(const LrBatch B, const Layout L) {
+    const int bz = blockIdx.z;
+    if (lr_skipped(B, L, bz)) return;
+    const bf16 *vb = B.at<bf16>(bz, L.off_vb);
+    const bf16 *pt = B.at<bf16>(bz, L.off_pt);
+    float *zp = B.at<float>(bz, L.off_zp);
+    const int64_t T = L.T, Tp = L.Tp, C = L.C;
+    const int rp = L.rp;
     __shared__ float Vs[64][65];
     __shared__ float Ps[64][65];
     const int tid = threadIdx.x;
@@ -470,7 +551,15 @@ lr_backproject_simt(const bf16 *vb, const bf16 *pt, float *zp, int64_t T, int64_
 // On the last iteration (amax != null) it folds max |Q[:, k]| into amax[k].
 template <int RP>
 __global__ void __launch_bounds__(128)
-lr_reduce_q_kernel(const float *zp, float *q, bf16 *qt, int64_t C, int splits, uint32_t *amax) {
+lr_reduce_q_kernel(const LrBatch B, const Layout L, int want_amax) {
+    const int bz = blockIdx.z;
+    if (lr_skipped(B, L, bz)) return;
+    const float *zp = B.at<float>(bz, L.off_zp);
+    float *q = B.at<float>(bz, L.off_q);
+    bf16 *qt = B.at<bf16>(bz, L.off_qt);
+    const int64_t C = L.C;
+    const int splits = L.splitsB;
+    uint32_t *amax = want_amax ? B.at<uint32_t>(bz, L.off_amax) + RP : nullptr;
     __shared__ float Wm[4][RP];
     const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     float v[RP];
@@ -536,8 +625,16 @@ __device__ __forceinline__ int int4_code(float v, float s) {
 
 // INT4 per column: s_k = amax_k / 7; codes packed two per byte, the even
 // column in the low nibble; the scales are written by the first r threads.
-__global__ void lr_int4_pack_kernel(const float *f, int64_t rows, int r, int rp,
-                                    const uint32_t *amax, uint8_t *codes, float *scales) {
+__global__ void lr_int4_pack_kernel(const LrBatch B, const Layout L, int which) {
+    const int bz = blockIdx.z;
+    if (lr_skipped(B, L, bz)) return;
+    const LrPtrs pp = B.get(bz);
+    const int r = L.r, rp = L.rp;
+    const float *f = B.at<float>(bz, which == 0 ? L.off_p : L.off_q);
+    const int64_t rows = which == 0 ? L.T : L.C;
+    const uint32_t *amax = B.at<uint32_t>(bz, L.off_amax) + (which == 0 ? 0 : rp);
+    uint8_t *codes = which == 0 ? pp.pc_out : pp.qc_out;
+    float *scales = which == 0 ? pp.ps_out : pp.qs_out;
     const int nb = (r + 1) / 2;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < r) scales[i] = __fdiv_rn(__uint_as_float(amax[i]), 7.0f);
@@ -557,6 +654,20 @@ __device__ __forceinline__ float int4_dequant(const uint8_t *row_codes, int k, c
     return __fmul_rn((float)q, __ldg(scales + k));
 }
 
+// Batched decode: the caller's pointers of buffer b (no workspace to hold a
+// per-buffer status); a bad buffer is skipped and reported once.
+__device__ __forceinline__ bool lr_dec_ptrs_ok(const LrBatch &B, const LrPtrs &p) {
+    int code = CF_OK;
+    if (!p.pc || !p.ps || !p.qc || !p.qs || !p.recon)
+        code = CF_ERR_INVALID_ARG;
+    else if (misaligned16(p.recon) || (reinterpret_cast<uintptr_t>(p.ps) & 3u) ||
+             (reinterpret_cast<uintptr_t>(p.qs) & 3u))
+        code = CF_ERR_ALIGNMENT;
+    if (code != CF_OK && B.dec_status && threadIdx.x == 0)
+        atomicCAS(B.dec_status, (int32_t)CF_OK, (int32_t)code);
+    return code == CF_OK;
+}
+
 // D = (qP sP)(qQ sQ)^T, then
 //   sender:   v = x - recon ; err = v - D ; recon = recon + D
 //   receiver: recon = recon + D
@@ -569,8 +680,17 @@ __device__ __forceinline__ float int4_dequant(const uint8_t *row_codes, int k, c
 // values from the same payload.
 template <bool SENDER>
 __global__ void __launch_bounds__(256, 2)
-lr_apply_kernel(const uint16_t *x, float *recon, float *err, const uint8_t *pc, const float *ps,
-                const uint8_t *qc, const float *qs, int64_t T, int64_t C, int r) {
+lr_apply_kernel(const LrBatch B, const Layout L) {
+    const int bz = blockIdx.z;
+    if (lr_skipped(B, L, bz)) return;
+    const LrPtrs pp = B.get(bz);
+    if (!SENDER && B.dec && !lr_dec_ptrs_ok(B, pp)) return;
+    const uint16_t *x = pp.x;
+    float *recon = pp.recon, *err = pp.err;
+    const uint8_t *pc = pp.pc, *qc = pp.qc;
+    const float *ps = pp.ps, *qs = pp.qs;
+    const int64_t T = L.T, C = L.C;
+    const int r = L.r;
     constexpr int TM = cf_lowrank::kApplyTok, TN = cf_lowrank::kApplyCh;
     extern __shared__ float sm[];
     float *Bs = sm;                   // [r][TN]

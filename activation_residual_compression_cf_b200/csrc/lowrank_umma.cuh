@@ -24,6 +24,7 @@
 #include <stdint.h>
 
 #include "cf.h"
+#include "lowrank_api.cuh"
 
 namespace cf {
 namespace umma {
@@ -71,6 +72,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
         "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// 3-D tile load: coordinates (x, y) inside buffer z of a [buffers][rows][cols]
+// map whose buffer stride is the per-buffer workspace stride.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int32_t x, int32_t y, int32_t z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
         : "memory");
 }
 
@@ -160,8 +172,8 @@ struct StageGeom {
 //   kbeg, nkb  : first K element of this split and number of 64-wide blocks
 template <int BN, bool A_MN>
 __device__ __forceinline__ void gemm_tile(const CUtensorMap *mapA, const CUtensorMap *mapB,
-                                          int32_t rows0, int32_t kbeg, int nkb, float *out,
-                                          int64_t out_rows, int32_t *status) {
+                                          int32_t rows0, int32_t kbeg, int nkb, int32_t zb,
+                                          float *out, int64_t out_rows, int32_t *status) {
     using G = StageGeom<BN>;
     extern __shared__ uint8_t dsmem[];
     const uint32_t base = (smem_u32(dsmem) + 1023u) & ~1023u;
@@ -211,12 +223,12 @@ __device__ __forceinline__ void gemm_tile(const CUtensorMap *mapA, const CUtenso
             mbar_expect_tx(full(s), (uint32_t)G::kBytes);
             const int32_t k = kbeg + kb * kBK;
             if (!A_MN) {
-                tma_load_2d(sa, mapA, full(s), k, rows0);          // box {64 ch, 128 tok}
+                tma_load_3d(sa, mapA, full(s), k, rows0, zb);      // box {64 ch, 128 tok, 1}
             } else {
-                tma_load_2d(sa, mapA, full(s), rows0, k);          // box {64 ch, 64 tok}
-                tma_load_2d(sa + kTileBytesA / 2, mapA, full(s), rows0 + 64, k);
+                tma_load_3d(sa, mapA, full(s), rows0, k, zb);      // box {64 ch, 64 tok, 1}
+                tma_load_3d(sa + kTileBytesA / 2, mapA, full(s), rows0 + 64, k, zb);
             }
-            tma_load_2d(sb, mapB, full(s), k, 0);                  // box {64 k, BN rows}
+            tma_load_3d(sb, mapB, full(s), k, 0, zb);              // box {64 k, BN rows, 1}
         }
     } else if (warp == 1 && lane == 0) {
         // MMA issuer
@@ -280,30 +292,38 @@ __device__ __forceinline__ void gemm_tile(const CUtensorMap *mapA, const CUtenso
     }
 }
 
-// Yp[split][t][0..BN) for the token block blockIdx.x, channel split blockIdx.y.
+// Yp[split][t][0..BN) of buffer blockIdx.z for the token block blockIdx.x and
+// channel split blockIdx.y.
 template <int BN>
 __global__ void __launch_bounds__(128, 1)
 project_kernel(const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapQt,
-               float *yp, int64_t T, int64_t C, int64_t chunk, int32_t *status) {
+               const cf_lowrank::LrBatch B, const cf_lowrank::Layout L) {
+    const int bz = blockIdx.z;
+    if (B.at<int32_t>(bz, L.off_status)[cf_lowrank::kSkipWord]) return;
     const int32_t t0 = blockIdx.x * 128;
-    const int64_t kb = (int64_t)blockIdx.y * chunk;
-    const int64_t ke = (kb + chunk < C) ? kb + chunk : C;
+    const int64_t kb = (int64_t)blockIdx.y * cf_lowrank::kChunkA;
+    const int64_t ke = (kb + cf_lowrank::kChunkA < L.C) ? kb + cf_lowrank::kChunkA : L.C;
     const int nkb = (int)((ke - kb + kBK - 1) / kBK);
-    gemm_tile<BN, false>(&mapV, &mapQt, t0, (int32_t)kb, nkb, yp + (int64_t)blockIdx.y * T * BN, T,
-                         status);
+    float *yp = B.at<float>(bz, L.off_yp) + (int64_t)blockIdx.y * L.T * BN;
+    gemm_tile<BN, false>(&mapV, &mapQt, t0, (int32_t)kb, nkb, bz, yp, L.T,
+                         B.at<int32_t>(bz, L.off_status) + cf_lowrank::kStatusWord);
 }
 
-// Zp[split][c][0..BN) for the channel block blockIdx.x, token split blockIdx.y.
+// Zp[split][c][0..BN) of buffer blockIdx.z for the channel block blockIdx.x
+// and token split blockIdx.y.
 template <int BN>
 __global__ void __launch_bounds__(128, 1)
 backproject_kernel(const __grid_constant__ CUtensorMap mapVt, const __grid_constant__ CUtensorMap mapPt,
-                   float *zp, int64_t T, int64_t C, int64_t chunk, int32_t *status) {
+                   const cf_lowrank::LrBatch B, const cf_lowrank::Layout L) {
+    const int bz = blockIdx.z;
+    if (B.at<int32_t>(bz, L.off_status)[cf_lowrank::kSkipWord]) return;
     const int32_t c0 = blockIdx.x * 128;
-    const int64_t kb = (int64_t)blockIdx.y * chunk;
-    const int64_t ke = (kb + chunk < T) ? kb + chunk : T;
+    const int64_t kb = (int64_t)blockIdx.y * cf_lowrank::kChunkB;
+    const int64_t ke = (kb + cf_lowrank::kChunkB < L.T) ? kb + cf_lowrank::kChunkB : L.T;
     const int nkb = (int)((ke - kb + kBK - 1) / kBK);
-    gemm_tile<BN, true>(&mapVt, &mapPt, c0, (int32_t)kb, nkb, zp + (int64_t)blockIdx.y * C * BN, C,
-                        status);
+    float *zp = B.at<float>(bz, L.off_zp) + (int64_t)blockIdx.y * L.C * BN;
+    gemm_tile<BN, true>(&mapVt, &mapPt, c0, (int32_t)kb, nkb, bz, zp, L.C,
+                        B.at<int32_t>(bz, L.off_status) + cf_lowrank::kStatusWord);
 }
 
 }  // namespace umma

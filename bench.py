@@ -161,7 +161,7 @@ class ClockSampler:
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "activation_residual_compression_cf_b200", "csrc")
-    for fn in ("quant_tma.cuh", "quant_kernels.cuh", "cf_common.cuh"):
+    for fn in ("quant_tma.cuh", "quant_kernels.cuh", "cf_common.cuh", "cf_api.cu"):
         h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
 
@@ -199,6 +199,49 @@ def oracle_sample(wl, seconds, max_buffer_steps=10**9):
         i += 1
     gbs = 2 * wl.elems * done / t_work / 1e9
     return gbs, done, t_work
+
+
+def blas_threads():
+    """Threads the host BLAS that numpy calls into actually uses."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+class LowrankOracleStepper:
+    """The oracle's low-rank sender + receiver on host copies of buffer 0's
+    trajectory (cycled), one buffer-step per call."""
+
+    def __init__(self, wl):
+        from oracle import lowrank as OL
+        self.OL, self.wl = OL, wl
+        xs = W.trajectory(wl, 0, steps=min(wl.steps, 4), device="cpu")
+        self.xb = [W.bf16_bits(x) for x in xs]
+        self.om = [W.omega(wl, 0, s, device="cpu").numpy() for s in range(len(xs))]
+        self.recon_s = OL.bf16_bits_to_f32(self.xb[0]).copy()
+        self.recon_r = self.recon_s.copy()
+        self.i = 0
+
+    def __call__(self):
+        k = 1 + self.i % (len(self.xb) - 1)
+        o = self.OL.lowrank_encode(self.xb[k], self.recon_s, self.om[k], self.wl.iters)
+        self.OL.lowrank_decode(o["p_codes"], o["p_scales"], o["q_codes"], o["q_scales"],
+                               self.recon_r, self.wl.rank)
+        self.i += 1
+
+
+def lowrank_oracle_sample(wl, seconds):
+    step = LowrankOracleStepper(wl)
+    done, t_work = 0, 0.0
+    while t_work < seconds:
+        t0 = time.perf_counter()
+        step()
+        t_work += time.perf_counter() - t0
+        done += 1
+    return 2 * wl.elems * done / t_work / 1e9, done, t_work
 
 
 # ------------------------------------------------------------ GPU leg
@@ -407,6 +450,26 @@ def run_lowrank(args, world, rank, local):
     enc_bytes = n * T * C * 14
     dec_bytes = n * T * C * 8
     status = max(cf.cf_lowrank_status(ws[b * wsb:]) for b in range(n))
+    # Launches per step: the sender runs prep, residual, omega, five kernels
+    # per subspace iteration (project, Gram+Cholesky, orthogonalise,
+    # back-project, reduce), two INT4 packs and the apply; the receiver one.
+    launches_per_step = 6 + 5 * it + 1
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_lowrank_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, OM, pc, ps,
+                              qc, qs, ws)
+        e2e["ms"] = R.reduce_scalar(e2e["ms"], "max")
+        e2e = {"value": round(2 * T * C * n * args.steps * world / (e2e["ms"] / 1e3) / 1e9, 3),
+               "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
+               "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(e2e["ms"] / args.steps, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, done, tw = lowrank_oracle_sample(wl, args.cpu_seconds)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{done} buffer-steps of {args.workload} buffer 0 ({T}x{C}, rank {r}, "
+                         f"{it} iterations, encode+decode), {tw:.1f} s of numpy fp64"}
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
@@ -415,7 +478,7 @@ def run_lowrank(args, world, rank, local):
         "config": {"workload": args.workload, "tokens": T, "channels": C, "buffers": n,
                    "rank": r, "iters": it, "mode": "low-rank INT4 + EF",
                    "parallelism": f"replicas x{world}", "l2": "inputs larger than L2",
-                   "launches_per_step": None},
+                   "launches_per_step": launches_per_step},
         "roofline": {"bound": "hbm", "achieved": round(enc_bytes / (enc_ms / 1e3) / 1e9, 1),
                      "peak": peak, "unit": "GB/s",
                      "frac": round(enc_bytes / (enc_ms / 1e3) / 1e9 / peak, 4), "traffic": None,
@@ -426,9 +489,54 @@ def run_lowrank(args, world, rank, local):
                    "avg_ms_per_step": round(dec_ms, 4)},
         "encode_ms_per_step": round(enc_ms, 4), "lowrank_status": status,
         "payload_ratio": round(2 * T * C / cf.cf_payload_bytes(d), 2),
-        "cpu_baseline": None, "e2e": None, "gpu_launches": None, "clocks": clocks,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
     }
     return out
+
+
+def run_lowrank_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, OM, pc, ps, qc, qs, ws):
+    """Low-rank end to end: every step copies the pinned host activations of
+    all buffers in, runs the batched sender and receiver, and reads the INT4
+    payload (factor codes and scales) back to the host."""
+    n, T, C = wl.buffers, wl.tokens, wl.channels
+    tr = W.Trajectory(wl, 0, device=dev)
+    tr.next()
+    x_host = []
+    for _ in range(2):
+        xk = tr.next().unsqueeze(0).expand(n, T, C).contiguous().cpu()
+        x_host.append(xk.pin_memory())
+        del xk
+    x_dev = torch.empty((n, T, C), dtype=torch.bfloat16, device=dev)
+    x16 = x_dev.view(torch.int16)
+    wsb = cf.cf_lowrank_workspace_bytes(d)
+    enc = cf.lowrank_buffer_array([(x16[b], recon_s[b], err[b], OM[1, b], pc[b], ps[b], qc[b],
+                                    qs[b]) for b in range(n)], dev)
+    dec = cf.lowrank_dec_buffer_array([(pc[b], ps[b], qc[b], qs[b], recon_r[b])
+                                       for b in range(n)], dev)
+    outs = [pc, ps, qc, qs]
+    host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+
+    def step(i):
+        x_dev.copy_(x_host[i % 2], non_blocking=True)
+        cf.cf_lowrank_encode_batched(d, n, enc, ws, stream=stream)
+        cf.cf_lowrank_decode_batched(d, n, dec, stream=stream)
+        for h, t in zip(host, outs):
+            h.copy_(t, non_blocking=True)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(args.steps):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    st = max(cf.cf_lowrank_status(ws[k * wsb:]) for k in range(n))
+    assert st in (0, 6), cf.cf_status_string(st)
+    return {"ms": a.elapsed_time(b), "h2d": n * T * C * 2,
+            "d2h": sum(t.numel() * t.element_size() for t in outs)}
 
 
 def run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, status):
@@ -477,17 +585,25 @@ def run_reference(args, world, rank):
         return None
     wl = W.WORKLOADS[args.workload]
     per_step = 1
-    import oracle
-    xs = W.trajectory(wl, 0, steps=min(wl.steps, 4), device="cpu")
-    xb = [W.bf16_bits(x) for x in xs]
-    recon_s, _ = oracle.state_init(xb[0])
-    recon_r = recon_s.copy()
+    cores, kind = 1, "single-threaded C oracle"
+    if wl.mode == "lowrank":
+        lr_step = LowrankOracleStepper(wl)
+        cores, kind = blas_threads(), "numpy fp64 oracle"
 
-    def one(i):
-        for _ in range(per_step):
-            x = xb[1 + i % (len(xb) - 1)]
-            c, s, _ = oracle.encode(x, recon_s, wl.bits)
-            oracle.decode(c, s, recon_r, wl.bits)
+        def one(i):
+            lr_step()
+    else:
+        import oracle
+        xs = W.trajectory(wl, 0, steps=min(wl.steps, 4), device="cpu")
+        xb = [W.bf16_bits(x) for x in xs]
+        recon_s, _ = oracle.state_init(xb[0])
+        recon_r = recon_s.copy()
+
+        def one(i):
+            for _ in range(per_step):
+                x = xb[1 + i % (len(xb) - 1)]
+                c, s, _ = oracle.encode(x, recon_s, wl.bits)
+                oracle.decode(c, s, recon_r, wl.bits)
 
     for i in range(args.warmup):
         one(i)
@@ -502,12 +618,13 @@ def run_reference(args, world, rank):
         "ms_per_step": round(sec * 1e3 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 state",
         "data": "synthetic",
-        "config": {"workload": args.workload, "tokens": wl.tokens, "channels": wl.channels,
-                   "buffers": wl.buffers, "bits": wl.bits,
-                   "sample": f"each step = {per_step} of the {wl.buffers} buffers"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{per_step} buffer(s) per step, {args.steps} steps, "
-                                   "single-threaded C oracle"},
+        "config": dict({"workload": args.workload, "tokens": wl.tokens, "channels": wl.channels,
+                        "buffers": wl.buffers},
+                       **({"rank": wl.rank, "iters": wl.iters} if wl.mode == "lowrank"
+                          else {"bits": wl.bits}),
+                       sample=f"each step = {per_step} of the {wl.buffers} buffers"),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{per_step} buffer(s) per step, {args.steps} steps, {kind}"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -187,7 +187,9 @@ int64_t cf_lowrank_workspace_bytes(const cf_desc *d);
 /* Bytes of one packed INT4 factor with `rows` rows at rank `rank`. */
 int64_t cf_lowrank_factor_bytes(int64_t rows, int32_t rank);
 
-/* Sender, low-rank mode.  x: bf16 [T][C]; recon_s: fp32 [T][C] updated;
+/* Sender, low-rank mode.  Alignment: x, recon_s, err 16 bytes; omega and the
+ * scales 4 bytes; the code arrays 1 byte.
+ * x: bf16 [T][C]; recon_s: fp32 [T][C] updated;
  * err: fp32 [T][C] written; omega: fp32 [C][r] Gaussian start block chosen
  * by the caller; p_codes: [T][ceil(r/2)] bytes, p_scales: fp32 [r];
  * q_codes: [C][ceil(r/2)] bytes, q_scales: fp32 [r] (all written);
@@ -202,6 +204,51 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
                             float *p_scales, uint8_t *q_codes, float *q_scales,
                             void *workspace, size_t workspace_bytes,
                             void *stream);
+
+/* One buffer of a batched low-rank encode (device pointers; rules as for
+ * cf_lowrank_encode). */
+typedef struct cf_lowrank_buffer {
+    const uint16_t *x;       /* bf16 [T][C]                                  */
+    float *recon_s;          /* fp32 [T][C], updated                         */
+    float *err;              /* fp32 [T][C], written                         */
+    const float *omega;      /* fp32 [C][r], subspace-iteration start        */
+    uint8_t *p_codes;        /* [T][ceil(r/2)], written                      */
+    float *p_scales;         /* fp32 [r], written                            */
+    uint8_t *q_codes;        /* [C][ceil(r/2)], written                      */
+    float *q_scales;         /* fp32 [r], written                            */
+} cf_lowrank_buffer;
+
+/* One buffer of a batched low-rank decode. */
+typedef struct cf_lowrank_dec_buffer {
+    const uint8_t *p_codes;
+    const float *p_scales;
+    const uint8_t *q_codes;
+    const float *q_scales;
+    float *recon_r;          /* fp32 [T][C], updated                         */
+} cf_lowrank_dec_buffer;
+
+/* Batched low-rank sender: `n` buffers of the same shape, every stage of the
+ * method launched once for all of them (the latency-bound small steps of
+ * different buffers then overlap).  bufs_dev: DEVICE array of n
+ * cf_lowrank_buffer, valid until the work completes.  workspace: device,
+ * 256-byte aligned, >= n * cf_lowrank_workspace_bytes(d) bytes; buffer b
+ * uses the slice at b * cf_lowrank_workspace_bytes(d), and its status word
+ * is read with cf_lowrank_status(workspace + that offset, stream).  Pointers
+ * inside bufs_dev are checked on the device: a buffer with a null pointer or
+ * a misaligned x/recon_s/err (16 B) or omega/scales (4 B) is skipped and
+ * its status word gets CF_ERR_INVALID_ARG / CF_ERR_ALIGNMENT. */
+cf_status cf_lowrank_encode_batched(const cf_desc *d, int32_t n,
+                                    const cf_lowrank_buffer *bufs_dev, void *workspace,
+                                    size_t workspace_bytes, void *stream);
+
+/* Batched low-rank receiver: recon_r += D for `n` buffers in one launch.
+ * bufs_dev: DEVICE array of n cf_lowrank_dec_buffer.  A buffer with a null
+ * pointer or misaligned recon_r (16 B) / scales (4 B) is skipped and, when
+ * status_dev (device int32, zeroed by the caller) is given, the first such
+ * error is stored there. */
+cf_status cf_lowrank_decode_batched(const cf_desc *d, int32_t n,
+                                    const cf_lowrank_dec_buffer *bufs_dev,
+                                    int32_t *status_dev, void *stream);
 
 /* Receiver, low-rank mode: recon_r += D, with D formed from the payload by
  * the same device routine the sender uses (so recon_r == recon_s bit for

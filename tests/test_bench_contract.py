@@ -32,3 +32,11 @@ def test_reference_arm_json_line():
 
 def test_reference_arm_other_ranks_print_nothing():
     assert _run({"RANK": "1", "WORLD_SIZE": "2"}, args=("--workload", "tiny")) == []
+
+
+def test_reference_arm_lowrank_line():
+    lines = _run(args=("--workload", "lowrank"))
+    d = json.loads(lines[-1])
+    assert d["impl"] == "reference" and d["value"] > 0
+    assert d["config"]["rank"] == 32 and d["config"]["iters"] == 2 and "bits" not in d["config"]
+    assert d["cpu_baseline"]["cores"] >= 1

@@ -205,3 +205,51 @@ def test_workspace_too_small_is_rejected():
         cf.cf_lowrank_encode(g.d, x.view(torch.int16), g.recon_s, g.err, om, g.pc, g.ps, g.qc,
                              g.qs, small)
     assert ei.value.status == 4
+
+
+@pytest.mark.parametrize("T,C,r,n", [(4096, 3072, 32, 4), (300, 136, 16, 3), (77, 64, 33, 2)])
+def test_batched_lowrank_equals_single_calls(T, C, r, n):
+    """One batched call over n buffers computes exactly what n single calls do
+    (same kernels, fixed reduction orders), for the sender and the receiver;
+    a buffer with a misaligned pointer is skipped and reported in its own
+    workspace status word."""
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r)
+    d = cf.desc(T, C, 0, r, 2)
+    wsb = cf.cf_lowrank_workspace_bytes(d)
+    xs = [W.trajectory(wl, b, steps=2, device="cuda") for b in range(n)]
+    oms = [W.omega(wl, b, 1, device="cuda") for b in range(n)]
+    single = [GpuLowrank(T, C, r, 2) for _ in range(n)]
+    batch = [GpuLowrank(T, C, r, 2) for _ in range(n)]
+    for b in range(n):
+        for g in (single[b], batch[b]):
+            g.init(xs[b][0].clone())
+    for b in range(n):
+        single[b].step(xs[b][1].clone(), oms[b])
+    xb = [xs[b][1].clone() for b in range(n)]
+    ws = torch.empty(n * wsb, dtype=torch.uint8, device="cuda")
+    enc = cf.lowrank_buffer_array([(xb[b].view(torch.int16), batch[b].recon_s, batch[b].err, oms[b],
+                                    batch[b].pc, batch[b].ps, batch[b].qc, batch[b].qs)
+                                   for b in range(n)], "cuda")
+    dec = cf.lowrank_dec_buffer_array([(batch[b].pc, batch[b].ps, batch[b].qc, batch[b].qs,
+                                        batch[b].recon_r) for b in range(n)], "cuda")
+    cf.cf_lowrank_encode_batched(d, n, enc, ws)
+    cf.cf_lowrank_decode_batched(d, n, dec)
+    torch.cuda.synchronize()
+    nb = (r + 1) // 2
+    for b in range(n):
+        assert cf.cf_lowrank_status(ws[b * wsb:]) == 0
+        for k in ("recon_s", "recon_r", "err", "ps", "qs"):
+            assert torch.equal(getattr(batch[b], k), getattr(single[b], k)), (b, k)
+        # the code arrays carry 16 spare bytes past the payload; compare the payload
+        assert torch.equal(batch[b].pc[:T * nb], single[b].pc[:T * nb]), b
+        assert torch.equal(batch[b].qc[:C * nb], single[b].qc[:C * nb]), b
+    # a misaligned recon pointer: that buffer is skipped, the others run
+    bad = GpuLowrank(T, C, r, 2)
+    bad.init(xs[0][0].clone())
+    before = bad.recon_s.clone()
+    rows = [(xb[0].view(torch.int16), bad.recon_s.data_ptr() + 4, bad.err, oms[0], bad.pc, bad.ps,
+             bad.qc, bad.qs)]
+    cf.cf_lowrank_encode_batched(d, 1, cf.lowrank_buffer_array(rows, "cuda"), ws)
+    torch.cuda.synchronize()
+    assert cf.cf_lowrank_status(ws) == 2
+    assert torch.equal(bad.recon_s, before)
