@@ -62,14 +62,14 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v) {
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Staging of x and recon: the tile's 128 tokens are 8 stages of 16 token
-// rows; a stage holds the rows' recon (16 x 128 fp32) and, for the sender,
-// x (16 x 128 bf16).  Ring depth per kernel, sized so that the sender with
+// Staging of x and recon: a tile's 128 tokens are 8 stages of 16 token rows;
+// a stage holds the rows' recon (16 x 128 fp32) and, for the sender, x
+// (16 x 128 bf16).  Ring depth per kernel, sized so that the sender with
 // rank <= 32 keeps two CTAs per SM.
 constexpr int kApplyStageTok = 16;
-constexpr int kApplyStagesPerTile = kApplyTile / kApplyStageTok;
 constexpr int kApplyConsumers = 256;            // 8 warps: 4 channel quarters x 2 token halves
 constexpr int kApplyThreads = kApplyConsumers + 32;  // + one producer warp
+constexpr int kApplyMaxTilesPerCta = 8;
 
 template <bool SENDER>
 __host__ __device__ constexpr int apply_stage_bytes() {
@@ -97,22 +97,53 @@ __device__ __forceinline__ void consumers_sync() {
     asm volatile("bar.sync 1, %0;" ::"r"(kApplyConsumers) : "memory");
 }
 
-// Warp roles (288 threads):
-//   warps 0-7 : build the MMA operands, thread 0 issues the MMAs; then each
+// B operand of one token tile: b[t][k] = qP[t][k] * (sP[k] sQ[k]) split into
+// the tf32-exact hi part and the remainder; 16-byte chunks of 4 consecutive k.
+template <int KP>
+__device__ __forceinline__ void apply_build_b(uint8_t *gbh, uint8_t *gbl, const uint8_t *pc,
+                                              const float *ps, const float *qs, int64_t t0,
+                                              int64_t T, int r, int nb, int tid) {
+    for (int idx = tid; idx < kApplyTile * (KP / 4); idx += kApplyConsumers) {
+        const int row = idx / (KP / 4), k0 = (idx - row * (KP / 4)) * 4;
+        const int64_t t = t0 + row;
+        float h[4], l[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int k = k0 + u;
+            float b = 0.0f;
+            if (t < T && k < r)
+                b = __fmul_rn((float)int4_code_at(pc + t * nb, k), __fmul_rn(__ldg(ps + k), __ldg(qs + k)));
+            h[u] = __uint_as_float(__float_as_uint(b) & 0xFFFFE000u);
+            l[u] = __fsub_rn(b, h[u]);
+        }
+        const uint32_t off = sw128_f32_offset(row, k0);
+        *reinterpret_cast<float4 *>(gbh + off) = make_float4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<float4 *>(gbl + off) = make_float4(l[0], l[1], l[2], l[3]);
+    }
+}
+
+// Persistent over a run of token tiles: CTA (x, y, z) owns channel block x of
+// buffer z and token tiles [y * tpc, (y + 1) * tpc).  Warp roles (288
+// threads):
+//   warps 0-7 : build the A operand (Q codes of the channel block) once and
+//               the B operand of each token tile; thread 0 issues the MMAs
+//               into one of two TMEM accumulators (128 columns each), so the
+//               next tile's product runs while this tile is combined; each
 //               warp combines one channel quarter (w % 4, its TMEM lanes) x
 //               one half (w / 4) of every 16-token stage, reading x and recon
-//               from shared memory and D from TMEM, and writes err and recon
-//               to global memory;
+//               from shared memory and D from TMEM, and writes err and recon;
 //   warp 8    : one lane issues 1-D bulk copies (cp.async.bulk, no multicast)
-//               of every token row's 128-channel segment of recon (and x)
-//               into the ring, from the kernel's first instructions on, so the
-//               HBM reads overlap the operand build and the MMA.
+//               of every token row's 128-channel segment of recon (and x) of
+//               all the CTA's tiles into the ring, from the kernel's first
+//               instructions on.
+// The B operand is single-buffered: tile i+1's is written after tile i's MMA
+// has completed (its commit barrier), before tile i is combined.
 // Every wait is bounded; on expiry CF_ERR_TIMEOUT goes to the buffer's status
-// word, the warps stop, the producer waits (bounded) for its copies still in
-// flight, and TMEM is freed.
+// word, the consumer warps leave together at the next tile boundary, the
+// producer waits (bounded) for its copies still in flight, and TMEM is freed.
 template <bool SENDER, int KP>
 __global__ void __launch_bounds__(kApplyThreads, (KP <= 32 ? 2 : 1))
-lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L) {
+lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int tpc) {
     const int bz = blockIdx.z;
     if (lr_skipped(B, L, bz)) return;
     const cf_lowrank::LrPtrs pp = B.get(bz);
@@ -136,24 +167,28 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L) {
     const uint32_t sA = base, sBh = base + OPB, sBl = base + 2 * OPB;
     const uint32_t ring = base + 3 * OPB;
     uint8_t *gring = gb + 3 * OPB;
-    const uint32_t bars = ring + S * SB;       // mma, full[S], empty[S]
-    const uint32_t mma_bar = bars;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(gring + S * SB + 8 * (1 + 2 * S));
+    const uint32_t bars = ring + S * SB;       // mma[2], full[S], empty[S]
+    const uint32_t full0 = bars + 16u, empty0 = bars + 16u + 8u * S;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(gring + S * SB + 8 * (2 + 2 * S));
     int *abort_flag = reinterpret_cast<int *>(tslot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t c0 = (int64_t)blockIdx.x * kApplyTile;
-    const int64_t t0 = (int64_t)blockIdx.y * kApplyTile;
+    const int64_t ntt = (T + kApplyTile - 1) / kApplyTile;
+    const int64_t ty0 = (int64_t)blockIdx.y * tpc;
+    if (ty0 >= ntt) return;
+    const int nt = (int)((ntt - ty0 < tpc) ? ntt - ty0 : tpc);        // tiles of this CTA
+    const int64_t tbeg = ty0 * kApplyTile;
+    const int64_t tend = (tbeg + (int64_t)nt * kApplyTile < T) ? tbeg + (int64_t)nt * kApplyTile : T;
     const int nb = (r + 1) / 2;
-    const int64_t cw = (C - c0 < kApplyTile) ? C - c0 : kApplyTile;   // channels in this tile
-    const int64_t tw = (T - t0 < kApplyTile) ? T - t0 : kApplyTile;   // tokens in this tile
-    const int ns = (int)((tw + kApplyStageTok - 1) / kApplyStageTok);  // stages in this tile
+    const int64_t cw = (C - c0 < kApplyTile) ? C - c0 : kApplyTile;   // channels in the block
 
     if (tid == 0) {
-        mbar_init(mma_bar, 1);
+        mbar_init(bars, 1);
+        mbar_init(bars + 8u, 1);
         for (int s = 0; s < S; ++s) {
-            mbar_init(bars + 8u * (1 + s), 1);                  // full: producer + tx bytes
-            mbar_init(bars + 8u * (1 + S + s), kApplyConsumers / 32);  // empty: one per warp
+            mbar_init(full0 + 8u * s, 1);                        // producer + tx bytes
+            mbar_init(empty0 + 8u * s, kApplyConsumers / 32);    // one per consumer warp
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -161,7 +196,7 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L) {
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tslot)),
-                     "r"(128u)
+                     "r"(256u)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -171,29 +206,31 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L) {
     const uint32_t tmem = *tslot;
 
     if (warp == kApplyConsumers / 32) {
-        // ---------------- producer ----------------
+        // ---------------- producer: stages of 16 rows over [tbeg, tend) ----------------
         if (lane == 0) {
             const uint32_t rbytes = (uint32_t)cw * 4u, xbytes = (uint32_t)cw * 2u;
             int issued = 0;
             bool ok = true;
-            for (int st = 0; st < ns; ++st) {
-                const int slot = st % S;
-                if (st >= S && !mbar_wait(bars + 8u * (1 + S + slot), (uint32_t)((st / S - 1) & 1))) {
-                    ok = false;
-                    break;
+            for (int it = 0; it < nt && ok; ++it) {
+                const int64_t t0 = tbeg + (int64_t)it * kApplyTile;
+                for (int64_t tb = t0; tb < t0 + kApplyTile && tb < tend; tb += kApplyStageTok) {
+                    const int slot = issued % S;
+                    if (issued >= S && !mbar_wait(empty0 + 8u * slot, (uint32_t)((issued / S - 1) & 1))) {
+                        ok = false;
+                        break;
+                    }
+                    const int rows = (int)((tend - tb < kApplyStageTok) ? tend - tb : kApplyStageTok);
+                    const uint32_t full = full0 + 8u * slot;
+                    const uint32_t dst = ring + (uint32_t)(slot * SB);
+                    mbar_expect_tx(full, (uint32_t)rows * (rbytes + (SENDER ? xbytes : 0u)));
+                    for (int j = 0; j < rows; ++j) {
+                        const int64_t o = (tb + j) * C + c0;
+                        bulk_g2s(dst + (uint32_t)(j * kApplyTile * 4), recon + o, rbytes, full);
+                        if (SENDER)
+                            bulk_g2s(dst + (uint32_t)(RB + j * kApplyTile * 2), x + o, xbytes, full);
+                    }
+                    ++issued;
                 }
-                const int64_t tb = t0 + (int64_t)st * kApplyStageTok;
-                const int rows = (int)((T - tb < kApplyStageTok) ? T - tb : kApplyStageTok);
-                const uint32_t full = bars + 8u * (1 + slot);
-                const uint32_t dst = ring + (uint32_t)(slot * SB);
-                mbar_expect_tx(full, (uint32_t)rows * (rbytes + (SENDER ? xbytes : 0u)));
-                for (int j = 0; j < rows; ++j) {
-                    const int64_t o = (tb + j) * C + c0;
-                    bulk_g2s(dst + (uint32_t)(j * kApplyTile * 4), recon + o, rbytes, full);
-                    if (SENDER)
-                        bulk_g2s(dst + (uint32_t)(RB + j * kApplyTile * 2), x + o, xbytes, full);
-                }
-                ++issued;
             }
             if (!ok && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
             // Copies of the last stages issued may still be landing if a
@@ -201,68 +238,78 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L) {
             // shared memory is released.  In a normal run these phases have
             // completed already and each wait returns at once.
             for (int st = (issued > S ? issued - S : 0); st < issued; ++st)
-                (void)mbar_wait(bars + 8u * (1 + st % S), (uint32_t)((st / S) & 1));
+                (void)mbar_wait(full0 + 8u * (st % S), (uint32_t)((st / S) & 1));
         }
     } else {
-        // ---------------- operands + MMA ----------------
-        // 16-byte chunks of 4 consecutive k per store
+        // ---------------- operands, MMAs, combine ----------------
+        // A = the INT4 codes of Q for this channel block, once.
         for (int idx = tid; idx < kApplyTile * (KP / 4); idx += kApplyConsumers) {
             const int row = idx / (KP / 4), k0 = (idx - row * (KP / 4)) * 4;
-            const int64_t c = c0 + row, t = t0 + row;
-            float a[4], h[4], l[4];
+            const int64_t c = c0 + row;
+            float a[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int k = k0 + u;
                 a[u] = (c < C && k < r) ? (float)int4_code_at(qc + c * nb, k) : 0.0f;
-                float b = 0.0f;
-                if (t < T && k < r)
-                    b = __fmul_rn((float)int4_code_at(pc + t * nb, k), __fmul_rn(__ldg(ps + k), __ldg(qs + k)));
-                h[u] = __uint_as_float(__float_as_uint(b) & 0xFFFFE000u);
-                l[u] = __fsub_rn(b, h[u]);
             }
-            const uint32_t off = sw128_f32_offset(row, k0);
-            *reinterpret_cast<float4 *>(gb + off) = make_float4(a[0], a[1], a[2], a[3]);
-            *reinterpret_cast<float4 *>(gb + OPB + off) = make_float4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<float4 *>(gb + 2 * OPB + off) = make_float4(l[0], l[1], l[2], l[3]);
+            *reinterpret_cast<float4 *>(gb + sw128_f32_offset(row, k0)) = make_float4(a[0], a[1], a[2], a[3]);
         }
+        apply_build_b<KP>(gb + OPB, gb + 2 * OPB, pc, ps, qs, tbeg, T, r, nb, tid);
+        const int ksteps = (r + 7) / 8;
+        constexpr uint32_t idesc = idesc_tf32(kApplyTile);
+        auto issue_mma = [&](int i) {
+            const uint32_t acc = tmem + (uint32_t)(128 * (i & 1));
+            for (int kk = 0; kk < ksteps; ++kk) {
+                const uint32_t off = (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32);
+                const uint64_t da = sw128_desc(sA + off, 16, 1024);
+                mma_tf32(acc, da, sw128_desc(sBh + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                mma_tf32(acc, da, sw128_desc(sBl + off, 16, 1024), idesc, 1u);
+            }
+            mma_commit(bars + 8u * (i & 1));
+        };
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         fence_before_sync();
         consumers_sync();
         fence_after_sync();
-        if (tid == 0) {
-            constexpr uint32_t idesc = idesc_tf32(kApplyTile);
-            const int ksteps = (r + 7) / 8;
-            for (int kk = 0; kk < ksteps; ++kk) {
-                const uint32_t off = (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32);
-                const uint64_t da = sw128_desc(sA + off, 16, 1024);
-                mma_tf32(tmem, da, sw128_desc(sBh + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
-                mma_tf32(tmem, da, sw128_desc(sBl + off, 16, 1024), idesc, 1u);
-            }
-            mma_commit(mma_bar);
-        }
-        const bool ok = __all_sync(kFullMask, mbar_wait(mma_bar, 0));
-        if (!ok && lane == 0) *(volatile int *)abort_flag = 1;
-        consumers_sync();
-        if (*(volatile int *)abort_flag) {
-            if (tid == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
-        } else {
+        if (tid == 0) issue_mma(0);
+
+        const int q = warp & 3, half = warp >> 2;
+        const int cl = 32 * q + lane;              // channel within the block
+        const int64_t c = c0 + cl;
+        const bool col_ok = cl < cw;
+        const uint32_t tlane = (uint32_t)(32 * q) << 16;
+        int g = 0;                                 // stages consumed so far
+        for (int i = 0; i < nt; ++i) {
+            // tile i's product is done: its accumulator may be read and the
+            // B operand rewritten
+            if (!__all_sync(kFullMask, mbar_wait(bars + 8u * (i & 1), (uint32_t)((i >> 1) & 1))))
+                if (lane == 0) *(volatile int *)abort_flag = 1;
             fence_after_sync();
-            // ---------------- combine ----------------
-            const int q = warp & 3, half = warp >> 2;
-            const int cl = 32 * q + lane;              // channel within the tile
-            const int64_t c = c0 + cl;
-            const bool col_ok = cl < cw;
-            const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
-            for (int st = 0; st < ns; ++st) {
-                const int slot = st % S;
-                const bool got = __all_sync(kFullMask, mbar_wait(bars + 8u * (1 + slot), (uint32_t)((st / S) & 1)));
-                if (!got) {
-                    if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+            const int64_t t0 = tbeg + (int64_t)i * kApplyTile;
+            if (i + 1 < nt)
+                apply_build_b<KP>(gb + OPB, gb + 2 * OPB, pc, ps, qs, t0 + kApplyTile, T, r, nb, tid);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            fence_before_sync();
+            consumers_sync();
+            fence_after_sync();
+            if (*(volatile int *)abort_flag) {
+                if (tid == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+                break;  // every consumer warp reads the same flag after the barrier
+            }
+            if (tid == 0 && i + 1 < nt) issue_mma(i + 1);
+
+            const uint32_t acc = tmem + tlane + (uint32_t)(128 * (i & 1));
+            const int64_t tw = (T - t0 < kApplyTile) ? T - t0 : kApplyTile;
+            const int ns = (int)((tw + kApplyStageTok - 1) / kApplyStageTok);
+            for (int st = 0; st < ns; ++st, ++g) {
+                const int slot = g % S;
+                if (!__all_sync(kFullMask, mbar_wait(full0 + 8u * slot, (uint32_t)((g / S) & 1)))) {
+                    if (lane == 0) *(volatile int *)abort_flag = 1;
                     break;
                 }
                 const int tl = st * kApplyStageTok + 8 * half;   // first token column of this warp
                 float dv[8];
-                tmem_ld8(trow + (uint32_t)tl, dv);
+                tmem_ld8(acc + (uint32_t)tl, dv);
                 const float *sr = reinterpret_cast<const float *>(gring + slot * SB) + 8 * half * kApplyTile;
                 const uint16_t *sx = reinterpret_cast<const uint16_t *>(gring + slot * SB + RB) + 8 * half * kApplyTile;
                 if (col_ok) {
@@ -281,15 +328,16 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L) {
                 // generic reads of the slot before the next async copy into it
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bars + 8u * (1 + S + slot));
+                if (lane == 0) mbar_arrive(empty0 + 8u * slot);
             }
+            fence_before_sync();
         }
     }
     fence_before_sync();
     __syncthreads();
     if (warp == 0) {
         fence_after_sync();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128u)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256u)
                      : "memory");
     }
 }

@@ -207,7 +207,10 @@ def test_workspace_too_small_is_rejected():
     assert ei.value.status == 4
 
 
-@pytest.mark.parametrize("T,C,r,n", [(4096, 3072, 32, 4), (300, 136, 16, 3), (77, 64, 33, 2)])
+# The larger batches give the apply kernel several token tiles per CTA (its
+# persistent path), with ragged channel and token tails, at rank <= 32 and 64.
+@pytest.mark.parametrize("T,C,r,n", [(4096, 3072, 32, 4), (300, 136, 16, 3), (77, 64, 33, 2),
+                                     (1100, 264, 16, 64), (650, 520, 64, 32)])
 def test_batched_lowrank_equals_single_calls(T, C, r, n):
     """One batched call over n buffers computes exactly what n single calls do
     (same kernels, fixed reduction orders), for the sender and the receiver;
