@@ -28,7 +28,8 @@ EXPORTS = ("cf_status_string", "cf_abi_version", "cf_codes_words_per_row",
            "cf_lowrank_factor_bytes", "cf_lowrank_encode", "cf_lowrank_decode",
            "cf_lowrank_status", "cf_set_lowrank_engine", "cf_set_quant_pipeline",
            "cf_set_launch_override", "cf_lowrank_encode_noalloc", "cf_decode_emit",
-           "cf_decode_emit_batched", "cf_lowrank_encode_batched", "cf_lowrank_decode_batched")
+           "cf_decode_emit_batched", "cf_lowrank_encode_batched", "cf_lowrank_decode_batched",
+           "cf_lowrank_set_apply_events")
 
 
 class CFError(RuntimeError):
@@ -107,6 +108,7 @@ def lib():
             "cf_lowrank_decode_batched": ([D, i32, vp, vp, vp], ctypes.c_int),
             "cf_set_launch_override": ([i32, i32, i32, i32], ctypes.c_int),
             "cf_set_lowrank_engine": ([i32], ctypes.c_int),
+            "cf_lowrank_set_apply_events": ([vp, vp, vp, vp], ctypes.c_int),
             "cf_set_quant_pipeline": ([i32, i32, i32], ctypes.c_int),
             "cf_lowrank_encode_noalloc": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         }
@@ -243,6 +245,17 @@ def cf_lowrank_status(workspace, stream=None) -> int:
 
 def cf_set_lowrank_engine(engine: int):
     _chk(lib().cf_set_lowrank_engine(engine), "cf_set_lowrank_engine")
+
+
+def _ev(e):
+    """torch.cuda.Event (already recorded once, so that it exists) or None ->
+    its cudaEvent_t handle."""
+    return None if e is None else ctypes.c_void_p(e.cuda_event)
+
+
+def cf_lowrank_set_apply_events(enc_start=None, enc_stop=None, dec_start=None, dec_stop=None):
+    _chk(lib().cf_lowrank_set_apply_events(_ev(enc_start), _ev(enc_stop), _ev(dec_start),
+                                           _ev(dec_stop)), "cf_lowrank_set_apply_events")
 
 
 def cf_set_quant_pipeline(kernel: int, pipeline: int, stages: int = 0):

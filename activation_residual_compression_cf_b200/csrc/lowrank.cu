@@ -120,6 +120,15 @@ int sm_count() {
 
 std::atomic<int> g_engine{0};  // 0 = tensor cores (tcgen05), 1 = CUDA cores
 
+// Events recorded around the apply launch (measurement hook), per direction.
+std::atomic<void *> g_apply_ev[2][2] = {};
+
+cf_status record_apply_event(bool sender, int which, cudaStream_t st) {
+    void *ev = g_apply_ev[sender ? 0 : 1][which].load();
+    if (!ev) return CF_OK;
+    return cudaEventRecord(static_cast<cudaEvent_t>(ev), st) == cudaSuccess ? CF_OK : CF_ERR_CUDA;
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // dependency on libcuda).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -268,7 +277,7 @@ cf_status launch_apply_tc(const LrBatch &B, const Layout &L, int n, cudaStream_t
 // D = P^ Q^T applied to the state.  Engine 0: tensor cores (tcgen05 tf32,
 // hi/lo split); engine 1: CUDA-core FMA chain.  A buffer's sender and
 // receiver must use the same engine to stay bit-identical.
-cf_status apply(bool sender, const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
+cf_status apply_launch(bool sender, const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
     if (g_engine.load() == 0) {
         if (L.rp <= 32)
             return sender ? launch_apply_tc<true, 32>(B, L, n, st) : launch_apply_tc<false, 32>(B, L, n, st);
@@ -294,6 +303,14 @@ cf_status apply(bool sender, const LrBatch &B, const Layout &L, int n, cudaStrea
     }
     LR_LAUNCHED();
     return CF_OK;
+}
+
+cf_status apply(bool sender, const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
+    const cf_status e0 = record_apply_event(sender, 0, st);
+    const cf_status k = apply_launch(sender, B, L, n, st);
+    const cf_status e1 = record_apply_event(sender, 1, st);
+    if (k != CF_OK) return k;
+    return e0 != CF_OK ? e0 : e1;
 }
 
 // The whole sender for n buffers (n = 1 for the single-buffer call).
@@ -431,6 +448,18 @@ cf_status cf_lowrank_decode_batched(const cf_desc *d, int32_t n, const cf_lowran
 cf_status cf_set_lowrank_engine(int32_t engine) {
     if (engine < 0 || engine > 1) return CF_ERR_INVALID_ARG;
     g_engine.store(engine);
+    return CF_OK;
+}
+
+cf_status cf_lowrank_set_apply_events(void *enc_start, void *enc_stop, void *dec_start,
+                                      void *dec_stop) {
+    if ((enc_start == nullptr) != (enc_stop == nullptr) ||
+        (dec_start == nullptr) != (dec_stop == nullptr))
+        return CF_ERR_INVALID_ARG;
+    g_apply_ev[0][0].store(enc_start);
+    g_apply_ev[0][1].store(enc_stop);
+    g_apply_ev[1][0].store(dec_start);
+    g_apply_ev[1][1].store(dec_stop);
     return CF_OK;
 }
 

@@ -68,7 +68,9 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v) {
 // rank <= 32 keeps two CTAs per SM.
 constexpr int kApplyStageTok = 16;
 constexpr int kApplyConsumers = 256;            // 8 warps: 4 channel quarters x 2 token halves
-constexpr int kApplyThreads = kApplyConsumers + 32;  // + one producer warp
+constexpr int kApplyProducerWarp = kApplyConsumers / 32;   // warp 8: bulk copies
+constexpr int kApplyMmaWarp = kApplyProducerWarp + 1;      // warp 9: B operands + MMAs
+constexpr int kApplyThreads = kApplyConsumers + 64;
 constexpr int kApplyMaxTilesPerCta = 8;
 
 template <bool SENDER>
@@ -81,7 +83,7 @@ __host__ __device__ constexpr int apply_ring() {
 }
 template <bool SENDER, int KP>
 __host__ __device__ constexpr int apply_tc_smem() {
-    return 1024 + 3 * (KP / 32) * 16384 + apply_ring<SENDER, KP>() * apply_stage_bytes<SENDER>() + 256;
+    return 1024 + 3 * (KP / 32) * 16384 + apply_ring<SENDER, KP>() * apply_stage_bytes<SENDER>() + 512;
 }
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
@@ -93,17 +95,19 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void consumers_sync() {
-    asm volatile("bar.sync 1, %0;" ::"r"(kApplyConsumers) : "memory");
+// consumers + the MMA warp, once, after the first operands are built
+__device__ __forceinline__ void operand_sync() {
+    asm volatile("bar.sync 1, %0;" ::"r"(kApplyConsumers + 32) : "memory");
 }
 
-// B operand of one token tile: b[t][k] = qP[t][k] * (sP[k] sQ[k]) split into
-// the tf32-exact hi part and the remainder; 16-byte chunks of 4 consecutive k.
+// B operand of one token tile: b[t][k] = qP[t][k] * s[k] (s[k] = sP[k] sQ[k],
+// precomputed in shared memory) split into the tf32-exact hi part and the
+// remainder; 16-byte chunks of 4 consecutive k, threads [tid0, tid0 + nthr).
 template <int KP>
 __device__ __forceinline__ void apply_build_b(uint8_t *gbh, uint8_t *gbl, const uint8_t *pc,
-                                              const float *ps, const float *qs, int64_t t0,
-                                              int64_t T, int r, int nb, int tid) {
-    for (int idx = tid; idx < kApplyTile * (KP / 4); idx += kApplyConsumers) {
+                                              const float *sk, int64_t t0, int64_t T, int r,
+                                              int nb, int tid, int nthr) {
+    for (int idx = tid; idx < kApplyTile * (KP / 4); idx += nthr) {
         const int row = idx / (KP / 4), k0 = (idx - row * (KP / 4)) * 4;
         const int64_t t = t0 + row;
         float h[4], l[4];
@@ -111,8 +115,7 @@ __device__ __forceinline__ void apply_build_b(uint8_t *gbh, uint8_t *gbl, const 
         for (int u = 0; u < 4; ++u) {
             const int k = k0 + u;
             float b = 0.0f;
-            if (t < T && k < r)
-                b = __fmul_rn((float)int4_code_at(pc + t * nb, k), __fmul_rn(__ldg(ps + k), __ldg(qs + k)));
+            if (t < T && k < r) b = __fmul_rn((float)int4_code_at(pc + t * nb, k), sk[k]);
             h[u] = __uint_as_float(__float_as_uint(b) & 0xFFFFE000u);
             l[u] = __fsub_rn(b, h[u]);
         }
@@ -122,25 +125,64 @@ __device__ __forceinline__ void apply_build_b(uint8_t *gbh, uint8_t *gbl, const 
     }
 }
 
+// The same B operand built by one warp: lane l owns token rows l, l + 32,
+// l + 64, l + 96; each row's packed codes (nb bytes) are loaded with all
+// loads in flight before any is used, then the row's KP values are written
+// as hi and lo 16-byte chunks.
+template <int KP>
+__device__ __forceinline__ void apply_build_b_warp(uint8_t *gbh, uint8_t *gbl, const uint8_t *pc,
+                                                   const float *sk, int64_t t0, int64_t T, int r,
+                                                   int nb, int lane) {
+    constexpr int NBX = KP / 2;
+#pragma unroll 1
+    for (int rr = 0; rr < kApplyTile / 32; ++rr) {
+        const int row = lane + 32 * rr;
+        const int64_t t = t0 + row;
+        const bool live = t < T;
+        const uint8_t *src = pc + t * nb;
+        uint32_t by[NBX];
+#pragma unroll
+        for (int j = 0; j < NBX; ++j) by[j] = (live && j < nb) ? (uint32_t)__ldg(src + j) : 0u;
+#pragma unroll
+        for (int k0 = 0; k0 < KP; k0 += 4) {
+            float h[4], l[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int k = k0 + u;
+                const int q = (int)((by[k >> 1] >> ((k & 1) * 4)) & 0xFu);
+                const float b = k < r ? __fmul_rn((float)(q >= 8 ? q - 16 : q), sk[k]) : 0.0f;
+                h[u] = __uint_as_float(__float_as_uint(b) & 0xFFFFE000u);
+                l[u] = __fsub_rn(b, h[u]);
+            }
+            const uint32_t off = sw128_f32_offset(row, k0);
+            *reinterpret_cast<float4 *>(gbh + off) = make_float4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<float4 *>(gbl + off) = make_float4(l[0], l[1], l[2], l[3]);
+        }
+    }
+}
+
 // Persistent over a run of token tiles: CTA (x, y, z) owns channel block x of
-// buffer z and token tiles [y * tpc, (y + 1) * tpc).  Warp roles (288
+// buffer z and token tiles [y * tpc, (y + 1) * tpc).  Warp roles (320
 // threads):
-//   warps 0-7 : build the A operand (Q codes of the channel block) once and
-//               the B operand of each token tile; thread 0 issues the MMAs
-//               into one of two TMEM accumulators (128 columns each), so the
-//               next tile's product runs while this tile is combined; each
-//               warp combines one channel quarter (w % 4, its TMEM lanes) x
-//               one half (w / 4) of every 16-token stage, reading x and recon
-//               from shared memory and D from TMEM, and writes err and recon;
+//   warps 0-7 : with warp 9, build the A operand (Q codes of the channel
+//               block) and tile 0's B operand; then each warp combines one
+//               channel quarter (w % 4, its TMEM lanes) x one half (w / 4) of
+//               every 16-token stage of every tile, reading x and recon from
+//               shared memory and D from TMEM, and writes err and recon;
 //   warp 8    : one lane issues 1-D bulk copies (cp.async.bulk, no multicast)
 //               of every token row's 128-channel segment of recon (and x) of
 //               all the CTA's tiles into the ring, from the kernel's first
-//               instructions on.
-// The B operand is single-buffered: tile i+1's is written after tile i's MMA
-// has completed (its commit barrier), before tile i is combined.
+//               instructions on;
+//   warp 9    : for tile i, once tile i-1's product is done (its commit
+//               barrier) writes tile i's B operand (single buffer), and once
+//               the consumers have released accumulator i % 2 (tile i-2
+//               combined) issues the MMAs of tile i into it.
+// So the consumers never wait on operand building: the product of the next
+// tile is formed while the current one is combined.
 // Every wait is bounded; on expiry CF_ERR_TIMEOUT goes to the buffer's status
-// word, the consumer warps leave together at the next tile boundary, the
-// producer waits (bounded) for its copies still in flight, and TMEM is freed.
+// word and the waiting warp stops (the others then run out of their own
+// waits), the producer waits (bounded) for its copies still in flight, and
+// TMEM is freed.
 template <bool SENDER, int KP>
 __global__ void __launch_bounds__(kApplyThreads, (KP <= 32 ? 2 : 1))
 lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int tpc) {
@@ -167,10 +209,11 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
     const uint32_t sA = base, sBh = base + OPB, sBl = base + 2 * OPB;
     const uint32_t ring = base + 3 * OPB;
     uint8_t *gring = gb + 3 * OPB;
-    const uint32_t bars = ring + S * SB;       // mma[2], full[S], empty[S]
-    const uint32_t full0 = bars + 16u, empty0 = bars + 16u + 8u * S;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(gring + S * SB + 8 * (2 + 2 * S));
-    int *abort_flag = reinterpret_cast<int *>(tslot + 1);
+    // barriers: mma[2], acc_free[2], full[S], empty[S]
+    const uint32_t bars = ring + S * SB;
+    const uint32_t mma0 = bars, accf0 = bars + 16u, full0 = bars + 32u, empty0 = bars + 32u + 8u * S;
+    float *sk = reinterpret_cast<float *>(gring + S * SB + 8 * (4 + 2 * S));   // [KP]
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sk + KP);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t c0 = (int64_t)blockIdx.x * kApplyTile;
@@ -184,15 +227,17 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
     const int64_t cw = (C - c0 < kApplyTile) ? C - c0 : kApplyTile;   // channels in the block
 
     if (tid == 0) {
-        mbar_init(bars, 1);
-        mbar_init(bars + 8u, 1);
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(mma0 + 8u * j, 1);                         // tcgen05.commit
+            mbar_init(accf0 + 8u * j, kApplyConsumers / 32);     // one per consumer warp
+        }
         for (int s = 0; s < S; ++s) {
             mbar_init(full0 + 8u * s, 1);                        // producer + tx bytes
             mbar_init(empty0 + 8u * s, kApplyConsumers / 32);    // one per consumer warp
         }
-        *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    if (tid < KP) sk[tid] = tid < r ? __fmul_rn(__ldg(ps + tid), __ldg(qs + tid)) : 0.0f;
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tslot)),
@@ -205,7 +250,7 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
     fence_after_sync();
     const uint32_t tmem = *tslot;
 
-    if (warp == kApplyConsumers / 32) {
+    if (warp == kApplyProducerWarp) {
         // ---------------- producer: stages of 16 rows over [tbeg, tend) ----------------
         if (lane == 0) {
             const uint32_t rbytes = (uint32_t)cw * 4u, xbytes = (uint32_t)cw * 2u;
@@ -241,9 +286,11 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
                 (void)mbar_wait(full0 + 8u * (st % S), (uint32_t)((st / S) & 1));
         }
     } else {
-        // ---------------- operands, MMAs, combine ----------------
-        // A = the INT4 codes of Q for this channel block, once.
-        for (int idx = tid; idx < kApplyTile * (KP / 4); idx += kApplyConsumers) {
+        // A = the INT4 codes of Q for this channel block, and tile 0's B:
+        // built once by the consumers and the MMA warp together.
+        const int ot = warp == kApplyMmaWarp ? kApplyConsumers + lane : tid;
+        constexpr int kOpThreads = kApplyConsumers + 32;
+        for (int idx = ot; idx < kApplyTile * (KP / 4); idx += kOpThreads) {
             const int row = idx / (KP / 4), k0 = (idx - row * (KP / 4)) * 4;
             const int64_t c = c0 + row;
             float a[4];
@@ -254,83 +301,101 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
             }
             *reinterpret_cast<float4 *>(gb + sw128_f32_offset(row, k0)) = make_float4(a[0], a[1], a[2], a[3]);
         }
-        apply_build_b<KP>(gb + OPB, gb + 2 * OPB, pc, ps, qs, tbeg, T, r, nb, tid);
-        const int ksteps = (r + 7) / 8;
-        constexpr uint32_t idesc = idesc_tf32(kApplyTile);
-        auto issue_mma = [&](int i) {
-            const uint32_t acc = tmem + (uint32_t)(128 * (i & 1));
-            for (int kk = 0; kk < ksteps; ++kk) {
-                const uint32_t off = (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32);
-                const uint64_t da = sw128_desc(sA + off, 16, 1024);
-                mma_tf32(acc, da, sw128_desc(sBh + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
-                mma_tf32(acc, da, sw128_desc(sBl + off, 16, 1024), idesc, 1u);
-            }
-            mma_commit(bars + 8u * (i & 1));
-        };
+        apply_build_b<KP>(gb + OPB, gb + 2 * OPB, pc, sk, tbeg, T, r, nb, ot, kOpThreads);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         fence_before_sync();
-        consumers_sync();
+        operand_sync();
         fence_after_sync();
-        if (tid == 0) issue_mma(0);
 
-        const int q = warp & 3, half = warp >> 2;
-        const int cl = 32 * q + lane;              // channel within the block
-        const int64_t c = c0 + cl;
-        const bool col_ok = cl < cw;
-        const uint32_t tlane = (uint32_t)(32 * q) << 16;
-        int g = 0;                                 // stages consumed so far
-        for (int i = 0; i < nt; ++i) {
-            // tile i's product is done: its accumulator may be read and the
-            // B operand rewritten
-            if (!__all_sync(kFullMask, mbar_wait(bars + 8u * (i & 1), (uint32_t)((i >> 1) & 1))))
-                if (lane == 0) *(volatile int *)abort_flag = 1;
-            fence_after_sync();
-            const int64_t t0 = tbeg + (int64_t)i * kApplyTile;
-            if (i + 1 < nt)
-                apply_build_b<KP>(gb + OPB, gb + 2 * OPB, pc, ps, qs, t0 + kApplyTile, T, r, nb, tid);
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            fence_before_sync();
-            consumers_sync();
-            fence_after_sync();
-            if (*(volatile int *)abort_flag) {
-                if (tid == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
-                break;  // every consumer warp reads the same flag after the barrier
-            }
-            if (tid == 0 && i + 1 < nt) issue_mma(i + 1);
-
-            const uint32_t acc = tmem + tlane + (uint32_t)(128 * (i & 1));
-            const int64_t tw = (T - t0 < kApplyTile) ? T - t0 : kApplyTile;
-            const int ns = (int)((tw + kApplyStageTok - 1) / kApplyStageTok);
-            for (int st = 0; st < ns; ++st, ++g) {
-                const int slot = g % S;
-                if (!__all_sync(kFullMask, mbar_wait(full0 + 8u * slot, (uint32_t)((g / S) & 1)))) {
-                    if (lane == 0) *(volatile int *)abort_flag = 1;
+        if (warp == kApplyMmaWarp) {
+            // ---------------- B operands and MMAs ----------------
+            const int ksteps = (r + 7) / 8;
+            constexpr uint32_t idesc = idesc_tf32(kApplyTile);
+            for (int i = 0; i < nt; ++i) {
+                if (i > 0) {
+                    // tile i-1's product has read the B buffer
+                    if (!__all_sync(kFullMask, mbar_wait(mma0 + 8u * ((i - 1) & 1), (uint32_t)(((i - 1) >> 1) & 1)))) {
+                        if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+                        break;
+                    }
+                    apply_build_b_warp<KP>(gb + OPB, gb + 2 * OPB, pc, sk, tbeg + (int64_t)i * kApplyTile,
+                                           T, r, nb, lane);
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                }
+                // accumulator i % 2 is free once tile i-2 has been combined
+                if (i >= 2 && !__all_sync(kFullMask, mbar_wait(accf0 + 8u * (i & 1), (uint32_t)(((i - 2) >> 1) & 1)))) {
+                    if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
                     break;
                 }
-                const int tl = st * kApplyStageTok + 8 * half;   // first token column of this warp
-                float dv[8];
-                tmem_ld8(acc + (uint32_t)tl, dv);
-                const float *sr = reinterpret_cast<const float *>(gring + slot * SB) + 8 * half * kApplyTile;
-                const uint16_t *sx = reinterpret_cast<const uint16_t *>(gring + slot * SB + RB) + 8 * half * kApplyTile;
-                if (col_ok) {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        if (tl + j >= tw) break;
-                        const float rv = sr[j * kApplyTile + cl];
-                        const int64_t o = (t0 + tl + j) * C + c;
-                        if (SENDER) {
-                            const float v = __fsub_rn(bf16_bits_to_f32(sx[j * kApplyTile + cl]), rv);
-                            __stcs(err + o, __fsub_rn(v, dv[j]));
-                        }
-                        __stcs(recon + o, __fadd_rn(rv, dv[j]));
-                    }
-                }
-                // generic reads of the slot before the next async copy into it
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(empty0 + 8u * slot);
+                fence_after_sync();
+                if (lane == 0) {
+                    const uint32_t acc = tmem + (uint32_t)(128 * (i & 1));
+                    for (int kk = 0; kk < ksteps; ++kk) {
+                        const uint32_t off = (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32);
+                        const uint64_t da = sw128_desc(sA + off, 16, 1024);
+                        mma_tf32(acc, da, sw128_desc(sBh + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                        mma_tf32(acc, da, sw128_desc(sBl + off, 16, 1024), idesc, 1u);
+                    }
+                    mma_commit(mma0 + 8u * (i & 1));
+                }
+                __syncwarp();
             }
-            fence_before_sync();
+        } else {
+            // ---------------- combine ----------------
+            const int q = warp & 3, half = warp >> 2;
+            const int cl = 32 * q + lane;              // channel within the block
+            const int64_t c = c0 + cl;
+            const bool col_ok = cl < cw;
+            const uint32_t tlane = (uint32_t)(32 * q) << 16;
+            int g = 0;                                 // stages consumed so far
+            bool ok = true;
+            for (int i = 0; i < nt && ok; ++i) {
+                if (!__all_sync(kFullMask, mbar_wait(mma0 + 8u * (i & 1), (uint32_t)((i >> 1) & 1)))) {
+                    if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+                    break;
+                }
+                fence_after_sync();
+                const int64_t t0 = tbeg + (int64_t)i * kApplyTile;
+                const uint32_t acc = tmem + tlane + (uint32_t)(128 * (i & 1));
+                const int64_t tw = (T - t0 < kApplyTile) ? T - t0 : kApplyTile;
+                const int ns = (int)((tw + kApplyStageTok - 1) / kApplyStageTok);
+                for (int st = 0; st < ns; ++st, ++g) {
+                    const int slot = g % S;
+                    if (!__all_sync(kFullMask, mbar_wait(full0 + 8u * slot, (uint32_t)((g / S) & 1)))) {
+                        if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                    const int tl = st * kApplyStageTok + 8 * half;   // first token column of this warp
+                    float dv[8];
+                    tmem_ld8(acc + (uint32_t)tl, dv);
+                    const float *sr = reinterpret_cast<const float *>(gring + slot * SB) + 8 * half * kApplyTile;
+                    const uint16_t *sx = reinterpret_cast<const uint16_t *>(gring + slot * SB + RB) + 8 * half * kApplyTile;
+                    if (col_ok) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            if (tl + j >= tw) break;
+                            const float rv = sr[j * kApplyTile + cl];
+                            const int64_t o = (t0 + tl + j) * C + c;
+                            if (SENDER) {
+                                const float v = __fsub_rn(bf16_bits_to_f32(sx[j * kApplyTile + cl]), rv);
+                                __stcs(err + o, __fsub_rn(v, dv[j]));
+                            }
+                            __stcs(recon + o, __fadd_rn(rv, dv[j]));
+                        }
+                    }
+                    // generic reads of the slot before the next async copy into it
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(empty0 + 8u * slot);
+                }
+                if (!ok) break;
+                // this warp's reads of accumulator i % 2 are complete
+                fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(accf0 + 8u * (i & 1));
+            }
         }
     }
     fence_before_sync();

@@ -158,22 +158,27 @@ class ClockSampler:
                 "window": "timed region" if win else "whole run (timed region shorter than one sample)"}
 
 
-def kernel_source_hash():
+QUANT_SOURCES = ("quant_tma.cuh", "quant_kernels.cuh", "cf_common.cuh", "cf_api.cu")
+LOWRANK_APPLY_SOURCES = ("lowrank_apply_tc.cuh", "lowrank_umma.cuh", "lowrank_kernels.cuh",
+                         "lowrank_api.cuh", "lowrank.cu", "cf_common.cuh")
+
+
+def kernel_source_hash(files=QUANT_SOURCES):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "activation_residual_compression_cf_b200", "csrc")
-    for fn in ("quant_tma.cuh", "quant_kernels.cuh", "cf_common.cuh", "cf_api.cu"):
+    for fn in files:
         h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, workload: str):
+def recorded_traffic(kernel: str, workload: str, files=QUANT_SOURCES):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current kernel source; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(f"{kernel}:{workload}")
-    if not d or d.get("source_hash") != kernel_source_hash():
+    if not d or d.get("source_hash") != kernel_source_hash(files):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -429,26 +434,45 @@ def run_lowrank(args, world, rank, local):
         enc(i)
         dec()
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+
+    def events(k):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(k)]
+
+    ev = [events(3) for _ in range(args.steps)]
+    # events the library records around the sender's and the receiver's
+    # apply kernel (recorded once here so that they exist)
+    aev = [events(4) for _ in range(args.steps)]
+    for e in aev:
+        for x_ in e:
+            x_.record(stream)
+    torch.cuda.synchronize()
     with R.bracket():
         wall0 = time.time()
         for i in range(args.steps):
             e0, e1, e2 = ev[i]
+            cf.cf_lowrank_set_apply_events(*aev[i])
             e0.record(stream)
             enc(args.warmup + i)
             e1.record(stream)
             dec()
             e2.record(stream)
+    cf.cf_lowrank_set_apply_events()
     clocks = sampler.stop(wall0, time.time())
     ms = ev[0][0].elapsed_time(ev[-1][2])
     enc_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
     dec_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    app_enc_ms = statistics.mean(a[0].elapsed_time(a[1]) for a in aev)
+    app_dec_ms = statistics.mean(a[2].elapsed_time(a[3]) for a in aev)
     ms = R.reduce_scalar(ms, "max")
     peak, peak_kind = peaks()
     value = 2 * T * C * n * args.steps * world / (ms / 1e3) / 1e9
     enc_bytes = n * T * C * 14
     dec_bytes = n * T * C * 8
+    # apply kernels: x, recon r/w, err (sender) or recon r/w (receiver), plus
+    # the packed factors and their scales
+    fac_bytes = n * ((T + C) * nb + 2 * 4 * r)
+    app_enc_bytes = enc_bytes + fac_bytes
+    app_dec_bytes = dec_bytes + fac_bytes
     status = max(cf.cf_lowrank_status(ws[b * wsb:]) for b in range(n))
     # Launches per step: the sender runs prep, residual, omega, five kernels
     # per subspace iteration (project, Gram+Cholesky, orthogonalise,
@@ -479,15 +503,25 @@ def run_lowrank(args, world, rank, local):
                    "rank": r, "iters": it, "mode": "low-rank INT4 + EF",
                    "parallelism": f"replicas x{world}", "l2": "inputs larger than L2",
                    "launches_per_step": launches_per_step},
-        "roofline": {"bound": "hbm", "achieved": round(enc_bytes / (enc_ms / 1e3) / 1e9, 1),
+        "roofline": {"bound": "hbm",
+                     "achieved": round(app_enc_bytes / (app_enc_ms / 1e3) / 1e9, 1),
                      "peak": peak, "unit": "GB/s",
-                     "frac": round(enc_bytes / (enc_ms / 1e3) / 1e9 / peak, 4), "traffic": None,
-                     "kernel": "cf_lowrank_encode (whole call, 14 B/elem unavoidable I/O)",
-                     "peak_kind": peak_kind},
-        "decode": {"achieved": round(dec_bytes / (dec_ms / 1e3) / 1e9, 1),
-                   "frac": round(dec_bytes / (dec_ms / 1e3) / 1e9 / peak, 4),
-                   "avg_ms_per_step": round(dec_ms, 4)},
-        "encode_ms_per_step": round(enc_ms, 4), "lowrank_status": status,
+                     "frac": round(app_enc_bytes / (app_enc_ms / 1e3) / 1e9 / peak, 4),
+                     "traffic": recorded_traffic("apply_sender", args.workload,
+                                                 LOWRANK_APPLY_SOURCES),
+                     "kernel": "lr_apply_tc_kernel<sender> (batched; D, EF update)",
+                     "peak_kind": peak_kind, "algorithmic_bytes_per_launch": app_enc_bytes,
+                     "avg_launch_ms": round(app_enc_ms, 4)},
+        "decode": {"kernel": "lr_apply_tc_kernel<receiver> (batched)",
+                   "achieved": round(app_dec_bytes / (app_dec_ms / 1e3) / 1e9, 1),
+                   "frac": round(app_dec_bytes / (app_dec_ms / 1e3) / 1e9 / peak, 4),
+                   "algorithmic_bytes_per_launch": app_dec_bytes,
+                   "avg_launch_ms": round(app_dec_ms, 4)},
+        "whole_call": {"encode_ms_per_step": round(enc_ms, 4),
+                       "decode_ms_per_step": round(dec_ms, 4),
+                       "encode_frac_of_14B_per_elem": round(
+                           enc_bytes / (enc_ms / 1e3) / 1e9 / peak, 4)},
+        "lowrank_status": status,
         "payload_ratio": round(2 * T * C / cf.cf_payload_bytes(d), 2),
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,

@@ -303,6 +303,20 @@ cf_status cf_lowrank_status(void *workspace, void *stream);
  * other value. */
 cf_status cf_set_lowrank_engine(int32_t engine);
 
+/* Measurement hook (no counterpart in the paper): CUDA events (cudaEvent_t,
+ * passed as void*) that the low-rank calls record around their apply kernel
+ * -- the kernel that forms D and updates the state -- so a caller can time
+ * that one kernel inside a whole call.  When enc_start/enc_stop are non-null,
+ * every later cf_lowrank_encode(_batched) records enc_start on its stream
+ * immediately before the apply launch and enc_stop immediately after it;
+ * dec_start/dec_stop likewise for cf_lowrank_decode(_batched).  Null pairs
+ * (the default) record nothing.  Process-wide; the events stay the caller's
+ * (create them before, destroy them after the calls that record them).  An
+ * event that fails to record makes the call return CF_ERR_CUDA after its
+ * launches.  Returns CF_ERR_INVALID_ARG if exactly one of a pair is null. */
+cf_status cf_lowrank_set_apply_events(void *enc_start, void *enc_stop, void *dec_start,
+                                      void *dec_stop);
+
 /* Memory pipeline of the quantize-mode kernels in this process: kernel 0 =
  * encode, 1 = decode; pipeline 0 = register-resident rows (each thread
  * loads its channel groups straight into registers), 1 = TMA row staging

@@ -107,6 +107,11 @@ def test_pipeline_and_engine_knobs_validate(L):
     assert L.cf_set_quant_pipeline(0, 1, 0) == 0   # restore the default
     assert L.cf_set_lowrank_engine(2) == 1
     assert L.cf_set_lowrank_engine(0) == 0
+    # the apply-event hook takes pairs: half a pair is rejected, all-null clears
+    one = ctypes.c_void_p(1)
+    assert L.cf_lowrank_set_apply_events(one, None, None, None) == 1
+    assert L.cf_lowrank_set_apply_events(None, None, None, one) == 1
+    assert L.cf_lowrank_set_apply_events(None, None, None, None) == 0
 
 
 def test_binding_raises_when_library_missing(monkeypatch, tmp_path):

@@ -256,3 +256,35 @@ def test_batched_lowrank_equals_single_calls(T, C, r, n):
     torch.cuda.synchronize()
     assert cf.cf_lowrank_status(ws) == 2
     assert torch.equal(bad.recon_s, before)
+
+
+def test_apply_event_hook_times_the_apply_kernel_only():
+    """Events handed to cf_lowrank_set_apply_events bracket the apply kernel
+    of the next encode and decode: they are recorded (elapsed time > 0, less
+    than the whole encode), results are unchanged, and clearing the hook
+    stops the recording."""
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=1024, channels=3072)
+    xs = W.trajectory(wl, 0, steps=2, device="cuda")
+    om = W.omega(wl, 0, 1, device="cuda")
+    plain, hooked = GpuLowrank(1024, 3072, 32, 2), GpuLowrank(1024, 3072, 32, 2)
+    for g in (plain, hooked):
+        g.init(xs[0].clone())
+    plain.step(xs[1].clone(), om)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for e in ev:
+        e.record()
+    torch.cuda.synchronize()
+    try:
+        cf.cf_lowrank_set_apply_events(ev[0], ev[1], ev[2], ev[3])
+        ev[4].record()
+        hooked.step(xs[1].clone(), om)
+        ev[5].record()
+    finally:
+        cf.cf_lowrank_set_apply_events()
+    torch.cuda.synchronize()
+    for k in ("recon_s", "recon_r", "err"):
+        assert torch.equal(getattr(plain, k), getattr(hooked, k)), k
+    t_enc, t_dec, t_all = ev[0].elapsed_time(ev[1]), ev[2].elapsed_time(ev[3]), ev[4].elapsed_time(ev[5])
+    assert 0 < t_enc < t_all and 0 < t_dec < t_all
+    # the encode's apply ends before the decode's begins
+    assert ev[1].elapsed_time(ev[2]) >= 0
