@@ -57,16 +57,28 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v) {
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
                    "=r"(r[6]), "=r"(r[7])
                  : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    // the wait takes the destination registers as operands, so no use of
+    // them can be scheduled above it
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7])
+                 :
+                 : "memory");
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Staging of x and recon: a tile's 128 tokens are 8 stages of 16 token rows;
-// a stage holds the rows' recon (16 x 128 fp32) and, for the sender, x
-// (16 x 128 bf16).  Ring depth per kernel, sized so that the sender with
-// rank <= 32 keeps two CTAs per SM.
-constexpr int kApplyStageTok = 16;
+// Staging of x and recon: a tile's 128 tokens are stages of STOK token rows;
+// a stage holds the rows' recon (STOK x 128 fp32) and, for the sender, x
+// (STOK x 128 bf16).  Each consumer warp takes STOK / 2 tokens of a stage.
+// The receiver moves half the bytes per element, so its stages are twice as
+// long to spread the fixed per-stage cost (barrier, TMEM load, release) over
+// as many bytes.  Ring depth per kernel, sized so that rank <= 32 keeps two
+// CTAs per SM.
+template <bool SENDER>
+__host__ __device__ constexpr int apply_stage_tok() {
+    return SENDER ? 16 : 32;
+}
 constexpr int kApplyConsumers = 256;            // 8 warps: 4 channel quarters x 2 token halves
 constexpr int kApplyProducerWarp = kApplyConsumers / 32;   // warp 8: bulk copies
 constexpr int kApplyMmaWarp = kApplyProducerWarp + 1;      // warp 9: B operands + MMAs
@@ -75,11 +87,11 @@ constexpr int kApplyMaxTilesPerCta = 8;
 
 template <bool SENDER>
 __host__ __device__ constexpr int apply_stage_bytes() {
-    return kApplyStageTok * kApplyTile * (SENDER ? 6 : 4);
+    return apply_stage_tok<SENDER>() * kApplyTile * (SENDER ? 6 : 4);
 }
 template <bool SENDER, int KP>
 __host__ __device__ constexpr int apply_ring() {
-    return KP <= 32 ? (SENDER ? 4 : 6) : 8;
+    return KP <= 32 ? (SENDER ? 4 : 3) : (SENDER ? 8 : 4);
 }
 template <bool SENDER, int KP>
 __host__ __device__ constexpr int apply_tc_smem() {
@@ -126,37 +138,61 @@ __device__ __forceinline__ void apply_build_b(uint8_t *gbh, uint8_t *gbl, const 
 }
 
 // The same B operand built by one warp: lane l owns token rows l, l + 32,
-// l + 64, l + 96; each row's packed codes (nb bytes) are loaded with all
-// loads in flight before any is used, then the row's KP values are written
-// as hi and lo 16-byte chunks.
+// l + 64, l + 96.  The packed codes of all four rows are loaded before any
+// is used -- as 32-bit words when the rows are 4-byte aligned (nb % 4 == 0
+// and an aligned code array: the usual case), else byte by byte one row at
+// a time -- then each row's KP values are written as hi and lo 16-byte chunks.
+template <int KP>
+__device__ __forceinline__ void apply_b_row(uint8_t *gbh, uint8_t *gbl, const uint32_t *w,
+                                            const float *sk, int row, int r) {
+#pragma unroll
+    for (int k0 = 0; k0 < KP; k0 += 4) {
+        float h[4], l[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int k = k0 + u;
+            const int q = (int)((w[k >> 3] >> ((k & 7) * 4)) & 0xFu);
+            const float b = k < r ? __fmul_rn((float)(q >= 8 ? q - 16 : q), sk[k]) : 0.0f;
+            h[u] = __uint_as_float(__float_as_uint(b) & 0xFFFFE000u);
+            l[u] = __fsub_rn(b, h[u]);
+        }
+        const uint32_t off = sw128_f32_offset(row, k0);
+        *reinterpret_cast<float4 *>(gbh + off) = make_float4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<float4 *>(gbl + off) = make_float4(l[0], l[1], l[2], l[3]);
+    }
+}
+
 template <int KP>
 __device__ __forceinline__ void apply_build_b_warp(uint8_t *gbh, uint8_t *gbl, const uint8_t *pc,
                                                    const float *sk, int64_t t0, int64_t T, int r,
                                                    int nb, int lane) {
-    constexpr int NBX = KP / 2;
+    constexpr int NW = KP / 8;                 // 32-bit words of codes per row (at most)
+    constexpr int RPL = kApplyTile / 32;       // rows per lane
+    const bool words = (nb & 3) == 0 && (reinterpret_cast<uintptr_t>(pc) & 3u) == 0;
+    if (words) {
+        const int nw = nb >> 2;
+        uint32_t w[RPL][NW];
+#pragma unroll
+        for (int rr = 0; rr < RPL; ++rr) {
+            const int64_t t = t0 + lane + 32 * rr;
+            const uint32_t *src = reinterpret_cast<const uint32_t *>(pc + t * nb);
+#pragma unroll
+            for (int j = 0; j < NW; ++j) w[rr][j] = (t < T && j < nw) ? __ldg(src + j) : 0u;
+        }
+#pragma unroll
+        for (int rr = 0; rr < RPL; ++rr) apply_b_row<KP>(gbh, gbl, w[rr], sk, lane + 32 * rr, r);
+    } else {
 #pragma unroll 1
-    for (int rr = 0; rr < kApplyTile / 32; ++rr) {
-        const int row = lane + 32 * rr;
-        const int64_t t = t0 + row;
-        const bool live = t < T;
-        const uint8_t *src = pc + t * nb;
-        uint32_t by[NBX];
+        for (int rr = 0; rr < RPL; ++rr) {
+            const int64_t t = t0 + lane + 32 * rr;
+            const uint8_t *src = pc + t * nb;
+            uint32_t w[NW];
 #pragma unroll
-        for (int j = 0; j < NBX; ++j) by[j] = (live && j < nb) ? (uint32_t)__ldg(src + j) : 0u;
+            for (int j = 0; j < NW; ++j) w[j] = 0u;
 #pragma unroll
-        for (int k0 = 0; k0 < KP; k0 += 4) {
-            float h[4], l[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int k = k0 + u;
-                const int q = (int)((by[k >> 1] >> ((k & 1) * 4)) & 0xFu);
-                const float b = k < r ? __fmul_rn((float)(q >= 8 ? q - 16 : q), sk[k]) : 0.0f;
-                h[u] = __uint_as_float(__float_as_uint(b) & 0xFFFFE000u);
-                l[u] = __fsub_rn(b, h[u]);
-            }
-            const uint32_t off = sw128_f32_offset(row, k0);
-            *reinterpret_cast<float4 *>(gbh + off) = make_float4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<float4 *>(gbl + off) = make_float4(l[0], l[1], l[2], l[3]);
+            for (int j = 0; j < 4 * NW; ++j)
+                if (t < T && j < nb) w[j >> 2] |= (uint32_t)__ldg(src + j) << (8 * (j & 3));
+            apply_b_row<KP>(gbh, gbl, w, sk, lane + 32 * rr, r);
         }
     }
 }
@@ -202,7 +238,9 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
     constexpr int OPB = NA * 16384;   // bytes per operand tile
     constexpr int S = apply_ring<SENDER, KP>();
     constexpr int SB = apply_stage_bytes<SENDER>();
-    constexpr int RB = kApplyStageTok * kApplyTile * 4;  // recon part of a stage
+    constexpr int STOK = apply_stage_tok<SENDER>();
+    constexpr int TPW = STOK / 2;                        // tokens per warp per stage
+    constexpr int RB = STOK * kApplyTile * 4;            // recon part of a stage
     extern __shared__ uint8_t dsm[];
     const uint32_t base = (smem_u32(dsm) + 1023u) & ~1023u;
     uint8_t *gb = dsm + (base - smem_u32(dsm));
@@ -258,13 +296,13 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
             bool ok = true;
             for (int it = 0; it < nt && ok; ++it) {
                 const int64_t t0 = tbeg + (int64_t)it * kApplyTile;
-                for (int64_t tb = t0; tb < t0 + kApplyTile && tb < tend; tb += kApplyStageTok) {
+                for (int64_t tb = t0; tb < t0 + kApplyTile && tb < tend; tb += STOK) {
                     const int slot = issued % S;
                     if (issued >= S && !mbar_wait(empty0 + 8u * slot, (uint32_t)((issued / S - 1) & 1))) {
                         ok = false;
                         break;
                     }
-                    const int rows = (int)((tend - tb < kApplyStageTok) ? tend - tb : kApplyStageTok);
+                    const int rows = (int)((tend - tb < STOK) ? tend - tb : STOK);
                     const uint32_t full = full0 + 8u * slot;
                     const uint32_t dst = ring + (uint32_t)(slot * SB);
                     mbar_expect_tx(full, (uint32_t)rows * (rbytes + (SENDER ? xbytes : 0u)));
@@ -359,7 +397,7 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
                 const int64_t t0 = tbeg + (int64_t)i * kApplyTile;
                 const uint32_t acc = tmem + tlane + (uint32_t)(128 * (i & 1));
                 const int64_t tw = (T - t0 < kApplyTile) ? T - t0 : kApplyTile;
-                const int ns = (int)((tw + kApplyStageTok - 1) / kApplyStageTok);
+                const int ns = (int)((tw + STOK - 1) / STOK);
                 for (int st = 0; st < ns; ++st, ++g) {
                     const int slot = g % S;
                     if (!__all_sync(kFullMask, mbar_wait(full0 + 8u * slot, (uint32_t)((g / S) & 1)))) {
@@ -367,14 +405,17 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
                         ok = false;
                         break;
                     }
-                    const int tl = st * kApplyStageTok + 8 * half;   // first token column of this warp
-                    float dv[8];
-                    tmem_ld8(acc + (uint32_t)tl, dv);
-                    const float *sr = reinterpret_cast<const float *>(gring + slot * SB) + 8 * half * kApplyTile;
-                    const uint16_t *sx = reinterpret_cast<const uint16_t *>(gring + slot * SB + RB) + 8 * half * kApplyTile;
+                    const int tl = st * STOK + TPW * half;   // first token column of this warp
+                    float dv[TPW];
+                    if (TPW == 16)
+                        tmem_ld16(acc + (uint32_t)tl, dv);
+                    else
+                        tmem_ld8(acc + (uint32_t)tl, dv);
+                    const float *sr = reinterpret_cast<const float *>(gring + slot * SB) + TPW * half * kApplyTile;
+                    const uint16_t *sx = reinterpret_cast<const uint16_t *>(gring + slot * SB + RB) + TPW * half * kApplyTile;
                     if (col_ok) {
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
+                        for (int j = 0; j < TPW; ++j) {
                             if (tl + j >= tw) break;
                             const float rv = sr[j * kApplyTile + cl];
                             const int64_t o = (t0 + tl + j) * C + c;

@@ -288,3 +288,28 @@ def test_apply_event_hook_times_the_apply_kernel_only():
     assert 0 < t_enc < t_all and 0 < t_dec < t_all
     # the encode's apply ends before the decode's begins
     assert ev[1].elapsed_time(ev[2]) >= 0
+
+
+@pytest.mark.parametrize("r", [32, 33])
+def test_decode_with_unaligned_codes_matches_aligned(r):
+    """Code arrays need only 1-byte alignment: a receiver given the same
+    payload at an odd address (and so reading it byte by byte) adds exactly
+    the same D as one reading it from an aligned copy."""
+    T, C = 700, 264
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r)
+    xs = W.trajectory(wl, 0, steps=2, device="cuda")
+    g = GpuLowrank(T, C, r, 2)
+    g.init(xs[0].clone())
+    g.step(xs[1].clone(), W.omega(wl, 0, 1, device="cuda"))
+    nb = (r + 1) // 2
+    odd_p = torch.zeros(T * nb + 32, dtype=torch.uint8, device="cuda")
+    odd_q = torch.zeros(C * nb + 32, dtype=torch.uint8, device="cuda")
+    odd_p[1:1 + T * nb] = g.pc[:T * nb]
+    odd_q[3:3 + C * nb] = g.qc[:C * nb]
+    ref = torch.zeros(T, C, dtype=torch.float32, device="cuda")
+    got = torch.zeros(T, C, dtype=torch.float32, device="cuda")
+    cf.cf_lowrank_decode(g.d, g.pc, g.ps, g.qc, g.qs, ref)
+    cf.cf_lowrank_decode(g.d, odd_p.data_ptr() + 1, g.ps, odd_q.data_ptr() + 3, g.qs, got)
+    torch.cuda.synchronize()
+    assert torch.equal(ref, got)
+    assert ref.abs().max() > 0
