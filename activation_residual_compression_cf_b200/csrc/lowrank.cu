@@ -56,6 +56,8 @@ Layout make_layout(int64_t T, int64_t C, int r) {
     L.splitsB = (int)((T + kChunkB - 1) / kChunkB);
     L.nGram = (int)((T + kGramTok - 1) / kGramTok);
     L.nGroups = (L.nGram + kGramGroup - 1) / kGramGroup;
+    L.nTileT = (int)((T + kTileRows - 1) / kTileRows);
+    L.nTileC = (int)((C + kTileRows - 1) / kTileRows);
     size_t off = 0;
     auto take = [&](size_t bytes) {
         size_t o = off;
@@ -64,6 +66,8 @@ Layout make_layout(int64_t T, int64_t C, int r) {
     };
     L.off_status = take(16);                          // status word, final ticket
     L.off_gt = take((size_t)L.nGroups * 4);           // group tickets
+    // partial Grams: per 32-token block (CUDA-core engine) or per 128-token
+    // tile (tensor-core engine); the former count is the larger
     L.off_gp = take((size_t)L.nGram * L.rp * L.rp * 8);
     L.off_gg = take((size_t)L.nGroups * L.rp * L.rp * 8);
     L.off_rmat = take((size_t)L.rp * L.rp * 4 + (size_t)L.rp * 4);
@@ -178,13 +182,13 @@ cf_status launch_project(const LrBatch &B, const Layout &L, int n, cudaStream_t 
     const int smem = cf::umma::StageGeom<BN>::kSmem;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return CF_ERR_CUDA;
-    dim3 grid((unsigned)((L.T + 127) / 128), (unsigned)L.splitsA, (unsigned)n);
+    dim3 grid((unsigned)L.nTileT, 1, (unsigned)n);
     k<<<grid, 128, smem, st>>>(mv, mq, B, L);
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 
 template <int BN>
-cf_status launch_backproject(const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
+cf_status launch_backproject(const LrBatch &B, const Layout &L, int n, bool last, cudaStream_t st) {
     CUtensorMap mv, mp;
     if (!make_map(&mv, B.ws + L.off_vb, L.C, L.T, L.C, n, B.ws_stride, 64) ||
         !make_map(&mp, B.ws + L.off_pt, L.Tp, L.rp, L.Tp, n, B.ws_stride, BN))
@@ -193,8 +197,8 @@ cf_status launch_backproject(const LrBatch &B, const Layout &L, int n, cudaStrea
     const int smem = cf::umma::StageGeom<BN>::kSmem;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return CF_ERR_CUDA;
-    dim3 grid((unsigned)((L.C + 127) / 128), (unsigned)L.splitsB, (unsigned)n);
-    k<<<grid, 128, smem, st>>>(mv, mp, B, L);
+    dim3 grid((unsigned)L.nTileC, 1, (unsigned)n);
+    k<<<grid, 128, smem, st>>>(mv, mp, B, L, last ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 
@@ -212,13 +216,13 @@ cf_status project(const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 
-cf_status backproject(const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
+cf_status backproject(const LrBatch &B, const Layout &L, int n, bool last, cudaStream_t st) {
     if (g_engine.load() == 0) {
         switch (L.rp) {
-            case 16: return launch_backproject<16>(B, L, n, st);
-            case 32: return launch_backproject<32>(B, L, n, st);
-            case 48: return launch_backproject<48>(B, L, n, st);
-            case 64: return launch_backproject<64>(B, L, n, st);
+            case 16: return launch_backproject<16>(B, L, n, last, st);
+            case 32: return launch_backproject<32>(B, L, n, last, st);
+            case 48: return launch_backproject<48>(B, L, n, last, st);
+            case 64: return launch_backproject<64>(B, L, n, last, st);
         }
     }
     cf::lr_backproject_simt<<<dim3((unsigned)((L.C + 63) / 64), (unsigned)L.splitsB, (unsigned)n), 256,
@@ -329,14 +333,22 @@ cf_status encode_impl(const cf_desc *d, const Layout &L, int n, const LrBatch &B
         cf::lr_omega_kernel<<<dim3((unsigned)((nq + 255) / 256), 1, (unsigned)n), 256, 0, st>>>(B, L);
         LR_LAUNCHED();
     }
+    // Tensor-core engine: each projection CTA accumulates its whole K range,
+    // so the projection also forms G and factors it (last tile of the
+    // buffer) and the back-projection writes Q's transpose and maxima: an
+    // iteration is three launches.  CUDA-core engine: split-K partials with
+    // separate Gram / Cholesky and Q-reduction kernels.
+    const bool fused = g_engine.load() == 0;
     for (int it = 0; it < d->iters; ++it) {
         const bool last = (it == d->iters - 1);
         LR_TRY(project(B, L, n, st));
-        cf::lr_gram_chol_kernel<<<dim3((unsigned)L.nGram, 1, (unsigned)n), 256, 0, st>>>(B, L);
-        LR_LAUNCHED();
+        if (!fused) {
+            cf::lr_gram_chol_kernel<<<dim3((unsigned)L.nGram, 1, (unsigned)n), 256, 0, st>>>(B, L);
+            LR_LAUNCHED();
+        }
         LR_TRY(orth(B, L, n, last, st));
-        LR_TRY(backproject(B, L, n, st));
-        LR_TRY(reduce_q(B, L, n, last, st));
+        LR_TRY(backproject(B, L, n, last, st));
+        if (!fused) LR_TRY(reduce_q(B, L, n, last, st));
     }
     // INT4 factors: quantise and pack against the column maxima.
     cf::lr_int4_pack_kernel<<<dim3((unsigned)((L.T * nb + 255) / 256), 1, (unsigned)n), 256, 0, st>>>(B, L, 0);

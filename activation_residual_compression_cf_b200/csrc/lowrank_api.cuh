@@ -19,6 +19,7 @@ constexpr int kGramGroup = 16;     // Gram partial blocks summed per first-level
 constexpr int kApplyTok = 32;      // D tile: tokens
 constexpr int kApplyCh = 256;      // D tile: channels
 constexpr int kApplyThreads = 256;
+constexpr int64_t kTileRows = 128;  // output rows per tcgen05 projection tile
 
 // Workspace layout (byte offsets, each region 256-byte aligned).  rp is
 // the rank padded to a multiple of 16 (MMA N granularity); Tp the token
@@ -28,8 +29,9 @@ struct Layout {
     int r, rp;
     int64_t Tp;
     int splitsA, splitsB, nGram, nGroups;
-    size_t off_status, off_gt, off_gp, off_gg, off_rmat, off_amax, off_vb, off_qt, off_yp, off_y, off_p, off_pt,
-        off_zp, off_q, total;
+    int nTileT, nTileC;  // 128-row tiles of the two projections
+    size_t off_status, off_gt, off_gp, off_gg, off_rmat, off_amax, off_vb, off_qt, off_yp, off_y,
+        off_p, off_pt, off_zp, off_q, total;
 };
 
 // Descriptor checks shared by cf_payload_bytes and the low-rank entry points.

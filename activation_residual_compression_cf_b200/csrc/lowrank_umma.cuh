@@ -1,10 +1,14 @@
 // lowrank_umma.cuh -- tcgen05 (5th-generation tensor core) kernels for the two
 // dense products of subspace iteration:
-//   project:     Yp[s] = Vb[tok block, channel split s] . Qt[:, split s]^T
-//                M = 128 tokens, N = rp, K = channels (K-major A and B)
-//   backproject: Zp[s] = Vb[token split s, ch block]^T . Pt[:, split s]^T
-//                M = 128 channels, N = rp, K = tokens (A is MN-major: V is
-//                stored token-major and the reduction runs over tokens)
+//   project:     Y[tok tile] = Vb[tok tile, :] . Qt^T
+//                M = 128 tokens, N = rp, K = all channels (K-major A and B)
+//   backproject: Q[ch block] = Vb[:, ch block]^T . Pt^T
+//                M = 128 channels, N = rp, K = all tokens (A is MN-major: V
+//                is stored token-major and the reduction runs over tokens)
+// Each CTA accumulates its whole K range in TMEM (no split-K), so its rows
+// are final when the MMAs end: the projection's tail forms the tile's
+// partial Gram and the buffer's last tile factors G; the back-projection's
+// tail writes the bf16 transpose and the column maxima.
 //
 // One CTA of 4 warps per output tile and K split:
 //   warp 0, one lane : TMA producer (cp.async.bulk.tensor, no multicast) into
@@ -25,6 +29,7 @@
 
 #include "cf.h"
 #include "lowrank_api.cuh"
+#include "lowrank_kernels.cuh"
 
 namespace cf {
 namespace umma {
@@ -299,8 +304,167 @@ __device__ __forceinline__ void gemm_tile(const CUtensorMap *mapA, const CUtenso
     }
 }
 
-// Yp[split][t][0..BN) of buffer blockIdx.z for the token block blockIdx.x and
-// channel split blockIdx.y.
+// Tail of the projection Y = Vb Q, run after a CTA has written the complete
+// Y rows of token tile `tile` (all channels in one accumulation): the
+// tile's fp64 partial Gram Y_tile^T Y_tile (upper triangle, rows in order);
+// the last tile of the buffer to finish (per-buffer ticket) sums the partial
+// Grams in tile order and factors G = R^T R.  Every sum runs in a fixed
+// order, so the result does not depend on which CTA finishes last.  (A
+// reduction whose order varied from run to run would be amplified by the
+// bf16 operand roundings of later iterations into visible differences.)
+// A pivot not above 1e-10 of its original diagonal entry marks the column
+// dead: its row of R and its inverse diagonal are zero (P gets a zero
+// column) and CF_ERR_NUMERIC is recorded.  Output: R (fp32 [rp][rp], upper)
+// and 1/diag(R) (fp32 [rp], 0 where dead).  The ticket is reset by its last
+// user.  The pipeline's shared memory is reused: every stage has been
+// consumed once the tile's product is done.
+template <int BN>
+__device__ __forceinline__ void project_tail(const cf_lowrank::LrBatch &B, const cf_lowrank::Layout &L,
+                                             int bz, int tile) {
+    extern __shared__ uint8_t dsmem[];
+    const uint32_t base = (smem_u32(dsmem) + 1023u) & ~1023u;
+    uint8_t *gbase = dsmem + (base - smem_u32(dsmem));
+    constexpr int LDY = BN + 1;
+    constexpr int kYsBytes = (128 * LDY * 4 + 255) & ~255;
+    static_assert(kYsBytes + BN * (BN + 1) * 8 <= kStages * StageGeom<BN>::kBytes, "tail scratch");
+    float *ys = reinterpret_cast<float *>(gbase);                 // [128][LDY] Y of the tile
+    double *A = reinterpret_cast<double *>(gbase + kYsBytes);     // [BN][BN + 1] G, then R
+    __shared__ double gdiag[64], invd[64];
+    __shared__ double rowbuf[2][33];
+    __shared__ int dead[64];
+    __shared__ int is_last;
+    const int tid = threadIdx.x;
+
+    // this thread's Y row (written by this thread in the epilogue)
+    const int64_t T = L.T;
+    const int64_t t = (int64_t)tile * 128 + tid;
+    if (t < T) {
+        const float4 *yr = reinterpret_cast<const float4 *>(B.at<float>(bz, L.off_y) + t * BN);
+#pragma unroll
+        for (int q = 0; q < BN / 4; ++q) {
+            const float4 v = yr[q];
+            ys[tid * LDY + 4 * q] = v.x;
+            ys[tid * LDY + 4 * q + 1] = v.y;
+            ys[tid * LDY + 4 * q + 2] = v.z;
+            ys[tid * LDY + 4 * q + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < BN; ++k) ys[tid * LDY + k] = 0.0f;
+    }
+    __syncthreads();
+
+    // the tile's partial Gram, rows in order (two interleaved fp64 sums)
+    double *gp = B.at<double>(bz, L.off_gp);
+    for (int e = tid; e < BN * BN; e += 128) {
+        const int i = e / BN, j = e - (e / BN) * BN;
+        if (i > j) continue;
+        double a0 = 0.0, a1 = 0.0;
+#pragma unroll 4
+        for (int u = 0; u < 128; u += 2) {
+            a0 = fma((double)ys[u * LDY + i], (double)ys[u * LDY + j], a0);
+            a1 = fma((double)ys[(u + 1) * LDY + i], (double)ys[(u + 1) * LDY + j], a1);
+        }
+        gp[(int64_t)tile * BN * BN + e] = a0 + a1;
+    }
+    __threadfence();
+    __syncthreads();
+    uint32_t *fin = B.at<uint32_t>(bz, L.off_status) + cf_lowrank::kTicketWord;
+    if (tid == 0) is_last = atomicAdd(fin, 1u) == (uint32_t)(L.nTileT - 1) ? 1 : 0;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+
+    // G = sum of the tiles' partial Grams in tile order (8 loads in flight)
+    const int ld = BN + 1, r = L.r, ntile = L.nTileT;
+    for (int e = tid; e < BN * BN; e += 128) {
+        const int i = e / BN, j = e - (e / BN) * BN;
+        if (i > j) continue;
+        double a[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+        int g = 0;
+        for (; g + 8 <= ntile; g += 8) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) a[u] += __ldcg(gp + (int64_t)(g + u) * BN * BN + e);
+        }
+        for (; g < ntile; ++g) a[0] += __ldcg(gp + (int64_t)g * BN * BN + e);
+        const double v = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+        A[i * ld + j] = v;
+        if (i == j) gdiag[i] = v;
+    }
+    __syncthreads();
+    if (BN <= 32) {
+        quad_cholesky(A, ld, r, gdiag, dead, invd, rowbuf);   // all 128 threads
+    } else if (tid < 32) {
+        warp_cholesky_smem(A, ld, r, gdiag, dead, invd);
+    }
+    __syncthreads();
+    float *rmat = B.at<float>(bz, L.off_rmat);
+    float *rinvd = rmat + BN * BN;
+    int nd = 0;
+    for (int e = tid; e < BN * BN; e += 128) {
+        const int i = e / BN, c = e - (e / BN) * BN;
+        rmat[e] = (i <= c && c < r) ? (float)A[i * ld + c] : 0.0f;
+    }
+    for (int j = tid; j < BN; j += 128) {
+        const bool live = j < r && !dead[j];
+        rinvd[j] = live ? (float)invd[j] : 0.0f;
+        nd += (j < r && dead[j]) ? 1 : 0;
+    }
+    if (nd) atomicCAS(B.at<int32_t>(bz, L.off_status) + cf_lowrank::kStatusWord, (int32_t)CF_OK,
+                      (int32_t)CF_ERR_NUMERIC);
+    if (tid == 0) *fin = 0u;
+}
+
+// Tail of the back-projection Q = Vb^T P for channel block `cblk`, run after
+// the CTA has written the block's complete Q rows (all tokens in one
+// accumulation): the bf16 transpose Qt [rp][C] for the next projection and,
+// on the last iteration, max |Q[:, k]| folded into the column maxima (float
+// bits, atomicMax).
+template <int BN>
+__device__ __forceinline__ void backproject_tail(const cf_lowrank::LrBatch &B, const cf_lowrank::Layout &L,
+                                                 int bz, int cblk, int want_amax) {
+    __shared__ float Wm[4][BN];
+    const int tid = threadIdx.x;
+    const int64_t C = L.C;
+    const int64_t c = (int64_t)cblk * 128 + tid;
+    float v[BN];
+    if (c < C) {
+        const float4 *qr = reinterpret_cast<const float4 *>(B.at<float>(bz, L.off_q) + c * BN);
+#pragma unroll
+        for (int q = 0; q < BN / 4; ++q) {
+            const float4 z = qr[q];
+            v[4 * q] = z.x;
+            v[4 * q + 1] = z.y;
+            v[4 * q + 2] = z.z;
+            v[4 * q + 3] = z.w;
+        }
+        bf16 *qt = B.at<bf16>(bz, L.off_qt);
+#pragma unroll
+        for (int k = 0; k < BN; ++k) qt[(int64_t)k * C + c] = __float2bfloat16_rn(v[k]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < BN; ++k) v[k] = 0.0f;
+    }
+    if (want_amax) {
+        const int warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+        for (int k = 0; k < BN; ++k) {
+            float m = fabsf(v[k]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) Wm[warp][k] = m;
+        }
+        __syncthreads();
+        uint32_t *amax = B.at<uint32_t>(bz, L.off_amax) + BN;
+        for (int k = tid; k < BN; k += 128) {
+            const float m = fmaxf(fmaxf(Wm[0][k], Wm[1][k]), fmaxf(Wm[2][k], Wm[3][k]));
+            atomicMax(amax + k, __float_as_uint(m));
+        }
+    }
+}
+
+// Y[t][0..BN) of buffer blockIdx.z for the token tile blockIdx.x, over all
+// channels, then the tile's share of G and R (above).
 template <int BN>
 __global__ void __launch_bounds__(128, 1)
 project_kernel(const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapQt,
@@ -308,29 +472,25 @@ project_kernel(const __grid_constant__ CUtensorMap mapV, const __grid_constant__
     const int bz = blockIdx.z;
     if (B.at<int32_t>(bz, L.off_status)[cf_lowrank::kSkipWord]) return;
     const int32_t t0 = blockIdx.x * 128;
-    const int64_t kb = (int64_t)blockIdx.y * cf_lowrank::kChunkA;
-    const int64_t ke = (kb + cf_lowrank::kChunkA < L.C) ? kb + cf_lowrank::kChunkA : L.C;
-    const int nkb = (int)((ke - kb + kBK - 1) / kBK);
-    float *yp = B.at<float>(bz, L.off_yp) + (int64_t)blockIdx.y * L.T * BN;
-    gemm_tile<BN, false>(&mapV, &mapQt, t0, (int32_t)kb, nkb, bz, yp, L.T,
+    const int nkb = (int)((L.C + kBK - 1) / kBK);
+    gemm_tile<BN, false>(&mapV, &mapQt, t0, 0, nkb, bz, B.at<float>(bz, L.off_y), L.T,
                          B.at<int32_t>(bz, L.off_status) + cf_lowrank::kStatusWord);
+    project_tail<BN>(B, L, bz, blockIdx.x);
 }
 
-// Zp[split][c][0..BN) of buffer blockIdx.z for the channel block blockIdx.x
-// and token split blockIdx.y.
+// Q[c][0..BN) of buffer blockIdx.z for the channel block blockIdx.x, over
+// all tokens, then the block's Qt and column maxima (above).
 template <int BN>
 __global__ void __launch_bounds__(128, 1)
 backproject_kernel(const __grid_constant__ CUtensorMap mapVt, const __grid_constant__ CUtensorMap mapPt,
-                   const cf_lowrank::LrBatch B, const cf_lowrank::Layout L) {
+                   const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int want_amax) {
     const int bz = blockIdx.z;
     if (B.at<int32_t>(bz, L.off_status)[cf_lowrank::kSkipWord]) return;
     const int32_t c0 = blockIdx.x * 128;
-    const int64_t kb = (int64_t)blockIdx.y * cf_lowrank::kChunkB;
-    const int64_t ke = (kb + cf_lowrank::kChunkB < L.T) ? kb + cf_lowrank::kChunkB : L.T;
-    const int nkb = (int)((ke - kb + kBK - 1) / kBK);
-    float *zp = B.at<float>(bz, L.off_zp) + (int64_t)blockIdx.y * L.C * BN;
-    gemm_tile<BN, true>(&mapVt, &mapPt, c0, (int32_t)kb, nkb, bz, zp, L.C,
+    const int nkb = (int)((L.T + kBK - 1) / kBK);
+    gemm_tile<BN, true>(&mapVt, &mapPt, c0, 0, nkb, bz, B.at<float>(bz, L.off_q), L.C,
                         B.at<int32_t>(bz, L.off_status) + cf_lowrank::kStatusWord);
+    backproject_tail<BN>(B, L, bz, blockIdx.x, want_amax);
 }
 
 }  // namespace umma
