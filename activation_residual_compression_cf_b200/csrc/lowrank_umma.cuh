@@ -324,7 +324,9 @@ __device__ __forceinline__ void project_tail(const cf_lowrank::LrBatch &B, const
     extern __shared__ uint8_t dsmem[];
     const uint32_t base = (smem_u32(dsmem) + 1023u) & ~1023u;
     uint8_t *gbase = dsmem + (base - smem_u32(dsmem));
-    constexpr int LDY = BN + 1;
+    // Y tile in shared memory, fp32, row pitch BN + 8 words so that the
+    // 4 x 8 fragment reads below fall in 32 distinct banks
+    constexpr int LDY = BN + 8;
     constexpr int kYsBytes = (128 * LDY * 4 + 255) & ~255;
     static_assert(kYsBytes + BN * (BN + 1) * 8 <= kStages * StageGeom<BN>::kBytes, "tail scratch");
     float *ys = reinterpret_cast<float *>(gbase);                 // [128][LDY] Y of the tile
@@ -341,32 +343,66 @@ __device__ __forceinline__ void project_tail(const cf_lowrank::LrBatch &B, const
     if (t < T) {
         const float4 *yr = reinterpret_cast<const float4 *>(B.at<float>(bz, L.off_y) + t * BN);
 #pragma unroll
-        for (int q = 0; q < BN / 4; ++q) {
-            const float4 v = yr[q];
-            ys[tid * LDY + 4 * q] = v.x;
-            ys[tid * LDY + 4 * q + 1] = v.y;
-            ys[tid * LDY + 4 * q + 2] = v.z;
-            ys[tid * LDY + 4 * q + 3] = v.w;
-        }
+        for (int q = 0; q < BN / 4; ++q)
+            *reinterpret_cast<float4 *>(ys + tid * LDY + 4 * q) = yr[q];
     } else {
 #pragma unroll
-        for (int k = 0; k < BN; ++k) ys[tid * LDY + k] = 0.0f;
+        for (int q = 0; q < BN / 4; ++q)
+            *reinterpret_cast<float4 *>(ys + tid * LDY + 4 * q) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
 
-    // the tile's partial Gram, rows in order (two interleaved fp64 sums)
-    double *gp = B.at<double>(bz, L.off_gp);
-    for (int e = tid; e < BN * BN; e += 128) {
-        const int i = e / BN, j = e - (e / BN) * BN;
-        if (i > j) continue;
-        double a0 = 0.0, a1 = 0.0;
-#pragma unroll 4
-        for (int u = 0; u < 128; u += 2) {
-            a0 = fma((double)ys[u * LDY + i], (double)ys[u * LDY + j], a0);
-            a1 = fma((double)ys[(u + 1) * LDY + i], (double)ys[(u + 1) * LDY + j], a1);
+    // The tile's partial Gram Y^T Y on the fp64 tensor path (mma.sync
+    // m8n8k4 f64; tcgen05 has no fp64 kind): 8 x 8 output blocks (I, J),
+    // I <= J, dealt to the 4 warps round robin; each warp runs its blocks'
+    // accumulators side by side over the 128 rows, 4 rows per step.  The
+    // fp32 values are exact in fp64, so every product is exact and only the
+    // fp64 sums round.  A fragment: A[i][k] = Y[k][8I + i] (i = lane / 4,
+    // k = lane % 4); B fragment: B[k][j] = Y[k][8J + j] (k = lane % 4,
+    // j = lane / 4); D: row lane / 4, columns 2 (lane % 4) + {0, 1}.
+    {
+        constexpr int NB = BN / 8;
+        constexpr int NU = NB * (NB + 1) / 2;
+        constexpr int MT = (NU + 3) / 4;               // blocks per warp, at most
+        const int warp = tid >> 5, lane = tid & 31;
+        const int fr = lane >> 2, fk = lane & 3;
+        int bi[MT], bj[MT];
+        double acc[MT][2];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            int u = warp + 4 * m, I = 0;
+            while (u >= NB - I && I < NB) { u -= NB - I; ++I; }  // u-th upper block, row-major
+            bi[m] = I < NB ? I : -1;
+            bj[m] = I < NB ? I + u : -1;
+            acc[m][0] = acc[m][1] = 0.0;
         }
-        gp[(int64_t)tile * BN * BN + e] = a0 + a1;
+#pragma unroll 2
+        for (int k0 = 0; k0 < 128; k0 += 4) {
+            const float *row = ys + (k0 + fk) * LDY;
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                if (bi[m] < 0) continue;
+                const double a = (double)row[8 * bi[m] + fr];
+                const double b = (double)row[8 * bj[m] + fr];
+                asm volatile(
+                    "mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                    : "+d"(acc[m][0]), "+d"(acc[m][1])
+                    : "d"(a), "d"(b));
+            }
+        }
+        double *gpt = B.at<double>(bz, L.off_gp) + (int64_t)tile * BN * BN;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            if (bi[m] < 0) continue;
+            const int i = 8 * bi[m] + fr;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int j = 8 * bj[m] + 2 * fk + c;
+                if (i <= j) gpt[i * BN + j] = acc[m][c];
+            }
+        }
     }
+    double *gp = B.at<double>(bz, L.off_gp);
     __threadfence();
     __syncthreads();
     uint32_t *fin = B.at<uint32_t>(bz, L.off_status) + cf_lowrank::kTicketWord;
