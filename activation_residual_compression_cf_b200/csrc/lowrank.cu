@@ -383,7 +383,7 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
     LR_TRY(check_ptr(x));
     LR_TRY(check_ptr(recon_s));
     LR_TRY(check_ptr(err));
-    LR_TRY(check_ptr(omega, 4));
+    if (omega) LR_TRY(check_ptr(omega, 4));   // NULL: warm start
     LR_TRY(check_ptr(p_codes, 1));
     LR_TRY(check_ptr(p_scales, 4));
     LR_TRY(check_ptr(q_codes, 1));

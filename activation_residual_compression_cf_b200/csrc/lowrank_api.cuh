@@ -39,8 +39,12 @@ cf_status check_desc(const cf_desc *d);
 Layout make_layout(int64_t T, int64_t C, int r);
 
 // Per-buffer status region (off_status): [0] status word, [1] final Gram
-// ticket, [2] skip flag (set when the buffer's pointers failed validation).
-constexpr int kStatusWord = 0, kTicketWord = 1, kSkipWord = 2;
+// ticket, [2] skip flag (set when the buffer's pointers failed validation),
+// all cleared at the start of every encode; [4] and [5] the warm-start tag,
+// kept across encodes: kWarmMagic | r and C once an encode has left a
+// usable Q (its bf16 copy Qt) in the workspace.
+constexpr int kStatusWord = 0, kTicketWord = 1, kSkipWord = 2, kWarmTag = 4, kWarmC = 5;
+constexpr uint32_t kWarmMagic = 0x51570000u;
 
 // One buffer's caller pointers (sender fields; the receiver uses the payload
 // and recon).

@@ -29,7 +29,9 @@ __device__ __forceinline__ bool lr_skipped(const LrBatch &B, const Layout &L, in
 // Per-buffer set-up of a low-rank encode: zero the status word, the Gram
 // tickets and the column maxima of this buffer's workspace slice, then check
 // its pointers (x, recon, err: 16-byte aligned; omega, scales: 4-byte; all
-// non-null) and mark the buffer skipped with the error in its status word.
+// non-null except omega, whose null means a warm start and needs the warm
+// tag of an earlier encode of this shape) and mark the buffer skipped with
+// the error in its status word.
 __global__ void lr_prep_kernel(const LrBatch B, const Layout L) {
     const int b = blockIdx.x;
     int32_t *st = B.at<int32_t>(b, L.off_status);
@@ -42,8 +44,13 @@ __global__ void lr_prep_kernel(const LrBatch B, const Layout L) {
     if (threadIdx.x == 0) {
         const LrPtrs p = B.get(b);
         int code = CF_OK;
-        if (!p.x || !p.recon || !p.err || !p.omega || !p.pc_out || !p.ps_out || !p.qc_out || !p.qs_out)
+        const uint32_t *wt = reinterpret_cast<const uint32_t *>(st);
+        const bool warm_ok = wt[cf_lowrank::kWarmTag] == (cf_lowrank::kWarmMagic | (uint32_t)L.r) &&
+                             wt[cf_lowrank::kWarmC] == (uint32_t)L.C;
+        if (!p.x || !p.recon || !p.err || !p.pc_out || !p.ps_out || !p.qc_out || !p.qs_out)
             code = CF_ERR_INVALID_ARG;
+        else if (!p.omega && !warm_ok)
+            code = CF_ERR_INVALID_ARG;   // warm start without an earlier encode
         else if (misaligned16(p.x) || misaligned16(p.recon) || misaligned16(p.err) ||
                  (reinterpret_cast<uintptr_t>(p.omega) & 3u) || (reinterpret_cast<uintptr_t>(p.ps_out) & 3u) ||
                  (reinterpret_cast<uintptr_t>(p.qs_out) & 3u))
@@ -87,6 +94,7 @@ __global__ void lr_omega_kernel(const LrBatch B, const Layout L) {
     const int bz = blockIdx.z;
     if (lr_skipped(B, L, bz)) return;
     const float *omega = B.get(bz).omega;
+    if (!omega) return;   // warm start: Qt still holds the previous encode's Q
     bf16 *qt = B.at<bf16>(bz, L.off_qt);
     const int64_t C = L.C;
     const int r = L.r, rp = L.rp;
@@ -638,6 +646,13 @@ __global__ void lr_int4_pack_kernel(const LrBatch B, const Layout L, int which) 
     const int nb = (r + 1) / 2;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < r) scales[i] = __fdiv_rn(__uint_as_float(amax[i]), 7.0f);
+    if (which == 1 && i == 0) {
+        // the workspace now holds this encode's final Q (Qt): a later
+        // encode of this shape may start from it
+        uint32_t *wt = B.at<uint32_t>(bz, L.off_status);
+        wt[cf_lowrank::kWarmTag] = cf_lowrank::kWarmMagic | (uint32_t)r;
+        wt[cf_lowrank::kWarmC] = (uint32_t)L.C;
+    }
     if (i >= rows * nb) return;
     const int64_t row = i / nb;
     const int b = (int)(i - row * nb);

@@ -61,6 +61,7 @@ extern "C" cf_status cf_lowrank_encode_noalloc(const cf_desc *d, const uint16_t 
                                                uint8_t *q_codes, float *q_scales, void *stream) {
     const cf_status ds = cf_lowrank::check_desc(d);
     if (ds != CF_OK) return ds;
+    if (!omega) return CF_ERR_INVALID_ARG;
     const int64_t need = cf_lowrank_workspace_bytes(d);
     if (need <= 0 || (uint64_t)need > (uint64_t)CF_LOWRANK_NOALLOC_SCRATCH_BYTES)
         return CF_ERR_WORKSPACE;

@@ -56,6 +56,11 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--iters", type=int, default=0,
+                    help="low-rank: subspace iterations (default: the workload's)")
+    ap.add_argument("--rank", type=int, default=0, help="low-rank: rank (default: the workload's)")
+    ap.add_argument("--warm", action="store_true",
+                    help="low-rank: warm start every encode after the first from the previous Q")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="budget of the oracle timing sample")
     ap.add_argument("--buffers", type=int, default=0,
@@ -387,6 +392,10 @@ def run_lowrank(args, world, rank, local):
     wl = W.WORKLOADS[args.workload]
     if args.buffers:
         wl = W.replace(wl, buffers=args.buffers)
+    if args.iters:
+        wl = W.replace(wl, iters=args.iters)
+    if args.rank:
+        wl = W.replace(wl, rank=args.rank)
     n, T, C, r, it = wl.buffers, wl.tokens, wl.channels, wl.rank, wl.iters
     d = cf.desc(T, C, 0, r, it)
     step_bytes = n * T * C * 2
@@ -419,11 +428,15 @@ def run_lowrank(args, world, rank, local):
     # one batched call per step for all buffers (encode) and one for decode
     encs = [cf.lowrank_buffer_array([(X16[s, b], recon_s[b], err[b], OM[s, b], pc[b], ps[b],
                                       qc[b], qs[b]) for b in range(n)], dev) for s in range(S)]
+    # warm start: omega NULL, the iteration starts from the previous Q
+    warms = [cf.lowrank_buffer_array([(X16[s, b], recon_s[b], err[b], None, pc[b], ps[b],
+                                       qc[b], qs[b]) for b in range(n)], dev) for s in range(S)]
     decs = cf.lowrank_dec_buffer_array([(pc[b], ps[b], qc[b], qs[b], recon_r[b]) for b in range(n)],
                                        dev)
 
     def enc(i):
-        cf.cf_lowrank_encode_batched(d, n, encs[1 + i % (S - 1)], ws, stream=stream)
+        src = warms if (args.warm and i > 0) else encs
+        cf.cf_lowrank_encode_batched(d, n, src[1 + i % (S - 1)], ws, stream=stream)
 
     def dec():
         cf.cf_lowrank_decode_batched(d, n, decs, stream=stream)
@@ -501,7 +514,8 @@ def run_lowrank(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 in, fp32 state, bf16 tensor products", "data": "synthetic",
         "config": {"workload": args.workload, "tokens": T, "channels": C, "buffers": n,
-                   "rank": r, "iters": it, "mode": "low-rank INT4 + EF",
+                   "rank": r, "iters": it,
+                   "mode": "low-rank INT4 + EF" + (", warm start" if args.warm else ""),
                    "parallelism": f"replicas x{world}", "l2": "inputs larger than L2",
                    "launches_per_step": launches_per_step},
         "roofline": {"bound": "hbm",

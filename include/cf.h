@@ -191,7 +191,13 @@ int64_t cf_lowrank_factor_bytes(int64_t rows, int32_t rank);
  * scales 4 bytes; the code arrays 1 byte.
  * x: bf16 [T][C]; recon_s: fp32 [T][C] updated;
  * err: fp32 [T][C] written; omega: fp32 [C][r] Gaussian start block chosen
- * by the caller; p_codes: [T][ceil(r/2)] bytes, p_scales: fp32 [r];
+ * by the caller, or NULL for a warm start ("Builds on": PowerSGD reuses the
+ * previous step's factor as the next start block): the iteration then starts
+ * from the Q that the previous encode left in this workspace, rounded to
+ * bf16 as every Q operand is.  A warm start needs an earlier encode of the
+ * same shape and rank on the same workspace (slice); without one the buffer
+ * is skipped and CF_ERR_INVALID_ARG is recorded in its status word.
+ * p_codes: [T][ceil(r/2)] bytes, p_scales: fp32 [r];
  * q_codes: [C][ceil(r/2)] bytes, q_scales: fp32 [r] (all written);
  * workspace: device, >= cf_lowrank_workspace_bytes(d) bytes, 256-byte
  * aligned, contents need not be initialised.  If the fp64 Gram matrix of an
@@ -211,7 +217,7 @@ typedef struct cf_lowrank_buffer {
     const uint16_t *x;       /* bf16 [T][C]                                  */
     float *recon_s;          /* fp32 [T][C], updated                         */
     float *err;              /* fp32 [T][C], written                         */
-    const float *omega;      /* fp32 [C][r], subspace-iteration start        */
+    const float *omega;      /* fp32 [C][r] start block, or NULL: warm start */
     uint8_t *p_codes;        /* [T][ceil(r/2)], written                      */
     float *p_scales;         /* fp32 [r], written                            */
     uint8_t *q_codes;        /* [C][ceil(r/2)], written                      */
@@ -282,7 +288,9 @@ cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes,
  *    Calls whose work overlaps on the GPU -- different streams without
  *    ordering between them -- race on the array and corrupt each other.
  *  - The status word is in the array as well: cf_lowrank_status cannot
- *    reach it; CF_ERR_NUMERIC cases still yield a valid, lower-rank D. */
+ *    reach it; CF_ERR_NUMERIC cases still yield a valid, lower-rank D.
+ *  - omega must not be NULL (a warm start would read whichever buffer the
+ *    shared array saw last): CF_ERR_INVALID_ARG. */
 cf_status cf_lowrank_encode_noalloc(const cf_desc *d, const uint16_t *x, float *recon_s,
                                     float *err, const float *omega, uint8_t *p_codes,
                                     float *p_scales, uint8_t *q_codes, float *q_scales,

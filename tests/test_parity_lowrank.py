@@ -63,15 +63,22 @@ def _check_codes(packed, scales, r):
     assert not np.any(q[:, ~live])
 
 
-def _run(wl, steps, buffer=0, check_frob=True):
+def _run(wl, steps, buffer=0, check_frob=True, warm=False):
+    """Teacher-forced parity over a trajectory.  warm=True: from the second
+    compressed step on, the GPU starts from the Q its previous encode left
+    in the workspace (omega NULL) and the oracle from its own previous Q."""
     T, C, r, it = wl.tokens, wl.channels, wl.rank, wl.iters
     xs = W.trajectory(wl, buffer, steps=steps, device="cuda")
     g = GpuLowrank(T, C, r, it)
     g.init(xs[0].clone())
     errs = []
+    q_prev = None
     for s in range(1, steps):
         x = xs[s].clone()
         om = W.omega(wl, buffer, s, device="cuda")
+        om_ora = om.cpu().numpy()
+        if warm and q_prev is not None:
+            om, om_ora = None, q_prev
         recon_before = g.recon_s.cpu().numpy()
         g.step(x, om)
         torch.cuda.synchronize()
@@ -94,7 +101,8 @@ def _run(wl, steps, buffer=0, check_frob=True):
         assert np.max(np.abs(d_pay - d_gpu)) <= tol
         # oracle on the same input
         ro = recon_before.copy()
-        out = L.lowrank_encode(xb, ro, om.cpu().numpy(), it)
+        out = L.lowrank_encode(xb, ro, om_ora, it)
+        q_prev = out["Q"]
         e_gpu, e_ora = _rel_err(v, d_pay), _rel_err(out["V"], out["D"])
         errs.append((e_gpu, e_ora))
         if check_frob:
@@ -313,3 +321,71 @@ def test_decode_with_unaligned_codes_matches_aligned(r):
     torch.cuda.synchronize()
     assert torch.equal(ref, got)
     assert ref.abs().max() > 0
+
+
+def test_warm_start_trajectory():
+    """omega NULL after the first compressed step: the iteration starts from
+    the previous encode's Q (PowerSGD-style warm start); each step stays
+    within the parity bar of the oracle started from its own previous Q."""
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=512, channels=384, iters=1)
+    errs = _run(wl, steps=6, warm=True)
+    assert len(errs) == 5
+
+
+def test_warm_start_without_earlier_encode_is_refused():
+    """A warm start on a workspace that never held this shape's Q skips the
+    buffer (state untouched) and records CF_ERR_INVALID_ARG."""
+    T, C, r = 256, 128, 8
+    g = GpuLowrank(T, C, r, 2)
+    g.ws.zero_()
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r)
+    xs = W.trajectory(wl, 0, steps=2, device="cuda")
+    g.init(xs[0].clone())
+    before = g.recon_s.clone()
+    g.step(xs[1].clone(), None)
+    torch.cuda.synchronize()
+    assert cf.cf_lowrank_status(g.ws) == 1
+    assert torch.equal(g.recon_s, before)
+    # after one cold encode the same workspace accepts a warm start
+    g.step(xs[1].clone(), W.omega(wl, 0, 1, device="cuda"))
+    assert cf.cf_lowrank_status(g.ws) == 0
+    g.step(xs[1].clone(), None)
+    assert cf.cf_lowrank_status(g.ws) == 0
+    # another rank on the same workspace does not match the tag
+    d2 = cf.desc(T, C, 0, r - 1, 2)
+    before = g.recon_s.clone()
+    cf.cf_lowrank_encode(d2, xs[1].clone().view(torch.int16), g.recon_s, g.err, None, g.pc, g.ps,
+                         g.qc, g.qs, g.ws)
+    assert cf.cf_lowrank_status(g.ws) == 1
+    assert torch.equal(g.recon_s, before)
+
+
+def test_warm_start_batched_equals_single():
+    """Warm-started batched encodes compute exactly what warm-started single
+    encodes do, buffer by buffer."""
+    T, C, r, n = 300, 136, 16, 3
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r)
+    d = cf.desc(T, C, 0, r, 1)
+    wsb = cf.cf_lowrank_workspace_bytes(d)
+    xs = [W.trajectory(wl, b, steps=3, device="cuda") for b in range(n)]
+    single = [GpuLowrank(T, C, r, 1) for _ in range(n)]
+    batch = [GpuLowrank(T, C, r, 1) for _ in range(n)]
+    ws = torch.empty(n * wsb, dtype=torch.uint8, device="cuda")
+    for b in range(n):
+        for g in (single[b], batch[b]):
+            g.init(xs[b][0].clone())
+    for step in (1, 2):
+        xb = [xs[b][step].clone() for b in range(n)]
+        oms = [W.omega(wl, b, step, device="cuda") if step == 1 else None for b in range(n)]
+        for b in range(n):
+            single[b].step(xb[b], oms[b])
+        enc = cf.lowrank_buffer_array([(xb[b].view(torch.int16), batch[b].recon_s, batch[b].err,
+                                        oms[b], batch[b].pc, batch[b].ps, batch[b].qc, batch[b].qs)
+                                       for b in range(n)], "cuda")
+        cf.cf_lowrank_encode_batched(d, n, enc, ws)
+        torch.cuda.synchronize()
+        for b in range(n):
+            assert cf.cf_lowrank_status(ws[b * wsb:]) == 0
+            assert cf.cf_lowrank_status(single[b].ws) == 0
+            for k in ("recon_s", "err", "ps", "qs"):
+                assert torch.equal(getattr(batch[b], k), getattr(single[b], k)), (step, b, k)
