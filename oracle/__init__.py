@@ -36,6 +36,8 @@ def _load():
         lib.orc_state_init.restype = None
         lib.orc_encode.argtypes = [i64, i64, i32, vp, vp, vp, vp, vp, vp]
         lib.orc_encode.restype = ctypes.c_int
+        lib.orc_encode_delta.argtypes = [i64, i64, i32, vp, vp, vp, vp, vp, vp]
+        lib.orc_encode_delta.restype = ctypes.c_int
         lib.orc_decode.argtypes = [i64, i64, i32, vp, vp, vp]
         lib.orc_decode.restype = ctypes.c_int
         lib.orc_decode_emit.argtypes = [i64, i64, i32, vp, vp, vp, vp]
@@ -87,6 +89,25 @@ def encode(x_bits: np.ndarray, recon_s: np.ndarray, bits: int):
     if rc != 0:
         raise ValueError(f"oracle encode: unsupported bits={bits}")
     return codes, scales, err
+
+
+def encode_delta(x_bits: np.ndarray, xprev_bits: np.ndarray, err: np.ndarray, bits: int):
+    """Delta-state sender step: v = ((float)x - (float)x_prev) + err, then
+    as encode without the mirror; ``err`` is updated in place.
+    Returns (codes uint32 [T, W], scales float32 [T])."""
+    T, C = x_bits.shape
+    _check(x_bits, np.uint16, (T, C), "x")
+    _check(xprev_bits, np.uint16, (T, C), "x_prev")
+    _check(err, np.float32, (T, C), "err")
+    W = words_per_row(C, bits) if bits in (1, 2) else 0
+    codes = np.empty((T, W), np.uint32)
+    scales = np.empty((T,), np.float32)
+    scratch = np.empty((max(C, 1),), np.float32)
+    rc = _load().orc_encode_delta(T, C, bits, _ptr(x_bits), _ptr(xprev_bits), _ptr(err),
+                                  _ptr(codes), _ptr(scales), _ptr(scratch))
+    if rc != 0:
+        raise ValueError(f"oracle encode: unsupported bits={bits}")
+    return codes, scales
 
 
 def decode(codes: np.ndarray, scales: np.ndarray, recon_r: np.ndarray, bits: int):

@@ -78,6 +78,46 @@ void orc_state_init(int64_t T, int64_t C, const uint16_t *x0, float *recon,
     }
 }
 
+/* Steps 2-6 for one token row: scale, codes, error feedback, mirror update
+ * (when rr is not NULL) and packing, from the row's residual v. */
+static void quantize_row(int64_t C, int32_t bits, const float *v, float *er, float *rr,
+                         uint32_t *cw, int64_t W, float *scale_out) {
+    /* 2. per-token scale */
+    float scale;
+    if (bits == 1) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < C; ++c) acc += fabs((double)v[c]);
+        float sum32 = (float)acc;
+        scale = (C > 0) ? sum32 / (float)C : 0.0f;
+    } else {
+        float a = 0.0f;
+        for (int64_t c = 0; c < C; ++c) {
+            float m = fabsf(v[c]);
+            if (m > a) a = m;
+        }
+        scale = a;
+    }
+    *scale_out = scale;
+
+    /* 3-6. quantise, error feedback, mirror update, pack */
+    for (int64_t w = 0; w < W; ++w) cw[w] = 0u;
+    const float half = 0.5f * scale;
+    for (int64_t c = 0; c < C; ++c) {
+        uint32_t code;
+        if (bits == 1) {
+            code = (v[c] >= 0.0f) ? 1u : 0u;
+        } else {
+            code = (uint32_t)(v[c] >= -half) + (uint32_t)(v[c] >= 0.0f) +
+                   (uint32_t)(v[c] >= half);
+        }
+        float d = dequant(bits, code, scale);
+        er[c] = v[c] - d;
+        if (rr) rr[c] = rr[c] + d;
+        int64_t bitpos = c * (int64_t)bits;
+        cw[bitpos / 32] |= code << (bitpos % 32);
+    }
+}
+
 /* One compressed step of the sender for T token rows.  Returns 0, or -1 for
  * an unsupported bit width.  v_scratch must hold C floats. */
 int orc_encode(int64_t T, int64_t C, int32_t bits, const uint16_t *x,
@@ -88,47 +128,36 @@ int orc_encode(int64_t T, int64_t C, int32_t bits, const uint16_t *x,
     for (int64_t t = 0; t < T; ++t) {
         const uint16_t *xr = x + t * C;
         float *rr = recon_s + t * C;
-        float *er = err + t * C;
-        uint32_t *cw = codes + t * W;
         float *v = v_scratch;
-
         /* 1. residual against the sender's copy of the receiver state */
         for (int64_t c = 0; c < C; ++c) v[c] = bf16_bits_to_float(xr[c]) - rr[c];
+        quantize_row(C, bits, v, err + t * C, rr, codes + t * W, W, scales + t);
+    }
+    return 0;
+}
 
-        /* 2. per-token scale */
-        float scale;
-        if (bits == 1) {
-            double acc = 0.0;
-            for (int64_t c = 0; c < C; ++c) acc += fabs((double)v[c]);
-            float sum32 = (float)acc;
-            scale = (C > 0) ? sum32 / (float)C : 0.0f;
-        } else {
-            float a = 0.0f;
-            for (int64_t c = 0; c < C; ++c) {
-                float m = fabsf(v[c]);
-                if (m > a) a = m;
-            }
-            scale = a;
-        }
-        scales[t] = scale;
-
-        /* 3-6. quantise, error feedback, mirror update, pack */
-        for (int64_t w = 0; w < W; ++w) cw[w] = 0u;
-        const float half = 0.5f * scale;
+/* The same sender with its state kept as the previous activation x_prev
+ * and the error buffer err (read, then overwritten) instead of a
+ * reconstruction copy:
+ *   1'. v_c = ((float)x_t[c] - (float)x_prev[c]) + err[c]    two roundings
+ * then steps 2-6 as above, without the mirror update.  In exact arithmetic
+ * v equals step 1's residual, because recon_s + err == x after every step
+ * (the "Approach" section's error feedback, kept in another form). */
+int orc_encode_delta(int64_t T, int64_t C, int32_t bits, const uint16_t *x,
+                     const uint16_t *x_prev, float *err, uint32_t *codes, float *scales,
+                     float *v_scratch) {
+    if (bits != 1 && bits != 2) return -1;
+    const int64_t W = orc_words_per_row(C, bits);
+    for (int64_t t = 0; t < T; ++t) {
+        const uint16_t *xr = x + t * C;
+        const uint16_t *pr = x_prev + t * C;
+        float *er = err + t * C;
+        float *v = v_scratch;
         for (int64_t c = 0; c < C; ++c) {
-            uint32_t code;
-            if (bits == 1) {
-                code = (v[c] >= 0.0f) ? 1u : 0u;
-            } else {
-                code = (uint32_t)(v[c] >= -half) + (uint32_t)(v[c] >= 0.0f) +
-                       (uint32_t)(v[c] >= half);
-            }
-            float d = dequant(bits, code, scale);
-            er[c] = v[c] - d;
-            rr[c] = rr[c] + d;
-            int64_t bitpos = c * (int64_t)bits;
-            cw[bitpos / 32] |= code << (bitpos % 32);
+            float d = bf16_bits_to_float(xr[c]) - bf16_bits_to_float(pr[c]);
+            v[c] = d + er[c];
         }
+        quantize_row(C, bits, v, er, NULL, codes + t * W, W, scales + t);
     }
     return 0;
 }

@@ -232,3 +232,54 @@ def test_decode_emit_is_decode_then_bf16():
     assert np.array_equal(recon_r, recon_s)
     ref = torch.from_numpy(recon_r).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(out, ref)
+
+
+@pytest.mark.parametrize("name", ["tiny", "flux_sp"])
+def test_delta_state_first_step_equals_standard_sender(name):
+    """At the first compressed step after the warmup (err = 0, x_prev = x_0
+    = recon_s) the delta-state residual ((x - x_prev) + 0) is the standard
+    residual x - recon_s rounded once: codes, scales and err are identical."""
+    kw = {} if name == "tiny" else dict(tokens=48, buffers=1)
+    wl, xs = _traj(name, steps=2, **kw)
+    recon_s, err0 = oracle.state_init(xs[0])
+    c_std, s_std, e_std = oracle.encode(xs[1], recon_s, wl.bits)
+    err = err0.copy()
+    c_del, s_del = oracle.encode_delta(xs[1], xs[0], err, wl.bits)
+    assert np.array_equal(c_std, c_del) and np.array_equal(s_std, s_del)
+    assert np.array_equal(e_std.view(np.uint32), err.view(np.uint32))
+
+
+@pytest.mark.parametrize("name", ["tiny", "flux_sp"])
+def test_delta_state_ef_identity_drifts_only_by_its_roundings(name):
+    """Delta-state bookkeeping: recon_r + err - x_t changes per step by
+    exactly the four fp32 roundings of the step (x_t - x_prev, + err, the
+    error, the receiver's add), so |recon_r + err - x_t| stays within their
+    accumulated half-ulps (an exact accounting, element by element)."""
+    kw = {} if name == "tiny" else dict(tokens=32, buffers=1)
+    wl, xs = _traj(name, steps=8, **kw)
+    recon_r, err = oracle.state_init(xs[0])
+    bound = np.zeros(recon_r.shape, np.float64)
+    for t in range(1, len(xs)):
+        d1 = (_f32_from_bits(xs[t]) - _f32_from_bits(xs[t - 1])).astype(np.float32)
+        v = (d1 + err).astype(np.float32)
+        codes, scales = oracle.encode_delta(xs[t], xs[t - 1], err, wl.bits)
+        oracle.decode(codes, scales, recon_r, wl.bits)
+        bound += 0.5 * (_ulp32(d1) + _ulp32(v) + _ulp32(err) + _ulp32(recon_r))
+        gap = np.abs(recon_r.astype(np.float64) + err.astype(np.float64)
+                     - _f32_from_bits(xs[t]).astype(np.float64))
+        assert np.all(gap <= bound * (1 + 1e-12) + 1e-300)
+        assert np.all(np.abs(err) <= np.abs(v) + (scales[:, None] if wl.bits == 1 else 0.25 * scales[:, None]) + 1e-30)
+
+
+@pytest.mark.parametrize("bits", [1, 2])
+def test_delta_state_zero_residual(bits):
+    """x_t == x_prev with err = 0 gives v = 0: zero scales, zero error, and a
+    receiver that does not move."""
+    _, xs = _traj("tiny", steps=1)
+    _, err = oracle.state_init(xs[0])
+    codes, scales = oracle.encode_delta(xs[0], xs[0], err, bits)
+    assert not np.any(scales) and not np.any(err)
+    recon_r, _ = oracle.state_init(xs[0])
+    before = recon_r.copy()
+    oracle.decode(codes, scales, recon_r, bits)
+    assert np.array_equal(recon_r.view(np.uint32), before.view(np.uint32))
