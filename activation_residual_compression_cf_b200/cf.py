@@ -29,7 +29,7 @@ EXPORTS = ("cf_status_string", "cf_abi_version", "cf_codes_words_per_row",
            "cf_lowrank_status", "cf_set_lowrank_engine", "cf_set_quant_pipeline",
            "cf_set_launch_override", "cf_lowrank_encode_noalloc", "cf_decode_emit",
            "cf_decode_emit_batched", "cf_lowrank_encode_batched", "cf_lowrank_decode_batched",
-           "cf_lowrank_set_apply_events")
+           "cf_lowrank_set_apply_events", "cf_encode_delta", "cf_encode_delta_batched")
 
 
 class CFError(RuntimeError):
@@ -47,6 +47,12 @@ class cf_desc(ctypes.Structure):
 
 class cf_enc_buffer(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("recon_s", ctypes.c_void_p),
+                ("err", ctypes.c_void_p), ("codes", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p)]
+
+
+class cf_enc_delta_buffer(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("x_prev", ctypes.c_void_p),
                 ("err", ctypes.c_void_p), ("codes", ctypes.c_void_p),
                 ("scales", ctypes.c_void_p)]
 
@@ -96,6 +102,8 @@ def lib():
             "cf_encode": ([D, vp, vp, vp, vp, vp, vp], ctypes.c_int),
             "cf_decode": ([D, vp, vp, vp, vp], ctypes.c_int),
             "cf_encode_batched": ([D, i32, vp, vp, vp], ctypes.c_int),
+            "cf_encode_delta": ([D, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+            "cf_encode_delta_batched": ([D, i32, vp, vp, vp], ctypes.c_int),
             "cf_decode_batched": ([D, i32, vp, vp, vp], ctypes.c_int),
             "cf_decode_emit": ([D, vp, vp, vp, vp, vp], ctypes.c_int),
             "cf_decode_emit_batched": ([D, i32, vp, vp, vp], ctypes.c_int),
@@ -169,6 +177,16 @@ def cf_state_init(d, x0, recon, err=None, stream=None):
 def cf_encode(d, x, recon_s, err, codes, scales, stream=None):
     _chk(lib().cf_encode(ctypes.byref(d), _p(x), _p(recon_s), _p(err), _p(codes),
                          _p(scales), _s(stream)), "cf_encode")
+
+
+def cf_encode_delta(d, x, x_prev, err, codes, scales, stream=None):
+    _chk(lib().cf_encode_delta(ctypes.byref(d), _p(x), _p(x_prev), _p(err), _p(codes),
+                               _p(scales), _s(stream)), "cf_encode_delta")
+
+
+def cf_encode_delta_batched(d, n, bufs_dev, status_dev=None, stream=None):
+    _chk(lib().cf_encode_delta_batched(ctypes.byref(d), n, _p(bufs_dev), _p(status_dev),
+                                       _s(stream)), "cf_encode_delta_batched")
 
 
 def cf_decode(d, codes, scales, recon_r, stream=None):
@@ -279,6 +297,14 @@ def enc_buffer_array(sets, device) -> torch.Tensor:
         arr[i] = cf_enc_buffer(_p(x), _p(r), _p(e), _p(c), _p(s))
     host = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8)
     return host.to(device)
+
+
+def enc_delta_buffer_array(sets, device) -> torch.Tensor:
+    """Device array of cf_enc_delta_buffer from [(x, x_prev, err, codes, scales), ...]."""
+    arr = (cf_enc_delta_buffer * len(sets))()
+    for i, t in enumerate(sets):
+        arr[i] = cf_enc_delta_buffer(*[_p(v) for v in t])
+    return torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
 
 
 def dec_buffer_array(sets, device) -> torch.Tensor:

@@ -81,14 +81,17 @@ struct Shape {
 // Launch shape per row: threads (a multiple of 32) x groups of 8 channels
 // per thread.  Chosen from sweeps on B200 timed in the encode -> decode
 // sequence (C = 3072, 114 x 1024 and 114 x 4096 rows): TMA encode is fastest
-// with 4 groups per thread at 2 bits and 3 at 1 bit, TMA decode with 3; the
-// register pipeline with 2.
-Shape choose_shape(int kernel, int64_t C, int pipeline, int bits) {
+// with 4 groups per thread at 2 bits and 3 at 1 bit (delta-state encode: 4
+// and 2), TMA decode with 3; the register pipeline with 2.
+Shape choose_shape(int kernel, int64_t C, int pipeline, int bits, bool delta = false) {
     const int64_t G = (C + 7) / 8;
     Shape s;
     int gpt;
     if (pipeline == 1) {
-        gpt = kernel == 0 ? (bits == 1 ? 3 : 4) : 3;
+        if (kernel == 0)
+            gpt = bits == 1 ? (delta ? 2 : 3) : 4;
+        else
+            gpt = 3;
     } else {
         gpt = (int)((G + 191) / 192);
         if (gpt < 2) gpt = 2;
@@ -158,12 +161,17 @@ template <bool ENC, int BITS, int GPT, class Src>
 cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t *status,
                      const Shape &s, int stages_req, cudaStream_t st) {
     const int64_t W = (C * BITS + 31) / 32;
-    const int64_t slot = ENC ? 6 * C : 4 * W + 4 * C;
+    int64_t slot = 4 * W + 4 * C;
+    if constexpr (ENC) slot = (Src::kDelta ? 8 : 6) * C;
     // Ring depth: measured on B200 (C = 1920 and 3072), 5 slots for both
-    // kernels are at or near the best; deeper rings cost CTAs per SM.
+    // kernels are at or near the best; deeper rings cost CTAs per SM.  The
+    // delta-state encode's slots are a third larger (8C bytes): 3 slots,
+    // which keep three CTAs per SM, beat 4 (two CTAs) by ~10 %.
     int stages = stages_req;
     if (stages <= 0) {
-        stages = (int)(120000 / slot);
+        bool delta = false;
+        if constexpr (ENC) delta = Src::kDelta;
+        stages = (int)((delta ? 75000 : 120000) / slot);
         if (stages > 5) stages = 5;
     }
     if (stages > 8) stages = 8;
@@ -212,10 +220,10 @@ cf_status launch_one(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
 // Runtime (bits, gpt, vec) -> template instance.
 // The TMA pipeline applies when rows are 16-byte multiples (C % 8 == 0),
 // decode code rows too (ceil(C*bits/32) % 4 == 0), and a 2-slot ring fits.
-bool tma_applies(bool enc, int bits, int64_t C) {
+bool tma_applies(bool enc, int bits, int64_t C, bool delta = false) {
     if (C % 8 != 0) return false;
     if (!enc && ((C * bits + 31) / 32) % 4 != 0) return false;
-    return 2 * (enc ? 6 * C : 4 * C + C * bits / 8) <= 200000;
+    return 2 * (enc ? (delta ? 8 : 6) * C : 4 * C + C * bits / 8) <= 200000;
 }
 
 template <bool ENC, class Src>
@@ -226,9 +234,11 @@ cf_status dispatch(const Src &src, int bits, int64_t T, int64_t C, int64_t rows,
         std::lock_guard<std::mutex> lk(g_mu);
         pipe = g_pipeline[ENC ? 0 : 1];
     }
-    if (pipe == 1 && !tma_applies(ENC, bits, C)) pipe = 0;
-    Shape s = choose_shape(ENC ? 0 : 1, C, pipe, bits);
-    if (pipe == 1 && s.threads > 480) s = choose_shape(ENC ? 0 : 1, C, pipe = 0, bits);
+    bool delta = false;
+    if constexpr (ENC) delta = Src::kDelta;
+    if (pipe == 1 && !tma_applies(ENC, bits, C, delta)) pipe = 0;
+    Shape s = choose_shape(ENC ? 0 : 1, C, pipe, bits, delta);
+    if (pipe == 1 && s.threads > 480) s = choose_shape(ENC ? 0 : 1, C, pipe = 0, bits, delta);
     s.pipeline = pipe;
     const bool vec = (C % 8) == 0;
 #define CF_CASE(B, G, V)                                     \
@@ -289,7 +299,8 @@ cf_status cf_state_init(const cf_desc *d, const uint16_t *x0, float *recon, floa
     const int64_t n = d->tokens * d->channels;
     if (n == 0) return CF_OK;
     CF_TRY(check_dev_ptr(x0));
-    CF_TRY(check_dev_ptr(recon));
+    if (!recon && !err) return CF_ERR_INVALID_ARG;
+    if (recon) CF_TRY(check_dev_ptr(recon));
     if (err) CF_TRY(check_dev_ptr(err));
     const int threads = 256;
     int64_t blocks = (n / 8 + threads - 1) / threads;
@@ -310,6 +321,20 @@ cf_status cf_encode(const cf_desc *d, const uint16_t *x, float *recon_s, float *
     CF_TRY(check_dev_ptr(codes));
     CF_TRY(check_dev_ptr(scales, 4));
     cf::EncSingle src{{x, recon_s, err, codes, scales}};
+    return dispatch<true>(src, d->bits, d->tokens, d->channels, d->tokens, nullptr,
+                          (cudaStream_t)stream);
+}
+
+cf_status cf_encode_delta(const cf_desc *d, const uint16_t *x, const uint16_t *x_prev, float *err,
+                          uint32_t *codes, float *scales, void *stream) {
+    CF_TRY(check_quant_desc(d));
+    if (d->tokens == 0) return CF_OK;
+    CF_TRY(check_dev_ptr(x));
+    CF_TRY(check_dev_ptr(x_prev));
+    CF_TRY(check_dev_ptr(err));
+    CF_TRY(check_dev_ptr(codes));
+    CF_TRY(check_dev_ptr(scales, 4));
+    cf::EncDeltaSingle src{{x, nullptr, err, codes, scales, x_prev}};
     return dispatch<true>(src, d->bits, d->tokens, d->channels, d->tokens, nullptr,
                           (cudaStream_t)stream);
 }
@@ -359,6 +384,18 @@ cf_status cf_encode_batched(const cf_desc *d, int32_t n, const cf_enc_buffer *bu
     CF_TRY(check_dev_ptr(bufs_dev));
     if (status_dev) CF_TRY(check_dev_ptr(status_dev));
     cf::EncArray src{bufs_dev};
+    return dispatch<true>(src, d->bits, d->tokens, d->channels, d->tokens * (int64_t)n,
+                          status_dev, (cudaStream_t)stream);
+}
+
+cf_status cf_encode_delta_batched(const cf_desc *d, int32_t n, const cf_enc_delta_buffer *bufs_dev,
+                                  int32_t *status_dev, void *stream) {
+    CF_TRY(check_quant_desc(d));
+    if (n < 0) return CF_ERR_INVALID_ARG;
+    if (n == 0 || d->tokens == 0) return CF_OK;
+    CF_TRY(check_dev_ptr(bufs_dev));
+    if (status_dev) CF_TRY(check_dev_ptr(status_dev));
+    cf::EncDeltaArray src{bufs_dev};
     return dispatch<true>(src, d->bits, d->tokens, d->channels, d->tokens * (int64_t)n,
                           status_dev, (cudaStream_t)stream);
 }

@@ -38,10 +38,11 @@ namespace cf {
 
 struct EncPtrs {
     const uint16_t *x;
-    float *recon;
+    float *recon;             // standard sender: the reconstruction copy
     float *err;
     uint32_t *codes;
     float *scales;
+    const uint16_t *xprev;    // delta-state sender: the previous activation
 };
 
 struct DecPtrs {
@@ -62,11 +63,35 @@ __device__ __forceinline__ P ldg_ptr(P const *field) {
 struct EncSingle {
     EncPtrs p;
     static constexpr bool kChecked = false;
+    static constexpr bool kDelta = false;
     __device__ __forceinline__ EncPtrs get(int64_t) const { return p; }
+};
+struct EncDeltaSingle {
+    EncPtrs p;
+    static constexpr bool kChecked = false;
+    static constexpr bool kDelta = true;
+    __device__ __forceinline__ EncPtrs get(int64_t) const { return p; }
+};
+struct EncDeltaArray {
+    const cf_enc_delta_buffer *a;
+    static constexpr bool kChecked = true;
+    static constexpr bool kDelta = true;
+    __device__ __forceinline__ EncPtrs get(int64_t i) const {
+        const cf_enc_delta_buffer *e = a + i;
+        EncPtrs p;
+        p.x = ldg_ptr(&e->x);
+        p.xprev = ldg_ptr(&e->x_prev);
+        p.recon = nullptr;
+        p.err = ldg_ptr(&e->err);
+        p.codes = ldg_ptr(&e->codes);
+        p.scales = ldg_ptr(&e->scales);
+        return p;
+    }
 };
 struct EncArray {
     const cf_enc_buffer *a;
     static constexpr bool kChecked = true;
+    static constexpr bool kDelta = false;
     __device__ __forceinline__ EncPtrs get(int64_t i) const {
         const cf_enc_buffer *e = a + i;
         EncPtrs p;
@@ -75,6 +100,7 @@ struct EncArray {
         p.err = ldg_ptr(&e->err);
         p.codes = ldg_ptr(&e->codes);
         p.scales = ldg_ptr(&e->scales);
+        p.xprev = nullptr;
         return p;
     }
 };
@@ -131,9 +157,11 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float *v) {
 __device__ __forceinline__ bool misaligned4(const void *p) {
     return (reinterpret_cast<uintptr_t>(p) & 3u) != 0;
 }
+template <bool DELTA>
 __device__ __forceinline__ int enc_ptr_status(const EncPtrs &p) {
-    if (!p.x || !p.recon || !p.err || !p.codes || !p.scales) return CF_ERR_INVALID_ARG;
-    if (misaligned16(p.x) || misaligned16(p.recon) || misaligned16(p.err) ||
+    const void *state = DELTA ? static_cast<const void *>(p.xprev) : static_cast<const void *>(p.recon);
+    if (!p.x || !state || !p.err || !p.codes || !p.scales) return CF_ERR_INVALID_ARG;
+    if (misaligned16(p.x) || misaligned16(state) || misaligned16(p.err) ||
         misaligned16(p.codes) || misaligned4(p.scales))
         return CF_ERR_ALIGNMENT;
     return CF_OK;
@@ -168,6 +196,25 @@ __device__ __forceinline__ float dequantize(uint32_t code, float scale) {
     return __fmul_rn(lvl, scale);
 }
 
+// Residual of 8 channels from their raw bf16 words.  Standard sender:
+// v = (float)x - recon.  Delta-state sender: v = ((float)x - (float)x_prev)
+// + err_old, two roundings in that order.  r holds recon or err_old.
+template <bool DELTA>
+__device__ __forceinline__ void residual8(const uint4 &xw, const uint4 &pw, const float *r, float *v) {
+    const uint32_t w4[4] = {xw.x, xw.y, xw.z, xw.w};
+    const uint32_t p4[4] = {pw.x, pw.y, pw.z, pw.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const float xf = bf16_bits_to_f32((w4[e >> 1] >> ((e & 1) * 16)) & 0xffffu);
+        if (DELTA) {
+            const float pf = bf16_bits_to_f32((p4[e >> 1] >> ((e & 1) * 16)) & 0xffffu);
+            v[e] = __fadd_rn(__fsub_rn(xf, pf), r[e]);
+        } else {
+            v[e] = __fsub_rn(xf, r[e]);
+        }
+    }
+}
+
 template <int BITS, int GPT, bool VEC, class Src>
 __global__ void __launch_bounds__(512)
 encode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status) {
@@ -189,19 +236,21 @@ encode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
         const int64_t t = row - b * T;
         const EncPtrs p = src.get(b);
         if (Src::kChecked) {
-            const int st = enc_ptr_status(p);
+            const int st = enc_ptr_status<Src::kDelta>(p);
             if (st != CF_OK) {
                 if (tid == 0) report(status, st);
                 continue;  // uniform across the CTA
             }
         }
         const uint16_t *xr = p.x + t * C;
-        float *rr = p.recon + t * C;
+        // r: the reconstruction (standard sender) or the old error (delta)
+        float *rr = (Src::kDelta ? p.err : p.recon) + t * C;
+        const uint16_t *pr = Src::kDelta ? p.xprev + t * C : nullptr;
         float *er = p.err + t * C;
         uint32_t *cw = p.codes + t * W;
 
         // Phase 1: issue every load of this thread's groups.
-        uint4 xraw[GPT];
+        uint4 xraw[GPT], praw[GPT];
         float r[GPT][8];
 #pragma unroll
         for (int j = 0; j < GPT; ++j) {
@@ -209,40 +258,38 @@ encode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
             if (VEC) {
                 if (g < G) {
                     xraw[j] = ld_ro_v4(xr + 8 * g);
+                    if (Src::kDelta) praw[j] = ld_ro_v4(pr + 8 * g);
                     const float4 a = ld_state_v4(rr + 8 * g);
                     const float4 c = ld_state_v4(rr + 8 * g + 4);
                     r[j][0] = a.x; r[j][1] = a.y; r[j][2] = a.z; r[j][3] = a.w;
                     r[j][4] = c.x; r[j][5] = c.y; r[j][6] = c.z; r[j][7] = c.w;
                 } else {
-                    xraw[j] = make_uint4(0, 0, 0, 0);
+                    xraw[j] = praw[j] = make_uint4(0, 0, 0, 0);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) r[j][e] = 0.0f;
                 }
             } else {
-                uint32_t h[8];
+                uint32_t h[8], hp[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int64_t c = 8 * g + e;
                     const bool ok = (g < G) && (c < C);
                     h[e] = ok ? (uint32_t)xr[c] : 0u;
+                    hp[e] = (Src::kDelta && ok) ? (uint32_t)pr[c] : 0u;
                     r[j][e] = ok ? rr[c] : 0.0f;
                 }
                 xraw[j] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16),
                                      h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+                praw[j] = make_uint4(hp[0] | (hp[1] << 16), hp[2] | (hp[3] << 16),
+                                     hp[4] | (hp[5] << 16), hp[6] | (hp[7] << 16));
             }
         }
 
-        // Phase 2: residual (padding lanes hold x = recon = 0, so v = 0).
+        // Phase 2: residual (padding lanes hold zeros, so v = 0).
         float v[GPT][8];
 #pragma unroll
-        for (int j = 0; j < GPT; ++j) {
-            const uint32_t w4[4] = {xraw[j].x, xraw[j].y, xraw[j].z, xraw[j].w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const uint32_t h = (w4[e >> 1] >> ((e & 1) * 16)) & 0xffffu;
-                v[j][e] = __fsub_rn(bf16_bits_to_f32(h), r[j][e]);
-            }
-        }
+        for (int j = 0; j < GPT; ++j)
+            residual8<Src::kDelta>(xraw[j], praw[j], r[j], v[j]);
 
         // Phase 3: per-token scale.
         float scale;
@@ -298,15 +345,17 @@ encode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
                 if (VEC) {
                     st_stream_v4(er + 8 * g, make_float4(eo[0], eo[1], eo[2], eo[3]));
                     st_stream_v4(er + 8 * g + 4, make_float4(eo[4], eo[5], eo[6], eo[7]));
-                    st_state_v4(rr + 8 * g, make_float4(ro[0], ro[1], ro[2], ro[3]));
-                    st_state_v4(rr + 8 * g + 4, make_float4(ro[4], ro[5], ro[6], ro[7]));
+                    if (!Src::kDelta) {
+                        st_state_v4(rr + 8 * g, make_float4(ro[0], ro[1], ro[2], ro[3]));
+                        st_state_v4(rr + 8 * g + 4, make_float4(ro[4], ro[5], ro[6], ro[7]));
+                    }
                 } else {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int64_t c = 8 * g + e;
                         if (c < C) {
                             er[c] = eo[e];
-                            rr[c] = ro[e];
+                            if (!Src::kDelta) rr[c] = ro[e];
                         }
                     }
                 }
@@ -405,16 +454,19 @@ decode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
 // Warmup: recon = (float)x0, err = 0 (err may be null).  Flat over n
 // elements; 8-element vector body, scalar tail.
 __global__ void state_init_kernel(const uint16_t *x0, float *recon, float *err, int64_t n) {
+    // recon or err may be null (not both; the host checks)
     const int64_t groups = n >> 3;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += stride) {
-        const uint4 xv = ld_ro_v4(x0 + 8 * g);
-        const uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
-        float f[8];
+        if (recon) {
+            const uint4 xv = ld_ro_v4(x0 + 8 * g);
+            const uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
+            float f[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = bf16_bits_to_f32((w4[e >> 1] >> ((e & 1) * 16)) & 0xffffu);
-        st_state_v4(recon + 8 * g, make_float4(f[0], f[1], f[2], f[3]));
-        st_state_v4(recon + 8 * g + 4, make_float4(f[4], f[5], f[6], f[7]));
+            for (int e = 0; e < 8; ++e) f[e] = bf16_bits_to_f32((w4[e >> 1] >> ((e & 1) * 16)) & 0xffffu);
+            st_state_v4(recon + 8 * g, make_float4(f[0], f[1], f[2], f[3]));
+            st_state_v4(recon + 8 * g + 4, make_float4(f[4], f[5], f[6], f[7]));
+        }
         if (err) {
             st_stream_v4(err + 8 * g, make_float4(0.f, 0.f, 0.f, 0.f));
             st_stream_v4(err + 8 * g + 4, make_float4(0.f, 0.f, 0.f, 0.f));
@@ -422,7 +474,7 @@ __global__ void state_init_kernel(const uint16_t *x0, float *recon, float *err, 
     }
     if (blockIdx.x == 0 && (int64_t)threadIdx.x < n - 8 * groups) {
         const int64_t i = 8 * groups + threadIdx.x;
-        recon[i] = bf16_bits_to_f32(x0[i]);
+        if (recon) recon[i] = bf16_bits_to_f32(x0[i]);
         if (err) err[i] = 0.0f;
     }
 }

@@ -64,7 +64,8 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
 }
 
 // Shared layout: [stages][slot bytes] then full[stages], empty[stages].
-// Encode slot: x row (2C bytes) then recon row (4C bytes).
+// Encode slot: x row (2C bytes) then recon row (4C bytes); delta-state
+// encode: x row (2C), x_prev row (2C), err row (4C).
 // Decode slot: codes row (4W bytes, padded to 16) then recon row (4C bytes).
 
 template <int BITS, int GPT, class Src>
@@ -77,7 +78,7 @@ encode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
     __shared__ int abort_row[2];  // set before the row's barrier, read after it
     const int64_t G = C >> 3;  // C % 8 == 0 on this path
     const int64_t W = (C * BITS + 31) >> 5;
-    const uint32_t slot = (uint32_t)(6 * C);
+    const uint32_t slot = (uint32_t)((Src::kDelta ? 8 : 6) * C);
     const uint32_t base = saddr(smem);
     const uint32_t bars = base + (uint32_t)stages * slot;
     const int tid = threadIdx.x;
@@ -98,7 +99,7 @@ encode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
         for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
             const int64_t b = row / T, t = row - b * T;
             const EncPtrs p = src.get(b);
-            if (Src::kChecked && enc_ptr_status(p) != CF_OK) continue;
+            if (Src::kChecked && enc_ptr_status<Src::kDelta>(p) != CF_OK) continue;
             const int s = i % stages;
             const uint32_t ph = (uint32_t)(i / stages) & 1u;
             if (!bar_wait(bars + 8u * (stages + s), ph ^ 1u)) {
@@ -110,7 +111,12 @@ encode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
             const uint32_t dst = base + (uint32_t)s * slot;
             bar_expect(bars + 8u * s, slot);
             bulk_g2s(dst, p.x + t * C, (uint32_t)(2 * C), bars + 8u * s);
-            bulk_g2s(dst + (uint32_t)(2 * C), p.recon + t * C, (uint32_t)(4 * C), bars + 8u * s);
+            if (Src::kDelta) {
+                bulk_g2s(dst + (uint32_t)(2 * C), p.xprev + t * C, (uint32_t)(2 * C), bars + 8u * s);
+                bulk_g2s(dst + (uint32_t)(4 * C), p.err + t * C, (uint32_t)(4 * C), bars + 8u * s);
+            } else {
+                bulk_g2s(dst + (uint32_t)(2 * C), p.recon + t * C, (uint32_t)(4 * C), bars + 8u * s);
+            }
             ++i;
         }
         return;
@@ -123,7 +129,7 @@ encode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
         const int64_t b = row / T, t = row - b * T;
         const EncPtrs p = src.get(b);
         if (Src::kChecked) {
-            const int st = enc_ptr_status(p);
+            const int st = enc_ptr_status<Src::kDelta>(p);
             if (st != CF_OK) {
                 if (ct == 0) report(status, st);
                 continue;
@@ -136,8 +142,10 @@ encode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
         ok = __shfl_sync(kFullMask, ok ? 1 : 0, 0) != 0;
         if (!ok && lane == 0) abort_row[par] = 1;  // acted on after the barrier
         const uint8_t *sx = smem + (size_t)s * slot;
-        const float *sr = reinterpret_cast<const float *>(sx + 2 * C);
-        float *rr = p.recon + t * C;
+        const uint8_t *sp = sx + 2 * C;   // x_prev row (delta-state sender)
+        // recon (standard) or the old err (delta-state)
+        const float *sr = reinterpret_cast<const float *>(sx + (Src::kDelta ? 4 : 2) * C);
+        float *rr = Src::kDelta ? nullptr : p.recon + t * C;
         float *er = p.err + t * C;
         uint32_t *cw = p.codes + t * W;
 
@@ -147,14 +155,13 @@ encode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
             const int64_t g = (int64_t)j * nc + ct;
             if (ok && g < G) {
                 const uint4 xw = *reinterpret_cast<const uint4 *>(sx + 16 * g);
+                const uint4 pw = Src::kDelta ? *reinterpret_cast<const uint4 *>(sp + 16 * g)
+                                             : make_uint4(0, 0, 0, 0);
                 const float4 a = *reinterpret_cast<const float4 *>(sr + 8 * g);
                 const float4 c = *reinterpret_cast<const float4 *>(sr + 8 * g + 4);
                 r[j][0] = a.x; r[j][1] = a.y; r[j][2] = a.z; r[j][3] = a.w;
                 r[j][4] = c.x; r[j][5] = c.y; r[j][6] = c.z; r[j][7] = c.w;
-                const uint32_t w4[4] = {xw.x, xw.y, xw.z, xw.w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    v[j][e] = __fsub_rn(bf16_bits_to_f32((w4[e >> 1] >> ((e & 1) * 16)) & 0xffffu), r[j][e]);
+                residual8<Src::kDelta>(xw, pw, r[j], v[j]);
             } else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) r[j][e] = v[j][e] = 0.0f;
@@ -227,8 +234,10 @@ encode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
             if (g < G) {
                 st_stream_v4(er + 8 * g, make_float4(eo[0], eo[1], eo[2], eo[3]));
                 st_stream_v4(er + 8 * g + 4, make_float4(eo[4], eo[5], eo[6], eo[7]));
-                st_state_v4(rr + 8 * g, make_float4(ro[0], ro[1], ro[2], ro[3]));
-                st_state_v4(rr + 8 * g + 4, make_float4(ro[4], ro[5], ro[6], ro[7]));
+                if (!Src::kDelta) {
+                    st_state_v4(rr + 8 * g, make_float4(ro[0], ro[1], ro[2], ro[3]));
+                    st_state_v4(rr + 8 * g + 4, make_float4(ro[4], ro[5], ro[6], ro[7]));
+                }
                 if ((lane % GPW) == 0) cw[g / GPW] = word;
             }
         }

@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--iters", type=int, default=0,
                     help="low-rank: subspace iterations (default: the workload's)")
     ap.add_argument("--rank", type=int, default=0, help="low-rank: rank (default: the workload's)")
+    ap.add_argument("--delta", action="store_true",
+                    help="quantize: delta-state sender (previous activation + error buffer)")
     ap.add_argument("--warm", action="store_true",
                     help="low-rank: warm start every encode after the first from the previous Q")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -294,13 +296,23 @@ def run_ours(args, world, rank, local):
     for b in range(n):
         cf.cf_state_init(d, X16[0, b], recon_s[b], err[b])
         cf.cf_state_init(d, X16[0, b], recon_r[b], None)
-    enc = [cf.enc_buffer_array([(X16[s, b], recon_s[b], err[b], codes[b], scales[b])
-                                for b in range(n)], dev) for s in range(S)]
+    if args.delta:
+        # delta-state sender: x_prev = the previous generated step; err = 0
+        for b in range(n):
+            cf.cf_state_init(d, X16[0, b], None, err[b])
+        enc = [cf.enc_delta_buffer_array([(X16[s, b], X16[s - 1, b], err[b], codes[b], scales[b])
+                                          for b in range(n)], dev) if s > 0 else None
+               for s in range(S)]
+        encode_batched = cf.cf_encode_delta_batched
+    else:
+        enc = [cf.enc_buffer_array([(X16[s, b], recon_s[b], err[b], codes[b], scales[b])
+                                    for b in range(n)], dev) for s in range(S)]
+        encode_batched = cf.cf_encode_batched
     dec = cf.dec_buffer_array([(codes[b], scales[b], recon_r[b]) for b in range(n)], dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
-        cf.cf_encode_batched(d, n, enc[1 + i % (S - 1)], status, stream)
+        encode_batched(d, n, enc[1 + i % (S - 1)], status, stream)
         cf.cf_decode_batched(d, n, dec, status, stream)
 
     sampler = ClockSampler(dev)
@@ -317,7 +329,7 @@ def run_ours(args, world, rank, local):
         for i in range(args.steps):
             e0, e1, e2 = ev[i]
             e0.record(stream)
-            cf.cf_encode_batched(d, n, enc[1 + (args.warmup + i) % (S - 1)], status, stream)
+            encode_batched(d, n, enc[1 + (args.warmup + i) % (S - 1)], status, stream)
             e1.record(stream)
             cf.cf_decode_batched(d, n, dec, status, stream)
             e2.record(stream)
@@ -332,7 +344,10 @@ def run_ours(args, world, rank, local):
 
     bytes_processed = 2 * T * C * n * args.steps * world
     value = bytes_processed / (ms / 1e3) / 1e9
-    enc_bytes = n * T * (C * 2 + C * 4 * 3 + Wd * 4 + 4)     # x, recon r/w, err w, codes, scale
+    if args.delta:
+        enc_bytes = n * T * (C * 2 * 2 + C * 4 * 2 + Wd * 4 + 4)  # x, x_prev, err r/w, codes, scale
+    else:
+        enc_bytes = n * T * (C * 2 + C * 4 * 3 + Wd * 4 + 4)     # x, recon r/w, err w, codes, scale
     dec_bytes = n * T * (Wd * 4 + 4 + C * 4 * 2)             # codes, scale, recon r/w
     peak, peak_kind = peaks()
     enc_gbs = enc_bytes / (enc_ms / 1e3) / 1e9
@@ -340,7 +355,7 @@ def run_ours(args, world, rank, local):
 
     # End to end through the public API: pinned host x in, payload out.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.delta:
         e2e = run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, status)
         e2e["ms"] = R.reduce_scalar(e2e["ms"], "max")
         e2e = {"value": round(bytes_processed / (e2e["ms"] / 1e3) / 1e9, 3), "unit": "GB/s",
@@ -354,21 +369,23 @@ def run_ours(args, world, rank, local):
                "sample": f"{done} buffer-steps of {args.workload} buffer 0 ({T}x{C}, "
                          f"{bits}-bit encode+decode), {tw:.1f} s single-threaded C"}
 
-    traffic = recorded_traffic("encode", args.workload)
+    traffic = recorded_traffic("encode_delta" if args.delta else "encode", args.workload)
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 in, fp32 state", "data": "synthetic",
         "config": {"workload": args.workload, "tokens": T, "channels": C, "buffers": n,
-                   "bits": bits, "mode": f"{bits}-bit {'mean-abs' if bits == 1 else 'absmax'} + EF",
+                   "bits": bits, "mode": f"{bits}-bit {'mean-abs' if bits == 1 else 'absmax'} + EF"
+                   + (", delta-state sender" if args.delta else ""),
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2 ({n * T * C * 14 / 1e9:.1f} GB touched per step)",
                    "launches_per_step": 2},
         "roofline": {"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(enc_gbs / peak, 4), "traffic": traffic,
                      "kernel": ("encode_tma_kernel (batched, TMA row staging)" if args.pipeline != 0
-                                else "encode_rows_kernel (batched, register rows)"),
+                                else "encode_rows_kernel (batched, register rows)")
+                     + (", delta-state sender" if args.delta else ""),
                      "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": enc_bytes, "avg_launch_ms": round(enc_ms, 4)},
         "decode": {"achieved": round(dec_gbs, 1), "frac": round(dec_gbs / peak, 4),

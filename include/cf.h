@@ -123,8 +123,10 @@ int64_t cf_codes_words_per_row(const cf_desc *d);
 int64_t cf_payload_bytes(const cf_desc *d);
 
 /* Warmup step ("Measured effects": the first step is sent uncompressed).
- * recon[i] = (float)x0[i]; err[i] = 0 when err != NULL.  Call it for the
- * sender (with err) and for the receiver (err = NULL) on the same x0.
+ * recon[i] = (float)x0[i] when recon != NULL; err[i] = 0 when err != NULL
+ * (at least one of them).  Call it for the sender (with err) and for the
+ * receiver (err = NULL) on the same x0; the delta-state sender below keeps
+ * no reconstruction and calls it with recon = NULL.
  * x0: bf16 [T][C] device; recon, err: fp32 [T][C] device. */
 cf_status cf_state_init(const cf_desc *d, const uint16_t *x0, float *recon,
                         float *err, void *stream);
@@ -167,6 +169,37 @@ cf_status cf_decode_batched(const cf_desc *d, int32_t n,
 cf_status cf_decode_emit_batched(const cf_desc *d, int32_t n,
                                  const cf_dec_emit_buffer *bufs_dev,
                                  int32_t *status_dev, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Delta-state sender: the same residual-with-error-feedback ("Approach") kept
+ * as the previous activation and the error buffer instead of a sender copy
+ * of the reconstruction.  With x_prev the previous step's activation (bf16,
+ * kept by the caller: x_0 after the warmup step) and err the error buffer:
+ *   v = ((float)x - (float)x_prev) + err       two fp32 roundings
+ * then the per-token scale, codes, packing and err = v - deq exactly as in
+ * cf_encode; the receiver is unchanged (cf_decode).  In exact arithmetic v
+ * equals cf_encode's x - recon_s (recon_s + err == x after every step), so
+ * the two senders agree up to fp32 rounding, and at the first compressed
+ * step after the warmup they are bit-identical.  It moves 12 bytes per
+ * element instead of 14 (recon_s is neither read nor written).  Warmup:
+ * cf_state_init(d, x0, NULL, err, stream), x_prev = x0.  Alignment as
+ * cf_encode (x_prev 16 bytes). */
+cf_status cf_encode_delta(const cf_desc *d, const uint16_t *x, const uint16_t *x_prev,
+                          float *err, uint32_t *codes, float *scales, void *stream);
+
+/* One sender buffer set of the batched delta-state encode. */
+typedef struct cf_enc_delta_buffer {
+    const uint16_t *x;       /* bf16 [T][C], this step's activation             */
+    const uint16_t *x_prev;  /* bf16 [T][C], the previous step's activation     */
+    float *err;              /* fp32 [T][C], error-feedback buffer (updated)    */
+    uint32_t *codes;         /* uint32 [T][ceil(C*bits/32)] (written)           */
+    float *scales;           /* fp32 [T] (written)                              */
+} cf_enc_delta_buffer;
+
+/* Batched delta-state encode: rules as cf_encode_batched. */
+cf_status cf_encode_delta_batched(const cf_desc *d, int32_t n,
+                                  const cf_enc_delta_buffer *bufs_dev,
+                                  int32_t *status_dev, void *stream);
 
 /* ------------------------------------------------------------------------
  * Low-rank mode ("Approach", "Key results", "Builds on": PowerSGD-style
