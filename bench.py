@@ -59,6 +59,9 @@ def parse():
     ap.add_argument("--iters", type=int, default=0,
                     help="low-rank: subspace iterations (default: the workload's)")
     ap.add_argument("--rank", type=int, default=0, help="low-rank: rank (default: the workload's)")
+    ap.add_argument("--e2e-chunks", type=int, default=6,
+                    help="end-to-end leg: buffers of a step split into this many chunks whose "
+                         "copies overlap the kernels of their neighbours")
     ap.add_argument("--delta", action="store_true",
                     help="quantize: delta-state sender (previous activation + error buffer)")
     ap.add_argument("--warm", action="store_true",
@@ -360,7 +363,8 @@ def run_ours(args, world, rank, local):
         e2e["ms"] = R.reduce_scalar(e2e["ms"], "max")
         e2e = {"value": round(bytes_processed / (e2e["ms"] / 1e3) / 1e9, 3), "unit": "GB/s",
                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-               "ms_per_step": round(e2e["ms"] / args.steps, 4)}
+               "ms_per_step": round(e2e["ms"] / args.steps, 4),
+               "overlap": f"{e2e['chunks']} chunks on copy-in / compute / copy-out streams"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -606,7 +610,17 @@ def run_lowrank_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, OM, pc,
 
 
 def run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, status):
+    """End to end through the C ABI with host buffers: every step copies the
+    pinned host activations of all buffers in, encodes and decodes them, and
+    reads the payload (codes, scales) back.  The step is split into chunks of
+    buffers on three streams -- host-to-device copies, the library calls,
+    device-to-host copies -- ordered by events, so the copies of one chunk
+    overlap the kernels of its neighbours (what a serving loop does with the
+    same calls).  The activations land in two alternating device slots, so a
+    step's copies never wait on the previous step's kernels."""
     n, T, C = wl.buffers, wl.tokens, wl.channels
+    nch = max(1, min(args.e2e_chunks, n))
+    bounds = [round(k * n / nch) for k in range(nch + 1)]
     # Two host steps of pinned input (buffer 0's trajectory replicated over
     # the buffers), alternated so consecutive steps see a real residual.
     tr = W.Trajectory(wl, 0, device=dev)
@@ -616,33 +630,63 @@ def run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, 
         xk = tr.next().unsqueeze(0).expand(n, T, C).contiguous().cpu()
         x_host.append(xk.pin_memory())
         del xk
-    x_dev = torch.empty((n, T, C), dtype=torch.bfloat16, device=dev)
-    x16 = x_dev.view(torch.int16)
-    enc = cf.enc_buffer_array([(x16[b], recon_s[b], err[b], codes[b], scales[b])
-                               for b in range(n)], dev)
-    dec = cf.dec_buffer_array([(codes[b], scales[b], recon_r[b]) for b in range(n)], dev)
+    x_dev = [torch.empty((n, T, C), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    enc = [[cf.enc_buffer_array([(x_dev[slot].view(torch.int16)[b], recon_s[b], err[b], codes[b],
+                                  scales[b]) for b in range(bounds[k], bounds[k + 1])], dev)
+            for k in range(nch)] for slot in range(2)]
+    dec = [cf.dec_buffer_array([(codes[b], scales[b], recon_r[b])
+                                for b in range(bounds[k], bounds[k + 1])], dev) for k in range(nch)]
     codes_h = torch.empty(codes.shape, dtype=codes.dtype).pin_memory()
     scales_h = torch.empty(scales.shape, dtype=scales.dtype).pin_memory()
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    d2h_done = [None] * nch      # last device-to-host copy of each chunk's payload
+    enc_done = [[None] * nch for _ in range(2)]   # last kernels reading a slot's chunk
 
     def step(i):
-        x_dev.copy_(x_host[i % 2], non_blocking=True)
-        cf.cf_encode_batched(d, n, enc, status, stream)
-        cf.cf_decode_batched(d, n, dec, status, stream)
-        codes_h.copy_(codes, non_blocking=True)
-        scales_h.copy_(scales, non_blocking=True)
+        slot = i % 2
+        for k in range(nch):
+            lo, hi = bounds[k], bounds[k + 1]
+            e_in, e_done, e_out = ev(), ev(), ev()
+            with torch.cuda.stream(s_in):
+                if enc_done[slot][k] is not None:
+                    s_in.wait_event(enc_done[slot][k])   # slot's chunk no longer read
+                x_dev[slot][lo:hi].copy_(x_host[slot][lo:hi], non_blocking=True)
+                e_in.record(s_in)
+            stream.wait_event(e_in)
+            if d2h_done[k] is not None:
+                stream.wait_event(d2h_done[k])   # payload of the last step read out
+            cf.cf_encode_batched(d, hi - lo, enc[slot][k], status, stream)
+            cf.cf_decode_batched(d, hi - lo, dec[k], status, stream)
+            e_done.record(stream)
+            enc_done[slot][k] = e_done
+            s_out.wait_event(e_done)
+            with torch.cuda.stream(s_out):
+                codes_h[lo:hi].copy_(codes[lo:hi], non_blocking=True)
+                scales_h[lo:hi].copy_(scales[lo:hi], non_blocking=True)
+                e_out.record(s_out)
+            d2h_done[k] = e_out
+
+    def settle():
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
 
     for i in range(max(3, args.warmup // 4)):
         step(i)
+    settle()
     torch.cuda.synchronize()
     steps = args.steps
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    s_in.wait_stream(stream)
     for i in range(steps):
         step(i)
+    settle()
     b.record(stream)
     torch.cuda.synchronize()
     return {"ms": a.elapsed_time(b), "h2d": n * T * C * 2,
-            "d2h": codes.numel() * 4 + scales.numel() * 4}
+            "d2h": codes.numel() * 4 + scales.numel() * 4, "chunks": nch}
 
 
 def run_reference(args, world, rank):
