@@ -568,7 +568,8 @@ def run_lowrank(args, world, rank, local):
         e2e["ms"] = R.reduce_scalar(e2e["ms"], "max")
         e2e = {"value": round(2 * T * C * n * args.steps * world / (e2e["ms"] / 1e3) / 1e9, 3),
                "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
-               "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(e2e["ms"] / args.steps, 4)}
+               "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(e2e["ms"] / args.steps, 4),
+               "overlap": f"{e2e['chunks']} chunks on copy-in / compute / copy-out streams"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -615,8 +616,11 @@ def run_lowrank(args, world, rank, local):
 def run_lowrank_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, OM, pc, ps, qc, qs, ws):
     """Low-rank end to end: every step copies the pinned host activations of
     all buffers in, runs the batched sender and receiver, and reads the INT4
-    payload (factor codes and scales) back to the host."""
+    payload (factor codes and scales) back to the host.  Chunks of buffers on
+    three streams overlap the copies with the kernels, as in run_e2e."""
     n, T, C = wl.buffers, wl.tokens, wl.channels
+    nch = max(1, min(args.e2e_chunks, n))
+    bounds = [round(k * n / nch) for k in range(nch + 1)]
     tr = W.Trajectory(wl, 0, device=dev)
     tr.next()
     x_host = []
@@ -624,36 +628,65 @@ def run_lowrank_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, OM, pc,
         xk = tr.next().unsqueeze(0).expand(n, T, C).contiguous().cpu()
         x_host.append(xk.pin_memory())
         del xk
-    x_dev = torch.empty((n, T, C), dtype=torch.bfloat16, device=dev)
-    x16 = x_dev.view(torch.int16)
+    x_dev = [torch.empty((n, T, C), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     wsb = cf.cf_lowrank_workspace_bytes(d)
-    enc = cf.lowrank_buffer_array([(x16[b], recon_s[b], err[b], OM[1, b], pc[b], ps[b], qc[b],
-                                    qs[b]) for b in range(n)], dev)
-    dec = cf.lowrank_dec_buffer_array([(pc[b], ps[b], qc[b], qs[b], recon_r[b])
-                                       for b in range(n)], dev)
+    enc = [[cf.lowrank_buffer_array([(x_dev[slot].view(torch.int16)[b], recon_s[b], err[b], OM[1, b],
+                                      pc[b], ps[b], qc[b], qs[b])
+                                     for b in range(bounds[k], bounds[k + 1])], dev)
+            for k in range(nch)] for slot in range(2)]
+    dec = [cf.lowrank_dec_buffer_array([(pc[b], ps[b], qc[b], qs[b], recon_r[b])
+                                        for b in range(bounds[k], bounds[k + 1])], dev)
+           for k in range(nch)]
     outs = [pc, ps, qc, qs]
     host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    d2h_done = [None] * nch
+    enc_done = [[None] * nch for _ in range(2)]
 
     def step(i):
-        x_dev.copy_(x_host[i % 2], non_blocking=True)
-        cf.cf_lowrank_encode_batched(d, n, enc, ws, stream=stream)
-        cf.cf_lowrank_decode_batched(d, n, dec, stream=stream)
-        for h, t in zip(host, outs):
-            h.copy_(t, non_blocking=True)
+        slot = i % 2
+        for k in range(nch):
+            lo, hi = bounds[k], bounds[k + 1]
+            e_in, e_done, e_out = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
+            with torch.cuda.stream(s_in):
+                if enc_done[slot][k] is not None:
+                    s_in.wait_event(enc_done[slot][k])
+                x_dev[slot][lo:hi].copy_(x_host[slot][lo:hi], non_blocking=True)
+                e_in.record(s_in)
+            stream.wait_event(e_in)
+            if d2h_done[k] is not None:
+                stream.wait_event(d2h_done[k])
+            cf.cf_lowrank_encode_batched(d, hi - lo, enc[slot][k], ws[lo * wsb:], stream=stream)
+            cf.cf_lowrank_decode_batched(d, hi - lo, dec[k], stream=stream)
+            e_done.record(stream)
+            enc_done[slot][k] = e_done
+            s_out.wait_event(e_done)
+            with torch.cuda.stream(s_out):
+                for h, t in zip(host, outs):
+                    h[lo:hi].copy_(t[lo:hi], non_blocking=True)
+                e_out.record(s_out)
+            d2h_done[k] = e_out
+
+    def settle():
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
 
     for i in range(max(3, args.warmup)):
         step(i)
+    settle()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    s_in.wait_stream(stream)
     for i in range(args.steps):
         step(i)
+    settle()
     b.record(stream)
     torch.cuda.synchronize()
     st = max(cf.cf_lowrank_status(ws[k * wsb:]) for k in range(n))
     assert st in (0, 6), cf.cf_status_string(st)
     return {"ms": a.elapsed_time(b), "h2d": n * T * C * 2,
-            "d2h": sum(t.numel() * t.element_size() for t in outs)}
+            "d2h": sum(t.numel() * t.element_size() for t in outs), "chunks": nch}
 
 
 def run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, status):

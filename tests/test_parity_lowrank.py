@@ -116,7 +116,11 @@ def test_small_lowrank_trajectory():
 
 
 @pytest.mark.parametrize("T,C,r,iters", [(100, 200, 5, 1), (300, 136, 16, 3), (77, 64, 33, 2),
-                                         (640, 512, 64, 2), (1000, 1000, 32, 2)])
+                                         (640, 512, 64, 2), (1000, 1000, 32, 2),
+                                         (64, 8, 1, 1),        # rank 1, the narrowest rows
+                                         (40, 64, 8, 16),      # the most iterations
+                                         (33, 264, 32, 2),     # barely more tokens than the rank
+                                         (17550, 1920, 32, 2)])  # 138 token tiles per Gram
 def test_lowrank_ragged_shapes(T, C, r, iters):
     wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r, iters=iters)
     _run(wl, 3)
