@@ -265,14 +265,15 @@ cf_status launch_apply_tc(const LrBatch &B, const Layout &L, int n, cudaStream_t
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return CF_ERR_CUDA;
     // Token tiles per CTA: enough CTAs for two waves of resident CTAs, and
-    // up to kApplyMaxTilesPerCta tiles each so the per-CTA set-up (TMEM,
+    // up to apply_max_tiles_per_cta tiles each so the per-CTA set-up (TMEM,
     // A operand, first product) is amortised.
     const int64_t ncb = (L.C + 127) / 128, ntt = (L.T + 127) / 128;
     const int64_t tiles = ncb * ntt * n;
     const int64_t slots = (int64_t)sm_count() * (KP <= 32 ? 2 : 1);
     int64_t tpc = tiles / (2 * slots);
     if (tpc < 1) tpc = 1;
-    if (tpc > cf::umma::kApplyMaxTilesPerCta) tpc = cf::umma::kApplyMaxTilesPerCta;
+    constexpr int max_tpc = cf::umma::apply_max_tiles_per_cta<SENDER>();
+    if (tpc > max_tpc) tpc = max_tpc;
     dim3 grid((unsigned)ncb, (unsigned)((ntt + tpc - 1) / tpc), (unsigned)n);
     k<<<grid, cf::umma::kApplyThreads, smem, st>>>(B, L, (int)tpc);
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;

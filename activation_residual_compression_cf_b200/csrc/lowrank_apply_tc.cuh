@@ -81,9 +81,16 @@ __host__ __device__ constexpr int apply_stage_tok() {
 }
 constexpr int kApplyConsumers = 256;            // 8 warps: 4 channel quarters x 2 token halves
 constexpr int kApplyProducerWarp = kApplyConsumers / 32;   // warp 8: bulk copies
-constexpr int kApplyMmaWarp = kApplyProducerWarp + 1;      // warp 9: B operands + MMAs
-constexpr int kApplyThreads = kApplyConsumers + 64;
-constexpr int kApplyMaxTilesPerCta = 8;
+constexpr int kApplyMmaWarp = kApplyProducerWarp + 1;      // warps 9, 10: B operands;
+constexpr int kApplyBuilders = 64;                          // warp 9 also issues the MMAs
+constexpr int kApplyThreads = kApplyConsumers + 32 + kApplyBuilders;
+// Token tiles per CTA at most: the receiver's tiles carry half the bytes of
+// the sender's, so it takes twice as many to amortise a CTA's set-up
+// (measured on B200: 16 tiles gave the receiver 0.92 of HBM against 0.89).
+template <bool SENDER>
+__host__ __device__ constexpr int apply_max_tiles_per_cta() {
+    return SENDER ? 8 : 16;
+}
 
 template <bool SENDER>
 __host__ __device__ constexpr int apply_stage_bytes() {
@@ -107,9 +114,13 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-// consumers + the MMA warp, once, after the first operands are built
+// consumers + the builder warps, once, after the first operands are built
 __device__ __forceinline__ void operand_sync() {
-    asm volatile("bar.sync 1, %0;" ::"r"(kApplyConsumers + 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"r"(kApplyConsumers + kApplyBuilders) : "memory");
+}
+// the two builder warps, once per token tile
+__device__ __forceinline__ void builder_sync() {
+    asm volatile("bar.sync 2, %0;" ::"r"(kApplyBuilders) : "memory");
 }
 
 // B operand of one token tile: b[t][k] = qP[t][k] * s[k] (s[k] = sP[k] sQ[k],
@@ -165,26 +176,27 @@ __device__ __forceinline__ void apply_b_row(uint8_t *gbh, uint8_t *gbl, const ui
 template <int KP>
 __device__ __forceinline__ void apply_build_b_warp(uint8_t *gbh, uint8_t *gbl, const uint8_t *pc,
                                                    const float *sk, int64_t t0, int64_t T, int r,
-                                                   int nb, int lane) {
+                                                   int nb, int lane, int part) {
     constexpr int NW = KP / 8;                 // 32-bit words of codes per row (at most)
-    constexpr int RPL = kApplyTile / 32;       // rows per lane
+    constexpr int NP = kApplyBuilders / 32;    // builder warps
+    constexpr int RPL = kApplyTile / 32 / NP;  // rows per lane: lane + 32 (NP rr + part)
     const bool words = (nb & 3) == 0 && (reinterpret_cast<uintptr_t>(pc) & 3u) == 0;
     if (words) {
         const int nw = nb >> 2;
         uint32_t w[RPL][NW];
 #pragma unroll
         for (int rr = 0; rr < RPL; ++rr) {
-            const int64_t t = t0 + lane + 32 * rr;
+            const int64_t t = t0 + lane + 32 * (NP * rr + part);
             const uint32_t *src = reinterpret_cast<const uint32_t *>(pc + t * nb);
 #pragma unroll
             for (int j = 0; j < NW; ++j) w[rr][j] = (t < T && j < nw) ? __ldg(src + j) : 0u;
         }
 #pragma unroll
-        for (int rr = 0; rr < RPL; ++rr) apply_b_row<KP>(gbh, gbl, w[rr], sk, lane + 32 * rr, r);
+        for (int rr = 0; rr < RPL; ++rr) apply_b_row<KP>(gbh, gbl, w[rr], sk, lane + 32 * (NP * rr + part), r);
     } else {
 #pragma unroll 1
         for (int rr = 0; rr < RPL; ++rr) {
-            const int64_t t = t0 + lane + 32 * rr;
+            const int64_t t = t0 + lane + 32 * (NP * rr + part);
             const uint8_t *src = pc + t * nb;
             uint32_t w[NW];
 #pragma unroll
@@ -192,15 +204,15 @@ __device__ __forceinline__ void apply_build_b_warp(uint8_t *gbh, uint8_t *gbl, c
 #pragma unroll
             for (int j = 0; j < 4 * NW; ++j)
                 if (t < T && j < nb) w[j >> 2] |= (uint32_t)__ldg(src + j) << (8 * (j & 3));
-            apply_b_row<KP>(gbh, gbl, w, sk, lane + 32 * rr, r);
+            apply_b_row<KP>(gbh, gbl, w, sk, lane + 32 * (NP * rr + part), r);
         }
     }
 }
 
 // Persistent over a run of token tiles: CTA (x, y, z) owns channel block x of
-// buffer z and token tiles [y * tpc, (y + 1) * tpc).  Warp roles (320
+// buffer z and token tiles [y * tpc, (y + 1) * tpc).  Warp roles (352
 // threads):
-//   warps 0-7 : with warp 9, build the A operand (Q codes of the channel
+//   warps 0-7 : with warps 9-10, build the A operand (Q codes of the channel
 //               block) and tile 0's B operand; then each warp combines one
 //               channel quarter (w % 4, its TMEM lanes) x one half (w / 4) of
 //               every 16-token stage of every tile, reading x and recon from
@@ -209,10 +221,11 @@ __device__ __forceinline__ void apply_build_b_warp(uint8_t *gbh, uint8_t *gbl, c
 //               of every token row's 128-channel segment of recon (and x) of
 //               all the CTA's tiles into the ring, from the kernel's first
 //               instructions on;
-//   warp 9    : for tile i, once tile i-1's product is done (its commit
-//               barrier) writes tile i's B operand (single buffer), and once
-//               the consumers have released accumulator i % 2 (tile i-2
-//               combined) issues the MMAs of tile i into it.
+//   warps 9-10: for tile i, once tile i-1's product is done (its commit
+//               barrier) write tile i's B operand (single buffer, half the
+//               rows each), and once the consumers have released accumulator
+//               i % 2 (tile i-2 combined) warp 9 issues the MMAs of tile i
+//               into it.
 // So the consumers never wait on operand building: the product of the next
 // tile is formed while the current one is combined.
 // Every wait is bounded; on expiry CF_ERR_TIMEOUT goes to the buffer's status
@@ -252,6 +265,7 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
     const uint32_t mma0 = bars, accf0 = bars + 16u, full0 = bars + 32u, empty0 = bars + 32u + 8u * S;
     float *sk = reinterpret_cast<float *>(gring + S * SB + 8 * (4 + 2 * S));   // [KP]
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sk + KP);
+    int *abort_flag = reinterpret_cast<int *>(tslot + 1);   // builder warps give up together
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t c0 = (int64_t)blockIdx.x * kApplyTile;
@@ -273,6 +287,7 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
             mbar_init(full0 + 8u * s, 1);                        // producer + tx bytes
             mbar_init(empty0 + 8u * s, kApplyConsumers / 32);    // one per consumer warp
         }
+        *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (tid < KP) sk[tid] = tid < r ? __fmul_rn(__ldg(ps + tid), __ldg(qs + tid)) : 0.0f;
@@ -326,8 +341,8 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
     } else {
         // A = the INT4 codes of Q for this channel block, and tile 0's B:
         // built once by the consumers and the MMA warp together.
-        const int ot = warp == kApplyMmaWarp ? kApplyConsumers + lane : tid;
-        constexpr int kOpThreads = kApplyConsumers + 32;
+        const int ot = warp >= kApplyMmaWarp ? kApplyConsumers + 32 * (warp - kApplyMmaWarp) + lane : tid;
+        constexpr int kOpThreads = kApplyConsumers + kApplyBuilders;
         for (int idx = ot; idx < kApplyTile * (KP / 4); idx += kOpThreads) {
             const int row = idx / (KP / 4), k0 = (idx - row * (KP / 4)) * 4;
             const int64_t c = c0 + row;
@@ -345,29 +360,35 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
         operand_sync();
         fence_after_sync();
 
-        if (warp == kApplyMmaWarp) {
+        if (warp >= kApplyMmaWarp) {
             // ---------------- B operands and MMAs ----------------
+            // Both builder warps reach builder_sync exactly once per tile and
+            // leave together on a shared flag, so a bounded wait that gives
+            // up in one of them cannot strand the other at the barrier.
+            const int part = warp - kApplyMmaWarp;
             const int ksteps = (r + 7) / 8;
             constexpr uint32_t idesc = idesc_tf32(kApplyTile);
             for (int i = 0; i < nt; ++i) {
+                bool ok = true;
                 if (i > 0) {
                     // tile i-1's product has read the B buffer
-                    if (!__all_sync(kFullMask, mbar_wait(mma0 + 8u * ((i - 1) & 1), (uint32_t)(((i - 1) >> 1) & 1)))) {
-                        if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
-                        break;
-                    }
-                    apply_build_b_warp<KP>(gb + OPB, gb + 2 * OPB, pc, sk, tbeg + (int64_t)i * kApplyTile,
-                                           T, r, nb, lane);
+                    ok = __all_sync(kFullMask, mbar_wait(mma0 + 8u * ((i - 1) & 1), (uint32_t)(((i - 1) >> 1) & 1)));
+                    if (ok)
+                        apply_build_b_warp<KP>(gb + OPB, gb + 2 * OPB, pc, sk, tbeg + (int64_t)i * kApplyTile,
+                                               T, r, nb, lane, part);
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 }
                 // accumulator i % 2 is free once tile i-2 has been combined
-                if (i >= 2 && !__all_sync(kFullMask, mbar_wait(accf0 + 8u * (i & 1), (uint32_t)(((i - 2) >> 1) & 1)))) {
-                    if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
-                    break;
+                if (ok && i >= 2)
+                    ok = __all_sync(kFullMask, mbar_wait(accf0 + 8u * (i & 1), (uint32_t)(((i - 2) >> 1) & 1)));
+                if (!ok && lane == 0) {
+                    *(volatile int *)abort_flag = 1;
+                    if (status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
                 }
-                __syncwarp();
+                builder_sync();
+                if (*(volatile int *)abort_flag) break;
                 fence_after_sync();
-                if (lane == 0) {
+                if (part == 0 && lane == 0) {
                     const uint32_t acc = tmem + (uint32_t)(128 * (i & 1));
                     for (int kk = 0; kk < ksteps; ++kk) {
                         const uint32_t off = (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32);
