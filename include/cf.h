@@ -108,6 +108,12 @@ typedef struct cf_dec_emit_buffer {
     uint16_t *out;       /* bf16 [T][C], written: bf16_rne(new recon_r)     */
 } cf_dec_emit_buffer;
 
+/* Streams and graphs: every call except cf_lowrank_status only enqueues
+ * work on the given stream (no allocation, no synchronisation, no host read
+ * of device memory), so a step of batched calls can be captured into a CUDA
+ * graph and replayed; the host-side argument checks run at capture time.
+ * cf_lowrank_encode_noalloc's first call on a device must precede capture. */
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *cf_status_string(cf_status s);
 
