@@ -188,6 +188,30 @@ cf_status launch_project(const LrBatch &B, const Layout &L, int n, cudaStream_t 
 }
 
 template <int BN>
+cf_status launch_project_residual(const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
+    CUtensorMap mq;
+    if (!make_map(&mq, B.ws + L.off_qt, L.C, L.rp, L.C, n, B.ws_stride, BN)) return CF_ERR_CUDA;
+    auto k = cf::umma::project_residual_kernel<BN>;
+    const int smem = cf::umma::StageGeom<BN>::kSmem;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return CF_ERR_CUDA;
+    dim3 grid((unsigned)L.nTileT, 1, (unsigned)n);
+    k<<<grid, cf::umma::kFusedThreads, smem, st>>>(mq, B, L);
+    return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
+}
+
+// First projection of a tensor-core encode, fused with the residual.
+cf_status project_residual(const LrBatch &B, const Layout &L, int n, cudaStream_t st) {
+    switch (L.rp) {
+        case 16: return launch_project_residual<16>(B, L, n, st);
+        case 32: return launch_project_residual<32>(B, L, n, st);
+        case 48: return launch_project_residual<48>(B, L, n, st);
+        case 64: return launch_project_residual<64>(B, L, n, st);
+    }
+    return CF_ERR_UNSUPPORTED;
+}
+
+template <int BN>
 cf_status launch_backproject(const LrBatch &B, const Layout &L, int n, bool last, cudaStream_t st) {
     CUtensorMap mv, mp;
     if (!make_map(&mv, B.ws + L.off_vb, L.C, L.T, L.C, n, B.ws_stride, 64) ||
@@ -321,15 +345,19 @@ cf_status apply(bool sender, const LrBatch &B, const Layout &L, int n, cudaStrea
 // The whole sender for n buffers (n = 1 for the single-buffer call).
 cf_status encode_impl(const cf_desc *d, const Layout &L, int n, const LrBatch &B, cudaStream_t st) {
     const int nb = (L.r + 1) / 2;
+    const bool fused = g_engine.load() == 0;
     cf::lr_prep_kernel<<<(unsigned)n, 128, 0, st>>>(B, L);
     LR_LAUNCHED();
     {
-        const int64_t groups = L.T * L.C / 8;
-        int64_t blocks = (groups + 255) / 256;
-        const int64_t cap = (int64_t)sm_count() * 8 / n + 1;
-        if (blocks > cap) blocks = cap;
-        cf::lr_residual_kernel<<<dim3((unsigned)blocks, 1, (unsigned)n), 256, 0, st>>>(B, L);
-        LR_LAUNCHED();
+        // tensor-core engine: the first projection forms Vb itself
+        if (!fused) {
+            const int64_t groups = L.T * L.C / 8;
+            int64_t blocks = (groups + 255) / 256;
+            const int64_t cap = (int64_t)sm_count() * 8 / n + 1;
+            if (blocks > cap) blocks = cap;
+            cf::lr_residual_kernel<<<dim3((unsigned)blocks, 1, (unsigned)n), 256, 0, st>>>(B, L);
+            LR_LAUNCHED();
+        }
         const int64_t nq = (int64_t)L.rp * L.C;
         cf::lr_omega_kernel<<<dim3((unsigned)((nq + 255) / 256), 1, (unsigned)n), 256, 0, st>>>(B, L);
         LR_LAUNCHED();
@@ -337,12 +365,13 @@ cf_status encode_impl(const cf_desc *d, const Layout &L, int n, const LrBatch &B
     // Tensor-core engine: each projection CTA accumulates its whole K range,
     // so the projection also forms G and factors it (last tile of the
     // buffer) and the back-projection writes Q's transpose and maxima: an
-    // iteration is three launches.  CUDA-core engine: split-K partials with
-    // separate Gram / Cholesky and Q-reduction kernels.
-    const bool fused = g_engine.load() == 0;
+    // iteration is three launches, and the first projection also forms the
+    // bf16 residual (no separate residual pass).  CUDA-core engine: the
+    // residual kernel, split-K partials with separate Gram / Cholesky and
+    // Q-reduction kernels.
     for (int it = 0; it < d->iters; ++it) {
         const bool last = (it == d->iters - 1);
-        LR_TRY(project(B, L, n, st));
+        LR_TRY(it == 0 && fused ? project_residual(B, L, n, st) : project(B, L, n, st));
         if (!fused) {
             cf::lr_gram_chol_kernel<<<dim3((unsigned)L.nGram, 1, (unsigned)n), 256, 0, st>>>(B, L);
             LR_LAUNCHED();

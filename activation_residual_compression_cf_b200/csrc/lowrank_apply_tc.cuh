@@ -111,9 +111,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
 // consumers + the builder warps, once, after the first operands are built
 __device__ __forceinline__ void operand_sync() {
     asm volatile("bar.sync 1, %0;" ::"r"(kApplyConsumers + kApplyBuilders) : "memory");

@@ -64,6 +64,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 // Bounded wait for the completion of phase `parity`; false on expiry.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     for (uint32_t i = 0; i < kWaitLimit; ++i)
@@ -318,6 +322,12 @@ __device__ __forceinline__ void gemm_tile(const CUtensorMap *mapA, const CUtenso
 // and 1/diag(R) (fp32 [rp], 0 where dead).  The ticket is reset by its last
 // user.  The pipeline's shared memory is reused: every stage has been
 // consumed once the tile's product is done.
+// The tail runs on the first 128 threads of the CTA (all of them in the
+// plain projection, the four converter warps in the fused one).
+__device__ __forceinline__ void tail_sync() {
+    asm volatile("bar.sync 3, 128;" ::: "memory");
+}
+
 template <int BN>
 __device__ __forceinline__ void project_tail(const cf_lowrank::LrBatch &B, const cf_lowrank::Layout &L,
                                              int bz, int tile) {
@@ -350,7 +360,7 @@ __device__ __forceinline__ void project_tail(const cf_lowrank::LrBatch &B, const
         for (int q = 0; q < BN / 4; ++q)
             *reinterpret_cast<float4 *>(ys + tid * LDY + 4 * q) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    __syncthreads();
+    tail_sync();
 
     // The tile's partial Gram Y^T Y on the fp64 tensor path (mma.sync
     // m8n8k4 f64; tcgen05 has no fp64 kind): 8 x 8 output blocks (I, J),
@@ -404,10 +414,10 @@ __device__ __forceinline__ void project_tail(const cf_lowrank::LrBatch &B, const
     }
     double *gp = B.at<double>(bz, L.off_gp);
     __threadfence();
-    __syncthreads();
+    tail_sync();
     uint32_t *fin = B.at<uint32_t>(bz, L.off_status) + cf_lowrank::kTicketWord;
     if (tid == 0) is_last = atomicAdd(fin, 1u) == (uint32_t)(L.nTileT - 1) ? 1 : 0;
-    __syncthreads();
+    tail_sync();
     if (!is_last) return;
     __threadfence();
 
@@ -427,13 +437,13 @@ __device__ __forceinline__ void project_tail(const cf_lowrank::LrBatch &B, const
         A[i * ld + j] = v;
         if (i == j) gdiag[i] = v;
     }
-    __syncthreads();
+    tail_sync();
     if (BN <= 32) {
         quad_cholesky(A, ld, r, gdiag, dead, invd, rowbuf);   // all 128 threads
     } else if (tid < 32) {
         warp_cholesky_smem(A, ld, r, gdiag, dead, invd);
     }
-    __syncthreads();
+    tail_sync();
     float *rmat = B.at<float>(bz, L.off_rmat);
     float *rinvd = rmat + BN * BN;
     int nd = 0;
@@ -527,6 +537,197 @@ backproject_kernel(const __grid_constant__ CUtensorMap mapVt, const __grid_const
     gemm_tile<BN, true>(&mapVt, &mapPt, c0, 0, nkb, bz, B.at<float>(bz, L.off_q), L.C,
                         B.at<int32_t>(bz, L.off_status) + cf_lowrank::kStatusWord);
     backproject_tail<BN>(B, L, bz, blockIdx.x, want_amax);
+}
+
+// First projection of an encode, fused with the residual: Y = Vb Q with
+// Vb = bf16((float)x - recon) formed here from the caller's x and recon
+// instead of being read back from the workspace.  One CTA per 128-token tile
+// over all channels (no split-K), 160 threads:
+//   warps 0-7 (converters): for every 64-channel k-block, coalesced loads of
+//     the tile's x (bf16) and recon (fp32) rows (16 rows per warp, all its
+//     loads in flight), v = x - recon rounded once to fp32 and once to bf16
+//     (the residual kernel's arithmetic), written into the ring's
+//     128-byte-swizzled A tile and to the workspace copy Vb that the later
+//     passes read; warps 0-3 then run the epilogue (Y rows from TMEM) and the
+//     tile's Gram / the buffer's Cholesky (project_tail);
+//   warp 8: allocates TMEM; one lane TMA-loads the Qt tiles (no multicast)
+//     and issues tcgen05.mma (kind::f16) per k-block; commits release slots.
+// Every wait is bounded; on expiry CF_ERR_TIMEOUT goes to the buffer's status
+// word, the loops end, and TMEM is freed.
+constexpr int kFusedConverters = 8;                        // warps 0-7
+constexpr int kFusedThreads = 32 * kFusedConverters + 32;  // + warp 8
+
+template <int BN>
+__global__ void __launch_bounds__(kFusedThreads, 2)
+project_residual_kernel(const __grid_constant__ CUtensorMap mapQt, const cf_lowrank::LrBatch B,
+                        const cf_lowrank::Layout L) {
+    using G = StageGeom<BN>;
+    const int bz = blockIdx.z;
+    if (B.at<int32_t>(bz, L.off_status)[cf_lowrank::kSkipWord]) return;
+    const cf_lowrank::LrPtrs pp = B.get(bz);
+    const int64_t T = L.T, C = L.C;
+    const int64_t t0 = (int64_t)blockIdx.x * 128;
+    const int nkb = (int)((C + kBK - 1) / kBK);
+    int32_t *status = B.at<int32_t>(bz, L.off_status) + cf_lowrank::kStatusWord;
+    bf16 *vb = B.at<bf16>(bz, L.off_vb);
+
+    extern __shared__ uint8_t dsmem[];
+    const uint32_t base = (smem_u32(dsmem) + 1023u) & ~1023u;
+    uint8_t *gbase = dsmem + (base - smem_u32(dsmem));
+    // barriers: a_full[S] (4 converter warps), b_full[S] (tx), empty[S]
+    // (commit), done (commit)
+    const uint32_t bars = base + kStages * G::kBytes;
+    auto a_full = [&](int q) { return bars + 8u * q; };
+    auto b_full = [&](int q) { return bars + 8u * (kStages + q); };
+    auto empty = [&](int q) { return bars + 8u * (2 * kStages + q); };
+    const uint32_t done = bars + 8u * (3 * kStages);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + kStages * G::kBytes + 8 * (3 * kStages + 1));
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int q = 0; q < kStages; ++q) {
+            mbar_init(a_full(q), kFusedConverters);
+            mbar_init(b_full(q), 1);
+            mbar_init(empty(q), 1);
+        }
+        mbar_init(done, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == kFusedConverters) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(G::kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    bool have = false;
+    if (warp == kFusedConverters) {
+        if (lane == 0) {
+            auto load_b = [&](int kb) {
+                const int q = kb % kStages;
+                mbar_expect_tx(b_full(q), (uint32_t)G::kBytesB);
+                tma_load_3d(base + q * G::kBytes + kTileBytesA, &mapQt, b_full(q), kb * kBK, 0, bz);
+            };
+            for (int kb = 0; kb < nkb && kb < kStages; ++kb) load_b(kb);
+            constexpr uint32_t idesc = idesc_bf16(BN, false);
+            bool ok = true;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int q = kb % kStages;
+                const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+                if (!mbar_wait(a_full(q), ph) || !mbar_wait(b_full(q), ph)) {
+                    ok = false;
+                    break;
+                }
+                fence_after_sync();
+                const uint32_t sa = base + q * G::kBytes, sb = sa + kTileBytesA;
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk)
+                    mma_bf16(tmem, sw128_desc(sa + kk * 32u, 16, 1024), sw128_desc(sb + kk * 32u, 16, 1024),
+                             idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(empty(q));
+                if (kb + kStages < nkb) {
+                    // this slot's B is read once its product is done
+                    if (!mbar_wait(empty(q), ph)) {
+                        ok = false;
+                        break;
+                    }
+                    load_b(kb + kStages);
+                }
+            }
+            if (ok)
+                mma_commit(done);
+            else
+                atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else {
+        // converters: warp w owns rows 16 w .. 16 w + 15 of the tile; one
+        // warp-wide load covers two rows (16 lanes x 4 channels each)
+        const int sub = lane >> 4, cl = (lane & 15) * 4;   // row within a pair, channel offset
+        bool ok = true;
+        for (int kb = 0; kb < nkb && ok; ++kb) {
+            const int q = kb % kStages;
+            if (kb >= kStages)
+                ok = __all_sync(kFullMask, mbar_wait(empty(q), (uint32_t)((kb / kStages - 1) & 1)));
+            if (!ok) break;
+            const int64_t c = (int64_t)kb * kBK + cl;
+            const bool cok = c < C;                  // C % 8 == 0: all 4 channels or none
+            uint8_t *sa = gbase + q * G::kBytes;
+            uint2 xw[8];
+            float4 rw[8];
+#pragma unroll
+            for (int pr = 0; pr < 8; ++pr) {
+                const int64_t t = t0 + 16 * warp + 2 * pr + sub;
+                if (cok && t < T) {
+                    xw[pr] = __ldcs(reinterpret_cast<const uint2 *>(pp.x + t * C + c));
+                    rw[pr] = __ldcs(reinterpret_cast<const float4 *>(pp.recon + t * C + c));
+                } else {
+                    xw[pr] = make_uint2(0u, 0u);
+                    rw[pr] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+#pragma unroll
+            for (int pr = 0; pr < 8; ++pr) {
+                const int row = 16 * warp + 2 * pr + sub;
+                const int64_t t = t0 + row;
+                const float v0 = __fsub_rn(bf16_bits_to_f32(xw[pr].x & 0xffffu), rw[pr].x);
+                const float v1 = __fsub_rn(bf16_bits_to_f32(xw[pr].x >> 16), rw[pr].y);
+                const float v2 = __fsub_rn(bf16_bits_to_f32(xw[pr].y & 0xffffu), rw[pr].z);
+                const float v3 = __fsub_rn(bf16_bits_to_f32(xw[pr].y >> 16), rw[pr].w);
+                const __nv_bfloat162 h0 = __floats2bfloat162_rn(v0, v1);
+                const __nv_bfloat162 h1 = __floats2bfloat162_rn(v2, v3);
+                const uint2 w = make_uint2(*reinterpret_cast<const uint32_t *>(&h0),
+                                           *reinterpret_cast<const uint32_t *>(&h1));
+                // 128-byte swizzle: 16-byte chunk j of row `row` sits at
+                // chunk j ^ (row & 7); this lane's 8 bytes are half a chunk
+                const int chunk = (cl >> 3) ^ (row & 7);
+                *reinterpret_cast<uint2 *>(sa + row * 128 + chunk * 16 + (cl & 4) * 2) = w;
+                if (cok && t < T) *reinterpret_cast<uint2 *>(vb + t * C + c) = w;
+            }
+            // generic writes of the A tile before the tensor cores read it
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(a_full(q));
+        }
+        if (!ok && lane == 0) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+        // epilogue (warps 0-3): TMEM lane 32 w + i holds Y row t0 + 32 w + i
+        if (warp < 4) have = __all_sync(kFullMask, ok && mbar_wait(done, 0));
+        if (have) {
+            fence_after_sync();
+            const int64_t row = t0 + 32 * warp + lane;
+            const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
+            float *y = B.at<float>(bz, L.off_y);
+#pragma unroll
+            for (int cc = 0; cc < BN; cc += 16) {
+                float v[16];
+                tmem_ld16(taddr + cc, v);
+                if (row < T) {
+                    float4 *dst = reinterpret_cast<float4 *>(y + row * BN + cc);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        dst[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                }
+            }
+        }
+    }
+    // every TMEM read is done: free it (the tail below uses only shared and
+    // global memory)
+    fence_before_sync();
+    __syncthreads();
+    if (warp == kFusedConverters) {
+        fence_after_sync();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(G::kTmemCols)
+                     : "memory");
+        return;
+    }
+    if (warp >= 4) return;   // the tail runs on warps 0-3
+    project_tail<BN>(B, L, bz, blockIdx.x);
 }
 
 }  // namespace umma
