@@ -555,11 +555,11 @@ def run_lowrank(args, world, rank, local):
     app_enc_bytes = enc_bytes + fac_bytes
     app_dec_bytes = dec_bytes + fac_bytes
     status = max(cf.cf_lowrank_status(ws[b * wsb:]) for b in range(n))
-    # Launches per step: the sender runs prep, residual, omega, three kernels
-    # per subspace iteration (project with its Gram/Cholesky tail,
-    # orthogonalise, back-project with its Q-reduction tail), two INT4 packs
-    # and the apply; the receiver one.
-    launches_per_step = 6 + 3 * it + 1
+    # Launches per step: the sender runs prep, omega, three kernels per
+    # subspace iteration (project with its Gram/Cholesky tail -- the first
+    # one also forms the bf16 residual --, orthogonalise, back-project with
+    # its Q-reduction tail), two INT4 packs and the apply; the receiver one.
+    launches_per_step = 5 + 3 * it + 1
 
     e2e = None
     if not args.no_e2e:
