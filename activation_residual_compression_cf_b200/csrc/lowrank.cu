@@ -5,16 +5,21 @@
 // style subspace iteration; "Measured effects" -- 2 vs 10 iterations).
 //
 // Per buffer and step, with V = (float)x - recon_s:
-//   Vb  = bf16(V)                       one pass over x, recon (8 B/elem)
-//   Qt  = bf16(Omega)^T                 [rp][C], K-major B operand
+//   Vb  = bf16(V)                       formed by the first projection from
+//                                       x and recon (tensor cores), or by a
+//                                       residual pass (CUDA cores)
+//   Qt  = bf16(Omega)^T                 [rp][C], K-major B operand (or the
+//                                       previous encode's, warm start)
 //   repeat iters:
-//     Y    = Vb Q          (split over channel ranges, fp32 partials)
-//     G    = Y^T Y         (fp64), R = chol(G), Rinv = R^-1
-//     P    = Y Rinv        (fp32 [T][rp], bf16 copy Pt [rp][Tp])
-//     Q    = Vb^T P        (split over token ranges, fp32 partials)
+//     Y    = Vb Q          128-token tiles over all channels; tile Grams
+//     G    = Y^T Y         (fp64, summed in tile order), R = chol(G)
+//     P    = Y R^-1        (fp32 [T][rp], bf16 copy Pt [rp][Tp])
+//     Q    = Vb^T P        128-channel blocks over all tokens
 //   INT4 per column of P and Q, packed
 //   D = (qP sP)(qQ sQ)^T ; err = V - D ; recon_s += D     (exact fp32 V)
-// The receiver adds the same D, formed by the same device routine.
+// The receiver adds the same D, formed by the same device routine.  The
+// CUDA-core engine (cross-checks) splits the two products over K and sums
+// the partials in fixed order instead.
 //
 // The workspace is caller-allocated (cf_lowrank_workspace_bytes); its
 // layout is computed here from (T, C, r).

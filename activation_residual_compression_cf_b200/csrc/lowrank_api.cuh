@@ -12,8 +12,8 @@ namespace cf_lowrank {
 constexpr int kMaxRank = 64;
 constexpr int kMaxIters = 16;
 
-constexpr int64_t kChunkA = 512;   // channels per split of the Y = V Q pass
-constexpr int64_t kChunkB = 512;   // tokens per split of the Q = V^T P pass
+constexpr int64_t kChunkA = 512;   // channels per split of Y = V Q (CUDA-core engine)
+constexpr int64_t kChunkB = 512;   // tokens per split of Q = V^T P (CUDA-core engine)
 constexpr int kGramTok = 32;       // tokens per Gram CTA
 constexpr int kGramGroup = 16;     // Gram partial blocks summed per first-level group
 constexpr int kApplyTok = 32;      // D tile: tokens

@@ -10,7 +10,7 @@
 // partial Gram and the buffer's last tile factors G; the back-projection's
 // tail writes the bf16 transpose and the column maxima.
 //
-// One CTA of 4 warps per output tile and K split:
+// One CTA of 4 warps per output tile:
 //   warp 0, one lane : TMA producer (cp.async.bulk.tensor, no multicast) into
 //                      a 4-stage ring of 128-byte-swizzled shared tiles
 //   warp 1           : allocates TMEM; one lane issues tcgen05.mma
@@ -18,6 +18,8 @@
 //                      tcgen05.commit releases each stage
 //   all 4 warps      : epilogue, tcgen05.ld 32 lanes x rp columns per warp,
 //                      one output row per thread, 16-byte stores
+// The first projection of an encode has its own kernel
+// (project_residual_kernel, below) that forms Vb from x and recon itself.
 // Every mbarrier wait is bounded; on expiry the kernel records
 // CF_ERR_TIMEOUT in the status word, stops issuing work, frees its TMEM and
 // returns.
@@ -185,7 +187,7 @@ struct StageGeom {
 // Common CTA skeleton.  A_MN: A operand is MN-major (backproject).
 //   rows0      : first output row of this tile (token for project, channel
 //                for backproject); TMA y (project) / x (backproject) base
-//   kbeg, nkb  : first K element of this split and number of 64-wide blocks
+//   kbeg, nkb  : first K element and number of 64-wide K blocks
 template <int BN, bool A_MN>
 __device__ __forceinline__ void gemm_tile(const CUtensorMap *mapA, const CUtensorMap *mapB,
                                           int32_t rows0, int32_t kbeg, int nkb, int32_t zb,
@@ -542,7 +544,7 @@ backproject_kernel(const __grid_constant__ CUtensorMap mapVt, const __grid_const
 // First projection of an encode, fused with the residual: Y = Vb Q with
 // Vb = bf16((float)x - recon) formed here from the caller's x and recon
 // instead of being read back from the workspace.  One CTA per 128-token tile
-// over all channels (no split-K), 160 threads:
+// over all channels (no split-K), 288 threads:
 //   warps 0-7 (converters): for every 64-channel k-block, coalesced loads of
 //     the tile's x (bf16) and recon (fp32) rows (16 rows per warp, all its
 //     loads in flight), v = x - recon rounded once to fp32 and once to bf16
