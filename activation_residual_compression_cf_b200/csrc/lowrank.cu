@@ -197,7 +197,7 @@ cf_status launch_project_residual(const LrBatch &B, const Layout &L, int n, cuda
     CUtensorMap mq;
     if (!make_map(&mq, B.ws + L.off_qt, L.C, L.rp, L.C, n, B.ws_stride, BN)) return CF_ERR_CUDA;
     auto k = cf::umma::project_residual_kernel<BN>;
-    const int smem = cf::umma::StageGeom<BN>::kSmem;
+    const int smem = cf::umma::FusedGeom<BN>::kSmem;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return CF_ERR_CUDA;
     dim3 grid((unsigned)L.nTileT, 1, (unsigned)n);

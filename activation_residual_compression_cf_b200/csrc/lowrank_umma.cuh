@@ -544,26 +544,59 @@ backproject_kernel(const __grid_constant__ CUtensorMap mapVt, const __grid_const
 // First projection of an encode, fused with the residual: Y = Vb Q with
 // Vb = bf16((float)x - recon) formed here from the caller's x and recon
 // instead of being read back from the workspace.  One CTA per 128-token tile
-// over all channels (no split-K), 288 threads:
-//   warps 0-7 (converters): for every 64-channel k-block, coalesced loads of
-//     the tile's x (bf16) and recon (fp32) rows (16 rows per warp, all its
-//     loads in flight), v = x - recon rounded once to fp32 and once to bf16
-//     (the residual kernel's arithmetic), written into the ring's
-//     128-byte-swizzled A tile and to the workspace copy Vb that the later
-//     passes read; warps 0-3 then run the epilogue (Y rows from TMEM) and the
-//     tile's Gram / the buffer's Cholesky (project_tail);
+// over all channels (no split-K), 288 threads, one CTA per SM:
+//   warps 0-7 (converters): warp w owns rows 16 w .. 16 w + 15 of the tile.
+//     For each 64-channel k-block it copies its rows' x (bf16) and recon
+//     (fp32) segments into a stage of a 4-deep shared ring with 16-byte
+//     asynchronous copies (cp.async, zero-filled past T and C), issued four
+//     k-blocks ahead so the loads never wait on the arithmetic; then it forms
+//     v = x - recon (rounded once to fp32, once to bf16: the residual
+//     kernel's arithmetic) and writes it in place over the stage's x rows in
+//     the 128-byte-swizzled layout the tensor cores read (a row's 16-byte
+//     chunks only permute within that row, and the warp owns its rows), and
+//     to the workspace copy Vb for the later passes.  Warps 0-3 then run the
+//     epilogue (Y rows from TMEM) and the tile's Gram / the buffer's Cholesky
+//     (project_tail);
 //   warp 8: allocates TMEM; one lane TMA-loads the Qt tiles (no multicast)
-//     and issues tcgen05.mma (kind::f16) per k-block; commits release slots.
+//     and issues tcgen05.mma (kind::f16) per k-block; commits release stages.
 // Every wait is bounded; on expiry CF_ERR_TIMEOUT goes to the buffer's status
 // word, the loops end, and TMEM is freed.
 constexpr int kFusedConverters = 8;                        // warps 0-7
 constexpr int kFusedThreads = 32 * kFusedConverters + 32;  // + warp 8
+constexpr int kFusedStages = 4;
+constexpr int kFusedX = 128 * 128;                         // x / A tile: 128 rows x 128 B
+constexpr int kFusedR = 128 * 256;                         // recon tile: 128 rows x 256 B
 
 template <int BN>
-__global__ void __launch_bounds__(kFusedThreads, 2)
+struct FusedGeom {
+    static constexpr int kBytesB = BN * kBK * 2;
+    static constexpr int kStage = kFusedX + kFusedR + kBytesB;   // multiple of 1 KB
+    static constexpr int kSmem = kFusedStages * kStage + 1024 + 256;
+    static constexpr uint32_t kTmemCols = BN <= 32 ? 32 : 64;
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+    // src-size 0 writes 16 zero bytes and reads nothing
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// wait until at most kFusedStages - 1 groups of this thread are in flight
+__device__ __forceinline__ void cp_async_wait_oldest() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(kFusedStages - 1) : "memory");
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kFusedThreads, 1)
 project_residual_kernel(const __grid_constant__ CUtensorMap mapQt, const cf_lowrank::LrBatch B,
                         const cf_lowrank::Layout L) {
-    using G = StageGeom<BN>;
+    using G = FusedGeom<BN>;
+    constexpr int S = kFusedStages;
+    static_assert(((128 * (BN + 8) * 4 + 255) & ~255) + BN * (BN + 1) * 8 <= S * G::kStage,
+                  "tail scratch");
     const int bz = blockIdx.z;
     if (B.at<int32_t>(bz, L.off_status)[cf_lowrank::kSkipWord]) return;
     const cf_lowrank::LrPtrs pp = B.get(bz);
@@ -576,18 +609,18 @@ project_residual_kernel(const __grid_constant__ CUtensorMap mapQt, const cf_lowr
     extern __shared__ uint8_t dsmem[];
     const uint32_t base = (smem_u32(dsmem) + 1023u) & ~1023u;
     uint8_t *gbase = dsmem + (base - smem_u32(dsmem));
-    // barriers: a_full[S] (4 converter warps), b_full[S] (tx), empty[S]
+    // barriers: a_full[S] (8 converter warps), b_full[S] (tx), empty[S]
     // (commit), done (commit)
-    const uint32_t bars = base + kStages * G::kBytes;
+    const uint32_t bars = base + S * G::kStage;
     auto a_full = [&](int q) { return bars + 8u * q; };
-    auto b_full = [&](int q) { return bars + 8u * (kStages + q); };
-    auto empty = [&](int q) { return bars + 8u * (2 * kStages + q); };
-    const uint32_t done = bars + 8u * (3 * kStages);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + kStages * G::kBytes + 8 * (3 * kStages + 1));
+    auto b_full = [&](int q) { return bars + 8u * (S + q); };
+    auto empty = [&](int q) { return bars + 8u * (2 * S + q); };
+    const uint32_t done = bars + 8u * (3 * S);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + S * G::kStage + 8 * (3 * S + 1));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int q = 0; q < kStages; ++q) {
+        for (int q = 0; q < S; ++q) {
             mbar_init(a_full(q), kFusedConverters);
             mbar_init(b_full(q), 1);
             mbar_init(empty(q), 1);
@@ -611,34 +644,34 @@ project_residual_kernel(const __grid_constant__ CUtensorMap mapQt, const cf_lowr
     if (warp == kFusedConverters) {
         if (lane == 0) {
             auto load_b = [&](int kb) {
-                const int q = kb % kStages;
+                const int q = kb % S;
                 mbar_expect_tx(b_full(q), (uint32_t)G::kBytesB);
-                tma_load_3d(base + q * G::kBytes + kTileBytesA, &mapQt, b_full(q), kb * kBK, 0, bz);
+                tma_load_3d(base + q * G::kStage + kFusedX + kFusedR, &mapQt, b_full(q), kb * kBK, 0, bz);
             };
-            for (int kb = 0; kb < nkb && kb < kStages; ++kb) load_b(kb);
+            for (int kb = 0; kb < nkb && kb < S; ++kb) load_b(kb);
             constexpr uint32_t idesc = idesc_bf16(BN, false);
             bool ok = true;
             for (int kb = 0; kb < nkb; ++kb) {
-                const int q = kb % kStages;
-                const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+                const int q = kb % S;
+                const uint32_t ph = (uint32_t)(kb / S) & 1u;
                 if (!mbar_wait(a_full(q), ph) || !mbar_wait(b_full(q), ph)) {
                     ok = false;
                     break;
                 }
                 fence_after_sync();
-                const uint32_t sa = base + q * G::kBytes, sb = sa + kTileBytesA;
+                const uint32_t sa = base + q * G::kStage, sb = sa + kFusedX + kFusedR;
 #pragma unroll
                 for (int kk = 0; kk < kBK / 16; ++kk)
                     mma_bf16(tmem, sw128_desc(sa + kk * 32u, 16, 1024), sw128_desc(sb + kk * 32u, 16, 1024),
                              idesc, (kb > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(empty(q));
-                if (kb + kStages < nkb) {
-                    // this slot's B is read once its product is done
+                if (kb + S < nkb) {
+                    // this stage's B is read once its product is done
                     if (!mbar_wait(empty(q), ph)) {
                         ok = false;
                         break;
                     }
-                    load_b(kb + kStages);
+                    load_b(kb + S);
                 }
             }
             if (ok)
@@ -648,54 +681,89 @@ project_residual_kernel(const __grid_constant__ CUtensorMap mapQt, const cf_lowr
         }
         __syncwarp();
     } else {
-        // converters: warp w owns rows 16 w .. 16 w + 15 of the tile; one
-        // warp-wide load covers two rows (16 lanes x 4 channels each)
-        const int sub = lane >> 4, cl = (lane & 15) * 4;   // row within a pair, channel offset
-        bool ok = true;
-        for (int kb = 0; kb < nkb && ok; ++kb) {
-            const int q = kb % kStages;
-            if (kb >= kStages)
-                ok = __all_sync(kFullMask, mbar_wait(empty(q), (uint32_t)((kb / kStages - 1) & 1)));
-            if (!ok) break;
-            const int64_t c = (int64_t)kb * kBK + cl;
-            const bool cok = c < C;                  // C % 8 == 0: all 4 channels or none
-            uint8_t *sa = gbase + q * G::kBytes;
-            uint2 xw[8];
-            float4 rw[8];
+        const int r0 = 16 * warp;   // this warp's first row in the tile
+        // Stage kb's copies of this warp's rows: 16 rows x (8 x-chunks + 16
+        // recon-chunks) of 16 bytes = 384 chunks, 12 per lane.
+        auto issue = [&](int kb) {
+            const int q = kb % S;
+            const uint32_t sx = base + q * G::kStage, sr = sx + kFusedX;
+            const int64_t cbase = (int64_t)kb * kBK;
 #pragma unroll
-            for (int pr = 0; pr < 8; ++pr) {
-                const int64_t t = t0 + 16 * warp + 2 * pr + sub;
-                if (cok && t < T) {
-                    xw[pr] = __ldcs(reinterpret_cast<const uint2 *>(pp.x + t * C + c));
-                    rw[pr] = __ldcs(reinterpret_cast<const float4 *>(pp.recon + t * C + c));
+            for (int j = 0; j < 12; ++j) {
+                const int ci = lane + 32 * j;
+                if (ci < 128) {
+                    const int row = r0 + (ci >> 3), cc = ci & 7;
+                    const int64_t t = t0 + row, c = cbase + 8 * cc;
+                    const bool ok = t < T && c < C;
+                    cp_async16(sx + row * 128 + cc * 16, ok ? (const void *)(pp.x + t * C + c) : pp.x, ok);
                 } else {
-                    xw[pr] = make_uint2(0u, 0u);
-                    rw[pr] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    const int cr = ci - 128;
+                    const int row = r0 + (cr >> 4), cc = cr & 15;
+                    const int64_t t = t0 + row, c = cbase + 4 * cc;
+                    const bool ok = t < T && c < C;
+                    cp_async16(sr + row * 256 + cc * 16, ok ? (const void *)(pp.recon + t * C + c) : pp.recon,
+                               ok);
                 }
             }
+            cp_async_commit();
+        };
+        for (int kb = 0; kb < S; ++kb) {
+            if (kb < nkb)
+                issue(kb);
+            else
+                cp_async_commit();   // keep one group per k-block
+        }
+        const int sub = lane >> 4, cl = (lane & 15) * 4;   // row within a pair, channel offset
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int q = kb % S;
+            cp_async_wait_oldest();
+            __syncwarp();
+            uint8_t *sx = gbase + q * G::kStage;
+            const uint8_t *sr = sx + kFusedX;
+            const int64_t c = (int64_t)kb * kBK + cl;
+            const bool cok = c < C;                  // C % 8 == 0: all 4 channels or none
+            uint2 w[8];
 #pragma unroll
             for (int pr = 0; pr < 8; ++pr) {
-                const int row = 16 * warp + 2 * pr + sub;
-                const int64_t t = t0 + row;
-                const float v0 = __fsub_rn(bf16_bits_to_f32(xw[pr].x & 0xffffu), rw[pr].x);
-                const float v1 = __fsub_rn(bf16_bits_to_f32(xw[pr].x >> 16), rw[pr].y);
-                const float v2 = __fsub_rn(bf16_bits_to_f32(xw[pr].y & 0xffffu), rw[pr].z);
-                const float v3 = __fsub_rn(bf16_bits_to_f32(xw[pr].y >> 16), rw[pr].w);
+                const int row = r0 + 2 * pr + sub;
+                const uint2 xv = *reinterpret_cast<const uint2 *>(sx + row * 128 + cl * 2);
+                const float4 rv = *reinterpret_cast<const float4 *>(sr + row * 256 + cl * 4);
+                const float v0 = __fsub_rn(bf16_bits_to_f32(xv.x & 0xffffu), rv.x);
+                const float v1 = __fsub_rn(bf16_bits_to_f32(xv.x >> 16), rv.y);
+                const float v2 = __fsub_rn(bf16_bits_to_f32(xv.y & 0xffffu), rv.z);
+                const float v3 = __fsub_rn(bf16_bits_to_f32(xv.y >> 16), rv.w);
                 const __nv_bfloat162 h0 = __floats2bfloat162_rn(v0, v1);
                 const __nv_bfloat162 h1 = __floats2bfloat162_rn(v2, v3);
-                const uint2 w = make_uint2(*reinterpret_cast<const uint32_t *>(&h0),
-                                           *reinterpret_cast<const uint32_t *>(&h1));
+                w[pr] = make_uint2(*reinterpret_cast<const uint32_t *>(&h0),
+                                   *reinterpret_cast<const uint32_t *>(&h1));
+            }
+            __syncwarp();   // every lane has read its rows' x before any is overwritten
+#pragma unroll
+            for (int pr = 0; pr < 8; ++pr) {
+                const int row = r0 + 2 * pr + sub;
                 // 128-byte swizzle: 16-byte chunk j of row `row` sits at
                 // chunk j ^ (row & 7); this lane's 8 bytes are half a chunk
                 const int chunk = (cl >> 3) ^ (row & 7);
-                *reinterpret_cast<uint2 *>(sa + row * 128 + chunk * 16 + (cl & 4) * 2) = w;
-                if (cok && t < T) *reinterpret_cast<uint2 *>(vb + t * C + c) = w;
+                *reinterpret_cast<uint2 *>(sx + row * 128 + chunk * 16 + (cl & 4) * 2) = w[pr];
+                const int64_t t = t0 + row;
+                if (cok && t < T) *reinterpret_cast<uint2 *>(vb + t * C + c) = w[pr];
             }
             // generic writes of the A tile before the tensor cores read it
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(a_full(q));
+            // refill this stage with k-block kb + S once its product is done
+            if (kb + S < nkb) {
+                ok = __all_sync(kFullMask, mbar_wait(empty(q), (uint32_t)((kb / S) & 1)));
+                if (!ok) break;
+                issue(kb + S);
+            } else {
+                cp_async_commit();
+            }
         }
+        // no copy may land after this CTA's shared memory is reused
+        asm volatile("cp.async.wait_all;" ::: "memory");
         if (!ok && lane == 0) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
         // epilogue (warps 0-3): TMEM lane 32 w + i holds Y row t0 + 32 w + i
         if (warp < 4) have = __all_sync(kFullMask, ok && mbar_wait(done, 0));
