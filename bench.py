@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--e2e-chunks", type=int, default=6,
                     help="end-to-end leg: buffers of a step split into this many chunks whose "
                          "copies overlap the kernels of their neighbours")
+    ap.add_argument("--emit", action="store_true",
+                    help="quantize: the receiver also writes the bf16 reconstruction")
     ap.add_argument("--delta", action="store_true",
                     help="quantize: delta-state sender (previous activation + error buffer)")
     ap.add_argument("--warm", action="store_true",
@@ -350,12 +352,20 @@ def run_ours(args, world, rank, local):
         enc = [cf.enc_buffer_array([(X16[s, b], recon_s[b], err[b], codes[b], scales[b])
                                     for b in range(n)], dev) for s in range(S)]
         encode_batched = cf.cf_encode_batched
-    dec = cf.dec_buffer_array([(codes[b], scales[b], recon_r[b]) for b in range(n)], dev)
+    if args.emit:
+        # the receiver also writes the bf16 reconstruction its attention reads
+        out_bf16 = torch.empty((n, T, C), dtype=torch.bfloat16, device=dev)
+        dec = cf.dec_emit_buffer_array([(codes[b], scales[b], recon_r[b], out_bf16[b].view(torch.int16))
+                                        for b in range(n)], dev)
+        decode_batched = cf.cf_decode_emit_batched
+    else:
+        dec = cf.dec_buffer_array([(codes[b], scales[b], recon_r[b]) for b in range(n)], dev)
+        decode_batched = cf.cf_decode_batched
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
         encode_batched(d, n, enc[1 + i % (S - 1)], status, stream)
-        cf.cf_decode_batched(d, n, dec, status, stream)
+        decode_batched(d, n, dec, status, stream)
 
     sampler = ClockSampler(dev)
     sampler.start()
@@ -373,7 +383,7 @@ def run_ours(args, world, rank, local):
             e0.record(stream)
             encode_batched(d, n, enc[1 + (args.warmup + i) % (S - 1)], status, stream)
             e1.record(stream)
-            cf.cf_decode_batched(d, n, dec, status, stream)
+            decode_batched(d, n, dec, status, stream)
             e2.record(stream)
         t_end.record(stream)
     wall1 = time.time()
@@ -391,13 +401,15 @@ def run_ours(args, world, rank, local):
     else:
         enc_bytes = n * T * (C * 2 + C * 4 * 3 + Wd * 4 + 4)     # x, recon r/w, err w, codes, scale
     dec_bytes = n * T * (Wd * 4 + 4 + C * 4 * 2)             # codes, scale, recon r/w
+    if args.emit:
+        dec_bytes += n * T * C * 2                           # bf16 copy out
     peak, peak_kind = peaks()
     enc_gbs = enc_bytes / (enc_ms / 1e3) / 1e9
     dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9
 
     # End to end through the public API: pinned host x in, payload out.
     e2e = None
-    if not args.no_e2e and not args.delta:
+    if not args.no_e2e and not args.delta and not args.emit:
         e2e = run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, status)
         e2e["ms"] = R.reduce_scalar(e2e["ms"], "max")
         e2e = {"value": round(bytes_processed / (e2e["ms"] / 1e3) / 1e9, 3), "unit": "GB/s",
@@ -428,7 +440,8 @@ def run_ours(args, world, rank, local):
         "dtype": "bf16 in, fp32 state", "data": "synthetic",
         "config": {"workload": args.workload, "tokens": T, "channels": C, "buffers": n,
                    "bits": bits, "mode": f"{bits}-bit {'mean-abs' if bits == 1 else 'absmax'} + EF"
-                   + (", delta-state sender" if args.delta else ""),
+                   + (", delta-state sender" if args.delta else "")
+                   + (", emitting decode" if args.emit else ""),
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2 ({n * T * C * 14 / 1e9:.1f} GB touched per step)",
                    "launches_per_step": 2},
@@ -436,7 +449,8 @@ def run_ours(args, world, rank, local):
                      "unit": "GB/s", "frac": round(enc_gbs / peak, 4), "traffic": traffic,
                      "kernel": ("encode_tma_kernel (batched, TMA row staging)" if args.pipeline != 0
                                 else "encode_rows_kernel (batched, register rows)")
-                     + (", delta-state sender" if args.delta else ""),
+                     + (", delta-state sender" if args.delta else "")
+                   + (", emitting decode" if args.emit else ""),
                      "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": enc_bytes, "avg_launch_ms": round(enc_ms, 4)},
         "decode": {"achieved": round(dec_gbs, 1), "frac": round(dec_gbs / peak, 4),
