@@ -24,8 +24,10 @@
  *    this with cudaPointerGetAttributes and return CF_ERR_INVALID_ARG for
  *    host memory instead of launching.
  *  - Every device pointer must be 16-byte aligned (CF_ERR_ALIGNMENT), except
- *    the per-token scale arrays of the quantize mode, which need 4 bytes
- *    (so [n][T] packed scales of any T are valid).
+ *    the scale arrays (per-token in the quantize mode, so [n][T] packed
+ *    scales of any T are valid; per-column in the low-rank mode) and the
+ *    low-rank start block omega, which need 4 bytes, and the low-rank INT4
+ *    code arrays, which need 1 byte.
  *  - Argument errors are reported synchronously and launch nothing.  A
  *    failed launch returns CF_ERR_CUDA.  Numeric trouble found on the
  *    device (low-rank mode) is written to a status word in the workspace.
@@ -63,13 +65,16 @@ extern "C" {
 typedef enum cf_status {
     CF_OK = 0,
     CF_ERR_INVALID_ARG = 1,  /* null/host pointer, negative size, bad field */
-    CF_ERR_ALIGNMENT = 2,    /* a device pointer is not 16-byte aligned     */
+    CF_ERR_ALIGNMENT = 2,    /* a device pointer is not aligned as required  */
     CF_ERR_UNSUPPORTED = 3,  /* bits/rank/scale_kind outside what is built  */
     CF_ERR_WORKSPACE = 4,    /* low-rank workspace too small                 */
     CF_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed         */
     CF_ERR_NUMERIC = 6,      /* low-rank: Gram matrix not positive definite */
-    CF_ERR_TIMEOUT = 7       /* a bounded device wait gave up (tensor-core
-                                products); recorded in the workspace status */
+    CF_ERR_TIMEOUT = 7       /* a bounded device wait (mbarrier of a TMA or
+                                tensor-core pipeline) gave up; recorded in
+                                the status word (batched status_dev or the
+                                low-rank workspace), never returned by a
+                                call                                         */
 } cf_status;
 
 /* Problem description, as the pages state the problem: one exchanged
