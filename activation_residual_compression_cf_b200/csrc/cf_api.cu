@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "cf.h"
+#include "cf_trace.h"
 #include "lowrank_api.cuh"
 #include "quant_kernels.cuh"
 #include "quant_tma.cuh"
@@ -294,6 +295,7 @@ int64_t cf_payload_bytes(const cf_desc *d) {
 
 cf_status cf_state_init(const cf_desc *d, const uint16_t *x0, float *recon, float *err,
                         void *stream) {
+    cf::TraceRange trace_("cf_state_init");
     if (!d || d->tokens < 0 || d->channels < 1) return CF_ERR_INVALID_ARG;
     if (d->tokens > (int64_t(1) << 40) / d->channels) return CF_ERR_INVALID_ARG;
     const int64_t n = d->tokens * d->channels;
@@ -313,6 +315,7 @@ cf_status cf_state_init(const cf_desc *d, const uint16_t *x0, float *recon, floa
 
 cf_status cf_encode(const cf_desc *d, const uint16_t *x, float *recon_s, float *err,
                     uint32_t *codes, float *scales, void *stream) {
+    cf::TraceRange trace_("cf_encode");
     CF_TRY(check_quant_desc(d));
     if (d->tokens == 0) return CF_OK;
     CF_TRY(check_dev_ptr(x));
@@ -327,6 +330,7 @@ cf_status cf_encode(const cf_desc *d, const uint16_t *x, float *recon_s, float *
 
 cf_status cf_encode_delta(const cf_desc *d, const uint16_t *x, const uint16_t *x_prev, float *err,
                           uint32_t *codes, float *scales, void *stream) {
+    cf::TraceRange trace_("cf_encode_delta");
     CF_TRY(check_quant_desc(d));
     if (d->tokens == 0) return CF_OK;
     CF_TRY(check_dev_ptr(x));
@@ -341,6 +345,7 @@ cf_status cf_encode_delta(const cf_desc *d, const uint16_t *x, const uint16_t *x
 
 cf_status cf_decode(const cf_desc *d, const uint32_t *codes, const float *scales, float *recon_r,
                     void *stream) {
+    cf::TraceRange trace_("cf_decode");
     CF_TRY(check_quant_desc(d));
     if (d->tokens == 0) return CF_OK;
     CF_TRY(check_dev_ptr(codes));
@@ -353,6 +358,7 @@ cf_status cf_decode(const cf_desc *d, const uint32_t *codes, const float *scales
 
 cf_status cf_decode_emit(const cf_desc *d, const uint32_t *codes, const float *scales,
                          float *recon_r, uint16_t *out, void *stream) {
+    cf::TraceRange trace_("cf_decode_emit");
     CF_TRY(check_quant_desc(d));
     if (d->tokens == 0) return CF_OK;
     CF_TRY(check_dev_ptr(codes));
@@ -366,6 +372,7 @@ cf_status cf_decode_emit(const cf_desc *d, const uint32_t *codes, const float *s
 
 cf_status cf_decode_emit_batched(const cf_desc *d, int32_t n, const cf_dec_emit_buffer *bufs_dev,
                                  int32_t *status_dev, void *stream) {
+    cf::TraceRange trace_("cf_decode_emit_batched");
     CF_TRY(check_quant_desc(d));
     if (n < 0) return CF_ERR_INVALID_ARG;
     if (n == 0 || d->tokens == 0) return CF_OK;
@@ -378,6 +385,7 @@ cf_status cf_decode_emit_batched(const cf_desc *d, int32_t n, const cf_dec_emit_
 
 cf_status cf_encode_batched(const cf_desc *d, int32_t n, const cf_enc_buffer *bufs_dev,
                             int32_t *status_dev, void *stream) {
+    cf::TraceRange trace_("cf_encode_batched");
     CF_TRY(check_quant_desc(d));
     if (n < 0) return CF_ERR_INVALID_ARG;
     if (n == 0 || d->tokens == 0) return CF_OK;
@@ -390,6 +398,7 @@ cf_status cf_encode_batched(const cf_desc *d, int32_t n, const cf_enc_buffer *bu
 
 cf_status cf_encode_delta_batched(const cf_desc *d, int32_t n, const cf_enc_delta_buffer *bufs_dev,
                                   int32_t *status_dev, void *stream) {
+    cf::TraceRange trace_("cf_encode_delta_batched");
     CF_TRY(check_quant_desc(d));
     if (n < 0) return CF_ERR_INVALID_ARG;
     if (n == 0 || d->tokens == 0) return CF_OK;
@@ -402,6 +411,7 @@ cf_status cf_encode_delta_batched(const cf_desc *d, int32_t n, const cf_enc_delt
 
 cf_status cf_decode_batched(const cf_desc *d, int32_t n, const cf_dec_buffer *bufs_dev,
                             int32_t *status_dev, void *stream) {
+    cf::TraceRange trace_("cf_decode_batched");
     CF_TRY(check_quant_desc(d));
     if (n < 0) return CF_ERR_INVALID_ARG;
     if (n == 0 || d->tokens == 0) return CF_OK;

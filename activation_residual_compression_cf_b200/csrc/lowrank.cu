@@ -30,6 +30,7 @@
 #include <atomic>
 
 #include "cf.h"
+#include "cf_trace.h"
 #include "cf_common.cuh"
 #include "lowrank_api.cuh"
 #include "lowrank_kernels.cuh"
@@ -411,6 +412,7 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
                             const float *omega, uint8_t *p_codes, float *p_scales,
                             uint8_t *q_codes, float *q_scales, void *workspace,
                             size_t workspace_bytes, void *stream) {
+    cf::TraceRange trace_("cf_lowrank_encode");
     LR_TRY(check_desc(d));
     if (d->tokens == 0) return CF_OK;
     const Layout L = make_layout(d->tokens, d->channels, d->rank);
@@ -441,6 +443,7 @@ cf_status cf_lowrank_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
 
 cf_status cf_lowrank_encode_batched(const cf_desc *d, int32_t n, const cf_lowrank_buffer *bufs_dev,
                                     void *workspace, size_t workspace_bytes, void *stream) {
+    cf::TraceRange trace_("cf_lowrank_encode_batched");
     LR_TRY(check_desc(d));
     if (n < 0) return CF_ERR_INVALID_ARG;
     if (n == 0 || d->tokens == 0) return CF_OK;
@@ -460,6 +463,7 @@ cf_status cf_lowrank_encode_batched(const cf_desc *d, int32_t n, const cf_lowran
 cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes, const float *p_scales,
                             const uint8_t *q_codes, const float *q_scales, float *recon_r,
                             void *stream) {
+    cf::TraceRange trace_("cf_lowrank_decode");
     LR_TRY(check_desc(d));
     if (d->tokens == 0) return CF_OK;
     LR_TRY(check_ptr(p_codes, 1));
@@ -479,6 +483,7 @@ cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes, const floa
 
 cf_status cf_lowrank_decode_batched(const cf_desc *d, int32_t n, const cf_lowrank_dec_buffer *bufs_dev,
                                     int32_t *status_dev, void *stream) {
+    cf::TraceRange trace_("cf_lowrank_decode_batched");
     LR_TRY(check_desc(d));
     if (n < 0) return CF_ERR_INVALID_ARG;
     if (n == 0 || d->tokens == 0) return CF_OK;
