@@ -12,7 +12,9 @@
 //
 // One CTA of 4 warps per output tile:
 //   warp 0, one lane : TMA producer (cp.async.bulk.tensor, no multicast) into
-//                      a 4-stage ring of 128-byte-swizzled shared tiles
+//                      a 3-stage ring of 128-byte-swizzled shared tiles
+//                      (three CTAs per SM: measured on B200, 3 stages beat
+//                      4 at two CTAs per SM and 6-8 at one)
 //   warp 1           : allocates TMEM; one lane issues tcgen05.mma
 //                      (kind::f16, bf16 in, fp32 accumulate in TMEM) and
 //                      tcgen05.commit releases each stage
@@ -36,7 +38,7 @@
 namespace cf {
 namespace umma {
 
-constexpr int kStages = 4;
+constexpr int kStages = 3;               // ring depth of the plain projections
 constexpr int kBK = 64;                 // K elements per stage (128 B of bf16)
 constexpr int kTileBytesA = 128 * kBK * 2;  // 16 KB
 constexpr uint32_t kWaitLimit = 1u << 22;
