@@ -364,8 +364,8 @@ cf_status encode_impl(const cf_desc *d, const Layout &L, int n, const LrBatch &B
             cf::lr_residual_kernel<<<dim3((unsigned)blocks, 1, (unsigned)n), 256, 0, st>>>(B, L);
             LR_LAUNCHED();
         }
-        const int64_t nq = (int64_t)L.rp * L.C;
-        cf::lr_omega_kernel<<<dim3((unsigned)((nq + 255) / 256), 1, (unsigned)n), 256, 0, st>>>(B, L);
+        cf::lr_omega_kernel<<<dim3((unsigned)((L.C + 31) / 32), (unsigned)((L.rp + 31) / 32), (unsigned)n),
+                              dim3(32, 8), 0, st>>>(B, L);
         LR_LAUNCHED();
     }
     // Tensor-core engine: each projection CTA accumulates its whole K range,

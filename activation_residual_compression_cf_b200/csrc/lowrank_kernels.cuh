@@ -91,18 +91,31 @@ __global__ void lr_residual_kernel(const LrBatch B, const Layout L) {
 
 // Qt[k][c] = bf16(omega[c][k]) for k < r, 0 for the padding rows.
 __global__ void lr_omega_kernel(const LrBatch B, const Layout L) {
+    // Qt[k][c] = bf16(Omega[c][k]) (0 for k >= r), one 32 x 32 tile per
+    // block (32 x 8 threads): coalesced reads of Omega's rows, transposed
+    // through shared memory, coalesced writes of Qt's rows.
     const int bz = blockIdx.z;
     if (lr_skipped(B, L, bz)) return;
     const float *omega = B.get(bz).omega;
     if (!omega) return;   // warm start: Qt still holds the previous encode's Q
     bf16 *qt = B.at<bf16>(bz, L.off_qt);
     const int64_t C = L.C;
-    const int r = L.r, rp = L.rp;
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (int64_t)rp * C) return;
-    const int k = (int)(i / C);
-    const int64_t c = i - (int64_t)k * C;
-    qt[i] = __float2bfloat16_rn(k < r ? omega[c * r + k] : 0.0f);
+    const int r = L.r;
+    __shared__ float tile[32][33];
+    const int64_t c0 = (int64_t)blockIdx.x * 32;
+    const int k0 = blockIdx.y * 32;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    for (int j = ty; j < 32; j += 8) {
+        const int64_t c = c0 + j;
+        const int k = k0 + tx;
+        tile[j][tx] = (c < C && k < r) ? omega[c * r + k] : 0.0f;
+    }
+    __syncthreads();
+    for (int j = ty; j < 32; j += 8) {
+        const int k = k0 + j;
+        const int64_t c = c0 + tx;
+        if (k < L.rp && c < C) qt[(int64_t)k * C + c] = __float2bfloat16_rn(tile[tx][j]);
+    }
 }
 
 // Yp[s][t][k] = sum over the channels of split s of Vb[t][c] * Qt[k][c].
@@ -645,7 +658,12 @@ __global__ void lr_int4_pack_kernel(const LrBatch B, const Layout L, int which) 
     float *scales = which == 0 ? pp.ps_out : pp.qs_out;
     const int nb = (r + 1) / 2;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < r) scales[i] = __fdiv_rn(__uint_as_float(amax[i]), 7.0f);
+    // the column scales, once per block (the same division every element
+    // would otherwise repeat)
+    __shared__ float sc[cf_lowrank::kMaxRank];
+    for (int k = threadIdx.x; k < r; k += blockDim.x) sc[k] = __fdiv_rn(__uint_as_float(amax[k]), 7.0f);
+    __syncthreads();
+    if (i < r) scales[i] = sc[i];
     if (which == 1 && i == 0) {
         // the workspace now holds this encode's final Q (Qt): a later
         // encode of this shape may start from it
@@ -657,8 +675,8 @@ __global__ void lr_int4_pack_kernel(const LrBatch B, const Layout L, int which) 
     const int64_t row = i / nb;
     const int b = (int)(i - row * nb);
     const int k0 = 2 * b, k1 = 2 * b + 1;
-    const int q0 = int4_code(f[row * rp + k0], __fdiv_rn(__uint_as_float(amax[k0]), 7.0f));
-    const int q1 = (k1 < r) ? int4_code(f[row * rp + k1], __fdiv_rn(__uint_as_float(amax[k1]), 7.0f)) : 0;
+    const int q0 = int4_code(f[row * rp + k0], sc[k0]);
+    const int q1 = (k1 < r) ? int4_code(f[row * rp + k1], sc[k1]) : 0;
     codes[i] = (uint8_t)((q0 & 0xF) | ((q1 & 0xF) << 4));
 }
 
