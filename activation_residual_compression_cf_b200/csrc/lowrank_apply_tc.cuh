@@ -80,10 +80,9 @@ __host__ __device__ constexpr int apply_stage_tok() {
     return SENDER ? 16 : 32;
 }
 constexpr int kApplyConsumers = 256;            // 8 warps: 4 channel quarters x 2 token halves
-constexpr int kApplyProducerWarp = kApplyConsumers / 32;   // warp 8: bulk copies
-constexpr int kApplyMmaWarp = kApplyProducerWarp + 1;      // warps 9, 10: B operands;
-constexpr int kApplyBuilders = 64;                          // warp 9 also issues the MMAs
-constexpr int kApplyThreads = kApplyConsumers + 32 + kApplyBuilders;
+constexpr int kApplyMmaWarp = kApplyConsumers / 32;        // warps 8, 9: B operands;
+constexpr int kApplyBuilders = 64;                          // warp 8 also issues the MMAs
+constexpr int kApplyThreads = kApplyConsumers + kApplyBuilders;
 // Token tiles per CTA at most: the receiver's tiles carry half the bytes of
 // the sender's, so it takes twice as many to amortise a CTA's set-up
 // (measured on B200: 16 tiles gave the receiver 0.92 of HBM against 0.89).
@@ -105,11 +104,17 @@ __host__ __device__ constexpr int apply_tc_smem() {
     return 1024 + 3 * (KP / 32) * 16384 + apply_ring<SENDER, KP>() * apply_stage_bytes<SENDER>() + 512;
 }
 
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
+// 16-byte asynchronous copy global -> shared (src-size 0: 16 zero bytes)
+__device__ __forceinline__ void apply_cp16(uint32_t dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void apply_cp_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void apply_cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 // consumers + the builder warps, once, after the first operands are built
 __device__ __forceinline__ void operand_sync() {
@@ -207,28 +212,28 @@ __device__ __forceinline__ void apply_build_b_warp(uint8_t *gbh, uint8_t *gbl, c
 }
 
 // Persistent over a run of token tiles: CTA (x, y, z) owns channel block x of
-// buffer z and token tiles [y * tpc, (y + 1) * tpc).  Warp roles (352
+// buffer z and token tiles [y * tpc, (y + 1) * tpc).  Warp roles (320
 // threads):
-//   warps 0-7 : with warps 9-10, build the A operand (Q codes of the channel
+//   warps 0-7 : with warps 8-9, build the A operand (Q codes of the channel
 //               block) and tile 0's B operand; then each warp combines one
 //               channel quarter (w % 4, its TMEM lanes) x one half (w / 4) of
-//               every 16-token stage of every tile, reading x and recon from
-//               shared memory and D from TMEM, and writes err and recon;
-//   warp 8    : one lane issues 1-D bulk copies (cp.async.bulk, no multicast)
-//               of every token row's 128-channel segment of recon (and x) of
-//               all the CTA's tiles into the ring, from the kernel's first
-//               instructions on;
-//   warps 9-10: for tile i, once tile i-1's product is done (its commit
+//               every stage of every tile, reading x and recon from shared
+//               memory and D from TMEM, and writes err and recon.  A warp
+//               stages exactly the rows and channels it combines itself:
+//               16-byte asynchronous copies (cp.async) into a ring of S
+//               stages, issued S stages ahead from the kernel's first
+//               instructions on, so its loads never wait on its arithmetic
+//               and no other warp has to hand it the data;
+//   warps 8-9 : for tile i, once tile i-1's product is done (its commit
 //               barrier) write tile i's B operand (single buffer, half the
 //               rows each), and once the consumers have released accumulator
-//               i % 2 (tile i-2 combined) warp 9 issues the MMAs of tile i
+//               i % 2 (tile i-2 combined) warp 8 issues the MMAs of tile i
 //               into it.
 // So the consumers never wait on operand building: the product of the next
 // tile is formed while the current one is combined.
 // Every wait is bounded; on expiry CF_ERR_TIMEOUT goes to the buffer's status
 // word and the waiting warp stops (the others then run out of their own
-// waits), the producer waits (bounded) for its copies still in flight, and
-// TMEM is freed.
+// waits), every warp drains its copies still in flight, and TMEM is freed.
 template <bool SENDER, int KP>
 __global__ void __launch_bounds__(kApplyThreads, (KP <= 32 ? 2 : 1))
 lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int tpc) {
@@ -257,10 +262,10 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
     const uint32_t sA = base, sBh = base + OPB, sBl = base + 2 * OPB;
     const uint32_t ring = base + 3 * OPB;
     uint8_t *gring = gb + 3 * OPB;
-    // barriers: mma[2], acc_free[2], full[S], empty[S]
+    // barriers: mma[2], acc_free[2]
     const uint32_t bars = ring + S * SB;
-    const uint32_t mma0 = bars, accf0 = bars + 16u, full0 = bars + 32u, empty0 = bars + 32u + 8u * S;
-    float *sk = reinterpret_cast<float *>(gring + S * SB + 8 * (4 + 2 * S));   // [KP]
+    const uint32_t mma0 = bars, accf0 = bars + 16u;
+    float *sk = reinterpret_cast<float *>(gring + S * SB + 8 * 4);   // [KP]
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sk + KP);
     int *abort_flag = reinterpret_cast<int *>(tslot + 1);   // builder warps give up together
 
@@ -280,10 +285,6 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
             mbar_init(mma0 + 8u * j, 1);                         // tcgen05.commit
             mbar_init(accf0 + 8u * j, kApplyConsumers / 32);     // one per consumer warp
         }
-        for (int s = 0; s < S; ++s) {
-            mbar_init(full0 + 8u * s, 1);                        // producer + tx bytes
-            mbar_init(empty0 + 8u * s, kApplyConsumers / 32);    // one per consumer warp
-        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -300,42 +301,46 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
     fence_after_sync();
     const uint32_t tmem = *tslot;
 
-    if (warp == kApplyProducerWarp) {
-        // ---------------- producer: stages of 16 rows over [tbeg, tend) ----------------
-        if (lane == 0) {
-            const uint32_t rbytes = (uint32_t)cw * 4u, xbytes = (uint32_t)cw * 2u;
-            int issued = 0;
-            bool ok = true;
-            for (int it = 0; it < nt && ok; ++it) {
-                const int64_t t0 = tbeg + (int64_t)it * kApplyTile;
-                for (int64_t tb = t0; tb < t0 + kApplyTile && tb < tend; tb += STOK) {
-                    const int slot = issued % S;
-                    if (issued >= S && !mbar_wait(empty0 + 8u * slot, (uint32_t)((issued / S - 1) & 1))) {
-                        ok = false;
-                        break;
+    {
+        // Consumer warps: their first S stages' copies go out before the
+        // operand build, so the loads overlap it.
+        const int q = warp & 3, half = warp >> 2;
+        const int cl = 32 * q + lane;              // channel within the block
+        const int64_t c = c0 + cl;
+        const bool col_ok = cl < cw;
+        const uint32_t tlane = (uint32_t)(32 * q) << 16;
+        // Global stage g covers tokens [tbeg + g STOK, +STOK) (tiles are
+        // full except possibly the CTA's last).  issue(g) stages this
+        // warp's TPW rows x 32 channels of it: recon in 16-byte chunks of
+        // 4 channels, x in chunks of 8; one commit group per stage.
+        const int64_t gstages = (tend - tbeg + STOK - 1) / STOK;
+        auto issue = [&](int64_t gg) {
+            if (gg < gstages) {
+                const uint32_t sr0 = ring + (uint32_t)((gg % S) * SB);
+                const int64_t tb = tbeg + gg * STOK + TPW * half;
+#pragma unroll
+                for (int id = lane; id < TPW * 8; id += 32) {
+                    const int row = id >> 3, ch = 32 * q + 4 * (id & 7);
+                    const int64_t t = tb + row;
+                    const bool ok = t < tend && ch < cw;
+                    apply_cp16(sr0 + (uint32_t)((TPW * half + row) * (kApplyTile * 4) + ch * 4),
+                               ok ? (const void *)(recon + t * C + c0 + ch) : (const void *)recon, ok);
+                }
+                if (SENDER) {
+#pragma unroll
+                    for (int id = lane; id < TPW * 4; id += 32) {
+                        const int row = id >> 2, ch = 32 * q + 8 * (id & 3);
+                        const int64_t t = tb + row;
+                        const bool ok = t < tend && ch < cw;
+                        apply_cp16(sr0 + (uint32_t)(RB + (TPW * half + row) * (kApplyTile * 2) + ch * 2),
+                                   ok ? (const void *)(x + t * C + c0 + ch) : (const void *)x, ok);
                     }
-                    const int rows = (int)((tend - tb < STOK) ? tend - tb : STOK);
-                    const uint32_t full = full0 + 8u * slot;
-                    const uint32_t dst = ring + (uint32_t)(slot * SB);
-                    mbar_expect_tx(full, (uint32_t)rows * (rbytes + (SENDER ? xbytes : 0u)));
-                    for (int j = 0; j < rows; ++j) {
-                        const int64_t o = (tb + j) * C + c0;
-                        bulk_g2s(dst + (uint32_t)(j * kApplyTile * 4), recon + o, rbytes, full);
-                        if (SENDER)
-                            bulk_g2s(dst + (uint32_t)(RB + j * kApplyTile * 2), x + o, xbytes, full);
-                    }
-                    ++issued;
                 }
             }
-            if (!ok && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
-            // Copies of the last stages issued may still be landing if a
-            // consumer gave up: wait for them (bounded) before this CTA's
-            // shared memory is released.  In a normal run these phases have
-            // completed already and each wait returns at once.
-            for (int st = (issued > S ? issued - S : 0); st < issued; ++st)
-                (void)mbar_wait(full0 + 8u * (st % S), (uint32_t)((st / S) & 1));
-        }
-    } else {
+            apply_cp_commit();
+        };
+        if (warp < kApplyMmaWarp)
+            for (int gg = 0; gg < S; ++gg) issue(gg);
         // A = the INT4 codes of Q for this channel block, and tile 0's B:
         // built once by the consumers and the MMA warp together.
         const int ot = warp >= kApplyMmaWarp ? kApplyConsumers + 32 * (warp - kApplyMmaWarp) + lane : tid;
@@ -399,14 +404,8 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
             }
         } else {
             // ---------------- combine ----------------
-            const int q = warp & 3, half = warp >> 2;
-            const int cl = 32 * q + lane;              // channel within the block
-            const int64_t c = c0 + cl;
-            const bool col_ok = cl < cw;
-            const uint32_t tlane = (uint32_t)(32 * q) << 16;
-            int g = 0;                                 // stages consumed so far
-            bool ok = true;
-            for (int i = 0; i < nt && ok; ++i) {
+            int64_t g = 0;                             // stages consumed so far
+            for (int i = 0; i < nt; ++i) {
                 if (!__all_sync(kFullMask, mbar_wait(mma0 + 8u * (i & 1), (uint32_t)((i >> 1) & 1)))) {
                     if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
                     break;
@@ -417,12 +416,11 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
                 const int64_t tw = (T - t0 < kApplyTile) ? T - t0 : kApplyTile;
                 const int ns = (int)((tw + STOK - 1) / STOK);
                 for (int st = 0; st < ns; ++st, ++g) {
-                    const int slot = g % S;
-                    if (!__all_sync(kFullMask, mbar_wait(full0 + 8u * slot, (uint32_t)((g / S) & 1)))) {
-                        if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
-                        ok = false;
-                        break;
-                    }
+                    const int slot = (int)(g % S);
+                    // this warp's copies of stage g have landed (one group
+                    // per stage, S in flight)
+                    apply_cp_wait<S - 1>();
+                    __syncwarp();
                     const int tl = st * STOK + TPW * half;   // first token column of this warp
                     float dv[TPW];
                     if (TPW == 16)
@@ -444,17 +442,17 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
                             __stcs(recon + o, __fadd_rn(rv, dv[j]));
                         }
                     }
-                    // generic reads of the slot before the next async copy into it
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    // every lane has read its rows of the slot: refill it
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(empty0 + 8u * slot);
+                    issue(g + S);
                 }
-                if (!ok) break;
                 // this warp's reads of accumulator i % 2 are complete
                 fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(accf0 + 8u * (i & 1));
             }
+            // no copy may land after this CTA's shared memory is released
+            asm volatile("cp.async.wait_all;" ::: "memory");
         }
     }
     fence_before_sync();
