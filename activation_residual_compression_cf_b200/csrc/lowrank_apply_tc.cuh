@@ -71,13 +71,13 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v) {
 // Staging of x and recon: a tile's 128 tokens are stages of STOK token rows;
 // a stage holds the rows' recon (STOK x 128 fp32) and, for the sender, x
 // (STOK x 128 bf16).  Each consumer warp takes STOK / 2 tokens of a stage.
-// The receiver moves half the bytes per element, so its stages are twice as
-// long to spread the fixed per-stage cost (barrier, TMEM load, release) over
-// as many bytes.  Ring depth per kernel, sized so that rank <= 32 keeps two
-// CTAs per SM.
+// Ring depth per kernel, sized so that rank <= 32 keeps two CTAs per SM
+// (measured on B200 with per-warp cp.async staging: 16-token stages 4 deep
+// for both directions; the receiver at 32-token stages 3 deep, or 16 x 6,
+// was slower).
 template <bool SENDER>
 __host__ __device__ constexpr int apply_stage_tok() {
-    return SENDER ? 16 : 32;
+    return 16;
 }
 constexpr int kApplyConsumers = 256;            // 8 warps: 4 channel quarters x 2 token halves
 constexpr int kApplyMmaWarp = kApplyConsumers / 32;        // warps 8, 9: B operands;
@@ -97,7 +97,7 @@ __host__ __device__ constexpr int apply_stage_bytes() {
 }
 template <bool SENDER, int KP>
 __host__ __device__ constexpr int apply_ring() {
-    return KP <= 32 ? (SENDER ? 4 : 3) : (SENDER ? 8 : 4);
+    return KP <= 32 ? 4 : 8;
 }
 template <bool SENDER, int KP>
 __host__ __device__ constexpr int apply_tc_smem() {
