@@ -168,46 +168,12 @@ lr_project_simt(const LrBatch B, const Layout L) {
     }
 }
 
-// Cholesky of the rp x rp matrix in shared memory A (leading dimension ld,
-// upper triangle valid), in one warp with every column in registers:
-// lane c owns column c (r <= 32).  Step j broadcasts row j of R by
-// shuffles; no shared-memory round trips inside the factorisation.
-// On return A's upper triangle holds R and dead[j] flags dead pivots.
-template <int RPW>
-__device__ __forceinline__ void warp_cholesky_regs(double *A, int ld, int r, const double *gdiag,
-                                                   int *dead, double *invd) {
-    const int lane = threadIdx.x & 31;
-    double col[RPW];
-#pragma unroll
-    for (int i = 0; i < RPW; ++i) col[i] = (lane < r && i <= lane) ? A[i * ld + lane] : 0.0;
-#pragma unroll
-    for (int j = 0; j < RPW; ++j) {
-        if (j >= r) break;
-        const double ajj = __shfl_sync(kFullMask, col[j], j);
-        const bool bad = !(ajj > 1e-10 * gdiag[j]);
-        // one reciprocal square root gives both R[j][j] = ajj * inv and 1/R[j][j]
-        const double inv = bad ? 0.0 : rsqrt(ajj);
-        const double rjj = ajj * inv;
-        if (lane > j) col[j] *= inv;
-        if (lane == j) col[j] = rjj;
-        const double rjc = col[j];
-#pragma unroll
-        for (int i = j + 1; i < RPW; ++i) {
-            const double rji = __shfl_sync(kFullMask, rjc, i);  // R[j][i] from lane i
-            if (lane >= i) col[i] = fma(-rji, rjc, col[i]);
-        }
-        if (lane == 0) {
-            dead[j] = bad ? 1 : 0;
-            invd[j] = inv;
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < RPW; ++i)
-        if (lane < r && i <= lane) A[i * ld + lane] = col[i];
-}
-
-// Same factorisation for r up to 64 with the matrix in shared memory (lane
-// l owns columns l and l + 32).
+// Cholesky G = R^T R of the rp x rp matrix in shared memory A (leading
+// dimension ld, upper triangle valid), in one warp, for r up to 64 (lane l
+// owns columns l and l + 32).  A pivot not above 1e-10 of its original
+// diagonal entry gdiag[j] is dead: its row of R and invd[j] become zero and
+// dead[j] is set.  On return A's upper triangle holds R and invd[j] =
+// 1/R[j][j] (0 where dead); one reciprocal square root gives both.
 __device__ __forceinline__ void warp_cholesky_smem(double *A, int ld, int r, const double *gdiag,
                                                    int *dead, double *invd) {
     const int lane = threadIdx.x & 31;
@@ -238,7 +204,7 @@ __device__ __forceinline__ void warp_cholesky_smem(double *A, int ld, int r, con
 // owns column c and the rows i = w, w + 4, ... of it in registers, so every
 // warp (one per SM sub-partition) shares the fp64 update work of a step.
 // Row j of R is broadcast through shared memory (double-buffered, one
-// barrier per step among the 128 threads).  Results as warp_cholesky_regs.
+// barrier per step among the 128 threads).  Results as warp_cholesky_smem.
 __device__ __forceinline__ void quad_cholesky(double *A, int ld, int r, const double *gdiag,
                                               int *dead, double *invd, double (*rowbuf)[33]) {
     const int tid = threadIdx.x;
