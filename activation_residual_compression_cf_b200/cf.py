@@ -29,7 +29,8 @@ EXPORTS = ("cf_status_string", "cf_abi_version", "cf_codes_words_per_row",
            "cf_lowrank_status", "cf_set_lowrank_engine", "cf_set_quant_pipeline",
            "cf_set_launch_override", "cf_lowrank_encode_noalloc", "cf_decode_emit",
            "cf_decode_emit_batched", "cf_lowrank_encode_batched", "cf_lowrank_decode_batched",
-           "cf_lowrank_set_apply_events", "cf_encode_delta", "cf_encode_delta_batched")
+           "cf_lowrank_set_apply_events", "cf_encode_delta", "cf_encode_delta_batched",
+           "cf_diag_bounded_wait")
 
 
 class CFError(RuntimeError):
@@ -117,6 +118,7 @@ def lib():
             "cf_set_launch_override": ([i32, i32, i32, i32], ctypes.c_int),
             "cf_set_lowrank_engine": ([i32], ctypes.c_int),
             "cf_lowrank_set_apply_events": ([vp, vp, vp, vp], ctypes.c_int),
+            "cf_diag_bounded_wait": ([i32, vp, vp], ctypes.c_int),
             "cf_set_quant_pipeline": ([i32, i32, i32], ctypes.c_int),
             "cf_lowrank_encode_noalloc": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         }
@@ -274,6 +276,10 @@ def _ev(e):
 def cf_lowrank_set_apply_events(enc_start=None, enc_stop=None, dec_start=None, dec_stop=None):
     _chk(lib().cf_lowrank_set_apply_events(_ev(enc_start), _ev(enc_stop), _ev(dec_start),
                                            _ev(dec_stop)), "cf_lowrank_set_apply_events")
+
+
+def cf_diag_bounded_wait(polls: int, out_dev, stream=None):
+    _chk(lib().cf_diag_bounded_wait(polls, _p(out_dev), _s(stream)), "cf_diag_bounded_wait")
 
 
 def cf_set_quant_pipeline(kernel: int, pipeline: int, stages: int = 0):

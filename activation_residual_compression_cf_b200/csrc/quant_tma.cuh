@@ -18,39 +18,19 @@
 
 #include "cf.h"
 #include "cf_common.cuh"
+#include "mbar.cuh"
 #include "quant_kernels.cuh"
 
 namespace cf {
 namespace tma {
 
-constexpr uint32_t kWaitLimit = 1u << 22;
-
 __device__ __forceinline__ uint32_t saddr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ void bar_init(uint32_t b, uint32_t n) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(b), "r"(n) : "memory");
-}
-__device__ __forceinline__ void bar_expect(uint32_t b, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void bar_arrive(uint32_t b) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(b) : "memory");
-}
-__device__ __forceinline__ bool bar_wait(uint32_t b, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(b), "r"(parity)
-            : "memory");
-        if (ok) return true;
-    }
-    return false;
-}
+__device__ __forceinline__ void bar_init(uint32_t b, uint32_t n) { mbar_init(b, n); }
+__device__ __forceinline__ void bar_expect(uint32_t b, uint32_t bytes) { mbar_expect_tx(b, bytes); }
+__device__ __forceinline__ void bar_arrive(uint32_t b) { mbar_arrive(b); }
+__device__ __forceinline__ bool bar_wait(uint32_t b, uint32_t parity) { return mbar_wait(b, parity); }
 // 1-D bulk copy global -> shared; both addresses 16-byte aligned, bytes a
 // multiple of 16.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {

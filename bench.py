@@ -170,9 +170,9 @@ class ClockSampler:
                 "window": "timed region" if win else "whole run (timed region shorter than one sample)"}
 
 
-QUANT_SOURCES = ("quant_tma.cuh", "quant_kernels.cuh", "cf_common.cuh", "cf_api.cu")
+QUANT_SOURCES = ("quant_tma.cuh", "quant_kernels.cuh", "cf_common.cuh", "mbar.cuh", "cf_api.cu")
 LOWRANK_APPLY_SOURCES = ("lowrank_apply_tc.cuh", "lowrank_umma.cuh", "lowrank_kernels.cuh",
-                         "lowrank_api.cuh", "lowrank.cu", "cf_common.cuh")
+                         "lowrank_api.cuh", "lowrank.cu", "cf_common.cuh", "mbar.cuh")
 
 
 def kernel_source_hash(files=QUANT_SOURCES):

@@ -119,6 +119,15 @@ typedef struct cf_dec_emit_buffer {
  * graph and replayed; the host-side argument checks run at capture time.
  * cf_lowrank_encode_noalloc's first call on a device must precede capture. */
 
+/* Diagnostic (no counterpart in the paper): checks on the device that the
+ * bounded wait every TMA and tensor-core pipeline uses ends.  One CTA waits,
+ * with at most `polls` polls (1 .. 65536), on an mbarrier it has signalled
+ * itself and on one that nothing signals, and writes out_dev[0..1] (device
+ * int32[2], 4-byte aligned): [0] = 1 if the signalled wait completed;
+ * [1] = CF_ERR_TIMEOUT if the unsignalled wait gave up (CF_OK otherwise).
+ * The GPU never hangs or faults: the unsignalled wait stops after `polls`. */
+cf_status cf_diag_bounded_wait(int32_t polls, int32_t *out_dev, void *stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *cf_status_string(cf_status s);
 

@@ -114,6 +114,13 @@ def test_pipeline_and_engine_knobs_validate(L):
     assert L.cf_lowrank_set_apply_events(None, None, None, None) == 0
 
 
+def test_bounded_wait_diagnostic_validates_before_any_cuda_call(L):
+    assert L.cf_diag_bounded_wait(0, 16, None) == 1        # no polls
+    assert L.cf_diag_bounded_wait(65537, 16, None) == 1    # above the cap
+    assert L.cf_diag_bounded_wait(256, None, None) == 1    # null output
+    assert L.cf_diag_bounded_wait(256, 18, None) == 2      # not 4-byte aligned
+
+
 def test_binding_raises_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(cf, "_lib", None)
     monkeypatch.setattr(cf, "LIB_PATH", str(tmp_path / "nope.so"))
