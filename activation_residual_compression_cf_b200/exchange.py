@@ -1,0 +1,247 @@
+"""Sequence-parallel exchange of compressed activations between ranks.
+
+In sequence-parallel serving every GPU computes the activations (K and V of
+every layer) of its own token shard and needs every other shard's for
+attention.  CompactFusion ("Accelerating Parallel Diffusion Model Serving
+with Residual Compression", sections "Approach" and "Key results") sends,
+instead of an activation, the compressed difference between it and the
+reconstruction the receivers already hold; each receiver keeps one
+reconstruction per (peer, buffer) and adds the decoded residual to it.  The
+first step (the warmup) exchanges the activations uncompressed.
+
+One compressed step on each rank is three device operations, all enqueued on
+the current stream:
+
+1. one batched encode of the rank's buffers, writing codes and scales
+   straight into one contiguous payload (``PayloadLayout``);
+2. one all-gather of the payloads over the process group (NCCL over NVLink
+   on GPUs);
+3. one batched decode of every peer's payload into that peer's receiver
+   states.
+
+The arithmetic runs in libcf's kernels (``CudaCodec``); this module lays out
+memory and orders the calls.  A caller may pass another codec object with
+the same four methods (the CPU tests drive the host logic that way).
+"""
+from __future__ import annotations
+
+import collections
+import dataclasses
+
+import torch
+import torch.distributed as dist
+
+from . import cf
+
+
+def _align16(n: int) -> int:
+    return (n + 15) & ~15
+
+
+@dataclasses.dataclass(frozen=True)
+class PayloadLayout:
+    """Where each buffer's codes and scales sit in one rank's payload.
+
+    Per buffer, in buffer order: the packed codes (uint32 [tokens, words]),
+    then the per-token fp32 scales, each segment starting on a 16-byte
+    boundary (the library's alignment rule), so the payload of a rank is one
+    contiguous byte range and the all-gather is a single collective."""
+    tokens: int
+    channels: int
+    bits: int
+    buffers: int
+
+    @property
+    def words_per_row(self) -> int:
+        return (self.channels * self.bits + 31) // 32
+
+    @property
+    def codes_bytes(self) -> int:
+        return self.tokens * self.words_per_row * 4
+
+    @property
+    def scales_bytes(self) -> int:
+        return self.tokens * 4
+
+    @property
+    def stride(self) -> int:
+        return _align16(self.codes_bytes) + _align16(self.scales_bytes)
+
+    @property
+    def bytes_per_rank(self) -> int:
+        return self.buffers * self.stride
+
+    def codes_offset(self, b: int) -> int:
+        return b * self.stride
+
+    def scales_offset(self, b: int) -> int:
+        return b * self.stride + _align16(self.codes_bytes)
+
+    def codes(self, payload: torch.Tensor, b: int) -> torch.Tensor:
+        """int32 [tokens, words] view of buffer b's codes in a payload."""
+        o = self.codes_offset(b)
+        return payload[o:o + self.codes_bytes].view(torch.int32).view(self.tokens, self.words_per_row)
+
+    def scales(self, payload: torch.Tensor, b: int) -> torch.Tensor:
+        """float32 [tokens] view of buffer b's scales in a payload."""
+        o = self.scales_offset(b)
+        return payload[o:o + self.scales_bytes].view(torch.float32)
+
+
+class CudaCodec:
+    """The product path: libcf's batched encode / decode kernels.  The device
+    arrays of buffer pointers are kept for the last `cache` pointer sets, so
+    inputs that cycle through a fixed set of tensors cost no host-to-device
+    copy of pointers per step."""
+
+    def __init__(self, device: torch.device, cache: int = 64):
+        self.device = device
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self._cache = collections.OrderedDict()
+        self._cache_size = cache
+
+    def _array(self, kind, sets, make):
+        key = (kind,) + tuple(t.data_ptr() for s in sets for t in s)
+        arr = self._cache.get(key)
+        if arr is None:
+            arr = make(sets, self.device)
+            self._cache[key] = arr
+            if len(self._cache) > self._cache_size:
+                self._cache.popitem(last=False)
+        else:
+            self._cache.move_to_end(key)
+        return arr
+
+    def state_init(self, d, x, recon, err):
+        cf.cf_state_init(d, x, recon, err)
+
+    def prepare_encode(self, d, sets):
+        self._array("enc", sets, cf.enc_buffer_array)
+
+    def encode_batched(self, d, sets):
+        cf.cf_encode_batched(d, len(sets), self._array("enc", sets, cf.enc_buffer_array), self.status)
+
+    def decode_batched(self, d, sets):
+        if sets:
+            cf.cf_decode_batched(d, len(sets), self._array("dec", sets, cf.dec_buffer_array), self.status)
+
+    def status_value(self) -> int:
+        """First error any batched call recorded (synchronises)."""
+        return int(self.status.item())
+
+
+class ShardExchange:
+    """Sender state for this rank's shard of `buffers` activations and
+    receiver states for every peer's shard, plus the payload buffers.
+
+    tokens, channels: this rank's shard of one buffer (every rank's shard has
+    the same shape); bits: 1 or 2.  `loopback` also keeps a receiver for the
+    rank's own shard and decodes its own payload, which on one GPU runs the
+    whole path (its reconstruction must equal the sender's mirror bit for
+    bit).  recon_r[p][b] is the reconstruction of peer p's buffer b (None for
+    the rank's own shard unless `loopback`)."""
+
+    def __init__(self, tokens: int, channels: int, bits: int, buffers: int, *, group=None,
+                 device=None, codec=None, loopback: bool = False):
+        if bits not in (1, 2):
+            raise ValueError(f"bits must be 1 or 2, got {bits}")
+        if tokens < 1 or channels < 1 or buffers < 1:
+            raise ValueError("tokens, channels and buffers must be positive")
+        self.group = group
+        if dist.is_available() and dist.is_initialized():
+            self.world = dist.get_world_size(group)
+            self.rank = dist.get_rank(group)
+            self.backend = dist.get_backend(group)
+        else:
+            self.world, self.rank, self.backend = 1, 0, None
+        if device is None:
+            device = torch.device("cuda", torch.cuda.current_device())
+        self.device = torch.device(device)
+        self.codec = codec if codec is not None else CudaCodec(self.device)
+        self.layout = PayloadLayout(tokens, channels, bits, buffers)
+        self.d = cf.desc(tokens, channels, bits)
+        n = self.layout.bytes_per_rank
+        self.send = torch.zeros(n, dtype=torch.uint8, device=self.device)
+        self.recv = torch.zeros(self.world * n, dtype=torch.uint8, device=self.device)
+        f32 = dict(dtype=torch.float32, device=self.device)
+        self.recon_s = [torch.empty(tokens, channels, **f32) for _ in range(buffers)]
+        self.err = [torch.empty(tokens, channels, **f32) for _ in range(buffers)]
+        self.peers = [p for p in range(self.world) if loopback or p != self.rank]
+        self.recon_r = [[torch.empty(tokens, channels, **f32) for _ in range(buffers)]
+                        if p in self.peers else None for p in range(self.world)]
+        self._dec_sets = [(self.layout.codes(self._payload(p), b), self.layout.scales(self._payload(p), b),
+                           self.recon_r[p][b]) for p in self.peers for b in range(buffers)]
+
+    def _payload(self, p: int) -> torch.Tensor:
+        n = self.layout.bytes_per_rank
+        return self.recv[p * n:(p + 1) * n]
+
+    def _all_gather(self, out: torch.Tensor, inp: torch.Tensor) -> None:
+        if self.backend is None:
+            out.copy_(inp)
+        elif self.backend == "nccl":
+            dist.all_gather_into_tensor(out, inp, group=self.group)
+        else:
+            dist.all_gather(list(out.chunk(self.world)), inp, group=self.group)
+
+    def _check(self, xs):
+        L = self.layout
+        if len(xs) != L.buffers:
+            raise ValueError(f"expected {L.buffers} activations, got {len(xs)}")
+        for x in xs:
+            if x.dtype != torch.bfloat16 or tuple(x.shape) != (L.tokens, L.channels) or not x.is_contiguous():
+                raise ValueError("each activation must be a contiguous bf16 [tokens, channels] tensor")
+            if x.data_ptr() % 16:
+                raise ValueError("each activation must start on a 16-byte boundary")
+
+    def warmup(self, xs) -> None:
+        """Step 0: exchange the activations uncompressed; every receiver
+        state starts from the exact activation and the error buffers from 0."""
+        self._check(xs)
+        L = self.layout
+        n = L.tokens * L.channels * 2
+        seg = _align16(n)            # every activation starts on a 16-byte boundary
+
+        def at(buf, i):
+            return buf[i * seg:i * seg + n].view(torch.bfloat16).view(L.tokens, L.channels)
+
+        local = torch.zeros(L.buffers * seg, dtype=torch.uint8, device=self.device)
+        for b in range(L.buffers):
+            at(local, b).copy_(xs[b])
+        every = torch.empty(self.world * L.buffers * seg, dtype=torch.uint8, device=self.device)
+        self._all_gather(every, local)
+        for b in range(L.buffers):
+            self.codec.state_init(self.d, xs[b], self.recon_s[b], self.err[b])
+            for p in self.peers:
+                self.codec.state_init(self.d, at(every, p * L.buffers + b), self.recon_r[p][b], None)
+
+    def _enc_sets(self, xs):
+        L = self.layout
+        return [(xs[b], self.recon_s[b], self.err[b], L.codes(self.send, b), L.scales(self.send, b))
+                for b in range(L.buffers)]
+
+    def prepare(self, xs) -> None:
+        """Optional: build the codec's per-call state (the device array of
+        buffer pointers) for these input tensors ahead of their step."""
+        self._check(xs)
+        if hasattr(self.codec, "prepare_encode"):
+            self.codec.prepare_encode(self.d, self._enc_sets(xs))
+
+    def step(self, xs, events=None) -> None:
+        """One compressed step: encode into the payload, all-gather, decode
+        every peer's payload into its receiver states.  `events`, four CUDA
+        events, are recorded on the current stream before the encode, after
+        it, after the all-gather and after the decode."""
+        self._check(xs)
+        mark = (lambda i: events[i].record()) if events is not None else (lambda i: None)
+        mark(0)
+        self.codec.encode_batched(self.d, self._enc_sets(xs))
+        mark(1)
+        self._all_gather(self.recv, self.send)
+        mark(2)
+        self.codec.decode_batched(self.d, self._dec_sets)
+        mark(3)
+
+    def payload_bytes_per_step(self) -> int:
+        """Bytes this rank sends per compressed step."""
+        return self.layout.bytes_per_rank

@@ -66,6 +66,10 @@ def parse():
                     help="quantize: the receiver also writes the bf16 reconstruction")
     ap.add_argument("--delta", action="store_true",
                     help="quantize: delta-state sender (previous activation + error buffer)")
+    ap.add_argument("--exchange", action="store_true",
+                    help="quantize mode: the sequence-parallel exchange (encode into one payload, "
+                         "all-gather over the process group, decode every peer's shard; one GPU "
+                         "alone decodes its own payload)")
     ap.add_argument("--warm", action="store_true",
                     help="low-rank: warm start every encode after the first from the previous Q")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -463,6 +467,89 @@ def run_ours(args, world, rank, local):
     return out
 
 
+def run_exchange(args, world, rank, local):
+    """The sequence-parallel exchange: per step one batched encode into the
+    payload, one all-gather of the payloads, one batched decode of every
+    peer's shard (of its own too when alone)."""
+    from activation_residual_compression_cf_b200 import build, cf
+    from activation_residual_compression_cf_b200.exchange import ShardExchange
+    build.build()
+    cf.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = W.WORKLOADS[args.workload]
+    if args.buffers:
+        wl = W.replace(wl, buffers=args.buffers)
+    n, T, C, bits = wl.buffers, wl.tokens, wl.channels, wl.bits
+    S = max(2, min(wl.steps, int(40e9 // (n * T * C * 2))))
+    if args.gen_steps:
+        S = max(2, min(S, args.gen_steps))
+    X = torch.empty((S, n, T, C), dtype=torch.bfloat16, device=dev)
+    for b in range(n):
+        tr = W.Trajectory(wl, b, device=dev, seed=rank)
+        for s in range(S):
+            X[s, b] = tr.next()
+    ex = ShardExchange(T, C, bits, n, device=dev, loopback=(world == 1))
+    ex.warmup([X[0, b] for b in range(n)])
+    stream = torch.cuda.current_stream(dev)
+
+    def xs(i):
+        return [X[1 + i % (S - 1), b] for b in range(n)]
+
+    for i in range(S - 1):
+        ex.prepare(xs(i))
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for i in range(args.warmup):
+        ex.step(xs(i))
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with R.bracket():
+        wall0 = time.time()
+        t_start.record(stream)
+        for i in range(args.steps):
+            ex.step(xs(args.warmup + i), events=ev[i])
+        t_end.record(stream)
+    wall1 = time.time()
+    clocks = sampler.stop(wall0, wall1)
+    st = ex.codec.status_value()
+    assert st == 0, cf.cf_status_string(st)
+    ms = R.reduce_scalar(t_start.elapsed_time(t_end), "max")
+    phase = [statistics.mean(e[k].elapsed_time(e[k + 1]) for e in ev) for k in range(3)]
+    Wd = ex.layout.words_per_row
+    enc_bytes = n * T * (C * 2 + C * 4 * 3 + Wd * 4 + 4)
+    dec_bytes = len(ex.peers) * n * T * (Wd * 4 + 4 + C * 4 * 2)
+    peak, peak_kind = peaks()
+    enc_gbs = enc_bytes / (phase[0] / 1e3) / 1e9
+    value = 2 * T * C * n * args.steps * world / (ms / 1e3) / 1e9
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 in, fp32 state", "data": "synthetic",
+        "config": {"workload": args.workload, "tokens": T, "channels": C, "buffers": n,
+                   "bits": bits, "mode": f"{bits}-bit + EF, sequence-parallel exchange",
+                   "parallelism": f"sp{world} (all-gather of payloads)",
+                   "l2": "inputs larger than L2", "launches_per_step": 2},
+        "roofline": {"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(enc_gbs / peak, 4),
+                     "traffic": recorded_traffic("encode", args.workload),
+                     "kernel": "encode_tma_kernel (batched, codes written into the payload)",
+                     "peak_kind": peak_kind, "algorithmic_bytes_per_launch": enc_bytes,
+                     "avg_launch_ms": round(phase[0], 4)},
+        "exchange": {"encode_ms": round(phase[0], 4), "all_gather_ms": round(phase[1], 4),
+                     "decode_ms": round(phase[2], 4), "payload_bytes_per_rank": ex.payload_bytes_per_step(),
+                     "decoded_shards": len(ex.peers) * n,
+                     "decode_frac": round(dec_bytes / (phase[2] / 1e3) / 1e9 / peak, 4),
+                     "collective": ex.backend or "local copy (one rank)"},
+        "cpu_baseline": None, "e2e": None,
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+
+
 def run_lowrank(args, world, rank, local):
     """Low-rank mode: per step, cf_lowrank_encode then cf_lowrank_decode for
     every buffer (one workspace, reused in stream order)."""
@@ -846,6 +933,8 @@ def main():
     try:
         if W.WORKLOADS[args.workload].mode == "lowrank":
             out = run_lowrank(args, world, rank, local)
+        elif args.exchange:
+            out = run_exchange(args, world, rank, local)
         else:
             out = run_ours(args, world, rank, local)
         if rank == 0:

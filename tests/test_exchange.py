@@ -1,0 +1,142 @@
+"""Host logic of the sequence-parallel exchange (exchange.py) on CPU ranks:
+payload layout, the warmup's uncompressed all-gather, and the routing of
+every peer's payload into that peer's receiver states.  The ranks run on the
+gloo backend with the oracle standing in for libcf's kernels (the codec is
+injected by the test); each rank regenerates every shard's trajectory from
+the shared seeds and checks each receiver state bit for bit against the
+oracle run directly on that peer's shard."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+from activation_residual_compression_cf_b200.exchange import PayloadLayout
+
+
+class OracleCodec:
+    """The four codec methods of ShardExchange on CPU tensors, computed by
+    the oracle in place through numpy views."""
+
+    def __init__(self, bits):
+        self.bits = bits
+
+    def state_init(self, d, x, recon, err):
+        import oracle
+        from activation_residual_compression_cf_b200 import workloads as W
+        r, e = oracle.state_init(W.bf16_bits(x))
+        recon.copy_(torch.from_numpy(r))
+        if err is not None:
+            err.copy_(torch.from_numpy(e))
+
+    def encode_batched(self, d, sets):
+        import oracle
+        from activation_residual_compression_cf_b200 import workloads as W
+        for x, rs, e, c, s in sets:
+            codes, scales, err = oracle.encode(W.bf16_bits(x), rs.numpy(), self.bits)
+            c.numpy().view(np.uint32)[...] = codes
+            s.numpy()[...] = scales
+            e.numpy()[...] = err
+
+    def decode_batched(self, d, sets):
+        import oracle
+        for c, s, rr in sets:
+            oracle.decode(c.numpy().view(np.uint32).copy(), s.numpy().copy(), rr.numpy(), self.bits)
+
+
+@pytest.mark.parametrize("T,C,bits,B", [(48, 200, 1, 3), (1024, 3072, 2, 114), (7, 8, 2, 2),
+                                        (3, 33, 1, 5)])
+def test_payload_layout_is_aligned_and_disjoint(T, C, bits, B):
+    L = PayloadLayout(T, C, bits, B)
+    assert L.words_per_row == (C * bits + 31) // 32
+    spans = []
+    for b in range(B):
+        for off, n in ((L.codes_offset(b), L.codes_bytes), (L.scales_offset(b), L.scales_bytes)):
+            assert off % 16 == 0
+            spans.append((off, off + n))
+    spans.sort()
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+    assert spans[-1][1] <= L.bytes_per_rank
+    # the padding costs at most 30 bytes per buffer over the packed payload
+    assert L.bytes_per_rank - B * (L.codes_bytes + L.scales_bytes) <= 30 * B
+    p = torch.zeros(L.bytes_per_rank, dtype=torch.uint8)
+    assert L.codes(p, B - 1).shape == (T, L.words_per_row) and L.scales(p, 0).shape == (T,)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q, bits, loopback):
+    import datetime
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    try:
+        import torch.distributed as dist
+        import oracle
+        from activation_residual_compression_cf_b200 import workloads as W
+        from activation_residual_compression_cf_b200.exchange import ShardExchange
+        from test_exchange import OracleCodec
+        dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                                world_size=world, timeout=datetime.timedelta(seconds=60))
+        T, C, B, steps = 37, 203, 3, 4          # ragged: segments need padding
+        wl = W.replace(W.WORKLOADS["flux_sp"], tokens=world * T, channels=C, bits=bits, buffers=B)
+        trajs = [W.trajectory(wl, b, steps=steps) for b in range(B)]
+
+        def shard(x, p):
+            return x[p * T:(p + 1) * T].clone()
+
+        ex = ShardExchange(T, C, bits, B, device="cpu", codec=OracleCodec(bits), loopback=loopback)
+        ex.warmup([shard(trajs[b][0], rank) for b in range(B)])
+        for t in range(1, steps):
+            ex.step([shard(trajs[b][t], rank) for b in range(B)])
+        bad = []
+        for p in range(world):
+            for b in range(B):
+                r, _ = oracle.state_init(W.bf16_bits(shard(trajs[b][0], p)))
+                for t in range(1, steps):
+                    oracle.encode(W.bf16_bits(shard(trajs[b][t], p)), r, bits)
+                if p == rank and not np.array_equal(ex.recon_s[b].numpy(), r):
+                    bad.append(("sender", p, b))
+                if p in ex.peers and not np.array_equal(ex.recon_r[p][b].numpy(), r):
+                    bad.append(("receiver", p, b))
+                if p not in ex.peers and ex.recon_r[p] is not None:
+                    bad.append(("unexpected receiver", p))
+        q.put((rank, "ok" if not bad else "bad", bad, len(ex.peers)))
+        dist.destroy_process_group()
+    except Exception as e:
+        q.put((rank, "fail", repr(e), 0))
+
+
+@pytest.mark.parametrize("bits,loopback", [(1, False), (2, True)])
+def test_exchange_routes_every_peer_payload_world2(bits, loopback):
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_worker, args=(r, world, port, q, bits, loopback)) for r in range(world)]
+    for p in ps:
+        p.start()
+    out = sorted([q.get(timeout=180) for _ in range(world)], key=lambda t: t[0])
+    for p in ps:
+        p.join(timeout=60)
+    for rank, status, info, npeers in out:
+        assert status == "ok", (rank, info)
+        assert npeers == (world if loopback else world - 1)
+
+
+def test_exchange_rejects_bad_shapes():
+    from activation_residual_compression_cf_b200.exchange import ShardExchange
+    ex = ShardExchange(8, 64, 1, 2, device="cpu", codec=OracleCodec(1))
+    with pytest.raises(ValueError):
+        ex.step([torch.zeros(8, 64, dtype=torch.bfloat16)])
+    with pytest.raises(ValueError):
+        ex.step([torch.zeros(8, 64, dtype=torch.float32)] * 2)
+    with pytest.raises(ValueError):
+        ShardExchange(8, 64, 3, 2, device="cpu", codec=OracleCodec(1))

@@ -138,3 +138,27 @@ def test_ablations_reproduce_the_pages_ordering(bits):
     # error feedback keeps the reconstruction close; without it error builds
     # up; compressing full activations is worst of all
     assert errs["ef"] < 0.85 * errs["no_ef"] and errs["no_ef"] < 0.5 * errs["naive"], errs
+
+
+@pytest.mark.parametrize("bits", [1, 2])
+def test_two_step_warmup_matches_oracle(bits):
+    """The 2-step warmup the page reports as a variant ("Measured effects"):
+    steps 0 and 1 go uncompressed, i.e. both sides are initialised on x_0 and
+    again on x_1, and compression starts at step 2.  Teacher-forced parity
+    from there; the receiver mirrors the sender bit for bit."""
+    wl = W.replace(W.WORKLOADS["flux_sp"], tokens=96, bits=bits)
+    xs = [x.clone() for x in W.trajectory(wl, 3, steps=6, device="cuda")]
+    g = GpuBuffer(wl.tokens, wl.channels, bits)
+    g.init(xs[0])
+    g.init(xs[1])
+    h = g.host()
+    r1, e1 = oracle.state_init(W.bf16_bits(xs[1]))
+    assert np.array_equal(h["recon_s"], r1) and np.array_equal(h["recon_r"], r1)
+    assert not np.any(h["err"]) and not np.any(e1)
+    for t in range(2, len(xs)):
+        r0 = g.host()["recon_s"]
+        g.step(xs[t])
+        v, ora = oracle_step(W.bf16_bits(xs[t]), r0, bits)
+        gpu = g.host()
+        compare_step(bits, v, ora, gpu)
+        assert np.array_equal(gpu["recon_r"], gpu["recon_s"])

@@ -1,0 +1,81 @@
+"""The sequence-parallel exchange (exchange.py) on one GPU through libcf's
+kernels and a one-rank NCCL group, in loopback: the rank encodes its buffers
+into the payload, all-gathers it and decodes its own payload.  Every
+receiver state must equal the sender's mirror bit for bit, the payload's
+codes and scales must equal the single-buffer calls on the same inputs, and
+buffer 0 is checked step by step against the oracle (teacher-forced, the
+quantize parity bar)."""
+import datetime
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+
+import oracle
+from activation_residual_compression_cf_b200 import cf
+from activation_residual_compression_cf_b200 import workloads as W
+from activation_residual_compression_cf_b200.exchange import ShardExchange
+from _parity import compare_step, f32_of
+
+pytestmark = pytest.mark.gpu
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+@pytest.fixture(scope="module")
+def nccl_group():
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    yield
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("T,C,bits,B", [(1024, 3072, 2, 6), (100, 1003, 1, 3)])
+def test_exchange_loopback_matches_single_calls_and_oracle(nccl_group, T, C, bits, B):
+    wl = W.replace(W.WORKLOADS["flux_sp"], tokens=T, channels=C, bits=bits, buffers=B)
+    trajs = [W.trajectory(wl, b, steps=4, device="cuda") for b in range(B)]
+    ex = ShardExchange(T, C, bits, B, loopback=True)
+    assert ex.world == 1 and ex.backend == "nccl"
+    xs0 = [trajs[b][0].clone() for b in range(B)]
+    ex.warmup(xs0)
+    # the same buffers through the single-buffer calls
+    d = cf.desc(T, C, bits)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    ref = []
+    for b in range(B):
+        rs, e = torch.empty(T, C, **f32), torch.empty(T, C, **f32)
+        cf.cf_state_init(d, xs0[b], rs, e)
+        ref.append((rs, e, torch.empty(T, ex.layout.words_per_row, dtype=torch.int32, device="cuda"),
+                    torch.empty(T, **f32)))
+    for t in range(1, 4):
+        xs = [trajs[b][t].clone() for b in range(B)]
+        r0 = ex.recon_s[0].cpu().numpy()
+        ex.step(xs)
+        for b in range(B):
+            rs, e, c, s = ref[b]
+            cf.cf_encode(d, xs[b], rs, e, c, s)
+        torch.cuda.synchronize()
+        assert ex.codec.status_value() == 0
+        for b in range(B):
+            rs, e, c, s = ref[b]
+            assert torch.equal(ex.layout.codes(ex.recv, b), c), (t, b)
+            assert torch.equal(ex.layout.scales(ex.recv, b), s), (t, b)
+            assert torch.equal(ex.recon_s[b], rs) and torch.equal(ex.err[b], e), (t, b)
+            assert torch.equal(ex.recon_r[0][b], ex.recon_s[b]), (t, b)
+        xb = W.bf16_bits(xs[0])
+        v = (f32_of(xb) - r0).astype(np.float32)
+        ro = r0.copy()
+        co, so, eo = oracle.encode(xb, ro, bits)
+        gpu = dict(codes=ex.layout.codes(ex.send, 0).cpu().numpy().view(np.uint32),
+                   scales=ex.layout.scales(ex.send, 0).cpu().numpy(),
+                   err=ex.err[0].cpu().numpy(), recon_s=ex.recon_s[0].cpu().numpy())
+        compare_step(bits, v, dict(codes=co, scales=so, err=eo, recon_s=ro), gpu)
