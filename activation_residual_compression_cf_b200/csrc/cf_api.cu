@@ -158,6 +158,8 @@ cf_status launch_decode_t(const Src &src, int64_t T, int64_t C, int64_t rows, in
 
 // TMA-staged variants: C % 8 == 0 (16-byte rows) and, for decode, 16-byte
 // code rows (W % 4 == 0); at most 480 consumer threads.
+constexpr int kDecodeConsumerWarpsPerSM = 12;
+
 template <bool ENC, int BITS, int GPT, class Src>
 cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t *status,
                      const Shape &s, int stages_req, cudaStream_t st) {
@@ -191,7 +193,15 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
         (void)cudaGetLastError();
         occ = 1;
     }
-    if (s.blocks_per_sm > 0 && s.blocks_per_sm < occ) occ = s.blocks_per_sm;
+    if (s.blocks_per_sm > 0) {
+        if (s.blocks_per_sm < occ) occ = s.blocks_per_sm;
+    } else if constexpr (!ENC) {
+        // Decode: measured on B200 (C = 1920 and 3072, ring depths 3-7), the
+        // rate depends on the consumer warps per SM and peaks at 12 (6.4-6.6
+        // TB/s); 15 or 9 lose 10-14 %.  Cap the CTAs per SM accordingly.
+        const int cap = kDecodeConsumerWarpsPerSM / (s.threads / 32);
+        if (cap >= 1 && cap < occ) occ = cap;
+    }
     int64_t grid = (int64_t)device_sm_count() * occ;
     if (grid > rows) grid = rows;
     if (grid < 1) grid = 1;
