@@ -238,3 +238,39 @@ def _full_size_steps(wl, d, n, steps, sample, trs, st, x_buf, enc, dec, status, 
                       scales=st["scales"][b].cpu().numpy(), err=st["err"][b].cpu().numpy(),
                       recon_s=st["recon_s"][b].cpu().numpy())
             compare_step(wl.bits, v, ora, gh)
+
+
+@pytest.mark.parametrize("pipeline,bits", [(1, 2), (0, 1)])
+def test_single_buffer_beyond_2_pow_31_elements(pipeline, bits):
+    """One buffer of 700,000 x 3072 = 2.15e9 elements, past 2^31, so every
+    element offset beyond row 699,050 needs 64-bit arithmetic (about 35 GB on
+    the device).  Rows on both sides of that boundary, the first and last
+    rows and random rows are checked against the oracle, which computes rows
+    independently; the receiver must equal the sender everywhere."""
+    T, C = 700_000, 3072
+    assert T * C > 2 ** 31
+    gen = torch.Generator(device="cuda").manual_seed(11)
+    gain = torch.exp(0.5 * torch.randn(C, device="cuda", generator=gen))
+    x0 = (torch.randn(T, C, device="cuda", generator=gen) * gain).to(torch.bfloat16)
+    x1 = (x0.float() + 0.05 * gain * torch.randn(T, C, device="cuda", generator=gen)).to(torch.bfloat16)
+    cf.cf_set_quant_pipeline(0, pipeline, 0)
+    cf.cf_set_quant_pipeline(1, pipeline, 0)
+    try:
+        g = GpuBuffer(T, C, bits)
+        g.init(x0)
+        g.step(x1)
+        torch.cuda.synchronize()
+        assert torch.equal(g.recon_r, g.recon_s)
+        edge = 2 ** 31 // C
+        rng = np.random.default_rng(5)
+        rows = np.unique(np.concatenate([[0, 1, T - 2, T - 1], np.arange(edge - 3, edge + 4),
+                                         rng.integers(0, T, 16)]))
+        idx = torch.from_numpy(rows).cuda()
+        r0, _ = oracle.state_init(W.bf16_bits(x0[idx]))
+        v, ora = oracle_step(W.bf16_bits(x1[idx]), r0, bits)
+        gpu = dict(codes=g.codes[idx].cpu().numpy().view(np.uint32), scales=g.scales[idx].cpu().numpy(),
+                   err=g.err[idx].cpu().numpy(), recon_s=g.recon_s[idx].cpu().numpy())
+        compare_step(bits, v, ora, gpu)
+    finally:
+        cf.cf_set_quant_pipeline(0, 1, 0)
+        cf.cf_set_quant_pipeline(1, 1, 0)
