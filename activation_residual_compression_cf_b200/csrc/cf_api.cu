@@ -90,7 +90,7 @@ Shape choose_shape(int kernel, int64_t C, int pipeline, int bits, bool delta = f
     int gpt;
     if (pipeline == 1) {
         if (kernel == 0)
-            gpt = bits == 1 ? (delta ? 2 : 3) : 4;
+            gpt = delta ? (bits == 1 ? 2 : 4) : 2;
         else
             gpt = 3;
     } else {
@@ -166,8 +166,10 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
     const int64_t W = (C * BITS + 31) / 32;
     int64_t slot = 4 * W + 4 * C;
     if constexpr (ENC) slot = (Src::kDelta ? 8 : 6) * C;
-    // Ring depth: measured on B200 (C = 1920 and 3072), 5 slots for both
-    // kernels are at or near the best; deeper rings cost CTAs per SM.  The
+    // Ring depth, measured on B200 (C = 1920 and 3072) in runs long enough
+    // for the power cap to hold the SM clock down, as in sustained use:
+    // encode 4 slots (with 2 groups per thread that keeps 3-4 CTAs and 16-18
+    // consumer warps per SM, 6-8 % above 5 slots at 2 CTAs); decode 5.  The
     // delta-state encode's slots are a third larger (8C bytes): 3 slots,
     // which keep three CTAs per SM, beat 4 (two CTAs) by ~10 %.
     int stages = stages_req;
@@ -175,7 +177,8 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
         bool delta = false;
         if constexpr (ENC) delta = Src::kDelta;
         stages = (int)((delta ? 75000 : 120000) / slot);
-        if (stages > 5) stages = 5;
+        const int cap = (ENC && !delta) ? 4 : 5;
+        if (stages > cap) stages = cap;
     }
     if (stages > 8) stages = 8;
     if (stages < 2) stages = 2;
