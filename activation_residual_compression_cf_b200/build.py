@@ -9,6 +9,7 @@ the driver (libcuda) at run time.
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import subprocess
 import sys
@@ -18,6 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libcf.so")
+STAMP = LIB + ".sources"    # hash of the inputs the library was built from
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -34,16 +36,31 @@ def _deps():
             + glob.glob(os.path.join(INCLUDE, "*.h")) + [__file__])
 
 
+def _inputs_hash() -> str:
+    """Content hash of every source, header and flag the library depends on.
+    File times are not used: a copy of the tree to another machine may round
+    them, and a source edited within the same second as the build would then
+    look older than the library."""
+    h = hashlib.sha256()
+    h.update(" ".join([NVCC, *ARCH, *FLAGS]).encode())
+    for p in sorted(_deps()):
+        h.update(os.path.relpath(p, ROOT).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(p) <= t for p in _deps())
+    with open(STAMP) as f:
+        return f.read().strip() == _inputs_hash()
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
+    digest = _inputs_hash()
     objdir = os.path.join(ROOT, "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = []
@@ -58,6 +75,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     tmp = LIB + f".tmp{os.getpid()}"
     subprocess.check_call([NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp])
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(digest + "\n")
     return LIB
 
 

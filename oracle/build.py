@@ -6,6 +6,7 @@ rounding sequence its comments state.
 """
 from __future__ import annotations
 
+import hashlib
 import os
 import subprocess
 import sys
@@ -17,13 +18,28 @@ CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
           "-fno-fast-math", "-fno-finite-math-only", "-Wall", "-Wextra"]
 
 
+STAMP = LIB + ".sources"    # hash of the source and flags the library was built from
+
+
+def _inputs_hash() -> str:
+    # content, not file times: a copy of the tree may round the times
+    h = hashlib.sha256(" ".join(CFLAGS).encode())
+    with open(SRC, "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()
+
+
 def build(force: bool = False) -> str:
-    if (not force and os.path.exists(LIB)
-            and os.path.getmtime(LIB) >= os.path.getmtime(SRC)):
-        return LIB
+    digest = _inputs_hash()
+    if not force and os.path.exists(LIB) and os.path.exists(STAMP):
+        with open(STAMP) as f:
+            if f.read().strip() == digest:
+                return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     subprocess.check_call(["gcc", *CFLAGS, SRC, "-o", tmp, "-lm"])
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(digest + "\n")
     return LIB
 
 
