@@ -1,11 +1,11 @@
 """Replica plumbing for multi-GPU runs of the codec (one process per GPU).
 
-In this build the codec has no exchange between GPUs: each rank compresses
-and decompresses its own buffers (in sequence-parallel serving each GPU owns
-its shard's activations).  N ranks are therefore N independent replicas; the
-only cross-rank operations are host-side plumbing: a barrier around a timed
-region and a max/sum of per-rank numbers.  torch.distributed provides it
-(NCCL on GPUs, gloo on CPU).
+In the default multi-GPU run each rank compresses and decompresses its own
+buffers, so N ranks are N independent replicas.  The only cross-rank
+operations are host-side plumbing: a barrier around a timed region and a
+max or sum of per-rank numbers.  torch.distributed provides them (NCCL on
+GPUs, gloo on CPU).  The exchange of payloads between ranks is in
+exchange.py.
 """
 from __future__ import annotations
 

@@ -15,13 +15,16 @@ seeded synthetic drift trajectories, pre-generated in HBM before timing; one
 step touches ~5 GB (FLUX-like shard), far more than the 126 MB L2, so no L2
 flush is needed between steps.
 
-Multi-GPU: the path has no exchange between GPUs in this build (sender and
-receiver share a device), so N ranks run N independent replicas of the
-workload ("weak" scaling); the timed region is bracketed by barriers and the
-max over ranks is reported.
+Multi-GPU: by default sender and receiver share a device, so N ranks run N
+independent replicas of the workload ("weak" scaling).  The timed region is
+bracketed by barriers and the max over ranks is reported.  --exchange runs
+the sequence-parallel exchange instead: each step encodes into one payload,
+all-gathers the payloads over NCCL and decodes every peer's shard.
 
---impl reference times the CPU oracle (plain C, one core) on a bounded
-sample of the same workload, with the same metric and unit.
+--workload lowrank times the low-rank mode (rank 32, INT4 factors).
+--impl reference times the CPU oracle on a bounded sample of the same
+workload, with the same metric and unit: the plain C oracle on one core for
+the quantize workloads, the numpy fp64 oracle for the low-rank one.
 """
 from __future__ import annotations
 
