@@ -21,7 +21,7 @@ the current stream:
 
 The arithmetic runs in libcf's kernels (``CudaCodec``); this module lays out
 memory and orders the calls.  A caller may pass another codec object with
-the same four methods (the CPU tests drive the host logic that way).
+the same methods (the CPU tests drive the host logic that way).
 """
 from __future__ import annotations
 
@@ -125,6 +125,11 @@ class CudaCodec:
         if sets:
             cf.cf_decode_batched(d, len(sets), self._array("dec", sets, cf.dec_buffer_array), self.status)
 
+    def decode_emit_batched(self, d, sets):
+        if sets:
+            cf.cf_decode_emit_batched(d, len(sets), self._array("emit", sets, cf.dec_emit_buffer_array),
+                                      self.status)
+
     def status_value(self) -> int:
         """First error any batched call recorded (synchronises)."""
         return int(self.status.item())
@@ -139,10 +144,12 @@ class ShardExchange:
     rank's own shard and decodes its own payload, which on one GPU runs the
     whole path (its reconstruction must equal the sender's mirror bit for
     bit).  recon_r[p][b] is the reconstruction of peer p's buffer b (None for
-    the rank's own shard unless `loopback`)."""
+    the rank's own shard unless `loopback`).  With `emit`, the decode also
+    writes out[p][b], the bf16 rounding of recon_r[p][b] that attention
+    reads, in the same pass (the codec's decode_emit_batched)."""
 
     def __init__(self, tokens: int, channels: int, bits: int, buffers: int, *, group=None,
-                 device=None, codec=None, loopback: bool = False):
+                 device=None, codec=None, loopback: bool = False, emit: bool = False):
         if bits not in (1, 2):
             raise ValueError(f"bits must be 1 or 2, got {bits}")
         if tokens < 1 or channels < 1 or buffers < 1:
@@ -169,8 +176,13 @@ class ShardExchange:
         self.peers = [p for p in range(self.world) if loopback or p != self.rank]
         self.recon_r = [[torch.empty(tokens, channels, **f32) for _ in range(buffers)]
                         if p in self.peers else None for p in range(self.world)]
+        self.emit = emit
+        self.out = [[torch.empty(tokens, channels, dtype=torch.bfloat16, device=self.device)
+                     for _ in range(buffers)] if emit and p in self.peers else None
+                    for p in range(self.world)]
         self._dec_sets = [(self.layout.codes(self._payload(p), b), self.layout.scales(self._payload(p), b),
-                           self.recon_r[p][b]) for p in self.peers for b in range(buffers)]
+                           self.recon_r[p][b]) + ((self.out[p][b],) if emit else ())
+                          for p in self.peers for b in range(buffers)]
 
     def _payload(self, p: int) -> torch.Tensor:
         n = self.layout.bytes_per_rank
@@ -214,6 +226,8 @@ class ShardExchange:
             self.codec.state_init(self.d, xs[b], self.recon_s[b], self.err[b])
             for p in self.peers:
                 self.codec.state_init(self.d, at(every, p * L.buffers + b), self.recon_r[p][b], None)
+                if self.emit:
+                    self.out[p][b].copy_(at(every, p * L.buffers + b))
 
     def _enc_sets(self, xs):
         L = self.layout
@@ -239,7 +253,10 @@ class ShardExchange:
         mark(1)
         self._all_gather(self.recv, self.send)
         mark(2)
-        self.codec.decode_batched(self.d, self._dec_sets)
+        if self.emit:
+            self.codec.decode_emit_batched(self.d, self._dec_sets)
+        else:
+            self.codec.decode_batched(self.d, self._dec_sets)
         mark(3)
 
     def payload_bytes_per_step(self) -> int:

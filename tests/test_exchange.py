@@ -45,6 +45,13 @@ class OracleCodec:
         for c, s, rr in sets:
             oracle.decode(c.numpy().view(np.uint32).copy(), s.numpy().copy(), rr.numpy(), self.bits)
 
+    def decode_emit_batched(self, d, sets):
+        import oracle
+        for c, s, rr, o in sets:
+            out = oracle.decode_emit(c.numpy().view(np.uint32).copy(), s.numpy().copy(), rr.numpy(),
+                                     self.bits)
+            o.view(torch.int16).numpy().view(np.uint16)[...] = out
+
 
 @pytest.mark.parametrize("T,C,bits,B", [(48, 200, 1, 3), (1024, 3072, 2, 114), (7, 8, 2, 2),
                                         (3, 33, 1, 5)])
@@ -73,7 +80,7 @@ def _free_port():
     return p
 
 
-def _worker(rank, world, port, q, bits, loopback):
+def _worker(rank, world, port, q, bits, loopback, emit=False):
     import datetime
     import sys
     sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
@@ -92,7 +99,8 @@ def _worker(rank, world, port, q, bits, loopback):
         def shard(x, p):
             return x[p * T:(p + 1) * T].clone()
 
-        ex = ShardExchange(T, C, bits, B, device="cpu", codec=OracleCodec(bits), loopback=loopback)
+        ex = ShardExchange(T, C, bits, B, device="cpu", codec=OracleCodec(bits), loopback=loopback,
+                           emit=emit)
         ex.warmup([shard(trajs[b][0], rank) for b in range(B)])
         for t in range(1, steps):
             ex.step([shard(trajs[b][t], rank) for b in range(B)])
@@ -106,6 +114,8 @@ def _worker(rank, world, port, q, bits, loopback):
                     bad.append(("sender", p, b))
                 if p in ex.peers and not np.array_equal(ex.recon_r[p][b].numpy(), r):
                     bad.append(("receiver", p, b))
+                if emit and p in ex.peers and not torch.equal(ex.out[p][b], torch.from_numpy(r).to(torch.bfloat16)):
+                    bad.append(("emitted bf16", p, b))
                 if p not in ex.peers and ex.recon_r[p] is not None:
                     bad.append(("unexpected receiver", p))
         q.put((rank, "ok" if not bad else "bad", bad, len(ex.peers)))
@@ -114,13 +124,14 @@ def _worker(rank, world, port, q, bits, loopback):
         q.put((rank, "fail", repr(e), 0))
 
 
-@pytest.mark.parametrize("bits,loopback", [(1, False), (2, True)])
-def test_exchange_routes_every_peer_payload_world2(bits, loopback):
+@pytest.mark.parametrize("bits,loopback,emit", [(1, False, False), (2, True, False), (2, False, True)])
+def test_exchange_routes_every_peer_payload_world2(bits, loopback, emit):
     world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    ps = [ctx.Process(target=_worker, args=(r, world, port, q, bits, loopback)) for r in range(world)]
+    ps = [ctx.Process(target=_worker, args=(r, world, port, q, bits, loopback, emit))
+          for r in range(world)]
     for p in ps:
         p.start()
     out = sorted([q.get(timeout=180) for _ in range(world)], key=lambda t: t[0])

@@ -79,3 +79,25 @@ def test_exchange_loopback_matches_single_calls_and_oracle(nccl_group, T, C, bit
                    scales=ex.layout.scales(ex.send, 0).cpu().numpy(),
                    err=ex.err[0].cpu().numpy(), recon_s=ex.recon_s[0].cpu().numpy())
         compare_step(bits, v, dict(codes=co, scales=so, err=eo, recon_s=ro), gpu)
+
+
+def test_exchange_emits_the_bf16_reconstruction(nccl_group):
+    """With emit, the receivers' bf16 copy equals the warmup activation after
+    the warmup and the bf16 rounding of the reconstruction after each step."""
+    T, C, bits, B = 256, 3072, 2, 4
+    wl = W.replace(W.WORKLOADS["flux_sp"], tokens=T, channels=C, bits=bits, buffers=B)
+    trajs = [W.trajectory(wl, b, steps=3, device="cuda") for b in range(B)]
+    ex = ShardExchange(T, C, bits, B, loopback=True, emit=True)
+    xs0 = [trajs[b][0].clone() for b in range(B)]
+    ex.warmup(xs0)
+    torch.cuda.synchronize()
+    for b in range(B):
+        assert torch.equal(ex.out[0][b], xs0[b])
+    for t in (1, 2):
+        ex.step([trajs[b][t].clone() for b in range(B)])
+        torch.cuda.synchronize()
+        assert ex.codec.status_value() == 0
+        for b in range(B):
+            assert torch.equal(ex.recon_r[0][b], ex.recon_s[b])
+            ref = ex.recon_r[0][b].to(torch.bfloat16)
+            assert torch.equal(ex.out[0][b].view(torch.int16), ref.view(torch.int16)), (t, b)
