@@ -17,7 +17,6 @@ import json
 import os
 
 import numpy as np
-import pytest
 
 from oracle import lowrank as L
 from conftest import GOLDEN

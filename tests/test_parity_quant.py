@@ -16,7 +16,7 @@ import oracle
 from activation_residual_compression_cf_b200 import cf
 from activation_residual_compression_cf_b200 import workloads as W
 
-from _parity import GpuBuffer, compare_step, f32_of, oracle_step
+from _parity import GpuBuffer, compare_step, oracle_step
 
 pytestmark = pytest.mark.gpu
 
