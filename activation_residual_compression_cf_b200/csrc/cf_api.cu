@@ -81,9 +81,9 @@ struct Shape {
 
 // Launch shape per row: threads (a multiple of 32) x groups of 8 channels
 // per thread.  Chosen from sweeps on B200 timed in the encode -> decode
-// sequence (C = 3072, 114 x 1024 and 114 x 4096 rows): TMA encode is fastest
-// with 4 groups per thread at 2 bits and 3 at 1 bit (delta-state encode: 4
-// and 2), TMA decode with 3; the register pipeline with 2.
+// sequence (C = 1920 and 3072): TMA encode 2 groups per thread under the
+// sustained power cap (delta-state encode: 2 at 1 bit, 4 at 2 bits), TMA
+// decode 3; the register pipeline 2.
 Shape choose_shape(int kernel, int64_t C, int pipeline, int bits, bool delta = false) {
     const int64_t G = (C + 7) / 8;
     Shape s;
