@@ -151,3 +151,49 @@ def test_exchange_rejects_bad_shapes():
         ex.step([torch.zeros(8, 64, dtype=torch.float32)] * 2)
     with pytest.raises(ValueError):
         ShardExchange(8, 64, 3, 2, device="cpu", codec=OracleCodec(1))
+
+
+def _leaver(rank, world, port, q):
+    import datetime
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    try:
+        import torch.distributed as dist
+        from activation_residual_compression_cf_b200 import workloads as W
+        from activation_residual_compression_cf_b200.exchange import ShardExchange
+        from test_exchange import OracleCodec
+        dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                                world_size=world, timeout=datetime.timedelta(seconds=5))
+        T, C, bits = 16, 64, 1
+        wl = W.replace(W.WORKLOADS["tiny"], tokens=world * T, channels=C)
+        xs = W.trajectory(wl, 0, steps=3)
+        ex = ShardExchange(T, C, bits, 1, device="cpu", codec=OracleCodec(bits))
+        ex.warmup([xs[0][rank * T:(rank + 1) * T].clone()])
+        ex.step([xs[1][rank * T:(rank + 1) * T].clone()])
+        if rank == 1:
+            q.put((rank, "left"))
+            q.close()
+            q.join_thread()
+            os._exit(0)                       # leaves between steps, nothing in flight
+        try:
+            ex.step([xs[2][rank * T:(rank + 1) * T].clone()])
+            q.put((rank, "no error"))
+        except Exception as e:                # the gather times out or the peer's socket closed
+            q.put((rank, "error", type(e).__name__))
+    except Exception as e:
+        q.put((rank, "fail", repr(e)))
+
+
+def test_a_rank_that_leaves_ends_the_survivors_next_step_with_an_error():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_leaver, args=(r, world, port, q)) for r in range(world)]
+    for p in ps:
+        p.start()
+    out = sorted([q.get(timeout=180) for _ in range(world)], key=lambda t: t[0])
+    for p in ps:
+        p.join(timeout=60)
+    assert out[1][1] == "left", out
+    assert out[0][1] == "error", out
