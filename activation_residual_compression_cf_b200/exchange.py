@@ -259,6 +259,35 @@ class ShardExchange:
             self.codec.decode_batched(self.d, self._dec_sets)
         mark(3)
 
+    def state_dict(self) -> dict:
+        """Everything a resumed exchange needs, as host copies, taken between
+        steps: this rank's sender state (recon_s, err) and its receivers'
+        reconstructions (and bf16 copies when emitting)."""
+        host = lambda ts: [t.detach().cpu().clone() for t in ts]  # noqa: E731
+        sd = {"layout": dataclasses.asdict(self.layout), "rank": self.rank, "world": self.world,
+              "recon_s": host(self.recon_s), "err": host(self.err),
+              "recon_r": {p: host(self.recon_r[p]) for p in self.peers}}
+        if self.emit:
+            sd["out"] = {p: host(self.out[p]) for p in self.peers}
+        return sd
+
+    def load_state_dict(self, sd: dict) -> None:
+        """Restore a state_dict taken on the same rank of an exchange with
+        the same layout, world size, peers and emit setting."""
+        if (sd["layout"] != dataclasses.asdict(self.layout) or sd["rank"] != self.rank
+                or sd["world"] != self.world or sorted(sd["recon_r"]) != self.peers
+                or ("out" in sd) != self.emit):
+            raise ValueError("state_dict was taken on a different exchange")
+        for dst, src in ((self.recon_s, sd["recon_s"]), (self.err, sd["err"])):
+            for d, s_ in zip(dst, src):
+                d.copy_(s_)
+        for p in self.peers:
+            for d, s_ in zip(self.recon_r[p], sd["recon_r"][p]):
+                d.copy_(s_)
+            if self.emit:
+                for d, s_ in zip(self.out[p], sd["out"][p]):
+                    d.copy_(s_)
+
     def payload_bytes_per_step(self) -> int:
         """Bytes this rank sends per compressed step."""
         return self.layout.bytes_per_rank

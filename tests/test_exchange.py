@@ -197,3 +197,68 @@ def test_a_rank_that_leaves_ends_the_survivors_next_step_with_an_error():
         p.join(timeout=60)
     assert out[1][1] == "left", out
     assert out[0][1] == "error", out
+
+
+def _resumer(rank, world, port, q):
+    import datetime
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    try:
+        import torch.distributed as dist
+        from activation_residual_compression_cf_b200 import workloads as W
+        from activation_residual_compression_cf_b200.exchange import ShardExchange
+        from test_exchange import OracleCodec
+        dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                                world_size=world, timeout=datetime.timedelta(seconds=60))
+        T, C, bits, B = 24, 96, 2, 2
+        wl = W.replace(W.WORKLOADS["flux_sp"], tokens=world * T, channels=C, bits=bits, buffers=B)
+        trajs = [W.trajectory(wl, b, steps=5) for b in range(B)]
+
+        def xs(t):
+            return [trajs[b][t][rank * T:(rank + 1) * T].clone() for b in range(B)]
+
+        def make():
+            return ShardExchange(T, C, bits, B, device="cpu", codec=OracleCodec(bits), emit=True)
+        whole, first = make(), make()
+        whole.warmup(xs(0))
+        first.warmup(xs(0))
+        for t in (1, 2):
+            whole.step(xs(t))
+            first.step(xs(t))
+        sd = first.state_dict()
+        del first
+        resumed = make()
+        resumed.load_state_dict(sd)
+        for t in (3, 4):
+            whole.step(xs(t))
+            resumed.step(xs(t))
+        same = all(torch.equal(a, b) for a, b in zip(whole.recon_s + whole.err, resumed.recon_s + resumed.err))
+        for p in whole.peers:
+            same &= all(torch.equal(a, b) for a, b in zip(whole.recon_r[p], resumed.recon_r[p]))
+            same &= all(torch.equal(a, b) for a, b in zip(whole.out[p], resumed.out[p]))
+        bad = make()
+        sd["world"] = world + 1
+        try:
+            bad.load_state_dict(sd)
+            rejected = False
+        except ValueError:
+            rejected = True
+        q.put((rank, "ok" if same and rejected else "bad", same, rejected))
+        dist.destroy_process_group()
+    except Exception as e:
+        q.put((rank, "fail", repr(e), None))
+
+
+def test_exchange_resumes_bit_for_bit_from_a_state_dict_world2():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_resumer, args=(r, world, port, q)) for r in range(world)]
+    for p in ps:
+        p.start()
+    out = sorted([q.get(timeout=180) for _ in range(world)], key=lambda t: t[0])
+    for p in ps:
+        p.join(timeout=60)
+    for o in out:
+        assert o[1] == "ok", o
