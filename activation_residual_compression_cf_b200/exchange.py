@@ -19,6 +19,10 @@ the current stream:
 3. one batched decode of every peer's payload into that peer's receiver
    states.
 
+``ShardExchange`` carries the quantize mode (1- or 2-bit codes and per-token
+scales), ``LowrankShardExchange`` the low-rank mode (INT4 factors P and Q
+and their column scales).
+
 The arithmetic runs in libcf's kernels (``CudaCodec``); this module lays out
 memory and orders the calls.  A caller may pass another codec object with
 the same methods (the CPU tests drive the host logic that way).
@@ -36,6 +40,10 @@ from . import cf
 
 def _align16(n: int) -> int:
     return (n + 15) & ~15
+
+
+def _seg(payload: torch.Tensor, off: int, nbytes: int) -> torch.Tensor:
+    return payload[off:off + nbytes]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -88,11 +96,57 @@ class PayloadLayout:
         return payload[o:o + self.scales_bytes].view(torch.float32)
 
 
+@dataclasses.dataclass(frozen=True)
+class LowrankPayloadLayout:
+    """Where each buffer's low-rank payload sits in one rank's payload.
+
+    Per buffer, in buffer order, each segment on a 16-byte boundary: the
+    packed INT4 codes of P (uint8 [tokens, ceil(rank/2)]), P's column scales
+    (fp32 [rank]), the packed codes of Q (uint8 [channels, ceil(rank/2)]),
+    Q's column scales (fp32 [rank])."""
+    tokens: int
+    channels: int
+    rank: int
+    buffers: int
+
+    @property
+    def nibble_bytes(self) -> int:
+        return (self.rank + 1) // 2
+
+    def _sizes(self):
+        nb = self.nibble_bytes
+        return (self.tokens * nb, 4 * self.rank, self.channels * nb, 4 * self.rank)
+
+    def _offsets(self):
+        offs, o = [], 0
+        for n in self._sizes():
+            offs.append(o)
+            o += _align16(n)
+        return offs, o
+
+    @property
+    def stride(self) -> int:
+        return self._offsets()[1]
+
+    @property
+    def bytes_per_rank(self) -> int:
+        return self.buffers * self.stride
+
+    def parts(self, payload: torch.Tensor, b: int):
+        """(p_codes, p_scales, q_codes, q_scales) views of buffer b."""
+        offs, _ = self._offsets()
+        base = b * self.stride
+        pc, ps, qc, qs = (_seg(payload, base + o, n) for o, n in zip(offs, self._sizes()))
+        nb = self.nibble_bytes
+        return (pc.view(self.tokens, nb), ps.view(torch.float32), qc.view(self.channels, nb),
+                qs.view(torch.float32))
+
+
 class CudaCodec:
-    """The product path: libcf's batched encode / decode kernels.  The device
-    arrays of buffer pointers are kept for the last `cache` pointer sets, so
-    inputs that cycle through a fixed set of tensors cost no host-to-device
-    copy of pointers per step."""
+    """The product path: libcf's batched kernels.  The device arrays of
+    buffer pointers are kept for the last `cache` pointer sets, so inputs
+    that cycle through a fixed set of tensors cost no host-to-device copy of
+    pointers per step."""
 
     def __init__(self, device: torch.device, cache: int = 64):
         self.device = device
@@ -101,7 +155,7 @@ class CudaCodec:
         self._cache_size = cache
 
     def _array(self, kind, sets, make):
-        key = (kind,) + tuple(t.data_ptr() for s in sets for t in s)
+        key = (kind,) + tuple(0 if t is None else t.data_ptr() for s in sets for t in s)
         arr = self._cache.get(key)
         if arr is None:
             arr = make(sets, self.device)
@@ -130,28 +184,33 @@ class CudaCodec:
             cf.cf_decode_emit_batched(d, len(sets), self._array("emit", sets, cf.dec_emit_buffer_array),
                                       self.status)
 
+    def lowrank_workspace_bytes(self, d) -> int:
+        return cf.cf_lowrank_workspace_bytes(d)
+
+    def lowrank_status(self, workspace_slice) -> int:
+        return cf.cf_lowrank_status(workspace_slice)
+
+    def lowrank_encode_batched(self, d, sets, workspace):
+        cf.cf_lowrank_encode_batched(d, len(sets), self._array("lr_enc", sets, cf.lowrank_buffer_array),
+                                     workspace)
+
+    def lowrank_decode_batched(self, d, sets):
+        if sets:
+            cf.cf_lowrank_decode_batched(d, len(sets),
+                                         self._array("lr_dec", sets, cf.lowrank_dec_buffer_array),
+                                         self.status)
+
     def status_value(self) -> int:
         """First error any batched call recorded (synchronises)."""
         return int(self.status.item())
 
 
-class ShardExchange:
-    """Sender state for this rank's shard of `buffers` activations and
-    receiver states for every peer's shard, plus the payload buffers.
+class _Exchange:
+    """What both modes share: the process group, this rank's sender state
+    for its shard of `buffers` activations, a receiver state per peer, the
+    payload buffers, the warmup and checkpoints."""
 
-    tokens, channels: this rank's shard of one buffer (every rank's shard has
-    the same shape); bits: 1 or 2.  `loopback` also keeps a receiver for the
-    rank's own shard and decodes its own payload, which on one GPU runs the
-    whole path (its reconstruction must equal the sender's mirror bit for
-    bit).  recon_r[p][b] is the reconstruction of peer p's buffer b (None for
-    the rank's own shard unless `loopback`).  With `emit`, the decode also
-    writes out[p][b], the bf16 rounding of recon_r[p][b] that attention
-    reads, in the same pass (the codec's decode_emit_batched)."""
-
-    def __init__(self, tokens: int, channels: int, bits: int, buffers: int, *, group=None,
-                 device=None, codec=None, loopback: bool = False, emit: bool = False):
-        if bits not in (1, 2):
-            raise ValueError(f"bits must be 1 or 2, got {bits}")
+    def __init__(self, layout, d, tokens, channels, buffers, group, device, codec, loopback):
         if tokens < 1 or channels < 1 or buffers < 1:
             raise ValueError("tokens, channels and buffers must be positive")
         self.group = group
@@ -165,9 +224,9 @@ class ShardExchange:
             device = torch.device("cuda", torch.cuda.current_device())
         self.device = torch.device(device)
         self.codec = codec if codec is not None else CudaCodec(self.device)
-        self.layout = PayloadLayout(tokens, channels, bits, buffers)
-        self.d = cf.desc(tokens, channels, bits)
-        n = self.layout.bytes_per_rank
+        self.layout, self.d = layout, d
+        self.tokens, self.channels, self.buffers = tokens, channels, buffers
+        n = layout.bytes_per_rank
         self.send = torch.zeros(n, dtype=torch.uint8, device=self.device)
         self.recv = torch.zeros(self.world * n, dtype=torch.uint8, device=self.device)
         f32 = dict(dtype=torch.float32, device=self.device)
@@ -176,13 +235,8 @@ class ShardExchange:
         self.peers = [p for p in range(self.world) if loopback or p != self.rank]
         self.recon_r = [[torch.empty(tokens, channels, **f32) for _ in range(buffers)]
                         if p in self.peers else None for p in range(self.world)]
-        self.emit = emit
-        self.out = [[torch.empty(tokens, channels, dtype=torch.bfloat16, device=self.device)
-                     for _ in range(buffers)] if emit and p in self.peers else None
-                    for p in range(self.world)]
-        self._dec_sets = [(self.layout.codes(self._payload(p), b), self.layout.scales(self._payload(p), b),
-                           self.recon_r[p][b]) + ((self.out[p][b],) if emit else ())
-                          for p in self.peers for b in range(buffers)]
+        self.emit = False
+        self.out = [None] * self.world
 
     def _payload(self, p: int) -> torch.Tensor:
         n = self.layout.bytes_per_rank
@@ -197,11 +251,11 @@ class ShardExchange:
             dist.all_gather(list(out.chunk(self.world)), inp, group=self.group)
 
     def _check(self, xs):
-        L = self.layout
-        if len(xs) != L.buffers:
-            raise ValueError(f"expected {L.buffers} activations, got {len(xs)}")
+        if len(xs) != self.buffers:
+            raise ValueError(f"expected {self.buffers} activations, got {len(xs)}")
         for x in xs:
-            if x.dtype != torch.bfloat16 or tuple(x.shape) != (L.tokens, L.channels) or not x.is_contiguous():
+            if (x.dtype != torch.bfloat16 or tuple(x.shape) != (self.tokens, self.channels)
+                    or not x.is_contiguous()):
                 raise ValueError("each activation must be a contiguous bf16 [tokens, channels] tensor")
             if x.data_ptr() % 16:
                 raise ValueError("each activation must start on a 16-byte boundary")
@@ -210,54 +264,24 @@ class ShardExchange:
         """Step 0: exchange the activations uncompressed; every receiver
         state starts from the exact activation and the error buffers from 0."""
         self._check(xs)
-        L = self.layout
-        n = L.tokens * L.channels * 2
+        T, C, B = self.tokens, self.channels, self.buffers
+        n = T * C * 2
         seg = _align16(n)            # every activation starts on a 16-byte boundary
 
         def at(buf, i):
-            return buf[i * seg:i * seg + n].view(torch.bfloat16).view(L.tokens, L.channels)
+            return buf[i * seg:i * seg + n].view(torch.bfloat16).view(T, C)
 
-        local = torch.zeros(L.buffers * seg, dtype=torch.uint8, device=self.device)
-        for b in range(L.buffers):
+        local = torch.zeros(B * seg, dtype=torch.uint8, device=self.device)
+        for b in range(B):
             at(local, b).copy_(xs[b])
-        every = torch.empty(self.world * L.buffers * seg, dtype=torch.uint8, device=self.device)
+        every = torch.empty(self.world * B * seg, dtype=torch.uint8, device=self.device)
         self._all_gather(every, local)
-        for b in range(L.buffers):
+        for b in range(B):
             self.codec.state_init(self.d, xs[b], self.recon_s[b], self.err[b])
             for p in self.peers:
-                self.codec.state_init(self.d, at(every, p * L.buffers + b), self.recon_r[p][b], None)
+                self.codec.state_init(self.d, at(every, p * B + b), self.recon_r[p][b], None)
                 if self.emit:
-                    self.out[p][b].copy_(at(every, p * L.buffers + b))
-
-    def _enc_sets(self, xs):
-        L = self.layout
-        return [(xs[b], self.recon_s[b], self.err[b], L.codes(self.send, b), L.scales(self.send, b))
-                for b in range(L.buffers)]
-
-    def prepare(self, xs) -> None:
-        """Optional: build the codec's per-call state (the device array of
-        buffer pointers) for these input tensors ahead of their step."""
-        self._check(xs)
-        if hasattr(self.codec, "prepare_encode"):
-            self.codec.prepare_encode(self.d, self._enc_sets(xs))
-
-    def step(self, xs, events=None) -> None:
-        """One compressed step: encode into the payload, all-gather, decode
-        every peer's payload into its receiver states.  `events`, four CUDA
-        events, are recorded on the current stream before the encode, after
-        it, after the all-gather and after the decode."""
-        self._check(xs)
-        mark = (lambda i: events[i].record()) if events is not None else (lambda i: None)
-        mark(0)
-        self.codec.encode_batched(self.d, self._enc_sets(xs))
-        mark(1)
-        self._all_gather(self.recv, self.send)
-        mark(2)
-        if self.emit:
-            self.codec.decode_emit_batched(self.d, self._dec_sets)
-        else:
-            self.codec.decode_batched(self.d, self._dec_sets)
-        mark(3)
+                    self.out[p][b].copy_(at(every, p * B + b))
 
     def state_dict(self) -> dict:
         """Everything a resumed exchange needs, as host copies, taken between
@@ -291,3 +315,107 @@ class ShardExchange:
     def payload_bytes_per_step(self) -> int:
         """Bytes this rank sends per compressed step."""
         return self.layout.bytes_per_rank
+
+
+class ShardExchange(_Exchange):
+    """The quantize mode.  tokens, channels: this rank's shard of one buffer
+    (every rank's shard has the same shape); bits: 1 or 2.  `loopback` also
+    keeps a receiver for the rank's own shard and decodes its own payload,
+    which on one GPU runs the whole path (its reconstruction must equal the
+    sender's mirror bit for bit).  recon_r[p][b] is the reconstruction of
+    peer p's buffer b (None for the rank's own shard unless `loopback`).
+    With `emit`, the decode also writes out[p][b], the bf16 rounding of
+    recon_r[p][b] that attention reads, in the same pass."""
+
+    def __init__(self, tokens: int, channels: int, bits: int, buffers: int, *, group=None,
+                 device=None, codec=None, loopback: bool = False, emit: bool = False):
+        if bits not in (1, 2):
+            raise ValueError(f"bits must be 1 or 2, got {bits}")
+        super().__init__(PayloadLayout(tokens, channels, bits, buffers), cf.desc(tokens, channels, bits),
+                         tokens, channels, buffers, group, device, codec, loopback)
+        self.emit = emit
+        self.out = [[torch.empty(tokens, channels, dtype=torch.bfloat16, device=self.device)
+                     for _ in range(buffers)] if emit and p in self.peers else None
+                    for p in range(self.world)]
+        L = self.layout
+        self._dec_sets = [(L.codes(self._payload(p), b), L.scales(self._payload(p), b), self.recon_r[p][b])
+                          + ((self.out[p][b],) if emit else ())
+                          for p in self.peers for b in range(buffers)]
+
+    def _enc_sets(self, xs):
+        L = self.layout
+        return [(xs[b], self.recon_s[b], self.err[b], L.codes(self.send, b), L.scales(self.send, b))
+                for b in range(L.buffers)]
+
+    def prepare(self, xs) -> None:
+        """Optional: build the codec's per-call state (the device array of
+        buffer pointers) for these input tensors ahead of their step."""
+        self._check(xs)
+        if hasattr(self.codec, "prepare_encode"):
+            self.codec.prepare_encode(self.d, self._enc_sets(xs))
+
+    def step(self, xs, events=None) -> None:
+        """One compressed step: encode into the payload, all-gather, decode
+        every peer's payload into its receiver states.  `events`, four CUDA
+        events, are recorded on the current stream before the encode, after
+        it, after the all-gather and after the decode."""
+        self._check(xs)
+        mark = (lambda i: events[i].record()) if events is not None else (lambda i: None)
+        mark(0)
+        self.codec.encode_batched(self.d, self._enc_sets(xs))
+        mark(1)
+        self._all_gather(self.recv, self.send)
+        mark(2)
+        if self.emit:
+            self.codec.decode_emit_batched(self.d, self._dec_sets)
+        else:
+            self.codec.decode_batched(self.d, self._dec_sets)
+        mark(3)
+
+
+class LowrankShardExchange(_Exchange):
+    """The low-rank mode: rank `rank` factors from `iters` subspace
+    iterations, INT4-quantised.  Each step's encode takes one fp32 [C, rank]
+    Gaussian start block per buffer (`omegas`), or None for the warm start
+    from the previous step's Q (every step after the first).  The encode
+    uses a device workspace of cf_lowrank_workspace_bytes per buffer;
+    status() reads the numeric status of every buffer.  Otherwise as
+    ShardExchange (no bf16 emission)."""
+
+    def __init__(self, tokens: int, channels: int, rank: int, iters: int, buffers: int, *,
+                 group=None, device=None, codec=None, loopback: bool = False):
+        if rank < 1 or iters < 1:
+            raise ValueError("rank and iters must be positive")
+        super().__init__(LowrankPayloadLayout(tokens, channels, rank, buffers),
+                         cf.desc(tokens, channels, 0, rank, iters),
+                         tokens, channels, buffers, group, device, codec, loopback)
+        self.ws_bytes = self.codec.lowrank_workspace_bytes(self.d)
+        self.workspace = torch.zeros(buffers * self.ws_bytes, dtype=torch.uint8, device=self.device)
+        L = self.layout
+        self._dec_sets = [L.parts(self._payload(p), b) + (self.recon_r[p][b],)
+                          for p in self.peers for b in range(buffers)]
+
+    def step(self, xs, omegas=None) -> None:
+        """One compressed step: encode into the payload, all-gather, decode
+        every peer's payload into its receiver states."""
+        self._check(xs)
+        if omegas is None:
+            omegas = [None] * self.buffers
+        if len(omegas) != self.buffers:
+            raise ValueError(f"expected {self.buffers} start blocks, got {len(omegas)}")
+        for om in omegas:
+            if om is not None and (om.dtype != torch.float32 or tuple(om.shape) != (self.channels, self.layout.rank)
+                                   or not om.is_contiguous()):
+                raise ValueError("each start block must be a contiguous fp32 [channels, rank] tensor")
+        L = self.layout
+        sets = [(xs[b], self.recon_s[b], self.err[b], omegas[b]) + L.parts(self.send, b)
+                for b in range(self.buffers)]
+        self.codec.lowrank_encode_batched(self.d, sets, self.workspace)
+        self._all_gather(self.recv, self.send)
+        self.codec.lowrank_decode_batched(self.d, self._dec_sets)
+
+    def status(self) -> list:
+        """Per-buffer numeric status of the last encodes (synchronises; the
+        codec reads and clears each buffer's status word)."""
+        return [self.codec.lowrank_status(self.workspace[b * self.ws_bytes:(b + 1) * self.ws_bytes])
+                for b in range(self.buffers)]

@@ -53,6 +53,59 @@ class OracleCodec:
             o.view(torch.int16).numpy().view(np.uint16)[...] = out
 
 
+class OracleLowrankCodec(OracleCodec):
+    """The low-rank codec methods on CPU tensors, computed by the numpy
+    oracle in place through numpy views (cold start only)."""
+
+    def __init__(self, rank, iters):
+        super().__init__(0)
+        self.rank, self.iters = rank, iters
+
+    def lowrank_workspace_bytes(self, d):
+        return 16
+
+    def lowrank_status(self, workspace_slice):
+        return 0
+
+    def lowrank_encode_batched(self, d, sets, workspace):
+        from oracle import lowrank as OL
+        from activation_residual_compression_cf_b200 import workloads as W
+        for x, rs, e, om, pc, ps, qc, qs in sets:
+            out = OL.lowrank_encode(W.bf16_bits(x), rs.numpy(), om.numpy().astype(np.float64), self.iters)
+            pc.numpy()[...] = out["p_codes"]
+            ps.numpy()[...] = out["p_scales"]
+            qc.numpy()[...] = out["q_codes"]
+            qs.numpy()[...] = out["q_scales"]
+            e.numpy()[...] = out["err"]
+
+    def lowrank_decode_batched(self, d, sets):
+        from oracle import lowrank as OL
+        for pc, ps, qc, qs, rr in sets:
+            OL.lowrank_decode(pc.numpy().copy(), ps.numpy().copy(), qc.numpy().copy(), qs.numpy().copy(),
+                              rr.numpy(), self.rank)
+
+
+@pytest.mark.parametrize("T,C,r,B", [(40, 72, 4, 2), (4096, 3072, 32, 114), (3, 5, 3, 1)])
+def test_lowrank_payload_layout_is_aligned_and_disjoint(T, C, r, B):
+    from activation_residual_compression_cf_b200.exchange import LowrankPayloadLayout
+    L = LowrankPayloadLayout(T, C, r, B)
+    nb = (r + 1) // 2
+    spans = []
+    p = torch.zeros(L.bytes_per_rank, dtype=torch.uint8)
+    base = p.data_ptr()
+    for b in range(B):
+        parts = L.parts(p, b)
+        assert [tuple(t.shape) for t in parts] == [(T, nb), (r,), (C, nb), (r,)]
+        for t in parts:
+            off = t.data_ptr() - base
+            assert off % 16 == 0
+            spans.append((off, off + t.numel() * t.element_size()))
+    spans.sort()
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:])) and spans[-1][1] <= L.bytes_per_rank
+    # the payload is the page's factor bytes plus at most 60 bytes of padding per buffer
+    assert L.stride - ((T + C) * nb + 8 * r) <= 60
+
+
 @pytest.mark.parametrize("T,C,bits,B", [(48, 200, 1, 3), (1024, 3072, 2, 114), (7, 8, 2, 2),
                                         (3, 33, 1, 5)])
 def test_payload_layout_is_aligned_and_disjoint(T, C, bits, B):
@@ -262,3 +315,62 @@ def test_exchange_resumes_bit_for_bit_from_a_state_dict_world2():
         p.join(timeout=60)
     for o in out:
         assert o[1] == "ok", o
+
+
+def _lowrank_worker(rank, world, port, q):
+    import datetime
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    try:
+        import torch.distributed as dist
+        from oracle import lowrank as OL
+        from activation_residual_compression_cf_b200 import workloads as W
+        from activation_residual_compression_cf_b200.exchange import LowrankShardExchange
+        from test_exchange import OracleLowrankCodec
+        dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                                world_size=world, timeout=datetime.timedelta(seconds=60))
+        T, C, r, iters, B, steps = 40, 72, 4, 2, 2, 3
+        wl = W.replace(W.WORKLOADS["lowrank"], tokens=world * T, channels=C, rank=r, iters=iters,
+                       buffers=B)
+        trajs = [W.trajectory(wl, b, steps=steps) for b in range(B)]
+        oms = {(b, t): W.omega(wl, b, t) for b in range(B) for t in range(1, steps)}
+
+        def shard(x, p):
+            return x[p * T:(p + 1) * T].clone()
+
+        ex = LowrankShardExchange(T, C, r, iters, B, device="cpu", codec=OracleLowrankCodec(r, iters))
+        ex.warmup([shard(trajs[b][0], rank) for b in range(B)])
+        for t in range(1, steps):
+            ex.step([shard(trajs[b][t], rank) for b in range(B)], [oms[(b, t)] for b in range(B)])
+        bad = []
+        for p in range(world):
+            for b in range(B):
+                rec = W.bf16_bits(shard(trajs[b][0], p)).astype(np.uint32) << 16
+                rec = rec.view(np.float32).copy()
+                for t in range(1, steps):
+                    OL.lowrank_encode(W.bf16_bits(shard(trajs[b][t], p)), rec,
+                                      oms[(b, t)].numpy().astype(np.float64), iters)
+                if p == rank and not np.array_equal(ex.recon_s[b].numpy(), rec):
+                    bad.append(("sender", p, b))
+                if p in ex.peers and not np.array_equal(ex.recon_r[p][b].numpy(), rec):
+                    bad.append(("receiver", p, b))
+        q.put((rank, "ok" if not bad else "bad", bad, ex.status()))
+        dist.destroy_process_group()
+    except Exception as e:
+        q.put((rank, "fail", repr(e), None))
+
+
+def test_lowrank_exchange_routes_every_peer_payload_world2():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_lowrank_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in ps:
+        p.start()
+    out = sorted([q.get(timeout=180) for _ in range(world)], key=lambda t: t[0])
+    for p in ps:
+        p.join(timeout=60)
+    for rank, status, info, st in out:
+        assert status == "ok", (rank, info)
+        assert st == [0, 0]

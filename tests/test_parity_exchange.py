@@ -16,7 +16,7 @@ import torch.distributed as dist
 import oracle
 from activation_residual_compression_cf_b200 import cf
 from activation_residual_compression_cf_b200 import workloads as W
-from activation_residual_compression_cf_b200.exchange import ShardExchange
+from activation_residual_compression_cf_b200.exchange import LowrankShardExchange, ShardExchange
 from _parity import compare_step, f32_of
 
 pytestmark = pytest.mark.gpu
@@ -101,3 +101,51 @@ def test_exchange_emits_the_bf16_reconstruction(nccl_group):
             assert torch.equal(ex.recon_r[0][b], ex.recon_s[b])
             ref = ex.recon_r[0][b].to(torch.bfloat16)
             assert torch.equal(ex.out[0][b].view(torch.int16), ref.view(torch.int16)), (t, b)
+
+
+def test_lowrank_exchange_loopback_matches_single_calls_and_oracle(nccl_group):
+    """The low-rank exchange in loopback: the payload equals single-buffer
+    cf_lowrank_encode calls on the same inputs bit for bit, the receivers
+    mirror the senders, buffer 0's error is within 1 % of the oracle's, and
+    a warm-started step (no start blocks) runs clean."""
+    from oracle import lowrank as OL
+    T, C, r, iters, B = 256, 192, 8, 2, 3
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r, iters=iters, buffers=B)
+    trajs = [W.trajectory(wl, b, steps=4, device="cuda") for b in range(B)]
+    ex = LowrankShardExchange(T, C, r, iters, B, loopback=True)
+    ex.warmup([trajs[b][0].clone() for b in range(B)])
+    d = cf.desc(T, C, 0, r, iters)
+    ws = torch.empty(cf.cf_lowrank_workspace_bytes(d), dtype=torch.uint8, device="cuda")
+    nb = (r + 1) // 2
+    ref = [dict(rs=ex.recon_s[b].clone(), err=torch.empty_like(ex.err[b]),
+                pc=torch.empty(T * nb, dtype=torch.uint8, device="cuda"), ps=torch.empty(r, device="cuda"),
+                qc=torch.empty(C * nb, dtype=torch.uint8, device="cuda"), qs=torch.empty(r, device="cuda"))
+           for b in range(B)]
+    for t in (1, 2):
+        xs = [trajs[b][t].clone() for b in range(B)]
+        oms = [W.omega(wl, b, t, device="cuda") for b in range(B)]
+        before0 = ex.recon_s[0].cpu().numpy()
+        ex.step(xs, oms)
+        for b in range(B):
+            g = ref[b]
+            cf.cf_lowrank_encode(d, xs[b], g["rs"], g["err"], oms[b], g["pc"], g["ps"], g["qc"], g["qs"], ws)
+        torch.cuda.synchronize()
+        assert ex.status() == [0] * B
+        for b in range(B):
+            pc, ps, qc, qs = ex.layout.parts(ex.recv, b)
+            g = ref[b]
+            assert torch.equal(pc.reshape(-1), g["pc"]) and torch.equal(qc.reshape(-1), g["qc"]), (t, b)
+            assert torch.equal(ps, g["ps"]) and torch.equal(qs, g["qs"]), (t, b)
+            assert torch.equal(ex.recon_s[b], g["rs"]) and torch.equal(ex.err[b], g["err"]), (t, b)
+            assert torch.equal(ex.recon_r[0][b], ex.recon_s[b]), (t, b)
+        out = OL.lowrank_encode(W.bf16_bits(xs[0]), before0.copy(), oms[0].cpu().numpy(), iters)
+        v = out["V"].astype(np.float64)
+        pc, ps, qc, qs = (a.cpu().numpy() for a in ex.layout.parts(ex.send, 0))
+        e_gpu = np.linalg.norm(v - OL.reconstruct(pc, ps, qc, qs, r)) / np.linalg.norm(v)
+        e_ora = np.linalg.norm(v - out["D"]) / np.linalg.norm(v)
+        assert abs(e_gpu - e_ora) <= 0.01 * e_ora, (t, e_gpu, e_ora)
+    ex.step([trajs[b][3].clone() for b in range(B)])      # warm start from the previous Q
+    torch.cuda.synchronize()
+    assert ex.status() == [0] * B
+    for b in range(B):
+        assert torch.equal(ex.recon_r[0][b], ex.recon_s[b])
