@@ -414,6 +414,19 @@ class LowrankShardExchange(_Exchange):
         self._all_gather(self.recv, self.send)
         self.codec.lowrank_decode_batched(self.d, self._dec_sets)
 
+    def state_dict(self) -> dict:
+        """As for the quantize mode, plus the encode workspace: it holds each
+        buffer's last Q, the warm start of the next step."""
+        sd = super().state_dict()
+        sd["workspace"] = self.workspace.detach().cpu().clone()
+        return sd
+
+    def load_state_dict(self, sd: dict) -> None:
+        if "workspace" not in sd or sd["workspace"].numel() != self.workspace.numel():
+            raise ValueError("state_dict was taken on a different exchange")
+        super().load_state_dict(sd)
+        self.workspace.copy_(sd["workspace"])
+
     def status(self) -> list:
         """Per-buffer numeric status of the last encodes (synchronises; the
         codec reads and clears each buffer's status word)."""

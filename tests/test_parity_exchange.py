@@ -144,8 +144,15 @@ def test_lowrank_exchange_loopback_matches_single_calls_and_oracle(nccl_group):
         e_gpu = np.linalg.norm(v - OL.reconstruct(pc, ps, qc, qs, r)) / np.linalg.norm(v)
         e_ora = np.linalg.norm(v - out["D"]) / np.linalg.norm(v)
         assert abs(e_gpu - e_ora) <= 0.01 * e_ora, (t, e_gpu, e_ora)
-    ex.step([trajs[b][3].clone() for b in range(B)])      # warm start from the previous Q
+    # a checkpoint taken here resumes the warm start bit for bit
+    resumed = LowrankShardExchange(T, C, r, iters, B, loopback=True)
+    resumed.load_state_dict(ex.state_dict())
+    x3 = [trajs[b][3].clone() for b in range(B)]
+    ex.step(x3)                                           # warm start from the previous Q
+    resumed.step(x3)
     torch.cuda.synchronize()
-    assert ex.status() == [0] * B
+    assert ex.status() == [0] * B and resumed.status() == [0] * B
     for b in range(B):
         assert torch.equal(ex.recon_r[0][b], ex.recon_s[b])
+        assert torch.equal(resumed.recon_s[b], ex.recon_s[b]) and torch.equal(resumed.err[b], ex.err[b])
+        assert torch.equal(resumed.recon_r[0][b], ex.recon_r[0][b])
