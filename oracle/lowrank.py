@@ -31,7 +31,9 @@ nibble, one row of ceil(r/2) bytes per factor row.
 
 Parity pins live in tests/test_oracle_lowrank.py (Eckart-Young optimum from
 LAPACK SVD, exact recovery at rank <= r, orthonormality, INT4 bounds, the
-compression-ratio closed form).
+compression-ratio closed form; reconstruct: hand-worked payloads in
+tests/golden/lowrank_reconstruct_cases.json and the elementwise INT4
+rounding bound on |D - P Q^T|).
 """
 from __future__ import annotations
 

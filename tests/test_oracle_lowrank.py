@@ -178,3 +178,87 @@ def test_iteration_count_barely_matters_on_drift_residuals():
     _, q_prev = L.subspace_iteration(v0, omega, iters=2)
     pw, qw = L.subspace_iteration(v1, q_prev, iters=1)
     assert e10 * (1 - 1e-9) <= rel(v1, pw, qw) <= e2 * 1.05
+
+
+# ---------------------------------------------------------------- reconstruct
+
+def test_reconstruct_hand_worked_cases():
+    """D from a hand-packed payload.  A reconstruct that dropped either
+    factor's scales, multiplied raw codes, swapped the nibbles or transposed
+    a factor gives a different D in these cases."""
+    g = json.load(open(os.path.join(GOLDEN, "lowrank_reconstruct_cases.json")))
+    for case in g["cases"]:
+        r = case["rank"]
+        pp = np.array(case["p_packed"], np.uint8)
+        qp = np.array(case["q_packed"], np.uint8)
+        assert np.array_equal(L.int4_pack(np.array(case["p_codes"], np.int8)), pp)
+        assert np.array_equal(L.int4_pack(np.array(case["q_codes"], np.int8)), qp)
+        d = L.reconstruct(pp, np.array(case["p_scales"], np.float32), qp,
+                          np.array(case["q_scales"], np.float32), r)
+        assert d.dtype == np.float32
+        assert np.array_equal(d, np.array(case["D"], np.float32)), (case, d)
+
+
+def _quantised(v, r, iters, seed):
+    omega = np.random.default_rng(seed).standard_normal((v.shape[1], r))
+    p, q = L.subspace_iteration(v, omega, iters)
+    pc, ps = L.int4_quantize_columns(p)
+    qc, qs = L.int4_quantize_columns(q)
+    d = L.reconstruct(L.int4_pack(pc), ps, L.int4_pack(qc), qs, r)
+    return p, q, pc, ps, qc, qs, d
+
+
+def _int4_bound(q, ph, ps, qs):
+    """Elementwise bound on |D - P Q^T| from the INT4 rounding alone: with
+    P^ = P + dP, |dP_ij| <= s_P_j / 2, and Q^ = Q + dQ, |dQ_kj| <= s_Q_j / 2,
+    D - P Q^T = dP Q^T + P^ dQ^T, so
+    |D - P Q^T|_ik <= sum_j (s_P_j / 2) |Q_kj| + |P^_ij| (s_Q_j / 2)."""
+    hp = 0.5 * ps.astype(np.float64)
+    hq = 0.5 * qs.astype(np.float64)
+    return (np.abs(q) * hp[None, :]).sum(axis=1)[None, :] + (np.abs(ph) * hq[None, :]).sum(axis=1)[:, None]
+
+
+def test_reconstruct_within_the_int4_rounding_bound():
+    """|D - P Q^T| <= sum_j (s_P_j/2 |Q_kj| + |P^_ij| s_Q_j/2) + fp32 rounding,
+    elementwise, on a drift-shaped residual and on a spectral matrix.  The
+    bound is tight enough that D built without a scale (or from raw codes)
+    violates it."""
+    rng = np.random.default_rng(3)
+    T, C, r = 96, 80, 8
+    u, w = rng.standard_normal((T, 4)), rng.standard_normal((C, 4)) * 0.05
+    for v in (u @ w.T + 0.01 * rng.standard_normal((T, C)),
+              _spectral(T, C, list(np.linspace(6.0, 0.1, 40)), seed=4)):
+        p, q, pc, ps, qc, qs, d = _quantised(v, r, 2, 6)
+        pq = p @ q.T
+        ph = pc.astype(np.float64) * ps.astype(np.float64)[None, :]
+        # plus one fp32 rounding of D (half an ulp of |D| <= |PQ^T| + bound)
+        b = _int4_bound(q, ph, ps, qs)
+        bound = b + (np.abs(pq) + b) * 2.0 ** -24 + 1e-30
+        gap = np.abs(d.astype(np.float64) - pq)
+        assert np.all(gap <= bound), float(np.max(gap / bound))
+        assert np.max(gap) > 0   # the INT4 step does change the product
+        # wrong reconstructions break the bound
+        qh = qc.astype(np.float64) * qs.astype(np.float64)[None, :]
+        for bad in (pc.astype(np.float64) @ qh.T,                     # P's scales dropped
+                    ph @ qc.astype(np.float64).T,                     # Q's scales dropped
+                    pc.astype(np.float64) @ qc.astype(np.float64).T):  # raw codes
+            assert np.any(np.abs(bad - pq) > bound)
+
+
+def test_reconstruct_error_close_to_unquantised_error():
+    """On the Eckart-Young matrices, ||V - D||_F differs from ||V - P Q^T||_F
+    by at most ||D - P Q^T||_F (triangle inequality), and that difference is
+    within the Frobenius norm of the elementwise INT4 bound."""
+    T, C, r = 48, 40, 4
+    v = _spectral(T, C, [10, 9, 8, 7] + list(np.linspace(1.0, 0.05, 36)))
+    p, q, pc, ps, qc, qs, d = _quantised(v, r, 50, 1)
+    ph = pc.astype(np.float64) * ps.astype(np.float64)[None, :]
+    bound = _int4_bound(q, ph, ps, qs)
+    bound = bound + (np.abs(p @ q.T) + bound) * 2.0 ** -24
+    e_q = np.linalg.norm(v - d.astype(np.float64))
+    e_f = np.linalg.norm(v - p @ q.T)
+    assert abs(e_q - e_f) <= np.linalg.norm(d.astype(np.float64) - p @ q.T) * (1 + 1e-9) + 1e-12
+    assert np.linalg.norm(d.astype(np.float64) - p @ q.T) <= np.linalg.norm(bound) * (1 + 1e-6)
+    # and INT4 costs accuracy against the SVD optimum, but not more than the bound
+    opt = np.sqrt(np.sum(np.linalg.svd(v, compute_uv=False)[r:] ** 2))
+    assert opt * (1 - 1e-12) <= e_q <= opt + np.linalg.norm(bound) * (1 + 1e-6)
