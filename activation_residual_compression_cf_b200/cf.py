@@ -14,7 +14,9 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libcf.so")
+# CF_LIBRARY=debug loads the bounds-checked debug build (libcf_debug.so)
+LIB_PATH = os.path.join(_PKG, "libcf_debug.so" if os.environ.get("CF_LIBRARY") == "debug"
+                        else "libcf.so")
 
 CF_OK = 0
 STATUS_NAMES = {0: "CF_OK", 1: "CF_ERR_INVALID_ARG", 2: "CF_ERR_ALIGNMENT",
@@ -26,11 +28,15 @@ EXPORTS = ("cf_status_string", "cf_abi_version", "cf_codes_words_per_row",
            "cf_payload_bytes", "cf_state_init", "cf_encode", "cf_decode",
            "cf_encode_batched", "cf_decode_batched", "cf_lowrank_workspace_bytes",
            "cf_lowrank_factor_bytes", "cf_lowrank_encode", "cf_lowrank_decode",
-           "cf_lowrank_status", "cf_set_lowrank_engine", "cf_set_quant_pipeline",
-           "cf_set_launch_override", "cf_lowrank_encode_noalloc", "cf_decode_emit",
-           "cf_decode_emit_batched", "cf_lowrank_encode_batched", "cf_lowrank_decode_batched",
-           "cf_lowrank_set_apply_events", "cf_encode_delta", "cf_encode_delta_batched",
-           "cf_diag_bounded_wait")
+           "cf_lowrank_status", "cf_lowrank_status_async", "cf_lowrank_encode_noalloc",
+           "cf_decode_emit", "cf_decode_emit_batched", "cf_lowrank_encode_batched",
+           "cf_lowrank_decode_batched", "cf_encode_delta", "cf_encode_delta_batched",
+           "cf_encode_publish_batched", "cf_decode_wait_batched")
+# Every symbol include/cf_diag.h declares: tuning knobs, measurement hooks
+# and the bounded-wait self-test (process-wide state, not product calls).
+DIAG_EXPORTS = ("cf_set_lowrank_engine", "cf_set_quant_pipeline", "cf_set_launch_override",
+                "cf_set_quant_unit", "cf_lowrank_set_apply_events", "cf_diag_bounded_wait",
+                "cf_debug_bounds_checked", "cf_debug_bounds_take", "cf_diag_bounds_selftest")
 
 
 class CFError(RuntimeError):
@@ -81,6 +87,20 @@ class cf_dec_emit_buffer(ctypes.Structure):
                 ("recon_r", ctypes.c_void_p), ("out", ctypes.c_void_p)]
 
 
+class cf_publish_dst(ctypes.Structure):
+    _fields_ = [("payload", ctypes.c_void_p), ("ready", ctypes.c_void_p), ("ack", ctypes.c_void_p)]
+
+
+class cf_enc_publish_buffer(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("recon_s", ctypes.c_void_p), ("err", ctypes.c_void_p),
+                ("codes_offset", ctypes.c_int64), ("scales_offset", ctypes.c_int64)]
+
+
+class cf_dec_wait_buffer(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("recon_r", ctypes.c_void_p), ("ready", ctypes.c_void_p)]
+
+
 _lib = None
 
 
@@ -113,6 +133,7 @@ def lib():
             "cf_lowrank_encode": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
             "cf_lowrank_decode": ([D, vp, vp, vp, vp, vp, vp], ctypes.c_int),
             "cf_lowrank_status": ([vp, vp], ctypes.c_int),
+            "cf_lowrank_status_async": ([vp, i64, i32, vp, vp], ctypes.c_int),
             "cf_lowrank_encode_batched": ([D, i32, vp, vp, sz, vp], ctypes.c_int),
             "cf_lowrank_decode_batched": ([D, i32, vp, vp, vp], ctypes.c_int),
             "cf_set_launch_override": ([i32, i32, i32, i32], ctypes.c_int),
@@ -120,6 +141,12 @@ def lib():
             "cf_lowrank_set_apply_events": ([vp, vp, vp, vp], ctypes.c_int),
             "cf_diag_bounded_wait": ([i32, vp, vp], ctypes.c_int),
             "cf_set_quant_pipeline": ([i32, i32, i32], ctypes.c_int),
+            "cf_set_quant_unit": ([i32, i32], ctypes.c_int),
+            "cf_debug_bounds_checked": ([], i32),
+            "cf_debug_bounds_take": ([], i32),
+            "cf_diag_bounds_selftest": ([vp, i32, vp], ctypes.c_int),
+            "cf_encode_publish_batched": ([D, i32, vp, i32, vp, ctypes.c_uint64, vp, vp], ctypes.c_int),
+            "cf_decode_wait_batched": ([D, i32, vp, ctypes.c_uint64, i32, vp, vp, vp], ctypes.c_int),
             "cf_lowrank_encode_noalloc": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
@@ -263,6 +290,57 @@ def cf_lowrank_status(workspace, stream=None) -> int:
     return lib().cf_lowrank_status(_p(workspace), _s(stream))
 
 
+def cf_lowrank_status_async(workspace, slice_bytes: int, n: int, host_status, stream=None):
+    """Enqueues the copy of n status words (slice b at workspace + b *
+    slice_bytes) into host_status (a pinned int32 tensor of >= n elements);
+    returns without waiting."""
+    if host_status.dtype != torch.int32 or host_status.device.type != "cpu" or host_status.numel() < n:
+        raise ValueError("host_status must be a host int32 tensor with at least n elements")
+    _chk(lib().cf_lowrank_status_async(_p(workspace), slice_bytes, n, _p(host_status), _s(stream)),
+         "cf_lowrank_status_async")
+
+
+def cf_encode_publish_batched(d, n, bufs_dev, ndst, dsts_dev, ack_target=0, status=None,
+                              stream=None):
+    _chk(lib().cf_encode_publish_batched(ctypes.byref(d), n, _p(bufs_dev), ndst, _p(dsts_dev),
+                                         int(ack_target), _p(status), _s(stream)),
+         "cf_encode_publish_batched")
+
+
+def cf_decode_wait_batched(d, n, bufs_dev, ready_target, nack=0, acks_dev=None, status=None,
+                           stream=None):
+    _chk(lib().cf_decode_wait_batched(ctypes.byref(d), n, _p(bufs_dev), int(ready_target), nack,
+                                      _p(acks_dev), _p(status), _s(stream)),
+         "cf_decode_wait_batched")
+
+
+def cf_debug_bounds_checked() -> bool:
+    return lib().cf_debug_bounds_checked() == 1
+
+
+def cf_debug_bounds_take() -> int:
+    """First failed index check of the debug build since the last call, as
+    (file tag << 16) | line, or 0; clears it (synchronises)."""
+    return lib().cf_debug_bounds_take()
+
+
+def cf_diag_bounds_selftest(out_dev, stream=None):
+    _chk(lib().cf_diag_bounds_selftest(_p(out_dev), out_dev.numel(), _s(stream)),
+         "cf_diag_bounds_selftest")
+
+
+def bounds_file_tag(name: str) -> int:
+    """The debug build's 15-bit tag of a source file's base name (FNV-1a)."""
+    h = 2166136261
+    for ch in os.path.basename(name).encode():
+        h = ((h ^ ch) * 16777619) & 0xFFFFFFFF
+    return (h ^ (h >> 15)) & 0x7FFF
+
+
+def cf_set_quant_unit(kernel: int, channels: int):
+    _chk(lib().cf_set_quant_unit(kernel, channels), "cf_set_quant_unit")
+
+
 def cf_set_lowrank_engine(engine: int):
     _chk(lib().cf_set_lowrank_engine(engine), "cf_set_lowrank_engine")
 
@@ -338,6 +416,36 @@ def lowrank_dec_buffer_array(sets, device) -> torch.Tensor:
     for i, t in enumerate(sets):
         arr[i] = cf_lowrank_dec_buffer(*[_p(v) for v in t])
     return torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
+
+
+def publish_dst_array(dsts, device) -> torch.Tensor:
+    """Device array of cf_publish_dst from [(payload, ready, ack or None), ...]."""
+    arr = (cf_publish_dst * len(dsts))()
+    for i, (pl, rd, ak) in enumerate(dsts):
+        arr[i] = cf_publish_dst(_p(pl), _p(rd), _p(ak))
+    return torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
+
+
+def enc_publish_buffer_array(sets, device) -> torch.Tensor:
+    """Device array of cf_enc_publish_buffer from
+    [(x, recon_s, err, codes_offset, scales_offset), ...]."""
+    arr = (cf_enc_publish_buffer * len(sets))()
+    for i, (x, r, e, co, so) in enumerate(sets):
+        arr[i] = cf_enc_publish_buffer(_p(x), _p(r), _p(e), int(co), int(so))
+    return torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
+
+
+def dec_wait_buffer_array(sets, device) -> torch.Tensor:
+    """Device array of cf_dec_wait_buffer from [(codes, scales, recon_r, ready), ...]."""
+    arr = (cf_dec_wait_buffer * len(sets))()
+    for i, t in enumerate(sets):
+        arr[i] = cf_dec_wait_buffer(*[_p(v) for v in t])
+    return torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
+
+
+def pointer_array(ptrs, device) -> torch.Tensor:
+    """Device array of raw pointers (uint64) from tensors or ints."""
+    return torch.tensor([_p(t) for t in ptrs], dtype=torch.int64).to(device)
 
 
 def dec_emit_buffer_array(sets, device) -> torch.Tensor:

@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "cf.h"
+#include "cf_diag.h"
 #include "cf_trace.h"
 #include "lowrank_api.cuh"
 #include "quant_kernels.cuh"
@@ -27,6 +28,7 @@ struct Override {
 Override g_override[2];
 int g_pipeline[2] = {1, 1};  // 0 = register-resident rows, 1 = TMA row staging (default)
 int g_stages[2] = {0, 0};    // TMA ring depth (0 = built-in choice)
+int g_unit[2] = {0, 0};      // TMA channels per thread unit, 4 or 8 (0 = built-in choice)
 std::mutex g_mu;
 
 int device_sm_count() {
@@ -77,7 +79,23 @@ struct Shape {
     int threads;
     int blocks_per_sm;
     int pipeline = 0;
+    int unit = 8;    // TMA pipeline: channels per thread unit (4 or 8)
 };
+
+// Channels per thread unit of the TMA kernels, measured on B200 in the
+// encode -> decode sequence (two alternating repeats of 300 steps each):
+// 4-channel units make every warp store 512 contiguous bytes and remove the
+// shared-memory bank conflicts of the recon reads, which helped the 2-bit
+// encode at C = 3072 (+3.5 %), but cost the 1-bit encode at C = 3072 4 %
+// and the 2-bit decode at C = 1920 4 %; elsewhere the two tie.
+int choose_unit(int kernel, int bits, int64_t C, bool delta) {
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (g_unit[kernel]) return g_unit[kernel];
+    }
+    if (kernel == 0 && !delta && bits == 2 && C >= 2048) return 4;
+    return 8;
+}
 
 // Launch shape per row: threads (a multiple of 32) x groups of 8 channels
 // per thread.  Chosen from sweeps on B200 timed in the encode -> decode
@@ -160,7 +178,7 @@ cf_status launch_decode_t(const Src &src, int64_t T, int64_t C, int64_t rows, in
 // code rows (W % 4 == 0); at most 480 consumer threads.
 constexpr int kDecodeConsumerWarpsPerSM = 12;
 
-template <bool ENC, int BITS, int GPT, class Src>
+template <bool ENC, int BITS, int GPT, int K, class Src>
 cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t *status,
                      const Shape &s, int stages_req, cudaStream_t st) {
     const int64_t W = (C * BITS + 31) / 32;
@@ -185,10 +203,11 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
     const size_t smem = (size_t)stages * slot + 16 * (size_t)stages;
     const int threads = 32 + s.threads;
     void (*k)(Src, int64_t, int64_t, int64_t, int32_t *, int);
+    // a thread's GPT groups of 8 channels as 8 / K * GPT units of K
     if constexpr (ENC)
-        k = cf::tma::encode_tma_kernel<BITS, GPT, Src>;
+        k = cf::tma::encode_tma_kernel<BITS, K, 8 / K * GPT, Src>;
     else
-        k = cf::tma::decode_tma_kernel<BITS, GPT, Src>;
+        k = cf::tma::decode_tma_kernel<BITS, K, 8 / K * GPT, Src>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return CF_ERR_CUDA;
     int occ = 0;
@@ -215,6 +234,7 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
 template <bool ENC, int BITS, int GPT, bool VEC, class Src>
 cf_status launch_one(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t *status,
                      const Shape &s, cudaStream_t st) {
+    constexpr bool kFused = Src::kPublish || Src::kWait;   // TMA pipeline only
     if constexpr (VEC) {
         if (s.pipeline == 1) {
             int stages;
@@ -222,13 +242,17 @@ cf_status launch_one(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
                 std::lock_guard<std::mutex> lk(g_mu);
                 stages = g_stages[ENC ? 0 : 1];
             }
-            return launch_tma<ENC, BITS, GPT>(src, T, C, rows, status, s, stages, st);
+            if (s.unit == 4) return launch_tma<ENC, BITS, GPT, 4>(src, T, C, rows, status, s, stages, st);
+            return launch_tma<ENC, BITS, GPT, 8>(src, T, C, rows, status, s, stages, st);
         }
     }
-    if constexpr (ENC)
+    if constexpr (kFused) {
+        return CF_ERR_UNSUPPORTED;
+    } else if constexpr (ENC) {
         return launch_encode_t<BITS, GPT, VEC>(src, T, C, rows, status, s, st);
-    else
+    } else {
         return launch_decode_t<BITS, GPT, VEC>(src, T, C, rows, status, s, st);
+    }
 }
 
 // Runtime (bits, gpt, vec) -> template instance.
@@ -250,10 +274,14 @@ cf_status dispatch(const Src &src, int bits, int64_t T, int64_t C, int64_t rows,
     }
     bool delta = false;
     if constexpr (ENC) delta = Src::kDelta;
+    constexpr bool kFused = Src::kPublish || Src::kWait;
+    if (kFused) pipe = 1;     // the publishing and waiting kernels are TMA-staged
     if (pipe == 1 && !tma_applies(ENC, bits, C, delta)) pipe = 0;
     Shape s = choose_shape(ENC ? 0 : 1, C, pipe, bits, delta);
     if (pipe == 1 && s.threads > 480) s = choose_shape(ENC ? 0 : 1, C, pipe = 0, bits, delta);
+    if (kFused && pipe != 1) return CF_ERR_UNSUPPORTED;
     s.pipeline = pipe;
+    s.unit = choose_unit(ENC ? 0 : 1, bits, C, delta);
     const bool vec = (C % 8) == 0;
 #define CF_CASE(B, G, V)                                     \
     if (bits == B && s.gpt == G && vec == V)                 \
@@ -269,6 +297,26 @@ cf_status dispatch(const Src &src, int bits, int64_t T, int64_t C, int64_t rows,
 }
 
 }  // namespace
+
+// Bounds-checked debug build: this translation unit's first failed index
+// check, read and cleared (synchronises the device).
+#ifdef CF_DEBUG_BOUNDS
+int32_t cf_bounds_take_api() {
+    int32_t v = 0;
+    const int32_t z = 0;
+    if (cudaMemcpyFromSymbol(&v, cf::g_bounds_hit, sizeof v) != cudaSuccess ||
+        cudaMemcpyToSymbol(cf::g_bounds_hit, &z, sizeof z) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return -1;
+    }
+    return v;
+}
+#endif
+
+#ifdef CF_DEBUG_BOUNDS
+int32_t cf_bounds_take_lowrank();
+int32_t cf_bounds_take_diag();
+#endif
 
 // ------------------------------------------------------------------ C ABI
 
@@ -433,6 +481,66 @@ cf_status cf_decode_batched(const cf_desc *d, int32_t n, const cf_dec_buffer *bu
     cf::DecArray src{bufs_dev};
     return dispatch<false>(src, d->bits, d->tokens, d->channels, d->tokens * (int64_t)n,
                            status_dev, (cudaStream_t)stream);
+}
+
+cf_status cf_encode_publish_batched(const cf_desc *d, int32_t n, const cf_enc_publish_buffer *bufs_dev,
+                                    int32_t ndst, const cf_publish_dst *dsts_dev, uint64_t ack_target,
+                                    int32_t *status_dev, void *stream) {
+    cf::TraceRange trace_("cf_encode_publish_batched");
+    CF_TRY(check_quant_desc(d));
+    if (n < 0 || ndst < 1 || ndst > 8) return CF_ERR_INVALID_ARG;
+    if (n == 0 || d->tokens == 0) return CF_OK;
+    if (!tma_applies(true, d->bits, d->channels)) return CF_ERR_UNSUPPORTED;
+    CF_TRY(check_dev_ptr(bufs_dev));
+    CF_TRY(check_dev_ptr(dsts_dev));
+    if (status_dev) CF_TRY(check_dev_ptr(status_dev, 4));
+    cf::EncPublishArray src{bufs_dev, dsts_dev, ndst, ack_target};
+    return dispatch<true>(src, d->bits, d->tokens, d->channels, d->tokens * (int64_t)n,
+                          status_dev, (cudaStream_t)stream);
+}
+
+cf_status cf_decode_wait_batched(const cf_desc *d, int32_t n, const cf_dec_wait_buffer *bufs_dev,
+                                 uint64_t ready_target, int32_t nack, uint64_t *const *acks_dev,
+                                 int32_t *status_dev, void *stream) {
+    cf::TraceRange trace_("cf_decode_wait_batched");
+    CF_TRY(check_quant_desc(d));
+    if (n < 0 || nack < 0 || nack > 64) return CF_ERR_INVALID_ARG;
+    if (nack > 0) CF_TRY(check_dev_ptr(acks_dev, 8));
+    if (status_dev) CF_TRY(check_dev_ptr(status_dev, 4));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (n > 0 && d->tokens > 0) {
+        if (!tma_applies(false, d->bits, d->channels)) return CF_ERR_UNSUPPORTED;
+        CF_TRY(check_dev_ptr(bufs_dev));
+        cf::DecWaitArray src{bufs_dev, ready_target};
+        CF_TRY(dispatch<false>(src, d->bits, d->tokens, d->channels, d->tokens * (int64_t)n,
+                               status_dev, st));
+    }
+    if (nack > 0) {
+        cf::tma::exchange_ack_kernel<<<1, 64, 0, st>>>(acks_dev, nack);
+        return launch_result();
+    }
+    return CF_OK;
+}
+
+int32_t cf_debug_bounds_checked(void) { return cf::kBoundsChecked ? 1 : 0; }
+
+int32_t cf_debug_bounds_take(void) {
+#ifdef CF_DEBUG_BOUNDS
+    int32_t first = 0;
+    for (int32_t v : {cf_bounds_take_api(), cf_bounds_take_lowrank(), cf_bounds_take_diag()})
+        if (first == 0 && v != 0) first = v;
+    return first;
+#else
+    return 0;
+#endif
+}
+
+cf_status cf_set_quant_unit(int32_t kernel, int32_t channels) {
+    if (kernel < 0 || kernel > 1) return CF_ERR_INVALID_ARG;
+    if (channels != 0 && channels != 4 && channels != 8) return CF_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_unit[kernel] = channels;
+    return CF_OK;
 }
 
 cf_status cf_set_quant_pipeline(int32_t kernel, int32_t pipeline, int32_t stages) {

@@ -7,7 +7,9 @@
 // unsignalled wait gives up after `polls` polls.
 #include <cuda_runtime.h>
 
+#include "bounds.cuh"
 #include "cf.h"
+#include "cf_diag.h"
 #include "cf_trace.h"
 #include "mbar.cuh"
 
@@ -32,6 +34,37 @@ __global__ void diag_wait_kernel(uint32_t polls, int32_t *out) {
 }
 
 }  // namespace
+
+// Positive control of the debug build's index checks: writes out[i] = i for
+// every i < n, each write guarded by a check that declares an extent of n / 2.
+// Every write the check lets through stays inside out[0, n).
+__global__ void diag_bounds_kernel(int32_t *out, int n) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+        if (CF_IN(i < n / 2)) out[i] = i;
+}
+
+// Bounds-checked debug build: this translation unit's first failed index
+// check, read and cleared (synchronises the device).
+#ifdef CF_DEBUG_BOUNDS
+int32_t cf_bounds_take_diag() {
+    int32_t v = 0;
+    const int32_t z = 0;
+    if (cudaMemcpyFromSymbol(&v, cf::g_bounds_hit, sizeof v) != cudaSuccess ||
+        cudaMemcpyToSymbol(cf::g_bounds_hit, &z, sizeof z) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return -1;
+    }
+    return v;
+}
+#endif
+
+extern "C" cf_status cf_diag_bounds_selftest(int32_t *out_dev, int32_t n, void *stream) {
+    if (!cf::kBoundsChecked) return CF_ERR_UNSUPPORTED;
+    if (!out_dev || n < 2 || n > (1 << 20)) return CF_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(out_dev) & 3u) != 0) return CF_ERR_ALIGNMENT;
+    diag_bounds_kernel<<<1, 256, 0, (cudaStream_t)stream>>>(out_dev, n);
+    return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
+}
 
 extern "C" cf_status cf_diag_bounded_wait(int32_t polls, int32_t *out_dev, void *stream) {
     cf::TraceRange trace_("cf_diag_bounded_wait");

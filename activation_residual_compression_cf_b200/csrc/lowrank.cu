@@ -30,6 +30,7 @@
 #include <atomic>
 
 #include "cf.h"
+#include "cf_diag.h"
 #include "cf_trace.h"
 #include "cf_common.cuh"
 #include "lowrank_api.cuh"
@@ -396,6 +397,21 @@ cf_status encode_impl(const cf_desc *d, const Layout &L, int n, const LrBatch &B
 
 }  // namespace
 
+// Bounds-checked debug build: this translation unit's first failed index
+// check, read and cleared (synchronises the device).
+#ifdef CF_DEBUG_BOUNDS
+int32_t cf_bounds_take_lowrank() {
+    int32_t v = 0;
+    const int32_t z = 0;
+    if (cudaMemcpyFromSymbol(&v, cf::g_bounds_hit, sizeof v) != cudaSuccess ||
+        cudaMemcpyToSymbol(cf::g_bounds_hit, &z, sizeof z) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return -1;
+    }
+    return v;
+}
+#endif
+
 extern "C" {
 
 int64_t cf_lowrank_workspace_bytes(const cf_desc *d) {
@@ -527,6 +543,31 @@ cf_status cf_lowrank_status(void *workspace, void *stream) {
         return CF_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return CF_ERR_CUDA;
     return (cf_status)h;
+}
+
+cf_status cf_lowrank_status_async(const void *workspace, int64_t slice_bytes, int32_t n,
+                                  int32_t *host_status, void *stream) {
+    if (n < 0) return CF_ERR_INVALID_ARG;
+    if (n == 0) return CF_OK;
+    if (!workspace || !host_status || slice_bytes <= 0) return CF_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || slice_bytes % 256 != 0 ||
+        (reinterpret_cast<uintptr_t>(host_status) & 3u) != 0)
+        return CF_ERR_ALIGNMENT;
+    LR_TRY(check_ptr(workspace, 256));
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, host_status) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return CF_ERR_INVALID_ARG;
+    }
+    if (a.type != cudaMemoryTypeHost) return CF_ERR_INVALID_ARG;   // pageable or device memory
+    // one strided copy: row b is the first int32 of slice b
+    if (cudaMemcpy2DAsync(host_status, sizeof(int32_t), workspace, (size_t)slice_bytes,
+                          sizeof(int32_t), (size_t)n, cudaMemcpyDeviceToHost,
+                          (cudaStream_t)stream) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return CF_ERR_CUDA;
+    }
+    return CF_OK;
 }
 
 }  // extern "C"

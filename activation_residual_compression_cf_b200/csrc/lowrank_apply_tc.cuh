@@ -20,6 +20,7 @@
 
 #include <cuda_bf16.h>
 
+#include "bounds.cuh"
 #include "cf.h"
 #include "cf_common.cuh"
 #include "lowrank_kernels.cuh"
@@ -322,7 +323,7 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
                 for (int id = lane; id < TPW * 8; id += 32) {
                     const int row = id >> 3, ch = 32 * q + 4 * (id & 7);
                     const int64_t t = tb + row;
-                    const bool ok = t < tend && ch < cw;
+                    const bool ok = t < tend && ch < cw && CF_IN(t < T && c0 + ch + 4 <= C);
                     apply_cp16(sr0 + (uint32_t)((TPW * half + row) * (kApplyTile * 4) + ch * 4),
                                ok ? (const void *)(recon + t * C + c0 + ch) : (const void *)recon, ok);
                 }
@@ -331,7 +332,7 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
                     for (int id = lane; id < TPW * 4; id += 32) {
                         const int row = id >> 2, ch = 32 * q + 8 * (id & 3);
                         const int64_t t = tb + row;
-                        const bool ok = t < tend && ch < cw;
+                        const bool ok = t < tend && ch < cw && CF_IN(t < T && c0 + ch + 8 <= C);
                         apply_cp16(sr0 + (uint32_t)(RB + (TPW * half + row) * (kApplyTile * 2) + ch * 2),
                                    ok ? (const void *)(x + t * C + c0 + ch) : (const void *)x, ok);
                     }
@@ -433,6 +434,7 @@ lr_apply_tc_kernel(const cf_lowrank::LrBatch B, const cf_lowrank::Layout L, int 
 #pragma unroll
                         for (int j = 0; j < TPW; ++j) {
                             if (tl + j >= tw) break;
+                            if (!CF_IN(t0 + tl + j < T && c < C)) break;
                             const float rv = sr[j * kApplyTile + cl];
                             const int64_t o = (t0 + tl + j) * C + c;
                             if (SENDER) {

@@ -9,6 +9,7 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include "bounds.cuh"
 #include "cf.h"
 #include "cf_common.cuh"
 #include "lowrank_api.cuh"
@@ -72,6 +73,7 @@ __global__ void lr_residual_kernel(const LrBatch B, const Layout L) {
     const int64_t groups = n >> 3;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += stride) {
+        if (!CF_IN(8 * g + 8 <= n)) continue;
         const uint4 xv = ld_ro_v4(x + 8 * g);
         const float4 a = ld_state_v4(recon + 8 * g);
         const float4 b = ld_state_v4(recon + 8 * g + 4);
@@ -108,13 +110,14 @@ __global__ void lr_omega_kernel(const LrBatch B, const Layout L) {
     for (int j = ty; j < 32; j += 8) {
         const int64_t c = c0 + j;
         const int k = k0 + tx;
-        tile[j][tx] = (c < C && k < r) ? omega[c * r + k] : 0.0f;
+        tile[j][tx] = (c < C && k < r && CF_IN(c * r + k < C * r)) ? omega[c * r + k] : 0.0f;
     }
     __syncthreads();
     for (int j = ty; j < 32; j += 8) {
         const int k = k0 + j;
         const int64_t c = c0 + tx;
-        if (k < L.rp && c < C) qt[(int64_t)k * C + c] = __float2bfloat16_rn(tile[tx][j]);
+        if (k < L.rp && c < C && CF_IN((int64_t)k * C + c < (int64_t)L.rp * C))
+            qt[(int64_t)k * C + c] = __float2bfloat16_rn(tile[tx][j]);
     }
 }
 
@@ -639,6 +642,7 @@ __global__ void lr_int4_pack_kernel(const LrBatch B, const Layout L, int which) 
     }
     if (i >= rows * nb) return;
     const int64_t row = i / nb;
+    if (!CF_IN(row < rows && 2 * (i - row * nb) < rp)) return;
     const int b = (int)(i - row * nb);
     const int k0 = 2 * b, k1 = 2 * b + 1;
     const int q0 = int4_code(f[row * rp + k0], sc[k0]);

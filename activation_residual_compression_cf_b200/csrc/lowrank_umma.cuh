@@ -31,6 +31,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "bounds.cuh"
 #include "cf.h"
 #include "lowrank_api.cuh"
 #include "lowrank_kernels.cuh"
@@ -251,7 +252,7 @@ __device__ __forceinline__ void gemm_tile(const CUtensorMap *mapA, const CUtenso
         for (int c = 0; c < BN; c += 16) {
             float v[16];
             tmem_ld16(taddr + c, v);
-            if (row < out_rows) {
+            if (row < out_rows && CF_IN(row >= 0 && c + 16 <= BN)) {
                 float4 *dst = reinterpret_cast<float4 *>(out + row * BN + c);
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -449,7 +450,8 @@ __device__ __forceinline__ void backproject_tail(const cf_lowrank::LrBatch &B, c
         }
         bf16 *qt = B.at<bf16>(bz, L.off_qt);
 #pragma unroll
-        for (int k = 0; k < BN; ++k) qt[(int64_t)k * C + c] = __float2bfloat16_rn(v[k]);
+        for (int k = 0; k < BN; ++k)
+            if (CF_IN((int64_t)k * C + c < (int64_t)L.rp * C)) qt[(int64_t)k * C + c] = __float2bfloat16_rn(v[k]);
     } else {
 #pragma unroll
         for (int k = 0; k < BN; ++k) v[k] = 0.0f;
@@ -737,7 +739,7 @@ project_residual_kernel(const __grid_constant__ CUtensorMap mapQt, const cf_lowr
             for (int cc = 0; cc < BN; cc += 16) {
                 float v[16];
                 tmem_ld16(taddr + cc, v);
-                if (row < T) {
+                if (row < T && CF_IN(row >= 0 && cc + 16 <= BN)) {
                     float4 *dst = reinterpret_cast<float4 *>(y + row * BN + cc);
 #pragma unroll
                     for (int u = 0; u < 4; ++u)

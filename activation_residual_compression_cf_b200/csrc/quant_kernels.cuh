@@ -31,6 +31,7 @@
 
 #include <cuda_bf16.h>
 
+#include "bounds.cuh"
 #include "cf.h"
 #include "cf_common.cuh"
 
@@ -43,6 +44,8 @@ struct EncPtrs {
     uint32_t *codes;
     float *scales;
     const uint16_t *xprev;    // delta-state sender: the previous activation
+    int64_t codes_off = 0;    // publishing sender: byte offsets in a payload slot
+    int64_t scales_off = 0;
 };
 
 struct DecPtrs {
@@ -50,6 +53,7 @@ struct DecPtrs {
     const float *scales;
     float *recon;
     uint16_t *out;  // bf16 copy of the new reconstruction (emitting decode only)
+    const uint64_t *ready = nullptr;  // waiting decode: the sender's ready counter
 };
 
 template <class P>
@@ -64,18 +68,21 @@ struct EncSingle {
     EncPtrs p;
     static constexpr bool kChecked = false;
     static constexpr bool kDelta = false;
+    static constexpr bool kPublish = false, kWait = false;
     __device__ __forceinline__ EncPtrs get(int64_t) const { return p; }
 };
 struct EncDeltaSingle {
     EncPtrs p;
     static constexpr bool kChecked = false;
     static constexpr bool kDelta = true;
+    static constexpr bool kPublish = false, kWait = false;
     __device__ __forceinline__ EncPtrs get(int64_t) const { return p; }
 };
 struct EncDeltaArray {
     const cf_enc_delta_buffer *a;
     static constexpr bool kChecked = true;
     static constexpr bool kDelta = true;
+    static constexpr bool kPublish = false, kWait = false;
     __device__ __forceinline__ EncPtrs get(int64_t i) const {
         const cf_enc_delta_buffer *e = a + i;
         EncPtrs p;
@@ -92,6 +99,7 @@ struct EncArray {
     const cf_enc_buffer *a;
     static constexpr bool kChecked = true;
     static constexpr bool kDelta = false;
+    static constexpr bool kPublish = false, kWait = false;
     __device__ __forceinline__ EncPtrs get(int64_t i) const {
         const cf_enc_buffer *e = a + i;
         EncPtrs p;
@@ -109,6 +117,7 @@ struct DecSingleT {
     DecPtrs p;
     static constexpr bool kChecked = false;
     static constexpr bool kEmit = EMIT;
+    static constexpr bool kPublish = false, kWait = false;
     __device__ __forceinline__ DecPtrs get(int64_t) const { return p; }
 };
 using DecSingle = DecSingleT<false>;
@@ -117,6 +126,7 @@ struct DecArray {
     const cf_dec_buffer *a;
     static constexpr bool kChecked = true;
     static constexpr bool kEmit = false;
+    static constexpr bool kPublish = false, kWait = false;
     __device__ __forceinline__ DecPtrs get(int64_t i) const {
         const cf_dec_buffer *e = a + i;
         DecPtrs p;
@@ -131,6 +141,7 @@ struct DecEmitArray {
     const cf_dec_emit_buffer *a;
     static constexpr bool kChecked = true;
     static constexpr bool kEmit = true;
+    static constexpr bool kPublish = false, kWait = false;
     __device__ __forceinline__ DecPtrs get(int64_t i) const {
         const cf_dec_emit_buffer *e = a + i;
         DecPtrs p;
@@ -157,20 +168,28 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float *v) {
 __device__ __forceinline__ bool misaligned4(const void *p) {
     return (reinterpret_cast<uintptr_t>(p) & 3u) != 0;
 }
-template <bool DELTA>
+template <bool DELTA, bool PUBLISH = false>
 __device__ __forceinline__ int enc_ptr_status(const EncPtrs &p) {
     const void *state = DELTA ? static_cast<const void *>(p.xprev) : static_cast<const void *>(p.recon);
+    if (PUBLISH) {  // codes and scales go to the destinations, at these offsets
+        if (!p.x || !state || !p.err || p.codes_off < 0 || p.scales_off < 0) return CF_ERR_INVALID_ARG;
+        if (misaligned16(p.x) || misaligned16(state) || misaligned16(p.err) || (p.codes_off & 15) ||
+            (p.scales_off & 3))
+            return CF_ERR_ALIGNMENT;
+        return CF_OK;
+    }
     if (!p.x || !state || !p.err || !p.codes || !p.scales) return CF_ERR_INVALID_ARG;
     if (misaligned16(p.x) || misaligned16(state) || misaligned16(p.err) ||
         misaligned16(p.codes) || misaligned4(p.scales))
         return CF_ERR_ALIGNMENT;
     return CF_OK;
 }
-template <bool EMIT>
+template <bool EMIT, bool WAIT = false>
 __device__ __forceinline__ int dec_ptr_status(const DecPtrs &p) {
-    if (!p.codes || !p.scales || !p.recon || (EMIT && !p.out)) return CF_ERR_INVALID_ARG;
+    if (!p.codes || !p.scales || !p.recon || (EMIT && !p.out) || (WAIT && !p.ready))
+        return CF_ERR_INVALID_ARG;
     if (misaligned16(p.codes) || misaligned4(p.scales) || misaligned16(p.recon) ||
-        (EMIT && misaligned16(p.out)))
+        (EMIT && misaligned16(p.out)) || (WAIT && (reinterpret_cast<uintptr_t>(p.ready) & 7u)))
         return CF_ERR_ALIGNMENT;
     return CF_OK;
 }
@@ -178,6 +197,131 @@ __device__ __forceinline__ int dec_ptr_status(const DecPtrs &p) {
 __device__ __forceinline__ void report(int32_t *status, int code) {
     if (status) atomicCAS(status, (int32_t)CF_OK, (int32_t)code);
 }
+
+// ---- exchange counters (publishing encode / waiting decode)
+
+__device__ __forceinline__ uint64_t ld_acquire_sys(const uint64_t *p) {
+    uint64_t v;
+    asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Polls of a counter before a wait gives up; with the backoff below (up to
+// about a microsecond between polls) that is on the order of a second.
+constexpr uint32_t kCounterPolls = 1u << 20;
+
+// Bounded wait until *p >= target (system-scope acquire); false on expiry.
+__device__ __forceinline__ bool wait_counter(const uint64_t *p, uint64_t target,
+                                             uint32_t polls = kCounterPolls) {
+    uint32_t ns = 32;
+    for (uint32_t i = 0; i < polls; ++i) {
+        if (ld_acquire_sys(p) >= target) return true;
+        __nanosleep(ns);
+        if (ns < 1024) ns <<= 1;
+    }
+    return false;
+}
+
+// Publishing encode: buffers of cf_enc_publish_buffer, destinations of
+// cf_publish_dst (the library's host code caps ndst at 8).
+struct EncPublishArray {
+    const cf_enc_publish_buffer *a;
+    const cf_publish_dst *dst;
+    int ndst;
+    uint64_t ack_target;
+    static constexpr bool kChecked = true;
+    static constexpr bool kDelta = false;
+    static constexpr bool kPublish = true, kWait = false;
+    __device__ __forceinline__ EncPtrs get(int64_t i) const {
+        const cf_enc_publish_buffer *e = a + i;
+        EncPtrs p;
+        p.x = ldg_ptr(&e->x);
+        p.recon = ldg_ptr(&e->recon_s);
+        p.err = ldg_ptr(&e->err);
+        p.codes = nullptr;
+        p.scales = nullptr;
+        p.xprev = nullptr;
+        p.codes_off = __ldg(reinterpret_cast<const long long *>(&e->codes_offset));
+        p.scales_off = __ldg(reinterpret_cast<const long long *>(&e->scales_offset));
+        return p;
+    }
+    // Destination pointers valid and aligned, then every ack counter at the
+    // target (bounded).  On failure records the status and returns false.
+    __device__ bool check_and_wait(int32_t *status) const {
+        for (int d = 0; d < ndst; ++d) {
+            const uint8_t *pl = ldg_ptr(&dst[d].payload);
+            const uint64_t *rd = ldg_ptr(&dst[d].ready);
+            const uint64_t *ak = ldg_ptr(&dst[d].ack);
+            if (!pl || !rd) {
+                report(status, CF_ERR_INVALID_ARG);
+                return false;
+            }
+            if (misaligned16(pl) || (reinterpret_cast<uintptr_t>(rd) & 7u) ||
+                (reinterpret_cast<uintptr_t>(ak) & 7u)) {
+                report(status, CF_ERR_ALIGNMENT);
+                return false;
+            }
+        }
+        if (ack_target == 0) return true;
+        for (int d = 0; d < ndst; ++d) {
+            const uint64_t *ak = ldg_ptr(&dst[d].ack);
+            if (ak && !wait_counter(ak, ack_target)) {
+                report(status, CF_ERR_TIMEOUT);
+                return false;
+            }
+        }
+        return true;
+    }
+    // One row's code words (staged in shared memory) and scale into every
+    // destination; 16-byte stores when the code rows are 16-byte multiples.
+    __device__ __forceinline__ void store_row(const EncPtrs &p, const uint32_t *srow, int64_t W,
+                                              int64_t t, float scale, int ct, int nc) const {
+        for (int d = 0; d < ndst; ++d) {
+            uint8_t *pl = ldg_ptr(&dst[d].payload);
+            uint32_t *crow = reinterpret_cast<uint32_t *>(pl + p.codes_off) + t * W;
+            if ((W & 3) == 0) {
+                const int nv = (int)(W >> 2);
+                for (int k = ct; k < nv; k += nc)
+                    if (CF_IN(4 * k + 4 <= W)) reinterpret_cast<uint4 *>(crow)[k] = reinterpret_cast<const uint4 *>(srow)[k];
+            } else {
+                for (int k = ct; k < (int)W; k += nc) crow[k] = srow[k];
+            }
+            if (ct == 0) reinterpret_cast<float *>(pl + p.scales_off)[t] = scale;
+        }
+    }
+    // Release of this CTA's rows: the fence orders every store the CTA made
+    // (observed through the barrier before this call) before the adds.
+    __device__ __forceinline__ void publish(uint64_t rows) const {
+        __threadfence_system();
+        for (int d = 0; d < ndst; ++d)
+            atomicAdd_system(reinterpret_cast<unsigned long long *>(ldg_ptr(&dst[d].ready)),
+                             (unsigned long long)rows);
+    }
+};
+
+// Waiting decode: buffers of cf_dec_wait_buffer, all waited for up to the
+// same ready target.
+struct DecWaitArray {
+    const cf_dec_wait_buffer *a;
+    uint64_t target;
+    static constexpr bool kChecked = true;
+    static constexpr bool kEmit = false;
+    static constexpr bool kPublish = false, kWait = true;
+    __device__ __forceinline__ DecPtrs get(int64_t i) const {
+        const cf_dec_wait_buffer *e = a + i;
+        DecPtrs p;
+        p.codes = ldg_ptr(&e->codes);
+        p.scales = ldg_ptr(&e->scales);
+        p.recon = ldg_ptr(&e->recon_r);
+        p.out = nullptr;
+        p.ready = ldg_ptr(&e->ready);
+        return p;
+    }
+    __device__ __forceinline__ bool wait_ready(int64_t i) const {
+        return wait_counter(ldg_ptr(&a[i].ready), target);
+    }
+};
+
 
 // Code of one residual value.  1 bit: [v >= 0].  2 bits: number of the
 // thresholds -A/2, 0, A/2 that v reaches (ties go to the upper bin).
@@ -215,6 +359,30 @@ __device__ __forceinline__ void residual8(const uint4 &xw, const uint4 &pw, cons
     }
 }
 
+// The same for 4 channels (two bf16 words), used by the TMA pipeline.
+template <bool DELTA>
+__device__ __forceinline__ void residual4(const uint2 &xw, const uint2 &pw, const float *r, float *v) {
+    const uint32_t w2[2] = {xw.x, xw.y};
+    const uint32_t p2[2] = {pw.x, pw.y};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float xf = bf16_bits_to_f32((w2[e >> 1] >> ((e & 1) * 16)) & 0xffffu);
+        if (DELTA) {
+            const float pf = bf16_bits_to_f32((p2[e >> 1] >> ((e & 1) * 16)) & 0xffffu);
+            v[e] = __fadd_rn(__fsub_rn(xf, pf), r[e]);
+        } else {
+            v[e] = __fsub_rn(xf, r[e]);
+        }
+    }
+}
+
+// 4 fp32 values -> 4 bf16 (round to nearest even) packed in 8 bytes.
+__device__ __forceinline__ uint2 pack_bf16x4(const float *v) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+    return make_uint2(*reinterpret_cast<const uint32_t *>(&a), *reinterpret_cast<const uint32_t *>(&b));
+}
+
 template <int BITS, int GPT, bool VEC, class Src>
 __global__ void __launch_bounds__(512)
 encode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status) {
@@ -230,8 +398,12 @@ encode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
     __shared__ double sh_sum[2][32];
     __shared__ float sh_max[2][32];
 
+    // par alternates the scale slots between consecutive rows that reach
+    // the row barrier.  A skipped row (bad buffer) reaches no barrier, so it
+    // must not flip par: otherwise a fast warp could write the next row's
+    // slot while a slow one still reads it for the previous row.
     int par = 0;
-    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x, par ^= 1) {
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
         const int64_t b = row / T;
         const int64_t t = row - b * T;
         const EncPtrs p = src.get(b);
@@ -256,7 +428,7 @@ encode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
         for (int j = 0; j < GPT; ++j) {
             const int64_t g = (int64_t)j * nt + tid;
             if (VEC) {
-                if (g < G) {
+                if (g < G && CF_IN(8 * g + 8 <= C && t < T)) {
                     xraw[j] = ld_ro_v4(xr + 8 * g);
                     if (Src::kDelta) praw[j] = ld_ro_v4(pr + 8 * g);
                     const float4 a = ld_state_v4(rr + 8 * g);
@@ -320,6 +492,7 @@ encode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
             for (int w = 0; w < nw; ++w) tot = fmaxf(tot, sh_max[par][w]);
             scale = tot;
         }
+        par ^= 1;
         const float half = __fmul_rn(0.5f, scale);
 
         // Phase 4: quantise, error feedback, mirror update, pack, store.
@@ -341,7 +514,7 @@ encode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
             uint32_t word = field << ((lane % GPW) * 8 * BITS);
 #pragma unroll
             for (int o = 1; o < GPW; o <<= 1) word |= __shfl_xor_sync(kFullMask, word, o);
-            if (g < G) {
+            if (g < G && CF_IN(8 * g + (VEC ? 8 : 1) <= C && t < T)) {
                 if (VEC) {
                     st_stream_v4(er + 8 * g, make_float4(eo[0], eo[1], eo[2], eo[3]));
                     st_stream_v4(er + 8 * g + 4, make_float4(eo[4], eo[5], eo[6], eo[7]));
@@ -359,10 +532,10 @@ encode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
                         }
                     }
                 }
-                if ((lane % GPW) == 0) cw[g / GPW] = word;
+                if ((lane % GPW) == 0 && CF_IN(g / GPW < W)) cw[g / GPW] = word;
             }
         }
-        if (tid == 0) p.scales[t] = scale;
+        if (tid == 0 && CF_IN(t < T)) p.scales[t] = scale;
     }
 }
 
@@ -395,7 +568,7 @@ decode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
 #pragma unroll
         for (int j = 0; j < GPT; ++j) {
             const int64_t g = (int64_t)j * nt + tid;
-            if (g < G) {
+            if (g < G && CF_IN((g + 1) * BITS <= 4 * W && t < T)) {
                 // group g's 8*BITS bits: byte g (1 bit) or half-word g (2 bits)
                 if (BITS == 1)
                     field[j] = __ldg(reinterpret_cast<const uint8_t *>(cw) + g);
@@ -405,7 +578,7 @@ decode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
                 field[j] = 0u;
             }
             if (VEC) {
-                if (g < G) {
+                if (g < G && CF_IN(8 * g + 8 <= C)) {
                     const float4 a = ld_state_v4(rr + 8 * g);
                     const float4 c = ld_state_v4(rr + 8 * g + 4);
                     r[j][0] = a.x; r[j][1] = a.y; r[j][2] = a.z; r[j][3] = a.w;
@@ -422,7 +595,7 @@ decode_rows_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status)
 #pragma unroll
         for (int j = 0; j < GPT; ++j) {
             const int64_t g = (int64_t)j * nt + tid;
-            if (g >= G) continue;
+            if (g >= G || !CF_IN(8 * g + (VEC ? 8 : 1) <= C)) continue;
             float ro[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -458,6 +631,7 @@ __global__ void state_init_kernel(const uint16_t *x0, float *recon, float *err, 
     const int64_t groups = n >> 3;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += stride) {
+        if (!CF_IN(8 * g + 8 <= n)) continue;
         if (recon) {
             const uint4 xv = ld_ro_v4(x0 + 8 * g);
             const uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};

@@ -21,7 +21,10 @@ the current stream:
 
 ``ShardExchange`` carries the quantize mode (1- or 2-bit codes and per-token
 scales), ``LowrankShardExchange`` the low-rank mode (INT4 factors P and Q
-and their column scales).
+and their column scales).  ``FusedShardExchange`` is the quantize mode with
+the transfer fused into the kernels: the encode stores each row's payload
+straight into every receiver's slot (peer memory) and advances counters
+that the receivers' decode waits on, so no collective runs per step.
 
 The arithmetic runs in libcf's kernels (``CudaCodec``); this module lays out
 memory and orders the calls.  A caller may pass another codec object with
@@ -155,7 +158,8 @@ class CudaCodec:
         self._cache_size = cache
 
     def _array(self, kind, sets, make):
-        key = (kind,) + tuple(0 if t is None else t.data_ptr() for s in sets for t in s)
+        key = (kind,) + tuple(0 if t is None else t if isinstance(t, int) else t.data_ptr()
+                              for s in sets for t in s)
         arr = self._cache.get(key)
         if arr is None:
             arr = make(sets, self.device)
@@ -199,6 +203,17 @@ class CudaCodec:
             cf.cf_lowrank_decode_batched(d, len(sets),
                                          self._array("lr_dec", sets, cf.lowrank_dec_buffer_array),
                                          self.status)
+
+    def encode_publish_batched(self, d, sets, dsts, ack_target):
+        arr = self._array("pub", sets, cf.enc_publish_buffer_array)
+        dst = self._array("dst", dsts, cf.publish_dst_array)
+        cf.cf_encode_publish_batched(d, len(sets), arr, len(dsts), dst, ack_target, self.status)
+
+    def decode_wait_batched(self, d, sets, ready_target, acks):
+        arr = self._array("wait", sets, cf.dec_wait_buffer_array) if sets else None
+        ack = self._array("ack", [(a,) for a in acks], lambda v, dev: cf.pointer_array(
+            [t[0] for t in v], dev)) if acks else None
+        cf.cf_decode_wait_batched(d, len(sets), arr, ready_target, len(acks), ack, self.status)
 
     def status_value(self) -> int:
         """First error any batched call recorded (synchronises)."""
@@ -377,7 +392,8 @@ class LowrankShardExchange(_Exchange):
     """The low-rank mode: rank `rank` factors from `iters` subspace
     iterations, INT4-quantised.  Each step's encode takes one fp32 [C, rank]
     Gaussian start block per buffer (`omegas`), or None for the warm start
-    from the previous step's Q (every step after the first).  The encode
+    from the previous step's Q (allowed only for a buffer that an earlier
+    step encoded; otherwise step() raises ValueError).  The encode
     uses a device workspace of cf_lowrank_workspace_bytes per buffer;
     status() reads the numeric status of every buffer.  Otherwise as
     ShardExchange (no bf16 emission)."""
@@ -391,6 +407,9 @@ class LowrankShardExchange(_Exchange):
                          tokens, channels, buffers, group, device, codec, loopback)
         self.ws_bytes = self.codec.lowrank_workspace_bytes(self.d)
         self.workspace = torch.zeros(buffers * self.ws_bytes, dtype=torch.uint8, device=self.device)
+        # buffer b's workspace slice holds a Q to warm-start from only after
+        # an encode of that buffer with a start block
+        self.encoded = [False] * buffers
         L = self.layout
         self._dec_sets = [L.parts(self._payload(p), b) + (self.recon_r[p][b],)
                           for p in self.peers for b in range(buffers)]
@@ -403,6 +422,10 @@ class LowrankShardExchange(_Exchange):
             omegas = [None] * self.buffers
         if len(omegas) != self.buffers:
             raise ValueError(f"expected {self.buffers} start blocks, got {len(omegas)}")
+        cold = [b for b in range(self.buffers) if omegas[b] is None and not self.encoded[b]]
+        if cold:
+            raise ValueError(f"buffers {cold} have no earlier encode to warm-start from: "
+                             "the first compressed step needs a start block for every buffer")
         for om in omegas:
             if om is not None and (om.dtype != torch.float32 or tuple(om.shape) != (self.channels, self.layout.rank)
                                    or not om.is_contiguous()):
@@ -411,6 +434,7 @@ class LowrankShardExchange(_Exchange):
         sets = [(xs[b], self.recon_s[b], self.err[b], omegas[b]) + L.parts(self.send, b)
                 for b in range(self.buffers)]
         self.codec.lowrank_encode_batched(self.d, sets, self.workspace)
+        self.encoded = [True] * self.buffers
         self._all_gather(self.recv, self.send)
         self.codec.lowrank_decode_batched(self.d, self._dec_sets)
 
@@ -419,16 +443,135 @@ class LowrankShardExchange(_Exchange):
         buffer's last Q, the warm start of the next step."""
         sd = super().state_dict()
         sd["workspace"] = self.workspace.detach().cpu().clone()
+        sd["encoded"] = list(self.encoded)
         return sd
 
     def load_state_dict(self, sd: dict) -> None:
-        if "workspace" not in sd or sd["workspace"].numel() != self.workspace.numel():
+        if ("workspace" not in sd or sd["workspace"].numel() != self.workspace.numel()
+                or len(sd.get("encoded", ())) != self.buffers):
             raise ValueError("state_dict was taken on a different exchange")
         super().load_state_dict(sd)
         self.workspace.copy_(sd["workspace"])
+        self.encoded = list(sd["encoded"])
 
     def status(self) -> list:
         """Per-buffer numeric status of the last encodes (synchronises; the
         codec reads and clears each buffer's status word)."""
         return [self.codec.lowrank_status(self.workspace[b * self.ws_bytes:(b + 1) * self.ws_bytes])
                 for b in range(self.buffers)]
+
+
+# ---------------------------------------------------------------- fused exchange
+
+@dataclasses.dataclass
+class SlotMemory:
+    """The memory the fused exchange writes through, as seen from one rank.
+
+    For every rank r (all addressable from this rank: its own memory, and
+    each peer's through peer access):
+      recv[r]  uint8 [2, world, bytes_per_rank]: slot s of sender p's payload
+               at receiver r is recv[r][s, p];
+      ready[r] int64 [world]: rows sender p has published to receiver r;
+      ack[r]   int64 [world]: steps receiver q has decoded from r's payloads.
+    Counters only grow; a fresh SlotMemory starts them at zero."""
+    recv: list
+    ready: list
+    ack: list
+
+
+def local_slot_memory(layout, world: int, device) -> SlotMemory:
+    """One process owning every rank's memory (one rank in loopback on one
+    GPU, or a test that stands in for several ranks)."""
+    return SlotMemory(
+        recv=[torch.zeros(2, world, layout.bytes_per_rank, dtype=torch.uint8, device=device)
+              for _ in range(world)],
+        ready=[torch.zeros(world, dtype=torch.int64, device=device) for _ in range(world)],
+        ack=[torch.zeros(world, dtype=torch.int64, device=device) for _ in range(world)])
+
+
+def symmetric_slot_memory(layout, group, device) -> SlotMemory:
+    """Every rank's slots and counters in one symmetric allocation per rank
+    (torch symmetric memory), each peer's mapped for peer access.  The
+    kernels only store to and atomically add into the peers' memory; no TMA
+    load and no collective reads it."""
+    import torch.distributed._symmetric_memory as symm_mem
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    nrecv = 2 * world * layout.bytes_per_rank
+    total = nrecv + 16 * world                       # + ready[world] + ack[world], int64
+    buf = symm_mem.empty(total, dtype=torch.uint8, device=device)
+    buf.zero_()
+    hdl = symm_mem.rendezvous(buf, group)
+    dist.barrier(group)
+    mem = SlotMemory([], [], [])
+    for r in range(world):
+        t = buf if r == rank else hdl.get_buffer(r, (total,), torch.uint8)
+        mem.recv.append(t[:nrecv].view(2, world, layout.bytes_per_rank))
+        mem.ready.append(t[nrecv:nrecv + 8 * world].view(torch.int64))
+        mem.ack.append(t[nrecv + 8 * world:].view(torch.int64))
+    mem._keep = (buf, hdl)  # the mapping lives as long as the exchange
+    return mem
+
+
+class FusedShardExchange(_Exchange):
+    """The quantize-mode exchange with the transfer fused into the codec
+    kernels: each step is one publishing encode, which stores every row's
+    codes and scale straight into every receiver's slot for this rank and
+    then advances the receivers' ready counters, and one waiting decode of
+    every peer's slot, which reads a peer's rows once its counter shows them
+    and then acknowledges the step to every sender.  Two slots per (receiver,
+    sender) are used in turn; before it overwrites a slot the encode waits
+    until the receiver has acknowledged the step that last used it.  No
+    collective runs per step.  `memory` defaults to symmetric memory across
+    the process group (one local allocation for a single rank)."""
+
+    def __init__(self, tokens: int, channels: int, bits: int, buffers: int, *, group=None,
+                 device=None, codec=None, loopback: bool = False, memory: SlotMemory = None):
+        if bits not in (1, 2):
+            raise ValueError(f"bits must be 1 or 2, got {bits}")
+        super().__init__(PayloadLayout(tokens, channels, bits, buffers), cf.desc(tokens, channels, bits),
+                         tokens, channels, buffers, group, device, codec, loopback)
+        if not self.peers:
+            raise ValueError("a single rank needs loopback=True: it has no other receiver")
+        self.send = self.recv = None          # the slots replace the gather buffers
+        if memory is None:
+            memory = (local_slot_memory(self.layout, 1, self.device) if self.world == 1
+                      else symmetric_slot_memory(self.layout, group, self.device))
+        self.memory = memory
+        self.epoch = 0          # compressed steps taken
+        self.base = 0           # epoch at which this memory's counters were zero
+
+    def _receivers(self):
+        """Ranks whose slots this rank's payload goes to (the same set as the
+        ranks it decodes: the exchange is symmetric)."""
+        return self.peers
+
+    def step(self, xs) -> None:
+        self._check(xs)
+        self.epoch += 1
+        k = self.epoch - self.base           # steps on this memory's counters
+        s, me, L, m = self.epoch % 2, self.rank, self.layout, self.memory
+        dsts = [(m.recv[r][s, me], m.ready[r][me:me + 1], m.ack[me][r:r + 1]) for r in self._receivers()]
+        enc = [(xs[b], self.recon_s[b], self.err[b], L.codes_offset(b), L.scales_offset(b))
+               for b in range(self.buffers)]
+        self.codec.encode_publish_batched(self.d, enc, dsts, max(k - 2, 0))
+        dec, acks = [], []
+        for p in self.peers:
+            slot = m.recv[me][s, p]
+            dec += [(L.codes(slot, b), L.scales(slot, b), self.recon_r[p][b], m.ready[me][p:p + 1])
+                    for b in range(self.buffers)]
+            acks.append(m.ack[p][me:me + 1])
+        self.codec.decode_wait_batched(self.d, dec, k * self.buffers * self.tokens, acks)
+
+    def state_dict(self) -> dict:
+        sd = super().state_dict()
+        sd["epoch"] = self.epoch
+        return sd
+
+    def load_state_dict(self, sd: dict) -> None:
+        """Restores the states into this exchange, whose slot memory must be
+        fresh (counters at zero on every rank): the counters then count from
+        the restored step on."""
+        if "epoch" not in sd:
+            raise ValueError("state_dict was taken on a different exchange")
+        super().load_state_dict(sd)
+        self.epoch = self.base = int(sd["epoch"])

@@ -1,8 +1,9 @@
 #!/usr/bin/env python
 """Throughput of the residual-compression hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload flux_sp]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload cogvideox]
                     [--impl ours|reference] [--no-cpu-baseline] [--no-e2e]
+                    [--no-lowrank-leg]
 
 A "step" is one denoising step of the workload: every exchanged buffer is
 encoded by the sender (residual + error feedback + per-token scale +
@@ -12,8 +13,10 @@ quantise + pack + error/mirror update) and decoded by the receiver (unpack
 Metric: GB/s of bf16 activation processed = 2 bytes * T * C * buffers *
 steps / (encode + decode time), whole job (all ranks).  Inputs are the
 seeded synthetic drift trajectories, pre-generated in HBM before timing; one
-step touches ~5 GB (FLUX-like shard), far more than the 126 MB L2, so no L2
-flush is needed between steps.
+step of the default workload (CogVideoX-like, 60 buffers of 17550 x 1920)
+touches ~45 GB, far more than the 126 MB L2, so no L2 flush is needed
+between steps.  The same line also reports, under "lowrank", the low-rank
+mode on its own workload (114 x 4096 x 3072, rank 32, 2 iterations).
 
 Multi-GPU: by default sender and receiver share a device, so N ranks run N
 independent replicas of the workload ("weak" scaling).  The timed region is
@@ -55,7 +58,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="flux_sp", choices=list(W.WORKLOADS))
+    ap.add_argument("--workload", default="cogvideox", choices=list(W.WORKLOADS),
+                    help="default: cogvideox (60 x 17550 x 1920, 2-bit), the largest workload")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -84,6 +88,13 @@ def parse():
                          "-1 the library default")
     ap.add_argument("--gen-steps", type=int, default=0,
                     help="distinct pre-generated steps to cycle through (0 = all that fit)")
+    ap.add_argument("--e2e-steps", type=int, default=40,
+                    help="steps of the end-to-end leg (each moves a whole step's activations "
+                         "over PCIe, ~70 ms for cogvideox)")
+    ap.add_argument("--no-lowrank-leg", action="store_true",
+                    help="quantize workloads: skip the low-rank leg (114 x 4096 x 3072, rank 32) "
+                         "that the line also reports under 'lowrank'")
+    ap.add_argument("--lowrank-steps", type=int, default=60)
     return ap.parse_args()
 
 
@@ -307,6 +318,41 @@ def oracle_sample_all_cores(wl, seconds):
     return sum(rates) / 1e9, cores, model
 
 
+# ------------------------------------------------------------ config
+
+def quant_config(args, wl, world):
+    """The `config` of a quantize-mode line; both arms print this same dict."""
+    n, T, C, bits = wl.buffers, wl.tokens, wl.channels, wl.bits
+    return {"workload": args.workload, "tokens": T, "channels": C, "buffers": n,
+            "bits": bits, "mode": f"{bits}-bit {'mean-abs' if bits == 1 else 'absmax'} + EF"
+            + (", delta-state sender" if args.delta else "")
+            + (", emitting decode" if args.emit else ""),
+            "parallelism": f"replicas x{world}",
+            "l2": f"inputs larger than L2 ({n * T * C * 14 / 1e9:.1f} GB touched per step)",
+            "launches_per_step": 2}
+
+
+def lowrank_config(args, wl, world):
+    """The `config` of a low-rank line; both arms print this same dict."""
+    it = wl.iters
+    return {"workload": "lowrank", "tokens": wl.tokens, "channels": wl.channels,
+            "buffers": wl.buffers, "rank": wl.rank, "iters": it,
+            "mode": "low-rank INT4 + EF" + (", warm start" if args.warm else ""),
+            "parallelism": f"replicas x{world}", "l2": "inputs larger than L2",
+            "launches_per_step": 5 + 3 * it + 1}
+
+
+def lowrank_workload(args):
+    wl = W.WORKLOADS["lowrank"]
+    if args.workload == "lowrank" and args.buffers:
+        wl = W.replace(wl, buffers=args.buffers)
+    if args.iters:
+        wl = W.replace(wl, iters=args.iters)
+    if args.rank:
+        wl = W.replace(wl, rank=args.rank)
+    return wl
+
+
 # ------------------------------------------------------------ GPU leg
 
 def run_ours(args, world, rank, local):
@@ -419,9 +465,11 @@ def run_ours(args, world, rank, local):
     if not args.no_e2e and not args.delta and not args.emit:
         e2e = run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, status)
         e2e["ms"] = R.reduce_scalar(e2e["ms"], "max")
-        e2e = {"value": round(bytes_processed / (e2e["ms"] / 1e3) / 1e9, 3), "unit": "GB/s",
+        e_steps = e2e["steps"]
+        e2e = {"value": round(2 * T * C * n * e_steps * world / (e2e["ms"] / 1e3) / 1e9, 3),
+               "unit": "GB/s", "steps": e_steps,
                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-               "ms_per_step": round(e2e["ms"] / args.steps, 4),
+               "ms_per_step": round(e2e["ms"] / e_steps, 4),
                "overlap": f"{e2e['chunks']} chunks on copy-in / compute / copy-out streams"}
 
     cpu = None
@@ -445,13 +493,7 @@ def run_ours(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 in, fp32 state", "data": "synthetic",
-        "config": {"workload": args.workload, "tokens": T, "channels": C, "buffers": n,
-                   "bits": bits, "mode": f"{bits}-bit {'mean-abs' if bits == 1 else 'absmax'} + EF"
-                   + (", delta-state sender" if args.delta else "")
-                   + (", emitting decode" if args.emit else ""),
-                   "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2 ({n * T * C * 14 / 1e9:.1f} GB touched per step)",
-                   "launches_per_step": 2},
+        "config": quant_config(args, wl, world),
         "roofline": {"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(enc_gbs / peak, 4), "traffic": traffic,
                      "kernel": ("encode_tma_kernel (batched, TMA row staging)" if args.pipeline != 0
@@ -561,13 +603,7 @@ def run_lowrank(args, world, rank, local):
     cf.lib()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    wl = W.WORKLOADS[args.workload]
-    if args.buffers:
-        wl = W.replace(wl, buffers=args.buffers)
-    if args.iters:
-        wl = W.replace(wl, iters=args.iters)
-    if args.rank:
-        wl = W.replace(wl, rank=args.rank)
+    wl = lowrank_workload(args)
     n, T, C, r, it = wl.buffers, wl.tokens, wl.channels, wl.rank, wl.iters
     d = cf.desc(T, C, 0, r, it)
     step_bytes = n * T * C * 2
@@ -670,9 +706,10 @@ def run_lowrank(args, world, rank, local):
         e2e = run_lowrank_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, OM, pc, ps,
                               qc, qs, ws)
         e2e["ms"] = R.reduce_scalar(e2e["ms"], "max")
-        e2e = {"value": round(2 * T * C * n * args.steps * world / (e2e["ms"] / 1e3) / 1e9, 3),
-               "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
-               "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(e2e["ms"] / args.steps, 4),
+        e_steps = e2e["steps"]
+        e2e = {"value": round(2 * T * C * n * e_steps * world / (e2e["ms"] / 1e3) / 1e9, 3),
+               "unit": "GB/s", "steps": e_steps, "h2d_bytes_per_step": e2e["h2d"],
+               "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(e2e["ms"] / e_steps, 4),
                "overlap": f"{e2e['chunks']} chunks on copy-in / compute / copy-out streams"}
 
     cpu = None
@@ -686,11 +723,7 @@ def run_lowrank(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 in, fp32 state, bf16 tensor products", "data": "synthetic",
-        "config": {"workload": args.workload, "tokens": T, "channels": C, "buffers": n,
-                   "rank": r, "iters": it,
-                   "mode": "low-rank INT4 + EF" + (", warm start" if args.warm else ""),
-                   "parallelism": f"replicas x{world}", "l2": "inputs larger than L2",
-                   "launches_per_step": launches_per_step},
+        "config": lowrank_config(args, wl, world),
         "roofline": {"bound": "hbm",
                      "achieved": round(app_enc_bytes / (app_enc_ms / 1e3) / 1e9, 1),
                      "peak": peak, "unit": "GB/s",
@@ -715,6 +748,23 @@ def run_lowrank(args, world, rank, local):
         "clocks": clocks,
     }
     return out
+
+
+def lowrank_leg(args, world, rank, local):
+    """The low-rank mode on its own workload (114 x 4096 x 3072, rank 32, 2
+    iterations), timed like run_lowrank after the quantize line has freed its
+    memory: the part of its line that the quantize line does not carry."""
+    torch.cuda.empty_cache()
+    la = argparse.Namespace(**vars(args))
+    la.workload, la.buffers, la.warm = "lowrank", 0, False
+    la.steps = max(1, min(args.steps, args.lowrank_steps))
+    la.warmup = max(3, min(args.warmup, 5))
+    la.gen_steps, la.no_e2e, la.no_cpu_baseline = 3, True, True
+    o = run_lowrank(la, world, rank, local)
+    keys = ("metric", "value", "unit", "steps", "warmup", "ms_per_step", "config", "roofline",
+            "decode", "whole_call", "tensor_pipe", "lowrank_status", "payload_ratio",
+            "gpu_launches", "clocks")
+    return {k: o[k] for k in keys if k in o}
 
 
 def run_lowrank_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, OM, pc, ps, qc, qs, ws):
@@ -779,10 +829,11 @@ def run_lowrank_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, OM, pc,
         step(i)
     settle()
     torch.cuda.synchronize()
+    steps = max(1, min(args.steps, args.e2e_steps))
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     s_in.wait_stream(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         step(i)
     settle()
     b.record(stream)
@@ -790,7 +841,7 @@ def run_lowrank_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, OM, pc,
     st = max(cf.cf_lowrank_status(ws[k * wsb:]) for k in range(n))
     assert st in (0, 6), cf.cf_status_string(st)
     return {"ms": a.elapsed_time(b), "h2d": n * T * C * 2,
-            "d2h": sum(t.numel() * t.element_size() for t in outs), "chunks": nch}
+            "d2h": sum(t.numel() * t.element_size() for t in outs), "chunks": nch, "steps": steps}
 
 
 def run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, status):
@@ -860,7 +911,7 @@ def run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, 
         step(i)
     settle()
     torch.cuda.synchronize()
-    steps = args.steps
+    steps = max(1, min(args.steps, args.e2e_steps))
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     s_in.wait_stream(stream)
@@ -870,7 +921,7 @@ def run_e2e(cf, d, wl, args, dev, stream, recon_s, recon_r, err, codes, scales, 
     b.record(stream)
     torch.cuda.synchronize()
     return {"ms": a.elapsed_time(b), "h2d": n * T * C * 2,
-            "d2h": codes.numel() * 4 + scales.numel() * 4, "chunks": nch}
+            "d2h": codes.numel() * 4 + scales.numel() * 4, "chunks": nch, "steps": steps}
 
 
 def run_reference(args, world, rank):
@@ -878,6 +929,13 @@ def run_reference(args, world, rank):
     if rank != 0:
         return None
     wl = W.WORKLOADS[args.workload]
+    if wl.mode == "lowrank":
+        wl = lowrank_workload(args)
+        config = lowrank_config(args, wl, world)
+    else:
+        if args.buffers:
+            wl = W.replace(wl, buffers=args.buffers)
+        config = quant_config(args, wl, world)
     per_step = 1
     cores, kind = 1, "single-threaded C oracle"
     if wl.mode == "lowrank":
@@ -912,13 +970,10 @@ def run_reference(args, world, rank):
         "ms_per_step": round(sec * 1e3 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 state",
         "data": "synthetic",
-        "config": dict({"workload": args.workload, "tokens": wl.tokens, "channels": wl.channels,
-                        "buffers": wl.buffers},
-                       **({"rank": wl.rank, "iters": wl.iters} if wl.mode == "lowrank"
-                          else {"bits": wl.bits}),
-                       sample=f"each step = {per_step} of the {wl.buffers} buffers"),
+        "config": config,
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{per_step} buffer(s) per step, {args.steps} steps, {kind}"},
+                         "sample": f"each step is {per_step} of the {wl.buffers} buffers "
+                                   f"({wl.tokens}x{wl.channels}), {args.steps} steps, {kind}"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -940,6 +995,8 @@ def main():
             out = run_exchange(args, world, rank, local)
         else:
             out = run_ours(args, world, rank, local)
+            if not args.no_lowrank_leg:
+                out["lowrank"] = lowrank_leg(args, world, rank, local)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

@@ -119,14 +119,8 @@ typedef struct cf_dec_emit_buffer {
  * graph and replayed; the host-side argument checks run at capture time.
  * cf_lowrank_encode_noalloc's first call on a device must precede capture. */
 
-/* Diagnostic (no counterpart in the paper): checks on the device that the
- * bounded wait every TMA and tensor-core pipeline uses ends.  One CTA waits,
- * with at most `polls` polls (1 .. 65536), on an mbarrier it has signalled
- * itself and on one that nothing signals, and writes out_dev[0..1] (device
- * int32[2], 4-byte aligned): [0] = 1 if the signalled wait completed;
- * [1] = CF_ERR_TIMEOUT if the unsignalled wait gave up (CF_OK otherwise).
- * The GPU never hangs or faults: the unsignalled wait stops after `polls`. */
-cf_status cf_diag_bounded_wait(int32_t polls, int32_t *out_dev, void *stream);
+/* Tuning knobs, measurement hooks and the bounded-wait self-test are
+ * declared apart, in cf_diag.h: product callers need none of them. */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *cf_status_string(cf_status s);
@@ -135,11 +129,16 @@ const char *cf_status_string(cf_status s);
 int32_t cf_abi_version(void);
 
 /* uint32 code words per token row: ceil(channels * bits / 32); 0 for an
- * invalid descriptor. */
+ * invalid descriptor.  Cite: the 1- and 2-bit variants of the "Measured
+ * effects" table (b bits per element); the word layout is this library's
+ * (least significant bit first, see above). */
 int64_t cf_codes_words_per_row(const cf_desc *d);
 
 /* Bytes on the wire for one buffer: codes + scales (quantize mode) or INT4
- * factors + scales (low-rank mode); 0 for an invalid descriptor. */
+ * factors + scales (low-rank mode); 0 for an invalid descriptor.  Cite:
+ * "Key results" (rank 32 with INT4 factors compresses about 100x: at
+ * 1024 x 3072 this size gives 95.6x) and the 1/2-bit rows of "Measured
+ * effects" (16/b x before the per-token scales). */
 int64_t cf_payload_bytes(const cf_desc *d);
 
 /* Warmup step ("Measured effects": the first step is sent uncompressed).
@@ -153,14 +152,23 @@ cf_status cf_state_init(const cf_desc *d, const uint16_t *x0, float *recon,
 
 /* Sender, quantize mode, one buffer: residual with error feedback, per-token
  * scale, quantise, pack, error update and mirror update in one pass.
+ * Cite: "Approach" (transmit the residual against the previous
+ * reconstruction; keep a sender-side error-feedback buffer) and the
+ * Compact-1bit / Compact-2bit rows of the "Measured effects" table.
  * x: bf16 [T][C]; recon_s: fp32 [T][C] read and updated in place;
  * err: fp32 [T][C] written; codes: uint32 [T][words_per_row] written;
- * scales: fp32 [T] written.  All device pointers, non-overlapping. */
+ * scales: fp32 [T] written.  All device pointers, non-overlapping.
+ * Errors: CF_ERR_INVALID_ARG (null or host pointer, T < 0, C < 1, rank or
+ * iters set), CF_ERR_UNSUPPORTED (bits not 1 or 2, C > 16384, scale_kind
+ * not 0), CF_ERR_ALIGNMENT, CF_ERR_CUDA; nothing is launched on an error. */
 cf_status cf_encode(const cf_desc *d, const uint16_t *x, float *recon_s,
                     float *err, uint32_t *codes, float *scales, void *stream);
 
 /* Receiver, quantize mode, one buffer: unpack, dequantise, accumulate.
- * codes, scales as written by cf_encode; recon_r: fp32 [T][C] updated. */
+ * Cite: "Approach" (the receiver adds the decoded residual to its own
+ * reconstruction of the previous step).
+ * codes, scales as written by cf_encode; recon_r: fp32 [T][C] updated.
+ * Never reads sender state.  Errors as cf_encode. */
 cf_status cf_decode(const cf_desc *d, const uint32_t *codes,
                     const float *scales, float *recon_r, void *stream);
 
@@ -173,7 +181,10 @@ cf_status cf_decode_emit(const cf_desc *d, const uint32_t *codes, const float *s
                          float *recon_r, uint16_t *out, void *stream);
 
 /* Batched forms: `n` buffers of the same shape in ONE launch, with the same
- * per-buffer semantics as cf_encode / cf_decode.  `bufs_dev` is a DEVICE
+ * per-buffer semantics as cf_encode / cf_decode (cite: as those; a diffusion
+ * transformer exchanges the K and V buffers of every layer at every step,
+ * "Approach" and the sequence-parallel setting of "Key results").  n < 0 is
+ * CF_ERR_INVALID_ARG; n == 0 launches nothing.  `bufs_dev` is a DEVICE
  * array of n descriptors (it must stay valid until the work completes).
  * Pointers inside it are checked on the device: a buffer with a null or
  * misaligned pointer is skipped and, when `status_dev` (device int32) is
@@ -188,6 +199,95 @@ cf_status cf_decode_batched(const cf_desc *d, int32_t n,
                             void *stream);
 cf_status cf_decode_emit_batched(const cf_desc *d, int32_t n,
                                  const cf_dec_emit_buffer *bufs_dev,
+                                 int32_t *status_dev, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Publishing encode and waiting decode: the sequence-parallel exchange with
+ * the payload transfer fused into the codec kernels.  Cite: "Approach"
+ * (senders transmit the compressed residual; every receiver keeps its own
+ * reconstruction), the 6.7x communication-bound speed-up of "Key results"
+ * (the transfer is what the compression shortens) and the ring-attention row
+ * of "Measured effects" (each rank's K/V reach every other rank).
+ *
+ * The encode writes each row's codes and scale straight into the payload
+ * slot that every receiver keeps for this sender -- plain stores, 16 bytes
+ * wide where the code row allows it, to memory that may be another GPU's
+ * (peer access) or this GPU's own -- instead of into a local payload that a
+ * collective then copies.  Synchronisation is by monotonic 64-bit counters
+ * in the receivers' memory:
+ *  - ready: rows published.  After its last row every CTA of the encode
+ *    adds the rows it walked to each destination's ready counter with a
+ *    system-scope release (fence, then atomic add).  For step e (1, 2, ...)
+ *    of a sender publishing R = n * T rows per step, the counter reaches
+ *    e * R when step e is complete, since a sender's steps are ordered.
+ *  - ack: steps decoded.  After its decode the receiver adds 1 to an ack
+ *    counter per sender (in that sender's memory).  With two payload slots
+ *    per (receiver, sender) used alternately (step e writes slot e % 2), the
+ *    sender at step e waits, before its first store to a destination, until
+ *    that destination's ack is >= e - 2 (ack_target), i.e. until the slot's
+ *    previous contents were decoded.
+ * Every wait is bounded (about a second): on expiry the CTA records
+ * CF_ERR_TIMEOUT in status_dev and stops, and nothing hangs.  A sender that
+ * stopped publishes nothing, so its receivers time out in turn.
+ * Requirements: C % 8 == 0; the decode also ceil(C*bits/32) % 4 == 0 (the
+ * TMA row pipeline); otherwise CF_ERR_UNSUPPORTED.  No TMA load ever reads
+ * another GPU's memory: the sender's loads are local, the receiver's bulk
+ * copies read its own memory. */
+
+/* One destination of a publishing encode (all device pointers; the first
+ * two may be another GPU's memory mapped for peer access). */
+typedef struct cf_publish_dst {
+    uint8_t *payload;        /* this sender's payload slot at the receiver, 16-byte aligned */
+    uint64_t *ready;         /* the receiver's ready counter for this sender, 8-byte aligned */
+    const uint64_t *ack;     /* this sender's ack counter for that receiver, or NULL: no wait */
+} cf_publish_dst;
+
+/* One buffer of a publishing encode: the sender state as in cf_enc_buffer,
+ * and where the buffer's codes ([T][ceil(C*bits/32)] uint32) and scales
+ * ([T] fp32) sit in every destination's payload slot. */
+typedef struct cf_enc_publish_buffer {
+    const uint16_t *x;       /* bf16 [T][C], this step's activation             */
+    float *recon_s;          /* fp32 [T][C], updated                            */
+    float *err;              /* fp32 [T][C], written                            */
+    int64_t codes_offset;    /* bytes from a slot's base, multiple of 16        */
+    int64_t scales_offset;   /* bytes from a slot's base, multiple of 4         */
+} cf_enc_publish_buffer;
+
+/* Sender: cf_encode_batched's arithmetic for n buffers, with codes and
+ * scales stored into each of the ndst (1..8) destinations instead of local
+ * arrays, the ack wait before the stores and the ready publication after
+ * them.  bufs_dev: DEVICE array of n cf_enc_publish_buffer; dsts_dev: DEVICE
+ * array of ndst cf_publish_dst; both valid until the work completes.
+ * ack_target: see above (0 = no wait).  Buffer pointers are checked on the
+ * device as in cf_encode_batched (a bad buffer is skipped, its rows still
+ * count as published); a destination with a null or misaligned pointer
+ * stops every CTA before any store with CF_ERR_INVALID_ARG / ALIGNMENT in
+ * status_dev (device int32, zeroed by the caller; may be NULL). */
+cf_status cf_encode_publish_batched(const cf_desc *d, int32_t n,
+                                    const cf_enc_publish_buffer *bufs_dev, int32_t ndst,
+                                    const cf_publish_dst *dsts_dev, uint64_t ack_target,
+                                    int32_t *status_dev, void *stream);
+
+/* One buffer of a waiting decode: cf_dec_buffer plus the ready counter of
+ * the sender whose payload holds this buffer's codes and scales. */
+typedef struct cf_dec_wait_buffer {
+    const uint32_t *codes;
+    const float *scales;
+    float *recon_r;          /* fp32 [T][C], updated                            */
+    const uint64_t *ready;   /* 8-byte aligned, in this receiver's memory       */
+} cf_dec_wait_buffer;
+
+/* Receiver: cf_decode_batched for n buffers, where a CTA reads a buffer's
+ * codes only after that buffer's ready counter is >= ready_target (the
+ * sender's step e: e * rows published per step).  Then adds 1 to each of the
+ * nack (0..64) counters in acks_dev (DEVICE array of uint64_t*, each 8-byte
+ * aligned, possibly another GPU's memory), with a system-scope release after
+ * the decode.  A wait that expires records CF_ERR_TIMEOUT in status_dev,
+ * the CTA stops, and the acks are still sent (so that a sender does not
+ * block on a receiver that gave up). */
+cf_status cf_decode_wait_batched(const cf_desc *d, int32_t n,
+                                 const cf_dec_wait_buffer *bufs_dev, uint64_t ready_target,
+                                 int32_t nack, uint64_t *const *acks_dev,
                                  int32_t *status_dev, void *stream);
 
 /* ------------------------------------------------------------------------
@@ -234,10 +334,14 @@ cf_status cf_encode_delta_batched(const cf_desc *d, int32_t n,
  * nibbles, even column in the low nibble.  Scales: fp32 [r] per factor.
  * ---------------------------------------------------------------------- */
 
-/* Device workspace bytes cf_lowrank_encode needs for this descriptor. */
+/* Device workspace bytes cf_lowrank_encode needs for this descriptor (the
+ * subspace-iteration intermediates of "Approach" / "Builds on": the bf16
+ * residual copy, Y, P, Q, the Gram partials); 0 for an invalid descriptor. */
 int64_t cf_lowrank_workspace_bytes(const cf_desc *d);
 
-/* Bytes of one packed INT4 factor with `rows` rows at rank `rank`. */
+/* Bytes of one packed INT4 factor with `rows` rows at rank `rank`:
+ * rows * ceil(rank / 2) ("Key results": INT4 factors); 0 if rows < 0 or
+ * rank < 1. */
 int64_t cf_lowrank_factor_bytes(int64_t rows, int32_t rank);
 
 /* Sender, low-rank mode.  Alignment: x, recon_s, err 16 bytes; omega and the
@@ -335,7 +439,11 @@ cf_status cf_lowrank_decode(const cf_desc *d, const uint8_t *p_codes,
  *    CF_ERR_WORKSPACE without launching anything.
  *  - The first call on a device looks up the array's device address on the
  *    current device (cudaGetSymbolAddress) and caches it; make that first
- *    call before any stream capture on that device.
+ *    call before any stream capture on that device.  The cached address
+ *    belongs to the device's primary context: after cudaDeviceReset (or any
+ *    reset of the primary context) it is stale and this library does not
+ *    notice, so do not call this entry point again in a process that has
+ *    reset the device.
  *  - Every call on a device shares the one array, which keeps the previous
  *    call's contents (the implementation clears what must start at zero).
  *    Calls whose work overlaps on the GPU -- different streams without
@@ -354,48 +462,23 @@ cf_status cf_lowrank_encode_noalloc(const cf_desc *d, const uint16_t *x, float *
  * clears it.  Returns CF_ERR_CUDA if the copy or the sync fails. */
 cf_status cf_lowrank_status(void *workspace, void *stream);
 
-/* Engine of the low-rank dense products in this process: 0 (the default) =
- * tcgen05 tensor cores (the two subspace-iteration products with bf16
- * operands, and D = P^ Q^T in tf32 with a hi/lo split of the scaled P
- * factor, fp32 accumulation in TMEM), 1 = CUDA cores (same operands, fp32
- * FMA).  For cross-checks and diagnosis; both satisfy the same parity bar.
- * The sender and the receiver of a buffer must use the same engine: D is
- * bit-identical only within one engine.  Returns CF_ERR_INVALID_ARG for any
- * other value. */
-cf_status cf_set_lowrank_engine(int32_t engine);
-
-/* Measurement hook (no counterpart in the paper): CUDA events (cudaEvent_t,
- * passed as void*) that the low-rank calls record around their apply kernel
- * -- the kernel that forms D and updates the state -- so a caller can time
- * that one kernel inside a whole call.  When enc_start/enc_stop are non-null,
- * every later cf_lowrank_encode(_batched) records enc_start on its stream
- * immediately before the apply launch and enc_stop immediately after it;
- * dec_start/dec_stop likewise for cf_lowrank_decode(_batched).  Null pairs
- * (the default) record nothing.  Process-wide; the events stay the caller's
- * (create them before, destroy them after the calls that record them).  An
- * event that fails to record makes the call return CF_ERR_CUDA after its
- * launches.  Returns CF_ERR_INVALID_ARG if exactly one of a pair is null. */
-cf_status cf_lowrank_set_apply_events(void *enc_start, void *enc_stop, void *dec_start,
-                                      void *dec_stop);
-
-/* Memory pipeline of the quantize-mode kernels in this process: kernel 0 =
- * encode, 1 = decode; pipeline 0 = register-resident rows (each thread
- * loads its channel groups straight into registers), 1 = TMA row staging
- * (a producer warp streams whole rows into a ring of `stages` shared-memory
- * slots with 1-D bulk copies; consumer warps compute from shared memory;
- * the default).  stages 0 = built-in choice, else 2..8.  Both give bit-identical results;
- * the TMA pipeline applies when C % 8 == 0 (decode also needs
- * ceil(C*bits/32) % 4 == 0) and otherwise the call uses pipeline 0.
- * Returns CF_ERR_INVALID_ARG for out-of-range values. */
-cf_status cf_set_quant_pipeline(int32_t kernel, int32_t pipeline, int32_t stages);
-
-/* Launch-shape override for tuning sweeps: kernel 0 = encode, 1 = decode;
- * groups_per_thread in 1..4 (8 channels per group), threads a multiple of
- * 32 in 32..512, or 0 to restore the built-in choice; blocks_per_sm caps
- * the persistent grid (0 = occupancy limit).  Affects later launches in
- * this process only.  Returns CF_ERR_INVALID_ARG for out-of-range values. */
-cf_status cf_set_launch_override(int32_t kernel, int32_t groups_per_thread,
-                                 int32_t threads, int32_t blocks_per_sm);
+/* Non-blocking form for a batch: enqueues on `stream` one strided
+ * device-to-host copy of the status words of n workspace slices -- slice b
+ * at workspace + b * slice_bytes, slice_bytes normally
+ * cf_lowrank_workspace_bytes(d) -- into host_status[0..n-1] (int32), and
+ * returns without waiting.  The words are valid once the stream has passed
+ * this point (record an event after the call and wait on it, or read them
+ * after a later synchronisation), and they hold what the encodes enqueued
+ * before this call recorded.  Nothing is cleared: every encode resets its
+ * slice's word when it starts.  host_status must be page-locked host memory
+ * (cudaHostAlloc / cudaHostRegister), so that the copy is asynchronous;
+ * pageable memory is CF_ERR_INVALID_ARG.  workspace: device, 256-byte
+ * aligned; slice_bytes a positive multiple of 256 (CF_ERR_ALIGNMENT
+ * otherwise); n >= 0 (0 enqueues nothing).  Returns CF_ERR_CUDA if the copy
+ * cannot be enqueued.  Usable inside stream capture: the copy becomes a
+ * graph node. */
+cf_status cf_lowrank_status_async(const void *workspace, int64_t slice_bytes, int32_t n,
+                                  int32_t *host_status, void *stream);
 
 #ifdef __cplusplus
 }

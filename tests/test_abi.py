@@ -12,10 +12,10 @@ from activation_residual_compression_cf_b200 import build, cf
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _declared():
+def _declared(header=None):
     names = set()
     for fn in os.listdir(os.path.join(ROOT, "include")):
-        if fn.endswith(".h"):
+        if fn.endswith(".h") and (header is None or fn == header):
             src = open(os.path.join(ROOT, "include", fn)).read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
             names |= set(re.findall(r"\b(cf_\w+)\s*\(", src))
@@ -33,8 +33,22 @@ def test_every_declared_symbol_is_exported(L):
     assert declared, "no declarations found"
     for name in sorted(declared):
         assert hasattr(L, name), f"{name} declared in include/ but not exported"
-    assert declared <= set(cf.EXPORTS) | declared
-    assert set(cf.EXPORTS) <= declared
+    # the product header and the diagnostic header each match their list
+    assert _declared("cf.h") == set(cf.EXPORTS)
+    assert _declared("cf_diag.h") == set(cf.DIAG_EXPORTS)
+    assert not set(cf.EXPORTS) & set(cf.DIAG_EXPORTS)
+    assert declared == set(cf.EXPORTS) | set(cf.DIAG_EXPORTS)
+
+
+def test_async_status_validates_before_any_cuda_call(L):
+    h = ctypes.c_int32()
+    assert L.cf_lowrank_status_async(256, 256, 0, None, None) == 0           # n == 0: nothing
+    assert L.cf_lowrank_status_async(256, 256, -1, ctypes.byref(h), None) == 1
+    assert L.cf_lowrank_status_async(None, 256, 1, ctypes.byref(h), None) == 1
+    assert L.cf_lowrank_status_async(256, 256, 1, None, None) == 1
+    assert L.cf_lowrank_status_async(256, 0, 1, ctypes.byref(h), None) == 1
+    assert L.cf_lowrank_status_async(128, 256, 1, ctypes.byref(h), None) == 2  # workspace alignment
+    assert L.cf_lowrank_status_async(256, 100, 1, ctypes.byref(h), None) == 2  # slice alignment
 
 
 def test_abi_version_and_status_strings(L):
@@ -126,3 +140,18 @@ def test_binding_raises_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(cf, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="not built"):
         cf.lib()
+
+
+def test_publish_and_wait_validate_before_any_cuda_call(L):
+    d = ctypes.byref(cf.desc(4, 64, 2))
+    assert L.cf_encode_publish_batched(d, 1, None, 0, None, 0, None, None) == 1    # no destination
+    assert L.cf_encode_publish_batched(d, 1, None, 9, None, 0, None, None) == 1    # above 8
+    assert L.cf_encode_publish_batched(d, -1, None, 1, None, 0, None, None) == 1
+    assert L.cf_encode_publish_batched(d, 0, None, 1, None, 0, None, None) == 0    # nothing to do
+    assert L.cf_encode_publish_batched(ctypes.byref(cf.desc(4, 64, 3)), 1, None, 1, None, 0, None,
+                                       None) == 3
+    assert L.cf_decode_wait_batched(d, -1, None, 0, 0, None, None, None) == 1
+    assert L.cf_decode_wait_batched(d, 0, None, 0, 65, None, None, None) == 1      # acks above 64
+    assert L.cf_decode_wait_batched(d, 0, None, 0, 0, None, None, None) == 0
+    assert L.cf_set_quant_unit(0, 6) == 1 and L.cf_set_quant_unit(2, 4) == 1
+    assert L.cf_set_quant_unit(0, 4) == 0 and L.cf_set_quant_unit(0, 0) == 0

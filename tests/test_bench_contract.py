@@ -40,3 +40,23 @@ def test_reference_arm_lowrank_line():
     assert d["impl"] == "reference" and d["value"] > 0
     assert d["config"]["rank"] == 32 and d["config"]["iters"] == 2 and "bits" not in d["config"]
     assert d["cpu_baseline"]["cores"] >= 1
+
+
+def test_reference_arm_config_equals_the_gpu_arm_config():
+    """With no flags both arms run the default workload (the CogVideoX-like
+    one, the largest) and print the same `config` dict."""
+    lines = _run(args=("--steps", "1", "--warmup", "0"))
+    d = json.loads(lines[-1])
+    sys.path.insert(0, ROOT)
+    import bench
+    argv = sys.argv
+    try:
+        sys.argv = ["bench.py"]
+        args = bench.parse()
+    finally:
+        sys.argv = argv
+    assert args.workload == "cogvideox"
+    wl = bench.W.WORKLOADS[args.workload]
+    assert d["config"] == bench.quant_config(args, wl, 1)
+    assert d["config"]["tokens"] == 17550 and d["config"]["channels"] == 1920
+    assert d["config"]["buffers"] == 60 and d["config"]["bits"] == 2

@@ -13,7 +13,6 @@ def test_stamp_tracks_content_not_file_times(tmp_path, monkeypatch):
     lib = tmp_path / "libx.so"
     lib.write_bytes(b"\x7fELF")
     monkeypatch.setattr(B, "LIB", str(lib))
-    monkeypatch.setattr(B, "STAMP", str(lib) + ".sources")
     monkeypatch.setattr(B, "_deps", lambda: [str(src)])
     assert not B.up_to_date()                      # no stamp yet
     (tmp_path / "libx.so.sources").write_text(B._inputs_hash() + "\n")
@@ -40,6 +39,7 @@ def test_hash_covers_flags_and_file_names(tmp_path, monkeypatch):
     monkeypatch.setattr(B, "_deps", lambda: [str(a)])
     monkeypatch.setattr(B, "FLAGS", B.FLAGS + ["-DEXTRA"])
     assert B._inputs_hash() != h1                  # same file, other flags
+    assert B._inputs_hash(debug=True) != B._inputs_hash()   # the debug build has its own stamp
 
 
 def test_oracle_build_stamp(tmp_path, monkeypatch):

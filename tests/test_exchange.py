@@ -374,3 +374,173 @@ def test_lowrank_exchange_routes_every_peer_payload_world2():
     for rank, status, info, st in out:
         assert status == "ok", (rank, info)
         assert st == [0, 0]
+
+
+def test_lowrank_warm_start_before_any_encode_is_refused():
+    """A warm start (no start block) needs the Q of an earlier encode of that
+    buffer: on the first compressed step it raises at the call site instead
+    of starting subspace iteration from an empty workspace.  After a step
+    with start blocks it is accepted, and a checkpoint carries that state."""
+    from activation_residual_compression_cf_b200 import workloads as W
+    from activation_residual_compression_cf_b200.exchange import LowrankShardExchange
+    T, C, r, iters, B = 24, 48, 4, 2, 2
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r, iters=iters, buffers=B)
+    trajs = [W.trajectory(wl, b, steps=4) for b in range(B)]
+    ex = LowrankShardExchange(T, C, r, iters, B, device="cpu", codec=OracleLowrankCodec(r, iters),
+                              loopback=True)
+    ex.warmup([trajs[b][0] for b in range(B)])
+    with pytest.raises(ValueError, match="warm-start"):
+        ex.step([trajs[b][1] for b in range(B)])
+    with pytest.raises(ValueError, match=r"\[1\]"):
+        ex.step([trajs[b][1] for b in range(B)], [W.omega(wl, 0, 1), None])
+    ex.step([trajs[b][1] for b in range(B)], [W.omega(wl, b, 1) for b in range(B)])
+    sd = ex.state_dict()
+    fresh = LowrankShardExchange(T, C, r, iters, B, device="cpu", codec=OracleLowrankCodec(r, iters),
+                                 loopback=True)
+    with pytest.raises(ValueError):
+        fresh.step([trajs[b][2] for b in range(B)])
+    fresh.load_state_dict(sd)
+    assert fresh.encoded == [True, True]
+
+
+# ---------------------------------------------------------------- fused exchange
+
+class OracleFusedCodec(OracleCodec):
+    """The fused exchange's two calls on CPU tensors, computed by the oracle,
+    with the counter protocol of the publishing encode and the waiting decode
+    done by polling the shared counters (bounded by `timeout` seconds)."""
+
+    def __init__(self, bits, timeout=30.0):
+        super().__init__(bits)
+        self.timeout = timeout
+
+    def _wait(self, counter, target):
+        import time
+        t0 = time.time()
+        while int(counter[0]) < target:
+            if time.time() - t0 > self.timeout:
+                raise TimeoutError(f"counter {int(counter[0])} < {target}")
+            time.sleep(0.001)
+
+    def encode_publish_batched(self, d, sets, dsts, ack_target):
+        import oracle
+        from activation_residual_compression_cf_b200 import workloads as W
+        if ack_target:
+            for _, _, ack in dsts:
+                self._wait(ack, ack_target)
+        for x, rs, e, co, so in sets:
+            codes, scales, err = oracle.encode(W.bf16_bits(x), rs.numpy(), self.bits)
+            e.numpy()[...] = err
+            cb, sb = codes.view(np.uint8).reshape(-1), scales.view(np.uint8).reshape(-1)
+            for payload, _, _ in dsts:
+                payload[co:co + cb.size].copy_(torch.from_numpy(cb.copy()))
+                payload[so:so + sb.size].copy_(torch.from_numpy(sb.copy()))
+        for _, ready, _ in dsts:                 # after every store (one writer per counter)
+            ready[0] += d.tokens * len(sets)
+
+    def decode_wait_batched(self, d, sets, ready_target, acks):
+        import oracle
+        for c, s, rr, ready in sets:
+            self._wait(ready, ready_target)
+            oracle.decode(c.numpy().view(np.uint32).copy(), s.numpy().copy(), rr.numpy(), self.bits)
+        for a in acks:
+            a[0] += 1
+
+
+def _file_slot_memory(layout, world, folder):
+    """Every rank's slots and counters in files mapped shared by all the
+    rank processes (stands in for peer-mapped GPU memory)."""
+    from activation_residual_compression_cf_b200.exchange import SlotMemory
+    mem = SlotMemory([], [], [])
+    for r in range(world):
+        recv = torch.from_file(os.path.join(folder, f"recv{r}"), shared=True,
+                               size=2 * world * layout.bytes_per_rank, dtype=torch.uint8)
+        mem.recv.append(recv.view(2, world, layout.bytes_per_rank))
+        mem.ready.append(torch.from_file(os.path.join(folder, f"ready{r}"), shared=True, size=world,
+                                         dtype=torch.int64))
+        mem.ack.append(torch.from_file(os.path.join(folder, f"ack{r}"), shared=True, size=world,
+                                       dtype=torch.int64))
+    return mem
+
+
+def _fused_worker(rank, world, port, folder, leave_after, q):
+    import datetime
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    try:
+        import torch.distributed as dist
+        import oracle
+        from activation_residual_compression_cf_b200 import workloads as W
+        from activation_residual_compression_cf_b200.exchange import FusedShardExchange, PayloadLayout
+        from test_exchange import OracleFusedCodec, _file_slot_memory
+        dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                                world_size=world, timeout=datetime.timedelta(seconds=60))
+        T, C, bits, B, steps = 16, 64, 2, 2, 6
+        wl = W.replace(W.WORKLOADS["flux_sp"], tokens=world * T, channels=C, bits=bits, buffers=B)
+        trajs = [W.trajectory(wl, b, steps=steps) for b in range(B)]
+
+        def shard(x, p):
+            return x[p * T:(p + 1) * T].clone()
+
+        mem = _file_slot_memory(PayloadLayout(T, C, bits, B), world, folder)
+        codec = OracleFusedCodec(bits, timeout=3.0 if leave_after else 30.0)
+        ex = FusedShardExchange(T, C, bits, B, device="cpu", codec=codec, memory=mem)
+        ex.warmup([shard(trajs[b][0], rank) for b in range(B)])
+        for t in range(1, steps):
+            if leave_after and rank == 1 and t > leave_after:
+                q.put((rank, "left"))
+                q.close()
+                q.join_thread()
+                os._exit(0)                      # leaves between steps, nothing in flight
+            try:
+                ex.step([shard(trajs[b][t], rank) for b in range(B)])
+            except TimeoutError as e:
+                q.put((rank, "timeout", t, str(e)))
+                return
+        bad = []
+        for p in ex.peers:
+            for b in range(B):
+                rec, _ = oracle.state_init(W.bf16_bits(shard(trajs[b][0], p)))
+                for t in range(1, steps):
+                    oracle.encode(W.bf16_bits(shard(trajs[b][t], p)), rec, bits)
+                if not np.array_equal(ex.recon_r[p][b].numpy(), rec):
+                    bad.append((p, b))
+        counters = ([int(v) for v in mem.ready[rank]], [int(v) for v in mem.ack[rank]])
+        q.put((rank, "ok" if not bad else "bad", bad, counters))
+        dist.barrier()
+        dist.destroy_process_group()
+    except Exception as e:
+        q.put((rank, "fail", repr(e), None))
+
+
+def _run_fused(tmp_path, world, leave_after):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_fused_worker, args=(r, world, port, str(tmp_path), leave_after, q))
+          for r in range(world)]
+    for p in ps:
+        p.start()
+    out = sorted([q.get(timeout=240) for _ in range(world)], key=lambda t: t[0])
+    for p in ps:
+        p.join(timeout=60)
+    return out
+
+
+def test_fused_exchange_routes_every_payload_through_the_slots_world2(tmp_path):
+    """Two ranks exchange five compressed steps through each other's slots
+    (shared memory standing in for peer-mapped GPU memory): every receiver
+    state equals the oracle run on that peer's shard bit for bit, both slots
+    are reused under the ack protocol, and the counters end at five steps."""
+    out = _run_fused(tmp_path, 2, 0)
+    for rank, status, info, counters in out:
+        assert status == "ok", (rank, info)
+        ready, ack = counters
+        assert ready == [0 if p == rank else 5 * 2 * 16 for p in range(2)], (rank, ready)
+        assert ack == [0 if p == rank else 5 for p in range(2)], (rank, ack)
+
+
+def test_fused_exchange_a_rank_that_leaves_ends_the_survivors_next_step(tmp_path):
+    out = _run_fused(tmp_path, 2, 1)
+    assert out[1][1] == "left", out
+    assert out[0][1] == "timeout" and out[0][2] == 2, out

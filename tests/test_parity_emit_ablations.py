@@ -93,36 +93,44 @@ def test_decode_emit_batched_full_size_sampled():
         assert (out[b].cpu().numpy().view(np.uint16) == o_out).mean() > 0.9999
 
 
-def _final_error(mode, wl, xs, bits, side):
-    """Run all steps in one mode; return ||x_last - recon_r|| / ||x_last||."""
+def _lockstep(mode, wl, xs, bits):
+    """Runs all steps in one mode on the GPU and in the oracle side by side,
+    checks every step at the parity bar (the sender's codes, scales, error
+    and reconstruction, and the receiver's reconstruction against the
+    oracle's receiver), and returns ||x_last - recon_r|| / ||x_last|| of
+    the GPU and of the oracle.  Modes: "ef" (the method), "no_ef" (the
+    sender's reference is the true previous activation, no error feedback)
+    and "naive" (every step compresses the full activation: both sides
+    restart from zero)."""
     T, C = wl.tokens, wl.channels
-    if side == "gpu":
-        g = GpuBuffer(T, C, bits)
-        zero = torch.zeros(T, C, dtype=torch.bfloat16, device="cuda")
-        g.init(xs[0].clone())
-        for s in range(1, len(xs)):
-            if mode == "naive":
-                g.init(zero)
-            elif mode == "no_ef":
-                cf.cf_state_init(g.d, xs[s - 1].clone().view(torch.int16), g.recon_s, g.err)
-            g.step(xs[s].clone())
-        torch.cuda.synchronize()
-        rr = g.recon_r.cpu().numpy()
-    else:
-        xb = [W.bf16_bits(x) for x in xs]
-        recon_s, _ = oracle.state_init(xb[0])
-        rr = recon_s.copy()
-        zero = np.zeros((T, C), np.uint16)
-        for s in range(1, len(xb)):
-            if mode == "naive":
-                recon_s, _ = oracle.state_init(zero)
-                rr = recon_s.copy()
-            elif mode == "no_ef":
-                recon_s, _ = oracle.state_init(xb[s - 1])
-            codes, scales, _ = oracle.encode(xb[s], recon_s, bits)
-            oracle.decode(codes, scales, rr, bits)
-    xl = f32_of(W.bf16_bits(xs[-1])).astype(np.float64)
-    return float(np.linalg.norm(xl - rr) / np.linalg.norm(xl))
+    g = GpuBuffer(T, C, bits)
+    g.init(xs[0].clone())
+    xb = [W.bf16_bits(x) for x in xs]
+    ro, _ = oracle.state_init(xb[0])
+    rr_o = ro.copy()
+    zero_t = torch.zeros(T, C, dtype=torch.bfloat16, device="cuda")
+    zero_b = np.zeros((T, C), np.uint16)
+    for s in range(1, len(xs)):
+        if mode == "naive":
+            g.init(zero_t)
+            ro, _ = oracle.state_init(zero_b)
+            rr_o = ro.copy()
+        elif mode == "no_ef":
+            cf.cf_state_init(g.d, xs[s - 1].clone().view(torch.int16), g.recon_s, g.err)
+            ro, _ = oracle.state_init(xb[s - 1])
+        g.step(xs[s].clone())
+        v, ora = oracle_step(xb[s], ro, bits)
+        oracle.decode(ora["codes"], ora["scales"], rr_o, bits)
+        gh = g.host()
+        recv = gh.pop("recon_r")
+        compare_step(bits, v, ora, gh)
+        compare_step(bits, v, dict(ora, recon_s=rr_o), dict(gh, recon_s=recv))
+        if mode == "ef":
+            assert np.array_equal(recv.view(np.uint32), gh["recon_s"].view(np.uint32))
+    xl = f32_of(xb[-1]).astype(np.float64)
+    rr_g = g.recon_r.cpu().numpy().astype(np.float64)
+    return (float(np.linalg.norm(xl - rr_g) / np.linalg.norm(xl)),
+            float(np.linalg.norm(xl - rr_o) / np.linalg.norm(xl)))
 
 
 @pytest.mark.parametrize("bits", [1, 2])
@@ -131,9 +139,8 @@ def test_ablations_reproduce_the_pages_ordering(bits):
     xs = W.trajectory(wl, 8, steps=28, device="cuda")
     errs = {}
     for mode in ("ef", "no_ef", "naive"):
-        eg = _final_error(mode, wl, xs, bits, "gpu")
-        eo = _final_error(mode, wl, xs, bits, "oracle")
-        assert abs(eg - eo) <= 1e-3 * max(eo, 1e-6), (mode, eg, eo)
+        eg, eo = _lockstep(mode, wl, xs, bits)
+        assert abs(eg - eo) <= 1e-5 * max(eo, 1e-6), (mode, eg, eo)
         errs[mode] = eg
     # error feedback keeps the reconstruction close; without it error builds
     # up; compressing full activations is worst of all

@@ -16,7 +16,8 @@ import torch.distributed as dist
 import oracle
 from activation_residual_compression_cf_b200 import cf
 from activation_residual_compression_cf_b200 import workloads as W
-from activation_residual_compression_cf_b200.exchange import LowrankShardExchange, ShardExchange
+from activation_residual_compression_cf_b200.exchange import (FusedShardExchange, LowrankShardExchange,
+                                                                ShardExchange)
 from _parity import compare_step, f32_of
 
 pytestmark = pytest.mark.gpu
@@ -156,3 +157,51 @@ def test_lowrank_exchange_loopback_matches_single_calls_and_oracle(nccl_group):
         assert torch.equal(ex.recon_r[0][b], ex.recon_s[b])
         assert torch.equal(resumed.recon_s[b], ex.recon_s[b]) and torch.equal(resumed.err[b], ex.err[b])
         assert torch.equal(resumed.recon_r[0][b], ex.recon_r[0][b])
+
+
+@pytest.mark.parametrize("T,C,bits,B", [(1024, 3072, 2, 6), (200, 1920, 1, 3), (96, 1920, 2, 2)])
+def test_fused_exchange_loopback_equals_the_gather_exchange(nccl_group, T, C, bits, B):
+    """The fused exchange (publishing encode into the slots, waiting decode,
+    counters and acks) in loopback on one GPU: its slots hold exactly the
+    gather exchange's payload, every state equals the gather exchange's bit
+    for bit over five steps (both slots used twice, ack waits from step 3),
+    buffer 0 meets the oracle's bar every step, and a checkpoint resumes on
+    fresh slot memory bit for bit."""
+    wl = W.replace(W.WORKLOADS["flux_sp"], tokens=T, channels=C, bits=bits, buffers=B)
+    trajs = [W.trajectory(wl, b, steps=7, device="cuda") for b in range(B)]
+    gx = ShardExchange(T, C, bits, B, loopback=True)
+    fx = FusedShardExchange(T, C, bits, B, loopback=True)
+    for ex in (gx, fx):
+        ex.warmup([trajs[b][0].clone() for b in range(B)])
+    for t in range(1, 6):
+        xs = [trajs[b][t].clone() for b in range(B)]
+        r0 = fx.recon_s[0].cpu().numpy()
+        gx.step(xs)
+        fx.step(xs)
+        torch.cuda.synchronize()
+        assert gx.codec.status_value() == 0 and fx.codec.status_value() == 0
+        slot = fx.memory.recv[0][t % 2, 0]
+        assert torch.equal(slot, gx.recv), t
+        for b in range(B):
+            for a, g in ((fx.recon_s[b], gx.recon_s[b]), (fx.err[b], gx.err[b]),
+                         (fx.recon_r[0][b], gx.recon_r[0][b]), (fx.recon_r[0][b], fx.recon_s[b])):
+                assert torch.equal(a.view(torch.int32), g.view(torch.int32)), (t, b)
+        assert fx.memory.ready[0].item() == t * B * T and fx.memory.ack[0].item() == t
+        xb = W.bf16_bits(xs[0])
+        v = (f32_of(xb) - r0).astype(np.float32)
+        ro = r0.copy()
+        co, so, eo = oracle.encode(xb, ro, bits)
+        gpu = dict(codes=fx.layout.codes(slot, 0).cpu().numpy().view(np.uint32),
+                   scales=fx.layout.scales(slot, 0).cpu().numpy(),
+                   err=fx.err[0].cpu().numpy(), recon_s=fx.recon_s[0].cpu().numpy())
+        compare_step(bits, v, dict(codes=co, scales=so, err=eo, recon_s=ro), gpu)
+    resumed = FusedShardExchange(T, C, bits, B, loopback=True)
+    resumed.load_state_dict(fx.state_dict())
+    x6 = [trajs[b][6].clone() for b in range(B)]
+    fx.step(x6)
+    resumed.step(x6)
+    torch.cuda.synchronize()
+    assert resumed.codec.status_value() == 0
+    for b in range(B):
+        assert torch.equal(resumed.recon_s[b], fx.recon_s[b]) and torch.equal(resumed.err[b], fx.err[b])
+        assert torch.equal(resumed.recon_r[0][b], fx.recon_r[0][b])

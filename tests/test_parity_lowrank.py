@@ -393,3 +393,41 @@ def test_warm_start_batched_equals_single():
             assert cf.cf_lowrank_status(single[b].ws) == 0
             for k in ("recon_s", "err", "ps", "qs"):
                 assert torch.equal(getattr(batch[b], k), getattr(single[b], k)), (step, b, k)
+
+
+def test_async_status_reads_every_slice_without_waiting():
+    """cf_lowrank_status_async copies each buffer's status word of a batched
+    encode into pinned host memory: a normal buffer (CF_OK), a zero residual
+    (CF_ERR_NUMERIC), a misaligned pointer (CF_ERR_ALIGNMENT) and a warm
+    start without an earlier encode (CF_ERR_INVALID_ARG), in one strided
+    copy; the words agree with the blocking per-slice read."""
+    T, C, r = 256, 192, 8
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r)
+    d = cf.desc(T, C, 0, r, 2)
+    wsb = cf.cf_lowrank_workspace_bytes(d)
+    n = 4
+    xs = W.trajectory(wl, 0, steps=2, device="cuda")
+    gs = [GpuLowrank(T, C, r, 2) for _ in range(n)]
+    for g in gs:
+        g.init(xs[0].clone())
+    om = W.omega(wl, 0, 1, device="cuda")
+    x1 = xs[1].clone().view(torch.int16)
+    x0 = xs[0].clone().view(torch.int16)      # equals the state: zero residual
+    rows = [(x1, gs[0].recon_s, gs[0].err, om, gs[0].pc, gs[0].ps, gs[0].qc, gs[0].qs),
+            (x0, gs[1].recon_s, gs[1].err, om, gs[1].pc, gs[1].ps, gs[1].qc, gs[1].qs),
+            (x1, gs[2].recon_s.data_ptr() + 4, gs[2].err, om, gs[2].pc, gs[2].ps, gs[2].qc, gs[2].qs),
+            (x1, gs[3].recon_s, gs[3].err, None, gs[3].pc, gs[3].ps, gs[3].qc, gs[3].qs)]
+    ws = torch.empty(n * wsb, dtype=torch.uint8, device="cuda")
+    ws.fill_(0x11)   # no earlier encode on these slices: the warm tag is absent
+    host = torch.full((n,), -1, dtype=torch.int32).pin_memory()
+    cf.cf_lowrank_encode_batched(d, n, cf.lowrank_buffer_array(rows, "cuda"), ws)
+    cf.cf_lowrank_status_async(ws, wsb, n, host)
+    ev = torch.cuda.Event()
+    ev.record()
+    ev.synchronize()
+    assert host.tolist() == [0, 6, 2, 1]
+    assert [cf.cf_lowrank_status(ws[b * wsb:]) for b in range(n)] == [0, 6, 2, 1]
+    # pageable host memory is refused: the copy would not be asynchronous
+    with pytest.raises(cf.CFError) as ei:
+        cf.cf_lowrank_status_async(ws, wsb, n, torch.zeros(n, dtype=torch.int32))
+    assert ei.value.status == 1

@@ -274,3 +274,49 @@ def test_single_buffer_beyond_2_pow_31_elements(pipeline, bits):
     finally:
         cf.cf_set_quant_pipeline(0, 1, 0)
         cf.cf_set_quant_pipeline(1, 1, 0)
+
+
+@pytest.mark.parametrize("C", [3072, 3068])
+def test_rows_pipeline_bad_buffers_between_valid_ones(C):
+    """Register-row pipeline (C = 3072 vector path, C = 3068 scalar path)
+    with every other buffer of a batched call invalid (null pointer), on a
+    grid of one CTA per SM, so each CTA meets valid and skipped rows in turn.
+    The valid buffers must equal an all-valid run bit for bit and the oracle
+    within the parity bar; a skipped row must not shift the scale slots that
+    the next valid row shares with the previous one."""
+    n, T = 24, 16
+    wl = W.replace(W.WORKLOADS["flux_sp"], tokens=T, channels=C, buffers=n)
+    xs = torch.stack([W.trajectory(wl, b, steps=2, device="cuda") for b in range(n)], 1)
+    d = cf.desc(T, C, wl.bits)
+    x16 = xs[1].view(torch.int16)
+    runs = []
+    try:
+        cf.cf_set_quant_pipeline(0, 0, 0)
+        G = (C + 7) // 8
+        cf.cf_set_launch_override(0, 2, ((G + 1) // 2 + 31) // 32 * 32, 1)   # one CTA per SM
+        for skip in (False, True):
+            st = _batched_state(wl, n)
+            for b in range(n):
+                cf.cf_state_init(d, xs[0, b].view(torch.int16), st["recon_s"][b], st["err"][b])
+            sets = [(x16[b], st["recon_s"][b], st["err"][b], st["codes"][b], st["scales"][b])
+                    for b in range(n)]
+            if skip:
+                sets = [s if b % 2 == 0 else (0,) + s[1:] for b, s in enumerate(sets)]
+            status = torch.zeros(1, dtype=torch.int32, device="cuda")
+            cf.cf_encode_batched(d, n, cf.enc_buffer_array(sets, "cuda"), status)
+            torch.cuda.synchronize()
+            assert int(status.item()) == (1 if skip else 0)
+            runs.append(st)
+    finally:
+        cf.cf_set_quant_pipeline(0, 1, 0)
+        cf.cf_set_launch_override(0, 0, 0, 0)
+    full, part = runs
+    for b in range(0, n, 2):
+        for k in ("codes", "scales", "err", "recon_s"):
+            assert torch.equal(full[k][b].view(torch.int32), part[k][b].view(torch.int32)), (b, k)
+        r0, _ = oracle.state_init(W.bf16_bits(xs[0, b]))
+        v, ora = oracle_step(W.bf16_bits(xs[1, b]), r0, wl.bits)
+        gh = dict(codes=part["codes"][b].cpu().numpy().view(np.uint32),
+                  scales=part["scales"][b].cpu().numpy(), err=part["err"][b].cpu().numpy(),
+                  recon_s=part["recon_s"][b].cpu().numpy())
+        compare_step(wl.bits, v, ora, gh)
