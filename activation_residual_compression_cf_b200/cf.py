@@ -35,7 +35,8 @@ EXPORTS = ("cf_status_string", "cf_abi_version", "cf_codes_words_per_row",
 # Every symbol include/cf_diag.h declares: tuning knobs, measurement hooks
 # and the bounded-wait self-test (process-wide state, not product calls).
 DIAG_EXPORTS = ("cf_set_lowrank_engine", "cf_set_quant_pipeline", "cf_set_launch_override",
-                "cf_set_quant_unit", "cf_lowrank_set_apply_events", "cf_diag_bounded_wait",
+                "cf_set_quant_unit", "cf_set_lowrank_group", "cf_lowrank_set_apply_events",
+                "cf_diag_bounded_wait",
                 "cf_debug_bounds_checked", "cf_debug_bounds_take", "cf_diag_bounds_selftest")
 
 
@@ -142,6 +143,7 @@ def lib():
             "cf_diag_bounded_wait": ([i32, vp, vp], ctypes.c_int),
             "cf_set_quant_pipeline": ([i32, i32, i32], ctypes.c_int),
             "cf_set_quant_unit": ([i32, i32], ctypes.c_int),
+            "cf_set_lowrank_group": ([i32], ctypes.c_int),
             "cf_debug_bounds_checked": ([], i32),
             "cf_debug_bounds_take": ([], i32),
             "cf_diag_bounds_selftest": ([vp, i32, vp], ctypes.c_int),
@@ -335,6 +337,10 @@ def bounds_file_tag(name: str) -> int:
     for ch in os.path.basename(name).encode():
         h = ((h ^ ch) * 16777619) & 0xFFFFFFFF
     return (h ^ (h >> 15)) & 0x7FFF
+
+
+def cf_set_lowrank_group(buffers: int):
+    _chk(lib().cf_set_lowrank_group(buffers), "cf_set_lowrank_group")
 
 
 def cf_set_quant_unit(kernel: int, channels: int):

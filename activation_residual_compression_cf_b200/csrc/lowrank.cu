@@ -130,6 +130,7 @@ int sm_count() {
 }
 
 std::atomic<int> g_engine{0};  // 0 = tensor cores (tcgen05), 1 = CUDA cores
+std::atomic<int> g_group{0};   // batched encode: buffers per pass of every stage (0 = all)
 
 // Events recorded around the apply launch (measurement hook), per direction.
 std::atomic<void *> g_apply_ev[2][2] = {};
@@ -349,8 +350,25 @@ cf_status apply(bool sender, const LrBatch &B, const Layout &L, int n, cudaStrea
     return e0 != CF_OK ? e0 : e1;
 }
 
-// The whole sender for n buffers (n = 1 for the single-buffer call).
+cf_status encode_group(const cf_desc *d, const Layout &L, int n, const LrBatch &B, cudaStream_t st);
+
+// The whole sender for n buffers (n = 1 for the single-buffer call): every
+// stage launched once for all n, or, with a group size g set, for g buffers
+// at a time (the buffers of a group then share the L2 between the passes).
 cf_status encode_impl(const cf_desc *d, const Layout &L, int n, const LrBatch &B, cudaStream_t st) {
+    const int g = g_group.load();
+    if (g <= 0 || g >= n || !B.enc) return encode_group(d, L, n, B, st);
+    for (int b0 = 0; b0 < n; b0 += g) {
+        LrBatch Bg = B;
+        Bg.enc = B.enc + b0;
+        Bg.ws = B.ws + (int64_t)b0 * B.ws_stride;
+        const cf_status s = encode_group(d, L, n - b0 < g ? n - b0 : g, Bg, st);
+        if (s != CF_OK) return s;
+    }
+    return CF_OK;
+}
+
+cf_status encode_group(const cf_desc *d, const Layout &L, int n, const LrBatch &B, cudaStream_t st) {
     const int nb = (L.r + 1) / 2;
     const bool fused = g_engine.load() == 0;
     cf::lr_prep_kernel<<<(unsigned)n, 128, 0, st>>>(B, L);
@@ -511,6 +529,12 @@ cf_status cf_lowrank_decode_batched(const cf_desc *d, int32_t n, const cf_lowran
     B.dec = bufs_dev;
     B.dec_status = status_dev;
     return apply(false, B, L, n, (cudaStream_t)stream);
+}
+
+cf_status cf_set_lowrank_group(int32_t buffers) {
+    if (buffers < 0 || buffers > 65535) return CF_ERR_INVALID_ARG;
+    g_group.store(buffers);
+    return CF_OK;
 }
 
 cf_status cf_set_lowrank_engine(int32_t engine) {

@@ -77,6 +77,9 @@ def parse():
                     help="quantize mode: the sequence-parallel exchange (encode into one payload, "
                          "all-gather over the process group, decode every peer's shard; one GPU "
                          "alone decodes its own payload)")
+    ap.add_argument("--lowrank-group", type=int, default=-1,
+                    help="low-rank: buffers per pass of the batched encode (0 = all; -1 = the "
+                         "library default)")
     ap.add_argument("--warm", action="store_true",
                     help="low-rank: warm start every encode after the first from the previous Q")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -606,6 +609,8 @@ def run_lowrank(args, world, rank, local):
     wl = lowrank_workload(args)
     n, T, C, r, it = wl.buffers, wl.tokens, wl.channels, wl.rank, wl.iters
     d = cf.desc(T, C, 0, r, it)
+    if args.lowrank_group >= 0:
+        cf.cf_set_lowrank_group(args.lowrank_group)
     step_bytes = n * T * C * 2
     S = max(2, min(wl.steps, int(30e9 // step_bytes)))
     if args.gen_steps:

@@ -41,6 +41,13 @@ cf_status cf_diag_bounded_wait(int32_t polls, int32_t *out_dev, void *stream);
  * other value. */
 cf_status cf_set_lowrank_engine(int32_t engine);
 
+/* Buffers per pass of a batched low-rank encode in this process: 0 (the
+ * default) launches every stage once for all buffers of the call; g > 0
+ * runs the whole sender for g buffers at a time, so a group's bf16 residual
+ * copies can stay in L2 between the four projection passes.  Results are
+ * bit-identical either way.  Returns CF_ERR_INVALID_ARG outside 0..65535. */
+cf_status cf_set_lowrank_group(int32_t buffers);
+
 /* Measurement hook (no counterpart in the paper): CUDA events (cudaEvent_t,
  * passed as void*) that the low-rank calls record around their apply kernel
  * -- the kernel that forms D and updates the state -- so a caller can time

@@ -431,3 +431,37 @@ def test_async_status_reads_every_slice_without_waiting():
     with pytest.raises(cf.CFError) as ei:
         cf.cf_lowrank_status_async(ws, wsb, n, torch.zeros(n, dtype=torch.int32))
     assert ei.value.status == 1
+
+
+@pytest.mark.parametrize("group", [1, 3])
+def test_grouped_batched_encode_is_bit_identical(group):
+    """A batched encode run g buffers at a time (cf_set_lowrank_group)
+    computes exactly what the all-buffers launches do."""
+    T, C, r, n = 640, 384, 16, 7
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r)
+    d = cf.desc(T, C, 0, r, 2)
+    wsb = cf.cf_lowrank_workspace_bytes(d)
+    xs = [W.trajectory(wl, b, steps=2, device="cuda") for b in range(n)]
+    oms = [W.omega(wl, b, 1, device="cuda") for b in range(n)]
+    outs = []
+    try:
+        for g in (0, group):
+            cf.cf_set_lowrank_group(g)
+            gs = [GpuLowrank(T, C, r, 2) for _ in range(n)]
+            for b in range(n):
+                gs[b].init(xs[b][0].clone())
+            ws = torch.empty(n * wsb, dtype=torch.uint8, device="cuda")
+            enc = cf.lowrank_buffer_array([(xs[b][1].view(torch.int16), gs[b].recon_s, gs[b].err, oms[b],
+                                            gs[b].pc, gs[b].ps, gs[b].qc, gs[b].qs) for b in range(n)],
+                                          "cuda")
+            cf.cf_lowrank_encode_batched(d, n, enc, ws)
+            torch.cuda.synchronize()
+            assert [cf.cf_lowrank_status(ws[b * wsb:]) for b in range(n)] == [0] * n
+            outs.append(gs)
+    finally:
+        cf.cf_set_lowrank_group(0)
+    nb = (r + 1) // 2
+    for a, b in zip(*outs):
+        for k in ("recon_s", "err", "ps", "qs"):
+            assert torch.equal(getattr(a, k), getattr(b, k)), k
+        assert torch.equal(a.pc[:T * nb], b.pc[:T * nb]) and torch.equal(a.qc[:C * nb], b.qc[:C * nb])
