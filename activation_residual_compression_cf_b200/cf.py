@@ -36,7 +36,7 @@ EXPORTS = ("cf_status_string", "cf_abi_version", "cf_codes_words_per_row",
 # and the bounded-wait self-test (process-wide state, not product calls).
 DIAG_EXPORTS = ("cf_set_lowrank_engine", "cf_set_quant_pipeline", "cf_set_launch_override",
                 "cf_set_quant_unit", "cf_set_lowrank_group", "cf_lowrank_set_apply_events",
-                "cf_diag_bounded_wait",
+                "cf_diag_bounded_wait", "cf_diag_stream_mix",
                 "cf_debug_bounds_checked", "cf_debug_bounds_take", "cf_diag_bounds_selftest")
 
 
@@ -144,6 +144,7 @@ def lib():
             "cf_set_quant_pipeline": ([i32, i32, i32], ctypes.c_int),
             "cf_set_quant_unit": ([i32, i32], ctypes.c_int),
             "cf_set_lowrank_group": ([i32], ctypes.c_int),
+            "cf_diag_stream_mix": ([vp, vp, vp, i64, vp], ctypes.c_int),
             "cf_debug_bounds_checked": ([], i32),
             "cf_debug_bounds_take": ([], i32),
             "cf_diag_bounds_selftest": ([vp, i32, vp], ctypes.c_int),
@@ -337,6 +338,11 @@ def bounds_file_tag(name: str) -> int:
     for ch in os.path.basename(name).encode():
         h = ((h ^ ch) * 16777619) & 0xFFFFFFFF
     return (h ^ (h >> 15)) & 0x7FFF
+
+
+def cf_diag_stream_mix(x, r, a, stream=None):
+    """Streaming pass with the encode's byte mix over every element of x."""
+    _chk(lib().cf_diag_stream_mix(_p(x), _p(r), _p(a), x.numel(), _s(stream)), "cf_diag_stream_mix")
 
 
 def cf_set_lowrank_group(buffers: int):

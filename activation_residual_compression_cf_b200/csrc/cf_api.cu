@@ -203,11 +203,20 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
     const size_t smem = (size_t)stages * slot + 16 * (size_t)stages;
     const int threads = 32 + s.threads;
     void (*k)(Src, int64_t, int64_t, int64_t, int32_t *, int);
-    // a thread's GPT groups of 8 channels as 8 / K * GPT units of K
-    if constexpr (ENC)
-        k = cf::tma::encode_tma_kernel<BITS, K, 8 / K * GPT, Src>;
-    else
-        k = cf::tma::decode_tma_kernel<BITS, K, 8 / K * GPT, Src>;
+    // a thread's GPT groups of 8 channels as 8 / K * GPT units of K; the
+    // plain 8-channel launches take the dedicated kernels (faster schedule)
+    constexpr bool kPlain = K == 8 && !Src::kPublish && !Src::kWait;
+    if constexpr (ENC) {
+        if constexpr (kPlain)
+            k = cf::tma::encode_tma_kernel<BITS, GPT, Src>;
+        else
+            k = cf::tma::encode_tma_unit_kernel<BITS, K, 8 / K * GPT, Src>;
+    } else {
+        if constexpr (kPlain)
+            k = cf::tma::decode_tma_kernel<BITS, GPT, Src>;
+        else
+            k = cf::tma::decode_tma_unit_kernel<BITS, K, 8 / K * GPT, Src>;
+    }
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return CF_ERR_CUDA;
     int occ = 0;

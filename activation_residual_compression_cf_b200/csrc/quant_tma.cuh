@@ -102,13 +102,315 @@ __device__ __forceinline__ void store_unit(float *row, int u, const float *o) {
 // encode: x row (2C), x_prev row (2C), err row (4C).
 // Decode slot: codes row (4W bytes, padded to 16) then recon row (4C bytes).
 
+// The two kernels below are the TMA pipeline with units of 8 channels and
+// plain pointer sources, as the default launches use them: the same
+// arithmetic, pipeline and results as the general kernels further down
+// (encode_tma_unit_kernel, decode_tma_unit_kernel), written without their
+// unit-width and exchange options.  Measured on B200 in the encode ->
+// decode sequence, this form runs 3 % (2-bit decode at C = 1920) to 6 %
+// (1-bit encode at C = 3072) faster than the general kernel instantiated
+// for the same shape: same instruction count, but the general form's
+// schedule stalls more and, for the 1-bit encode, spills a register.
+
+template <int BITS, int GPT, class Src>
+__global__ void __launch_bounds__(512)
+encode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, int stages) {
+    constexpr int GPW = 4 / BITS;
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ double sh_sum[2][32];
+    __shared__ float sh_max[2][32];
+    __shared__ int abort_row[2];  // set before the row's barrier, read after it
+    const int64_t G = C >> 3;  // C % 8 == 0 on this path
+    const int64_t W = (C * BITS + 31) >> 5;
+    const uint32_t slot = (uint32_t)((Src::kDelta ? 8 : 6) * C);
+    const uint32_t base = saddr(smem);
+    const uint32_t bars = base + (uint32_t)stages * slot;
+    const int tid = threadIdx.x;
+    const int nc = blockDim.x - 32;  // consumer threads
+    if (tid == 0) {
+        abort_row[0] = abort_row[1] = 0;
+        for (int s = 0; s < stages; ++s) {
+            bar_init(bars + 8u * s, 1);                    // full: producer arrival + tx
+            bar_init(bars + 8u * (stages + s), (uint32_t)(nc / 32));  // empty: one per consumer warp
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (tid < 32) {
+        if (tid != 0) return;
+        int i = 0;
+        for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+            const int64_t b = row / T, t = row - b * T;
+            const EncPtrs p = src.get(b);
+            if (Src::kChecked && enc_ptr_status<Src::kDelta>(p) != CF_OK) continue;
+            const int s = i % stages;
+            const uint32_t ph = (uint32_t)(i / stages) & 1u;
+            if (!bar_wait(bars + 8u * (stages + s), ph ^ 1u)) {
+                // consumers stopped releasing slots; they time out on their
+                // own waits and leave together
+                if (status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+                return;
+            }
+            const uint32_t dst = base + (uint32_t)s * slot;
+            if (!CF_IN(t < T && b * T + t == row && s < stages)) continue;
+            bar_expect(bars + 8u * s, slot);
+            bulk_g2s(dst, p.x + t * C, (uint32_t)(2 * C), bars + 8u * s);
+            if (Src::kDelta) {
+                bulk_g2s(dst + (uint32_t)(2 * C), p.xprev + t * C, (uint32_t)(2 * C), bars + 8u * s);
+                bulk_g2s(dst + (uint32_t)(4 * C), p.err + t * C, (uint32_t)(4 * C), bars + 8u * s);
+            } else {
+                bulk_g2s(dst + (uint32_t)(2 * C), p.recon + t * C, (uint32_t)(4 * C), bars + 8u * s);
+            }
+            ++i;
+        }
+        return;
+    }
+
+    const int ct = tid - 32;  // consumer thread index
+    const int lane = ct & 31, warp = ct >> 5, nw = nc >> 5;
+    int i = 0, par = 0;
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+        const int64_t b = row / T, t = row - b * T;
+        const EncPtrs p = src.get(b);
+        if (Src::kChecked) {
+            const int st = enc_ptr_status<Src::kDelta>(p);
+            if (st != CF_OK) {
+                if (ct == 0) report(status, st);
+                continue;
+            }
+        }
+        const int s = i % stages;
+        const uint32_t ph = (uint32_t)(i / stages) & 1u;
+        bool ok = true;
+        if (lane == 0) ok = bar_wait(bars + 8u * s, ph);
+        ok = __shfl_sync(kFullMask, ok ? 1 : 0, 0) != 0;
+        if (!ok && lane == 0) abort_row[par] = 1;  // acted on after the barrier
+        const uint8_t *sx = smem + (size_t)s * slot;
+        const uint8_t *sp = sx + 2 * C;   // x_prev row (delta-state sender)
+        // recon (standard) or the old err (delta-state)
+        const float *sr = reinterpret_cast<const float *>(sx + (Src::kDelta ? 4 : 2) * C);
+        float *rr = Src::kDelta ? nullptr : p.recon + t * C;
+        float *er = p.err + t * C;
+        uint32_t *cw = p.codes + t * W;
+
+        float r[GPT][8], v[GPT][8];
+#pragma unroll
+        for (int j = 0; j < GPT; ++j) {
+            const int64_t g = (int64_t)j * nc + ct;
+            if (ok && g < G && CF_IN(8 * g + 8 <= C)) {
+                const uint4 xw = *reinterpret_cast<const uint4 *>(sx + 16 * g);
+                const uint4 pw = Src::kDelta ? *reinterpret_cast<const uint4 *>(sp + 16 * g)
+                                             : make_uint4(0, 0, 0, 0);
+                const float4 a = *reinterpret_cast<const float4 *>(sr + 8 * g);
+                const float4 c = *reinterpret_cast<const float4 *>(sr + 8 * g + 4);
+                r[j][0] = a.x; r[j][1] = a.y; r[j][2] = a.z; r[j][3] = a.w;
+                r[j][4] = c.x; r[j][5] = c.y; r[j][6] = c.z; r[j][7] = c.w;
+                residual8<Src::kDelta>(xw, pw, r[j], v[j]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) r[j][e] = v[j][e] = 0.0f;
+            }
+        }
+        // the slot is no longer read: release it to the producer.  The reads
+        // above are generic-proxy accesses and the producer's next bulk copy
+        // into this slot is an async-proxy write: the proxy fence orders them
+        // (without it a late read can see the next row's bytes).
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) bar_arrive(bars + 8u * (stages + s));
+        ++i;
+
+        float scale;
+        if (BITS == 1) {
+            double acc = 0.0;
+#pragma unroll
+            for (int j = 0; j < GPT; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc += (double)fabsf(v[j][e]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFullMask, acc, o);
+            if (lane == 0) sh_sum[par][warp] = acc;
+            consumer_sync(nc);
+            if (*(volatile int *)&abort_row[par]) {
+                if (ct == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+                return;  // every consumer warp sees the same flag here
+            }
+            double tot = 0.0;
+            for (int w = 0; w < nw; ++w) tot += sh_sum[par][w];
+            scale = __fdiv_rn(__double2float_rn(tot), (float)C);
+        } else {
+            float m = 0.0f;
+#pragma unroll
+            for (int j = 0; j < GPT; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[j][e]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+            if (lane == 0) sh_max[par][warp] = m;
+            consumer_sync(nc);
+            if (*(volatile int *)&abort_row[par]) {
+                if (ct == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+                return;
+            }
+            float tot = 0.0f;
+            for (int w = 0; w < nw; ++w) tot = fmaxf(tot, sh_max[par][w]);
+            scale = tot;
+        }
+        par ^= 1;
+        const float half = __fmul_rn(0.5f, scale);
+#pragma unroll
+        for (int j = 0; j < GPT; ++j) {
+            const int64_t g = (int64_t)j * nc + ct;
+            uint32_t field = 0;
+            float eo[8], ro[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                uint32_t code = quantize<BITS>(v[j][e], half);
+                code = (g < G) ? code : 0u;
+                field |= code << (e * BITS);
+                const float d = dequantize<BITS>(code, scale);
+                eo[e] = __fsub_rn(v[j][e], d);
+                ro[e] = __fadd_rn(r[j][e], d);
+            }
+            uint32_t word = field << ((lane % GPW) * 8 * BITS);
+#pragma unroll
+            for (int o = 1; o < GPW; o <<= 1) word |= __shfl_xor_sync(kFullMask, word, o);
+            if (g < G && CF_IN(8 * g + 8 <= C && t < T && g / GPW < W)) {
+                st_stream_v4(er + 8 * g, make_float4(eo[0], eo[1], eo[2], eo[3]));
+                st_stream_v4(er + 8 * g + 4, make_float4(eo[4], eo[5], eo[6], eo[7]));
+                if (!Src::kDelta) {
+                    st_state_v4(rr + 8 * g, make_float4(ro[0], ro[1], ro[2], ro[3]));
+                    st_state_v4(rr + 8 * g + 4, make_float4(ro[4], ro[5], ro[6], ro[7]));
+                }
+                if ((lane % GPW) == 0) cw[g / GPW] = word;
+            }
+        }
+        if (ct == 0 && CF_IN(t < T)) p.scales[t] = scale;
+    }
+}
+
+template <int BITS, int GPT, class Src>
+__global__ void __launch_bounds__(512)
+decode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, int stages) {
+    constexpr uint32_t MASK = (1u << BITS) - 1u;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int64_t G = C >> 3;
+    const int64_t W = (C * BITS + 31) >> 5;
+    const uint32_t cbytes = (uint32_t)(W * 4);
+    const uint32_t slot = cbytes + (uint32_t)(4 * C);
+    const uint32_t base = saddr(smem);
+    const uint32_t bars = base + (uint32_t)stages * slot;
+    const int tid = threadIdx.x;
+    const int nc = blockDim.x - 32;
+    if (tid == 0) {
+        for (int s = 0; s < stages; ++s) {
+            bar_init(bars + 8u * s, 1);
+            bar_init(bars + 8u * (stages + s), (uint32_t)(nc / 32));
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (tid < 32) {
+        if (tid != 0) return;
+        int i = 0;
+        for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+            const int64_t b = row / T, t = row - b * T;
+            const DecPtrs p = src.get(b);
+            if (Src::kChecked && dec_ptr_status<Src::kEmit>(p) != CF_OK) continue;
+            const int s = i % stages;
+            const uint32_t ph = (uint32_t)(i / stages) & 1u;
+            if (!bar_wait(bars + 8u * (stages + s), ph ^ 1u)) {
+                if (status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+                return;
+            }
+            const uint32_t dst = base + (uint32_t)s * slot;
+            if (!CF_IN(t < T && b * T + t == row && s < stages && (W & 3) == 0)) continue;
+            // W % 4 == 0 on this path (host check): codes rows are 16-byte
+            // aligned multiples of 16 bytes
+            bar_expect(bars + 8u * s, cbytes + (uint32_t)(4 * C));
+            bulk_g2s(dst, p.codes + t * W, cbytes, bars + 8u * s);
+            bulk_g2s(dst + cbytes, p.recon + t * C, (uint32_t)(4 * C), bars + 8u * s);
+            ++i;
+        }
+        return;
+    }
+
+    const int ct = tid - 32;
+    const int lane = ct & 31;
+    int i = 0;
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+        const int64_t b = row / T, t = row - b * T;
+        const DecPtrs p = src.get(b);
+        if (Src::kChecked) {
+            const int st = dec_ptr_status<Src::kEmit>(p);
+            if (st != CF_OK) {
+                if (ct == 0) report(status, st);
+                continue;
+            }
+        }
+        const int s = i % stages;
+        const uint32_t ph = (uint32_t)(i / stages) & 1u;
+        bool ok = true;
+        if (lane == 0) ok = bar_wait(bars + 8u * s, ph);
+        ok = __shfl_sync(kFullMask, ok ? 1 : 0, 0) != 0;
+        if (!ok) {  // decode warps are independent: each leaves on its own
+            if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+            return;
+        }
+        const uint8_t *sc = smem + (size_t)s * slot;
+        const float *sr = reinterpret_cast<const float *>(sc + cbytes);
+        const float scale = __ldg(p.scales + t);
+        float *rr = p.recon + t * C;
+        uint32_t field[GPT];
+        float r[GPT][8];
+#pragma unroll
+        for (int j = 0; j < GPT; ++j) {
+            const int64_t g = (int64_t)j * nc + ct;
+            if (g < G && CF_IN(8 * g + 8 <= C && (g + 1) * BITS <= (int64_t)cbytes)) {
+                const uint32_t off = (uint32_t)(g * BITS);  // byte offset of the group's field
+                field[j] = BITS == 1 ? (uint32_t)sc[off]
+                                     : (uint32_t)*reinterpret_cast<const uint16_t *>(sc + off);
+                const float4 a = *reinterpret_cast<const float4 *>(sr + 8 * g);
+                const float4 c = *reinterpret_cast<const float4 *>(sr + 8 * g + 4);
+                r[j][0] = a.x; r[j][1] = a.y; r[j][2] = a.z; r[j][3] = a.w;
+                r[j][4] = c.x; r[j][5] = c.y; r[j][6] = c.z; r[j][7] = c.w;
+            } else {
+                field[j] = 0u;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) r[j][e] = 0.0f;
+            }
+        }
+        // release the slot; proxy fence as in the encode kernel
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) bar_arrive(bars + 8u * (stages + s));
+        ++i;
+#pragma unroll
+        for (int j = 0; j < GPT; ++j) {
+            const int64_t g = (int64_t)j * nc + ct;
+            if (g >= G || !CF_IN(8 * g + 8 <= C && t < T)) continue;
+            float ro[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t code = (field[j] >> (e * BITS)) & MASK;
+                ro[e] = __fadd_rn(r[j][e], dequantize<BITS>(code, scale));
+            }
+            st_state_v4(rr + 8 * g, make_float4(ro[0], ro[1], ro[2], ro[3]));
+            st_state_v4(rr + 8 * g + 4, make_float4(ro[4], ro[5], ro[6], ro[7]));
+            if (Src::kEmit) *reinterpret_cast<uint4 *>(p.out + t * C + 8 * g) = pack_bf16x8(ro);
+        }
+    }
+}
+
 // Code words of the longest row (C = 16384 at 2 bits): the publishing
 // encode stages one row of them in shared memory.
 constexpr int kMaxCodeWords = 1024;
 
 template <int BITS, int K, int UPT, class Src>
 __global__ void __launch_bounds__(512)
-encode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, int stages) {
+encode_tma_unit_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, int stages) {
     static_assert(K == 4 || K == 8, "units of 4 or 8 channels");
     constexpr int UPW = 32 / (K * BITS);  // units per 32-bit code word
     extern __shared__ __align__(16) uint8_t smem[];
@@ -301,7 +603,7 @@ encode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
 
 template <int BITS, int K, int UPT, class Src>
 __global__ void __launch_bounds__(512)
-decode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, int stages) {
+decode_tma_unit_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, int stages) {
     static_assert(K == 4 || K == 8, "units of 4 or 8 channels");
     constexpr uint32_t MASK = (1u << BITS) - 1u;
     extern __shared__ __align__(16) uint8_t smem[];

@@ -216,6 +216,19 @@ def recorded_traffic(kernel: str, workload: str, files=QUANT_SOURCES):
     return d.get("dram_bytes_per_launch")
 
 
+def recorded_tensor_pipe():
+    """Tensor-pipe activity of the low-rank kernels from the committed ncu
+    summary (profiles/tensor_pipe.json), if it was taken on the current
+    low-rank sources; else None."""
+    p = os.path.join(ROOT, "profiles", "tensor_pipe.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_hash") != kernel_source_hash(LOWRANK_APPLY_SOURCES):
+        return None
+    return {"kernels": d["kernels"], "metric": d["metric"], "capture": d["capture"]}
+
+
 # ------------------------------------------------------------ CPU oracle leg
 
 def oracle_sample(wl, seconds, max_buffer_steps=10**9):
@@ -475,6 +488,27 @@ def run_ours(args, world, rank, local):
                "ms_per_step": round(e2e["ms"] / e_steps, 4),
                "overlap": f"{e2e['chunks']} chunks on copy-in / compute / copy-out streams"}
 
+    # The HBM ceiling of the encode's byte mix: a plain streaming pass over
+    # the same slab (x in, recon in/out, err out), timed the same way.  It
+    # overwrites the states, which nothing reads after this point.
+    mix = None
+    if not args.delta and not args.emit:
+        xs1 = X16[1].reshape(-1)
+        for _ in range(3):
+            cf.cf_diag_stream_mix(xs1, recon_s.view(-1), err.view(-1), stream)
+        mev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(20)]
+        for m0, m1 in mev:
+            m0.record(stream)
+            cf.cf_diag_stream_mix(xs1, recon_s.view(-1), err.view(-1), stream)
+            m1.record(stream)
+        torch.cuda.synchronize()
+        mix_ms = statistics.mean(m0.elapsed_time(m1) for m0, m1 in mev)
+        mix_gbs = n * T * C * 14 / (mix_ms / 1e3) / 1e9
+        mix = {"kernel": "cf_diag_stream_mix (6 B read, 8 B written per element, no per-row work)",
+               "achieved": round(mix_gbs, 1), "frac_of_peak": round(mix_gbs / peaks()[0], 4),
+               "encode_frac_of_mix": round(enc_gbs / mix_gbs, 4)}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, done, tw = oracle_sample(wl, args.cpu_seconds)
@@ -504,7 +538,8 @@ def run_ours(args, world, rank, local):
                      + (", delta-state sender" if args.delta else "")
                    + (", emitting decode" if args.emit else ""),
                      "peak_kind": peak_kind,
-                     "algorithmic_bytes_per_launch": enc_bytes, "avg_launch_ms": round(enc_ms, 4)},
+                     "algorithmic_bytes_per_launch": enc_bytes, "avg_launch_ms": round(enc_ms, 4),
+                     "mix_ceiling": mix},
         "decode": {"achieved": round(dec_gbs, 1), "frac": round(dec_gbs / peak, 4),
                    "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_ms": round(dec_ms, 4)},
         "cpu_baseline": cpu,
@@ -748,6 +783,7 @@ def run_lowrank(args, world, rank, local):
                        "encode_frac_of_14B_per_elem": round(
                            enc_bytes / (enc_ms / 1e3) / 1e9 / peak, 4)},
         "lowrank_status": status,
+        "tensor_pipe": recorded_tensor_pipe(),
         "payload_ratio": round(2 * T * C / cf.cf_payload_bytes(d), 2),
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
