@@ -34,7 +34,7 @@ __global__ void diag_wait_kernel(uint32_t polls, int32_t *out) {
     out[1] = cf::mbar_wait(never, 0, polls) ? (int32_t)CF_OK : (int32_t)CF_ERR_TIMEOUT;
 }
 
-// The memory ceiling of the encode's byte mix: a plain streaming pass that
+// A reference for the encode's byte mix: a plain streaming pass that
 // reads a bf16 array x and an fp32 array r and writes two fp32 arrays,
 // a = (float)x - r and r = (float)x + r (6 bytes read, 8 written per
 // element, as the encode reads x and recon and writes err and recon).

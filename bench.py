@@ -488,9 +488,12 @@ def run_ours(args, world, rank, local):
                "ms_per_step": round(e2e["ms"] / e_steps, 4),
                "overlap": f"{e2e['chunks']} chunks on copy-in / compute / copy-out streams"}
 
-    # The HBM ceiling of the encode's byte mix: a plain streaming pass over
-    # the same slab (x in, recon in/out, err out), timed the same way.  It
-    # overwrites the states, which nothing reads after this point.
+    # A reference for the encode's byte mix: a plain streaming pass over the
+    # same slab (x in, recon in/out, err out: 6 B read, 8 B written per
+    # element) with none of the per-row work, timed the same way.  Writes
+    # dominate the mix, and HBM serves it slower than a copy's even split;
+    # the encode is compared with this pass as well as with the copy peak.
+    # It overwrites the states, which nothing reads after this point.
     mix = None
     if not args.delta and not args.emit:
         xs1 = X16[1].reshape(-1)
@@ -507,7 +510,7 @@ def run_ours(args, world, rank, local):
         mix_gbs = n * T * C * 14 / (mix_ms / 1e3) / 1e9
         mix = {"kernel": "cf_diag_stream_mix (6 B read, 8 B written per element, no per-row work)",
                "achieved": round(mix_gbs, 1), "frac_of_peak": round(mix_gbs / peaks()[0], 4),
-               "encode_frac_of_mix": round(enc_gbs / mix_gbs, 4)}
+               "encode_over_reference": round(enc_gbs / mix_gbs, 4)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -539,7 +542,7 @@ def run_ours(args, world, rank, local):
                    + (", emitting decode" if args.emit else ""),
                      "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": enc_bytes, "avg_launch_ms": round(enc_ms, 4),
-                     "mix_ceiling": mix},
+                     "mix_reference": mix},
         "decode": {"achieved": round(dec_gbs, 1), "frac": round(dec_gbs / peak, 4),
                    "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_ms": round(dec_ms, 4)},
         "cpu_baseline": cpu,

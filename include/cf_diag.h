@@ -73,13 +73,13 @@ cf_status cf_lowrank_set_apply_events(void *enc_start, void *enc_stop, void *dec
  * Returns CF_ERR_INVALID_ARG for out-of-range values. */
 cf_status cf_set_quant_pipeline(int32_t kernel, int32_t pipeline, int32_t stages);
 
-/* The memory ceiling of the encode's byte mix (no counterpart in the
- * paper): one streaming pass over n elements (n % 8 == 0) that reads x (bf16
- * [n]) and r (fp32 [n]) and writes a = (float)x - r and r = (float)x + r
- * (fp32 [n] each), i.e. the 6 bytes read and 8 written per element of the
- * quantize encode with none of its per-row work.  Timing it next to the
- * encode separates what the kernel leaves on the table from what the
- * read/write mix of HBM costs.  Device pointers, 16-byte aligned,
+/* A reference for the encode's byte mix (no counterpart in the paper): one
+ * streaming pass over n elements (n % 8 == 0) that reads x (bf16 [n]) and r
+ * (fp32 [n]) and writes a = (float)x - r and r = (float)x + r (fp32 [n]
+ * each), i.e. the 6 bytes read and 8 written per element of the quantize
+ * encode with none of its per-row work.  Timed next to the encode, it shows
+ * what HBM gives a plain streaming kernel with that read/write mix, which
+ * is less than it gives a copy's even split.  Device pointers, 16-byte aligned,
  * non-overlapping; overwrites r and a.  n < 0 or n % 8 != 0:
  * CF_ERR_INVALID_ARG. */
 cf_status cf_diag_stream_mix(const uint16_t *x, float *r, float *a, int64_t n, void *stream);

@@ -125,7 +125,6 @@ def test_publish_then_wait_in_stream_order_over_steps():
     stream, with two slots used in turn and the ack target of each step
     (e - 2): the receiver tracks the sender bit for bit."""
     T, C, bits, n = 48, 1920, 2, 3
-    xs_all = None
     wl = W.replace(W.WORKLOADS["cogvideox"], tokens=T, buffers=n)
     xs_all = torch.stack([W.trajectory(wl, b, steps=5, device="cuda") for b in range(n)], 1)
     f32 = dict(dtype=torch.float32, device="cuda")
