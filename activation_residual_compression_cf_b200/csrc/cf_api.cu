@@ -209,6 +209,8 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
     if constexpr (ENC) {
         if constexpr (kPlain)
             k = cf::tma::encode_tma_kernel<BITS, GPT, Src>;
+        else if constexpr (Src::kPublish)
+            k = cf::tma::encode_tma_publish_kernel<BITS, K, 8 / K * GPT, Src>;
         else
             k = cf::tma::encode_tma_unit_kernel<BITS, K, 8 / K * GPT, Src>;
     } else {

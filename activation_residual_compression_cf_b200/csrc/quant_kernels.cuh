@@ -272,22 +272,28 @@ struct EncPublishArray {
         }
         return true;
     }
-    // One row's code words (staged in shared memory) and scale into every
-    // destination; 16-byte stores when the code rows are 16-byte multiples.
-    __device__ __forceinline__ void store_row(const EncPtrs &p, const uint32_t *srow, int64_t W,
-                                              int64_t t, float scale, int ct, int nc) const {
+    // A warp's gathered code words of one unit block into every destination:
+    // with 16-byte code rows (W % 4 == 0) lanes 0 .. nvec - 1 store q[0..3],
+    // words w0 + 4 lane .. + 3; otherwise each word's first lane (own) stores
+    // its word at index wi.  w0 is a multiple of 4, so a vector never
+    // straddles the end of a row.
+    __device__ __forceinline__ void store_words(const EncPtrs &p, int64_t t, int64_t W, int64_t w0, int lane,
+                                                int nvec, const uint32_t *q, uint32_t word, bool own,
+                                                int64_t wi) const {
+        const bool vec = (W & 3) == 0;
         for (int d = 0; d < ndst; ++d) {
-            uint8_t *pl = ldg_ptr(&dst[d].payload);
-            uint32_t *crow = reinterpret_cast<uint32_t *>(pl + p.codes_off) + t * W;
-            if ((W & 3) == 0) {
-                const int nv = (int)(W >> 2);
-                for (int k = ct; k < nv; k += nc)
-                    if (CF_IN(4 * k + 4 <= W)) reinterpret_cast<uint4 *>(crow)[k] = reinterpret_cast<const uint4 *>(srow)[k];
-            } else {
-                for (int k = ct; k < (int)W; k += nc) crow[k] = srow[k];
+            uint32_t *crow = reinterpret_cast<uint32_t *>(ldg_ptr(&dst[d].payload) + p.codes_off) + t * W;
+            if (vec) {
+                if (lane < nvec && w0 + 4 * lane + 4 <= W)
+                    *reinterpret_cast<uint4 *>(crow + w0 + 4 * lane) = make_uint4(q[0], q[1], q[2], q[3]);
+            } else if (own && CF_IN(wi < W)) {
+                crow[wi] = word;
             }
-            if (ct == 0) reinterpret_cast<float *>(pl + p.scales_off)[t] = scale;
         }
+    }
+    __device__ __forceinline__ void store_scale(const EncPtrs &p, int64_t t, float scale) const {
+        for (int d = 0; d < ndst; ++d)
+            reinterpret_cast<float *>(ldg_ptr(&dst[d].payload) + p.scales_off)[t] = scale;
     }
     // Release of this CTA's rows: the fence orders every store the CTA made
     // (observed through the barrier before this call) before the adds.

@@ -24,10 +24,10 @@
 // (when given) and the CTA stops.
 //
 // Publishing encode / waiting decode (the exchange with the payload transfer
-// fused in): with a publishing source the encode stages each row's code
-// words in shared memory and copies the row, with 16-byte stores where the
-// row allows, into every destination payload slot (which may be another
-// GPU's memory), writes the scale there too, and after its last row adds
+// fused in): with a publishing source the encode's warps gather their code
+// words with shuffles and store them, 16 bytes per lane where the row
+// allows, into every destination payload slot (which may be another GPU's
+// memory), write the scale there too, and after its last row add
 // the rows it walked to each destination's ready counter with a
 // system-scope release.  With a waiting source the decode's producer reads
 // a buffer's rows only after that buffer's ready counter has reached the
@@ -404,13 +404,9 @@ decode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
     }
 }
 
-// Code words of the longest row (C = 16384 at 2 bits): the publishing
-// encode stages one row of them in shared memory.
-constexpr int kMaxCodeWords = 1024;
-
 template <int BITS, int K, int UPT, class Src>
-__global__ void __launch_bounds__(512)
-encode_tma_unit_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, int stages) {
+__device__ __forceinline__ void encode_unit_body(const Src &src, int64_t T, int64_t C, int64_t rows,
+                                                 int32_t *status, int stages) {
     static_assert(K == 4 || K == 8, "units of 4 or 8 channels");
     constexpr int UPW = 32 / (K * BITS);  // units per 32-bit code word
     extern __shared__ __align__(16) uint8_t smem[];
@@ -418,7 +414,6 @@ encode_tma_unit_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *sta
     __shared__ float sh_max[2][32];
     __shared__ int abort_row[2];  // set before the row's barrier, read after it
     __shared__ int cta_abort;     // publishing: a destination check or an ack wait failed
-    __shared__ __align__(16) uint32_t srow[Src::kPublish ? kMaxCodeWords : 4];
     const int NU = (int)(C / K);  // units per row (C % 8 == 0 and C <= 16384 on this path)
     const int64_t W = (C * BITS + 31) >> 5;
     const uint32_t slot = (uint32_t)((Src::kDelta ? 8 : 6) * C);
@@ -557,7 +552,7 @@ encode_tma_unit_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *sta
         }
         par ^= 1;
         const float half = __fmul_rn(0.5f, scale);
-        uint32_t *cw = Src::kPublish ? srow : p.codes + t * W;
+        uint32_t *cw = Src::kPublish ? nullptr : p.codes + t * W;
 #pragma unroll
         for (int j = 0; j < UPT; ++j) {
             const int u = j * nc + ct;
@@ -581,14 +576,24 @@ encode_tma_unit_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *sta
             uint32_t word = field << ((lane % UPW) * K * BITS);
 #pragma unroll
             for (int o = 1; o < UPW; o <<= 1) word |= __shfl_xor_sync(kFullMask, word, o);
-            if (u < NU && (lane % UPW) == 0 && CF_IN(u / UPW < W)) cw[u / UPW] = word;
+            if constexpr (Src::kPublish) {
+                // This warp's code words of unit block j are contiguous: 32 / UPW
+                // words from w0, the word of lane group g (every lane of which
+                // holds it after the butterfly above) at w0 + g.  w0 is a
+                // multiple of 4 (nc is a multiple of 32), so lanes
+                // 0 .. 8 / UPW - 1 each gather four words and store them as one
+                // 16-byte vector to every destination.
+                const int64_t w0 = (int64_t)(j * nc + 32 * warp) / UPW;
+                uint32_t q[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) q[m] = __shfl_sync(kFullMask, word, ((4 * lane + m) * UPW) & 31);
+                src.store_words(p, t, W, w0, lane, 8 / UPW, q, word, u < NU && (lane % UPW) == 0, u / UPW);
+            } else if (u < NU && (lane % UPW) == 0 && CF_IN(u / UPW < W)) {
+                cw[u / UPW] = word;
+            }
         }
         if constexpr (Src::kPublish) {
-            // The row's code words are complete in shared memory after this
-            // barrier; the next row writes them only after its own scale
-            // barrier, which every consumer reaches after this copy-out.
-            consumer_sync(nc);
-            src.store_row(p, srow, W, t, scale, ct, nc);
+            if (ct == 0 && CF_IN(t < T)) src.store_scale(p, t, scale);
         } else {
             if (ct == 0 && CF_IN(t < T)) p.scales[t] = scale;
         }
@@ -599,6 +604,22 @@ encode_tma_unit_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *sta
         consumer_sync(nc);
         if (ct == 0) src.publish(walked);
     }
+}
+
+template <int BITS, int K, int UPT, class Src>
+__global__ void __launch_bounds__(512)
+encode_tma_unit_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, int stages) {
+    encode_unit_body<BITS, K, UPT, Src>(src, T, C, rows, status, stages);
+}
+
+// The publishing form: at most 96 registers a thread, so that three CTAs of
+// a C = 3072 or C = 1920 launch (224 or 160 threads) still fit on an SM as
+// they do for the plain encode; without the cap the destination stores
+// raise it past 110 and only two fit.
+template <int BITS, int K, int UPT, class Src>
+__global__ void __maxnreg__(96)
+encode_tma_publish_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, int stages) {
+    encode_unit_body<BITS, K, UPT, Src>(src, T, C, rows, status, stages);
 }
 
 template <int BITS, int K, int UPT, class Src>

@@ -209,6 +209,14 @@ class CudaCodec:
         dst = self._array("dst", dsts, cf.publish_dst_array)
         cf.cf_encode_publish_batched(d, len(sets), arr, len(dsts), dst, ack_target, self.status)
 
+    def prepare_publish(self, enc, dsts, dec, acks):
+        self._array("pub", enc, cf.enc_publish_buffer_array)
+        self._array("dst", dsts, cf.publish_dst_array)
+        if dec:
+            self._array("wait", dec, cf.dec_wait_buffer_array)
+        if acks:
+            self._array("ack", [(a,) for a in acks], lambda v, dev: cf.pointer_array([t[0] for t in v], dev))
+
     def decode_wait_batched(self, d, sets, ready_target, acks):
         arr = self._array("wait", sets, cf.dec_wait_buffer_array) if sets else None
         ack = self._array("ack", [(a,) for a in acks], lambda v, dev: cf.pointer_array(
@@ -358,9 +366,10 @@ class ShardExchange(_Exchange):
                           for p in self.peers for b in range(buffers)]
 
     def _enc_sets(self, xs):
-        L = self.layout
-        return [(xs[b], self.recon_s[b], self.err[b], L.codes(self.send, b), L.scales(self.send, b))
-                for b in range(L.buffers)]
+        if not hasattr(self, "_send_views"):   # built once: views cost host time every step
+            L = self.layout
+            self._send_views = [(L.codes(self.send, b), L.scales(self.send, b)) for b in range(L.buffers)]
+        return [(xs[b], self.recon_s[b], self.err[b]) + self._send_views[b] for b in range(self.buffers)]
 
     def prepare(self, xs) -> None:
         """Optional: build the codec's per-call state (the device array of
@@ -545,22 +554,54 @@ class FusedShardExchange(_Exchange):
         ranks it decodes: the exchange is symmetric)."""
         return self.peers
 
-    def step(self, xs) -> None:
-        self._check(xs)
-        self.epoch += 1
-        k = self.epoch - self.base           # steps on this memory's counters
-        s, me, L, m = self.epoch % 2, self.rank, self.layout, self.memory
-        dsts = [(m.recv[r][s, me], m.ready[r][me:me + 1], m.ack[me][r:r + 1]) for r in self._receivers()]
+    def _sets(self, xs, s):
+        """The encode's buffers, its destinations (slot s at every receiver)
+        and the decode's buffers and ack counters for one step.  The views of
+        a slot are built once and kept: a step would otherwise spend more
+        host time making hundreds of tensor views than the GPU spends on its
+        kernels."""
+        me, L, m = self.rank, self.layout, self.memory
+        cache = self.__dict__.setdefault("_slot_sets", {})
+        if s not in cache:
+            dsts = [(m.recv[r][s, me], m.ready[r][me:me + 1], m.ack[me][r:r + 1])
+                    for r in self._receivers()]
+            dec, acks = [], []
+            for p in self.peers:
+                slot = m.recv[me][s, p]
+                dec += [(L.codes(slot, b), L.scales(slot, b), self.recon_r[p][b], m.ready[me][p:p + 1])
+                        for b in range(self.buffers)]
+                acks.append(m.ack[p][me:me + 1])
+            cache[s] = (dsts, dec, acks)
+        dsts, dec, acks = cache[s]
         enc = [(xs[b], self.recon_s[b], self.err[b], L.codes_offset(b), L.scales_offset(b))
                for b in range(self.buffers)]
+        return enc, dsts, dec, acks
+
+    def prepare(self, xs) -> None:
+        """Optional: build the codec's device arrays of pointers for these
+        input tensors (both slots) ahead of their steps."""
+        self._check(xs)
+        if hasattr(self.codec, "prepare_publish"):
+            for s in (0, 1):
+                enc, dsts, dec, acks = self._sets(xs, s)
+                self.codec.prepare_publish(enc, dsts, dec, acks)
+
+    def step(self, xs, events=None) -> None:
+        """One compressed step: the publishing encode, then the waiting
+        decode of every peer's slot.  `events`, four CUDA events, are
+        recorded on the current stream before the encode, after it (twice:
+        there is no collective in between) and after the decode."""
+        self._check(xs)
+        mark = (lambda i: events[i].record()) if events is not None else (lambda i: None)
+        self.epoch += 1
+        k = self.epoch - self.base           # steps on this memory's counters
+        enc, dsts, dec, acks = self._sets(xs, self.epoch % 2)
+        mark(0)
         self.codec.encode_publish_batched(self.d, enc, dsts, max(k - 2, 0))
-        dec, acks = [], []
-        for p in self.peers:
-            slot = m.recv[me][s, p]
-            dec += [(L.codes(slot, b), L.scales(slot, b), self.recon_r[p][b], m.ready[me][p:p + 1])
-                    for b in range(self.buffers)]
-            acks.append(m.ack[p][me:me + 1])
+        mark(1)
+        mark(2)
         self.codec.decode_wait_batched(self.d, dec, k * self.buffers * self.tokens, acks)
+        mark(3)
 
     def state_dict(self) -> dict:
         sd = super().state_dict()

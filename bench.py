@@ -80,6 +80,9 @@ def parse():
     ap.add_argument("--lowrank-group", type=int, default=-1,
                     help="low-rank: buffers per pass of the batched encode (0 = all; -1 = the "
                          "library default)")
+    ap.add_argument("--fused", action="store_true",
+                    help="with --exchange: the fused exchange (publishing encode into the receivers' "
+                         "slots, waiting decode; no collective)")
     ap.add_argument("--warm", action="store_true",
                     help="low-rank: warm start every encode after the first from the previous Q")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -558,7 +561,7 @@ def run_exchange(args, world, rank, local):
     payload, one all-gather of the payloads, one batched decode of every
     peer's shard (of its own too when alone)."""
     from activation_residual_compression_cf_b200 import build, cf
-    from activation_residual_compression_cf_b200.exchange import ShardExchange
+    from activation_residual_compression_cf_b200.exchange import FusedShardExchange, ShardExchange
     build.build()
     cf.lib()
     dev = torch.device("cuda", local)
@@ -575,7 +578,8 @@ def run_exchange(args, world, rank, local):
         tr = W.Trajectory(wl, b, device=dev, seed=rank)
         for s in range(S):
             X[s, b] = tr.next()
-    ex = ShardExchange(T, C, bits, n, device=dev, loopback=(world == 1))
+    kind = FusedShardExchange if args.fused else ShardExchange
+    ex = kind(T, C, bits, n, device=dev, loopback=(world == 1))
     ex.warmup([X[0, b] for b in range(n)])
     stream = torch.cuda.current_stream(dev)
 
@@ -616,20 +620,25 @@ def run_exchange(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 in, fp32 state", "data": "synthetic",
         "config": {"workload": args.workload, "tokens": T, "channels": C, "buffers": n,
-                   "bits": bits, "mode": f"{bits}-bit + EF, sequence-parallel exchange",
+                   "bits": bits, "mode": f"{bits}-bit + EF, sequence-parallel exchange"
+                   + (", fused" if args.fused else ""),
                    "parallelism": f"sp{world} (all-gather of payloads)",
                    "l2": "inputs larger than L2", "launches_per_step": 2},
         "roofline": {"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(enc_gbs / peak, 4),
                      "traffic": recorded_traffic("encode", args.workload),
-                     "kernel": "encode_tma_kernel (batched, codes written into the payload)",
+                     "kernel": ("encode_tma_unit_kernel (publishing: codes and scales stored into "
+                                "the receivers' slots)" if args.fused
+                                else "encode_tma_kernel (batched, codes written into the payload)"),
                      "peak_kind": peak_kind, "algorithmic_bytes_per_launch": enc_bytes,
                      "avg_launch_ms": round(phase[0], 4)},
         "exchange": {"encode_ms": round(phase[0], 4), "all_gather_ms": round(phase[1], 4),
                      "decode_ms": round(phase[2], 4), "payload_bytes_per_rank": ex.payload_bytes_per_step(),
                      "decoded_shards": len(ex.peers) * n,
                      "decode_frac": round(dec_bytes / (phase[2] / 1e3) / 1e9 / peak, 4),
-                     "collective": ex.backend or "local copy (one rank)"},
+                     "collective": ("none: the encode stores into the receivers' slots, the decode "
+                                    "waits on their counters" if args.fused
+                                    else ex.backend or "local copy (one rank)")},
         "cpu_baseline": None, "e2e": None,
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,

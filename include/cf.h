@@ -232,7 +232,10 @@ cf_status cf_decode_emit_batched(const cf_desc *d, int32_t n,
  * Requirements: C % 8 == 0; the decode also ceil(C*bits/32) % 4 == 0 (the
  * TMA row pipeline); otherwise CF_ERR_UNSUPPORTED.  No TMA load ever reads
  * another GPU's memory: the sender's loads are local, the receiver's bulk
- * copies read its own memory. */
+ * copies read its own memory.  Both calls only enqueue work, so they can be
+ * stream-captured; the counter targets are arguments of the captured
+ * launches, so a captured step waits for the same counts on every replay
+ * (capture per step, or call them eagerly). */
 
 /* One destination of a publishing encode (all device pointers; the first
  * two may be another GPU's memory mapped for peer access). */

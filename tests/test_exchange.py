@@ -505,6 +505,7 @@ def _fused_worker(rank, world, port, folder, leave_after, q):
                     oracle.encode(W.bf16_bits(shard(trajs[b][t], p)), rec, bits)
                 if not np.array_equal(ex.recon_r[p][b].numpy(), rec):
                     bad.append((p, b))
+        dist.barrier()        # every rank's last decode (and its acks) is done
         counters = ([int(v) for v in mem.ready[rank]], [int(v) for v in mem.ack[rank]])
         q.put((rank, "ok" if not bad else "bad", bad, counters))
         dist.barrier()

@@ -123,3 +123,55 @@ def test_lowrank_step_graph_replay_equals_eager():
         for b in range(n):
             assert cf.cf_lowrank_status(graph["ws"][b * wsb:]) == 0
     del g
+
+
+def test_async_status_read_inside_a_captured_step():
+    """cf_lowrank_status_async enqueues one strided device-to-host copy, so
+    it captures with the batched encode: after each replay the pinned host
+    words hold what the blocking per-slice read returns."""
+    T, C, r, n = 256, 192, 8, 3
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r)
+    d = cf.desc(T, C, 0, r, 2)
+    wsb = cf.cf_lowrank_workspace_bytes(d)
+    nb = (r + 1) // 2
+    f32 = dict(dtype=torch.float32, device="cuda")
+    xs = [W.trajectory(wl, b, steps=3, device="cuda") for b in range(n)]
+    rs = torch.empty(n, T, C, **f32)
+    er = torch.empty(n, T, C, **f32)
+    x = torch.empty(n, T, C, dtype=torch.bfloat16, device="cuda")
+    pc = torch.empty(n, T * nb + 16, dtype=torch.uint8, device="cuda")
+    qc = torch.empty(n, C * nb + 16, dtype=torch.uint8, device="cuda")
+    ps, qs = torch.empty(n, r, **f32), torch.empty(n, r, **f32)
+    om = torch.stack([W.omega(wl, b, 1, device="cuda") for b in range(n)])
+    for b in range(n):
+        cf.cf_state_init(d, xs[b][0].view(torch.int16), rs[b], er[b])
+    x16 = x.view(torch.int16)
+    # buffer 1 gets a zero residual (CF_ERR_NUMERIC), the others real steps;
+    # the capture warm-up below is step 1 of every buffer
+    enc = cf.lowrank_buffer_array([(x16[b], rs[b], er[b], om[b], pc[b], ps[b], qc[b], qs[b])
+                                   for b in range(n)], "cuda")
+    ws = torch.empty(n * wsb, dtype=torch.uint8, device="cuda")
+    host = torch.full((n,), -1, dtype=torch.int32).pin_memory()
+    for b in range(n):
+        x[b].copy_(xs[1][0] if b == 1 else xs[b][1])
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        cf.cf_lowrank_encode_batched(d, n, enc, ws, stream=s)    # first-call set-up outside capture
+        s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        cf.cf_lowrank_encode_batched(d, n, enc, ws, stream=s)
+        cf.cf_lowrank_status_async(ws, wsb, n, host, stream=s)
+    for t in (1, 2):
+        # buffer 1 stays at its warmup activation: its state equals it
+        # exactly, so its residual is zero at every step
+        for b in range(n):
+            x[b].copy_(xs[1][0] if b == 1 else xs[b][t])
+        host.fill_(-1)
+        g.replay()
+        torch.cuda.synchronize()
+        got = host.tolist()
+        want = [cf.cf_lowrank_status(ws[b * wsb:]) for b in range(n)]
+        assert got == want, (t, got, want)
+        assert got[0] == 0 and got[2] == 0 and got[1] == 6, got
