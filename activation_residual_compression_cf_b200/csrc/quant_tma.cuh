@@ -612,12 +612,14 @@ encode_tma_unit_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *sta
     encode_unit_body<BITS, K, UPT, Src>(src, T, C, rows, status, stages);
 }
 
-// The publishing form: at most 96 registers a thread, so that three CTAs of
-// a C = 3072 or C = 1920 launch (224 or 160 threads) still fit on an SM as
-// they do for the plain encode; without the cap the destination stores
-// raise it past 110 and only two fit.
+// The publishing form: at most 80 registers a thread, so that three CTAs of
+// a C = 3072 launch (7 warps each) still fit on an SM as they do for the
+// plain encode: the warps of an SM's CTAs spread over its four 16K-register
+// sub-partitions, and the sub-partition that holds 6 of the 21 warps needs
+// 6 x 32 x R <= 16384.  Without the cap the destination stores raise R past
+// 110, and at 96 only two CTAs fit (measured: 296-CTA grid, 40 % slower).
 template <int BITS, int K, int UPT, class Src>
-__global__ void __maxnreg__(96)
+__global__ void __maxnreg__(80)
 encode_tma_publish_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, int stages) {
     encode_unit_body<BITS, K, UPT, Src>(src, T, C, rows, status, stages);
 }

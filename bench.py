@@ -479,6 +479,26 @@ def run_ours(args, world, rank, local):
     enc_gbs = enc_bytes / (enc_ms / 1e3) / 1e9
     dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9
 
+    # Invariants of the state after the run (no oracle): the receiver equals
+    # the sender's mirror bit for bit, and recon_s + err == x of the last
+    # step within the three fp32 roundings of a step (residual v, error,
+    # mirror update: u (|v| + |err| + |recon|), with |v| <= |err| + the
+    # row's scale since |deq| <= scale), for every buffer.
+    invariants = None
+    if not args.delta:
+        last = X[1 + (args.warmup + args.steps - 1) % (S - 1)]
+        gap_ok = True
+        for b in range(n):
+            xb = last[b].double()
+            rs, er = recon_s[b].double(), err[b].double()
+            sc = scales[b].double()[:, None]
+            bound = (2 * er.abs() + sc + rs.abs()) * 2.0 ** -24 * (1 + 1e-6) + 3 * 2.0 ** -149
+            gap_ok &= bool(((rs + er - xb).abs() <= bound).all())
+            del xb, rs, er, sc, bound
+        invariants = {"receiver_equals_sender": bool(torch.equal(recon_r.view(torch.int32),
+                                                                 recon_s.view(torch.int32))),
+                      "ef_identity_within_roundings": gap_ok, "buffers_checked": n}
+
     # End to end through the public API: pinned host x in, payload out.
     e2e = None
     if not args.no_e2e and not args.delta and not args.emit:
@@ -550,6 +570,7 @@ def run_ours(args, world, rank, local):
                    "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_ms": round(dec_ms, 4)},
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "invariants": invariants,
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
     }
