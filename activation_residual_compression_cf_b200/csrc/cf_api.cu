@@ -293,6 +293,13 @@ cf_status dispatch(const Src &src, int bits, int64_t T, int64_t C, int64_t rows,
     if (kFused && pipe != 1) return CF_ERR_UNSUPPORTED;
     s.pipeline = pipe;
     s.unit = choose_unit(ENC ? 0 : 1, bits, C, delta);
+    if constexpr (Src::kPublish) {
+        // the publishing encode at 4-channel units needs more registers than
+        // the 80 that keep three CTAs per SM (it spills): 8-channel units
+        // unless a sweep overrides it
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_unit[0]) s.unit = 8;
+    }
     const bool vec = (C % 8) == 0;
 #define CF_CASE(B, G, V)                                     \
     if (bits == B && s.gpt == G && vec == V)                 \
