@@ -280,8 +280,10 @@ encode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
                 st_stream_v4(er + 8 * g, make_float4(eo[0], eo[1], eo[2], eo[3]));
                 st_stream_v4(er + 8 * g + 4, make_float4(eo[4], eo[5], eo[6], eo[7]));
                 if (!Src::kDelta) {
-                    st_state_v4(rr + 8 * g, make_float4(ro[0], ro[1], ro[2], ro[3]));
-                    st_state_v4(rr + 8 * g + 4, make_float4(ro[4], ro[5], ro[6], ro[7]));
+                    // streaming (evict-first) like err: measured 0.3-1.3 % faster
+                    // than a plain store for the reconstruction too
+                    st_stream_v4(rr + 8 * g, make_float4(ro[0], ro[1], ro[2], ro[3]));
+                    st_stream_v4(rr + 8 * g + 4, make_float4(ro[4], ro[5], ro[6], ro[7]));
                 }
                 if ((lane % GPW) == 0) cw[g / GPW] = word;
             }
