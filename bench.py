@@ -555,7 +555,8 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16 in, fp32 state", "data": "synthetic",
+        "dtype": "f32", "dtype_note": "bf16 activations in; fp32 state and arithmetic (fp64 1-bit sums)",
+        "data": "synthetic",
         "config": quant_config(args, wl, world),
         "roofline": {"bound": "hbm", "achieved": round(enc_gbs, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(enc_gbs / peak, 4), "traffic": traffic,
@@ -639,7 +640,8 @@ def run_exchange(args, world, rank, local):
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16 in, fp32 state", "data": "synthetic",
+        "dtype": "f32", "dtype_note": "bf16 activations in; fp32 state and arithmetic (fp64 1-bit sums)",
+        "data": "synthetic",
         "config": {"workload": args.workload, "tokens": T, "channels": C, "buffers": n,
                    "bits": bits, "mode": f"{bits}-bit + EF, sequence-parallel exchange"
                    + (", fused" if args.fused else ""),
@@ -795,7 +797,9 @@ def run_lowrank(args, world, rank, local):
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16 in, fp32 state, bf16 tensor products", "data": "synthetic",
+        "dtype": "f32", "dtype_note": "bf16 activations in; fp32 state; bf16 and tf32 tensor products "
+                                      "with fp32 accumulation",
+        "data": "synthetic",
         "config": lowrank_config(args, wl, world),
         "roofline": {"bound": "hbm",
                      "achieved": round(app_enc_bytes / (app_enc_ms / 1e3) / 1e9, 1),
@@ -1042,7 +1046,8 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(sec * 1e3 / args.steps, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 state",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "dtype_note": "bf16 activations in; fp32 state and arithmetic (the oracle's fp64 sums and products)",
         "data": "synthetic",
         "config": config,
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
