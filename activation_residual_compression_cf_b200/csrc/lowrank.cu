@@ -263,8 +263,8 @@ cf_status backproject(const LrBatch &B, const Layout &L, int n, bool last, cudaS
 }
 
 cf_status orth(const LrBatch &B, const Layout &L, int n, bool last, cudaStream_t st) {
-    const dim3 grid((unsigned)((L.Tp + 63) / 64), 1, (unsigned)n);
-#define CF_ORTH(RP) cf::lr_orth_kernel<RP><<<grid, 64, 0, st>>>(B, L, last ? 1 : 0)
+    const dim3 grid((unsigned)((L.Tp + cf::kOrthThreads - 1) / cf::kOrthThreads), 1, (unsigned)n);
+#define CF_ORTH(RP) cf::lr_orth_kernel<RP><<<grid, cf::kOrthThreads, 0, st>>>(B, L, last ? 1 : 0)
     switch (L.rp) {
         case 16: CF_ORTH(16); break;
         case 32: CF_ORTH(32); break;
@@ -369,7 +369,6 @@ cf_status encode_impl(const cf_desc *d, const Layout &L, int n, const LrBatch &B
 }
 
 cf_status encode_group(const cf_desc *d, const Layout &L, int n, const LrBatch &B, cudaStream_t st) {
-    const int nb = (L.r + 1) / 2;
     const bool fused = g_engine.load() == 0;
     cf::lr_prep_kernel<<<(unsigned)n, 128, 0, st>>>(B, L);
     LR_LAUNCHED();
@@ -383,7 +382,9 @@ cf_status encode_group(const cf_desc *d, const Layout &L, int n, const LrBatch &
             cf::lr_residual_kernel<<<dim3((unsigned)blocks, 1, (unsigned)n), 256, 0, st>>>(B, L);
             LR_LAUNCHED();
         }
-        cf::lr_omega_kernel<<<dim3((unsigned)((L.C + 31) / 32), (unsigned)((L.rp + 31) / 32), (unsigned)n),
+        const int64_t ctiles = (L.C + 31) / 32;
+        cf::lr_omega_kernel<<<dim3((unsigned)((ctiles + cf::kOmegaTilesPerBlock - 1) / cf::kOmegaTilesPerBlock),
+                                   (unsigned)((L.rp + 31) / 32), (unsigned)n),
                               dim3(32, 8), 0, st>>>(B, L);
         LR_LAUNCHED();
     }
@@ -406,10 +407,13 @@ cf_status encode_group(const cf_desc *d, const Layout &L, int n, const LrBatch &
         if (!fused) LR_TRY(reduce_q(B, L, n, last, st));
     }
     // INT4 factors: quantise and pack against the column maxima.
-    cf::lr_int4_pack_kernel<<<dim3((unsigned)((L.T * nb + 255) / 256), 1, (unsigned)n), 256, 0, st>>>(B, L, 0);
-    LR_LAUNCHED();
-    cf::lr_int4_pack_kernel<<<dim3((unsigned)((L.C * nb + 255) / 256), 1, (unsigned)n), 256, 0, st>>>(B, L, 1);
-    LR_LAUNCHED();
+    {
+        const int64_t rows = L.T > L.C ? L.T : L.C;
+        cf::lr_int4_pack_kernel<<<dim3((unsigned)((rows + cf::kPackThreads - 1) / cf::kPackThreads), 2,
+                                       (unsigned)n),
+                                  cf::kPackThreads, 0, st>>>(B, L);
+        LR_LAUNCHED();
+    }
     return apply(true, B, L, n, st);
 }
 

@@ -92,10 +92,13 @@ __global__ void lr_residual_kernel(const LrBatch B, const Layout L) {
 }
 
 // Qt[k][c] = bf16(omega[c][k]) for k < r, 0 for the padding rows.
+constexpr int kOmegaTilesPerBlock = 4;
+
 __global__ void lr_omega_kernel(const LrBatch B, const Layout L) {
-    // Qt[k][c] = bf16(Omega[c][k]) (0 for k >= r), one 32 x 32 tile per
-    // block (32 x 8 threads): coalesced reads of Omega's rows, transposed
-    // through shared memory, coalesced writes of Qt's rows.
+    // Qt[k][c] = bf16(Omega[c][k]) (0 for k >= r), 32 x 32 tiles (32 x 8
+    // threads), kOmegaTilesPerBlock of them a grid stride apart along the
+    // channels: coalesced reads of Omega's rows, transposed through shared
+    // memory, coalesced writes of Qt's rows.
     const int bz = blockIdx.z;
     if (lr_skipped(B, L, bz)) return;
     const float *omega = B.get(bz).omega;
@@ -104,20 +107,22 @@ __global__ void lr_omega_kernel(const LrBatch B, const Layout L) {
     const int64_t C = L.C;
     const int r = L.r;
     __shared__ float tile[32][33];
-    const int64_t c0 = (int64_t)blockIdx.x * 32;
     const int k0 = blockIdx.y * 32;
     const int tx = threadIdx.x, ty = threadIdx.y;
-    for (int j = ty; j < 32; j += 8) {
-        const int64_t c = c0 + j;
-        const int k = k0 + tx;
-        tile[j][tx] = (c < C && k < r && CF_IN(c * r + k < C * r)) ? omega[c * r + k] : 0.0f;
-    }
-    __syncthreads();
-    for (int j = ty; j < 32; j += 8) {
-        const int k = k0 + j;
-        const int64_t c = c0 + tx;
-        if (k < L.rp && c < C && CF_IN((int64_t)k * C + c < (int64_t)L.rp * C))
-            qt[(int64_t)k * C + c] = __float2bfloat16_rn(tile[tx][j]);
+    for (int64_t c0 = (int64_t)blockIdx.x * 32; c0 < C; c0 += (int64_t)gridDim.x * 32) {
+        for (int j = ty; j < 32; j += 8) {
+            const int64_t c = c0 + j;
+            const int k = k0 + tx;
+            tile[j][tx] = (c < C && k < r && CF_IN(c * r + k < C * r)) ? omega[c * r + k] : 0.0f;
+        }
+        __syncthreads();
+        for (int j = ty; j < 32; j += 8) {
+            const int k = k0 + j;
+            const int64_t c = c0 + tx;
+            if (k < L.rp && c < C && CF_IN((int64_t)k * C + c < (int64_t)L.rp * C))
+                qt[(int64_t)k * C + c] = __float2bfloat16_rn(tile[tx][j]);
+        }
+        __syncthreads();   // the tile is refilled by the next pass
     }
 }
 
@@ -420,8 +425,16 @@ lr_gram_chol_kernel(const LrBatch B, const Layout L) {
 // past T) that the back-projection reads.  On the last iteration (amax !=
 // null) it also folds max |P[:, k]| into amax[k] (float bits, atomicMax once
 // per CTA and column).
+//
+// The substitution runs column by column: once P[t][j] is final, it is taken
+// out of every later column, reading row j of R as 16-byte shared-memory
+// loads (a row-at-a-time sweep needs one scalar load per product).  Each
+// column k still receives its products in ascending j, so the sums are
+// exactly those of the row-at-a-time form.
+constexpr int kOrthThreads = 256;
+
 template <int RP>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kOrthThreads)
 lr_orth_kernel(const LrBatch B, const Layout L, int want_amax) {
     const int bz = blockIdx.z;
     if (lr_skipped(B, L, bz)) return;
@@ -432,13 +445,15 @@ lr_orth_kernel(const LrBatch B, const Layout L, int want_amax) {
     bf16 *pt = B.at<bf16>(bz, L.off_pt);
     const int64_t T = L.T, Tp = L.Tp;
     uint32_t *amax = want_amax ? B.at<uint32_t>(bz, L.off_amax) : nullptr;
-    __shared__ float Rs[RP * RP];
+    constexpr int NW = kOrthThreads / 32;
+    __shared__ __align__(16) float Rs[RP * RP];
     __shared__ float Id[RP];
-    __shared__ float Wm[4][RP];
-    for (int i = threadIdx.x; i < RP * RP; i += blockDim.x) Rs[i] = rmat[i];
-    for (int i = threadIdx.x; i < RP; i += blockDim.x) Id[i] = rinvd[i];
+    __shared__ float Wm[NW][RP];
+    for (int i = threadIdx.x; i < RP * RP; i += kOrthThreads) Rs[i] = rmat[i];
+    for (int i = threadIdx.x; i < RP; i += kOrthThreads) Id[i] = rinvd[i];
     __syncthreads();
-    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const float4 *R4 = reinterpret_cast<const float4 *>(Rs);
+    const int64_t t = (int64_t)blockIdx.x * kOrthThreads + threadIdx.x;
     float pv[RP];
     if (t < T) {
         const float4 *yr = reinterpret_cast<const float4 *>(y + t * RP);
@@ -451,11 +466,17 @@ lr_orth_kernel(const LrBatch B, const Layout L, int want_amax) {
             pv[4 * q + 3] = v.w;
         }
 #pragma unroll
-        for (int k = 0; k < RP; ++k) {
-            float acc = pv[k];
+        for (int j = 0; j < RP; ++j) {
+            pv[j] = pv[j] * Id[j];
+            const float nj = -pv[j];
 #pragma unroll
-            for (int j = 0; j < k; ++j) acc = fmaf(-pv[j], Rs[j * RP + k], acc);
-            pv[k] = acc * Id[k];
+            for (int q = (j + 1) / 4; q < RP / 4; ++q) {
+                const float4 rv = R4[(j * RP) / 4 + q];
+                const float re[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (4 * q + e > j) pv[4 * q + e] = fmaf(nj, re[e], pv[4 * q + e]);
+            }
         }
         float4 *pr = reinterpret_cast<float4 *>(p + t * RP);
 #pragma unroll
@@ -479,9 +500,9 @@ lr_orth_kernel(const LrBatch B, const Layout L, int want_amax) {
             if (lane == 0) Wm[warp][k] = m;
         }
         __syncthreads();
-        for (int k = threadIdx.x; k < RP; k += blockDim.x) {
+        for (int k = threadIdx.x; k < RP; k += kOrthThreads) {
             float m = 0.0f;
-            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, Wm[w][k]);
+            for (int w = 0; w < NW; ++w) m = fmaxf(m, Wm[w][k]);
             atomicMax(amax + k, __float_as_uint(m));
         }
     }
@@ -614,40 +635,76 @@ __device__ __forceinline__ int int4_code(float v, float s) {
 }
 
 // INT4 per column: s_k = amax_k / 7; codes packed two per byte, the even
-// column in the low nibble; the scales are written by the first r threads.
-__global__ void lr_int4_pack_kernel(const LrBatch B, const Layout L, int which) {
+// column in the low nibble.  One launch packs both factors: blockIdx.y = 0
+// packs P (T rows), 1 packs Q (C rows).  A thread owns one row: it reads the
+// row's rp floats as float4s and writes the row's nb bytes, as one 16-byte
+// store per 32 columns when the row's codes are 16-byte aligned, else byte
+// by byte (same bytes either way).  Block 0 of each factor writes the
+// column scales.
+constexpr int kPackThreads = 128;
+
+__global__ void __launch_bounds__(kPackThreads) lr_int4_pack_kernel(const LrBatch B, const Layout L) {
     const int bz = blockIdx.z;
     if (lr_skipped(B, L, bz)) return;
+    const int which = blockIdx.y;
+    const int64_t rows = which == 0 ? L.T : L.C;
+    const int64_t row0 = (int64_t)blockIdx.x * kPackThreads;
+    if (row0 >= rows) return;   // the shorter factor's grid tail (never block 0)
     const LrPtrs pp = B.get(bz);
     const int r = L.r, rp = L.rp;
     const float *f = B.at<float>(bz, which == 0 ? L.off_p : L.off_q);
-    const int64_t rows = which == 0 ? L.T : L.C;
     const uint32_t *amax = B.at<uint32_t>(bz, L.off_amax) + (which == 0 ? 0 : rp);
     uint8_t *codes = which == 0 ? pp.pc_out : pp.qc_out;
     float *scales = which == 0 ? pp.ps_out : pp.qs_out;
     const int nb = (r + 1) / 2;
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     // the column scales, once per block (the same division every element
-    // would otherwise repeat)
+    // would otherwise repeat); zero past r, so padded columns code to 0
     __shared__ float sc[cf_lowrank::kMaxRank];
-    for (int k = threadIdx.x; k < r; k += blockDim.x) sc[k] = __fdiv_rn(__uint_as_float(amax[k]), 7.0f);
+    for (int k = threadIdx.x; k < rp; k += kPackThreads)
+        sc[k] = k < r ? __fdiv_rn(__uint_as_float(amax[k]), 7.0f) : 0.0f;
     __syncthreads();
-    if (i < r) scales[i] = sc[i];
-    if (which == 1 && i == 0) {
-        // the workspace now holds this encode's final Q (Qt): a later
-        // encode of this shape may start from it
-        uint32_t *wt = B.at<uint32_t>(bz, L.off_status);
-        wt[cf_lowrank::kWarmTag] = cf_lowrank::kWarmMagic | (uint32_t)r;
-        wt[cf_lowrank::kWarmC] = (uint32_t)L.C;
+    if (blockIdx.x == 0) {
+        for (int k = threadIdx.x; k < r; k += kPackThreads) scales[k] = sc[k];
+        if (which == 1 && threadIdx.x == 0) {
+            // the workspace now holds this encode's final Q (Qt): a later
+            // encode of this shape may start from it
+            uint32_t *wt = B.at<uint32_t>(bz, L.off_status);
+            wt[cf_lowrank::kWarmTag] = cf_lowrank::kWarmMagic | (uint32_t)r;
+            wt[cf_lowrank::kWarmC] = (uint32_t)L.C;
+        }
     }
-    if (i >= rows * nb) return;
-    const int64_t row = i / nb;
-    if (!CF_IN(row < rows && 2 * (i - row * nb) < rp)) return;
-    const int b = (int)(i - row * nb);
-    const int k0 = 2 * b, k1 = 2 * b + 1;
-    const int q0 = int4_code(f[row * rp + k0], sc[k0]);
-    const int q1 = (k1 < r) ? int4_code(f[row * rp + k1], sc[k1]) : 0;
-    codes[i] = (uint8_t)((q0 & 0xF) | ((q1 & 0xF) << 4));
+    const int64_t row = row0 + threadIdx.x;
+    if (row >= rows) return;
+    const float4 *fr = reinterpret_cast<const float4 *>(f + row * rp);
+    uint8_t *cr = codes + row * nb;
+    const bool vec = (nb % 16) == 0 && (reinterpret_cast<uintptr_t>(cr) & 15u) == 0;
+    // 32 columns (16 bytes) at a time; rp is a multiple of 16, so the last
+    // block may hold 16 columns (8 bytes)
+    for (int k0 = 0; k0 < rp; k0 += 32) {
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        const int kn = rp - k0 < 32 ? rp - k0 : 32;
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+            if (4 * q4 >= kn || !CF_IN(k0 + 4 * q4 + 4 <= rp)) break;
+            const float4 v = __ldcg(fr + (k0 / 4 + q4));
+            const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int k = k0 + 4 * q4 + j;
+                const uint32_t nib = (uint32_t)int4_code(e[j], sc[k]) & 0xFu;
+                const int c = 4 * q4 + j;   // column within the 32-column block
+                w[c >> 3] |= nib << (4 * (c & 7));
+            }
+        }
+        const int bytes = (nb - k0 / 2) < 16 ? (nb - k0 / 2) : 16;
+        if (vec && bytes == 16) {
+            *reinterpret_cast<uint4 *>(cr + k0 / 2) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+#pragma unroll
+            for (int bi = 0; bi < 16; ++bi)
+                if (bi < bytes && CF_IN(k0 / 2 + bi < nb)) cr[k0 / 2 + bi] = (uint8_t)(w[bi >> 2] >> (8 * (bi & 3)));
+        }
+    }
 }
 
 __device__ __forceinline__ float int4_dequant(const uint8_t *row_codes, int k, const float *scales) {

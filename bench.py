@@ -358,7 +358,7 @@ def lowrank_config(args, wl, world):
             "buffers": wl.buffers, "rank": wl.rank, "iters": it,
             "mode": "low-rank INT4 + EF" + (", warm start" if args.warm else ""),
             "parallelism": f"replicas x{world}", "l2": "inputs larger than L2",
-            "launches_per_step": 5 + 3 * it + 1}
+            "launches_per_step": 4 + 3 * it + 1}
 
 
 def lowrank_workload(args):
@@ -773,8 +773,9 @@ def run_lowrank(args, world, rank, local):
     # Launches per step: the sender runs prep, omega, three kernels per
     # subspace iteration (project with its Gram/Cholesky tail -- the first
     # one also forms the bf16 residual --, orthogonalise, back-project with
-    # its Q-reduction tail), two INT4 packs and the apply; the receiver one.
-    launches_per_step = 5 + 3 * it + 1
+    # its Q-reduction tail), one INT4 pack of both factors and the apply; the
+    # receiver one.
+    launches_per_step = 4 + 3 * it + 1
 
     e2e = None
     if not args.no_e2e:
