@@ -263,8 +263,10 @@ cf_status backproject(const LrBatch &B, const Layout &L, int n, bool last, cudaS
 }
 
 cf_status orth(const LrBatch &B, const Layout &L, int n, bool last, cudaStream_t st) {
-    const dim3 grid((unsigned)((L.Tp + cf::kOrthThreads - 1) / cf::kOrthThreads), 1, (unsigned)n);
-#define CF_ORTH(RP) cf::lr_orth_kernel<RP><<<grid, cf::kOrthThreads, 0, st>>>(B, L, last ? 1 : 0)
+#define CF_ORTH(RP)                                                                                   \
+    cf::lr_orth_kernel<RP><<<dim3((unsigned)((L.Tp + cf::orth_threads<RP>() - 1) / cf::orth_threads<RP>()), \
+                                  1, (unsigned)n),                                                        \
+                             cf::orth_threads<RP>(), 0, st>>>(B, L, last ? 1 : 0)
     switch (L.rp) {
         case 16: CF_ORTH(16); break;
         case 32: CF_ORTH(32); break;
@@ -409,9 +411,14 @@ cf_status encode_group(const cf_desc *d, const Layout &L, int n, const LrBatch &
     // INT4 factors: quantise and pack against the column maxima.
     {
         const int64_t rows = L.T > L.C ? L.T : L.C;
-        cf::lr_int4_pack_kernel<<<dim3((unsigned)((rows + cf::kPackThreads - 1) / cf::kPackThreads), 2,
-                                       (unsigned)n),
-                                  cf::kPackThreads, 0, st>>>(B, L);
+        const dim3 grid((unsigned)((rows + cf::kPackThreads - 1) / cf::kPackThreads), 2, (unsigned)n);
+        switch (L.rp) {
+            case 16: cf::lr_int4_pack_kernel<16><<<grid, cf::kPackThreads, 0, st>>>(B, L); break;
+            case 32: cf::lr_int4_pack_kernel<32><<<grid, cf::kPackThreads, 0, st>>>(B, L); break;
+            case 48: cf::lr_int4_pack_kernel<48><<<grid, cf::kPackThreads, 0, st>>>(B, L); break;
+            case 64: cf::lr_int4_pack_kernel<64><<<grid, cf::kPackThreads, 0, st>>>(B, L); break;
+            default: return CF_ERR_UNSUPPORTED;
+        }
         LR_LAUNCHED();
     }
     return apply(true, B, L, n, st);

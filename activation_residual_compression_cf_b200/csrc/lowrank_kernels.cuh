@@ -419,6 +419,28 @@ lr_gram_chol_kernel(const LrBatch B, const Layout L) {
     if (tid == 0) *ticket = 0u;
 }
 
+// Row staging for the one-row-per-thread kernels below: a warp copies the
+// RP-float rows row0 .. row0 + 31 of a row-major [rows][RP] fp32 array into
+// its shared-memory tile [32][RP + 4] with coalesced 16-byte loads (rows past
+// `rows` read as 0), so that afterwards lane l holds row row0 + l in the
+// tile's row l.  The 4-float pad keeps the lanes' 16-byte row reads free of
+// bank conflicts.
+template <int RP>
+__device__ __forceinline__ void warp_stage_rows(const float *src, int64_t row0, int64_t rows, float *tile,
+                                                int lane) {
+    constexpr int Q = RP / 4;   // float4 per row
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+    for (int i = 0; i < Q; ++i) {
+        const int idx = i * 32 + lane;   // float4 index within the warp's 32 rows
+        const int rr = idx / Q, c4 = idx - (idx / Q) * Q;
+        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (row0 + rr < rows) v = __ldcg(s4 + row0 * Q + idx);
+        *reinterpret_cast<float4 *>(tile + rr * (RP + 4) + 4 * c4) = v;
+    }
+    __syncwarp();
+}
+
 // P = Y R^-1 by forward substitution, one token row per thread:
 //   P[t][k] = (Y[t][k] - sum_{j<k} P[t][j] R[j][k]) / R[k][k]
 // written as fp32 P [T][rp] and as the bf16 transpose Pt [rp][Tp] (zero
@@ -426,16 +448,24 @@ lr_gram_chol_kernel(const LrBatch B, const Layout L) {
 // null) it also folds max |P[:, k]| into amax[k] (float bits, atomicMax once
 // per CTA and column).
 //
-// The substitution runs column by column: once P[t][j] is final, it is taken
-// out of every later column, reading row j of R as 16-byte shared-memory
-// loads (a row-at-a-time sweep needs one scalar load per product).  Each
-// column k still receives its products in ascending j, so the sums are
-// exactly those of the row-at-a-time form.
-constexpr int kOrthThreads = 256;
+// Each warp moves its 32 rows of Y in and of P out through a shared-memory
+// tile with coalesced 16-byte accesses.  The substitution runs column by
+// column: once P[t][j] is final, it is taken out of every later column,
+// reading row j of R as 16-byte shared-memory loads (a row-at-a-time sweep
+// needs one scalar load per product).  Each column k still receives its
+// products in ascending j, so the sums are exactly those of the row-at-a-time
+// form.
+// Threads per block: 4 warps, 2 at rank 64 (the R matrix and the staging
+// tiles stay within 48 KB of static shared memory).
+template <int RP>
+__host__ __device__ constexpr int orth_threads() {
+    return RP > 48 ? 64 : 128;
+}
 
 template <int RP>
-__global__ void __launch_bounds__(kOrthThreads)
+__global__ void __launch_bounds__(orth_threads<RP>())
 lr_orth_kernel(const LrBatch B, const Layout L, int want_amax) {
+    constexpr int kOrthThreads = orth_threads<RP>();
     const int bz = blockIdx.z;
     if (lr_skipped(B, L, bz)) return;
     const float *y = B.at<float>(bz, L.off_y);
@@ -446,31 +476,37 @@ lr_orth_kernel(const LrBatch B, const Layout L, int want_amax) {
     const int64_t T = L.T, Tp = L.Tp;
     uint32_t *amax = want_amax ? B.at<uint32_t>(bz, L.off_amax) : nullptr;
     constexpr int NW = kOrthThreads / 32;
+    constexpr int Q = RP / 4;
     __shared__ __align__(16) float Rs[RP * RP];
+    __shared__ __align__(16) float tiles[NW][32 * (RP + 4)];
     __shared__ float Id[RP];
     __shared__ float Wm[NW][RP];
     for (int i = threadIdx.x; i < RP * RP; i += kOrthThreads) Rs[i] = rmat[i];
     for (int i = threadIdx.x; i < RP; i += kOrthThreads) Id[i] = rinvd[i];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row0 = (int64_t)blockIdx.x * kOrthThreads + 32 * warp;
+    float *tile = tiles[warp];
+    warp_stage_rows<RP>(y, row0, T, tile, lane);
     __syncthreads();
     const float4 *R4 = reinterpret_cast<const float4 *>(Rs);
-    const int64_t t = (int64_t)blockIdx.x * kOrthThreads + threadIdx.x;
+    float4 *mine = reinterpret_cast<float4 *>(tile + lane * (RP + 4));
+    const int64_t t = row0 + lane;
     float pv[RP];
-    if (t < T) {
-        const float4 *yr = reinterpret_cast<const float4 *>(y + t * RP);
 #pragma unroll
-        for (int q = 0; q < RP / 4; ++q) {
-            const float4 v = yr[q];
-            pv[4 * q] = v.x;
-            pv[4 * q + 1] = v.y;
-            pv[4 * q + 2] = v.z;
-            pv[4 * q + 3] = v.w;
-        }
+    for (int q = 0; q < Q; ++q) {
+        const float4 v = mine[q];
+        pv[4 * q] = v.x;
+        pv[4 * q + 1] = v.y;
+        pv[4 * q + 2] = v.z;
+        pv[4 * q + 3] = v.w;
+    }
+    if (t < T) {
 #pragma unroll
         for (int j = 0; j < RP; ++j) {
             pv[j] = pv[j] * Id[j];
             const float nj = -pv[j];
 #pragma unroll
-            for (int q = (j + 1) / 4; q < RP / 4; ++q) {
+            for (int q = (j + 1) / 4; q < Q; ++q) {
                 const float4 rv = R4[(j * RP) / 4 + q];
                 const float re[4] = {rv.x, rv.y, rv.z, rv.w};
 #pragma unroll
@@ -478,20 +514,22 @@ lr_orth_kernel(const LrBatch B, const Layout L, int want_amax) {
                     if (4 * q + e > j) pv[4 * q + e] = fmaf(nj, re[e], pv[4 * q + e]);
             }
         }
-        float4 *pr = reinterpret_cast<float4 *>(p + t * RP);
+    }   // rows past T stay 0 (the staging read them as 0)
 #pragma unroll
-        for (int q = 0; q < RP / 4; ++q)
-            pr[q] = make_float4(pv[4 * q], pv[4 * q + 1], pv[4 * q + 2], pv[4 * q + 3]);
-    } else {
+    for (int q = 0; q < Q; ++q) mine[q] = make_float4(pv[4 * q], pv[4 * q + 1], pv[4 * q + 2], pv[4 * q + 3]);
+    __syncwarp();
+    float4 *p4 = reinterpret_cast<float4 *>(p);
 #pragma unroll
-        for (int k = 0; k < RP; ++k) pv[k] = 0.0f;
+    for (int i = 0; i < Q; ++i) {
+        const int idx = i * 32 + lane;
+        const int rr = idx / Q, c4 = idx - (idx / Q) * Q;
+        if (row0 + rr < T) p4[row0 * Q + idx] = *reinterpret_cast<const float4 *>(tile + rr * (RP + 4) + 4 * c4);
     }
     if (t < Tp) {
 #pragma unroll
         for (int k = 0; k < RP; ++k) pt[(int64_t)k * Tp + t] = __float2bfloat16_rn(pv[k]);
     }
     if (amax) {
-        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
         for (int k = 0; k < RP; ++k) {
             float m = fabsf(pv[k]);
@@ -636,32 +674,39 @@ __device__ __forceinline__ int int4_code(float v, float s) {
 
 // INT4 per column: s_k = amax_k / 7; codes packed two per byte, the even
 // column in the low nibble.  One launch packs both factors: blockIdx.y = 0
-// packs P (T rows), 1 packs Q (C rows).  A thread owns one row: it reads the
-// row's rp floats as float4s and writes the row's nb bytes, as one 16-byte
-// store per 32 columns when the row's codes are 16-byte aligned, else byte
-// by byte (same bytes either way).  Block 0 of each factor writes the
-// column scales.
+// packs P (T rows), 1 packs Q (C rows).  Each warp stages its 32 rows through
+// shared memory with coalesced loads; a thread then codes one row and writes
+// the row's nb bytes, as one 16-byte store per 32 columns when the row's
+// codes are 16-byte aligned, else byte by byte (same bytes either way).
+// Block 0 of each factor writes the column scales.
 constexpr int kPackThreads = 128;
 
+template <int RP>
 __global__ void __launch_bounds__(kPackThreads) lr_int4_pack_kernel(const LrBatch B, const Layout L) {
     const int bz = blockIdx.z;
     if (lr_skipped(B, L, bz)) return;
     const int which = blockIdx.y;
     const int64_t rows = which == 0 ? L.T : L.C;
-    const int64_t row0 = (int64_t)blockIdx.x * kPackThreads;
-    if (row0 >= rows) return;   // the shorter factor's grid tail (never block 0)
+    const int64_t blk0 = (int64_t)blockIdx.x * kPackThreads;
+    if (blk0 >= rows) return;   // the shorter factor's grid tail (never block 0)
     const LrPtrs pp = B.get(bz);
-    const int r = L.r, rp = L.rp;
+    const int r = L.r;
     const float *f = B.at<float>(bz, which == 0 ? L.off_p : L.off_q);
-    const uint32_t *amax = B.at<uint32_t>(bz, L.off_amax) + (which == 0 ? 0 : rp);
+    const uint32_t *amax = B.at<uint32_t>(bz, L.off_amax) + (which == 0 ? 0 : RP);
     uint8_t *codes = which == 0 ? pp.pc_out : pp.qc_out;
     float *scales = which == 0 ? pp.ps_out : pp.qs_out;
     const int nb = (r + 1) / 2;
+    constexpr int NW = kPackThreads / 32;
     // the column scales, once per block (the same division every element
     // would otherwise repeat); zero past r, so padded columns code to 0
-    __shared__ float sc[cf_lowrank::kMaxRank];
-    for (int k = threadIdx.x; k < rp; k += kPackThreads)
+    __shared__ float sc[RP];
+    __shared__ __align__(16) float tiles[NW][32 * (RP + 4)];
+    for (int k = threadIdx.x; k < RP; k += kPackThreads)
         sc[k] = k < r ? __fdiv_rn(__uint_as_float(amax[k]), 7.0f) : 0.0f;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row0 = blk0 + 32 * warp;
+    float *tile = tiles[warp];
+    warp_stage_rows<RP>(f, row0, rows, tile, lane);
     __syncthreads();
     if (blockIdx.x == 0) {
         for (int k = threadIdx.x; k < r; k += kPackThreads) scales[k] = sc[k];
@@ -673,20 +718,21 @@ __global__ void __launch_bounds__(kPackThreads) lr_int4_pack_kernel(const LrBatc
             wt[cf_lowrank::kWarmC] = (uint32_t)L.C;
         }
     }
-    const int64_t row = row0 + threadIdx.x;
+    const int64_t row = row0 + lane;
     if (row >= rows) return;
-    const float4 *fr = reinterpret_cast<const float4 *>(f + row * rp);
+    const float4 *fr = reinterpret_cast<const float4 *>(tile + lane * (RP + 4));
     uint8_t *cr = codes + row * nb;
     const bool vec = (nb % 16) == 0 && (reinterpret_cast<uintptr_t>(cr) & 15u) == 0;
-    // 32 columns (16 bytes) at a time; rp is a multiple of 16, so the last
+    // 32 columns (16 bytes) at a time; RP is a multiple of 16, so the last
     // block may hold 16 columns (8 bytes)
-    for (int k0 = 0; k0 < rp; k0 += 32) {
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-        const int kn = rp - k0 < 32 ? rp - k0 : 32;
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-            if (4 * q4 >= kn || !CF_IN(k0 + 4 * q4 + 4 <= rp)) break;
-            const float4 v = __ldcg(fr + (k0 / 4 + q4));
+    for (int k0 = 0; k0 < RP; k0 += 32) {
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        constexpr int kMax = 8;
+#pragma unroll
+        for (int q4 = 0; q4 < kMax; ++q4) {
+            if (k0 + 4 * q4 >= RP) break;
+            const float4 v = fr[k0 / 4 + q4];
             const float e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -697,6 +743,7 @@ __global__ void __launch_bounds__(kPackThreads) lr_int4_pack_kernel(const LrBatc
             }
         }
         const int bytes = (nb - k0 / 2) < 16 ? (nb - k0 / 2) : 16;
+        if (bytes <= 0) break;
         if (vec && bytes == 16) {
             *reinterpret_cast<uint4 *>(cr + k0 / 2) = make_uint4(w[0], w[1], w[2], w[3]);
         } else {
