@@ -327,6 +327,35 @@ def test_decode_with_unaligned_codes_matches_aligned(r):
     assert ref.abs().max() > 0
 
 
+@pytest.mark.parametrize("r", [32, 64, 33])
+def test_encode_into_unaligned_codes_matches_aligned(r):
+    """The encode writes a row's INT4 codes as 16-byte vectors only where the
+    row is 16-byte aligned (even rank 32 or 64) and byte by byte otherwise:
+    code arrays at odd addresses receive exactly the bytes an aligned
+    encode of the same input writes, and the states stay identical."""
+    T, C = 700, 264
+    wl = W.replace(W.WORKLOADS["lowrank"], tokens=T, channels=C, rank=r)
+    xs = W.trajectory(wl, 0, steps=2, device="cuda")
+    om = W.omega(wl, 0, 1, device="cuda")
+    a, b = GpuLowrank(T, C, r, 2), GpuLowrank(T, C, r, 2)
+    a.init(xs[0].clone())
+    b.init(xs[0].clone())
+    nb = (r + 1) // 2
+    odd_p = torch.zeros(T * nb + 32, dtype=torch.uint8, device="cuda")
+    odd_q = torch.zeros(C * nb + 32, dtype=torch.uint8, device="cuda")
+    a.step(xs[1].clone(), om)
+    cf.cf_lowrank_encode(b.d, xs[1].clone().view(torch.int16), b.recon_s, b.err, om,
+                         odd_p.data_ptr() + 1, b.ps, odd_q.data_ptr() + 5, b.qs, b.ws)
+    torch.cuda.synchronize()
+    assert cf.cf_lowrank_status(a.ws) == 0 and cf.cf_lowrank_status(b.ws) == 0
+    assert torch.equal(odd_p[1:1 + T * nb], a.pc[:T * nb])
+    assert torch.equal(odd_q[5:5 + C * nb], a.qc[:C * nb])
+    assert not odd_p[0].item() and not odd_p[1 + T * nb:].any()      # nothing outside the rows
+    assert not odd_q[:5].any() and not odd_q[5 + C * nb:].any()
+    assert torch.equal(a.ps, b.ps) and torch.equal(a.qs, b.qs)
+    assert torch.equal(a.recon_s, b.recon_s) and torch.equal(a.err, b.err)
+
+
 def test_warm_start_trajectory():
     """omega NULL after the first compressed step: the iteration starts from
     the previous encode's Q (PowerSGD-style warm start); each step stays
