@@ -10,6 +10,7 @@ an out-of-range access in a status word and skip it (include/cf_diag.h).
 """
 from __future__ import annotations
 
+import fcntl
 import glob
 import hashlib
 import os
@@ -70,10 +71,25 @@ def up_to_date(debug: bool = False) -> bool:
 
 def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
     """Compile every source (in parallel) and link the library; nothing is
-    done when the stamp shows it was built from the same inputs."""
+    done when the stamp shows it was built from the same inputs.  Processes
+    that build at the same time (one per GPU of a multi-rank run) take turns
+    on a lock file, and a process that finds the library current once it
+    holds the lock does nothing."""
     lib = _lib(debug)
     if not force and up_to_date(debug):
         return lib
+    os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
+    with open(os.path.join(ROOT, "_build", ".lock"), "w") as lk:
+        fcntl.flock(lk, fcntl.LOCK_EX)
+        try:
+            if not force and up_to_date(debug):
+                return lib
+            return _compile(lib, verbose, debug)
+        finally:
+            fcntl.flock(lk, fcntl.LOCK_UN)
+
+
+def _compile(lib: str, verbose: bool, debug: bool) -> str:
     digest = _inputs_hash(debug)
     objdir = os.path.join(ROOT, "_build", "debug" if debug else "release")
     os.makedirs(objdir, exist_ok=True)

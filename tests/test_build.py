@@ -3,6 +3,8 @@ not from file times (a copied tree can round the times, which once made a
 rebuilt source look older than a stale library).  No compiler runs here:
 the hash and the up-to-date check are exercised on temporary files."""
 import os
+import threading
+import time
 
 from activation_residual_compression_cf_b200 import build as B
 
@@ -50,3 +52,36 @@ def test_oracle_build_stamp(tmp_path, monkeypatch):
     h1 = OB._inputs_hash()
     src.write_text("int f(void){return 2;}\n")
     assert OB._inputs_hash() != h1
+
+
+def test_concurrent_builds_take_turns(tmp_path, monkeypatch):
+    """Ranks of a multi-GPU run that find the library stale at the same time
+    compile one after another under the lock file, and the ones that get the
+    lock after the first build find the library current and compile nothing
+    (no two compilers write the same object files)."""
+    monkeypatch.setattr(B, "ROOT", str(tmp_path))
+    state = {"built": False, "active": 0, "most": 0, "compiles": 0}
+    mu = threading.Lock()
+
+    def fake_up_to_date(debug=False):
+        return state["built"]
+
+    def fake_compile(lib, verbose, debug):
+        with mu:
+            state["active"] += 1
+            state["most"] = max(state["most"], state["active"])
+        time.sleep(0.2)
+        with mu:
+            state["active"] -= 1
+            state["compiles"] += 1
+            state["built"] = True
+        return lib
+
+    monkeypatch.setattr(B, "up_to_date", fake_up_to_date)
+    monkeypatch.setattr(B, "_compile", fake_compile)
+    ts = [threading.Thread(target=B.build) for _ in range(4)]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    assert state["most"] == 1 and state["compiles"] == 1
