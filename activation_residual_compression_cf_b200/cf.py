@@ -36,7 +36,7 @@ EXPORTS = ("cf_status_string", "cf_abi_version", "cf_codes_words_per_row",
 # and the bounded-wait self-test (process-wide state, not product calls).
 DIAG_EXPORTS = ("cf_set_lowrank_engine", "cf_set_quant_pipeline", "cf_set_launch_override",
                 "cf_set_quant_unit", "cf_set_lowrank_group", "cf_lowrank_set_apply_events",
-                "cf_diag_bounded_wait", "cf_diag_stream_mix",
+                "cf_diag_bounded_wait", "cf_diag_stream_mix", "cf_diag_stream_mix_tma",
                 "cf_debug_bounds_checked", "cf_debug_bounds_take", "cf_diag_bounds_selftest")
 
 
@@ -145,6 +145,7 @@ def lib():
             "cf_set_quant_unit": ([i32, i32], ctypes.c_int),
             "cf_set_lowrank_group": ([i32], ctypes.c_int),
             "cf_diag_stream_mix": ([vp, vp, vp, i64, vp], ctypes.c_int),
+            "cf_diag_stream_mix_tma": ([vp, vp, vp, i64, i64, vp, vp], ctypes.c_int),
             "cf_debug_bounds_checked": ([], i32),
             "cf_debug_bounds_take": ([], i32),
             "cf_diag_bounds_selftest": ([vp, i32, vp], ctypes.c_int),
@@ -343,6 +344,13 @@ def bounds_file_tag(name: str) -> int:
 def cf_diag_stream_mix(x, r, a, stream=None):
     """Streaming pass with the encode's byte mix over every element of x."""
     _chk(lib().cf_diag_stream_mix(_p(x), _p(r), _p(a), x.numel(), _s(stream)), "cf_diag_stream_mix")
+
+
+def cf_diag_stream_mix_tma(x, r, a, rows, channels, status=None, stream=None):
+    """The encode's byte mix through the encode's TMA row pipeline (rows x
+    channels), without its per-row work."""
+    _chk(lib().cf_diag_stream_mix_tma(_p(x), _p(r), _p(a), rows, channels, _p(status), _s(stream)),
+         "cf_diag_stream_mix_tma")
 
 
 def cf_set_lowrank_group(buffers: int):

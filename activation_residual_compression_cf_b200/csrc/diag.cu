@@ -41,6 +41,10 @@ __global__ void diag_wait_kernel(uint32_t polls, int32_t *out) {
 // Each thread takes kMixUnroll groups of 8 elements a grid stride apart and
 // issues all their loads before any store.
 constexpr int kMixUnroll = 4;
+// Longest row the staged reference accepts (two 6C-byte slots fit in
+// shared memory; rows longer than 15360 channels need more than 480
+// consumer threads and are refused as unsupported).
+constexpr int64_t kMixTmaMaxC = 16384;
 
 __global__ void __launch_bounds__(128) diag_stream_mix_kernel(const uint4 *x, float4 *r, float4 *a,
                                                               int64_t n8) {
@@ -80,6 +84,114 @@ __global__ void __launch_bounds__(128) diag_stream_mix_kernel(const uint4 *x, fl
     }
 }
 
+// 1-D bulk copy global -> shared (no multicast) completing on an mbarrier;
+// both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void mix_bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// The same byte mix moved by the encode's own memory pipeline: a producer
+// lane bulk-copies each row's x (bf16, 2C bytes) and r (fp32, 4C bytes) into
+// a ring of shared-memory slots (no multicast); consumer warps read the row
+// from shared memory, release the slot and write a = (float)x - r and
+// r = (float)x + r with streaming stores, GPT groups of 8 channels per
+// thread.  None of the encode's per-row work (scale reduction and its
+// barrier, quantisation, codes).  Every wait is bounded: on expiry the
+// status word gets CF_ERR_TIMEOUT and the warp stops.
+template <int GPT>
+__global__ void __launch_bounds__(512) diag_stream_mix_tma_kernel(const uint16_t *x, float *r, float *a,
+                                                                  int64_t rows, int64_t C, int stages,
+                                                                  int32_t *status) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int64_t G = C >> 3;
+    const uint32_t slot = (uint32_t)(6 * C);
+    const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    const uint32_t bars = base + (uint32_t)stages * slot;
+    const int tid = threadIdx.x;
+    const int nc = blockDim.x - 32;
+    if (tid == 0) {
+        for (int s = 0; s < stages; ++s) {
+            cf::mbar_init(bars + 8u * s, 1);
+            cf::mbar_init(bars + 8u * (stages + s), (uint32_t)(nc / 32));
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (tid < 32) {
+        if (tid != 0) return;
+        int i = 0;
+        for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+            const int s = i % stages;
+            const uint32_t ph = (uint32_t)(i / stages) & 1u;
+            if (!cf::mbar_wait(bars + 8u * (stages + s), ph ^ 1u)) {
+                if (status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+                return;
+            }
+            if (!CF_IN(row < rows && s < stages)) continue;
+            const uint32_t dst = base + (uint32_t)s * slot;
+            cf::mbar_expect_tx(bars + 8u * s, slot);
+            mix_bulk_g2s(dst, x + row * C, (uint32_t)(2 * C), bars + 8u * s);
+            mix_bulk_g2s(dst + (uint32_t)(2 * C), r + row * C, (uint32_t)(4 * C), bars + 8u * s);
+            ++i;
+        }
+        return;
+    }
+    const int ct = tid - 32, lane = ct & 31;
+    int i = 0;
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+        const int s = i % stages;
+        const uint32_t ph = (uint32_t)(i / stages) & 1u;
+        bool ok = true;
+        if (lane == 0) ok = cf::mbar_wait(bars + 8u * s, ph);
+        if (__shfl_sync(cf::kFullMask, ok ? 1 : 0, 0) == 0) {
+            if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+            return;
+        }
+        const uint8_t *sx = smem + (size_t)s * slot;
+        const float *sr = reinterpret_cast<const float *>(sx + 2 * C);
+        float f[GPT][8], rr[GPT][8];
+#pragma unroll
+        for (int j = 0; j < GPT; ++j) {
+            const int64_t g = (int64_t)j * nc + ct;
+            if (g < G && CF_IN(8 * g + 8 <= C)) {
+                const uint4 xw = *reinterpret_cast<const uint4 *>(sx + 16 * g);
+                const float4 p0 = *reinterpret_cast<const float4 *>(sr + 8 * g);
+                const float4 p1 = *reinterpret_cast<const float4 *>(sr + 8 * g + 4);
+                const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[j][e] = cf::bf16_bits_to_f32((w[e >> 1] >> ((e & 1) * 16)) & 0xffffu);
+                rr[j][0] = p0.x; rr[j][1] = p0.y; rr[j][2] = p0.z; rr[j][3] = p0.w;
+                rr[j][4] = p1.x; rr[j][5] = p1.y; rr[j][6] = p1.z; rr[j][7] = p1.w;
+            }
+        }
+        // the slot is no longer read (generic-proxy reads before the next
+        // async-proxy bulk write into it)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) cf::mbar_arrive(bars + 8u * (stages + s));
+        ++i;
+        float *ar = a + row * C, *rw = r + row * C;
+#pragma unroll
+        for (int j = 0; j < GPT; ++j) {
+            const int64_t g = (int64_t)j * nc + ct;
+            if (g >= G || !CF_IN(8 * g + 8 <= C)) continue;
+            float d[8], t[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                d[e] = __fsub_rn(f[j][e], rr[j][e]);
+                t[e] = __fadd_rn(f[j][e], rr[j][e]);
+            }
+            cf::st_stream_v4(ar + 8 * g, make_float4(d[0], d[1], d[2], d[3]));
+            cf::st_stream_v4(ar + 8 * g + 4, make_float4(d[4], d[5], d[6], d[7]));
+            cf::st_stream_v4(rw + 8 * g, make_float4(t[0], t[1], t[2], t[3]));
+            cf::st_stream_v4(rw + 8 * g + 4, make_float4(t[4], t[5], t[6], t[7]));
+        }
+    }
+}
+
 }  // namespace
 
 extern "C" cf_status cf_diag_stream_mix(const uint16_t *x, float *r, float *a, int64_t n, void *stream) {
@@ -99,6 +211,50 @@ extern "C" cf_status cf_diag_stream_mix(const uint16_t *x, float *r, float *a, i
     if (blocks > need) blocks = need;
     diag_stream_mix_kernel<<<(unsigned)blocks, 128, 0, (cudaStream_t)stream>>>(
         reinterpret_cast<const uint4 *>(x), reinterpret_cast<float4 *>(r), reinterpret_cast<float4 *>(a), n / 8);
+    return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
+}
+
+extern "C" cf_status cf_diag_stream_mix_tma(const uint16_t *x, float *r, float *a, int64_t rows, int64_t C,
+                                             int32_t *status_dev, void *stream) {
+    cf::TraceRange trace_("cf_diag_stream_mix_tma");
+    if (rows < 0 || C < 8 || C % 8 != 0 || C > kMixTmaMaxC) return CF_ERR_INVALID_ARG;
+    if (rows == 0) return CF_OK;
+    if (!x || !r || !a) return CF_ERR_INVALID_ARG;
+    if (((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(a)) &
+         15u) != 0 ||
+        (reinterpret_cast<uintptr_t>(status_dev) & 3u) != 0)
+        return CF_ERR_ALIGNMENT;
+    // the encode's launch shape for the row length: 2 groups of 8 channels
+    // per consumer thread (4 where that keeps the CTA within 512 threads),
+    // a ring of up to 4 slots of 6C bytes
+    const int64_t G = C / 8;
+    int gpt = 2;
+    int64_t nc = ((G + gpt - 1) / gpt + 31) / 32 * 32;
+    if (nc > 480) {
+        gpt = 4;
+        nc = ((G + gpt - 1) / gpt + 31) / 32 * 32;
+    }
+    if (nc > 480) return CF_ERR_UNSUPPORTED;
+    const int64_t slot = 6 * C;
+    int stages = (int)(120000 / slot);
+    if (stages > 4) stages = 4;
+    if (stages < 2) stages = 2;
+    const size_t smem = (size_t)stages * slot + 16 * (size_t)stages;
+    void (*k)(const uint16_t *, float *, float *, int64_t, int64_t, int, int32_t *) =
+        gpt == 2 ? diag_stream_mix_tma_kernel<2> : diag_stream_mix_tma_kernel<4>;
+    const int threads = (int)nc + 32;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return CF_ERR_CUDA;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, threads, smem) != cudaSuccess || occ < 1) {
+        (void)cudaGetLastError();
+        occ = 1;
+    }
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t grid = (int64_t)sms * occ;
+    if (grid > rows) grid = rows;
+    k<<<(unsigned)grid, threads, smem, (cudaStream_t)stream>>>(x, r, a, rows, C, stages, status_dev);
     return cudaGetLastError() == cudaSuccess ? CF_OK : CF_ERR_CUDA;
 }
 

@@ -84,6 +84,21 @@ cf_status cf_set_quant_pipeline(int32_t kernel, int32_t pipeline, int32_t stages
  * CF_ERR_INVALID_ARG. */
 cf_status cf_diag_stream_mix(const uint16_t *x, float *r, float *a, int64_t n, void *stream);
 
+/* The same byte mix moved by the quantize encode's own memory pipeline (no
+ * counterpart in the paper): rows x rows of C channels, x bf16 [rows][C] and
+ * r fp32 [rows][C] read, a = (float)x - r and r = (float)x + r written
+ * (fp32 [rows][C] each).  A producer lane bulk-copies each row's x and r into
+ * a ring of shared-memory slots (the encode's ring depth and threads per row
+ * for this C); consumer warps write a and r with streaming stores.  It does
+ * none of the encode's per-row work (scale reduction, quantisation, codes),
+ * so the encode's time over this kernel's time is what that work costs.
+ * Device pointers, 16-byte aligned, non-overlapping; overwrites r and a.
+ * status_dev: optional device int32 (4-byte aligned) that receives
+ * CF_ERR_TIMEOUT if a bounded pipeline wait expires.  rows < 0, C < 8,
+ * C % 8 != 0 or C > 16384: CF_ERR_INVALID_ARG; C > 15360: CF_ERR_UNSUPPORTED. */
+cf_status cf_diag_stream_mix_tma(const uint16_t *x, float *r, float *a, int64_t rows, int64_t C,
+                                 int32_t *status_dev, void *stream);
+
 /* Bounds-checked debug build.  The library built with CF_DEBUG_BOUNDS
  * (libcf_debug.so) checks, at the global and shared-memory accesses of its
  * kernels, that the index arithmetic stays inside the array; a failed check

@@ -1,6 +1,7 @@
-"""The byte-mix ceiling pass (cf_diag_stream_mix) computes what it states,
-so the time bench.py reports for it is the time of that work: a = x - r and
-r = x + r elementwise in fp32, over a ragged number of elements."""
+"""The byte-mix reference passes (cf_diag_stream_mix, and
+cf_diag_stream_mix_tma through the encode's row pipeline) compute what they
+state, so the times bench.py reports for them are the times of that work:
+a = x - r and r = x + r elementwise in fp32, over ragged sizes."""
 import pytest
 import torch
 
@@ -28,3 +29,34 @@ def test_stream_mix_rejects_ragged_groups():
     with pytest.raises(cf.CFError) as ei:
         cf.cf_diag_stream_mix(x, r, r.clone())
     assert ei.value.status == 1
+
+
+@pytest.mark.parametrize("rows,C", [(1, 8), (37, 1920), (3 * 148 * 4 + 5, 1920), (300, 3072), (5, 15360)])
+def test_stream_mix_tma_computes_difference_and_sum(rows, C):
+    g = torch.Generator(device="cuda").manual_seed(rows * C)
+    x = torch.randn(rows, C, device="cuda", generator=g).to(torch.bfloat16)
+    r = torch.randn(rows, C, device="cuda", generator=g)
+    a = torch.full((rows, C), float("nan"), device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    r0 = r.clone()
+    cf.cf_diag_stream_mix_tma(x.view(torch.int16), r, a, rows, C, st)
+    torch.cuda.synchronize()
+    xf = x.float()
+    assert st.item() == 0
+    assert torch.equal(a, xf - r0) and torch.equal(r, xf + r0)
+
+
+def test_stream_mix_tma_rejects_bad_shapes():
+    x = torch.zeros(4, 24, dtype=torch.int16, device="cuda")
+    r = torch.zeros(4, 24, device="cuda")
+    for rows, C, code in ((4, 12, 1), (-1, 24, 1), (1, 16392, 1)):
+        with pytest.raises(cf.CFError) as ei:
+            cf.cf_diag_stream_mix_tma(x, r, r.clone(), rows, C)
+        assert ei.value.status == code
+    big = torch.zeros(1, 15368, device="cuda")
+    with pytest.raises(cf.CFError) as ei:
+        cf.cf_diag_stream_mix_tma(torch.zeros(1, 15368, dtype=torch.int16, device="cuda"), big, big.clone(),
+                                  1, 15368)
+    assert ei.value.status == 3
+    # nothing to do
+    cf.cf_diag_stream_mix_tma(x, r, r.clone(), 0, 24)
