@@ -19,6 +19,7 @@ namespace {
 // ---------------------------------------------------------------- helpers
 
 constexpr int kMaxGroupsPerThread = 4;
+constexpr int64_t kMaxDynSmem = 227 * 1024;   // dynamic shared memory a CTA may opt into
 constexpr int kMaxThreads = 512;
 constexpr int64_t kMaxChannels = 8LL * kMaxGroupsPerThread * kMaxThreads;  // 16384
 
@@ -178,6 +179,16 @@ cf_status launch_decode_t(const Src &src, int64_t T, int64_t C, int64_t rows, in
 // code rows (W % 4 == 0); at most 480 consumer threads.
 constexpr int kDecodeConsumerWarpsPerSM = 12;
 
+// The standard sender's encode (not the delta-state one): the sources whose
+// dedicated TMA kernel stores err and recon with bulk copies.
+template <bool ENC, class Src>
+constexpr bool standard_encode() {
+    if constexpr (ENC)
+        return !Src::kDelta;
+    else
+        return false;
+}
+
 template <bool ENC, int BITS, int GPT, int K, class Src>
 cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t *status,
                      const Shape &s, int stages_req, cudaStream_t st) {
@@ -190,25 +201,50 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
     // consumer warps per SM, 6-8 % above 5 slots at 2 CTAs); decode 5.  The
     // delta-state encode's slots are a third larger (8C bytes): 3 slots,
     // which keep three CTAs per SM, beat 4 (two CTAs) by ~10 %.
+    // a thread's GPT groups of 8 channels as 8 / K * GPT units of K; the
+    // plain 8-channel launches take the dedicated kernels (faster schedule),
+    // and the standard sender's dedicated encode stores err and recon with
+    // bulk copies from two shared-memory output rows (8C bytes each)
+    constexpr bool kPlain = K == 8 && !Src::kPublish && !Src::kWait;
+    bool delta = false;
+    if constexpr (ENC) delta = Src::kDelta;
+    constexpr bool kBulk = kPlain && standard_encode<ENC, Src>();
+    const int threads = 32 + s.threads;
+    void (*k)(Src, int64_t, int64_t, int64_t, int32_t *, int);
+    // Bulk-store encode: measured on B200 in the encode -> decode sequence,
+    // it beats the per-thread stores when a 2-slot ring plus the two output
+    // rows still lets four CTAs share an SM (C = 1920: encode +4 %), and
+    // loses where fewer fit (C = 3072, two CTAs: -15 %; C = 1920 with 3 or 4
+    // slots: -4 to -22 %).  So it runs with 2 slots, and only where the
+    // occupancy query gives four CTAs.
+    bool bulk = false;
+    if constexpr (kBulk) {
+        const size_t smem2 = 2 * (size_t)slot + 16 * (size_t)C + 32;
+        auto kb = cf::tma::encode_tma_kernel<BITS, GPT, Src, true>;
+        int occ_b = 0;
+        if (smem2 <= (size_t)kMaxDynSmem &&
+            cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) == cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_b, kb, threads, smem2) == cudaSuccess)
+            bulk = occ_b >= 4;
+        (void)cudaGetLastError();
+    }
+    const int64_t out_rows = bulk ? 16 * C : 0;
     int stages = stages_req;
     if (stages <= 0) {
-        bool delta = false;
-        if constexpr (ENC) delta = Src::kDelta;
-        stages = (int)((delta ? 75000 : 120000) / slot);
+        stages = bulk ? 2 : (int)((delta ? 75000 : 120000) / slot);
         const int cap = (ENC && !delta) ? 4 : 5;
         if (stages > cap) stages = cap;
     }
     if (stages > 8) stages = 8;
     if (stages < 2) stages = 2;
-    const size_t smem = (size_t)stages * slot + 16 * (size_t)stages;
-    const int threads = 32 + s.threads;
-    void (*k)(Src, int64_t, int64_t, int64_t, int32_t *, int);
-    // a thread's GPT groups of 8 channels as 8 / K * GPT units of K; the
-    // plain 8-channel launches take the dedicated kernels (faster schedule)
-    constexpr bool kPlain = K == 8 && !Src::kPublish && !Src::kWait;
+    size_t smem = (size_t)stages * slot + (size_t)out_rows + 16 * (size_t)stages;
+    while (smem > (size_t)kMaxDynSmem && stages > 2)
+        smem = (size_t)--stages * slot + (size_t)out_rows + 16 * (size_t)stages;
+    if (smem > (size_t)kMaxDynSmem) return CF_ERR_UNSUPPORTED;
     if constexpr (ENC) {
         if constexpr (kPlain)
-            k = cf::tma::encode_tma_kernel<BITS, GPT, Src>;
+            k = bulk ? cf::tma::encode_tma_kernel<BITS, GPT, Src, kBulk>
+                     : cf::tma::encode_tma_kernel<BITS, GPT, Src, false>;
         else if constexpr (Src::kPublish)
             k = cf::tma::encode_tma_publish_kernel<BITS, K, 8 / K * GPT, Src>;
         else
