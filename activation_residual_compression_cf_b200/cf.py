@@ -145,7 +145,7 @@ def lib():
             "cf_set_quant_unit": ([i32, i32], ctypes.c_int),
             "cf_set_lowrank_group": ([i32], ctypes.c_int),
             "cf_diag_stream_mix": ([vp, vp, vp, i64, vp], ctypes.c_int),
-            "cf_diag_stream_mix_tma": ([vp, vp, vp, i64, i64, vp, vp], ctypes.c_int),
+            "cf_diag_stream_mix_tma": ([vp, vp, vp, i64, i64, i32, vp, vp], ctypes.c_int),
             "cf_debug_bounds_checked": ([], i32),
             "cf_debug_bounds_take": ([], i32),
             "cf_diag_bounds_selftest": ([vp, i32, vp], ctypes.c_int),
@@ -346,11 +346,12 @@ def cf_diag_stream_mix(x, r, a, stream=None):
     _chk(lib().cf_diag_stream_mix(_p(x), _p(r), _p(a), x.numel(), _s(stream)), "cf_diag_stream_mix")
 
 
-def cf_diag_stream_mix_tma(x, r, a, rows, channels, status=None, stream=None):
+def cf_diag_stream_mix_tma(x, r, a, rows, channels, status=None, stream=None, bulk=False):
     """The encode's byte mix through the encode's TMA row pipeline (rows x
-    channels), without its per-row work."""
-    _chk(lib().cf_diag_stream_mix_tma(_p(x), _p(r), _p(a), rows, channels, _p(status), _s(stream)),
-         "cf_diag_stream_mix_tma")
+    channels) and its store path (bulk=True: bulk stores from shared-memory
+    output rows), without its per-row work."""
+    _chk(lib().cf_diag_stream_mix_tma(_p(x), _p(r), _p(a), rows, channels, 1 if bulk else 0, _p(status),
+                                      _s(stream)), "cf_diag_stream_mix_tma")
 
 
 def cf_set_lowrank_group(buffers: int):

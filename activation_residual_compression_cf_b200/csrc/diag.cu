@@ -93,26 +93,42 @@ __device__ __forceinline__ void mix_bulk_g2s(uint32_t dst, const void *src, uint
         : "memory");
 }
 
+__device__ __forceinline__ void mix_bulk_s2g(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
+
 // The same byte mix moved by the encode's own memory pipeline: a producer
 // lane bulk-copies each row's x (bf16, 2C bytes) and r (fp32, 4C bytes) into
 // a ring of shared-memory slots (no multicast); consumer warps read the row
-// from shared memory, release the slot and write a = (float)x - r and
-// r = (float)x + r with streaming stores, GPT groups of 8 channels per
-// thread.  None of the encode's per-row work (scale reduction and its
-// barrier, quantisation, codes).  Every wait is bounded: on expiry the
-// status word gets CF_ERR_TIMEOUT and the warp stops.
-template <int GPT>
+// from shared memory, release the slot and form a = (float)x - r and
+// r = (float)x + r, GPT groups of 8 channels per thread.  BULK = false:
+// they write a and r with streaming 16-byte stores.  BULK = true (the
+// standard encode's store path): they write them into one of two
+// shared-memory output rows, and one thread has the copy engine store the
+// row after the next row's barrier (every consumer passes a barrier per
+// row, as the encode's do for the scale); before that barrier it waits
+// until the previous store has read its output row.  None of the encode's
+// per-row work (scale, quantisation, codes).  Every mbarrier wait is
+// bounded: on expiry the status word gets CF_ERR_TIMEOUT and the CTA's
+// consumers leave together at the next barrier (BULK) or each warp leaves
+// (otherwise).
+template <int GPT, bool BULK>
 __global__ void __launch_bounds__(512) diag_stream_mix_tma_kernel(const uint16_t *x, float *r, float *a,
                                                                   int64_t rows, int64_t C, int stages,
                                                                   int32_t *status) {
     extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ int abort_row[2];   // BULK: set before a row's barrier, read after it
     const int64_t G = C >> 3;
     const uint32_t slot = (uint32_t)(6 * C);
     const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-    const uint32_t bars = base + (uint32_t)stages * slot;
+    const uint32_t obytes = BULK ? (uint32_t)(8 * C) : 0u;   // output row: a (4C) then r (4C)
+    const uint32_t obase = base + (uint32_t)stages * slot;
+    const uint32_t bars = obase + 2u * obytes;
     const int tid = threadIdx.x;
     const int nc = blockDim.x - 32;
     if (tid == 0) {
+        abort_row[0] = abort_row[1] = 0;
         for (int s = 0; s < stages; ++s) {
             cf::mbar_init(bars + 8u * s, 1);
             cf::mbar_init(bars + 8u * (stages + s), (uint32_t)(nc / 32));
@@ -140,15 +156,19 @@ __global__ void __launch_bounds__(512) diag_stream_mix_tma_kernel(const uint16_t
         return;
     }
     const int ct = tid - 32, lane = ct & 31;
-    int i = 0;
+    int i = 0, par = 0, orow = 0;
+    float *pend_a = nullptr, *pend_r = nullptr;   // BULK, thread ct 0: the row waiting in output row pend_o
+    int pend_o = 0;
     for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
         const int s = i % stages;
         const uint32_t ph = (uint32_t)(i / stages) & 1u;
         bool ok = true;
         if (lane == 0) ok = cf::mbar_wait(bars + 8u * s, ph);
-        if (__shfl_sync(cf::kFullMask, ok ? 1 : 0, 0) == 0) {
+        ok = __shfl_sync(cf::kFullMask, ok ? 1 : 0, 0) != 0;
+        if (!ok) {
             if (lane == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
-            return;
+            if constexpr (!BULK) return;
+            if (lane == 0) abort_row[par] = 1;   // acted on after the barrier
         }
         const uint8_t *sx = smem + (size_t)s * slot;
         const float *sr = reinterpret_cast<const float *>(sx + 2 * C);
@@ -156,7 +176,7 @@ __global__ void __launch_bounds__(512) diag_stream_mix_tma_kernel(const uint16_t
 #pragma unroll
         for (int j = 0; j < GPT; ++j) {
             const int64_t g = (int64_t)j * nc + ct;
-            if (g < G && CF_IN(8 * g + 8 <= C)) {
+            if (ok && g < G && CF_IN(8 * g + 8 <= C)) {
                 const uint4 xw = *reinterpret_cast<const uint4 *>(sx + 16 * g);
                 const float4 p0 = *reinterpret_cast<const float4 *>(sr + 8 * g);
                 const float4 p1 = *reinterpret_cast<const float4 *>(sr + 8 * g + 4);
@@ -171,9 +191,27 @@ __global__ void __launch_bounds__(512) diag_stream_mix_tma_kernel(const uint16_t
         // async-proxy bulk write into it)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        if (lane == 0) cf::mbar_arrive(bars + 8u * (stages + s));
+        if (lane == 0 && ok) cf::mbar_arrive(bars + 8u * (stages + s));
         ++i;
         float *ar = a + row * C, *rw = r + row * C;
+        float *oa = nullptr, *orr = nullptr;
+        if constexpr (BULK) {
+            if (ct == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            asm volatile("bar.sync 1, %0;" ::"r"(nc) : "memory");
+            if (*(volatile int *)&abort_row[par]) {
+                if (ct == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+                return;   // every consumer warp sees the same flag here
+            }
+            par ^= 1;
+            if (ct == 0 && pend_a) {
+                const uint32_t ob = obase + (uint32_t)(pend_o & 1) * obytes;
+                mix_bulk_s2g(pend_a, ob, (uint32_t)(4 * C));
+                mix_bulk_s2g(pend_r, ob + (uint32_t)(4 * C), (uint32_t)(4 * C));
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            }
+            oa = reinterpret_cast<float *>(smem + (size_t)stages * slot + (size_t)(orow & 1) * obytes);
+            orr = oa + C;
+        }
 #pragma unroll
         for (int j = 0; j < GPT; ++j) {
             const int64_t g = (int64_t)j * nc + ct;
@@ -184,10 +222,39 @@ __global__ void __launch_bounds__(512) diag_stream_mix_tma_kernel(const uint16_t
                 d[e] = __fsub_rn(f[j][e], rr[j][e]);
                 t[e] = __fadd_rn(f[j][e], rr[j][e]);
             }
-            cf::st_stream_v4(ar + 8 * g, make_float4(d[0], d[1], d[2], d[3]));
-            cf::st_stream_v4(ar + 8 * g + 4, make_float4(d[4], d[5], d[6], d[7]));
-            cf::st_stream_v4(rw + 8 * g, make_float4(t[0], t[1], t[2], t[3]));
-            cf::st_stream_v4(rw + 8 * g + 4, make_float4(t[4], t[5], t[6], t[7]));
+            if constexpr (BULK) {
+                *reinterpret_cast<float4 *>(oa + 8 * g) = make_float4(d[0], d[1], d[2], d[3]);
+                *reinterpret_cast<float4 *>(oa + 8 * g + 4) = make_float4(d[4], d[5], d[6], d[7]);
+                *reinterpret_cast<float4 *>(orr + 8 * g) = make_float4(t[0], t[1], t[2], t[3]);
+                *reinterpret_cast<float4 *>(orr + 8 * g + 4) = make_float4(t[4], t[5], t[6], t[7]);
+            } else {
+                cf::st_stream_v4(ar + 8 * g, make_float4(d[0], d[1], d[2], d[3]));
+                cf::st_stream_v4(ar + 8 * g + 4, make_float4(d[4], d[5], d[6], d[7]));
+                cf::st_stream_v4(rw + 8 * g, make_float4(t[0], t[1], t[2], t[3]));
+                cf::st_stream_v4(rw + 8 * g + 4, make_float4(t[4], t[5], t[6], t[7]));
+            }
+        }
+        if constexpr (BULK) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            if (ct == 0) {
+                pend_a = ar;
+                pend_r = rw;
+                pend_o = orow;
+            }
+            ++orow;
+        }
+    }
+    if constexpr (BULK) {
+        // the last row's outputs: every consumer has written its part
+        asm volatile("bar.sync 1, %0;" ::"r"(nc) : "memory");
+        if (ct == 0) {
+            if (pend_a) {
+                const uint32_t ob = obase + (uint32_t)(pend_o & 1) * obytes;
+                mix_bulk_s2g(pend_a, ob, (uint32_t)(4 * C));
+                mix_bulk_s2g(pend_r, ob + (uint32_t)(4 * C), (uint32_t)(4 * C));
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            }
+            asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
         }
     }
 }
@@ -215,20 +282,21 @@ extern "C" cf_status cf_diag_stream_mix(const uint16_t *x, float *r, float *a, i
 }
 
 extern "C" cf_status cf_diag_stream_mix_tma(const uint16_t *x, float *r, float *a, int64_t rows, int64_t C,
-                                             int32_t *status_dev, void *stream) {
+                                             int32_t bulk, int32_t *status_dev, void *stream) {
     cf::TraceRange trace_("cf_diag_stream_mix_tma");
-    if (rows < 0 || C < 8 || C % 8 != 0 || C > kMixTmaMaxC) return CF_ERR_INVALID_ARG;
+    if (rows < 0 || C < 8 || C % 8 != 0 || C > kMixTmaMaxC || (bulk != 0 && bulk != 1)) return CF_ERR_INVALID_ARG;
     if (rows == 0) return CF_OK;
     if (!x || !r || !a) return CF_ERR_INVALID_ARG;
     if (((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(a)) &
          15u) != 0 ||
         (reinterpret_cast<uintptr_t>(status_dev) & 3u) != 0)
         return CF_ERR_ALIGNMENT;
-    // the encode's launch shape for the row length: 2 groups of 8 channels
-    // per consumer thread (4 where that keeps the CTA within 512 threads),
-    // a ring of up to 4 slots of 6C bytes
+    // the encode's launch shapes: per-thread stores with 2 groups of 8
+    // channels per consumer thread (4 where that keeps the CTA within 512
+    // threads) and a ring of up to 4 slots of 6C bytes; bulk stores with 4
+    // groups, 2 slots and two 8C-byte output rows
     const int64_t G = C / 8;
-    int gpt = 2;
+    int gpt = bulk ? 4 : 2;
     int64_t nc = ((G + gpt - 1) / gpt + 31) / 32 * 32;
     if (nc > 480) {
         gpt = 4;
@@ -236,12 +304,14 @@ extern "C" cf_status cf_diag_stream_mix_tma(const uint16_t *x, float *r, float *
     }
     if (nc > 480) return CF_ERR_UNSUPPORTED;
     const int64_t slot = 6 * C;
-    int stages = (int)(120000 / slot);
+    int stages = bulk ? 2 : (int)(120000 / slot);
     if (stages > 4) stages = 4;
     if (stages < 2) stages = 2;
-    const size_t smem = (size_t)stages * slot + 16 * (size_t)stages;
+    const size_t smem = (size_t)stages * slot + (bulk ? 16 * (size_t)C : 0) + 16 * (size_t)stages;
+    if (smem > 227 * 1024) return CF_ERR_UNSUPPORTED;
     void (*k)(const uint16_t *, float *, float *, int64_t, int64_t, int, int32_t *) =
-        gpt == 2 ? diag_stream_mix_tma_kernel<2> : diag_stream_mix_tma_kernel<4>;
+        bulk ? (gpt == 2 ? diag_stream_mix_tma_kernel<2, true> : diag_stream_mix_tma_kernel<4, true>)
+             : (gpt == 2 ? diag_stream_mix_tma_kernel<2, false> : diag_stream_mix_tma_kernel<4, false>);
     const int threads = (int)nc + 32;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return CF_ERR_CUDA;

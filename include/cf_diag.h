@@ -88,15 +88,21 @@ cf_status cf_diag_stream_mix(const uint16_t *x, float *r, float *a, int64_t n, v
  * counterpart in the paper): rows x rows of C channels, x bf16 [rows][C] and
  * r fp32 [rows][C] read, a = (float)x - r and r = (float)x + r written
  * (fp32 [rows][C] each).  A producer lane bulk-copies each row's x and r into
- * a ring of shared-memory slots (the encode's ring depth and threads per row
- * for this C); consumer warps write a and r with streaming stores.  It does
- * none of the encode's per-row work (scale reduction, quantisation, codes),
- * so the encode's time over this kernel's time is what that work costs.
- * Device pointers, 16-byte aligned, non-overlapping; overwrites r and a.
+ * a ring of shared-memory slots; consumer warps compute from shared memory
+ * and write a and r with the encode's store path: bulk = 0, per-thread
+ * streaming stores (the encode's launch shape for long rows); bulk = 1,
+ * two shared-memory output rows stored by the copy engine after each row's
+ * barrier, 4 groups of 8 channels per thread and 2 slots (the standard
+ * encode's shape where four CTAs fit on an SM).  It does none of the
+ * encode's per-row work (scale reduction, quantisation, codes), so the
+ * encode's time over this kernel's time is what that work costs.  Device
+ * pointers, 16-byte aligned, non-overlapping; overwrites r and a.
  * status_dev: optional device int32 (4-byte aligned) that receives
  * CF_ERR_TIMEOUT if a bounded pipeline wait expires.  rows < 0, C < 8,
- * C % 8 != 0 or C > 16384: CF_ERR_INVALID_ARG; C > 15360: CF_ERR_UNSUPPORTED. */
-cf_status cf_diag_stream_mix_tma(const uint16_t *x, float *r, float *a, int64_t rows, int64_t C,
+ * C % 8 != 0, C > 16384 or bulk not 0 or 1: CF_ERR_INVALID_ARG; rows needing
+ * more than 480 consumer threads (C > 15360) or more shared memory than a
+ * CTA may have (bulk: C > 8300): CF_ERR_UNSUPPORTED. */
+cf_status cf_diag_stream_mix_tma(const uint16_t *x, float *r, float *a, int64_t rows, int64_t C, int32_t bulk,
                                  int32_t *status_dev, void *stream);
 
 /* Bounds-checked debug build.  The library built with CF_DEBUG_BOUNDS

@@ -31,15 +31,18 @@ def test_stream_mix_rejects_ragged_groups():
     assert ei.value.status == 1
 
 
+@pytest.mark.parametrize("bulk", [False, True])
 @pytest.mark.parametrize("rows,C", [(1, 8), (37, 1920), (3 * 148 * 4 + 5, 1920), (300, 3072), (5, 15360)])
-def test_stream_mix_tma_computes_difference_and_sum(rows, C):
+def test_stream_mix_tma_computes_difference_and_sum(rows, C, bulk):
+    if bulk and C > 8296:
+        pytest.skip("bulk stores: two ring slots and two output rows exceed a CTA's shared memory")
     g = torch.Generator(device="cuda").manual_seed(rows * C)
     x = torch.randn(rows, C, device="cuda", generator=g).to(torch.bfloat16)
     r = torch.randn(rows, C, device="cuda", generator=g)
     a = torch.full((rows, C), float("nan"), device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     r0 = r.clone()
-    cf.cf_diag_stream_mix_tma(x.view(torch.int16), r, a, rows, C, st)
+    cf.cf_diag_stream_mix_tma(x.view(torch.int16), r, a, rows, C, st, bulk=bulk)
     torch.cuda.synchronize()
     xf = x.float()
     assert st.item() == 0
@@ -53,6 +56,11 @@ def test_stream_mix_tma_rejects_bad_shapes():
         with pytest.raises(cf.CFError) as ei:
             cf.cf_diag_stream_mix_tma(x, r, r.clone(), rows, C)
         assert ei.value.status == code
+    with pytest.raises(cf.CFError) as ei:     # bulk: 2 slots + 2 output rows beyond a CTA's shared memory
+        cf.cf_diag_stream_mix_tma(torch.zeros(1, 8304, dtype=torch.int16, device="cuda"),
+                                  torch.zeros(1, 8304, device="cuda"), torch.zeros(1, 8304, device="cuda"),
+                                  1, 8304, bulk=True)
+    assert ei.value.status == 3
     big = torch.zeros(1, 15368, device="cuda")
     with pytest.raises(cf.CFError) as ei:
         cf.cf_diag_stream_mix_tma(torch.zeros(1, 15368, dtype=torch.int16, device="cuda"), big, big.clone(),
