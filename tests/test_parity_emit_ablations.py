@@ -26,10 +26,12 @@ from _parity import GpuBuffer, compare_step, f32_of, oracle_step
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("pipe", [0, 1])
+@pytest.mark.parametrize("pipe,unit", [(0, 0), (1, 0), (1, 8)])
 @pytest.mark.parametrize("T,C,bits", [(64, 3072, 2), (64, 3072, 1), (37, 1920, 2), (9, 200, 2),
                                       (13, 33, 1), (5, 16384, 2)])
-def test_decode_emit_matches_oracle(T, C, bits, pipe):
+def test_decode_emit_matches_oracle(T, C, bits, pipe, unit):
+    """unit 0: the built-in choice (4-channel units for the emitting decode
+    on the TMA pipeline); unit 8: the 8-channel kernel, same results."""
     wl = W.replace(W.WORKLOADS["flux_sp"], tokens=T, channels=C, bits=bits)
     xs = W.trajectory(wl, 6, steps=3, device="cuda")
     xb = [W.bf16_bits(x) for x in xs]
@@ -39,6 +41,7 @@ def test_decode_emit_matches_oracle(T, C, bits, pipe):
     rr = ro.copy()
     try:
         cf.cf_set_quant_pipeline(1, pipe, 0)
+        cf.cf_set_quant_unit(1, unit)
         g.init(xs[0].clone())
         for s in (1, 2):
             cf.cf_encode(g.d, xs[s].clone().view(torch.int16), g.recon_s, g.err, g.codes, g.scales)
@@ -57,6 +60,7 @@ def test_decode_emit_matches_oracle(T, C, bits, pipe):
             assert same.mean() > 0.999 and np.array_equal(gout[same], o_out[same])
     finally:
         cf.cf_set_quant_pipeline(1, 1, 0)
+        cf.cf_set_quant_unit(1, 0)
 
 
 def test_decode_emit_batched_full_size_sampled():
