@@ -198,10 +198,12 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
     if constexpr (ENC) slot = (Src::kDelta ? 8 : 6) * C;
     // Ring depth, measured on B200 (C = 1920 and 3072) in runs long enough
     // for the power cap to hold the SM clock down, as in sustained use:
-    // encode 4 slots (with 2 groups per thread that keeps 3-4 CTAs and 16-18
-    // consumer warps per SM, 6-8 % above 5 slots at 2 CTAs); decode 5.  The
-    // delta-state encode's slots are a third larger (8C bytes): 3 slots,
-    // which keep three CTAs per SM, beat 4 (two CTAs) by ~10 %.
+    // encode with per-thread stores 4 slots (with 2 groups per thread that
+    // keeps 3-4 CTAs and 16-18 consumer warps per SM, 6-8 % above 5 slots at
+    // 2 CTAs); the bulk-store encode 2 (below); decode 5.  The delta-state
+    // encode's slots are a third larger (8C bytes): at C = 3072, 3 slots,
+    // which keep three CTAs per SM, beat 4 (two CTAs) by ~10 %; at C <= 2048
+    // it takes 2 (below).
     // a thread's GPT groups of 8 channels as 8 / K * GPT units of K; the
     // plain 8-channel launches take the dedicated kernels (faster schedule),
     // and the standard sender's dedicated encode stores err and recon with
@@ -232,7 +234,16 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
     const int64_t out_rows = bulk ? 16 * C : 0;
     int stages = stages_req;
     if (stages <= 0) {
-        stages = bulk ? 2 : (int)((delta ? 75000 : 120000) / slot);
+        // delta-state encode: 2 slots where a slot (8C bytes) is at most
+        // 16 KB, measured on B200 at C = 1920 (4 groups per thread):
+        // 6042-6060 GB/s against 5052 with 4 slots, as more CTAs share an
+        // SM; at C = 3072, 3 slots (75 KB) stay best (2: -4 to -6 %)
+        if (bulk)
+            stages = 2;
+        else if (delta)
+            stages = slot <= 16384 ? 2 : (int)(75000 / slot);
+        else
+            stages = (int)(120000 / slot);
         const int cap = (ENC && !delta) ? 4 : 5;
         if (stages > cap) stages = cap;
     }
