@@ -320,3 +320,51 @@ def test_rows_pipeline_bad_buffers_between_valid_ones(C):
                   scales=part["scales"][b].cpu().numpy(), err=part["err"][b].cpu().numpy(),
                   recon_s=part["recon_s"][b].cpu().numpy())
         compare_step(wl.bits, v, ora, gh)
+
+
+@pytest.mark.parametrize("C", [1920, 1024])
+def test_bulk_encode_bad_buffers_between_valid_ones(C):
+    """TMA encode with bulk stores (rows short enough for four CTAs per SM)
+    on a grid of one CTA per SM, every other buffer of the batched call
+    invalid: each CTA meets valid and skipped rows in turn, so a row's
+    outputs wait in shared memory across skipped rows before their bulk
+    store.  The valid buffers must equal an all-valid run bit for bit and
+    the oracle within the parity bar; the skipped buffers stay untouched."""
+    n, T = 24, 16
+    wl = W.replace(W.WORKLOADS["cogvideox"], tokens=T, channels=C, buffers=n)
+    xs = torch.stack([W.trajectory(wl, b, steps=2, device="cuda") for b in range(n)], 1)
+    d = cf.desc(T, C, wl.bits)
+    x16 = xs[1].view(torch.int16)
+    runs = []
+    G = C // 8
+    try:
+        cf.cf_set_launch_override(0, 4, ((G + 3) // 4 + 31) // 32 * 32, 1)   # one CTA per SM
+        for skip in (False, True):
+            st = _batched_state(wl, n)
+            for b in range(n):
+                cf.cf_state_init(d, xs[0, b].view(torch.int16), st["recon_s"][b], st["err"][b])
+            before = st["recon_s"].clone()
+            sets = [(x16[b], st["recon_s"][b], st["err"][b], st["codes"][b], st["scales"][b])
+                    for b in range(n)]
+            if skip:
+                sets = [s if b % 2 == 0 else (0,) + s[1:] for b, s in enumerate(sets)]
+            status = torch.zeros(1, dtype=torch.int32, device="cuda")
+            cf.cf_encode_batched(d, n, cf.enc_buffer_array(sets, "cuda"), status)
+            torch.cuda.synchronize()
+            assert int(status.item()) == (1 if skip else 0)
+            if skip:
+                for b in range(1, n, 2):
+                    assert torch.equal(st["recon_s"][b], before[b])
+            runs.append(st)
+    finally:
+        cf.cf_set_launch_override(0, 0, 0, 0)
+    full, part = runs
+    for b in range(0, n, 2):
+        for k in ("codes", "scales", "err", "recon_s"):
+            assert torch.equal(full[k][b].view(torch.int32), part[k][b].view(torch.int32)), (b, k)
+        r0, _ = oracle.state_init(W.bf16_bits(xs[0, b]))
+        v, ora = oracle_step(W.bf16_bits(xs[1, b]), r0, wl.bits)
+        gh = dict(codes=part["codes"][b].cpu().numpy().view(np.uint32),
+                  scales=part["scales"][b].cpu().numpy(), err=part["err"][b].cpu().numpy(),
+                  recon_s=part["recon_s"][b].cpu().numpy())
+        compare_step(wl.bits, v, ora, gh)
