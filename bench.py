@@ -599,6 +599,11 @@ def run_ours(args, world, rank, local):
                      "mix_reference": mix},
         "decode": {"achieved": round(dec_gbs, 1), "frac": round(dec_gbs / peak, 4),
                    "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_ms": round(dec_ms, 4)},
+        # the whole timed step against the same roofline: both launches'
+        # algorithmic bytes over the step time (the slowest rank's)
+        "step_roofline": {"algorithmic_bytes_per_step": enc_bytes + dec_bytes,
+                          "achieved": round((enc_bytes + dec_bytes) * args.steps / (ms / 1e3) / 1e9, 1),
+                          "frac": round((enc_bytes + dec_bytes) * args.steps / (ms / 1e3) / 1e9 / peak, 4)},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "invariants": invariants,
