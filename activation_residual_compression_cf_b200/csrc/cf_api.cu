@@ -220,10 +220,18 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
     // loses where fewer fit (C = 3072, two CTAs: -15 %; C = 1920 with 3 or 4
     // slots: -4 to -22 %).  So it runs with 2 slots, and only where the
     // occupancy query gives four CTAs.
+    // The publishing encode (8-channel units) takes the same bulk-store path
+    // for its local err and recon rows under the same condition; its codes
+    // and scales still go straight to the receivers' slots.
+    constexpr bool kBulkPub = ENC && Src::kPublish && K == 8;
     bool bulk = false;
-    if constexpr (kBulk) {
+    if constexpr (kBulk || kBulkPub) {
         const size_t smem2 = 2 * (size_t)slot + 16 * (size_t)C + 32;
-        auto kb = cf::tma::encode_tma_kernel<BITS, GPT, Src, true>;
+        void (*kb)(Src, int64_t, int64_t, int64_t, int32_t *, int);
+        if constexpr (kBulk)
+            kb = cf::tma::encode_tma_kernel<BITS, GPT, Src, true>;
+        else
+            kb = cf::tma::encode_tma_publish_kernel<BITS, K, 8 / K * GPT, Src, true>;
         int occ_b = 0;
         if (smem2 <= (size_t)kMaxDynSmem &&
             cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) == cudaSuccess &&
@@ -258,7 +266,8 @@ cf_status launch_tma(const Src &src, int64_t T, int64_t C, int64_t rows, int32_t
             k = bulk ? cf::tma::encode_tma_kernel<BITS, GPT, Src, kBulk>
                      : cf::tma::encode_tma_kernel<BITS, GPT, Src, false>;
         else if constexpr (Src::kPublish)
-            k = cf::tma::encode_tma_publish_kernel<BITS, K, 8 / K * GPT, Src>;
+            k = bulk ? cf::tma::encode_tma_publish_kernel<BITS, K, 8 / K * GPT, Src, kBulkPub>
+                     : cf::tma::encode_tma_publish_kernel<BITS, K, 8 / K * GPT, Src, false>;
         else
             k = cf::tma::encode_tma_unit_kernel<BITS, K, 8 / K * GPT, Src>;
     } else {

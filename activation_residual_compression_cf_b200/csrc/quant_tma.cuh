@@ -97,6 +97,14 @@ __device__ __forceinline__ void load_unit(const uint8_t *sx, const uint8_t *sp, 
     }
 }
 
+// K fp32 values of unit u to a row in shared memory (an output row of the
+// bulk-store path): one or two 16-byte stores.
+template <int K>
+__device__ __forceinline__ void store_unit_shared(float *row, int u, const float *o) {
+    *reinterpret_cast<float4 *>(row + K * u) = make_float4(o[0], o[1], o[2], o[3]);
+    if constexpr (K == 8) *reinterpret_cast<float4 *>(row + K * u + 4) = make_float4(o[4], o[5], o[6], o[7]);
+}
+
 // K fp32 values of unit u to a row: one or two 16-byte stores.
 template <int K, bool STREAM>
 __device__ __forceinline__ void store_unit(float *row, int u, const float *o) {
@@ -477,10 +485,14 @@ decode_tma_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, 
     }
 }
 
-template <int BITS, int K, int UPT, class Src>
+// BULK: the standard encode's bulk-store path (two shared-memory output
+// rows, stores issued after the next row's scale barrier), as in
+// encode_tma_kernel.
+template <int BITS, int K, int UPT, class Src, bool BULK = false>
 __device__ __forceinline__ void encode_unit_body(const Src &src, int64_t T, int64_t C, int64_t rows,
                                                  int32_t *status, int stages) {
     static_assert(K == 4 || K == 8, "units of 4 or 8 channels");
+    static_assert(!(BULK && Src::kDelta), "bulk stores serve the standard sender");
     constexpr int UPW = 32 / (K * BITS);  // units per 32-bit code word
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ double sh_sum[2][32];
@@ -491,7 +503,9 @@ __device__ __forceinline__ void encode_unit_body(const Src &src, int64_t T, int6
     const int64_t W = (C * BITS + 31) >> 5;
     const uint32_t slot = (uint32_t)((Src::kDelta ? 8 : 6) * C);
     const uint32_t base = saddr(smem);
-    const uint32_t bars = base + (uint32_t)stages * slot;
+    const uint32_t obytes = BULK ? (uint32_t)(8 * C) : 0u;   // BULK output row: err, then recon
+    const uint32_t obase = base + (uint32_t)stages * slot;
+    const uint32_t bars = obase + 2u * obytes;
     const int tid = threadIdx.x;
     const int nc = blockDim.x - 32;  // consumer threads
     if (tid == 0) {
@@ -543,6 +557,17 @@ __device__ __forceinline__ void encode_unit_body(const Src &src, int64_t T, int6
     const int lane = ct & 31, warp = ct >> 5, nw = nc >> 5;
     int i = 0, par = 0;
     uint64_t walked = 0;  // rows this CTA walked, skipped ones included (publishing)
+    float *pend_err = nullptr, *pend_rec = nullptr;   // BULK, thread ct 0: the row in output row pend_o
+    int pend_o = 0, orow = 0;
+    auto flush_pending = [&]() {
+        if (BULK && ct == 0 && pend_err) {
+            const uint32_t ob = obase + (uint32_t)(pend_o & 1) * obytes;
+            bulk_s2g(pend_err, ob, (uint32_t)(4 * C));
+            bulk_s2g(pend_rec, ob + (uint32_t)(4 * C), (uint32_t)(4 * C));
+            bulk_commit();
+            pend_err = pend_rec = nullptr;
+        }
+    };
     for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
         const int64_t b = row / T, t = row - b * T;
         const EncPtrs p = src.get(b);
@@ -597,11 +622,14 @@ __device__ __forceinline__ void encode_unit_body(const Src &src, int64_t T, int6
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFullMask, acc, o);
             if (lane == 0) sh_sum[par][warp] = acc;
+            if (BULK && ct == 0) bulk_wait_read();   // output row orow % 2 is free after the barrier
             consumer_sync(nc);
             if (*(volatile int *)&abort_row[par]) {
                 if (ct == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+                if (BULK && ct == 0) bulk_wait_all();
                 return;  // every consumer warp sees the same flag here
             }
+            flush_pending();
             double tot = 0.0;
             for (int w = 0; w < nw; ++w) tot += sh_sum[par][w];
             scale = __fdiv_rn(__double2float_rn(tot), (float)C);
@@ -614,11 +642,14 @@ __device__ __forceinline__ void encode_unit_body(const Src &src, int64_t T, int6
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
             if (lane == 0) sh_max[par][warp] = m;
+            if (BULK && ct == 0) bulk_wait_read();   // output row orow % 2 is free after the barrier
             consumer_sync(nc);
             if (*(volatile int *)&abort_row[par]) {
                 if (ct == 0 && status) atomicCAS(status, (int32_t)CF_OK, (int32_t)CF_ERR_TIMEOUT);
+                if (BULK && ct == 0) bulk_wait_all();
                 return;
             }
+            flush_pending();
             float tot = 0.0f;
             for (int w = 0; w < nw; ++w) tot = fmaxf(tot, sh_max[par][w]);
             scale = tot;
@@ -641,8 +672,14 @@ __device__ __forceinline__ void encode_unit_body(const Src &src, int64_t T, int6
                 ro[e] = __fadd_rn(r[j][e], d);
             }
             if (u < NU && CF_IN(K * u + K <= C && t < T)) {
-                store_unit<K, true>(er, u, eo);
-                if (!Src::kDelta) store_unit<K, false>(rr, u, ro);
+                if constexpr (BULK) {
+                    float *oe = reinterpret_cast<float *>(smem + (size_t)stages * slot + (size_t)(orow & 1) * obytes);
+                    store_unit_shared<K>(oe, u, eo);
+                    store_unit_shared<K>(oe + C, u, ro);
+                } else {
+                    store_unit<K, true>(er, u, eo);
+                    if (!Src::kDelta) store_unit<K, false>(rr, u, ro);
+                }
             }
             // nc is a multiple of 32, so u % UPW == lane % UPW: the UPW
             // lanes of one code word are adjacent and aligned
@@ -670,12 +707,28 @@ __device__ __forceinline__ void encode_unit_body(const Src &src, int64_t T, int6
         } else {
             if (ct == 0 && CF_IN(t < T)) p.scales[t] = scale;
         }
+        if constexpr (BULK) {
+            // this thread's output-row writes, visible to the copy engine
+            // once every consumer has passed the next barrier
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            if (ct == 0) {
+                pend_err = er;
+                pend_rec = rr;
+                pend_o = orow;
+            }
+            ++orow;
+        }
     }
-    if constexpr (Src::kPublish) {
+    if constexpr (Src::kPublish || BULK) {
         // every consumer's stores of this CTA precede the barrier; the
-        // system-scope fence of the publishing thread is cumulative over them
+        // system-scope fence of the publishing thread is cumulative over
+        // them; BULK: the last row's outputs are in shared memory
         consumer_sync(nc);
-        if (ct == 0) src.publish(walked);
+        flush_pending();
+        if constexpr (Src::kPublish) {
+            if (ct == 0) src.publish(walked);
+        }
+        if (BULK && ct == 0) bulk_wait_all();
     }
 }
 
@@ -691,10 +744,10 @@ encode_tma_unit_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *sta
 // sub-partitions, and the sub-partition that holds 6 of the 21 warps needs
 // 6 x 32 x R <= 16384.  Without the cap the destination stores raise R past
 // 110, and at 96 only two CTAs fit (measured: 296-CTA grid, 40 % slower).
-template <int BITS, int K, int UPT, class Src>
+template <int BITS, int K, int UPT, class Src, bool BULK = false>
 __global__ void __maxnreg__(80)
 encode_tma_publish_kernel(Src src, int64_t T, int64_t C, int64_t rows, int32_t *status, int stages) {
-    encode_unit_body<BITS, K, UPT, Src>(src, T, C, rows, status, stages);
+    encode_unit_body<BITS, K, UPT, Src, BULK>(src, T, C, rows, status, stages);
 }
 
 template <int BITS, int K, int UPT, class Src>
